@@ -1,0 +1,48 @@
+"""Pins for the replay certificate (CPU only): it accepts correct greedy
+codes and rejects planted mistakes (a wrong pick, a wrong coefficient)."""
+
+import numpy as np
+
+import oracle
+
+
+def _setup(seed=0, n=256, d=32, m=6):
+    rng = np.random.default_rng(seed)
+    D = rng.standard_normal((n, d))
+    D /= np.linalg.norm(D, axis=1, keepdims=True)
+    X = rng.standard_normal((m, d))
+    return D, X
+
+
+def _words(ref):
+    return oracle.pack_words(ref["idx"], oracle.store_coef_fp16(ref["coef"]))
+
+
+def test_certificate_accepts_oracle_codes():
+    D, X = _setup()
+    ref = oracle.encode_ref(X, D)
+    c = oracle.certify_codes(X, D, _words(ref))
+    assert c["ok_pick"].all() and c["ok_coef"].all()
+    assert np.allclose(c["pick_ratio"], 1.0)
+
+
+def test_certificate_rejects_wrong_pick():
+    D, X = _setup(1)
+    ref = oracle.encode_ref(X, D)
+    bad = ref["idx"].copy()
+    # swap the pick of vector 2 at step 4 for a clearly worse atom
+    bad[2, 4] = (bad[2, 4] + 17) % D.shape[0]
+    words = oracle.pack_words(bad, oracle.store_coef_fp16(ref["coef"]))
+    c = oracle.certify_codes(X, D, words)
+    assert not c["ok_pick"][2, 4]
+
+
+def test_certificate_rejects_wrong_coefficient():
+    D, X = _setup(2)
+    ref = oracle.encode_ref(X, D)
+    coef = ref["coef"].copy()
+    coef[1, 3] *= 1.01
+    words = oracle.pack_words(ref["idx"], oracle.store_coef_fp16(coef))
+    c = oracle.certify_codes(X, D, words)
+    assert not c["ok_coef"][1, 3]
+    assert c["ok_pick"].all()
