@@ -1,0 +1,579 @@
+"""Benchmark of the dictionary-coded KV cache hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sdk|reference]
+                    [--workload layer4k|decode256k|decode32k_b4|prefill256k_vec]
+
+Default workload 'layer4k' (one Llama-3.1-8B attention layer, batch 1, 32 q /
+8 KV heads, d=128, 32768-atom bf16 K and V dictionaries, 4096 tokens): one
+step is the whole hot path on that layer -- greedy-pursuit encode of all
+4096 x 8 x 2 = 65,536 K/V vectors written into the code store (sdk_append),
+then one decode-attention step over the 4096 tokens (sdk_decode_attn).
+'decode256k' / 'decode32k_b4' time a 32-layer decode step, 'prefill256k_vec'
+the encode of 262,144 vectors.
+
+Timing: W untimed warm-up steps, then K steps, each timed with CUDA events on
+the launching stream; the L2 is flushed (256 MiB memset) between steps,
+outside the events.  Multi-GPU (torchrun): every rank runs its own
+independent copy of the workload (weak scaling, no collective on the data
+path); the time is the max over ranks.  Rank 0 prints one JSON line.
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("decode ctx tokens/s/step & encoded KV vecs/s (1 B200), "
+          "% HBM/tensor roofline")
+ENC_FLOP_PER_VEC_PER_ATOM_STEP = 2  # one multiply-add per (atom, dim)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="sdk", choices=["sdk", "reference"])
+    ap.add_argument("--workload", default="layer4k",
+                    choices=["layer4k", "decode256k", "decode32k_b4",
+                             "prefill256k_vec"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return dict(hbm=j["hbm_gbs"], bf16=j["bf16_tflops"],
+                    bf16_sus=j["bf16_tflops_sustained"],
+                    sm_max=j.get("sm_max_mhz", 1965.0), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, sm_max=1965.0,
+                src="fallback")
+
+
+# ----------------------------------------------------------------- clocks
+
+class Clocks:
+    """nvidia-smi samples (200 ms) of one GPU while the timed region runs."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                smax.append(float(f[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------- distributed
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "sdk":
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif args.impl == "sdk":
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ helpers
+
+def timed_steps(step, steps, warmup, flush, world, clocks=None):
+    """Runs warm-up steps, then `steps` steps each between CUDA events on
+    the current stream with an L2 flush before each (outside the events).
+    Returns (per-step ms list, total device ms)."""
+    import torch
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+    evs = []
+    for _ in range(steps):
+        flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        step()
+        b.record()
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ck = clocks.stop() if clocks else None
+    ms = [a.elapsed_time(b) for a, b in evs]
+    return ms, ck
+
+
+def make_flush():
+    import torch
+    buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def flush():
+        buf.zero_()
+    return flush
+
+
+def union_bytes(sdk, ws_list, lay, B, Hq, Hkv, N, k, full):
+    """Algorithmic code bytes of one decode layer from the selected sets in
+    the workspaces: 12 B per token per KV head (Klow scan) + 52 B per token
+    of the GQA-group union U (Khigh rescore beyond the first 3 words) + 64 B
+    per value code read (U, or every token with the full-softmax flag)."""
+    import torch
+    g = Hq // Hkv
+    total = 0
+    usum = 0
+    for ws in ws_list:
+        lst = ws[lay["list"]:lay["list"] + B * Hq * N * 4].view(torch.int32)
+        lst = lst.view(B, Hkv, g, N)[..., :k].long()
+        mark = torch.zeros(B, Hkv, N, dtype=torch.bool, device=lst.device)
+        mark.scatter_(2, lst.reshape(B, Hkv, g * k), True)
+        U = int(mark.sum())
+        usum += U
+        total += 12 * N * B * Hkv + 52 * U + (64 * N * B * Hkv if full else 64 * U)
+    return total, usum
+
+
+# ---------------------------------------------------------- workloads
+
+def bench_layer4k(args, world, rank, pk):
+    import torch
+    import workloads
+    import sparse_dictionary_coded_b200 as sdk
+    w = workloads.layer4k(device="cuda")
+    d, n, N, Hkv, Hq = w["d"], w["n_atoms"], w["n_tokens"], w["Hkv"], w["Hq"]
+    if rank:
+        # every rank encodes its own independent sequence (weak scaling)
+        w["xk"] = torch.roll(w["xk"], shifts=rank * 7, dims=2).contiguous()
+        w["xv"] = torch.roll(w["xv"], shifts=rank * 7, dims=2).contiguous()
+    DK, DV, xk, xv = w["DK"], w["DV"], w["xk"], w["xv"]
+    q = (w["q"] / w["q"].norm(dim=-1, keepdim=True)).contiguous()
+    store = sdk.CodeStore(1, Hkv, N)
+    aws = sdk.new_workspace(sdk.sdk_append_workspace_bytes(1, Hkv, N, d, n))
+    dws = sdk.new_workspace(sdk.sdk_decode_workspace_bytes(1, Hq, d, n, N))
+    out = torch.empty(1, Hq, d, device="cuda")
+    n_vec = 2 * Hkv * N
+    ev = {"enc": [], "dec": []}
+
+    def step(record=False):
+        store.lens = [0]
+        if record:
+            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            e0.record()
+        sdk.sdk_append(store, xk, xv, DK, DV, workspace=aws)
+        if record:
+            e1.record()
+        sdk.sdk_decode_attn(q, DK, DV, store, out=out, workspace=dws)
+        if record:
+            e2.record()
+            ev["enc"].append((e0, e1))
+            ev["dec"].append((e1, e2))
+
+    flush = make_flush()
+    clocks = Clocks(torch.cuda.current_device())
+    ms, ck = timed_steps(lambda: step(True), args.steps, args.warmup, flush,
+                         world, clocks)
+    ev["enc"] = ev["enc"][args.warmup:]
+    ev["dec"] = ev["dec"][args.warmup:]
+    rc, hdr = sdk.sdk_check_status(aws)
+    assert rc == 0, "device check failed in append"
+    rc, _ = sdk.sdk_check_status(dws)
+    assert rc == 0, "device check failed in decode"
+    enc_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["enc"])
+    dec_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["dec"])
+    step_ms = max_over_ranks(statistics.mean(ms), world)
+    lay = sdk.sdk_decode_layout_of(1, Hq, d, n, N)
+    k = (N + 9) // 10
+    dec_bytes, U = union_bytes(sdk, [dws], lay, 1, Hq, Hkv, N, k, False)
+    dec_bytes += 2 * n * d * 2
+    flops = n_vec * 2 * n * d * 16
+    enc_bound = "alu"
+    # CUDA-core fp32 FMA peak: 148 SMs x 128 lanes x 2 flop x max clock
+    alu_peak = 148 * 128 * 2 * pk["sm_max"] * 1e6 / 1e12
+    enc_tflops = flops / (enc_ms * 1e-3) / 1e12
+    res = {
+        "value": world * n_vec / (step_ms * 1e-3),
+        "unit": "encoded KV vecs/s (whole step: encode+append 65,536 vectors, "
+                "then one decode step over 4096 tokens)",
+        "ms_per_step": step_ms,
+        "encode": {"value": n_vec / (enc_ms * 1e-3), "unit": "vecs/s",
+                   "ms": enc_ms, "tflops": enc_tflops},
+        "decode": {"value": N / (dec_ms * 1e-3), "unit": "ctx tokens/s/step",
+                   "ms": dec_ms, "alg_bytes": dec_bytes, "union_tokens": U,
+                   "gbs": dec_bytes / (dec_ms * 1e-3) / 1e9,
+                   "frac_hbm": dec_bytes / (dec_ms * 1e-3) / 1e9 / pk["hbm"]},
+        "roofline": {"bound": enc_bound, "kernel": "encode (sdk_append)",
+                     "achieved": enc_tflops, "peak": alu_peak,
+                     "unit": "TFLOP/s", "frac": enc_tflops / alu_peak,
+                     "traffic": None,
+                     "peak_note": "fp32 FMA: 148 SMs x 128 lanes x 2 x "
+                                  "%.0f MHz" % pk["sm_max"]},
+        "clocks": ck,
+        "config": {"workload": "layer4k", "B": 1, "Hq": Hq, "Hkv": Hkv,
+                   "head_dim": d, "n_atoms": n, "n_tokens": N, "k_atoms": 16,
+                   "klow": 3, "khigh": 16, "top": "1/10",
+                   "l2": "flushed between steps (256 MiB memset outside the "
+                         "per-step events)"},
+        "dtype": "f32 (bf16 dictionaries, fp16 coefficients)",
+        # kernels per step: append = 2 x (encode + scatter); decode = 8
+        "gpu_launches": args.steps * (4 + 8),
+        "enc_fallback_rows": hdr[2],
+    }
+    if not args.no_e2e:
+        res["e2e"] = e2e_layer4k(args, sdk, store, aws, dws, xk, xv, q, DK, DV,
+                                 out, world, n_vec)
+    return res
+
+
+def e2e_layer4k(args, sdk, store, aws, dws, xk, xv, q, DK, DV, out, world,
+                n_vec):
+    """Same step through the public API with inputs copied from pinned host
+    memory every step and the decode output read back."""
+    import torch
+    hxk = xk.cpu().pin_memory()
+    hxv = xv.cpu().pin_memory()
+    hq = q.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dxk, dxv, dq = torch.empty_like(xk), torch.empty_like(xv), torch.empty_like(q)
+
+    def step():
+        dxk.copy_(hxk, non_blocking=True)
+        dxv.copy_(hxv, non_blocking=True)
+        dq.copy_(hq, non_blocking=True)
+        store.lens = [0]
+        sdk.sdk_append(store, dxk, dxv, DK, DV, workspace=aws)
+        sdk.sdk_decode_attn(dq, DK, DV, store, out=out, workspace=dws)
+        hout.copy_(out, non_blocking=True)
+
+    flush = make_flush()
+    ms, _ = timed_steps(step, max(2, args.steps // 2), 1, flush, world)
+    t = max_over_ranks(statistics.mean(ms), world)
+    return {"value": world * n_vec / (t * 1e-3), "unit": "encoded KV vecs/s",
+            "h2d_bytes_per_step": hxk.numel() * 4 + hxv.numel() * 4 + hq.numel() * 4,
+            "d2h_bytes_per_step": hout.numel() * 4, "ms_per_step": t}
+
+
+def bench_decode(args, world, rank, pk, name):
+    import torch
+    import workloads
+    import sparse_dictionary_coded_b200 as sdk
+    W = workloads.WORKLOADS[name]
+    L, B, Hq, Hkv, d, n, N = (W["L"], W["B"], W["Hq"], W["Hkv"], W["d"],
+                              W["n_atoms"], W["n_tokens"])
+    layers = []
+    for l in range(L):
+        lay = workloads.decode_layer(name, l + 1000 * rank, device="cuda")
+        k_lo, k_full, v_full = workloads.layout(lay["kwords"], lay["vwords"])
+        del lay["kwords"], lay["vwords"]
+        store = sdk.CodeStore.from_tensors(k_lo, k_full, v_full, [N] * B)
+        q = (lay["q"] / lay["q"].norm(dim=-1, keepdim=True)).contiguous()
+        ws = sdk.new_workspace(sdk.sdk_decode_workspace_bytes(B, Hq, d, n, N))
+        layers.append(dict(DK=lay["DK"], DV=lay["DV"], store=store, q=q, ws=ws,
+                           out=torch.empty(B, Hq, d, device="cuda")))
+    torch.cuda.synchronize()
+
+    def step():
+        for ly in layers:
+            sdk.sdk_decode_attn(ly["q"], ly["DK"], ly["DV"], ly["store"],
+                                out=ly["out"], workspace=ly["ws"])
+
+    # capture the 32 layer calls in one CUDA graph
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    flush = make_flush()
+    clocks = Clocks(torch.cuda.current_device())
+    ms, ck = timed_steps(g.replay, args.steps, args.warmup, flush, world, clocks)
+    # serialised-layer variant without the graph, for reference
+    ms_nog, _ = timed_steps(step, max(2, args.steps // 2), 1, flush, world)
+    for ly in layers:
+        rc, _ = sdk.sdk_check_status(ly["ws"])
+        assert rc == 0, "device check failed in decode"
+    step_ms = max_over_ranks(statistics.mean(ms), world)
+    lay = sdk.sdk_decode_layout_of(B, Hq, d, n, N)
+    k = (N + 9) // 10
+    code_bytes, U = union_bytes(sdk, [ly["ws"] for ly in layers], lay, B, Hq,
+                                Hkv, N, k, False)
+    alg = code_bytes + L * 2 * n * d * 2
+    gbs = alg / (step_ms * 1e-3) / 1e9
+    return {
+        "value": world * B * N / (step_ms * 1e-3),
+        "unit": "ctx tokens/s/step (%d layers)" % L,
+        "ms_per_step": step_ms,
+        "ms_per_step_no_graph": statistics.mean(ms_nog),
+        "roofline": {"bound": "hbm", "kernel": "decode step (all kernels, "
+                     "%d layers)" % L, "achieved": gbs, "peak": pk["hbm"],
+                     "unit": "GB/s", "frac": gbs / pk["hbm"],
+                     "traffic": None, "alg_bytes_per_step": alg,
+                     "union_tokens_per_step": U},
+        "clocks": ck,
+        "config": {"workload": name, "layers": L, "B": B, "Hq": Hq,
+                   "Hkv": Hkv, "head_dim": d, "n_atoms": n, "n_tokens": N,
+                   "klow": 3, "khigh": 16, "top": "1/10",
+                   "l2": "flushed between steps; codes (%.1f GB) exceed L2"
+                         % (L * B * Hkv * N * 140 / 1e9)},
+        "dtype": "f32 (bf16 dictionaries, fp16 coefficients)",
+        "gpu_launches": args.steps * L * 8,
+    }
+
+
+def bench_prefill(args, world, rank, pk):
+    import torch
+    import workloads
+    import sparse_dictionary_coded_b200 as sdk
+    w = workloads.prefill(device="cuda")
+    d, n = w["d"], w["n_atoms"]
+    xk = w["xk"].reshape(-1, d)
+    xv = w["xv"].reshape(-1, d)
+    if rank:
+        xk, xv = xv.flip(0).contiguous(), xk.flip(0).contiguous()
+    nv = xk.shape[0]
+    ck_ = torch.empty(nv, 16, dtype=torch.int32, device="cuda")
+    cv_ = torch.empty(nv, 16, dtype=torch.int32, device="cuda")
+    ws = sdk.new_workspace(sdk.sdk_encode_workspace_bytes(nv, d, n))
+
+    def step():
+        sdk.sdk_encode(xk, w["DK"], codes=ck_, workspace=ws)
+        sdk.sdk_encode(xv, w["DV"], codes=cv_, workspace=ws)
+
+    flush = make_flush()
+    clocks = Clocks(torch.cuda.current_device())
+    ms, ck = timed_steps(step, args.steps, args.warmup, flush, world, clocks)
+    rc, hdr = sdk.sdk_check_status(ws)
+    assert rc == 0
+    step_ms = max_over_ranks(statistics.mean(ms), world)
+    flops = 2 * nv * 2 * n * d * 16
+    tfl = flops / (step_ms * 1e-3) / 1e12
+    alu_peak = 148 * 128 * 2 * pk["sm_max"] * 1e6 / 1e12
+    return {
+        "value": world * 2 * nv / (step_ms * 1e-3), "unit": "encoded KV vecs/s",
+        "ms_per_step": step_ms,
+        "roofline": {"bound": "alu", "kernel": "encode", "achieved": tfl,
+                     "peak": alu_peak, "unit": "TFLOP/s",
+                     "frac": tfl / alu_peak, "traffic": None},
+        "clocks": ck,
+        "config": {"workload": "prefill256k_vec", "n_vectors": 2 * nv,
+                   "head_dim": d, "n_atoms": n, "k_atoms": 16,
+                   "l2": "flushed between steps"},
+        "dtype": "f32 (bf16 dictionaries)",
+        "gpu_launches": args.steps * 2,
+        "enc_fallback_rows": hdr[2],
+    }
+
+
+# ------------------------------------------------------ oracle timings
+
+def cpu_baseline(name, budget_s=15.0):
+    """The fp64 oracle on this host's cores, on a bounded sample of the
+    workload, scaled to the metric's unit."""
+    import numpy as np
+    import torch
+    import oracle
+    import workloads
+    cores = len(os.sched_getaffinity(0))
+    torch.set_num_threads(cores)
+    if name in ("layer4k", "prefill256k_vec"):
+        if name == "layer4k":
+            w = workloads.layer4k()
+            x = w["xk"].reshape(-1, w["d"])
+            D = w["DK"]
+            per_step = 2 * w["Hkv"] * w["n_tokens"]
+        else:
+            w = workloads.prefill(n_tokens=64)
+            x = w["xk"].reshape(-1, w["d"])
+            D = w["DK"]
+            per_step = 2 * 8 * 16384
+        Dn = D.float().double().numpy()
+        xs = x.double().numpy()
+        t0 = time.perf_counter()
+        nvec = 0
+        while time.perf_counter() - t0 < budget_s * 0.8 and nvec < xs.shape[0]:
+            oracle.encode_ref(xs[nvec:nvec + 4], Dn)
+            nvec += 4
+        t_enc = (time.perf_counter() - t0) / nvec
+        sample = "%d vectors encoded by the oracle" % nvec
+        t_step = t_enc * per_step
+        if name == "layer4k":
+            # plus one decode head over 4096 tokens (x32 heads)
+            g = workloads.make_gen(5)
+            kw = workloads.random_codes((4096,), 32768, g).numpy().view(np.uint32)
+            vw = workloads.random_codes((4096,), 32768, g).numpy().view(np.uint32)
+            qh = np.random.default_rng(0).standard_normal(128)
+            t1 = time.perf_counter()
+            oracle.decode_head_ref(qh, kw, vw, Dn, Dn)
+            t_dec = (time.perf_counter() - t1) * 32
+            t_step += t_dec
+            sample += " + 1 of 32 decode heads (4096 tokens)"
+        return {"value": per_step / t_step, "unit": "encoded KV vecs/s",
+                "cores": cores, "kind": "oracle",
+                "sample": sample + "; extrapolated to the full step"}
+    # decode workloads: one head of one layer, x (L*B*Hq)
+    W = workloads.WORKLOADS[name]
+    lay = workloads.decode_layer(name, 0, B=1)
+    kw = lay["kwords"][0, 0].numpy().view(np.uint32)
+    vw = lay["vwords"][0, 0].numpy().view(np.uint32)
+    qn = lay["q"][0, 0].double().numpy()
+    Dk = lay["DK"].float().double().numpy()
+    Dv = lay["DV"].float().double().numpy()
+    t0 = time.perf_counter()
+    oracle.decode_head_ref(qn, kw, vw, Dk, Dv)
+    t_head = time.perf_counter() - t0
+    t_step = t_head * W["L"] * W["B"] * W["Hq"]
+    return {"value": W["B"] * W["n_tokens"] / t_step,
+            "unit": "ctx tokens/s/step", "cores": cores, "kind": "oracle",
+            "sample": "1 query head of 1 layer (%d tokens), extrapolated x%d"
+                      % (W["n_tokens"], W["L"] * W["B"] * W["Hq"])}
+
+
+def reference_arm(args):
+    """The oracle as the reference implementation, timed on the host cores
+    with the same metric, unit and config as the sdk arm."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    name = args.workload
+    vals = []
+    for _ in range(args.warmup):
+        pass
+    t0 = time.perf_counter()
+    for _ in range(max(1, args.steps)):
+        vals.append(cpu_baseline(name, budget_s=min(20.0, 120.0 / max(1, args.steps))))
+    wall = time.perf_counter() - t0
+    v = statistics.mean(x["value"] for x in vals)
+    cb = dict(vals[0])
+    cb["value"] = v
+    line = {"impl": "reference", "metric": METRIC, "value": v,
+            "unit": vals[0]["unit"], "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": wall * 1e3 / max(1, args.steps),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": {"workload": name}, "cpu_baseline": cb,
+            "e2e": {"value": v, "unit": vals[0]["unit"],
+                    "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        reference_arm(args)
+        return
+    import torch
+    world, rank, local = dist_setup(args)
+    import sparse_dictionary_coded_b200 as sdk
+    sdk.load()
+    pk = peaks()
+    if args.workload == "layer4k":
+        res = bench_layer4k(args, world, rank, pk)
+    elif args.workload == "prefill256k_vec":
+        res = bench_prefill(args, world, rank, pk)
+    else:
+        res = bench_decode(args, world, rank, pk, args.workload)
+    if rank == 0:
+        line = {"metric": METRIC, "value": res.pop("value"),
+                "unit": res.pop("unit"), "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": res.pop("ms_per_step"),
+                "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": res.pop("dtype"),
+                "data": "synthetic (seeded; shapes of the Llama-3.1-8B KV "
+                        "workloads, no model or dataset)"}
+        line.update(res)
+        line["roofline"]["peak_source"] = pk["src"]
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(args.workload)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

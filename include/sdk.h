@@ -1,0 +1,259 @@
+/*
+ * sdk.h -- dictionary-coded KV cache, encode and decode-attention hot path
+ *          for NVIDIA B200 (sm_100a).  C ABI of libsdk.so.
+ *
+ * Method: "LLM Inference in a Flash!" (Zhao, Kim, Hooper, Manolache, Mahoney,
+ * Shao, Keutzer, Gholami).  The evolve.pub review of the paper, section
+ * "Summary", and its FAQ entry "What is the 15x KV cache compression ..."
+ * describe what is computed here:
+ *   - every key and value vector is stored as K=16 (atom index, coefficient)
+ *     pairs over a static, per-layer, per-stream (key or value) overcomplete
+ *     dictionary of 32,768 atoms;
+ *   - the encoder is a projection-based greedy pursuit replacing OMP, so no
+ *     least-squares refit is done;
+ *   - decoding uses query-aware hierarchical sparsity: every token is scored
+ *     from Klow=3 atoms, the top 10% are refined with Khigh=16 atoms.
+ * The authors' abstract (readsearch.ai listing) states the goal: represent
+ * each KV vector as a linear combination of static dictionary vectors.
+ *
+ * Conventions for every entry point
+ *   - Pointers marked "device" are CUDA device pointers (or managed memory)
+ *     owned by the caller; pointers marked "host" are host memory read
+ *     during the call only.  The library allocates nothing.
+ *   - Calls are stream-ordered and asynchronous on `stream` (NULL = the
+ *     legacy default stream).  Host-side argument checks return an error
+ *     BEFORE anything is launched; a launch failure returns SDK_ERR_CUDA.
+ *   - Conditions found on the device (an atom index >= n_atoms, an
+ *     inconsistent selection count) are recorded in the workspace header and
+ *     read by sdk_check_status(); no kernel traps.
+ *   - Thread safety: concurrent calls must use distinct workspaces.
+ *   - Tensors are dense, row-major, with no padding between rows.
+ *
+ * Code word (32 bits): bits 31..16 = fp16 bits of the coefficient (round to
+ * nearest even, saturated to +-65504), bit 15 = 0, bits 14..0 = atom index.
+ *
+ * Code store of one layer (capacity `cap` tokens per sequence):
+ *   k_lo   uint32 [B][Hkv][3][cap]  words 0..2 (greedy order) of every key
+ *                                   code, one plane per word: the Klow scan
+ *                                   reads 12 bytes per token, coalesced.
+ *   k_full uint32 [B][Hkv][cap][16] all 16 words of every key code: one
+ *                                   64-byte record per token for the
+ *                                   Khigh rescore of selected tokens.
+ *   v_full uint32 [B][Hkv][cap][16] all 16 words of every value code.
+ * Query head h of a sequence reads KV head h / (Hq / Hkv).
+ */
+#ifndef SDK_H
+#define SDK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SDK_API __attribute__((visibility("default")))
+#else
+#define SDK_API
+#endif
+
+/* A cudaStream_t, declared without including the CUDA headers. */
+typedef struct CUstream_st* sdk_stream_t;
+
+typedef enum {
+  SDK_OK = 0,
+  SDK_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned buffer */
+  SDK_ERR_UNSUPPORTED = 2,   /* valid but outside what is built (head_dim) */
+  SDK_ERR_CAPACITY = 3,      /* append past `cap`, workspace too small     */
+  SDK_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed       */
+  SDK_ERR_TIMEOUT = 5,       /* a bounded device wait gave up              */
+  SDK_ERR_DEVICE_CHECK = 6   /* a device-side check failed (bad atom index) */
+} sdk_status;
+
+typedef enum { SDK_F32 = 0, SDK_BF16 = 1 } sdk_dtype;
+
+#define SDK_MAX_ATOMS 32768   /* 15-bit atom index                         */
+#define SDK_K_ATOMS 16        /* atoms per stored code                     */
+#define SDK_KLOW_PLANES 3     /* words kept in the k_lo planes             */
+#define SDK_MAX_BATCH 64      /* sequences per decode / append call        */
+#define SDK_WS_ALIGN 256      /* required alignment of workspaces (bytes)  */
+
+/* Human-readable name of a status code (static string, never NULL). */
+SDK_API const char* sdk_status_string(int status);
+
+/* Library ABI version (incremented on any signature change). */
+SDK_API int32_t sdk_version(void);
+
+/* ------------------------------------------------------------------ encode
+ * Greedy pursuit ("LLM Inference in a Flash!", review Summary): for every
+ * input vector x, r = x; 16 times: i* = argmax_i |<r, d_i>| (ties: lowest
+ * i), coef = <r, d_i*>, r -= coef * d_i*.  The pick is made exactly in
+ * fp32: candidate atoms come from a bf16 tensor-core correlation GEMM with
+ * fp32 accumulation, and every atom that can be the fp32 argmax within the
+ * rounding bound of that GEMM is re-scored in fp32 before the pick.
+ *
+ *   x           device, [n_vec][head_dim], fp32 or bf16 (x_dtype)
+ *   n_vec       number of vectors, >= 0 (0 launches nothing)
+ *   head_dim    64 or 128
+ *   dict        device, bf16 [n_atoms][head_dim], unit-norm rows expected
+ *               (used as given), 16-byte aligned
+ *   n_atoms     1 .. 32768
+ *   k_atoms     1 .. 16 picks per vector
+ *   codes_out   device, uint32 [n_vec][k_atoms], words in pick order
+ *   resid_sqnorm_out  device, float [n_vec] = ||r_final||^2, or NULL
+ *   workspace   device, >= sdk_encode_workspace_bytes(), 256-byte aligned,
+ *               initialised once by sdk_workspace_init()
+ * Errors: SDK_ERR_INVALID_ARG (null/misaligned pointers, sizes out of
+ * range), SDK_ERR_UNSUPPORTED (head_dim), SDK_ERR_CAPACITY (ws_bytes too
+ * small), SDK_ERR_CUDA.
+ */
+SDK_API sdk_status sdk_encode(const void* x, int32_t x_dtype, int64_t n_vec,
+                      int32_t head_dim, const void* dict, int32_t n_atoms,
+                      int32_t k_atoms, uint32_t* codes_out,
+                      float* resid_sqnorm_out, void* workspace,
+                      size_t ws_bytes, sdk_stream_t stream);
+
+/* Same contract as sdk_encode, computed by the plain CUDA-core kernel:
+ * every correlation in fp32 FMA order k = 0..head_dim-1, exact argmax over
+ * all atoms.  A second, independent GPU path for cross-checks and for
+ * head_dim / n_atoms the tensor-core kernel does not take. */
+SDK_API sdk_status sdk_encode_simt(const void* x, int32_t x_dtype, int64_t n_vec,
+                           int32_t head_dim, const void* dict,
+                           int32_t n_atoms, int32_t k_atoms,
+                           uint32_t* codes_out, float* resid_sqnorm_out,
+                           void* workspace, size_t ws_bytes,
+                           sdk_stream_t stream);
+
+SDK_API size_t sdk_encode_workspace_bytes(int64_t n_vec, int32_t head_dim,
+                                  int32_t n_atoms);
+
+/* ------------------------------------------------------------------ append
+ * Encode n_new new key and value vectors per (sequence, KV head) and write
+ * them into the code store at token positions [lens[b], lens[b] + n_new).
+ * The review's FAQ describes the store: compact per-token codes referencing
+ * a fixed dictionary, appended at every generated token while the
+ * dictionary stays static.
+ *
+ *   xk, xv      device, [B][Hkv][n_new][head_dim], fp32 or bf16
+ *   dict_k/_v   device, bf16 [n_atoms][head_dim]
+ *   k_lo, k_full, v_full  device, the code store (layout above)
+ *   cap         capacity in tokens per sequence
+ *   lens_host   host, int32 [B]: current lengths; lens[b] + n_new <= cap.
+ *               The library does not update it.
+ * Errors: as sdk_encode, plus SDK_ERR_CAPACITY when lens[b] + n_new > cap.
+ */
+SDK_API sdk_status sdk_append(const void* xk, const void* xv, int32_t x_dtype,
+                      int32_t B, int32_t Hkv, int32_t n_new, int32_t head_dim,
+                      const void* dict_k, const void* dict_v, int32_t n_atoms,
+                      uint32_t* k_lo, uint32_t* k_full, uint32_t* v_full,
+                      int64_t cap, const int32_t* lens_host, void* workspace,
+                      size_t ws_bytes, sdk_stream_t stream);
+
+SDK_API size_t sdk_append_workspace_bytes(int32_t B, int32_t Hkv, int32_t n_new,
+                                  int32_t head_dim, int32_t n_atoms);
+
+/* ------------------------------------------------------------ decode attn
+ * One layer of decode attention for B sequences over their code stores
+ * (review Summary: score all tokens at Klow=3, refine the top 10% at
+ * Khigh=16).  Per query head (b, h), with N = lens[b]:
+ *   QD      = D_K q                       (all n_atoms correlations)
+ *   s_lo_t  = sum_{j<klow} c_tj QD[idx_tj]           for every token t
+ *   S       = the k = ceil(top_num*N/top_den) tokens with the largest s_lo
+ *             (ties: lower token index)
+ *   s_t     = scale * sum_{j<khigh} c_tj QD[idx_tj]  for t in S
+ *   p       = softmax of s over S; with full_softmax != 0 the softmax runs
+ *             over all N tokens, t outside S using scale * s_lo_t
+ *   w[a]    = sum_t p_t sum_j c^V_tj [idx^V_tj == a] (over the softmax domain)
+ *   out     = w D_V
+ *
+ *   q          device, float [B][Hq][head_dim]
+ *   dict_k/_v  device, bf16 [n_atoms][head_dim]
+ *   lens_host  host, int32 [B], 1 <= lens[b] <= cap
+ *   klow       1 .. khigh;  khigh  klow .. 16
+ *   top_num, top_den   0 < top_num <= top_den
+ *   scale      logit scale (1/sqrt(head_dim) for standard attention)
+ *   out        device, float [B][Hq][head_dim]
+ *   workspace  device, >= sdk_decode_workspace_bytes(B, Hq, head_dim,
+ *              n_atoms, max_len) with max_len >= every lens[b]
+ * Limits: B <= 64, Hq % Hkv == 0, head_dim in {64, 128}, B*Hq <= 2048,
+ *         scale > 0.
+ */
+SDK_API sdk_status sdk_decode_attn(const float* q, int32_t B, int32_t Hq, int32_t Hkv,
+                           int32_t head_dim, const void* dict_k,
+                           const void* dict_v, int32_t n_atoms,
+                           const uint32_t* k_lo, const uint32_t* k_full,
+                           const uint32_t* v_full, int64_t cap,
+                           const int32_t* lens_host, int32_t klow,
+                           int32_t khigh, int32_t top_num, int32_t top_den,
+                           int32_t full_softmax, float scale, float* out,
+                           void* workspace, size_t ws_bytes,
+                           sdk_stream_t stream);
+
+SDK_API size_t sdk_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t head_dim,
+                                  int32_t n_atoms, int64_t max_len);
+
+/* Byte offsets of the decode workspace regions, for inspection by tests
+ * and tools after a call (contents are valid until the next call using the
+ * same workspace).  R = B*Hq query heads, L = max_len. */
+typedef struct {
+  size_t header;     /* 256-byte status header                            */
+  size_t qd;         /* float  [R][n_atoms]   QD = D_K q                  */
+  size_t keys;       /* uint32 [R][L]  order-preserving keys of s_lo      */
+  size_t hist1;      /* uint32 [R][4096] histogram of key bits 31..20     */
+  size_t hist2;      /* uint32 [R][4096] bits 19..8 inside the bucket     */
+  size_t state;      /* sdk_select_state [R]                              */
+  size_t list;       /* int32  [R][L]  the selected tokens at the front
+                        (unordered); with full_softmax the other tokens
+                        fill the back                                     */
+  size_t cand_t;     /* int32  [R][L]  tokens inside the pass-1 bucket    */
+  size_t cand_key;   /* uint32 [R][L]  their keys                         */
+  size_t sel_score;  /* float  [R][L]  s_t of list[r][i], i < k           */
+  size_t w;          /* float  [R][n_atoms] unnormalised per-atom weights */
+  size_t part;       /* float  partial sums of w D_V                      */
+  size_t total;      /* total bytes                                       */
+} sdk_decode_layout;
+
+/* Per-head selection state in the decode workspace (region `state`).
+ * Keys map a float score s to a uint32 whose unsigned order is the order
+ * of s (+0 and -0 map to the same key). */
+typedef struct {
+  uint32_t kth_key;    /* key of the k-th largest s_lo                     */
+  uint32_t k;          /* selected-set size                                */
+  uint32_t n_above;    /* tokens above the pass-1 bucket                   */
+  uint32_t n_cand;     /* tokens inside the pass-1 bucket                  */
+  uint32_t n_sel;      /* entries written at the front of `list`           */
+  uint32_t n_comp;     /* entries written at the back of `list`            */
+  uint32_t eq_total;   /* tokens with key == kth_key                       */
+  uint32_t eq_taken;   /* how many of those are in the selected set        */
+  uint32_t max_score;  /* key of max s_t over the selected set             */
+  uint32_t max_comp;   /* key of the largest s_lo outside it (0 = none)    */
+  float z;             /* softmax denominator                              */
+  uint32_t pad[5];
+} sdk_select_state;
+
+SDK_API sdk_status sdk_decode_layout_of(int32_t B, int32_t Hq, int32_t head_dim,
+                                int32_t n_atoms, int64_t max_len,
+                                sdk_decode_layout* layout_out /* host */);
+
+/* ------------------------------------------------------------ workspaces
+ * Every workspace starts with a 256-byte header:
+ *   uint32 [0] status recorded on the device (0 = none; sticky)
+ *   uint32 [1] detail of the first recorded failure (e.g. the bad index)
+ *   uint32 [2] encode: rows that needed the exact fallback scan
+ *   uint32 [3] encode: candidate atoms re-scored in fp32
+ * sdk_workspace_init zeroes the header (stream-ordered); call it once per
+ * new workspace.  sdk_check_status synchronises `stream`, returns the
+ * recorded status (SDK_OK if none) and clears it; `counters_out` (host,
+ * nullable) receives words [0..3] before the clear.
+ */
+SDK_API sdk_status sdk_workspace_init(void* workspace, size_t ws_bytes,
+                              sdk_stream_t stream);
+SDK_API sdk_status sdk_check_status(void* workspace, sdk_stream_t stream,
+                            uint32_t* counters_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDK_H */

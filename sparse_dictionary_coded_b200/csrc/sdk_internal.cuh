@@ -1,0 +1,176 @@
+// Internal helpers shared by the kernels of libsdk.so (not installed).
+//
+// Code word format (review of "LLM Inference in a Flash!", FAQ on the 15x
+// KV compression: each vector is stored as the indices and coefficients of
+// its 16 atoms): bits 31..16 = fp16 coefficient, bit 15 = 0, bits 14..0 =
+// atom index.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/sdk.h"
+
+namespace sdk {
+
+constexpr int kMaxAtoms = SDK_MAX_ATOMS;
+constexpr int kAtoms = SDK_K_ATOMS;
+constexpr int kLoPlanes = SDK_KLOW_PLANES;
+constexpr int kMaxBatch = SDK_MAX_BATCH;
+
+// Header at offset 0 of every workspace (256 bytes).
+struct WsHeader {
+  unsigned int err;          // first recorded sdk_status (0 = none)
+  unsigned int info;         // detail of that failure
+  unsigned int enc_fallback; // encode rows re-scanned exactly
+  unsigned int enc_cands;    // encode candidates re-scored in fp32
+  unsigned int pad[60];
+};
+static_assert(sizeof(WsHeader) == 256, "header size");
+
+__device__ __forceinline__ void record_error(WsHeader* h, unsigned code,
+                                             unsigned info) {
+  if (atomicCAS(&h->err, 0u, code) == 0u) atomicExch(&h->info, info);
+}
+
+// ---- code words -----------------------------------------------------------
+__device__ __forceinline__ uint32_t word_idx(uint32_t w) { return w & 0x7FFFu; }
+__device__ __forceinline__ float word_coef(uint32_t w) {
+  return __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+}
+// fp16 round-to-nearest-even with saturation to +-65504.
+__device__ __forceinline__ uint32_t make_word(float coef, uint32_t idx) {
+  float c = fminf(fmaxf(coef, -65504.0f), 65504.0f);
+  uint32_t hb = (uint32_t)__half_as_ushort(__float2half_rn(c));
+  return (hb << 16) | (idx & 0x7FFFu);
+}
+
+// ---- order-preserving float keys -------------------------------------------
+// Larger key <=> larger score; -0 and +0 share the key of +0.
+__device__ __forceinline__ uint32_t score_key(float s) {
+  uint32_t b = __float_as_uint(s);
+  if ((b << 1) == 0u) b = 0u;  // -0 -> +0
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_score(uint32_t k) {
+  uint32_t b = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+  return __uint_as_float(b);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) {
+  return __uint_as_float(v << 16);
+}
+__device__ __forceinline__ float bf16_hi(uint32_t v) {
+  return __uint_as_float(v & 0xFFFF0000u);
+}
+
+// ---- block-wide helpers (blockDim.x a multiple of 32, <= 1024) -------------
+// Inclusive scan of one uint32 per thread; returns the block total in *total.
+__device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, uint32_t* s_warp,
+                                                    uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint32_t t = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += t;
+  }
+  __syncthreads();
+  if (lane == 31) s_warp[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t t = lane < nw ? s_warp[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      uint32_t u = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += u;
+    }
+    if (lane < nw) s_warp[lane] = t;
+  }
+  __syncthreads();
+  uint32_t base = warp > 0 ? s_warp[warp - 1] : 0u;
+  *total = s_warp[nw - 1];
+  __syncthreads();
+  return base + v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ uint32_t warp_umax(uint32_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+
+// ---- kernel parameter blocks (passed by value) ------------------------------
+// Decode: one layer, B sequences, R = B*Hq query heads.  Per sequence b:
+// lens = tokens, kcnt = selected-set size, dcnt = softmax-domain size;
+// *_off = prefix sums over sequences of Hq * (that count).
+struct DecodeParams {
+  const float* q;
+  const uint16_t* dk;
+  const uint16_t* dv;
+  const uint32_t* k_lo;
+  const uint32_t* k_full;
+  const uint32_t* v_full;
+  float* out;
+  float* qd;
+  uint32_t* keys;
+  uint32_t* hist1;
+  uint32_t* hist2;
+  sdk_select_state* st;
+  int32_t* list;
+  int32_t* cand_t;
+  uint32_t* cand_key;
+  float* sel_score;
+  float* w;
+  float* part;
+  WsHeader* hdr;
+  int64_t cap;
+  int64_t L;
+  int B, Hq, Hkv, g, d, n, klow, khigh, full, R, n_out_tiles;
+  float scale;
+  int lens[kMaxBatch];
+  int kcnt[kMaxBatch];
+  int dcnt[kMaxBatch];
+  int64_t tok_off[kMaxBatch + 1];
+  int64_t sel_off[kMaxBatch + 1];
+  int64_t dom_off[kMaxBatch + 1];
+};
+
+// Encode: n_vec vectors of head_dim over n dictionary atoms, k_atoms picks.
+struct EncodeParams {
+  const void* x;
+  int x_dtype;
+  int64_t n_vec;
+  const uint16_t* dict;
+  int n;
+  int k_atoms;
+  uint32_t* codes;
+  float* rsq;
+  WsHeader* hdr;
+};
+
+int num_sms();  // cached multiprocessor count of the current device
+
+sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream);
+sdk_decode_layout decode_layout(int B, int Hq, int d, int n, int64_t L);
+sdk_status launch_encode_simt(const EncodeParams& p, int head_dim, cudaStream_t stream);
+// Tensor-core encoder; sets *taken = false when it does not handle the
+// shape (the caller then runs the CUDA-core encoder).
+sdk_status launch_encode_tc(const EncodeParams& p, int head_dim, void* scratch,
+                            size_t scratch_bytes, cudaStream_t stream, bool* taken);
+size_t encode_tc_scratch_bytes(int64_t n_vec, int head_dim, int n_atoms);
+
+}  // namespace sdk

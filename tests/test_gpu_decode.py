@@ -1,0 +1,266 @@
+"""GPU parity of decode attention (sdk_decode_attn through the C ABI) against
+the fp64 oracle, on identical codes (oracle-encoded or drawn by the input
+generator; never produced by the CUDA path)."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import sparse_dictionary_coded_b200 as sdk
+from parity import (OUT_TOL, check_selection, words_np)
+
+pytestmark = pytest.mark.gpu
+
+
+def _store(kw, vw, lens=None, cap=None):
+    """Code store on the GPU from [B, Hkv, N, 16] int32 word tensors."""
+    k_lo, k_full, v_full = workloads.layout(kw, vw, cap)
+    B = kw.shape[0]
+    lens = [kw.shape[2]] * B if lens is None else lens
+    return sdk.CodeStore.from_tensors(k_lo.cuda(), k_full.cuda(),
+                                      v_full.cuda(), lens)
+
+
+def _unit(q):
+    return q / q.norm(dim=-1, keepdim=True)
+
+
+def _run(q, DK, DV, store, **kw):
+    B, Hq, d = q.shape
+    ws = sdk.new_workspace(sdk.sdk_decode_workspace_bytes(
+        B, Hq, d, DK.shape[0], max(store.lens)))
+    out = sdk.sdk_decode_attn(q.cuda(), DK.cuda(), DV.cuda(), store,
+                              workspace=ws, **kw)
+    torch.cuda.synchronize()
+    rc, hdr = sdk.sdk_check_status(ws)
+    lay = sdk.sdk_decode_layout_of(B, Hq, d, DK.shape[0], max(store.lens))
+    return out.cpu().double().numpy(), ws, lay, rc
+
+
+def _gpu_sets(ws, lay, R, L, ks):
+    lst = ws[lay["list"]:lay["list"] + R * L * 4].view(torch.int32)
+    lst = lst.view(R, L).cpu().numpy()
+    return [lst[r, :ks[r]] for r in range(R)]
+
+
+def _gpu_keys(ws, lay, R, L):
+    k = ws[lay["keys"]:lay["keys"] + R * L * 4].view(torch.int32)
+    return k.view(R, L).cpu().numpy().view(np.uint32)
+
+
+def _key_to_float(keys):
+    keys = keys.astype(np.uint32)
+    neg = (keys & 0x80000000) == 0
+    b = np.where(neg, ~keys, keys & 0x7FFFFFFF).astype(np.uint32)
+    return b.view(np.float32)
+
+
+def _compare(q, DK, DV, kw, vw, lens, klow=3, khigh=16, top_num=1, top_den=10,
+             full=False, heads=None):
+    """Runs GPU decode and checks sets, s_lo and outputs against the oracle
+    for the given (b, h) heads (all if None)."""
+    B, Hq, d = q.shape
+    store = _store(kw, vw, lens)
+    out, ws, lay, rc = _run(q, DK, DV, store, klow=klow, khigh=khigh,
+                            top_num=top_num, top_den=top_den,
+                            full_softmax=full)
+    assert rc == 0, "device check failed"
+    L = max(lens)
+    R = B * Hq
+    ks = [oracle.topk_count(lens[r // Hq], top_num, top_den) for r in range(R)]
+    sets = _gpu_sets(ws, lay, R, L, ks)
+    keys = _gpu_keys(ws, lay, R, L)
+    st = sdk.read_select_state(ws, lay, R)
+    qn = q.double().numpy()
+    kwn, vwn = words_np(kw), words_np(vw)
+    DKn, DVn = DK.float().double().numpy(), DV.float().double().numpy()
+    Hkv = kw.shape[1]
+    g = Hq // Hkv
+    ndiff = 0
+    for r in range(R):
+        b, h = divmod(r, Hq)
+        if heads is not None and (b, h) not in heads:
+            continue
+        n_b = lens[b]
+        kvh = h // g
+        assert int(st["n_sel"][r]) == ks[r]
+        ref = oracle.decode_head_ref(qn[b, h], kwn[b, kvh, :n_b],
+                                     vwn[b, kvh, :n_b], DKn, DVn, klow, khigh,
+                                     top_num, top_den, full)
+        # s_lo of the GPU within fp32 rounding of the oracle's
+        s_gpu = _key_to_float(keys[r, :n_b]).astype(np.float64)
+        scale_lo = np.max(np.abs(ref["s_lo"])) + 1e-30
+        assert np.max(np.abs(s_gpu - ref["s_lo"])) <= 1e-5 * scale_lo
+        nd = check_selection(sets[r], ref["s_lo"], ks[r])
+        ndiff += nd
+        if nd:
+            ref = oracle.decode_head_ref(qn[b, h], kwn[b, kvh, :n_b],
+                                         vwn[b, kvh, :n_b], DKn, DVn, klow,
+                                         khigh, top_num, top_den, full,
+                                         force_set=sets[r])
+        err = np.max(np.abs(out[b, h] - ref["out"]))
+        assert err <= OUT_TOL, (b, h, err)
+        if full:
+            assert int(st["n_sel"][r]) + int(st["n_comp"][r]) == n_b
+    return out, ndiff
+
+
+def _random_case(seed, B, Hq, Hkv, N, d, n, lens=None, outliers=0):
+    g = workloads.make_gen(seed)
+    DK = workloads.gaussian_dictionary(n, d, g)
+    DV = workloads.gaussian_dictionary(n, d, g)
+    kw = workloads.random_codes((B, Hkv, N), n, g)
+    vw = workloads.random_codes((B, Hkv, N), n, g)
+    q = _unit(workloads.queries(B, Hq, d, g, n_outlier=outliers))
+    lens = [N] * B if lens is None else lens
+    return q, DK, DV, kw, vw, lens
+
+
+def test_tiny_workload_oracle_encoded_codes():
+    """Workload 'tiny': codes from the oracle's own greedy pursuit."""
+    w = workloads.tiny()
+    d, N = w["d"], w["n_tokens"]
+    DK = w["DK"].float().double().numpy()
+    DV = w["DV"].float().double().numpy()
+    rk = oracle.encode_ref(w["xk"].reshape(N, d).double().numpy(), DK)
+    rv = oracle.encode_ref(w["xv"].reshape(N, d).double().numpy(), DV)
+    kw = oracle.pack_words(rk["idx"], oracle.store_coef_fp16(rk["coef"]))
+    vw = oracle.pack_words(rv["idx"], oracle.store_coef_fp16(rv["coef"]))
+    kw = torch.from_numpy(kw.view(np.int32)).view(1, 1, N, 16)
+    vw = torch.from_numpy(vw.view(np.int32)).view(1, 1, N, 16)
+    q = _unit(w["q"])
+    for full in (False, True):
+        _compare(q, w["DK"], w["DV"], kw, vw, [N], full=full)
+
+
+@pytest.mark.parametrize("full", [False, True])
+def test_layer4k_shape_random_codes(full):
+    """Workload 'layer4k' shape: 32 q / 8 KV heads, d=128, 32768 atoms,
+    4096 tokens (random codes from the input generator)."""
+    q, DK, DV, kw, vw, lens = _random_case(77, 1, 32, 8, 4096, 128, 32768)
+    _compare(q, DK, DV, kw, vw, lens, full=full)
+
+
+def test_ragged_batch_small_and_odd_sizes():
+    """B=3 with lengths 1, 5 and 333 (k = 1, 1, 34), GQA 6/2, d=64, 1000
+    atoms (not a multiple of any tile)."""
+    q, DK, DV, kw, vw, _ = _random_case(5, 3, 6, 2, 333, 64, 1000)
+    lens = [1, 5, 333]
+    for full in (False, True):
+        _compare(q, DK, DV, kw, vw, lens, full=full)
+
+
+def test_dense_special_case_matches_sdpa():
+    """Klow=Khigh=16, top 100%: dense attention over the decoded keys and
+    values, checked against torch SDPA in fp64 on the CPU."""
+    q, DK, DV, kw, vw, lens = _random_case(9, 1, 4, 2, 300, 128, 2048)
+    out, _ = _compare(q, DK, DV, kw, vw, lens, klow=16, khigh=16, top_num=1,
+                      top_den=1)
+    DKn, DVn = DK.double(), DV.double()
+    kwn, vwn = words_np(kw), words_np(vw)
+    for h in range(4):
+        K = torch.from_numpy(oracle.decode_vectors(kwn[0, h // 2], DKn.numpy(), 16))
+        V = torch.from_numpy(oracle.decode_vectors(vwn[0, h // 2], DVn.numpy(), 16))
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q[0, h].double().view(1, 1, 1, -1), K.view(1, 1, 300, -1),
+            V.view(1, 1, 300, -1)).view(-1).numpy()
+        assert np.max(np.abs(out[0, h] - ref)) <= 2e-3
+
+
+@pytest.mark.parametrize("full", [False, True])
+def test_all_tokens_tie(full):
+    """Every token carries the same key code: all s_lo tie, the selected
+    set is the k lowest token indices (tie rule), p is uniform over it."""
+    g = workloads.make_gen(3)
+    n, d, N = 512, 64, 1000
+    DK = workloads.gaussian_dictionary(n, d, g)
+    DV = workloads.gaussian_dictionary(n, d, g)
+    one = workloads.random_codes((1, 1, 1), n, g)
+    kw = one.expand(1, 1, N, 16).contiguous()
+    vw = workloads.random_codes((1, 1, N), n, g)
+    q = _unit(workloads.queries(1, 2, d, g))
+    store = _store(kw, vw)
+    out, ws, lay, rc = _run(q, DK, DV, store, full_softmax=full)
+    assert rc == 0
+    sets = _gpu_sets(ws, lay, 2, N, [100, 100])
+    for r in range(2):
+        assert sorted(sets[r].tolist()) == list(range(100))
+    _compare(q, DK, DV, kw, vw, [N], full=full)
+
+
+def test_partial_ties_at_threshold():
+    """Half the tokens share one code (ties across the k-th score), the rest
+    random: the tie rule takes the lowest indices among the tied tokens."""
+    g = workloads.make_gen(4)
+    n, d, N = 512, 64, 2000
+    DK = workloads.gaussian_dictionary(n, d, g)
+    DV = workloads.gaussian_dictionary(n, d, g)
+    kw = workloads.random_codes((1, 1, N), n, g)
+    kw[0, 0, 1::2] = kw[0, 0, 7]
+    vw = workloads.random_codes((1, 1, N), n, g)
+    q = _unit(workloads.queries(1, 4, d, g))
+    _compare(q, DK, DV, kw, vw, [N])
+    _compare(q, DK, DV, kw, vw, [N], full=True)
+
+
+def test_klow_and_khigh_variants():
+    q, DK, DV, kw, vw, lens = _random_case(12, 2, 8, 4, 700, 128, 4096)
+    _compare(q, DK, DV, kw, vw, lens, klow=1, khigh=8, top_num=1, top_den=4)
+    _compare(q, DK, DV, kw, vw, lens, klow=5, khigh=16, top_num=3, top_den=10)
+
+
+def test_bad_atom_index_is_reported_not_trapped():
+    """Codes naming atom 1500 of a 1000-atom dictionary: the kernels skip
+    the term and record SDK_ERR_DEVICE_CHECK with the index."""
+    q, DK, DV, kw, vw, lens = _random_case(13, 1, 2, 1, 64, 64, 1000)
+    kw[0, 0, 10, 0] = (kw[0, 0, 10, 0] & ~0x7FFF) | 1500
+    store = _store(kw, vw)
+    _, ws, _, rc = _run(q, DK, DV, store)
+    assert rc == 6
+    rc2, _ = sdk.sdk_check_status(ws)
+    assert rc2 == 0                      # cleared by the first read
+
+
+@pytest.mark.parametrize("name", ["decode32k_b4", "decode256k"])
+def test_full_size_layer_sampled_heads(name):
+    """One layer of the full-size decode workloads in the bench's launch
+    configuration; the oracle checks two sampled heads one by one and every
+    head's set size and softmax mass."""
+    lay = workloads.decode_layer(name, 0, device="cuda")
+    B, Hq = lay["B"], lay["Hq"]
+    N = lay["n_tokens"]
+    q = _unit(lay["q"])
+    k_lo, k_full, v_full = workloads.layout(lay["kwords"], lay["vwords"])
+    store = sdk.CodeStore.from_tensors(k_lo, k_full, v_full, [N] * B)
+    ws = sdk.new_workspace(sdk.sdk_decode_workspace_bytes(
+        B, Hq, 128, 32768, N))
+    out = sdk.sdk_decode_attn(q, lay["DK"], lay["DV"], store, workspace=ws)
+    torch.cuda.synchronize()
+    rc, _ = sdk.sdk_check_status(ws)
+    assert rc == 0
+    layd = sdk.sdk_decode_layout_of(B, Hq, 128, 32768, N)
+    st = sdk.read_select_state(ws, layd, B * Hq)
+    k = oracle.topk_count(N, 1, 10)
+    assert torch.all(st["n_sel"] == k)
+    assert torch.all(st["z"] >= 1.0)          # the max term contributes 1
+    assert torch.isfinite(out).all()
+    R = B * Hq
+    sets = _gpu_sets(ws, layd, R, N, [k] * R)
+    qn = q.cpu().double().numpy()
+    DKn = lay["DK"].cpu().float().double().numpy()
+    DVn = lay["DV"].cpu().float().double().numpy()
+    outn = out.cpu().double().numpy()
+    for (b, h) in [(0, 0), (B - 1, Hq - 1)]:
+        kvh = h // (Hq // lay["Hkv"])
+        kwn = words_np(lay["kwords"][b, kvh])
+        vwn = words_np(lay["vwords"][b, kvh])
+        ref = oracle.decode_head_ref(qn[b, h], kwn, vwn, DKn, DVn)
+        r = b * Hq + h
+        if check_selection(sets[r], ref["s_lo"], k):
+            ref = oracle.decode_head_ref(qn[b, h], kwn, vwn, DKn, DVn,
+                                         force_set=sets[r])
+        assert np.max(np.abs(outn[b, h] - ref["out"])) <= OUT_TOL
