@@ -44,6 +44,8 @@ def greedy_pursuit(x, D, k_atoms=16):
         gap = (|c|_(1) - |c|_(2)) / |c|_(1)   (0 when |c|_(1) == 0)
         r  <- r - coef * D[i*]
     Returns (idx[int64, k], coef[fp64, k], gap[fp64, k], r_final[fp64, d]).
+    ``greedy_pursuit.last_rnorm`` holds ||r|| before every step (a
+    diagnostic for the parity tests).
     """
     D = np.asarray(D, dtype=np.float64)
     r = np.array(x, dtype=np.float64, copy=True)
@@ -51,7 +53,9 @@ def greedy_pursuit(x, D, k_atoms=16):
     idx = np.zeros(k_atoms, dtype=np.int64)
     coef = np.zeros(k_atoms, dtype=np.float64)
     gap = np.zeros(k_atoms, dtype=np.float64)
+    rnorm = np.zeros(k_atoms, dtype=np.float64)
     for j in range(k_atoms):
+        rnorm[j] = np.sqrt(np.sum(r * r))
         c = D @ r
         a = np.abs(c)
         i = int(np.argmax(a))
@@ -64,6 +68,7 @@ def greedy_pursuit(x, D, k_atoms=16):
         idx[j] = i
         coef[j] = c[i]
         r = r - c[i] * D[i]
+    greedy_pursuit.last_rnorm = rnorm
     return idx, coef, gap, r
 
 
@@ -71,7 +76,8 @@ def encode_ref(X, D, k_atoms=16):
     """Greedy pursuit of every row of ``X`` ([m, d]); one vector at a time.
 
     Returns dict with idx [m,k] int64, coef [m,k] fp64, gap [m,k] fp64,
-    resid [m,d] fp64 (the final residuals).
+    resid [m,d] fp64 (the final residuals), rnorm [m,k] (||r|| before each
+    step) and xnorm [m].
     """
     X = np.asarray(X, dtype=np.float64)
     m = X.shape[0]
@@ -79,11 +85,14 @@ def encode_ref(X, D, k_atoms=16):
     out_coef = np.zeros((m, k_atoms), dtype=np.float64)
     out_gap = np.zeros((m, k_atoms), dtype=np.float64)
     out_r = np.zeros_like(X)
+    out_rn = np.zeros((m, k_atoms), dtype=np.float64)
     Dd = np.asarray(D, dtype=np.float64)
     for v in range(m):
         i, c, g, r = greedy_pursuit(X[v], Dd, k_atoms)
         out_idx[v], out_coef[v], out_gap[v], out_r[v] = i, c, g, r
-    return {"idx": out_idx, "coef": out_coef, "gap": out_gap, "resid": out_r}
+        out_rn[v] = greedy_pursuit.last_rnorm
+    return {"idx": out_idx, "coef": out_coef, "gap": out_gap, "resid": out_r,
+            "rnorm": out_rn, "xnorm": np.sqrt(np.sum(X * X, axis=1))}
 
 
 def store_coef_fp16(coef):

@@ -1,14 +1,722 @@
-// Tensor-core greedy pursuit encoder (placeholder until the sm_100a kernel
-// lands): declines every shape, so sdk_encode runs the CUDA-core encoder.
+// Greedy pursuit encoder on the 5th-generation tensor cores (sm_100a).
+//
+// Method ("LLM Inference in a Flash!", evolve.pub review, Summary): every
+// vector x gets K picks; a pick is i* = argmax_i |<r, d_i>| over the whole
+// dictionary, coef = <r, d_i*>, r -= coef * d_i* (projection-based greedy
+// pursuit, no least-squares refit).
+//
+// Design (one persistent CTA per SM, 10 warps, warp-specialised):
+//   warp 0      TMA producer: streams the bf16 dictionary through a 4-stage
+//               shared-memory ring in 128-atom tiles (128B-swizzled,
+//               K-major), the same dictionary 16 times per row tile.
+//   warp 1      MMA issuer: allocates 512 TMEM columns; for every atom tile
+//               issues tcgen05.mma kind::f16 (bf16 x bf16 -> fp32, M=128,
+//               N=128, K=16) for two 128-row sets of residuals (A operand,
+//               bf16, in shared memory) into one of two TMEM accumulator
+//               buffers; tcgen05.commit frees the ring stage and hands the
+//               buffer to the epilogue.
+//   warps 2..9  epilogue: one thread per residual row.  tcgen05.ld brings
+//               the row's 128 correlations to registers, the buffer is
+//               released at once, and the row keeps the running maximum
+//               B of |c~| plus every atom with |c~| >= B - band.  band is
+//               twice a rigorous bound on |c~ - c| (bf16 rounding of r by
+//               Cauchy-Schwarz, plus accumulation slack), so the exact
+//               fp32 argmax is always among the kept candidates.  After the
+//               last atom tile of a step the candidates are re-scored in
+//               fp32 (k = 0..D-1 FMA order, the same arithmetic as the
+//               CUDA-core encoder), the pick is written, r is updated in
+//               fp32 (global scratch, L2-resident) and its bf16 copy
+//               becomes the next step's A operand.  A row whose candidate
+//               list overflows falls back to an exact fp32 scan of all
+//               atoms (counted in the workspace header).
+// Every wait on an mbarrier is bounded (1 s of %globaltimer); on expiry the
+// CTA records SDK_ERR_TIMEOUT, stops issuing work, lets in-flight copies and
+// MMAs finish (bounded), frees its TMEM and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "sdk_internal.cuh"
 
 namespace sdk {
+namespace tc {
 
-size_t encode_tc_scratch_bytes(int64_t, int, int) { return 0; }
+constexpr int kRows = 128;                 // rows per set (TMEM lanes, MMA M)
+constexpr int kSets = 2;                   // row sets per CTA
+constexpr int kTileRows = kRows * kSets;   // vectors per row tile
+constexpr int kAtomTile = 128;             // atoms per B tile (MMA N)
+constexpr int kStages = 4;
+constexpr int kCand = 8;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (2 + kEpiWarps);
+constexpr int kMaxCtas = 160;
+constexpr int kTmemCols = 512;
+constexpr unsigned long long kWaitNs = 1000000000ull;
 
-sdk_status launch_encode_tc(const EncodeParams&, int, void*, size_t, cudaStream_t, bool* taken) {
+template <int D>
+struct Cfg {
+  static constexpr int KB = D / 64;                   // 128-byte K blocks
+  static constexpr int KSTEPS = D / 16;               // MMAs per row set
+  static constexpr int kStageBytes = kAtomTile * D * 2;
+  static constexpr int kABytes = kRows * D * 2;       // one row set
+  static constexpr int kOffA = kStages * kStageBytes;
+  static constexpr int kOffCi = kOffA + kSets * kABytes;
+  static constexpr int kOffCv = kOffCi + kTileRows * kCand * 4;
+  static constexpr int kOffBar = kOffCv + kTileRows * kCand * 4;
+  static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1 + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  // + alignment slack; at least 116 KB so that one CTA (which holds all 512
+  // TMEM columns) is resident per SM
+  static constexpr int kSmemUsed = kOffMisc + 64 + 1024;
+  static constexpr int kSmem = kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024;
+};
+
+struct TcParams {
+  const void* x;
+  int x_dtype;
+  int64_t n_vec;
+  const uint16_t* dict;
+  int n;
+  int k_atoms;
+  uint32_t* codes;
+  float* rsq;
+  WsHeader* hdr;
+  float* resid;        // [grid][D][kTileRows] fp32
+  const float* dmax;   // max_i ||d_i||
+  int n_tiles;
+  int n_atom_tiles;
+};
+
+// ---- PTX wrappers -----------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0u;
+}
+// Bounded wait: false when the phase did not complete within kWaitNs or the
+// CTA is aborting.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          volatile uint32_t* abort_flag,
+                                          unsigned long long limit = kWaitNs) {
+#pragma unroll 1
+  for (int i = 0; i < 128; ++i)
+    if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+#pragma unroll 1
+  while (true) {
+    if (mbar_try(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > limit) return false;
+  }
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  const uint32_t z = 0u;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(z), "r"(z), "r"(z), "r"(z)
+      : "memory");
+}
+// 32 lanes x 32 bits, 64 consecutive columns per thread.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&v)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31]),
+        "=r"(v[32]), "=r"(v[33]), "=r"(v[34]), "=r"(v[35]), "=r"(v[36]), "=r"(v[37]),
+        "=r"(v[38]), "=r"(v[39]), "=r"(v[40]), "=r"(v[41]), "=r"(v[42]), "=r"(v[43]),
+        "=r"(v[44]), "=r"(v[45]), "=r"(v[46]), "=r"(v[47]), "=r"(v[48]), "=r"(v[49]),
+        "=r"(v[50]), "=r"(v[51]), "=r"(v[52]), "=r"(v[53]), "=r"(v[54]), "=r"(v[55]),
+        "=r"(v[56]), "=r"(v[57]), "=r"(v[58]), "=r"(v[59]), "=r"(v[60]), "=r"(v[61]),
+        "=r"(v[62]), "=r"(v[63])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (the canonical layout TMA SWIZZLE_128B writes).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) |
+         ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+// Instruction descriptor: D f32, A bf16, B bf16, both K-major, N=128, M=128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                            ((uint32_t)(kAtomTile >> 3) << 17) | ((uint32_t)(kRows >> 4) << 24);
+
+__device__ __forceinline__ float bf16_round(float v) {
+  return __bfloat162float(__float2bfloat16_rn(v));
+}
+
+// ---- the kernel --------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    encode_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcParams p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint32_t* s_ci = reinterpret_cast<uint32_t*>(smem + C::kOffCi);
+  float* s_cv = reinterpret_cast<float*>(smem + C::kOffCv);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile uint32_t* s_abort = misc + 0;
+  volatile uint32_t* s_tmem = misc + 1;
+
+  const uint32_t sB = smem_u32(smem);
+  const uint32_t sA = smem_u32(smem + C::kOffA);
+  auto bar_full = [&](int s) { return smem_u32(&bars[s]); };
+  auto bar_empty = [&](int s) { return smem_u32(&bars[kStages + s]); };
+  auto bar_tfull = [&](int b) { return smem_u32(&bars[2 * kStages + b]); };
+  auto bar_tempty = [&](int b) { return smem_u32(&bars[2 * kStages + 2 + b]); };
+  const uint32_t bar_afull = smem_u32(&bars[2 * kStages + 4]);
+  const uint32_t bar_done = smem_u32(&bars[2 * kStages + 5]);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    *s_abort = 0u;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar_full(s), 1);
+      mbar_init(bar_empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_tfull(b), 1);
+      mbar_init(bar_tempty(b), kEpiWarps);
+    }
+    mbar_init(bar_afull, kEpiWarps);
+    mbar_init(bar_done, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32((const void*)s_tmem)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const int steps_total = p.k_atoms;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, last_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x)
+        for (int j = 0; ok && j < steps_total; ++j)
+          for (int a = 0; a < p.n_atom_tiles; ++a) {
+            if (!mbar_wait(bar_empty(stage), phase ^ 1u, s_abort)) {
+              ok = false;
+              break;
+            }
+            mbar_expect_tx(bar_full(stage), (uint32_t)C::kStageBytes);
+#pragma unroll
+            for (int kb = 0; kb < C::KB; ++kb)
+              tma_load_2d(sB + stage * C::kStageBytes + kb * (kAtomTile * 128), &tmap, kb * 64,
+                          a * kAtomTile, bar_full(stage));
+            issued_mask |= 1u << stage;
+            last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
+            if (++stage == kStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+      if (!ok) {
+        record_error(p.hdr, SDK_ERR_TIMEOUT, 0x40000000u | blockIdx.x);
+        *s_abort = 1u;
+      }
+      // let every issued copy land before the CTA can exit
+      for (int s = 0; s < kStages; ++s)
+        if (issued_mask & (1u << s)) {
+          uint32_t dummy = 0u;
+          mbar_wait(bar_full(s), (last_phase >> s) & 1u, &dummy, 100000000ull);
+        }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, tbuf = 0, tphase = 0, aphase = 0;
+      bool ok = true;
+      bool issued = false;
+      for (int tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x)
+        for (int j = 0; ok && j < steps_total; ++j) {
+          if (!mbar_wait(bar_afull, aphase, s_abort)) {
+            ok = false;
+            break;
+          }
+          aphase ^= 1u;
+          tc_fence_after();
+          for (int a = 0; a < p.n_atom_tiles; ++a) {
+            if (!mbar_wait(bar_full(stage), phase, s_abort) ||
+                !mbar_wait(bar_tempty(tbuf), tphase ^ 1u, s_abort)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t bbase = sB + stage * C::kStageBytes;
+#pragma unroll
+            for (int rs = 0; rs < kSets; ++rs) {
+              const uint32_t d_tmem = tmem + tbuf * (kSets * kAtomTile) + rs * kAtomTile;
+              const uint32_t abase = sA + rs * C::kABytes;
+#pragma unroll
+              for (int ks = 0; ks < C::KSTEPS; ++ks) {
+                const uint32_t koff = (ks >> 2) * (kRows * 128) + (ks & 3) * 32;
+                const uint32_t boff = (ks >> 2) * (kAtomTile * 128) + (ks & 3) * 32;
+                tc_mma(d_tmem, smem_desc(abase + koff), smem_desc(bbase + boff), kIdesc,
+                       ks > 0 ? 1u : 0u);
+              }
+            }
+            issued = true;
+            tc_commit(bar_empty(stage));
+            tc_commit(bar_tfull(tbuf));
+            if (++stage == kStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            tbuf ^= 1u;
+            if (tbuf == 0u) tphase ^= 1u;
+          }
+        }
+      if (!ok) {
+        record_error(p.hdr, SDK_ERR_TIMEOUT, 0x41000000u | blockIdx.x);
+        *s_abort = 1u;
+      }
+      if (issued) {
+        // all MMAs of this thread complete before TMEM is released
+        tc_commit(bar_done);
+        uint32_t dummy = 0u;
+        mbar_wait(bar_done, 0u, &dummy, 100000000ull);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - 2;
+    const int rs = e >> 2;               // row set
+    const int q = warp & 3;              // TMEM lane quarter of this warp
+    const int rin = q * 32 + lane;       // row within the set (TMEM lane)
+    const int row = rs * kRows + rin;    // row within the tile
+    float* rres = p.resid + (int64_t)blockIdx.x * D * kTileRows + row;  // stride kTileRows
+    uint32_t* ci = s_ci + row * kCand;
+    float* cv = s_cv + row * kCand;
+    const float dmax = *p.dmax;
+    uint8_t* arow = smem + C::kOffA + rs * C::kABytes + rin * 128;
+    uint32_t tbuf = 0, tphase = 0;
+    uint32_t n_rescored = 0;
+    bool ok = true;
+
+    // writes bf16(r) of this row into the swizzled A operand and returns
+    // (||r - bf16(r)||^2, ||r||^2) accumulated from the fp32 values
+    auto write_a_chunk = [&](int kc, const float (&r8)[8], float& e2, float& n2) {
+      uint32_t w[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float a0 = r8[2 * u], a1 = r8[2 * u + 1];
+        const __nv_bfloat162 h = __floats2bfloat162_rn(a0, a1);
+        const float b0 = __low2float(h), b1 = __high2float(h);
+        e2 = fmaf(a0 - b0, a0 - b0, e2);
+        e2 = fmaf(a1 - b1, a1 - b1, e2);
+        n2 = fmaf(a0, a0, n2);
+        n2 = fmaf(a1, a1, n2);
+        w[u] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      const int kb = kc >> 3, c16 = kc & 7;
+      uint4* dst = reinterpret_cast<uint4*>(arow + kb * (kRows * 128) +
+                                            ((c16 ^ (rin & 7)) << 4));
+      *dst = make_uint4(w[0], w[1], w[2], w[3]);
+    };
+    auto band_of = [&](float e2, float n2) {
+      return 2.0f * dmax * sqrtf(e2) + 0.0009765625f * dmax * sqrtf(n2);
+    };
+    // fp32 correlation in k order (the CUDA-core encoder's arithmetic)
+    auto dot_atom = [&](uint32_t i) {
+      const uint4* dp = reinterpret_cast<const uint4*>(p.dict + (int64_t)i * D);
+      float s = 0.0f;
+#pragma unroll 4
+      for (int kc = 0; kc < D / 8; ++kc) {
+        const uint4 dv = __ldg(dp + kc);
+        const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          s = fmaf(rres[(kc * 8 + 2 * u) * kTileRows], bf16_lo(dw[u]), s);
+          s = fmaf(rres[(kc * 8 + 2 * u + 1) * kTileRows], bf16_hi(dw[u]), s);
+        }
+      }
+      return s;
+    };
+
+    for (int tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x) {
+      const int64_t grow = (int64_t)tile * kTileRows + row;
+      const bool valid = grow < p.n_vec;
+      // residual <- x; A <- bf16(x)
+      float e2 = 0.0f, n2 = 0.0f;
+#pragma unroll 1
+      for (int kc = 0; kc < D / 8; ++kc) {
+        float r8[8];
+        if (valid) {
+          if (p.x_dtype == SDK_F32) {
+            const float4* xp = reinterpret_cast<const float4*>(
+                reinterpret_cast<const float*>(p.x) + grow * D + kc * 8);
+            const float4 a = __ldg(xp), b = __ldg(xp + 1);
+            r8[0] = a.x; r8[1] = a.y; r8[2] = a.z; r8[3] = a.w;
+            r8[4] = b.x; r8[5] = b.y; r8[6] = b.z; r8[7] = b.w;
+          } else {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(
+                reinterpret_cast<const uint16_t*>(p.x) + grow * D + kc * 8));
+            const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              r8[2 * u] = bf16_lo(vw[u]);
+              r8[2 * u + 1] = bf16_hi(vw[u]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) r8[u] = 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) rres[(kc * 8 + u) * kTileRows] = r8[u];
+        write_a_chunk(kc, r8, e2, n2);
+      }
+      float band = band_of(e2, n2);
+      bool active = valid && n2 > 0.0f;
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_afull);
+
+      for (int j = 0; j < steps_total; ++j) {
+        float best = -INFINITY, thr = -INFINITY;
+        int cnt = 0;
+        bool ovf = false;
+#pragma unroll 1
+        for (int a = 0; a < p.n_atom_tiles; ++a) {
+          // one lane waits so the warp stays converged for tcgen05.ld
+          const bool got = lane == 0 ? mbar_wait(bar_tfull(tbuf), tphase, s_abort) : true;
+          if (!__shfl_sync(0xffffffffu, got ? 1 : 0, 0)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t v[2][64];
+          const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + tbuf * (kSets * kAtomTile) +
+                                 rs * kAtomTile;
+          tmem_ld64(taddr, v[0]);
+          tmem_ld64(taddr + 64, v[1]);
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_tempty(tbuf));
+          tbuf ^= 1u;
+          if (tbuf == 0u) tphase ^= 1u;
+          if (!active) continue;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            float m = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) m = fmaxf(m, fabsf(__uint_as_float(v[c][i])));
+            if (m >= thr) {
+              // rare: the chunk holds a value within `band` of the running
+              // maximum.  Drop stale candidates, then keep every column of
+              // the chunk at or above the new threshold.
+              best = fmaxf(best, m);
+              thr = best - band;
+              int w = 0;
+#pragma unroll 1
+              for (int t = 0; t < cnt; ++t)
+                if (cv[t] >= thr) {
+                  ci[w] = ci[t];
+                  cv[w] = cv[t];
+                  ++w;
+                }
+              cnt = w;
+              const int lim = p.n - (a * kAtomTile + c * 64);
+              const uint32_t cbase = (uint32_t)(a * kAtomTile + c * 64);
+#pragma unroll
+              for (int i = 0; i < 64; ++i) {
+                const float av = fabsf(__uint_as_float(v[c][i]));
+                if (av >= thr && i < lim) {
+                  if (cnt < kCand) {
+                    ci[cnt] = cbase + i;
+                    cv[cnt] = av;
+                    ++cnt;
+                  } else {
+                    ovf = true;
+                  }
+                }
+              }
+            }
+          }
+        }
+        if (!ok) break;
+
+        // ---- pick: exact fp32 re-score of the candidates
+        uint32_t pick = 0u;
+        float coef = 0.0f;
+        if (active) {
+          float babs = -1.0f;
+          if (ovf) {
+            atomicAdd(&p.hdr->enc_fallback, 1u);
+#pragma unroll 1
+            for (int i = 0; i < p.n; ++i) {
+              const float c = dot_atom((uint32_t)i);
+              if (fabsf(c) > babs) {
+                babs = fabsf(c);
+                coef = c;
+                pick = (uint32_t)i;
+              }
+            }
+          } else {
+            int used = 0;
+#pragma unroll 1
+            for (int t = 0; t < cnt; ++t) {
+              if (cv[t] < thr) continue;
+              const uint32_t i = ci[t];
+              const float c = dot_atom(i);
+              ++used;
+              if (fabsf(c) > babs || (fabsf(c) == babs && i < pick)) {
+                babs = fabsf(c);
+                coef = c;
+                pick = i;
+              }
+            }
+            n_rescored += (uint32_t)used;
+          }
+        }
+        if (valid) p.codes[grow * p.k_atoms + j] = make_word(coef, pick);
+
+        // ---- residual update r -= coef * d_pick; next A operand
+        if (j + 1 < steps_total) {
+          if (active) {
+            e2 = 0.0f;
+            n2 = 0.0f;
+            const uint4* dp = reinterpret_cast<const uint4*>(p.dict + (int64_t)pick * D);
+#pragma unroll 1
+            for (int kc = 0; kc < D / 8; ++kc) {
+              const uint4 dv = __ldg(dp + kc);
+              const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
+              float r8[8];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                float* r0 = rres + (kc * 8 + 2 * u) * kTileRows;
+                float* r1 = rres + (kc * 8 + 2 * u + 1) * kTileRows;
+                r8[2 * u] = fmaf(-coef, bf16_lo(dw[u]), *r0);
+                r8[2 * u + 1] = fmaf(-coef, bf16_hi(dw[u]), *r1);
+                *r0 = r8[2 * u];
+                *r1 = r8[2 * u + 1];
+              }
+              write_a_chunk(kc, r8, e2, n2);
+            }
+            band = band_of(e2, n2);
+            active = n2 > 0.0f;
+          }
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_afull);
+        } else if (active) {
+          // last step: update the fp32 residual only (for ||r||^2)
+          const uint4* dp = reinterpret_cast<const uint4*>(p.dict + (int64_t)pick * D);
+#pragma unroll 1
+          for (int kc = 0; kc < D / 8; ++kc) {
+            const uint4 dv = __ldg(dp + kc);
+            const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              float* r0 = rres + (kc * 8 + 2 * u) * kTileRows;
+              float* r1 = rres + (kc * 8 + 2 * u + 1) * kTileRows;
+              *r0 = fmaf(-coef, bf16_lo(dw[u]), *r0);
+              *r1 = fmaf(-coef, bf16_hi(dw[u]), *r1);
+            }
+          }
+        }
+      }
+      if (!ok) break;
+      if (valid && p.rsq != nullptr) {
+        float s = 0.0f;
+        for (int k = 0; k < D; ++k) {
+          const float r = rres[k * kTileRows];
+          s = fmaf(r, r, s);
+        }
+        p.rsq[grow] = s;
+      }
+    }
+    if (!ok) {
+      record_error(p.hdr, SDK_ERR_TIMEOUT, 0x42000000u | blockIdx.x);
+      *s_abort = 1u;
+    }
+    n_rescored = __reduce_add_sync(0xffffffffu, n_rescored);
+    if (lane == 0 && n_rescored) atomicAdd(&p.hdr->enc_cands, n_rescored);
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// max_i ||d_i|| (one warp per atom); *out must be zero before the launch
+__global__ void dict_norm_kernel(const uint16_t* dict, int n, int D, float* out) {
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  const int w0 = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  float mx = 0.0f;
+  for (int i = w0; i < n; i += warps) {
+    float s = 0.0f;
+    for (int k = lane; k < D; k += 32) {
+      const float v = bf16_lo(dict[(int64_t)i * D + k]);
+      s = fmaf(v, v, s);
+    }
+    s = warp_sum(s);
+    mx = fmaxf(mx, sqrtf(s));
+  }
+  if (lane == 0 && mx > 0.0f) atomicMax(reinterpret_cast<int*>(out), __float_as_int(mx));
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000,
+                                         cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+}  // namespace tc
+
+size_t encode_tc_scratch_bytes(int64_t n_vec, int head_dim, int n_atoms) {
+  (void)n_atoms;
+  if (head_dim != 64 && head_dim != 128) return 256;
+  int64_t tiles = (n_vec + tc::kTileRows - 1) / tc::kTileRows;
+  if (tiles > tc::kMaxCtas) tiles = tc::kMaxCtas;
+  return 256 + (size_t)tiles * head_dim * tc::kTileRows * 4;
+}
+
+sdk_status launch_encode_tc(const EncodeParams& p, int head_dim, void* scratch,
+                            size_t scratch_bytes, cudaStream_t stream, bool* taken) {
   *taken = false;
-  return SDK_OK;
+  if (head_dim != 64 && head_dim != 128) return SDK_OK;
+  if (p.n_vec <= 0) return SDK_OK;
+  // vectorised 16-byte loads of x rows need a 16-byte aligned x
+  if ((reinterpret_cast<uintptr_t>(p.x) & 15u) != 0u) return SDK_OK;
+  auto fn = tc::encode_fn();
+  if (fn == nullptr) return SDK_OK;  // no driver entry point: CUDA-core path
+  const int64_t tiles = (p.n_vec + tc::kTileRows - 1) / tc::kTileRows;
+  int64_t grid = tiles;
+  const int sms = num_sms();
+  if (grid > sms) grid = sms;
+  if (grid > tc::kMaxCtas) grid = tc::kMaxCtas;
+  const size_t per_cta = (size_t)head_dim * tc::kTileRows * 4;
+  if (scratch_bytes < 256 + (size_t)grid * per_cta) return SDK_ERR_CAPACITY;
+
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)p.n};
+  const cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+  const cuuint32_t box[2] = {64u, (cuuint32_t)tc::kAtomTile};
+  const cuuint32_t estr[2] = {1u, 1u};
+  CUresult cr = fn(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(p.dict), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return SDK_ERR_INVALID_ARG;
+  *taken = true;
+
+  float* dmax = reinterpret_cast<float*>(scratch);
+  if (cudaMemsetAsync(dmax, 0, sizeof(float), stream) != cudaSuccess) return SDK_ERR_CUDA;
+  tc::dict_norm_kernel<<<64, 256, 0, stream>>>(p.dict, p.n, head_dim, dmax);
+
+  tc::TcParams tp;
+  tp.x = p.x;
+  tp.x_dtype = p.x_dtype;
+  tp.n_vec = p.n_vec;
+  tp.dict = p.dict;
+  tp.n = p.n;
+  tp.k_atoms = p.k_atoms;
+  tp.codes = p.codes;
+  tp.rsq = p.rsq;
+  tp.hdr = p.hdr;
+  tp.resid = reinterpret_cast<float*>(reinterpret_cast<char*>(scratch) + 256);
+  tp.dmax = dmax;
+  tp.n_tiles = (int)tiles;
+  tp.n_atom_tiles = (p.n + tc::kAtomTile - 1) / tc::kAtomTile;
+
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(tc::encode_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         tc::Cfg<128>::kSmem);
+    cudaFuncSetAttribute(tc::encode_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         tc::Cfg<64>::kSmem);
+    attr = true;
+  }
+  if (head_dim == 128)
+    tc::encode_tc_kernel<128><<<(unsigned)grid, tc::kThreads, tc::Cfg<128>::kSmem, stream>>>(map, tp);
+  else
+    tc::encode_tc_kernel<64><<<(unsigned)grid, tc::kThreads, tc::Cfg<64>::kSmem, stream>>>(map, tp);
+  return cudaGetLastError() == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
 }
 
 }  // namespace sdk
