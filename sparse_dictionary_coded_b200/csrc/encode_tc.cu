@@ -27,8 +27,8 @@
 //               CUDA-core encoder), the pick is written, r is updated in
 //               fp32 (global scratch, L2-resident) and its bf16 copy
 //               becomes the next step's A operand.  A row whose candidate
-//               list overflows falls back to an exact fp32 scan of all
-//               atoms (counted in the workspace header).
+//               list overflows is re-picked by an exact fp32 scan of all
+//               atoms shared by its warp (counted in the workspace header).
 // Every wait on an mbarrier is bounded (1 s of %globaltimer); on expiry the
 // CTA records SDK_ERR_TIMEOUT, stops issuing work, lets in-flight copies and
 // MMAs finish (bounded), frees its TMEM and exits.
@@ -386,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       *dst = make_uint4(w[0], w[1], w[2], w[3]);
     };
     auto band_of = [&](float e2, float n2) {
-      return 2.0f * dmax * sqrtf(e2) + 0.0009765625f * dmax * sqrtf(n2);
+      return 2.0f * dmax * sqrtf(e2) + 0.000244140625f * dmax * sqrtf(n2);
     };
     // fp32 correlation in k order (the CUDA-core encoder's arithmetic)
     auto dot_atom = [&](uint32_t i) {
@@ -512,34 +512,72 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- pick: exact fp32 re-score of the candidates
         uint32_t pick = 0u;
         float coef = 0.0f;
-        if (active) {
+        if (active && !ovf) {
           float babs = -1.0f;
-          if (ovf) {
-            atomicAdd(&p.hdr->enc_fallback, 1u);
+          int used = 0;
 #pragma unroll 1
-            for (int i = 0; i < p.n; ++i) {
-              const float c = dot_atom((uint32_t)i);
-              if (fabsf(c) > babs) {
-                babs = fabsf(c);
-                coef = c;
-                pick = (uint32_t)i;
+          for (int t = 0; t < cnt; ++t) {
+            if (cv[t] < thr) continue;
+            const uint32_t i = ci[t];
+            const float c = dot_atom(i);
+            ++used;
+            if (fabsf(c) > babs || (fabsf(c) == babs && i < pick)) {
+              babs = fabsf(c);
+              coef = c;
+              pick = i;
+            }
+          }
+          n_rescored += (uint32_t)used;
+        }
+        // rows whose candidate list overflowed: exact fp32 scan of every atom
+        // by the whole warp, one such row at a time
+        uint32_t ovm = __ballot_sync(0xffffffffu, active && ovf);
+        if (ovm != 0u && lane == 0) atomicAdd(&p.hdr->enc_fallback, (uint32_t)__popc(ovm));
+#pragma unroll 1
+        while (ovm != 0u) {
+          const int src = __ffs(ovm) - 1;
+          ovm &= ovm - 1u;
+          const float* rsrc = p.resid + (int64_t)blockIdx.x * D * kTileRows +
+                              (rs * kRows + q * 32 + src);
+          float rr[D];
+#pragma unroll
+          for (int k = 0; k < D; ++k) rr[k] = rsrc[k * kTileRows];
+          float bab = -1.0f, bc = 0.0f;
+          uint32_t bi = 0u;
+#pragma unroll 1
+          for (int i = lane; i < p.n; i += 32) {
+            const uint4* dp = reinterpret_cast<const uint4*>(p.dict + (int64_t)i * D);
+            float sdot = 0.0f;
+#pragma unroll
+            for (int kc = 0; kc < D / 8; ++kc) {
+              const uint4 dv = __ldg(dp + kc);
+              const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                sdot = fmaf(rr[kc * 8 + 2 * u], bf16_lo(dw[u]), sdot);
+                sdot = fmaf(rr[kc * 8 + 2 * u + 1], bf16_hi(dw[u]), sdot);
               }
             }
-          } else {
-            int used = 0;
-#pragma unroll 1
-            for (int t = 0; t < cnt; ++t) {
-              if (cv[t] < thr) continue;
-              const uint32_t i = ci[t];
-              const float c = dot_atom(i);
-              ++used;
-              if (fabsf(c) > babs || (fabsf(c) == babs && i < pick)) {
-                babs = fabsf(c);
-                coef = c;
-                pick = i;
-              }
+            if (fabsf(sdot) > bab) {
+              bab = fabsf(sdot);
+              bc = sdot;
+              bi = (uint32_t)i;
             }
-            n_rescored += (uint32_t)used;
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            const float oa = __shfl_xor_sync(0xffffffffu, bab, o);
+            const float oc = __shfl_xor_sync(0xffffffffu, bc, o);
+            const uint32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (oa > bab || (oa == bab && oi < bi)) {
+              bab = oa;
+              bc = oc;
+              bi = oi;
+            }
+          }
+          if (lane == src) {
+            coef = bc;
+            pick = bi;
           }
         }
         if (valid) p.codes[grow * p.k_atoms + j] = make_word(coef, pick);
@@ -616,22 +654,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// max_i ||d_i|| (one warp per atom); *out must be zero before the launch
-__global__ void dict_norm_kernel(const uint16_t* dict, int n, int D, float* out) {
-  const int warps = gridDim.x * (blockDim.x >> 5);
-  const int w0 = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  float mx = 0.0f;
-  for (int i = w0; i < n; i += warps) {
-    float s = 0.0f;
-    for (int k = lane; k < D; k += 32) {
-      const float v = bf16_lo(dict[(int64_t)i * D + k]);
-      s = fmaf(v, v, s);
+// max_i ||d_i|| (one thread per atom, 16-byte loads); *out must be zero
+// before the launch
+template <int D>
+__global__ void __launch_bounds__(128) dict_norm_kernel(const uint16_t* dict, int n, float* out) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  float s = 0.0f;
+  if (i < n) {
+    const uint4* dp = reinterpret_cast<const uint4*>(dict + (int64_t)i * D);
+#pragma unroll
+    for (int kc = 0; kc < D / 8; ++kc) {
+      const uint4 v = __ldg(dp + kc);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        s = fmaf(bf16_lo(w[u]), bf16_lo(w[u]), s);
+        s = fmaf(bf16_hi(w[u]), bf16_hi(w[u]), s);
+      }
     }
-    s = warp_sum(s);
-    mx = fmaxf(mx, sqrtf(s));
   }
-  if (lane == 0 && mx > 0.0f) atomicMax(reinterpret_cast<int*>(out), __float_as_int(mx));
+  float m = sqrtf(s);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0 && m > 0.0f) atomicMax(reinterpret_cast<int*>(out), __float_as_int(m));
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -687,7 +732,10 @@ sdk_status launch_encode_tc(const EncodeParams& p, int head_dim, void* scratch,
 
   float* dmax = reinterpret_cast<float*>(scratch);
   if (cudaMemsetAsync(dmax, 0, sizeof(float), stream) != cudaSuccess) return SDK_ERR_CUDA;
-  tc::dict_norm_kernel<<<64, 256, 0, stream>>>(p.dict, p.n, head_dim, dmax);
+  if (head_dim == 128)
+    tc::dict_norm_kernel<128><<<(p.n + 127) / 128, 128, 0, stream>>>(p.dict, p.n, dmax);
+  else
+    tc::dict_norm_kernel<64><<<(p.n + 127) / 128, 128, 0, stream>>>(p.dict, p.n, dmax);
 
   tc::TcParams tp;
   tp.x = p.x;
