@@ -296,8 +296,9 @@ def bench_layer4k(args, world, rank, pk):
                    "l2": "flushed between steps (256 MiB memset outside the "
                          "per-step events)"},
         "dtype": "f32 (bf16 dictionaries, fp16 coefficients)",
-        # kernels per step: append = 2 x (encode + scatter); decode = 8
-        "gpu_launches": args.steps * (4 + 8),
+        # kernels per step: append = 2 x (dictionary norm + encode +
+        # scatter); decode = 7 (qd, klow, pass2, final, rescore, value, out)
+        "gpu_launches": args.steps * (6 + 7),
         "enc_fallback_rows": hdr[2],
     }
     if not args.no_e2e:
@@ -400,7 +401,7 @@ def bench_decode(args, world, rank, pk, name):
                    "l2": "flushed between steps; codes (%.1f GB) exceed L2"
                          % (L * B * Hkv * N * 140 / 1e9)},
         "dtype": "f32 (bf16 dictionaries, fp16 coefficients)",
-        "gpu_launches": args.steps * L * 8,
+        "gpu_launches": args.steps * L * 7,
     }
 
 
@@ -443,7 +444,7 @@ def bench_prefill(args, world, rank, pk):
                    "head_dim": d, "n_atoms": n, "k_atoms": 16,
                    "l2": "flushed between steps"},
         "dtype": "f32 (bf16 dictionaries)",
-        "gpu_launches": args.steps * 2,
+        "gpu_launches": args.steps * 2 * 2,
         "enc_fallback_rows": hdr[2],
     }
 

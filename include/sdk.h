@@ -173,7 +173,7 @@ SDK_API size_t sdk_append_workspace_bytes(int32_t B, int32_t Hkv, int32_t n_new,
  *   klow       1 .. khigh;  khigh  klow .. 16
  *   top_num, top_den   0 < top_num <= top_den
  *   scale      logit scale (1/sqrt(head_dim) for standard attention)
- *   out        device, float [B][Hq][head_dim]
+ *   out        device, float [B][Hq][head_dim], 16-byte aligned
  *   workspace  device, >= sdk_decode_workspace_bytes(B, Hq, head_dim,
  *              n_atoms, max_len) with max_len >= every lens[b]
  * Limits: B <= 64, Hq % Hkv == 0, head_dim in {64, 128}, B*Hq <= 2048,

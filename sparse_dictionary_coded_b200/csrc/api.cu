@@ -265,7 +265,7 @@ sdk_status sdk_decode_attn(const float* q, int32_t B, int32_t Hq, int32_t Hkv, i
     return SDK_ERR_INVALID_ARG;
   if (!aligned(workspace, SDK_WS_ALIGN) || !aligned(dict_k, 16) || !aligned(dict_v, 16) ||
       !aligned(k_full, 16) || !aligned(v_full, 16) || !aligned(k_lo, 4) || !aligned(q, 4) ||
-      !aligned(out, 4))
+      !aligned(out, 16))
     return SDK_ERR_INVALID_ARG;
   int64_t max_len = 0;
   for (int b = 0; b < B; ++b) {

@@ -21,9 +21,12 @@
 //                    selected tokens (64-byte k_full records).
 //   value_kernel     e_t = exp(s_t - max), z = sum e_t, and the scatter
 //                    w[idx^V_tj] += e_t c^V_tj (shared-memory atomics into a
-//                    per-atom weight tile, flushed to global).
-//   out_kernel       partial sums of w D_V over atom tiles;
-//   out_reduce       out = (sum of partials) / z.
+//                    per-atom weight tile per CTA; a cluster of CTAs per
+//                    head sums its tiles through distributed shared memory).
+//   out_kernel       out += (w D_V) / z over atom tiles (vector reductions
+//                    into `out`, zeroed by qd_kernel).
+#include <cooperative_groups.h>
+
 #include "sdk_internal.cuh"
 
 namespace sdk {
@@ -99,29 +102,33 @@ __device__ void block_find_desc(const uint32_t* hist, uint32_t k,
 }
 
 // ---------------------------------------------------------------- qd_kernel
-template <int D>
-__global__ void __launch_bounds__(256) qd_kernel(DecodeParams p) {
-  __shared__ float Ds[D][64];
-  __shared__ float Qs[D][32];
-  const int n = p.n, R = p.R;
-  const int a0 = blockIdx.x * 64, r0 = blockIdx.y * 32;
-  const int tid = threadIdx.x;
+// QD[r][a] = sum_k q[r][k] D_K[a][k] on a 128-atom x 32-row tile; thread
+// (ta, tr) owns atoms 4ta..4ta+3 and rows 8tr..8tr+7 (32 accumulators, fp32
+// FMA chains in k order).  The first kernel of a call also zeroes the
+// per-head selection state, both histograms and `out` (accumulated with
+// reductions by out_kernel).
+constexpr int kQdThreads = 128;
 
-  // zero the per-head selection state and histograms (grid-stride over the
-  // whole grid, block-linear order)
+template <int D>
+__global__ void __launch_bounds__(kQdThreads) qd_kernel(DecodeParams p) {
+  extern __shared__ float4 smem4[];
+  float* Ds = reinterpret_cast<float*>(smem4);   // [D][128]  atom tile, k-major
+  float* Qs = Ds + D * 128;                      // [D][32]   query rows, k-major
+  const int n = p.n, R = p.R, tid = threadIdx.x;
+  const int a0 = blockIdx.x * 128, r0 = blockIdx.y * 32;
   {
-    const int64_t nblk = (int64_t)gridDim.x * gridDim.y;
-    const int64_t bl = (int64_t)blockIdx.y * gridDim.x + blockIdx.x;
+    const int64_t nthr = (int64_t)gridDim.x * gridDim.y * kQdThreads;
+    const int64_t g0 = ((int64_t)blockIdx.y * gridDim.x + blockIdx.x) * kQdThreads + tid;
     const int64_t hwords = (int64_t)R * 4096;
-    for (int64_t e = bl * 256 + tid; e < hwords; e += nblk * 256) {
+    for (int64_t e = g0; e < hwords; e += nthr) {
       p.hist1[e] = 0u;
       p.hist2[e] = 0u;
     }
-    for (int64_t e = bl * 256 + tid; e < (int64_t)R; e += nblk * 256) {
+    for (int64_t e = g0; e < (int64_t)R * D; e += nthr) p.out[e] = 0.0f;
+    for (int64_t e = g0; e < (int64_t)R; e += nthr) {
       sdk_select_state s;
-      const int b = (int)(e / p.Hq);
       s.kth_key = 0u;
-      s.k = (uint32_t)p.kcnt[b];
+      s.k = (uint32_t)p.kcnt[e / p.Hq];
       s.n_above = s.n_cand = s.n_sel = s.n_comp = 0u;
       s.eq_total = s.eq_taken = 0u;
       s.max_score = 0u;
@@ -132,56 +139,54 @@ __global__ void __launch_bounds__(256) qd_kernel(DecodeParams p) {
       p.st[e] = s;
     }
   }
-
-  // atom tile, transposed to [k][a] in fp32
-  for (int e = tid; e < 64 * (D / 8); e += 256) {
-    const int a = e & 63, c = e >> 6;
+  for (int e = tid; e < 128 * (D / 8); e += kQdThreads) {
+    const int a = e & 127, c = e >> 7;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (a0 + a < n)
-      v = __ldg(reinterpret_cast<const uint4*>(p.dk + (int64_t)(a0 + a) * D) + c);
-    Ds[c * 8 + 0][a] = bf16_lo(v.x);
-    Ds[c * 8 + 1][a] = bf16_hi(v.x);
-    Ds[c * 8 + 2][a] = bf16_lo(v.y);
-    Ds[c * 8 + 3][a] = bf16_hi(v.y);
-    Ds[c * 8 + 4][a] = bf16_lo(v.z);
-    Ds[c * 8 + 5][a] = bf16_hi(v.z);
-    Ds[c * 8 + 6][a] = bf16_lo(v.w);
-    Ds[c * 8 + 7][a] = bf16_hi(v.w);
+    if (a0 + a < n) v = __ldg(reinterpret_cast<const uint4*>(p.dk + (int64_t)(a0 + a) * D) + c);
+    float* col = Ds + (c * 8) * 128 + a;
+    col[0 * 128] = bf16_lo(v.x);
+    col[1 * 128] = bf16_hi(v.x);
+    col[2 * 128] = bf16_lo(v.y);
+    col[3 * 128] = bf16_hi(v.y);
+    col[4 * 128] = bf16_lo(v.z);
+    col[5 * 128] = bf16_hi(v.z);
+    col[6 * 128] = bf16_lo(v.w);
+    col[7 * 128] = bf16_hi(v.w);
   }
-  for (int e = tid; e < 32 * D; e += 256) {
+  for (int e = tid; e < 32 * D; e += kQdThreads) {
     const int r = e & 31, k = e >> 5;
-    Qs[k][r] = (r0 + r < R) ? p.q[(int64_t)(r0 + r) * D + k] : 0.0f;
+    Qs[k * 32 + r] = (r0 + r < R) ? __ldg(p.q + (int64_t)(r0 + r) * D + k) : 0.0f;
   }
   __syncthreads();
-
   const int ta = tid & 31, tr = tid >> 5;
-  float acc[4][2];
+  float acc[8][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = 0.0f;
-#pragma unroll 8
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[i][u] = 0.0f;
+#pragma unroll 4
   for (int k = 0; k < D; ++k) {
-    const float2 dv = *reinterpret_cast<const float2*>(&Ds[k][2 * ta]);
-    const float4 qv = *reinterpret_cast<const float4*>(&Qs[k][4 * tr]);
-    acc[0][0] = fmaf(qv.x, dv.x, acc[0][0]);
-    acc[0][1] = fmaf(qv.x, dv.y, acc[0][1]);
-    acc[1][0] = fmaf(qv.y, dv.x, acc[1][0]);
-    acc[1][1] = fmaf(qv.y, dv.y, acc[1][1]);
-    acc[2][0] = fmaf(qv.z, dv.x, acc[2][0]);
-    acc[2][1] = fmaf(qv.z, dv.y, acc[2][1]);
-    acc[3][0] = fmaf(qv.w, dv.x, acc[3][0]);
-    acc[3][1] = fmaf(qv.w, dv.y, acc[3][1]);
+    const float4 dv = *reinterpret_cast<const float4*>(Ds + k * 128 + 4 * ta);
+    const float4 qa = *reinterpret_cast<const float4*>(Qs + k * 32 + 8 * tr);
+    const float4 qb = *reinterpret_cast<const float4*>(Qs + k * 32 + 8 * tr + 4);
+    const float dd[4] = {dv.x, dv.y, dv.z, dv.w};
+    const float qq[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) acc[i][u] = fmaf(qq[i], dd[u], acc[i][u]);
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = r0 + 4 * tr + i;
+  for (int i = 0; i < 8; ++i) {
+    const int r = r0 + 8 * tr + i;
     if (r >= R) continue;
+    float* dst = p.qd + (int64_t)r * n + a0 + 4 * ta;
+    if (a0 + 4 * ta + 3 < n && (n & 3) == 0) {
+      *reinterpret_cast<float4*>(dst) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+    } else {
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int a = a0 + 2 * ta + u;
-      if (a < n) {
-        p.qd[(int64_t)r * n + a] = acc[i][u];
-        p.w[(int64_t)r * n + a] = 0.0f;
-      }
+      for (int u = 0; u < 4; ++u)
+        if (a0 + 4 * ta + u < n) dst[u] = acc[i][u];
     }
   }
 }
@@ -197,6 +202,14 @@ __device__ __forceinline__ void stage_row(float* dst, const float* src, int n) {
   }
 }
 
+// Warp-aggregated shared-memory histogram increment (lanes with equal bins
+// add once); every lane of the warp must call it; bin 0xFFFFFFFF skips.
+__device__ __forceinline__ void hist_add_warp(uint32_t* sh, uint32_t bin) {
+  const unsigned mm = __match_any_sync(0xffffffffu, bin);
+  const int lane = threadIdx.x & 31;
+  if (bin != 0xFFFFFFFFu && lane == __ffs(mm) - 1) atomicAdd(&sh[bin], (uint32_t)__popc(mm));
+}
+
 // -------------------------------------------------------------- klow_kernel
 constexpr int kScanThreads = 512;
 
@@ -210,8 +223,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) klow_kernel(DecodeParams p) {
   const int64_t G1 = total * (blockIdx.x + 1) / gridDim.x;
   const int nlo = min(p.klow, kLoPlanes);
 
-  for_segments(p.tok_off, p.lens, p.B, G0, G1,
-               [&](int b, int h, int64_t t0, int64_t t1) {
+  for_segments(p.tok_off, p.lens, p.B, G0, G1, [&](int b, int h, int64_t t0, int64_t t1) {
     const int r = b * p.Hq + h, kvh = h / p.g;
     const float* qdr = p.qd + (int64_t)r * n;
     const bool stage = (t1 - t0) * p.klow >= (int64_t)(n / 2);
@@ -235,30 +247,33 @@ __global__ void __launch_bounds__(kScanThreads, 1) klow_kernel(DecodeParams p) {
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int64_t t = tb + tid + u * kScanThreads;
-        if (t >= t1) continue;
-        float s = 0.0f;
+        uint32_t bin = 0xFFFFFFFFu;
+        if (t < t1) {
+          float s = 0.0f;
 #pragma unroll
-        for (int j = 0; j < kLoPlanes; ++j) {
-          if (j >= nlo) break;
-          const uint32_t idx = word_idx(wv[u][j]);
-          if (idx >= (uint32_t)n) {
-            record_error(p.hdr, SDK_ERR_DEVICE_CHECK, idx);
-            continue;
+          for (int j = 0; j < kLoPlanes; ++j) {
+            if (j >= nlo) break;
+            const uint32_t idx = word_idx(wv[u][j]);
+            if (idx >= (uint32_t)n) {
+              record_error(p.hdr, SDK_ERR_DEVICE_CHECK, idx);
+              continue;
+            }
+            s = fmaf(word_coef(wv[u][j]), src[idx], s);
           }
-          s = fmaf(word_coef(wv[u][j]), src[idx], s);
-        }
-        for (int j = kLoPlanes; j < p.klow; ++j) {
-          const uint32_t wj = __ldg(rec + t * kAtoms + j);
-          const uint32_t idx = word_idx(wj);
-          if (idx >= (uint32_t)n) {
-            record_error(p.hdr, SDK_ERR_DEVICE_CHECK, idx);
-            continue;
+          for (int j = kLoPlanes; j < p.klow; ++j) {
+            const uint32_t wj = __ldg(rec + t * kAtoms + j);
+            const uint32_t idx = word_idx(wj);
+            if (idx >= (uint32_t)n) {
+              record_error(p.hdr, SDK_ERR_DEVICE_CHECK, idx);
+              continue;
+            }
+            s = fmaf(word_coef(wj), src[idx], s);
           }
-          s = fmaf(word_coef(wj), src[idx], s);
+          const uint32_t key = score_key(s);
+          keys[t] = key;
+          bin = key >> 20;
         }
-        const uint32_t key = score_key(s);
-        keys[t] = key;
-        atomicAdd(&sh[key >> 20], 1u);
+        hist_add_warp(sh, bin);
       }
     }
     __syncthreads();
@@ -270,25 +285,26 @@ __global__ void __launch_bounds__(kScanThreads, 1) klow_kernel(DecodeParams p) {
 }
 
 // ------------------------------------------------------------- pass2_kernel
-constexpr int kPass2PerThread = 4;
-
+// Tokens above the bucket of the k-th key are selected, tokens inside it
+// become candidates (with a histogram of key bits 19..8), the others go to
+// the complement.  Each warp compacts 128 tokens per iteration with ballots
+// and reserves its output slots with one atomic per category.
 __global__ void __launch_bounds__(kScanThreads) pass2_kernel(DecodeParams p) {
   __shared__ uint32_t s_tmp[48];
-  __shared__ uint32_t s_base[4];
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned lt = (1u << lane) - 1u;
   const int64_t total = p.tok_off[p.B];
   const int64_t G0 = total * blockIdx.x / gridDim.x;
   const int64_t G1 = total * (blockIdx.x + 1) / gridDim.x;
 
-  for_segments(p.tok_off, p.lens, p.B, G0, G1,
-               [&](int b, int h, int64_t t0, int64_t t1) {
+  for_segments(p.tok_off, p.lens, p.B, G0, G1, [&](int b, int h, int64_t t0, int64_t t1) {
     const int r = b * p.Hq + h;
     const int Nb = p.lens[b];
     sdk_select_state* st = p.st + r;
     uint32_t b1, above1, cnt1;
     bool bad;
-    block_find_desc<4096>(p.hist1 + (int64_t)r * 4096, (uint32_t)p.kcnt[b],
-                          s_tmp, b1, above1, cnt1, bad);
+    block_find_desc<4096>(p.hist1 + (int64_t)r * 4096, (uint32_t)p.kcnt[b], s_tmp, b1, above1,
+                          cnt1, bad);
     if (bad) {
       if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x10000000u | r);
       return;
@@ -300,86 +316,89 @@ __global__ void __launch_bounds__(kScanThreads) pass2_kernel(DecodeParams p) {
     uint32_t* ck = p.cand_key + (int64_t)r * p.L;
     uint32_t* h2 = p.hist2 + (int64_t)r * 4096;
     uint32_t cmax = 0u;
-    for (int64_t tb = t0; tb < t1; tb += kPass2PerThread * kScanThreads) {
-      uint32_t key[kPass2PerThread];
-      uint32_t nsel = 0, ncand = 0, ncomp = 0;
+    const int nwarps = kScanThreads / 32;
+    for (int64_t tb = t0 + (int64_t)warp * 128; tb < t1; tb += (int64_t)nwarps * 128) {
+      uint32_t key[4];
+      unsigned ms[4], mc[4], mo[4];
+      uint32_t ns = 0, nc = 0, no = 0;
 #pragma unroll
-      for (int u = 0; u < kPass2PerThread; ++u) {
-        const int64_t t = tb + tid + u * kScanThreads;
-        key[u] = t < t1 ? keys[t] : 0u;
-        if (t < t1) {
-          const uint32_t d1 = key[u] >> 20;
-          if (d1 > b1) ++nsel;
-          else if (d1 == b1) ++ncand;
-          else ++ncomp;
-        }
-      }
-      uint32_t tot_sc, tot_comp;
-      const uint32_t inc_sc = block_incl_scan(nsel | (ncand << 16), s_tmp, &tot_sc);
-      const uint32_t inc_comp = p.full ? block_incl_scan(ncomp, s_tmp, &tot_comp) : 0u;
-      if (tid == 0) {
-        s_base[0] = (tot_sc & 0xFFFFu) ? atomicAdd(&st->n_sel, tot_sc & 0xFFFFu) : 0u;
-        s_base[1] = (tot_sc >> 16) ? atomicAdd(&st->n_cand, tot_sc >> 16) : 0u;
-        s_base[2] = (p.full && tot_comp) ? atomicAdd(&st->n_comp, tot_comp) : 0u;
-      }
-      __syncthreads();
-      uint32_t psel = s_base[0] + (inc_sc & 0xFFFFu) - nsel;
-      uint32_t pcand = s_base[1] + (inc_sc >> 16) - ncand;
-      uint32_t pcomp = s_base[2] + inc_comp - ncomp;
-      __syncthreads();
-#pragma unroll
-      for (int u = 0; u < kPass2PerThread; ++u) {
-        const int64_t t = tb + tid + u * kScanThreads;
-        if (t >= t1) continue;
+      for (int u = 0; u < 4; ++u) {
+        const int64_t t = tb + lane + 32 * u;
+        const bool valid = t < t1;
+        key[u] = valid ? keys[t] : 0u;
         const uint32_t d1 = key[u] >> 20;
-        if (d1 > b1) {
-          if (psel < (uint32_t)Nb) list[psel] = (int32_t)t;
-          ++psel;
-        } else if (d1 == b1) {
-          if (pcand < (uint32_t)Nb) {
-            ct[pcand] = (int32_t)t;
-            ck[pcand] = key[u];
+        ms[u] = __ballot_sync(0xffffffffu, valid && d1 > b1);
+        mc[u] = __ballot_sync(0xffffffffu, valid && d1 == b1);
+        mo[u] = __ballot_sync(0xffffffffu, valid && d1 < b1 && p.full);
+        ns += __popc(ms[u]);
+        nc += __popc(mc[u]);
+        no += __popc(mo[u]);
+      }
+      uint32_t bs = 0, bc = 0, bo = 0;
+      if (lane == 0) {
+        if (ns) bs = atomicAdd(&st->n_sel, ns);
+        if (nc) bc = atomicAdd(&st->n_cand, nc);
+        if (no) bo = atomicAdd(&st->n_comp, no);
+      }
+      bs = __shfl_sync(0xffffffffu, bs, 0);
+      bc = __shfl_sync(0xffffffffu, bc, 0);
+      bo = __shfl_sync(0xffffffffu, bo, 0);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t t = tb + lane + 32 * u;
+        if ((ms[u] >> lane) & 1u) {
+          const uint32_t pos = bs + __popc(ms[u] & lt);
+          if (pos < (uint32_t)Nb) list[pos] = (int32_t)t;
+        } else if ((mc[u] >> lane) & 1u) {
+          const uint32_t pos = bc + __popc(mc[u] & lt);
+          if (pos < (uint32_t)Nb) {
+            ct[pos] = (int32_t)t;
+            ck[pos] = key[u];
           }
-          ++pcand;
           atomicAdd(&h2[(key[u] >> 8) & 0xFFFu], 1u);
-        } else if (p.full) {
-          if (pcomp < (uint32_t)Nb) list[Nb - 1 - (int64_t)pcomp] = (int32_t)t;
-          ++pcomp;
+        } else if ((mo[u] >> lane) & 1u) {
+          const uint32_t pos = bo + __popc(mo[u] & lt);
+          if (pos < (uint32_t)Nb) list[Nb - 1 - (int64_t)pos] = (int32_t)t;
           cmax = max(cmax, key[u]);
         }
+        bs += __popc(ms[u]);
+        bc += __popc(mc[u]);
+        bo += __popc(mo[u]);
       }
     }
     if (p.full) {
       cmax = warp_umax(cmax);
-      if ((tid & 31) == 0 && cmax) atomicMax(&st->max_comp, cmax);
+      if (lane == 0 && cmax) atomicMax(&st->max_comp, cmax);
     }
     __syncthreads();
   });
 }
 
 // ------------------------------------------------------------- final_kernel
-// One CTA per query head.
+// One CTA per query head: the last two radix digits over the candidates, the
+// exact k-th key, the tie rule (lower token index first) and the rest of the
+// selected set.
 __global__ void __launch_bounds__(kScanThreads) final_kernel(DecodeParams p) {
   __shared__ uint32_t s_tmp[48];
   __shared__ uint32_t sh[2048];
-  __shared__ uint32_t s_base[4];
-  const int r = blockIdx.x, tid = threadIdx.x;
+  __shared__ uint32_t s_cnt[2];
+  const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned lt = (1u << lane) - 1u;
   const int b = r / p.Hq;
   const int Nb = p.lens[b];
   const uint32_t k = (uint32_t)p.kcnt[b];
   sdk_select_state* st = p.st + r;
   const uint32_t n_cand = st->n_cand;
   const uint32_t n_above = st->n_above;
-  if (st->n_sel != n_above || n_above >= k || n_cand == 0u) {
+  if (st->n_sel != n_above || n_above >= k || n_cand == 0u || n_cand > (uint32_t)Nb) {
     if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x20000000u | r);
     return;
   }
   const uint32_t* ck = p.cand_key + (int64_t)r * p.L;
   const int32_t* ct = p.cand_t + (int64_t)r * p.L;
   int32_t* list = p.list + (int64_t)r * p.L;
-  const uint32_t k1 = k - n_above;  // rank inside the pass-1 bucket
+  const uint32_t k1 = k - n_above;
 
-  // digit 2 (bits 19..8) from the global histogram
   uint32_t b2, above2, cnt2, b3, above3, cnt3;
   bool bad;
   block_find_desc<4096>(p.hist2 + (int64_t)r * 4096, k1, s_tmp, b2, above2, cnt2, bad);
@@ -388,7 +407,6 @@ __global__ void __launch_bounds__(kScanThreads) final_kernel(DecodeParams p) {
     return;
   }
   const uint32_t k2 = k1 - above2;
-  // digit 3 (bits 7..0) over the candidates in bucket b2
   for (int i = tid; i < 256; i += kScanThreads) sh[i] = 0u;
   __syncthreads();
   for (uint32_t i = tid; i < n_cand; i += kScanThreads) {
@@ -406,17 +424,15 @@ __global__ void __launch_bounds__(kScanThreads) final_kernel(DecodeParams p) {
   const uint32_t eq_take = k2 - above3;
   const uint32_t eq_total = cnt3;
 
-  // With more ties than places, the places go to the lowest token indices:
-  // radix-select the eq_take-th smallest token index among the ties
-  // (digits 31..21, 20..10, 9..0; bins stored in reverse so the descending
-  // search walks ascending token indices).
+  // more ties than places: the eq_take-th smallest token index among the
+  // ties, by radix select over index digits 31..21, 20..10, 9..0 (bins kept
+  // in reverse so the descending search walks ascending indices)
   uint32_t t_cut = 0xFFFFFFFFu;
   if (eq_total > eq_take) {
     uint32_t prefix = 0u, rank = eq_take;
-    const int shifts[3] = {21, 10, 0};
-    const int widths[3] = {11, 11, 10};
     for (int ps = 0; ps < 3; ++ps) {
-      const int sh_lo = shifts[ps], wbits = widths[ps];
+      const int sh_lo = ps == 0 ? 21 : (ps == 1 ? 10 : 0);
+      const int wbits = ps == 2 ? 10 : 11;
       const uint32_t nb = 1u << wbits;
       for (int i = tid; i < 2048; i += kScanThreads) sh[i] = 0u;
       __syncthreads();
@@ -425,8 +441,7 @@ __global__ void __launch_bounds__(kScanThreads) final_kernel(DecodeParams p) {
         const uint32_t t = (uint32_t)ct[i];
         const uint32_t hi = (ps == 0) ? 0u : (t >> (sh_lo + wbits));
         if (hi != prefix) continue;
-        const uint32_t dg = (t >> sh_lo) & (nb - 1u);
-        atomicAdd(&sh[2047u - dg], 1u);
+        atomicAdd(&sh[2047u - ((t >> sh_lo) & (nb - 1u))], 1u);
       }
       __syncthreads();
       uint32_t bin, above, cnt;
@@ -435,65 +450,67 @@ __global__ void __launch_bounds__(kScanThreads) final_kernel(DecodeParams p) {
         if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x23000000u | r);
         return;
       }
-      const uint32_t dg = 2047u - bin;
-      prefix = (prefix << wbits) | dg;
+      prefix = (prefix << wbits) | (2047u - bin);
       rank -= above;
     }
-    t_cut = prefix;  // the eq_take-th smallest tie index
+    t_cut = prefix;
   }
 
-  // classify the candidates; write selected to the front, the rest (with
-  // full_softmax) to the back of the list
+  if (tid == 0) {
+    s_cnt[0] = n_above;
+    s_cnt[1] = st->n_comp;
+  }
+  __syncthreads();
   uint32_t cmax = 0u;
-  for (uint32_t i0 = 0; i0 < n_cand; i0 += kScanThreads) {
-    const uint32_t i = i0 + tid;
+  for (uint32_t i0 = (uint32_t)warp * 32; i0 < n_cand; i0 += kScanThreads) {
+    const uint32_t i = i0 + lane;
     uint32_t key = 0u, t = 0u;
     bool sel = false, comp = false;
     if (i < n_cand) {
       key = ck[i];
       t = (uint32_t)ct[i];
       sel = key > T || (key == T && t <= t_cut);
-      comp = !sel;
+      comp = !sel && p.full;
     }
-    uint32_t tot_s, tot_c;
-    const uint32_t inc = block_incl_scan((sel ? 1u : 0u) | ((comp && p.full) ? 0x10000u : 0u),
-                                         s_tmp, &tot_s);
-    (void)tot_c;
-    if (tid == 0) {
-      s_base[0] = atomicAdd(&st->n_sel, tot_s & 0xFFFFu);
-      s_base[1] = p.full ? atomicAdd(&st->n_comp, tot_s >> 16) : 0u;
+    const unsigned msel = __ballot_sync(0xffffffffu, sel);
+    const unsigned mcomp = __ballot_sync(0xffffffffu, comp);
+    uint32_t bs = 0, bo = 0;
+    if (lane == 0) {
+      if (msel) bs = atomicAdd(&s_cnt[0], (uint32_t)__popc(msel));
+      if (mcomp) bo = atomicAdd(&s_cnt[1], (uint32_t)__popc(mcomp));
     }
-    __syncthreads();
+    bs = __shfl_sync(0xffffffffu, bs, 0) + __popc(msel & lt);
+    bo = __shfl_sync(0xffffffffu, bo, 0) + __popc(mcomp & lt);
     if (sel) {
-      const uint32_t pos = s_base[0] + (inc & 0xFFFFu) - 1u;
-      if (pos < k) list[pos] = (int32_t)t;
+      if (bs < k) list[bs] = (int32_t)t;
       else record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x26000000u | r);
     }
-    if (comp && p.full) {
-      const uint32_t pos = s_base[1] + (inc >> 16) - 1u;
-      if (pos < (uint32_t)Nb) list[Nb - 1 - (int64_t)pos] = (int32_t)t;
+    if (comp) {
+      if (bo < (uint32_t)Nb) list[Nb - 1 - (int64_t)bo] = (int32_t)t;
       else record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x27000000u | r);
       cmax = max(cmax, key);
     }
-    __syncthreads();
   }
   if (p.full) {
     cmax = warp_umax(cmax);
-    if ((tid & 31) == 0 && cmax) atomicMax(&st->max_comp, cmax);
+    if (lane == 0 && cmax) atomicMax(&st->max_comp, cmax);
   }
   __syncthreads();
   if (tid == 0) {
     st->kth_key = T;
     st->eq_total = eq_total;
     st->eq_taken = eq_take;
-    __threadfence();
-    if (st->n_sel != k) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x24000000u | r);
-    if (p.full && st->n_sel + st->n_comp != (uint32_t)Nb)
+    st->n_sel = s_cnt[0];
+    st->n_comp = s_cnt[1];
+    if (s_cnt[0] != k) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x24000000u | r);
+    if (p.full && s_cnt[0] + s_cnt[1] != (uint32_t)Nb)
       record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x25000000u | r);
   }
 }
 
 // ----------------------------------------------------------- rescore_kernel
+// s_t = scale * sum_{j<khigh} c_tj QD[idx_tj] for the selected tokens; two
+// tokens per thread per iteration keep 128 bytes of records in flight.
 __global__ void __launch_bounds__(kScanThreads, 1) rescore_kernel(DecodeParams p) {
   extern __shared__ float4 smem4[];
   float* sq = reinterpret_cast<float*>(smem4);
@@ -502,96 +519,130 @@ __global__ void __launch_bounds__(kScanThreads, 1) rescore_kernel(DecodeParams p
   const int64_t G0 = total * blockIdx.x / gridDim.x;
   const int64_t G1 = total * (blockIdx.x + 1) / gridDim.x;
 
-  for_segments(p.sel_off, p.kcnt, p.B, G0, G1,
-               [&](int b, int h, int64_t i0, int64_t i1) {
+  for_segments(p.sel_off, p.kcnt, p.B, G0, G1, [&](int b, int h, int64_t i0, int64_t i1) {
     const int r = b * p.Hq + h, kvh = h / p.g;
     const float* qdr = p.qd + (int64_t)r * n;
     const bool stage = (i1 - i0) * p.khigh >= (int64_t)(n / 2);
     if (stage) stage_row(sq, qdr, n);
     __syncthreads();
     const float* src = stage ? sq : qdr;
-    const uint4* rec = reinterpret_cast<const uint4*>(
-        p.k_full + ((int64_t)b * p.Hkv + kvh) * p.cap * kAtoms);
+    const uint4* rec = reinterpret_cast<const uint4*>(p.k_full +
+                                                      ((int64_t)b * p.Hkv + kvh) * p.cap * kAtoms);
     const int32_t* list = p.list + (int64_t)r * p.L;
     float* out = p.sel_score + (int64_t)r * p.L;
-    float smax = -INFINITY;
     const int Nb = p.lens[b];
-    for (int64_t i = i0 + tid; i < i1; i += kScanThreads) {
-      const int64_t t = list[i];
-      if (t < 0 || t >= Nb) {
-        record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x30000000u | r);
-        out[i] = -INFINITY;
-        continue;
+    float smax = -INFINITY;
+    for (int64_t ib = i0; ib < i1; ib += 2 * kScanThreads) {
+      int64_t t[2];
+      uint4 wv[2][4];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int64_t i = ib + tid + u * kScanThreads;
+        t[u] = i < i1 ? (int64_t)list[i] : -1;
+        if (i < i1 && (t[u] < 0 || t[u] >= Nb)) {
+          record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x30000000u | r);
+          t[u] = -1;
+        }
       }
-      uint4 wv[4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) wv[c] = __ldcs(rec + t * 4 + c);
-      const uint32_t* wd = reinterpret_cast<const uint32_t*>(wv);
-      float s = 0.0f;
+      for (int u = 0; u < 2; ++u)
 #pragma unroll
-      for (int j = 0; j < kAtoms; ++j) {
-        if (j >= p.khigh) break;
-        const uint32_t idx = word_idx(wd[j]);
-        if (idx >= (uint32_t)n) {
-          record_error(p.hdr, SDK_ERR_DEVICE_CHECK, idx);
+        for (int c = 0; c < 4; ++c)
+          wv[u][c] = t[u] >= 0 ? __ldcs(rec + t[u] * 4 + c) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int64_t i = ib + tid + u * kScanThreads;
+        if (i >= i1) continue;
+        if (t[u] < 0) {
+          out[i] = -INFINITY;
           continue;
         }
-        s = fmaf(word_coef(wd[j]), src[idx], s);
+        const uint32_t* wd = reinterpret_cast<const uint32_t*>(wv[u]);
+        float s = 0.0f;
+#pragma unroll
+        for (int j = 0; j < kAtoms; ++j) {
+          if (j >= p.khigh) break;
+          const uint32_t idx = word_idx(wd[j]);
+          if (idx >= (uint32_t)n) {
+            record_error(p.hdr, SDK_ERR_DEVICE_CHECK, idx);
+            continue;
+          }
+          s = fmaf(word_coef(wd[j]), src[idx], s);
+        }
+        s *= p.scale;
+        out[i] = s;
+        smax = fmaxf(smax, s);
       }
-      s *= p.scale;
-      out[i] = s;
-      smax = fmaxf(smax, s);
     }
     smax = warp_max(smax);
-    if ((tid & 31) == 0 && smax > -INFINITY)
-      atomicMax(&p.st[r].max_score, score_key(smax));
+    if ((tid & 31) == 0 && smax > -INFINITY) atomicMax(&p.st[r].max_score, score_key(smax));
     __syncthreads();
   });
 }
 
 // ------------------------------------------------------------- value_kernel
-__global__ void __launch_bounds__(kScanThreads, 1) value_kernel(DecodeParams p) {
+// One cluster of C CTAs per query head.  Each CTA scatters
+// e_t * c^V_tj into a shared-memory per-atom weight tile for its share of
+// the head's softmax domain (e_t = exp(logit_t - max)); the cluster then
+// sums the C tiles through distributed shared memory and writes w[r] and
+// the softmax denominator z[r] once, with plain stores.
+__global__ void __launch_bounds__(kScanThreads, 1) value_kernel(DecodeParams p, int C) {
   extern __shared__ float4 smem4[];
   float* sw = reinterpret_cast<float*>(smem4);
-  __shared__ float s_red[32];
+  __shared__ float s_red[kScanThreads / 32];
+  __shared__ float s_z;
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
   const int n = p.n, tid = threadIdx.x;
-  const int64_t total = p.dom_off[p.B];
-  const int64_t G0 = total * blockIdx.x / gridDim.x;
-  const int64_t G1 = total * (blockIdx.x + 1) / gridDim.x;
+  const int r = blockIdx.x / C;
+  const int rank = (int)cluster.block_rank();
+  const int b = r / p.Hq, h = r % p.Hq, kvh = h / p.g;
+  const int64_t Dr = p.dcnt[b];
+  const int64_t i0 = Dr * rank / C, i1 = Dr * (rank + 1) / C;
+  const int k = p.kcnt[b];
+  const int Nb = p.lens[b];
+  const sdk_select_state* st = p.st + r;
+  float m = key_score(st->max_score);
+  if (p.full && st->n_comp > 0u) m = fmaxf(m, p.scale * key_score(st->max_comp));
 
-  for_segments(p.dom_off, p.dcnt, p.B, G0, G1,
-               [&](int b, int h, int64_t i0, int64_t i1) {
-    const int r = b * p.Hq + h, kvh = h / p.g;
-    const sdk_select_state* st = p.st + r;
-    const int k = p.kcnt[b];
-    float m = key_score(st->max_score);
-    if (p.full && st->n_comp > 0u) m = fmaxf(m, p.scale * key_score(st->max_comp));
-    const bool smem_w = (i1 - i0) * kAtoms >= (int64_t)(n / 2);
-    if (smem_w) {
-      for (int i = tid; i < n; i += kScanThreads) sw[i] = 0.0f;
-      __syncthreads();
-    }
-    float* wdst = smem_w ? sw : p.w + (int64_t)r * n;
-    const uint4* rec = reinterpret_cast<const uint4*>(
-        p.v_full + ((int64_t)b * p.Hkv + kvh) * p.cap * kAtoms);
-    const int32_t* list = p.list + (int64_t)r * p.L;
-    const float* ss = p.sel_score + (int64_t)r * p.L;
-    const uint32_t* keys = p.keys + (int64_t)r * p.L;
-    float z = 0.0f;
-    const int Nb = p.lens[b];
-    for (int64_t i = i0 + tid; i < i1; i += kScanThreads) {
-      const int64_t t = list[i];
-      if (t < 0 || t >= Nb) {
-        record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x31000000u | r);
-        continue;
-      }
-      const float logit = (i < k) ? ss[i] : p.scale * key_score(keys[t]);
-      const float e = expf(logit - m);
-      z += e;
-      uint4 wv[4];
+  for (int i = tid; i < n; i += kScanThreads) sw[i] = 0.0f;
+  __syncthreads();
+  const uint4* rec = reinterpret_cast<const uint4*>(p.v_full +
+                                                    ((int64_t)b * p.Hkv + kvh) * p.cap * kAtoms);
+  const int32_t* list = p.list + (int64_t)r * p.L;
+  const float* ss = p.sel_score + (int64_t)r * p.L;
+  const uint32_t* keys = p.keys + (int64_t)r * p.L;
+  float z = 0.0f;
+  for (int64_t ib = i0; ib < i1; ib += 2 * kScanThreads) {
+    int64_t t[2];
+    float e[2];
+    uint4 wv[2][4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) wv[c] = __ldcs(rec + t * 4 + c);
-      const uint32_t* wd = reinterpret_cast<const uint32_t*>(wv);
+    for (int u = 0; u < 2; ++u) {
+      const int64_t i = ib + tid + u * kScanThreads;
+      t[u] = i < i1 ? (int64_t)list[i] : -1;
+      if (i < i1 && (t[u] < 0 || t[u] >= Nb)) {
+        record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x31000000u | r);
+        t[u] = -1;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        wv[u][c] = t[u] >= 0 ? __ldcs(rec + t[u] * 4 + c) : make_uint4(0u, 0u, 0u, 0u);
+      const int64_t i = ib + tid + u * kScanThreads;
+      e[u] = 0.0f;
+      if (t[u] >= 0) {
+        const float logit = (i < k) ? ss[i] : p.scale * key_score(keys[t[u]]);
+        e[u] = expf(logit - m);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (t[u] < 0) continue;
+      z += e[u];
+      const uint32_t* wd = reinterpret_cast<const uint32_t*>(wv[u]);
 #pragma unroll
       for (int j = 0; j < kAtoms; ++j) {
         const uint32_t idx = word_idx(wd[j]);
@@ -599,57 +650,64 @@ __global__ void __launch_bounds__(kScanThreads, 1) value_kernel(DecodeParams p) 
           record_error(p.hdr, SDK_ERR_DEVICE_CHECK, idx);
           continue;
         }
-        atomicAdd(&wdst[idx], e * word_coef(wd[j]));
+        atomicAdd(&sw[idx], e[u] * word_coef(wd[j]));
       }
     }
-    z = warp_sum(z);
-    if ((tid & 31) == 0) s_red[tid >> 5] = z;
-    __syncthreads();
-    if (tid == 0) {
-      float zz = 0.0f;
-      for (int i = 0; i < kScanThreads / 32; ++i) zz += s_red[i];
-      atomicAdd(&p.st[r].z, zz);
-    }
-    if (smem_w) {
-      float* gw = p.w + (int64_t)r * n;
-      for (int i = tid; i < n; i += kScanThreads) {
-        const float v = sw[i];
-        if (v != 0.0f) atomicAdd(&gw[i], v);
-      }
-    }
-    __syncthreads();
-  });
+  }
+  z = warp_sum(z);
+  if ((tid & 31) == 0) s_red[tid >> 5] = z;
+  __syncthreads();
+  if (tid == 0) {
+    float zz = 0.0f;
+    for (int i = 0; i < kScanThreads / 32; ++i) zz += s_red[i];
+    s_z = zz;
+  }
+  cluster.sync();
+  // reduce this CTA's slice of the atoms over the C tiles of the cluster
+  const int a0 = (int)((int64_t)n * rank / C), a1 = (int)((int64_t)n * (rank + 1) / C);
+  float* gw = p.w + (int64_t)r * n;
+  for (int a = a0 + tid; a < a1; a += kScanThreads) {
+    float sum = 0.0f;
+    for (int c = 0; c < C; ++c) sum += cluster.map_shared_rank(sw, c)[a];
+    gw[a] = sum;
+  }
+  if (rank == 0 && tid == 0) {
+    float zz = 0.0f;
+    for (int c = 0; c < C; ++c) zz += *cluster.map_shared_rank(&s_z, c);
+    p.st[r].z = zz;
+  }
+  cluster.sync();
 }
 
 // --------------------------------------------------------------- out_kernel
-// part[tile][r][k] = sum_{a in tile} w[r][a] D_V[a][k]   (128-atom tiles,
-// 32-row blocks).
+// out[r][k] += (1/z[r]) sum_{a in tile} w[r][a] D_V[a][k] over a 128-atom
+// tile and a 32-row block; thread (tk, tr) owns columns tk*C.. and rows
+// 8tr..8tr+7; results are added with vector reductions.
 template <int D>
-__global__ void __launch_bounds__(256) out_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kQdThreads) out_kernel(DecodeParams p) {
   extern __shared__ float4 smem4[];
   float* Ds = reinterpret_cast<float*>(smem4);  // [128][D]
   float* Ws = Ds + 128 * D;                     // [128][32]
   const int n = p.n, R = p.R, tid = threadIdx.x;
   const int a0 = blockIdx.x * 128, r0 = blockIdx.y * 32;
-  for (int e = tid; e < 128 * (D / 8); e += 256) {
+  for (int e = tid; e < 128 * (D / 8); e += kQdThreads) {
     const int a = e / (D / 8), c = e % (D / 8);
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (a0 + a < n)
-      v = __ldg(reinterpret_cast<const uint4*>(p.dv + (int64_t)(a0 + a) * D) + c);
+    if (a0 + a < n) v = __ldg(reinterpret_cast<const uint4*>(p.dv + (int64_t)(a0 + a) * D) + c);
     float4* d = reinterpret_cast<float4*>(Ds + a * D + c * 8);
     d[0] = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
     d[1] = make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
   }
-  for (int e = tid; e < 128 * 32; e += 256) {
+  for (int e = tid; e < 128 * 32; e += kQdThreads) {
     const int r = e & 31, a = e >> 5;
     Ws[a * 32 + r] = (r0 + r < R && a0 + a < n) ? p.w[(int64_t)(r0 + r) * n + a0 + a] : 0.0f;
   }
   __syncthreads();
   constexpr int C = D / 32;
   const int tk = tid & 31, tr = tid >> 5;
-  float acc[4][C];
+  float acc[8][C];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int c = 0; c < C; ++c) acc[i][c] = 0.0f;
 #pragma unroll 4
@@ -662,31 +720,30 @@ __global__ void __launch_bounds__(256) out_kernel(DecodeParams p) {
       const float2 v = *reinterpret_cast<const float2*>(Ds + a * D + tk * 2);
       dv[0] = v.x; dv[1] = v.y;
     }
-    const float4 wv = *reinterpret_cast<const float4*>(Ws + a * 32 + 4 * tr);
-    const float wr[4] = {wv.x, wv.y, wv.z, wv.w};
+    const float4 wa = *reinterpret_cast<const float4*>(Ws + a * 32 + 8 * tr);
+    const float4 wb = *reinterpret_cast<const float4*>(Ws + a * 32 + 8 * tr + 4);
+    const float wr[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
       for (int c = 0; c < C; ++c) acc[i][c] = fmaf(wr[i], dv[c], acc[i][c]);
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = r0 + 4 * tr + i;
+  for (int i = 0; i < 8; ++i) {
+    const int r = r0 + 8 * tr + i;
     if (r >= R) continue;
-    float* dst = p.part + ((int64_t)blockIdx.x * R + r) * D + tk * C;
-#pragma unroll
-    for (int c = 0; c < C; ++c) dst[c] = acc[i][c];
+    const float iz = 1.0f / p.st[r].z;
+    float* dst = p.out + (int64_t)r * D + tk * C;
+    if constexpr (C == 4) {
+      asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(acc[i][0] * iz),
+                   "f"(acc[i][1] * iz), "f"(acc[i][2] * iz), "f"(acc[i][3] * iz)
+                   : "memory");
+    } else {
+      asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(dst), "f"(acc[i][0] * iz),
+                   "f"(acc[i][1] * iz)
+                   : "memory");
+    }
   }
-}
-
-__global__ void out_reduce_kernel(DecodeParams p) {
-  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t total = (int64_t)p.R * p.d;
-  if (e >= total) return;
-  const int r = (int)(e / p.d);
-  float s = 0.0f;
-  for (int t = 0; t < p.n_out_tiles; ++t) s += p.part[((int64_t)t * p.R) * p.d + e];
-  p.out[e] = s / p.st[r].z;
 }
 
 // --------------------------------------------------------------- launcher
@@ -701,6 +758,7 @@ sdk_decode_layout decode_layout(int B, int Hq, int d, int n, int64_t L) {
     off = align_up(off + bytes, 256);
     return o;
   };
+  (void)d;
   l.header = take(sizeof(WsHeader));
   l.qd = take(R * n * 4);
   l.keys = take(R * L * 4);
@@ -712,8 +770,7 @@ sdk_decode_layout decode_layout(int B, int Hq, int d, int n, int64_t L) {
   l.cand_key = take(R * L * 4);
   l.sel_score = take(R * L * 4);
   l.w = take(R * n * 4);
-  const size_t tiles = (size_t)(n + 127) / 128;
-  l.part = take(tiles * R * d * 4);
+  l.part = take(0);
   l.total = off;
   return l;
 }
@@ -725,58 +782,68 @@ static int grid_for(int64_t work, int64_t per_cta, int cap_ctas) {
   return (int)g;
 }
 
-sdk_status launch_decode(const DecodeParams& p0, cudaStream_t stream) {
-  DecodeParams p = p0;
+sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
   const int sms = num_sms();
   const size_t qd_smem = (size_t)((p.n + 3) & ~3) * 4;
-  cudaError_t e;
-
-  // qd + zeroing
-  {
-    dim3 grid((p.n + 63) / 64, (p.R + 31) / 32);
-    if (p.d == 128) qd_kernel<128><<<grid, 256, 0, stream>>>(p);
-    else qd_kernel<64><<<grid, 256, 0, stream>>>(p);
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(qd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 80 * 1024);
+    cudaFuncSetAttribute(qd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 80 * 1024);
+    cudaFuncSetAttribute(out_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 80 * 1024);
+    cudaFuncSetAttribute(out_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 80 * 1024);
+    cudaFuncSetAttribute(klow_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    cudaFuncSetAttribute(rescore_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    cudaFuncSetAttribute(value_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    cudaFuncSetAttribute(value_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+    attr = true;
   }
-  // klow scan
   {
-    const size_t smem = qd_smem + 4096 * 4;
-    static bool attr = false;
-    if (!attr) {
-      cudaFuncSetAttribute(klow_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-      cudaFuncSetAttribute(rescore_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-      cudaFuncSetAttribute(value_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-      cudaFuncSetAttribute(out_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-      cudaFuncSetAttribute(out_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-      attr = true;
-    }
+    dim3 grid((p.n + 127) / 128, (p.R + 31) / 32);
+    const size_t smem = (size_t)p.d * 128 * 4 + (size_t)p.d * 32 * 4;
+    if (p.d == 128) qd_kernel<128><<<grid, kQdThreads, smem, stream>>>(p);
+    else qd_kernel<64><<<grid, kQdThreads, smem, stream>>>(p);
+  }
+  {
     const int g = grid_for(p.tok_off[p.B], 2048, sms);
-    klow_kernel<<<g, kScanThreads, smem, stream>>>(p);
+    klow_kernel<<<g, kScanThreads, qd_smem + 4096 * 4, stream>>>(p);
   }
   {
-    const int g = grid_for(p.tok_off[p.B], 4096, 2 * sms);
+    const int g = grid_for(p.tok_off[p.B], 8192, 2 * sms);
     pass2_kernel<<<g, kScanThreads, 0, stream>>>(p);
   }
   final_kernel<<<p.R, kScanThreads, 0, stream>>>(p);
   {
-    const int g = grid_for(p.sel_off[p.B], 1024, sms);
+    int64_t per = p.sel_off[p.B] / (2 * sms);
+    if (per < 512) per = 512;
+    const int g = grid_for(p.sel_off[p.B], per, 2 * sms);
     rescore_kernel<<<g, kScanThreads, qd_smem, stream>>>(p);
   }
   {
-    const int g = grid_for(p.dom_off[p.B], 1024, sms);
-    value_kernel<<<g, kScanThreads, qd_smem, stream>>>(p);
+    int64_t dmax = 0;
+    for (int b = 0; b < p.B; ++b) dmax = p.dcnt[b] > dmax ? p.dcnt[b] : dmax;
+    int C = 1;
+    while (C < 8 && (int64_t)p.R * C * 2 <= sms && dmax / (2 * C) >= 1024) C *= 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.R * C));
+    cfg.blockDim = dim3(kScanThreads);
+    cfg.dynamicSmemBytes = qd_smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)C;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, value_kernel, p, C) != cudaSuccess) return SDK_ERR_CUDA;
   }
   {
-    dim3 grid(p.n_out_tiles, (p.R + 31) / 32);
+    dim3 grid((p.n + 127) / 128, (p.R + 31) / 32);
     const size_t smem = (size_t)128 * p.d * 4 + 128 * 32 * 4;
-    if (p.d == 128) out_kernel<128><<<grid, 256, smem, stream>>>(p);
-    else out_kernel<64><<<grid, 256, smem, stream>>>(p);
+    if (p.d == 128) out_kernel<128><<<grid, kQdThreads, smem, stream>>>(p);
+    else out_kernel<64><<<grid, kQdThreads, smem, stream>>>(p);
   }
-  {
-    const int64_t tot = (int64_t)p.R * p.d;
-    out_reduce_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, stream>>>(p);
-  }
-  e = cudaGetLastError();
-  return e == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
 }
 
 }  // namespace sdk

@@ -469,34 +469,48 @@ __global__ void __launch_bounds__(kThreads, 1)
           tbuf ^= 1u;
           if (tbuf == 0u) tphase ^= 1u;
           if (!active) continue;
+          // max |c~| of each 16-column group (balanced trees, no long
+          // dependent chains), then of the tile
+          float m16[8];
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            float m = 0.0f;
+          for (int g = 0; g < 8; ++g) {
+            const uint32_t* vg = &v[g >> 2][(g & 3) * 16];
+            float t8[8];
 #pragma unroll
-            for (int i = 0; i < 64; ++i) m = fmaxf(m, fabsf(__uint_as_float(v[c][i])));
-            if (m >= thr) {
-              // rare: the chunk holds a value within `band` of the running
-              // maximum.  Drop stale candidates, then keep every column of
-              // the chunk at or above the new threshold.
-              best = fmaxf(best, m);
-              thr = best - band;
-              int w = 0;
+            for (int i = 0; i < 8; ++i)
+              t8[i] = fmaxf(fabsf(__uint_as_float(vg[i])), fabsf(__uint_as_float(vg[i + 8])));
+#pragma unroll
+            for (int i = 0; i < 4; ++i) t8[i] = fmaxf(t8[i], t8[i + 4]);
+            m16[g] = fmaxf(fmaxf(t8[0], t8[2]), fmaxf(t8[1], t8[3]));
+          }
+          const float mt = fmaxf(fmaxf(fmaxf(m16[0], m16[1]), fmaxf(m16[2], m16[3])),
+                                 fmaxf(fmaxf(m16[4], m16[5]), fmaxf(m16[6], m16[7])));
+          if (mt >= thr) {
+            // rare: the tile holds a value within `band` of the running
+            // maximum.  Drop stale candidates, then keep every column at or
+            // above the new threshold.
+            best = fmaxf(best, mt);
+            thr = best - band;
+            int w = 0;
 #pragma unroll 1
-              for (int t = 0; t < cnt; ++t)
-                if (cv[t] >= thr) {
-                  ci[w] = ci[t];
-                  cv[w] = cv[t];
-                  ++w;
-                }
-              cnt = w;
-              const int lim = p.n - (a * kAtomTile + c * 64);
-              const uint32_t cbase = (uint32_t)(a * kAtomTile + c * 64);
+            for (int t = 0; t < cnt; ++t)
+              if (cv[t] >= thr) {
+                ci[w] = ci[t];
+                cv[w] = cv[t];
+                ++w;
+              }
+            cnt = w;
+            const int lim = p.n - a * kAtomTile;
 #pragma unroll
-              for (int i = 0; i < 64; ++i) {
-                const float av = fabsf(__uint_as_float(v[c][i]));
-                if (av >= thr && i < lim) {
+            for (int g = 0; g < 8; ++g) {
+              if (m16[g] < thr) continue;
+              const uint32_t* vg = &v[g >> 2][(g & 3) * 16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float av = fabsf(__uint_as_float(vg[i]));
+                if (av >= thr && g * 16 + i < lim) {
                   if (cnt < kCand) {
-                    ci[cnt] = cbase + i;
+                    ci[cnt] = (uint32_t)(a * kAtomTile + g * 16 + i);
                     cv[cnt] = av;
                     ++cnt;
                   } else {
