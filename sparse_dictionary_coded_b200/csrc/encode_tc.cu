@@ -5,7 +5,7 @@
 // dictionary, coef = <r, d_i*>, r -= coef * d_i* (projection-based greedy
 // pursuit, no least-squares refit).
 //
-// Design (one persistent CTA per SM, 10 warps, warp-specialised):
+// Design (one persistent CTA per SM, 18 warps, warp-specialised):
 //   warp 0      TMA producer: streams the bf16 dictionary through a 4-stage
 //               shared-memory ring in 128-atom tiles (128B-swizzled,
 //               K-major), the same dictionary 16 times per row tile.
@@ -15,16 +15,18 @@
 //               bf16, in shared memory) into one of two TMEM accumulator
 //               buffers; tcgen05.commit frees the ring stage and hands the
 //               buffer to the epilogue.
-//   warps 2..9  epilogue: one thread per residual row.  tcgen05.ld brings
-//               the row's 128 correlations to registers, the buffer is
-//               released at once, and the row keeps the running maximum
+//   warps 2..17 epilogue: two threads per residual row (64 columns each of
+//               every 128-atom tile).  tcgen05.ld brings a thread's
+//               correlations to registers, the buffer is released at once,
+//               and the thread keeps the running maximum
 //               B of |c~| plus every atom with |c~| >= B - band.  band is
 //               twice a rigorous bound on |c~ - c| (bf16 rounding of r by
 //               Cauchy-Schwarz, plus accumulation slack), so the exact
 //               fp32 argmax is always among the kept candidates.  After the
 //               last atom tile of a step the candidates are re-scored in
-//               fp32 (k = 0..D-1 FMA order, the same arithmetic as the
-//               CUDA-core encoder), the pick is written, r is updated in
+//               fp32 by the row's lead thread (k = 0..D-1 FMA order, the
+//               same arithmetic as the CUDA-core encoder), the pick is
+//               written, r is updated in
 //               fp32 (global scratch, L2-resident) and its bf16 copy
 //               becomes the next step's A operand.  A row whose candidate
 //               list overflows is re-picked by an exact fp32 scan of all
@@ -45,8 +47,10 @@ constexpr int kSets = 2;                   // row sets per CTA
 constexpr int kTileRows = kRows * kSets;   // vectors per row tile
 constexpr int kAtomTile = 128;             // atoms per B tile (MMA N)
 constexpr int kStages = 4;
-constexpr int kCand = 8;
-constexpr int kEpiWarps = 8;
+constexpr int kCand = 8;                   // candidates kept per thread
+constexpr int kEpiWarps = 16;
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kLeadWarps = kEpiWarps / 2;  // warps owning whole rows
 constexpr int kThreads = 32 * (2 + kEpiWarps);
 constexpr int kMaxCtas = 160;
 constexpr int kTmemCols = 512;
@@ -59,9 +63,13 @@ struct Cfg {
   static constexpr int kStageBytes = kAtomTile * D * 2;
   static constexpr int kABytes = kRows * D * 2;       // one row set
   static constexpr int kOffA = kStages * kStageBytes;
-  static constexpr int kOffCi = kOffA + kSets * kABytes;
-  static constexpr int kOffCv = kOffCi + kTileRows * kCand * 4;
-  static constexpr int kOffBar = kOffCv + kTileRows * kCand * 4;
+  static constexpr int kOffCw = kOffA + kSets * kABytes;          // candidate words
+  static constexpr int kOffBest = kOffCw + kEpiThreads * kCand * 4;
+  static constexpr int kOffCnt = kOffBest + kEpiThreads * 4;
+  static constexpr int kOffBand = kOffCnt + kEpiThreads * 4;
+  static constexpr int kOffAct = kOffBand + kTileRows * 4;
+  static constexpr int kOffFr = kOffAct + kTileRows * 4;          // fallback residuals
+  static constexpr int kOffBar = kOffFr + kLeadWarps * D * 4;
   static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   // + alignment slack; at least 116 KB so that one CTA (which holds all 512
@@ -206,14 +214,18 @@ __device__ __forceinline__ float bf16_round(float v) {
 
 // ---- the kernel --------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __maxnreg__(112)
     encode_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint32_t* s_ci = reinterpret_cast<uint32_t*>(smem + C::kOffCi);
-  float* s_cv = reinterpret_cast<float*>(smem + C::kOffCv);
+  uint32_t* s_cw = reinterpret_cast<uint32_t*>(smem + C::kOffCw);
+  float* s_best = reinterpret_cast<float*>(smem + C::kOffBest);
+  uint32_t* s_cnt = reinterpret_cast<uint32_t*>(smem + C::kOffCnt);
+  float* s_band = reinterpret_cast<float*>(smem + C::kOffBand);
+  uint32_t* s_act = reinterpret_cast<uint32_t*>(smem + C::kOffAct);
+  float* s_fr = reinterpret_cast<float*>(smem + C::kOffFr);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile uint32_t* s_abort = misc + 0;
@@ -239,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_tfull(b), 1);
       mbar_init(bar_tempty(b), kEpiWarps);
     }
-    mbar_init(bar_afull, kEpiWarps);
+    mbar_init(bar_afull, kLeadWarps);
     mbar_init(bar_done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -351,22 +363,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // 16 warps: (row set, column half) x TMEM lane quarter.  Thread `tix`
+    // scans 64 of the 128 columns of one residual row per atom tile; the
+    // "lead" thread of the row (column half 0) merges both candidate lists
+    // at the end of a step, picks, and updates the residual.
     const int e = warp - 2;
-    const int rs = e >> 2;               // row set
-    const int q = warp & 3;              // TMEM lane quarter of this warp
-    const int rin = q * 32 + lane;       // row within the set (TMEM lane)
-    const int row = rs * kRows + rin;    // row within the tile
+    const int combo = e >> 2;
+    const int rs = combo >> 1, half = combo & 1;
+    const bool lead = half == 0;
+    const int q = warp & 3;                   // TMEM lane quarter of this warp
+    const int rin = q * 32 + lane;            // row within the set (TMEM lane)
+    const int row = rs * kRows + rin;         // row within the tile
+    const int tix = e * 32 + lane;            // partner (other half): tix ^ 128
+    uint32_t* cw = s_cw + tix * kCand;
+    const uint32_t* pcw = s_cw + (tix ^ 128) * kCand;
     float* rres = p.resid + (int64_t)blockIdx.x * D * kTileRows + row;  // stride kTileRows
-    uint32_t* ci = s_ci + row * kCand;
-    float* cv = s_cv + row * kCand;
+    float* fr = s_fr + (rs * 4 + (e & 3)) * D;                           // lead warps only
     const float dmax = *p.dmax;
     uint8_t* arow = smem + C::kOffA + rs * C::kABytes + rin * 128;
     uint32_t tbuf = 0, tphase = 0;
     uint32_t n_rescored = 0;
-    bool ok = true;
+    auto epi_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); };
 
-    // writes bf16(r) of this row into the swizzled A operand and returns
-    // (||r - bf16(r)||^2, ||r||^2) accumulated from the fp32 values
+    // bf16(r) of this row into the swizzled A operand; accumulates
+    // ||r - bf16(r)||^2 and ||r||^2 from the fp32 values
     auto write_a_chunk = [&](int kc, const float (&r8)[8], float& e2, float& n2) {
       uint32_t w[4];
 #pragma unroll
@@ -381,68 +401,77 @@ __global__ void __launch_bounds__(kThreads, 1)
         w[u] = *reinterpret_cast<const uint32_t*>(&h);
       }
       const int kb = kc >> 3, c16 = kc & 7;
-      uint4* dst = reinterpret_cast<uint4*>(arow + kb * (kRows * 128) +
-                                            ((c16 ^ (rin & 7)) << 4));
+      uint4* dst = reinterpret_cast<uint4*>(arow + kb * (kRows * 128) + ((c16 ^ (rin & 7)) << 4));
       *dst = make_uint4(w[0], w[1], w[2], w[3]);
     };
+    // twice the bound on |c~ - c|: bf16 rounding of r (Cauchy-Schwarz with
+    // the largest atom norm) plus slack for the accumulation order
     auto band_of = [&](float e2, float n2) {
       return 2.0f * dmax * sqrtf(e2) + 0.000244140625f * dmax * sqrtf(n2);
     };
     // fp32 correlation in k order (the CUDA-core encoder's arithmetic)
     auto dot_atom = [&](uint32_t i) {
       const uint4* dp = reinterpret_cast<const uint4*>(p.dict + (int64_t)i * D);
-      float s = 0.0f;
+      float sd = 0.0f;
 #pragma unroll 4
       for (int kc = 0; kc < D / 8; ++kc) {
         const uint4 dv = __ldg(dp + kc);
         const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          s = fmaf(rres[(kc * 8 + 2 * u) * kTileRows], bf16_lo(dw[u]), s);
-          s = fmaf(rres[(kc * 8 + 2 * u + 1) * kTileRows], bf16_hi(dw[u]), s);
+          sd = fmaf(rres[(kc * 8 + 2 * u) * kTileRows], bf16_lo(dw[u]), sd);
+          sd = fmaf(rres[(kc * 8 + 2 * u + 1) * kTileRows], bf16_hi(dw[u]), sd);
         }
       }
-      return s;
+      return sd;
     };
+    // candidate word: bf16 of |c~| rounded up (order-preserving for
+    // non-negative values) in the high half, atom index in the low half
+    auto cand_val = [](uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); };
 
-    for (int tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x) {
+    for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
       const int64_t grow = (int64_t)tile * kTileRows + row;
       const bool valid = grow < p.n_vec;
-      // residual <- x; A <- bf16(x)
-      float e2 = 0.0f, n2 = 0.0f;
+      if (lead && !*s_abort) {
+        // residual <- x; A <- bf16(x)
+        float e2 = 0.0f, n2 = 0.0f;
 #pragma unroll 1
-      for (int kc = 0; kc < D / 8; ++kc) {
-        float r8[8];
-        if (valid) {
-          if (p.x_dtype == SDK_F32) {
-            const float4* xp = reinterpret_cast<const float4*>(
-                reinterpret_cast<const float*>(p.x) + grow * D + kc * 8);
-            const float4 a = __ldg(xp), b = __ldg(xp + 1);
-            r8[0] = a.x; r8[1] = a.y; r8[2] = a.z; r8[3] = a.w;
-            r8[4] = b.x; r8[5] = b.y; r8[6] = b.z; r8[7] = b.w;
-          } else {
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(
-                reinterpret_cast<const uint16_t*>(p.x) + grow * D + kc * 8));
-            const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+        for (int kc = 0; kc < D / 8; ++kc) {
+          float r8[8];
+          if (valid) {
+            if (p.x_dtype == SDK_F32) {
+              const float4* xp = reinterpret_cast<const float4*>(
+                  reinterpret_cast<const float*>(p.x) + grow * D + kc * 8);
+              const float4 xa = __ldg(xp), xb = __ldg(xp + 1);
+              r8[0] = xa.x; r8[1] = xa.y; r8[2] = xa.z; r8[3] = xa.w;
+              r8[4] = xb.x; r8[5] = xb.y; r8[6] = xb.z; r8[7] = xb.w;
+            } else {
+              const uint4 xv = __ldg(reinterpret_cast<const uint4*>(
+                  reinterpret_cast<const uint16_t*>(p.x) + grow * D + kc * 8));
+              const uint32_t vw[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              r8[2 * u] = bf16_lo(vw[u]);
-              r8[2 * u + 1] = bf16_hi(vw[u]);
+              for (int u = 0; u < 4; ++u) {
+                r8[2 * u] = bf16_lo(vw[u]);
+                r8[2 * u + 1] = bf16_hi(vw[u]);
+              }
             }
+          } else {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) r8[u] = 0.0f;
           }
-        } else {
 #pragma unroll
-          for (int u = 0; u < 8; ++u) r8[u] = 0.0f;
+          for (int u = 0; u < 8; ++u) rres[(kc * 8 + u) * kTileRows] = r8[u];
+          write_a_chunk(kc, r8, e2, n2);
         }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) rres[(kc * 8 + u) * kTileRows] = r8[u];
-        write_a_chunk(kc, r8, e2, n2);
+        s_band[row] = band_of(e2, n2);
+        s_act[row] = (valid && n2 > 0.0f) ? 1u : 0u;
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_afull);
       }
-      float band = band_of(e2, n2);
-      bool active = valid && n2 > 0.0f;
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_afull);
+      epi_sync();
+      float band = s_band[row];
+      bool active = s_act[row] != 0u;
 
       for (int j = 0; j < steps_total; ++j) {
         float best = -INFINITY, thr = -INFINITY;
@@ -450,18 +479,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ovf = false;
 #pragma unroll 1
         for (int a = 0; a < p.n_atom_tiles; ++a) {
+          if (*s_abort) continue;
           // one lane waits so the warp stays converged for tcgen05.ld
           const bool got = lane == 0 ? mbar_wait(bar_tfull(tbuf), tphase, s_abort) : true;
           if (!__shfl_sync(0xffffffffu, got ? 1 : 0, 0)) {
-            ok = false;
-            break;
+            if (lane == 0) {
+              record_error(p.hdr, SDK_ERR_TIMEOUT, 0x42000000u | blockIdx.x);
+              *s_abort = 1u;
+            }
+            continue;
           }
           tc_fence_after();
-          uint32_t v[2][64];
-          const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + tbuf * (kSets * kAtomTile) +
-                                 rs * kAtomTile;
-          tmem_ld64(taddr, v[0]);
-          tmem_ld64(taddr + 64, v[1]);
+          uint32_t v[64];
+          tmem_ld64(tmem + ((uint32_t)(q * 32) << 16) + tbuf * (kSets * kAtomTile) +
+                        rs * kAtomTile + half * 64,
+                    v);
           tmem_ld_wait();
           tc_fence_before();
           __syncwarp();
@@ -469,138 +501,138 @@ __global__ void __launch_bounds__(kThreads, 1)
           tbuf ^= 1u;
           if (tbuf == 0u) tphase ^= 1u;
           if (!active) continue;
-          // max |c~| of each 16-column group (balanced trees, no long
-          // dependent chains), then of the tile
-          float m16[8];
+          // max |c~| of each 16-column group (balanced trees), then overall
+          float m16[4];
 #pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            const uint32_t* vg = &v[g >> 2][(g & 3) * 16];
+          for (int g = 0; g < 4; ++g) {
             float t8[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-              t8[i] = fmaxf(fabsf(__uint_as_float(vg[i])), fabsf(__uint_as_float(vg[i + 8])));
+              t8[i] = fmaxf(fabsf(__uint_as_float(v[g * 16 + i])),
+                            fabsf(__uint_as_float(v[g * 16 + i + 8])));
 #pragma unroll
             for (int i = 0; i < 4; ++i) t8[i] = fmaxf(t8[i], t8[i + 4]);
             m16[g] = fmaxf(fmaxf(t8[0], t8[2]), fmaxf(t8[1], t8[3]));
           }
-          const float mt = fmaxf(fmaxf(fmaxf(m16[0], m16[1]), fmaxf(m16[2], m16[3])),
-                                 fmaxf(fmaxf(m16[4], m16[5]), fmaxf(m16[6], m16[7])));
+          const float mt = fmaxf(fmaxf(m16[0], m16[1]), fmaxf(m16[2], m16[3]));
           if (mt >= thr) {
-            // rare: the tile holds a value within `band` of the running
-            // maximum.  Drop stale candidates, then keep every column at or
-            // above the new threshold.
+            // rare: a value within `band` of the running maximum.  Drop
+            // stale candidates, then keep every column at or above the new
+            // threshold (predicated pushes, one 16-column group at a time).
             best = fmaxf(best, mt);
             thr = best - band;
             int w = 0;
 #pragma unroll 1
             for (int t = 0; t < cnt; ++t)
-              if (cv[t] >= thr) {
-                ci[w] = ci[t];
-                cv[w] = cv[t];
-                ++w;
-              }
+              if (cand_val(cw[t]) >= thr) cw[w++] = cw[t];
             cnt = w;
-            const int lim = p.n - a * kAtomTile;
+            const int col0 = a * kAtomTile + half * 64;
+            const int lim = p.n - col0;
 #pragma unroll
-            for (int g = 0; g < 8; ++g) {
+            for (int g = 0; g < 4; ++g) {
               if (m16[g] < thr) continue;
-              const uint32_t* vg = &v[g >> 2][(g & 3) * 16];
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
-                const float av = fabsf(__uint_as_float(vg[i]));
-                if (av >= thr && g * 16 + i < lim) {
-                  if (cnt < kCand) {
-                    ci[cnt] = (uint32_t)(a * kAtomTile + g * 16 + i);
-                    cv[cnt] = av;
-                    ++cnt;
-                  } else {
-                    ovf = true;
-                  }
-                }
+                const uint32_t ab = __float_as_uint(fabsf(__uint_as_float(v[g * 16 + i])));
+                const bool take = __uint_as_float(ab) >= thr && g * 16 + i < lim;
+                const bool room = cnt < kCand;
+                if (take && room)
+                  cw[cnt] = (((ab + 0xFFFFu) >> 16) << 16) | (uint32_t)(col0 + g * 16 + i);
+                ovf |= take && !room;
+                cnt += (take && room) ? 1 : 0;
               }
             }
           }
         }
-        if (!ok) break;
 
-        // ---- pick: exact fp32 re-score of the candidates
-        uint32_t pick = 0u;
-        float coef = 0.0f;
-        if (active && !ovf) {
-          float babs = -1.0f;
-          int used = 0;
+        // ---- step end: merge the two halves of every row, pick, update
+        s_best[tix] = best;
+        s_cnt[tix] = (uint32_t)cnt | (ovf ? 0x80000000u : 0u);
+        epi_sync();
+        if (lead && !*s_abort) {
+          const float pbest = s_best[tix ^ 128];
+          const uint32_t pc = s_cnt[tix ^ 128];
+          const float gthr = fmaxf(best, pbest) - band;
+          const bool anyovf = ovf || (pc >> 31) != 0u;
+          const int pcnt = (int)(pc & 0x7FFFFFFFu);
+          uint32_t pick = 0u;
+          float coef = 0.0f;
+          if (active && !anyovf) {
+            float babs = -1.0f;
 #pragma unroll 1
-          for (int t = 0; t < cnt; ++t) {
-            if (cv[t] < thr) continue;
-            const uint32_t i = ci[t];
-            const float c = dot_atom(i);
-            ++used;
-            if (fabsf(c) > babs || (fabsf(c) == babs && i < pick)) {
-              babs = fabsf(c);
-              coef = c;
-              pick = i;
-            }
-          }
-          n_rescored += (uint32_t)used;
-        }
-        // rows whose candidate list overflowed: exact fp32 scan of every atom
-        // by the whole warp, one such row at a time
-        uint32_t ovm = __ballot_sync(0xffffffffu, active && ovf);
-        if (ovm != 0u && lane == 0) atomicAdd(&p.hdr->enc_fallback, (uint32_t)__popc(ovm));
-#pragma unroll 1
-        while (ovm != 0u) {
-          const int src = __ffs(ovm) - 1;
-          ovm &= ovm - 1u;
-          const float* rsrc = p.resid + (int64_t)blockIdx.x * D * kTileRows +
-                              (rs * kRows + q * 32 + src);
-          float rr[D];
-#pragma unroll
-          for (int k = 0; k < D; ++k) rr[k] = rsrc[k * kTileRows];
-          float bab = -1.0f, bc = 0.0f;
-          uint32_t bi = 0u;
-#pragma unroll 1
-          for (int i = lane; i < p.n; i += 32) {
-            const uint4* dp = reinterpret_cast<const uint4*>(p.dict + (int64_t)i * D);
-            float sdot = 0.0f;
-#pragma unroll
-            for (int kc = 0; kc < D / 8; ++kc) {
-              const uint4 dv = __ldg(dp + kc);
-              const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                sdot = fmaf(rr[kc * 8 + 2 * u], bf16_lo(dw[u]), sdot);
-                sdot = fmaf(rr[kc * 8 + 2 * u + 1], bf16_hi(dw[u]), sdot);
+            for (int t = 0; t < cnt + pcnt; ++t) {
+              const uint32_t wv = t < cnt ? cw[t] : pcw[t - cnt];
+              if (cand_val(wv) < gthr) continue;
+              const uint32_t i = wv & 0x7FFFu;
+              const float c = dot_atom(i);
+              ++n_rescored;
+              if (fabsf(c) > babs || (fabsf(c) == babs && i < pick)) {
+                babs = fabsf(c);
+                coef = c;
+                pick = i;
               }
             }
-            if (fabsf(sdot) > bab) {
-              bab = fabsf(sdot);
-              bc = sdot;
-              bi = (uint32_t)i;
-            }
           }
+          // rows whose candidate list overflowed: exact fp32 scan of every
+          // atom shared by the warp, one such row at a time
+          uint32_t ovm = __ballot_sync(0xffffffffu, active && anyovf);
+          if (ovm != 0u && lane == 0) atomicAdd(&p.hdr->enc_fallback, (uint32_t)__popc(ovm));
+#pragma unroll 1
+          while (ovm != 0u) {
+            const int src = __ffs(ovm) - 1;
+            ovm &= ovm - 1u;
+            const float* rsrc = p.resid + (int64_t)blockIdx.x * D * kTileRows +
+                                (rs * kRows + q * 32 + src);
+            for (int k = lane; k < D; k += 32) fr[k] = rsrc[k * kTileRows];
+            __syncwarp();
+            float bab = -1.0f, bc = 0.0f;
+            uint32_t bi = 0u;
+#pragma unroll 1
+            for (int i = lane; i < p.n; i += 32) {
+              const uint4* dp = reinterpret_cast<const uint4*>(p.dict + (int64_t)i * D);
+              float sd = 0.0f;
+#pragma unroll 4
+              for (int kc = 0; kc < D / 8; ++kc) {
+                const uint4 dv = __ldg(dp + kc);
+                const float4 ra = *reinterpret_cast<const float4*>(fr + kc * 8);
+                const float4 rb = *reinterpret_cast<const float4*>(fr + kc * 8 + 4);
+                sd = fmaf(ra.x, bf16_lo(dv.x), sd);
+                sd = fmaf(ra.y, bf16_hi(dv.x), sd);
+                sd = fmaf(ra.z, bf16_lo(dv.y), sd);
+                sd = fmaf(ra.w, bf16_hi(dv.y), sd);
+                sd = fmaf(rb.x, bf16_lo(dv.z), sd);
+                sd = fmaf(rb.y, bf16_hi(dv.z), sd);
+                sd = fmaf(rb.z, bf16_lo(dv.w), sd);
+                sd = fmaf(rb.w, bf16_hi(dv.w), sd);
+              }
+              if (fabsf(sd) > bab) {
+                bab = fabsf(sd);
+                bc = sd;
+                bi = (uint32_t)i;
+              }
+            }
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            const float oa = __shfl_xor_sync(0xffffffffu, bab, o);
-            const float oc = __shfl_xor_sync(0xffffffffu, bc, o);
-            const uint32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (oa > bab || (oa == bab && oi < bi)) {
-              bab = oa;
-              bc = oc;
-              bi = oi;
+            for (int o = 16; o > 0; o >>= 1) {
+              const float oa = __shfl_xor_sync(0xffffffffu, bab, o);
+              const float oc = __shfl_xor_sync(0xffffffffu, bc, o);
+              const uint32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
+              if (oa > bab || (oa == bab && oi < bi)) {
+                bab = oa;
+                bc = oc;
+                bi = oi;
+              }
             }
+            if (lane == src) {
+              coef = bc;
+              pick = bi;
+            }
+            __syncwarp();
           }
-          if (lane == src) {
-            coef = bc;
-            pick = bi;
-          }
-        }
-        if (valid) p.codes[grow * p.k_atoms + j] = make_word(coef, pick);
+          if (valid) p.codes[grow * p.k_atoms + j] = make_word(coef, pick);
 
-        // ---- residual update r -= coef * d_pick; next A operand
-        if (j + 1 < steps_total) {
+          // residual update r -= coef * d_pick; next A operand
           if (active) {
-            e2 = 0.0f;
-            n2 = 0.0f;
+            float e2 = 0.0f, n2 = 0.0f;
             const uint4* dp = reinterpret_cast<const uint4*>(p.dict + (int64_t)pick * D);
 #pragma unroll 1
             for (int kc = 0; kc < D / 8; ++kc) {
@@ -616,44 +648,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *r0 = r8[2 * u];
                 *r1 = r8[2 * u + 1];
               }
-              write_a_chunk(kc, r8, e2, n2);
+              if (j + 1 < steps_total) write_a_chunk(kc, r8, e2, n2);
             }
-            band = band_of(e2, n2);
-            active = n2 > 0.0f;
+            if (j + 1 < steps_total) {
+              s_band[row] = band_of(e2, n2);
+              s_act[row] = n2 > 0.0f ? 1u : 0u;
+            }
           }
-          fence_proxy_async();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar_afull);
-        } else if (active) {
-          // last step: update the fp32 residual only (for ||r||^2)
-          const uint4* dp = reinterpret_cast<const uint4*>(p.dict + (int64_t)pick * D);
-#pragma unroll 1
-          for (int kc = 0; kc < D / 8; ++kc) {
-            const uint4 dv = __ldg(dp + kc);
-            const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              float* r0 = rres + (kc * 8 + 2 * u) * kTileRows;
-              float* r1 = rres + (kc * 8 + 2 * u + 1) * kTileRows;
-              *r0 = fmaf(-coef, bf16_lo(dw[u]), *r0);
-              *r1 = fmaf(-coef, bf16_hi(dw[u]), *r1);
-            }
+          if (j + 1 < steps_total) {
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_afull);
           }
         }
+        epi_sync();
+        band = s_band[row];
+        active = s_act[row] != 0u;
       }
-      if (!ok) break;
-      if (valid && p.rsq != nullptr) {
-        float s = 0.0f;
+      if (lead && valid && p.rsq != nullptr && !*s_abort) {
+        float sq = 0.0f;
         for (int k = 0; k < D; ++k) {
           const float r = rres[k * kTileRows];
-          s = fmaf(r, r, s);
+          sq = fmaf(r, r, sq);
         }
-        p.rsq[grow] = s;
+        p.rsq[grow] = sq;
       }
-    }
-    if (!ok) {
-      record_error(p.hdr, SDK_ERR_TIMEOUT, 0x42000000u | blockIdx.x);
-      *s_abort = 1u;
     }
     n_rescored = __reduce_add_sync(0xffffffffu, n_rescored);
     if (lane == 0 && n_rescored) atomicAdd(&p.hdr->enc_cands, n_rescored);
