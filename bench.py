@@ -45,6 +45,10 @@ def parse():
     ap.add_argument("--workload", default="layer4k",
                     choices=["layer4k", "decode256k", "decode32k_b4",
                              "prefill256k_vec"])
+    ap.add_argument("--layers", type=int, default=None,
+                    help="decode workloads: layers to instantiate (default: "
+                         "the workload's 32); fewer layers make small ncu "
+                         "captures and are recorded in config.layers")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -342,6 +346,8 @@ def bench_decode(args, world, rank, pk, name):
     W = workloads.WORKLOADS[name]
     L, B, Hq, Hkv, d, n, N = (W["L"], W["B"], W["Hq"], W["Hkv"], W["d"],
                               W["n_atoms"], W["n_tokens"])
+    if args.layers is not None:
+        L = max(1, min(L, args.layers))
     layers = []
     for l in range(L):
         lay = workloads.decode_layer(name, l + 1000 * rank, device="cuda")

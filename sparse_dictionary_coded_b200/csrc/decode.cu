@@ -19,12 +19,13 @@
 //                    the rest of the selected set.
 //   rescore_kernel   s_t = scale * sum_{j<khigh} c_tj QD[idx_tj] for the
 //                    selected tokens (64-byte k_full records).
-//   value_kernel     e_t = exp(s_t - max), z = sum e_t, and the scatter
-//                    w[idx^V_tj] += e_t c^V_tj (shared-memory atomics into a
-//                    per-atom weight tile per CTA; a cluster of CTAs per
-//                    head sums its tiles through distributed shared memory).
-//   out_kernel       out += (w D_V) / z over atom tiles (vector reductions
-//                    into `out`, zeroed by qd_kernel).
+//   value_kernel     p_t = exp(s_t - max) / z and the scatter
+//                    w[idx^V_tj] += p_t c^V_tj (shared-memory fixed-point
+//                    atomics into a per-atom weight tile per CTA; a cluster
+//                    of CTAs per head sums its tiles through distributed
+//                    shared memory).
+//   out_kernel       out += w D_V over atom tiles (vector reductions into
+//                    `out`, zeroed by qd_kernel).
 #include <cooperative_groups.h>
 
 #include "sdk_internal.cuh"
@@ -102,18 +103,18 @@ __device__ void block_find_desc(const uint32_t* hist, uint32_t k,
 }
 
 // ---------------------------------------------------------------- qd_kernel
-// QD[r][a] = sum_k q[r][k] D_K[a][k] on a 128-atom x 32-row tile; thread
-// (ta, tr) owns atoms 4ta..4ta+3 and rows 8tr..8tr+7 (32 accumulators, fp32
-// FMA chains in k order).  The first kernel of a call also zeroes the
-// per-head selection state, both histograms and `out` (accumulated with
-// reductions by out_kernel).
-constexpr int kQdThreads = 128;
+// QD[r][a] = sum_k q[r][k] D_K[a][k] on a 128-atom x 32-row tile.  The atom
+// tile is kept as bf16 in shared memory ([k][atom]); thread (ta, tr) owns
+// atoms 4ta..4ta+3 and rows 4tr..4tr+3 (16 accumulators, fp32 FMA chains in
+// k order).  48 KB of shared memory per CTA lets four CTAs share an SM.
+// The first kernel of a call also zeroes the per-head selection state, both
+// histograms and `out` (accumulated with reductions by out_kernel).
+constexpr int kQdThreads = 256;
 
 template <int D>
 __global__ void __launch_bounds__(kQdThreads) qd_kernel(DecodeParams p) {
-  extern __shared__ float4 smem4[];
-  float* Ds = reinterpret_cast<float*>(smem4);   // [D][128]  atom tile, k-major
-  float* Qs = Ds + D * 128;                      // [D][32]   query rows, k-major
+  __shared__ __align__(16) uint16_t Ds[D][128];   // atom tile, k-major, bf16
+  __shared__ __align__(16) float Qs[D][32];       // query rows, k-major
   const int n = p.n, R = p.R, tid = threadIdx.x;
   const int a0 = blockIdx.x * 128, r0 = blockIdx.y * 32;
   {
@@ -126,59 +127,55 @@ __global__ void __launch_bounds__(kQdThreads) qd_kernel(DecodeParams p) {
     }
     for (int64_t e = g0; e < (int64_t)R * D; e += nthr) p.out[e] = 0.0f;
     for (int64_t e = g0; e < (int64_t)R; e += nthr) {
-      sdk_select_state s;
-      s.kth_key = 0u;
-      s.k = (uint32_t)p.kcnt[e / p.Hq];
-      s.n_above = s.n_cand = s.n_sel = s.n_comp = 0u;
-      s.eq_total = s.eq_taken = 0u;
-      s.max_score = 0u;
-      s.max_comp = 0u;
-      s.z = 0.0f;
+      sdk_select_state st;
+      st.kth_key = 0u;
+      st.k = (uint32_t)p.kcnt[e / p.Hq];
+      st.n_above = st.n_cand = st.n_sel = st.n_comp = 0u;
+      st.eq_total = st.eq_taken = 0u;
+      st.max_score = 0u;
+      st.max_comp = 0u;
+      st.z = 0.0f;
 #pragma unroll
-      for (int u = 0; u < 5; ++u) s.pad[u] = 0u;
-      p.st[e] = s;
+      for (int u = 0; u < 5; ++u) st.pad[u] = 0u;
+      p.st[e] = st;
     }
   }
   for (int e = tid; e < 128 * (D / 8); e += kQdThreads) {
     const int a = e & 127, c = e >> 7;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (a0 + a < n) v = __ldg(reinterpret_cast<const uint4*>(p.dk + (int64_t)(a0 + a) * D) + c);
-    float* col = Ds + (c * 8) * 128 + a;
-    col[0 * 128] = bf16_lo(v.x);
-    col[1 * 128] = bf16_hi(v.x);
-    col[2 * 128] = bf16_lo(v.y);
-    col[3 * 128] = bf16_hi(v.y);
-    col[4 * 128] = bf16_lo(v.z);
-    col[5 * 128] = bf16_hi(v.z);
-    col[6 * 128] = bf16_lo(v.w);
-    col[7 * 128] = bf16_hi(v.w);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      Ds[c * 8 + 2 * u][a] = (uint16_t)(w[u] & 0xFFFFu);
+      Ds[c * 8 + 2 * u + 1][a] = (uint16_t)(w[u] >> 16);
+    }
   }
   for (int e = tid; e < 32 * D; e += kQdThreads) {
     const int r = e & 31, k = e >> 5;
-    Qs[k * 32 + r] = (r0 + r < R) ? __ldg(p.q + (int64_t)(r0 + r) * D + k) : 0.0f;
+    Qs[k][r] = (r0 + r < R) ? __ldg(p.q + (int64_t)(r0 + r) * D + k) : 0.0f;
   }
   __syncthreads();
   const int ta = tid & 31, tr = tid >> 5;
-  float acc[8][4];
+  float acc[4][4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int u = 0; u < 4; ++u) acc[i][u] = 0.0f;
-#pragma unroll 4
+#pragma unroll 8
   for (int k = 0; k < D; ++k) {
-    const float4 dv = *reinterpret_cast<const float4*>(Ds + k * 128 + 4 * ta);
-    const float4 qa = *reinterpret_cast<const float4*>(Qs + k * 32 + 8 * tr);
-    const float4 qb = *reinterpret_cast<const float4*>(Qs + k * 32 + 8 * tr + 4);
-    const float dd[4] = {dv.x, dv.y, dv.z, dv.w};
-    const float qq[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+    const uint2 dv = *reinterpret_cast<const uint2*>(&Ds[k][4 * ta]);
+    const float4 qv = *reinterpret_cast<const float4*>(&Qs[k][4 * tr]);
+    const float dd[4] = {bf16_lo(dv.x), bf16_hi(dv.x), bf16_lo(dv.y), bf16_hi(dv.y)};
+    const float qq[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int u = 0; u < 4; ++u) acc[i][u] = fmaf(qq[i], dd[u], acc[i][u]);
   }
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = r0 + 8 * tr + i;
+  for (int i = 0; i < 4; ++i) {
+    const int r = r0 + 4 * tr + i;
     if (r >= R) continue;
     float* dst = p.qd + (int64_t)r * n + a0 + 4 * ta;
     if (a0 + 4 * ta + 3 < n && (n & 3) == 0) {
@@ -202,18 +199,12 @@ __device__ __forceinline__ void stage_row(float* dst, const float* src, int n) {
   }
 }
 
-// Warp-aggregated shared-memory histogram increment (lanes with equal bins
-// add once); every lane of the warp must call it; bin 0xFFFFFFFF skips.
-__device__ __forceinline__ void hist_add_warp(uint32_t* sh, uint32_t bin) {
-  const unsigned mm = __match_any_sync(0xffffffffu, bin);
-  const int lane = threadIdx.x & 31;
-  if (bin != 0xFFFFFFFFu && lane == __ffs(mm) - 1) atomicAdd(&sh[bin], (uint32_t)__popc(mm));
-}
-
 // -------------------------------------------------------------- klow_kernel
 constexpr int kScanThreads = 512;
+constexpr int kKlowThreads = 1024;
+constexpr int kKlowU = 4;   // tokens per thread per batch
 
-__global__ void __launch_bounds__(kScanThreads, 1) klow_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p) {
   extern __shared__ float4 smem4[];
   float* sq = reinterpret_cast<float*>(smem4);
   uint32_t* sh = reinterpret_cast<uint32_t*>(sq + ((p.n + 3) & ~3));
@@ -228,57 +219,65 @@ __global__ void __launch_bounds__(kScanThreads, 1) klow_kernel(DecodeParams p) {
     const float* qdr = p.qd + (int64_t)r * n;
     const bool stage = (t1 - t0) * p.klow >= (int64_t)(n / 2);
     if (stage) stage_row(sq, qdr, n);
-    for (int i = tid; i < 4096; i += kScanThreads) sh[i] = 0u;
+    for (int i = tid; i < 4096; i += kKlowThreads) sh[i] = 0u;
     __syncthreads();
     const float* src = stage ? sq : qdr;
     const int64_t head = (int64_t)b * p.Hkv + kvh;
     const uint32_t* plane = p.k_lo + head * kLoPlanes * p.cap;
     const uint32_t* rec = p.k_full + head * p.cap * kAtoms;
     uint32_t* keys = p.keys + (int64_t)r * p.L;
-    for (int64_t tb = t0; tb < t1; tb += 4 * kScanThreads) {
-      uint32_t wv[4][kLoPlanes];
+    constexpr int64_t kBatch = (int64_t)kKlowU * kKlowThreads;
+    // register double buffer: the next batch's plane words are in flight
+    // while the current batch is scored
+    uint32_t wv[kKlowU][kLoPlanes], wn[kKlowU][kLoPlanes];
+    auto load_batch = [&](int64_t tb, uint32_t (&w)[kKlowU][kLoPlanes]) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t t = tb + tid + u * kScanThreads;
+      for (int u = 0; u < kKlowU; ++u) {
+        const int64_t t = tb + tid + u * kKlowThreads;
 #pragma unroll
         for (int j = 0; j < kLoPlanes; ++j)
-          wv[u][j] = (t < t1 && j < nlo) ? __ldcs(plane + j * p.cap + t) : 0u;
+          w[u][j] = (t < t1 && j < nlo) ? __ldcs(plane + j * p.cap + t) : 0u;
       }
+    };
+    load_batch(t0, wv);
+    for (int64_t tb = t0; tb < t1; tb += kBatch) {
+      if (tb + kBatch < t1) load_batch(tb + kBatch, wn);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t t = tb + tid + u * kScanThreads;
-        uint32_t bin = 0xFFFFFFFFu;
-        if (t < t1) {
-          float s = 0.0f;
+      for (int u = 0; u < kKlowU; ++u) {
+        const int64_t t = tb + tid + u * kKlowThreads;
+        if (t >= t1) continue;
+        float s = 0.0f;
 #pragma unroll
-          for (int j = 0; j < kLoPlanes; ++j) {
-            if (j >= nlo) break;
-            const uint32_t idx = word_idx(wv[u][j]);
-            if (idx >= (uint32_t)n) {
-              record_error(p.hdr, SDK_ERR_DEVICE_CHECK, idx);
-              continue;
-            }
-            s = fmaf(word_coef(wv[u][j]), src[idx], s);
+        for (int j = 0; j < kLoPlanes; ++j) {
+          if (j >= nlo) break;
+          const uint32_t idx = word_idx(wv[u][j]);
+          if (idx >= (uint32_t)n) {
+            record_error(p.hdr, SDK_ERR_DEVICE_CHECK, idx);
+            continue;
           }
-          for (int j = kLoPlanes; j < p.klow; ++j) {
-            const uint32_t wj = __ldg(rec + t * kAtoms + j);
-            const uint32_t idx = word_idx(wj);
-            if (idx >= (uint32_t)n) {
-              record_error(p.hdr, SDK_ERR_DEVICE_CHECK, idx);
-              continue;
-            }
-            s = fmaf(word_coef(wj), src[idx], s);
-          }
-          const uint32_t key = score_key(s);
-          keys[t] = key;
-          bin = key >> 20;
+          s = fmaf(word_coef(wv[u][j]), src[idx], s);
         }
-        hist_add_warp(sh, bin);
+        for (int j = kLoPlanes; j < p.klow; ++j) {
+          const uint32_t wj = __ldg(rec + t * kAtoms + j);
+          const uint32_t idx = word_idx(wj);
+          if (idx >= (uint32_t)n) {
+            record_error(p.hdr, SDK_ERR_DEVICE_CHECK, idx);
+            continue;
+          }
+          s = fmaf(word_coef(wj), src[idx], s);
+        }
+        const uint32_t key = score_key(s);
+        keys[t] = key;
+        atomicAdd(&sh[key >> 20], 1u);
       }
+#pragma unroll
+      for (int u = 0; u < kKlowU; ++u)
+#pragma unroll
+        for (int j = 0; j < kLoPlanes; ++j) wv[u][j] = wn[u][j];
     }
     __syncthreads();
     uint32_t* gh = p.hist1 + (int64_t)r * 4096;
-    for (int i = tid; i < 4096; i += kScanThreads)
+    for (int i = tid; i < 4096; i += kKlowThreads)
       if (sh[i]) atomicAdd(&gh[i], sh[i]);
     __syncthreads();
   });
@@ -289,7 +288,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) klow_kernel(DecodeParams p) {
 // become candidates (with a histogram of key bits 19..8), the others go to
 // the complement.  Each warp compacts 128 tokens per iteration with ballots
 // and reserves its output slots with one atomic per category.
-__global__ void __launch_bounds__(kScanThreads) pass2_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kScanThreads, 2) pass2_kernel(DecodeParams p) {
   __shared__ uint32_t s_tmp[48];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned lt = (1u << lane) - 1u;
@@ -317,16 +316,27 @@ __global__ void __launch_bounds__(kScanThreads) pass2_kernel(DecodeParams p) {
     uint32_t* h2 = p.hist2 + (int64_t)r * 4096;
     uint32_t cmax = 0u;
     const int nwarps = kScanThreads / 32;
-    for (int64_t tb = t0 + (int64_t)warp * 128; tb < t1; tb += (int64_t)nwarps * 128) {
-      uint32_t key[4];
-      unsigned ms[4], mc[4], mo[4];
+    constexpr int U = 4;                       // tokens per lane per batch
+    constexpr int64_t WB = 32 * U;             // tokens per warp batch
+    uint32_t kc[U], kn[U];
+    auto load_keys = [&](int64_t tb, uint32_t (&kk)[U]) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t t = tb + lane + 32 * u;
+        kk[u] = t < t1 ? keys[t] : 0u;
+      }
+    };
+    int64_t tb = t0 + (int64_t)warp * WB;
+    if (tb < t1) load_keys(tb, kc);
+    for (; tb < t1; tb += (int64_t)nwarps * WB) {
+      const int64_t tnext = tb + (int64_t)nwarps * WB;
+      if (tnext < t1) load_keys(tnext, kn);
+      unsigned ms[U], mc[U], mo[U];
       uint32_t ns = 0, nc = 0, no = 0;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t t = tb + lane + 32 * u;
-        const bool valid = t < t1;
-        key[u] = valid ? keys[t] : 0u;
-        const uint32_t d1 = key[u] >> 20;
+      for (int u = 0; u < U; ++u) {
+        const bool valid = tb + lane + 32 * u < t1;
+        const uint32_t d1 = kc[u] >> 20;
         ms[u] = __ballot_sync(0xffffffffu, valid && d1 > b1);
         mc[u] = __ballot_sync(0xffffffffu, valid && d1 == b1);
         mo[u] = __ballot_sync(0xffffffffu, valid && d1 < b1 && p.full);
@@ -344,7 +354,7 @@ __global__ void __launch_bounds__(kScanThreads) pass2_kernel(DecodeParams p) {
       bc = __shfl_sync(0xffffffffu, bc, 0);
       bo = __shfl_sync(0xffffffffu, bo, 0);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < U; ++u) {
         const int64_t t = tb + lane + 32 * u;
         if ((ms[u] >> lane) & 1u) {
           const uint32_t pos = bs + __popc(ms[u] & lt);
@@ -353,18 +363,20 @@ __global__ void __launch_bounds__(kScanThreads) pass2_kernel(DecodeParams p) {
           const uint32_t pos = bc + __popc(mc[u] & lt);
           if (pos < (uint32_t)Nb) {
             ct[pos] = (int32_t)t;
-            ck[pos] = key[u];
+            ck[pos] = kc[u];
           }
-          atomicAdd(&h2[(key[u] >> 8) & 0xFFFu], 1u);
+          atomicAdd(&h2[(kc[u] >> 8) & 0xFFFu], 1u);
         } else if ((mo[u] >> lane) & 1u) {
           const uint32_t pos = bo + __popc(mo[u] & lt);
           if (pos < (uint32_t)Nb) list[Nb - 1 - (int64_t)pos] = (int32_t)t;
-          cmax = max(cmax, key[u]);
+          cmax = max(cmax, kc[u]);
         }
         bs += __popc(ms[u]);
         bc += __popc(mc[u]);
         bo += __popc(mo[u]);
       }
+#pragma unroll
+      for (int u = 0; u < U; ++u) kc[u] = kn[u];
     }
     if (p.full) {
       cmax = warp_umax(cmax);
@@ -375,6 +387,7 @@ __global__ void __launch_bounds__(kScanThreads) pass2_kernel(DecodeParams p) {
 }
 
 // ------------------------------------------------------------- final_kernel
+constexpr int kFinalStage = 12288;   // candidates staged in shared memory
 // One CTA per query head: the last two radix digits over the candidates, the
 // exact k-th key, the tie rule (lower token index first) and the rest of the
 // selected set.
@@ -398,6 +411,18 @@ __global__ void __launch_bounds__(kScanThreads) final_kernel(DecodeParams p) {
   const int32_t* ct = p.cand_t + (int64_t)r * p.L;
   int32_t* list = p.list + (int64_t)r * p.L;
   const uint32_t k1 = k - n_above;
+  // candidates in shared memory when they fit (one coalesced pass over the
+  // global copy; the passes below then read shared memory)
+  extern __shared__ uint32_t s_cand[];
+  if (n_cand <= (uint32_t)kFinalStage) {
+    for (uint32_t i = tid; i < n_cand; i += kScanThreads) {
+      s_cand[i] = ck[i];
+      s_cand[kFinalStage + i] = (uint32_t)ct[i];
+    }
+    __syncthreads();
+    ck = s_cand;
+    ct = reinterpret_cast<const int32_t*>(s_cand + kFinalStage);
+  }
 
   uint32_t b2, above2, cnt2, b3, above3, cnt3;
   bool bad;
@@ -509,12 +534,21 @@ __global__ void __launch_bounds__(kScanThreads) final_kernel(DecodeParams p) {
 }
 
 // ----------------------------------------------------------- rescore_kernel
-// s_t = scale * sum_{j<khigh} c_tj QD[idx_tj] for the selected tokens; two
-// tokens per thread per iteration keep 128 bytes of records in flight.
-__global__ void __launch_bounds__(kScanThreads, 1) rescore_kernel(DecodeParams p) {
+// s_t = scale * sum_{j<khigh} c_tj QD[idx_tj] for the selected tokens.  Four
+// lanes share a token: lane c of the group loads words 4c..4c+3 of the
+// 64-byte record (one coalesced 16-byte load; the group reads the record in
+// full), gathers their QD terms and the group sums its partials with two
+// shuffles.  A ring of kRing iterations keeps list entries and records in
+// flight ahead of the one being scored.
+constexpr int kRecThreads = 1024;
+constexpr int kRing = 4;
+
+__global__ void __launch_bounds__(kRecThreads, 1) rescore_kernel(DecodeParams p) {
   extern __shared__ float4 smem4[];
   float* sq = reinterpret_cast<float*>(smem4);
-  const int n = p.n, tid = threadIdx.x;
+  const int n = p.n, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int grp = lane >> 2, c = lane & 3;
+  constexpr int kWarps = kRecThreads / 32;
   const int64_t total = p.sel_off[p.B];
   const int64_t G0 = total * blockIdx.x / gridDim.x;
   const int64_t G1 = total * (blockIdx.x + 1) / gridDim.x;
@@ -531,69 +565,87 @@ __global__ void __launch_bounds__(kScanThreads, 1) rescore_kernel(DecodeParams p
     const int32_t* list = p.list + (int64_t)r * p.L;
     float* out = p.sel_score + (int64_t)r * p.L;
     const int Nb = p.lens[b];
-    float smax = -INFINITY;
-    for (int64_t ib = i0; ib < i1; ib += 2 * kScanThreads) {
-      int64_t t[2];
-      uint4 wv[2][4];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int64_t i = ib + tid + u * kScanThreads;
-        t[u] = i < i1 ? (int64_t)list[i] : -1;
-        if (i < i1 && (t[u] < 0 || t[u] >= Nb)) {
-          record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x30000000u | r);
-          t[u] = -1;
-        }
+    const int jmax = min(p.khigh - 4 * c, 4);   // words of this lane that count
+    auto entry = [&](int64_t it) { return i0 + (it * kWarps + warp) * 8 + grp; };
+    auto fetch = [&](int64_t it, int& t, uint4& w) {
+      const int64_t i = entry(it);
+      t = i < i1 ? list[i] : -1;
+      if (i < i1 && (t < 0 || t >= Nb)) {
+        if (c == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x30000000u | r);
+        t = -1;
       }
+      w = t >= 0 ? __ldcs(rec + (int64_t)t * 4 + c) : make_uint4(0u, 0u, 0u, 0u);
+    };
+    int tq[kRing];
+    uint4 wq[kRing];
 #pragma unroll
-      for (int u = 0; u < 2; ++u)
+    for (int s2 = 0; s2 < kRing; ++s2) fetch(s2, tq[s2], wq[s2]);
+    float smax = -INFINITY;
+    for (int64_t it0 = 0; entry(it0) - grp < i1; it0 += kRing) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          wv[u][c] = t[u] >= 0 ? __ldcs(rec + t[u] * 4 + c) : make_uint4(0u, 0u, 0u, 0u);
+      for (int s2 = 0; s2 < kRing; ++s2) {
+        const int64_t it = it0 + s2;
+        const int64_t i = entry(it);
+        const int t = tq[s2];
+        const uint4 w = wq[s2];
+        fetch(it + kRing, tq[s2], wq[s2]);
+        const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+        float part = 0.0f;
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int64_t i = ib + tid + u * kScanThreads;
-        if (i >= i1) continue;
-        if (t[u] < 0) {
-          out[i] = -INFINITY;
-          continue;
-        }
-        const uint32_t* wd = reinterpret_cast<const uint32_t*>(wv[u]);
-        float s = 0.0f;
-#pragma unroll
-        for (int j = 0; j < kAtoms; ++j) {
-          if (j >= p.khigh) break;
-          const uint32_t idx = word_idx(wd[j]);
-          if (idx >= (uint32_t)n) {
+        for (int u = 0; u < 4; ++u) {
+          if (u >= jmax) break;
+          const uint32_t idx = word_idx(wd[u]);
+          if (t >= 0 && idx >= (uint32_t)n) {
             record_error(p.hdr, SDK_ERR_DEVICE_CHECK, idx);
             continue;
           }
-          s = fmaf(word_coef(wd[j]), src[idx], s);
+          if (t >= 0) part = fmaf(word_coef(wd[u]), src[idx], part);
         }
-        s *= p.scale;
-        out[i] = s;
-        smax = fmaxf(smax, s);
+        part += __shfl_xor_sync(0xffffffffu, part, 1);
+        part += __shfl_xor_sync(0xffffffffu, part, 2);
+        if (c == 0 && i < i1) {
+          const float sc = t >= 0 ? part * p.scale : -INFINITY;
+          out[i] = sc;
+          smax = fmaxf(smax, sc);
+        }
       }
     }
     smax = warp_max(smax);
-    if ((tid & 31) == 0 && smax > -INFINITY) atomicMax(&p.st[r].max_score, score_key(smax));
+    if (lane == 0 && smax > -INFINITY) atomicMax(&p.st[r].max_score, score_key(smax));
     __syncthreads();
   });
 }
 
 // ------------------------------------------------------------- value_kernel
-// One cluster of C CTAs per query head.  Each CTA scatters
-// e_t * c^V_tj into a shared-memory per-atom weight tile for its share of
-// the head's softmax domain (e_t = exp(logit_t - max)); the cluster then
-// sums the C tiles through distributed shared memory and writes w[r] and
-// the softmax denominator z[r] once, with plain stores.
-__global__ void __launch_bounds__(kScanThreads, 1) value_kernel(DecodeParams p, int C) {
+// One cluster of C CTAs per query head; CTA `rank` owns a contiguous share
+// of the head's softmax domain (the selected set, or every token with the
+// full-softmax flag).
+//   pass A  e_t = exp(logit_t - max); the cluster sums e_t into z
+//           (distributed shared memory).
+//   pass B  p_t = e_t / z; w[idx^V_tj] += p_t c^V_tj into a shared-memory
+//           tile of n bins, four lanes per token as in rescore_kernel.  The
+//           bins hold 2^-20 fixed point in int32 (native shared-memory
+//           integer atomics, exact and order-independent).  Since
+//           sum_t p_t = 1, a bin can leave the int32 range only if the
+//           CTA's sum of |p_t c_tj| reaches 2^10; a CTA that sees that
+//           re-runs pass B with fp32 atomics.
+//   reduce  each CTA sums its slice of the atoms over the cluster's tiles
+//           and writes w[r] (already normalised) with plain stores.
+constexpr float kFixScale = 1048576.0f;       // 2^20
+constexpr float kFixInv = 1.0f / 1048576.0f;
+
+__global__ void __launch_bounds__(kRecThreads, 1) value_kernel(DecodeParams p, int C) {
   extern __shared__ float4 smem4[];
-  float* sw = reinterpret_cast<float*>(smem4);
-  __shared__ float s_red[kScanThreads / 32];
+  int* siw = reinterpret_cast<int*>(smem4);
+  float* sfw = reinterpret_cast<float*>(smem4);
+  __shared__ float s_red[kRecThreads / 32];
   __shared__ float s_z;
+  __shared__ int s_float;
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
-  const int n = p.n, tid = threadIdx.x;
+  const int n = p.n, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int grp = lane >> 2, c = lane & 3;
+  constexpr int kWarps = kRecThreads / 32;
   const int r = blockIdx.x / C;
   const int rank = (int)cluster.block_rank();
   const int b = r / p.Hq, h = r % p.Hq, kvh = h / p.g;
@@ -604,143 +656,172 @@ __global__ void __launch_bounds__(kScanThreads, 1) value_kernel(DecodeParams p, 
   const sdk_select_state* st = p.st + r;
   float m = key_score(st->max_score);
   if (p.full && st->n_comp > 0u) m = fmaxf(m, p.scale * key_score(st->max_comp));
-
-  for (int i = tid; i < n; i += kScanThreads) sw[i] = 0.0f;
-  __syncthreads();
   const uint4* rec = reinterpret_cast<const uint4*>(p.v_full +
                                                     ((int64_t)b * p.Hkv + kvh) * p.cap * kAtoms);
   const int32_t* list = p.list + (int64_t)r * p.L;
   const float* ss = p.sel_score + (int64_t)r * p.L;
   const uint32_t* keys = p.keys + (int64_t)r * p.L;
+  auto logit_of = [&](int64_t i, int64_t t) {
+    return (i < k) ? ss[i] : p.scale * key_score(keys[t]);
+  };
+
+  for (int i = tid; i < n; i += kRecThreads) siw[i] = 0;
+  // ---- pass A: z
   float z = 0.0f;
-  for (int64_t ib = i0; ib < i1; ib += 2 * kScanThreads) {
-    int64_t t[2];
-    float e[2];
-    uint4 wv[2][4];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int64_t i = ib + tid + u * kScanThreads;
-      t[u] = i < i1 ? (int64_t)list[i] : -1;
-      if (i < i1 && (t[u] < 0 || t[u] >= Nb)) {
-        record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x31000000u | r);
-        t[u] = -1;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        wv[u][c] = t[u] >= 0 ? __ldcs(rec + t[u] * 4 + c) : make_uint4(0u, 0u, 0u, 0u);
-      const int64_t i = ib + tid + u * kScanThreads;
-      e[u] = 0.0f;
-      if (t[u] >= 0) {
-        const float logit = (i < k) ? ss[i] : p.scale * key_score(keys[t[u]]);
-        e[u] = expf(logit - m);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      if (t[u] < 0) continue;
-      z += e[u];
-      const uint32_t* wd = reinterpret_cast<const uint32_t*>(wv[u]);
-#pragma unroll
-      for (int j = 0; j < kAtoms; ++j) {
-        const uint32_t idx = word_idx(wd[j]);
-        if (idx >= (uint32_t)n) {
-          record_error(p.hdr, SDK_ERR_DEVICE_CHECK, idx);
-          continue;
-        }
-        atomicAdd(&sw[idx], e[u] * word_coef(wd[j]));
-      }
-    }
+  for (int64_t i = i0 + tid; i < i1; i += kRecThreads) {
+    const int64_t t = i < k ? 0 : (int64_t)list[i];
+    if (t < 0 || t >= Nb) continue;
+    z += expf(logit_of(i, t) - m);
   }
   z = warp_sum(z);
-  if ((tid & 31) == 0) s_red[tid >> 5] = z;
+  if (lane == 0) s_red[warp] = z;
   __syncthreads();
   if (tid == 0) {
     float zz = 0.0f;
-    for (int i = 0; i < kScanThreads / 32; ++i) zz += s_red[i];
+    for (int i = 0; i < kWarps; ++i) zz += s_red[i];
     s_z = zz;
+    s_float = 0;
+  }
+  cluster.sync();
+  float ztot = 0.0f;
+  for (int cc = 0; cc < C; ++cc) ztot += *cluster.map_shared_rank(&s_z, cc);
+  const float invz = 1.0f / ztot;
+
+  // ---- pass B: scatter p_t c_tj (fixed point; fp32 atomics on re-run)
+  auto entry = [&](int64_t it) { return i0 + (it * kWarps + warp) * 8 + grp; };
+  auto fetch = [&](int64_t it, int& t, uint4& w) {
+    const int64_t i = entry(it);
+    t = i < i1 ? list[i] : -1;
+    if (i < i1 && (t < 0 || t >= Nb)) {
+      if (c == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x31000000u | r);
+      t = -1;
+    }
+    w = t >= 0 ? __ldcs(rec + (int64_t)t * 4 + c) : make_uint4(0u, 0u, 0u, 0u);
+  };
+  for (int pass = 0; pass < 2; ++pass) {
+    const bool use_float = pass == 1;
+    if (use_float) {
+      if (!s_float) break;
+      __syncthreads();
+      for (int i = tid; i < n; i += kRecThreads) sfw[i] = 0.0f;
+    }
+    __syncthreads();
+    float absum = 0.0f;
+    int tq[kRing];
+    uint4 wq[kRing];
+#pragma unroll
+    for (int s2 = 0; s2 < kRing; ++s2) fetch(s2, tq[s2], wq[s2]);
+    for (int64_t it0 = 0; entry(it0) - grp < i1; it0 += kRing) {
+#pragma unroll
+      for (int s2 = 0; s2 < kRing; ++s2) {
+        const int64_t it = it0 + s2;
+        const int64_t i = entry(it);
+        const int t = tq[s2];
+        const uint4 w = wq[s2];
+        fetch(it + kRing, tq[s2], wq[s2]);
+        if (t < 0) continue;
+        const float pt = expf(logit_of(i, t) - m) * invz;
+        const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t idx = word_idx(wd[u]);
+          if (idx >= (uint32_t)n) {
+            record_error(p.hdr, SDK_ERR_DEVICE_CHECK, idx);
+            continue;
+          }
+          const float v = pt * word_coef(wd[u]);
+          if (use_float) {
+            atomicAdd(&sfw[idx], v);
+          } else {
+            absum += fabsf(v);
+            atomicAdd(&siw[idx], __float2int_rn(v * kFixScale));
+          }
+        }
+      }
+    }
+    if (!use_float) {
+      // exact int32 range guard (see above); also catches NaN
+      if (!(absum < 1024.0f)) s_float = 1;
+      __syncthreads();
+      if (s_float) continue;
+      break;
+    }
   }
   cluster.sync();
   // reduce this CTA's slice of the atoms over the C tiles of the cluster
   const int a0 = (int)((int64_t)n * rank / C), a1 = (int)((int64_t)n * (rank + 1) / C);
   float* gw = p.w + (int64_t)r * n;
-  for (int a = a0 + tid; a < a1; a += kScanThreads) {
+  for (int a = a0 + tid; a < a1; a += kRecThreads) {
     float sum = 0.0f;
-    for (int c = 0; c < C; ++c) sum += cluster.map_shared_rank(sw, c)[a];
+    for (int cc = 0; cc < C; ++cc) {
+      const bool f = *cluster.map_shared_rank(&s_float, cc) != 0;
+      const int* tile = cluster.map_shared_rank(siw, cc);
+      sum += f ? __int_as_float(tile[a]) : (float)tile[a] * kFixInv;
+    }
     gw[a] = sum;
   }
-  if (rank == 0 && tid == 0) {
-    float zz = 0.0f;
-    for (int c = 0; c < C; ++c) zz += *cluster.map_shared_rank(&s_z, c);
-    p.st[r].z = zz;
-  }
+  if (rank == 0 && tid == 0) p.st[r].z = ztot;
   cluster.sync();
 }
 
 // --------------------------------------------------------------- out_kernel
-// out[r][k] += (1/z[r]) sum_{a in tile} w[r][a] D_V[a][k] over a 128-atom
-// tile and a 32-row block; thread (tk, tr) owns columns tk*C.. and rows
-// 8tr..8tr+7; results are added with vector reductions.
+// out[r][k] += sum_{a in tile} w[r][a] D_V[a][k] over a 128-atom tile and a
+// 32-row block.  The atom tile stays bf16 in shared memory ([atom][k]);
+// thread (tk, tr) owns columns tk*C.. and rows 4tr..4tr+3; results are
+// added with vector reductions into `out` (zeroed by qd_kernel).
 template <int D>
 __global__ void __launch_bounds__(kQdThreads) out_kernel(DecodeParams p) {
-  extern __shared__ float4 smem4[];
-  float* Ds = reinterpret_cast<float*>(smem4);  // [128][D]
-  float* Ws = Ds + 128 * D;                     // [128][32]
+  __shared__ __align__(16) uint16_t Ds[128][D];   // atom tile, bf16
+  __shared__ __align__(16) float Ws[128][32];     // w tile, [atom][row]
   const int n = p.n, R = p.R, tid = threadIdx.x;
   const int a0 = blockIdx.x * 128, r0 = blockIdx.y * 32;
   for (int e = tid; e < 128 * (D / 8); e += kQdThreads) {
     const int a = e / (D / 8), c = e % (D / 8);
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (a0 + a < n) v = __ldg(reinterpret_cast<const uint4*>(p.dv + (int64_t)(a0 + a) * D) + c);
-    float4* d = reinterpret_cast<float4*>(Ds + a * D + c * 8);
-    d[0] = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
-    d[1] = make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
+    *reinterpret_cast<uint4*>(&Ds[a][c * 8]) = v;
   }
   for (int e = tid; e < 128 * 32; e += kQdThreads) {
     const int r = e & 31, a = e >> 5;
-    Ws[a * 32 + r] = (r0 + r < R && a0 + a < n) ? p.w[(int64_t)(r0 + r) * n + a0 + a] : 0.0f;
+    Ws[a][r] = (r0 + r < R && a0 + a < n) ? p.w[(int64_t)(r0 + r) * n + a0 + a] : 0.0f;
   }
   __syncthreads();
   constexpr int C = D / 32;
   const int tk = tid & 31, tr = tid >> 5;
-  float acc[8][C];
+  float acc[4][C];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int c = 0; c < C; ++c) acc[i][c] = 0.0f;
-#pragma unroll 4
+    for (int cc = 0; cc < C; ++cc) acc[i][cc] = 0.0f;
+#pragma unroll 8
   for (int a = 0; a < 128; ++a) {
     float dv[C];
     if constexpr (C == 4) {
-      const float4 v = *reinterpret_cast<const float4*>(Ds + a * D + tk * 4);
-      dv[0] = v.x; dv[1] = v.y; dv[2] = v.z; dv[3] = v.w;
+      const uint2 v = *reinterpret_cast<const uint2*>(&Ds[a][tk * 4]);
+      dv[0] = bf16_lo(v.x); dv[1] = bf16_hi(v.x); dv[2] = bf16_lo(v.y); dv[3] = bf16_hi(v.y);
     } else {
-      const float2 v = *reinterpret_cast<const float2*>(Ds + a * D + tk * 2);
-      dv[0] = v.x; dv[1] = v.y;
+      const uint32_t v = *reinterpret_cast<const uint32_t*>(&Ds[a][tk * 2]);
+      dv[0] = bf16_lo(v); dv[1] = bf16_hi(v);
     }
-    const float4 wa = *reinterpret_cast<const float4*>(Ws + a * 32 + 8 * tr);
-    const float4 wb = *reinterpret_cast<const float4*>(Ws + a * 32 + 8 * tr + 4);
-    const float wr[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+    const float4 wv = *reinterpret_cast<const float4*>(&Ws[a][4 * tr]);
+    const float wr[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int c = 0; c < C; ++c) acc[i][c] = fmaf(wr[i], dv[c], acc[i][c]);
+      for (int cc = 0; cc < C; ++cc) acc[i][cc] = fmaf(wr[i], dv[cc], acc[i][cc]);
   }
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = r0 + 8 * tr + i;
+  for (int i = 0; i < 4; ++i) {
+    const int r = r0 + 4 * tr + i;
     if (r >= R) continue;
-    const float iz = 1.0f / p.st[r].z;
     float* dst = p.out + (int64_t)r * D + tk * C;
     if constexpr (C == 4) {
-      asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(acc[i][0] * iz),
-                   "f"(acc[i][1] * iz), "f"(acc[i][2] * iz), "f"(acc[i][3] * iz)
+      asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(acc[i][0]),
+                   "f"(acc[i][1]), "f"(acc[i][2]), "f"(acc[i][3])
                    : "memory");
     } else {
-      asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(dst), "f"(acc[i][0] * iz),
-                   "f"(acc[i][1] * iz)
+      asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(dst), "f"(acc[i][0]),
+                   "f"(acc[i][1])
                    : "memory");
     }
   }
@@ -787,36 +868,32 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
   const size_t qd_smem = (size_t)((p.n + 3) & ~3) * 4;
   static bool attr = false;
   if (!attr) {
-    cudaFuncSetAttribute(qd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 80 * 1024);
-    cudaFuncSetAttribute(qd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 80 * 1024);
-    cudaFuncSetAttribute(out_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 80 * 1024);
-    cudaFuncSetAttribute(out_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 80 * 1024);
     cudaFuncSetAttribute(klow_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     cudaFuncSetAttribute(rescore_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    cudaFuncSetAttribute(final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     cudaFuncSetAttribute(value_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     cudaFuncSetAttribute(value_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
     attr = true;
   }
   {
     dim3 grid((p.n + 127) / 128, (p.R + 31) / 32);
-    const size_t smem = (size_t)p.d * 128 * 4 + (size_t)p.d * 32 * 4;
-    if (p.d == 128) qd_kernel<128><<<grid, kQdThreads, smem, stream>>>(p);
-    else qd_kernel<64><<<grid, kQdThreads, smem, stream>>>(p);
+    if (p.d == 128) qd_kernel<128><<<grid, kQdThreads, 0, stream>>>(p);
+    else qd_kernel<64><<<grid, kQdThreads, 0, stream>>>(p);
   }
   {
     const int g = grid_for(p.tok_off[p.B], 2048, sms);
-    klow_kernel<<<g, kScanThreads, qd_smem + 4096 * 4, stream>>>(p);
+    klow_kernel<<<g, kKlowThreads, qd_smem + 4096 * 4, stream>>>(p);
   }
   {
     const int g = grid_for(p.tok_off[p.B], 8192, 2 * sms);
     pass2_kernel<<<g, kScanThreads, 0, stream>>>(p);
   }
-  final_kernel<<<p.R, kScanThreads, 0, stream>>>(p);
+  final_kernel<<<p.R, kScanThreads, (size_t)2 * kFinalStage * 4, stream>>>(p);
   {
-    int64_t per = p.sel_off[p.B] / (2 * sms);
-    if (per < 512) per = 512;
-    const int g = grid_for(p.sel_off[p.B], per, 2 * sms);
-    rescore_kernel<<<g, kScanThreads, qd_smem, stream>>>(p);
+    int64_t per = p.sel_off[p.B] / sms;
+    if (per < 1024) per = 1024;
+    const int g = grid_for(p.sel_off[p.B], per, sms);
+    rescore_kernel<<<g, kRecThreads, qd_smem, stream>>>(p);
   }
   {
     int64_t dmax = 0;
@@ -825,7 +902,7 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
     while (C < 8 && (int64_t)p.R * C * 2 <= sms && dmax / (2 * C) >= 1024) C *= 2;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(p.R * C));
-    cfg.blockDim = dim3(kScanThreads);
+    cfg.blockDim = dim3(kRecThreads);
     cfg.dynamicSmemBytes = qd_smem;
     cfg.stream = stream;
     cudaLaunchAttribute at[1];
@@ -839,9 +916,8 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
   }
   {
     dim3 grid((p.n + 127) / 128, (p.R + 31) / 32);
-    const size_t smem = (size_t)128 * p.d * 4 + 128 * 32 * 4;
-    if (p.d == 128) out_kernel<128><<<grid, kQdThreads, smem, stream>>>(p);
-    else out_kernel<64><<<grid, kQdThreads, smem, stream>>>(p);
+    if (p.d == 128) out_kernel<128><<<grid, kQdThreads, 0, stream>>>(p);
+    else out_kernel<64><<<grid, kQdThreads, 0, stream>>>(p);
   }
   return cudaGetLastError() == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
 }

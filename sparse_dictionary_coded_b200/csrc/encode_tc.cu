@@ -69,7 +69,9 @@ struct Cfg {
   static constexpr int kOffBand = kOffCnt + kEpiThreads * 4;
   static constexpr int kOffAct = kOffBand + kTileRows * 4;
   static constexpr int kOffFr = kOffAct + kTileRows * 4;          // fallback residuals
-  static constexpr int kOffBar = kOffFr + kLeadWarps * D * 4;
+  static constexpr int kOffStg = kOffFr + kLeadWarps * D * 4;      // push staging
+  static constexpr int kOffRes = kOffStg + kEpiWarps * 16 * 4;     // per-thread picks
+  static constexpr int kOffBar = kOffRes + kEpiThreads * 12;
   static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   // + alignment slack; at least 116 KB so that one CTA (which holds all 512
@@ -194,6 +196,19 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&v)[64]) {
         "=r"(v[62]), "=r"(v[63])
       : "r"(taddr));
 }
+// 32 lanes x 32 bits, 32 consecutive columns per thread.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -214,7 +229,7 @@ __device__ __forceinline__ float bf16_round(float v) {
 
 // ---- the kernel --------------------------------------------------------------
 template <int D>
-__global__ void __maxnreg__(112)
+__global__ void __launch_bounds__(kThreads, 1)
     encode_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -226,6 +241,10 @@ __global__ void __maxnreg__(112)
   float* s_band = reinterpret_cast<float*>(smem + C::kOffBand);
   uint32_t* s_act = reinterpret_cast<uint32_t*>(smem + C::kOffAct);
   float* s_fr = reinterpret_cast<float*>(smem + C::kOffFr);
+  float* s_stg = reinterpret_cast<float*>(smem + C::kOffStg);
+  float* s_rabs = reinterpret_cast<float*>(smem + C::kOffRes);
+  uint32_t* s_ridx = reinterpret_cast<uint32_t*>(smem + C::kOffRes + kEpiThreads * 4);
+  float* s_rcoef = reinterpret_cast<float*>(smem + C::kOffRes + kEpiThreads * 8);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile uint32_t* s_abort = misc + 0;
@@ -376,7 +395,8 @@ __global__ void __maxnreg__(112)
     const int row = rs * kRows + rin;         // row within the tile
     const int tix = e * 32 + lane;            // partner (other half): tix ^ 128
     uint32_t* cw = s_cw + tix * kCand;
-    const uint32_t* pcw = s_cw + (tix ^ 128) * kCand;
+    float* stg = s_stg + e * 16;
+    const unsigned lt = (1u << lane) - 1u;
     float* rres = p.resid + (int64_t)blockIdx.x * D * kTileRows + row;  // stride kTileRows
     float* fr = s_fr + (rs * 4 + (e & 3)) * D;                           // lead warps only
     const float dmax = *p.dmax;
@@ -490,88 +510,176 @@ __global__ void __maxnreg__(112)
             continue;
           }
           tc_fence_after();
-          uint32_t v[64];
-          tmem_ld64(tmem + ((uint32_t)(q * 32) << 16) + tbuf * (kSets * kAtomTile) +
-                        rs * kAtomTile + half * 64,
-                    v);
-          tmem_ld_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar_tempty(tbuf));
-          tbuf ^= 1u;
-          if (tbuf == 0u) tphase ^= 1u;
-          if (!active) continue;
-          // max |c~| of each 16-column group (balanced trees), then overall
-          float m16[4];
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            float t8[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              t8[i] = fmaxf(fabsf(__uint_as_float(v[g * 16 + i])),
-                            fabsf(__uint_as_float(v[g * 16 + i + 8])));
-#pragma unroll
-            for (int i = 0; i < 4; ++i) t8[i] = fmaxf(t8[i], t8[i + 4]);
-            m16[g] = fmaxf(fmaxf(t8[0], t8[2]), fmaxf(t8[1], t8[3]));
-          }
-          const float mt = fmaxf(fmaxf(m16[0], m16[1]), fmaxf(m16[2], m16[3]));
-          if (mt >= thr) {
-            // rare: a value within `band` of the running maximum.  Drop
-            // stale candidates, then keep every column at or above the new
-            // threshold (predicated pushes, one 16-column group at a time).
-            best = fmaxf(best, mt);
-            thr = best - band;
-            int w = 0;
+          const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + tbuf * (kSets * kAtomTile) +
+                                 rs * kAtomTile + half * 64;
+          // two 32-column halves: 32 accumulator registers live at a time
 #pragma unroll 1
-            for (int t = 0; t < cnt; ++t)
-              if (cand_val(cw[t]) >= thr) cw[w++] = cw[t];
-            cnt = w;
-            const int col0 = a * kAtomTile + half * 64;
-            const int lim = p.n - col0;
+          for (int c = 0; c < 2; ++c) {
+            uint32_t v[32];
+            __syncwarp();  // reconverge (the previous half may have diverged)
+            tmem_ld32(taddr + c * 32, v);
+            tmem_ld_wait();
+            if (c == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(bar_tempty(tbuf));
+            }
+            // max |c~| of each 16-column group (balanced trees), then overall
+            float m16[2];
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              if (m16[g] < thr) continue;
+            for (int g = 0; g < 2; ++g) {
+              float t8[8];
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const uint32_t ab = __float_as_uint(fabsf(__uint_as_float(v[g * 16 + i])));
-                const bool take = __uint_as_float(ab) >= thr && g * 16 + i < lim;
-                const bool room = cnt < kCand;
-                if (take && room)
-                  cw[cnt] = (((ab + 0xFFFFu) >> 16) << 16) | (uint32_t)(col0 + g * 16 + i);
-                ovf |= take && !room;
-                cnt += (take && room) ? 1 : 0;
+              for (int i = 0; i < 8; ++i)
+                t8[i] = fmaxf(fabsf(__uint_as_float(v[g * 16 + i])),
+                              fabsf(__uint_as_float(v[g * 16 + i + 8])));
+#pragma unroll
+              for (int i = 0; i < 4; ++i) t8[i] = fmaxf(t8[i], t8[i + 4]);
+              m16[g] = fmaxf(fmaxf(t8[0], t8[2]), fmaxf(t8[1], t8[3]));
+            }
+            const float mt = fmaxf(m16[0], m16[1]);
+            if (active && mt >= thr) {
+              best = fmaxf(best, mt);
+              thr = best - band;
+            }
+            // Candidates: every column within `band` of the running maximum.
+            // A triggering lane stages its 16-column group in shared memory
+            // and 16 lanes of the warp test and append them to that lane's
+            // list together (cost per trigger independent of group width).
+            const int col0 = a * kAtomTile + half * 64 + c * 32;
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+              unsigned tm = __ballot_sync(0xffffffffu, active && m16[g] >= thr);
+              while (tm != 0u) {
+                const int L = __ffs(tm) - 1;
+                tm &= tm - 1u;
+                if (lane == L) {
+                  float4* s4 = reinterpret_cast<float4*>(stg);
+#pragma unroll
+                  for (int i = 0; i < 4; ++i)
+                    s4[i] = make_float4(fabsf(__uint_as_float(v[g * 16 + 4 * i])),
+                                        fabsf(__uint_as_float(v[g * 16 + 4 * i + 1])),
+                                        fabsf(__uint_as_float(v[g * 16 + 4 * i + 2])),
+                                        fabsf(__uint_as_float(v[g * 16 + 4 * i + 3])));
+                }
+                __syncwarp();
+                const float thrL = __shfl_sync(0xffffffffu, thr, L);
+                const float av = lane < 16 ? stg[lane] : 0.0f;
+                const int col = col0 + g * 16 + lane;
+                const bool take = lane < 16 && av >= thrL && col < p.n;
+                const unsigned pm = __ballot_sync(0xffffffffu, take);
+                const int np = __popc(pm);
+                int cntL = __shfl_sync(0xffffffffu, cnt, L);
+                if (cntL + np > kCand) {
+                  // make room: drop the owner's stale candidates
+                  if (lane == L) {
+                    int w = 0;
+                    for (int t = 0; t < cnt; ++t)
+                      if (cand_val(cw[t]) >= thr) cw[w++] = cw[t];
+                    cnt = w;
+                  }
+                  __syncwarp();
+                  cntL = __shfl_sync(0xffffffffu, cnt, L);
+                }
+                if (take) {
+                  const int pos = cntL + __popc(pm & lt);
+                  const uint32_t ab = __float_as_uint(av);
+                  if (pos < kCand)
+                    s_cw[(e * 32 + L) * kCand + pos] =
+                        (((ab + 0xFFFFu) >> 16) << 16) | (uint32_t)col;
+                }
+                if (lane == L) {
+                  const int nc = cntL + np;
+                  ovf |= nc > kCand;
+                  cnt = nc < kCand ? nc : kCand;
+                }
+                __syncwarp();
               }
             }
           }
+          tbuf ^= 1u;
+          if (tbuf == 0u) tphase ^= 1u;
         }
 
         // ---- step end: merge the two halves of every row, pick, update
         s_best[tix] = best;
         s_cnt[tix] = (uint32_t)cnt | (ovf ? 0x80000000u : 0u);
         epi_sync();
-        if (lead && !*s_abort) {
-          const float pbest = s_best[tix ^ 128];
-          const uint32_t pc = s_cnt[tix ^ 128];
+        const float pbest = s_best[tix ^ 128];
+        const uint32_t pcw_cnt = s_cnt[tix ^ 128];
+        const bool anyovf = ovf || (pcw_cnt >> 31) != 0u;
+        {
+          // each thread re-scores its own candidates that survive the row's
+          // threshold; the chunk-outer loop reads the fp32 residual once for
+          // all of them and keeps every dot in k order
           const float gthr = fmaxf(best, pbest) - band;
-          const bool anyovf = ovf || (pc >> 31) != 0u;
-          const int pcnt = (int)(pc & 0x7FFFFFFFu);
+          float babs = -1.0f, bcoef = 0.0f;
+          uint32_t bidx = 0xFFFFFFFFu;
+          if (active && !anyovf && !*s_abort) {
+            bool ok_e[kCand];
+            uint32_t ix[kCand];
+            float acc[kCand];
+#pragma unroll
+            for (int e2 = 0; e2 < kCand; ++e2) {
+              const uint32_t wv = cw[e2];
+              ok_e[e2] = e2 < cnt && cand_val(wv) >= gthr;
+              ix[e2] = wv & 0x7FFFu;
+              acc[e2] = 0.0f;
+              n_rescored += ok_e[e2] ? 1u : 0u;
+            }
+#pragma unroll 1
+            for (int kc = 0; kc < D / 8; ++kc) {
+              float r8[8];
+#pragma unroll
+              for (int u = 0; u < 8; ++u) r8[u] = rres[(kc * 8 + u) * kTileRows];
+#pragma unroll
+              for (int e2 = 0; e2 < kCand; ++e2) {
+                if (!ok_e[e2]) continue;
+                const uint4 dv = __ldg(reinterpret_cast<const uint4*>(p.dict + (int64_t)ix[e2] * D) + kc);
+                float sd = acc[e2];
+                sd = fmaf(r8[0], bf16_lo(dv.x), sd);
+                sd = fmaf(r8[1], bf16_hi(dv.x), sd);
+                sd = fmaf(r8[2], bf16_lo(dv.y), sd);
+                sd = fmaf(r8[3], bf16_hi(dv.y), sd);
+                sd = fmaf(r8[4], bf16_lo(dv.z), sd);
+                sd = fmaf(r8[5], bf16_hi(dv.z), sd);
+                sd = fmaf(r8[6], bf16_lo(dv.w), sd);
+                sd = fmaf(r8[7], bf16_hi(dv.w), sd);
+                acc[e2] = sd;
+              }
+            }
+#pragma unroll
+            for (int e2 = 0; e2 < kCand; ++e2) {
+              if (!ok_e[e2]) continue;
+              const float aa = fabsf(acc[e2]);
+              if (aa > babs || (aa == babs && ix[e2] < bidx)) {
+                babs = aa;
+                bcoef = acc[e2];
+                bidx = ix[e2];
+              }
+            }
+          }
+          s_rabs[tix] = babs;
+          s_ridx[tix] = bidx;
+          s_rcoef[tix] = bcoef;
+        }
+        epi_sync();
+        if (lead && !*s_abort) {
           uint32_t pick = 0u;
           float coef = 0.0f;
           if (active && !anyovf) {
-            float babs = -1.0f;
-#pragma unroll 1
-            for (int t = 0; t < cnt + pcnt; ++t) {
-              const uint32_t wv = t < cnt ? cw[t] : pcw[t - cnt];
-              if (cand_val(wv) < gthr) continue;
-              const uint32_t i = wv & 0x7FFFu;
-              const float c = dot_atom(i);
-              ++n_rescored;
-              if (fabsf(c) > babs || (fabsf(c) == babs && i < pick)) {
-                babs = fabsf(c);
-                coef = c;
-                pick = i;
-              }
+            // the better of the two halves' picks (ties: lower atom index)
+            float babs = s_rabs[tix];
+            uint32_t bidx = s_ridx[tix];
+            coef = s_rcoef[tix];
+            const float oabs = s_rabs[tix ^ 128];
+            const uint32_t oidx = s_ridx[tix ^ 128];
+            if (oabs > babs || (oabs == babs && oidx < bidx)) {
+              babs = oabs;
+              bidx = oidx;
+              coef = s_rcoef[tix ^ 128];
             }
+            pick = bidx;
           }
           // rows whose candidate list overflowed: exact fp32 scan of every
           // atom shared by the warp, one such row at a time
