@@ -6,36 +6,48 @@
 // pursuit, no least-squares refit).
 //
 // Design (one persistent CTA per SM, 18 warps, warp-specialised):
-//   warp 0      TMA producer: streams the bf16 dictionary through a 4-stage
-//               shared-memory ring in 128-atom tiles (128B-swizzled,
-//               K-major), the same dictionary 16 times per row tile.
+//   warp 0      TMA producer: streams the operand copy of the dictionary
+//               through a 4-stage shared-memory ring in 128-atom tiles
+//               (128B-swizzled, K-major), the same dictionary 16 times per
+//               row tile.
 //   warp 1      MMA issuer: allocates 512 TMEM columns; for every atom tile
-//               issues tcgen05.mma kind::f16 (bf16 x bf16 -> fp32, M=128,
-//               N=128, K=16) for two 128-row sets of residuals (A operand,
-//               bf16, in shared memory) into one of two TMEM accumulator
-//               buffers; tcgen05.commit frees the ring stage and hands the
-//               buffer to the epilogue.
+//               issues tcgen05.mma kind::f16 (M=128, N=128, K=16, fp32
+//               accumulate) for two 128-row sets of residuals (A operand in
+//               shared memory) into one of two TMEM accumulator buffers;
+//               tcgen05.commit frees the ring stage and hands the buffer to
+//               the epilogue.
 //   warps 2..17 epilogue: two threads per residual row (64 columns each of
 //               every 128-atom tile).  tcgen05.ld brings a thread's
 //               correlations to registers, the buffer is released at once,
 //               and the thread keeps the running maximum
 //               B of |c~| plus every atom with |c~| >= B - band.  band is
-//               twice a rigorous bound on |c~ - c| (bf16 rounding of r by
-//               Cauchy-Schwarz, plus accumulation slack), so the exact
-//               fp32 argmax is always among the kept candidates.  After the
-//               last atom tile of a step the candidates are re-scored in
-//               fp32 by the row's lead thread (k = 0..D-1 FMA order, the
-//               same arithmetic as the CUDA-core encoder), the pick is
-//               written, r is updated in
-//               fp32 (global scratch, L2-resident) and its bf16 copy
-//               becomes the next step's A operand.  A row whose candidate
-//               list overflows is re-picked by an exact fp32 scan of all
-//               atoms shared by its warp (counted in the workspace header).
+//               twice a rigorous bound on the error of c~ (operand rounding
+//               of r and of the dictionary by Cauchy-Schwarz, plus
+//               accumulation slack), so the exact fp32 argmax is always
+//               among the kept candidates.  After the last atom tile of a
+//               step the candidates are re-scored in fp32 (k = 0..D-1 FMA
+//               order over the bf16 atoms, the same arithmetic as the
+//               CUDA-core encoder), the row's lead thread writes the pick,
+//               r is updated in fp32 (global scratch, L2-resident) and its
+//               rounded copy becomes the next step's A operand.  A row whose
+//               candidate list overflows is re-picked by an exact fp32 scan
+//               of all atoms shared by its warp (counted in the workspace
+//               header).
+// Operands: fp16 by default.  The bf16 atoms are copied once per call as
+// fp16(t d) with a power-of-two t (exact for every entry within 29 binades
+// of the largest), and each A row holds fp16(s r) with a per-row power of
+// two s, so |c~ - s t c| is about 8x tighter than with bf16 operands at the
+// same MMA rate; fewer atoms fall inside the band.  Setting the environment
+// variable SDK_ENCODE_OPERANDS=bf16 selects bf16 operands (the atoms as
+// given, t = 1; the row scale s is kept).  Either way the picks are the
+// exact fp32 argmax.
 // Every wait on an mbarrier is bounded (1 s of %globaltimer); on expiry the
 // CTA records SDK_ERR_TIMEOUT, stops issuing work, lets in-flight copies and
 // MMAs finish (bounded), frees its TMEM and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "sdk_internal.cuh"
 
@@ -68,9 +80,12 @@ struct Cfg {
   static constexpr int kOffCnt = kOffBest + kEpiThreads * 4;
   static constexpr int kOffBand = kOffCnt + kEpiThreads * 4;
   static constexpr int kOffAct = kOffBand + kTileRows * 4;
-  static constexpr int kOffFr = kOffAct + kTileRows * 4;          // fallback residuals
-  static constexpr int kOffStg = kOffFr + kLeadWarps * D * 4;      // push staging
-  static constexpr int kOffRes = kOffStg + kEpiWarps * 16 * 4;     // per-thread picks
+  static constexpr int kOffScl = kOffAct + kTileRows * 4;          // per-row A scale
+  static constexpr int kOffFr = kOffScl + kTileRows * 4;          // fallback residuals
+  // push staging (tile loop) shares the fallback scratch (step end only)
+  static constexpr int kOffStg = kOffFr;
+  static_assert(kEpiWarps * 32 <= kLeadWarps * D, "staging must fit the fallback scratch");
+  static constexpr int kOffRes = kOffFr + kLeadWarps * D * 4;      // per-thread picks
   static constexpr int kOffBar = kOffRes + kEpiThreads * 12;
   static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -78,7 +93,20 @@ struct Cfg {
   // TMEM columns) is resident per SM
   static constexpr int kSmemUsed = kOffMisc + 64 + 1024;
   static constexpr int kSmem = kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024;
+  static_assert(kSmem <= 232448, "exceeds the 227 KB shared memory of one sm_100 CTA");
 };
+
+// power-of-two factor t with max|t v| in [2^14, 2^15) for amax = max|v|:
+// fp16 keeps its 11-bit significand over the largest entries and cannot
+// overflow.  The exponent is capped at 126 so t stays finite (amax below
+// 2^-112, subnormals included, gets t = 2^126 and max|t v| < 2^14); 1 for
+// zero or non-finite amax.
+__device__ __forceinline__ float pow2_scale(float amax) {
+  const uint32_t b = __float_as_uint(amax);
+  const int ex = (int)((b >> 23) & 0xFFu);
+  if (!(amax > 0.0f) || ex == 0xFF) return 1.0f;
+  return ldexpf(1.0f, min(14 - (ex - 127), 126));
+}
 
 struct TcParams {
   const void* x;
@@ -91,7 +119,9 @@ struct TcParams {
   float* rsq;
   WsHeader* hdr;
   float* resid;        // [grid][D][kTileRows] fp32
-  const float* dmax;   // max_i ||d_i||
+  // dictionary statistics: [0] max_i ||d_i||, [1] max_i ||t d_i - fp16(t d_i)||
+  // (f16 operands; 0 for bf16), [2] max_ij |d_ij| as bits; t = dict_scale([2])
+  const float* dmax;
   int n_tiles;
   int n_atom_tiles;
 };
@@ -108,14 +138,17 @@ __device__ __forceinline__ uint64_t globaltimer() {
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+// try_wait suspends the thread until the phase completes or ~hint_ns pass,
+// so a waiting warp issues few instructions
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity,
+                                         uint32_t hint_ns = 20000u) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.b32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0u;
 }
@@ -124,9 +157,7 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile uint32_t* abort_flag,
                                           unsigned long long limit = kWaitNs) {
-#pragma unroll 1
-  for (int i = 0; i < 128; ++i)
-    if (mbar_try(bar, parity)) return true;
+  if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
 #pragma unroll 1
   while (true) {
@@ -213,22 +244,35 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// max(|a|, |b|) in one instruction (the sign of the result is the xor of
+// the operands' signs; only its magnitude is used)
+__device__ __forceinline__ float absmax2(float a, float b) {
+  float r;
+  asm("max.xorsign.abs.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
 // 1024 bytes apart (the canonical layout TMA SWIZZLE_128B writes).
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
   return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) |
          ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
 }
-// Instruction descriptor: D f32, A bf16, B bf16, both K-major, N=128, M=128.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                            ((uint32_t)(kAtomTile >> 3) << 17) | ((uint32_t)(kRows >> 4) << 24);
+// Instruction descriptor: D f32, A and B both f16 (F16=true) or both bf16,
+// both K-major, N=128, M=128.
+template <bool F16>
+struct Idesc {
+  static constexpr uint32_t value = (1u << 4) | ((F16 ? 0u : 1u) << 7) | ((F16 ? 0u : 1u) << 10) |
+                                    ((uint32_t)(kAtomTile >> 3) << 17) |
+                                    ((uint32_t)(kRows >> 4) << 24);
+};
 
 __device__ __forceinline__ float bf16_round(float v) {
   return __bfloat162float(__float2bfloat16_rn(v));
 }
 
 // ---- the kernel --------------------------------------------------------------
-template <int D>
+template <int D, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
     encode_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcParams p) {
   using C = Cfg<D>;
@@ -240,6 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* s_cnt = reinterpret_cast<uint32_t*>(smem + C::kOffCnt);
   float* s_band = reinterpret_cast<float*>(smem + C::kOffBand);
   uint32_t* s_act = reinterpret_cast<uint32_t*>(smem + C::kOffAct);
+  float* s_scl = reinterpret_cast<float*>(smem + C::kOffScl);
   float* s_fr = reinterpret_cast<float*>(smem + C::kOffFr);
   float* s_stg = reinterpret_cast<float*>(smem + C::kOffStg);
   float* s_rabs = reinterpret_cast<float*>(smem + C::kOffRes);
@@ -354,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int ks = 0; ks < C::KSTEPS; ++ks) {
                 const uint32_t koff = (ks >> 2) * (kRows * 128) + (ks & 3) * 32;
                 const uint32_t boff = (ks >> 2) * (kAtomTile * 128) + (ks & 3) * 32;
-                tc_mma(d_tmem, smem_desc(abase + koff), smem_desc(bbase + boff), kIdesc,
+                tc_mma(d_tmem, smem_desc(abase + koff), smem_desc(bbase + boff), Idesc<F16>::value,
                        ks > 0 ? 1u : 0u);
               }
             }
@@ -395,39 +440,74 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = rs * kRows + rin;         // row within the tile
     const int tix = e * 32 + lane;            // partner (other half): tix ^ 128
     uint32_t* cw = s_cw + tix * kCand;
-    float* stg = s_stg + e * 16;
+    float* stg = s_stg + e * 32;
     const unsigned lt = (1u << lane) - 1u;
     float* rres = p.resid + (int64_t)blockIdx.x * D * kTileRows + row;  // stride kTileRows
     float* fr = s_fr + (rs * 4 + (e & 3)) * D;                           // lead warps only
-    const float dmax = *p.dmax;
+    // f16 operands: the MMA reads fp16(t d_i) for a power-of-two t, so a
+    // tensor-core value approximates s t <r, d_i> for the row scale s; econv
+    // is the largest conversion error ||t d_i - fp16(t d_i)|| and dmax bounds
+    // the operand atom norms ||fp16(t d_i)||
+    // (read where used, to keep them out of the scan loop's registers)
+    auto tdict_of = [&] {
+      return F16 ? pow2_scale(__int_as_float(__ldg(reinterpret_cast<const int*>(p.dmax) + 2)))
+                 : 1.0f;
+    };
     uint8_t* arow = smem + C::kOffA + rs * C::kABytes + rin * 128;
     uint32_t tbuf = 0, tphase = 0;
     uint32_t n_rescored = 0;
     auto epi_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); };
 
-    // bf16(r) of this row into the swizzled A operand; accumulates
-    // ||r - bf16(r)||^2 and ||r||^2 from the fp32 values
-    auto write_a_chunk = [&](int kc, const float (&r8)[8], float& e2, float& n2) {
+    // A operand row: the residual times the row's power-of-two scale s,
+    // rounded to the operand type.  Accumulates
+    // the scaled rounding error ||s r - A||^2 and ||s r||^2.
+    auto write_a_chunk = [&](int kc, const float (&r8)[8], float sc, float& e2, float& n2) {
       uint32_t w[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const float a0 = r8[2 * u], a1 = r8[2 * u + 1];
-        const __nv_bfloat162 h = __floats2bfloat162_rn(a0, a1);
-        const float b0 = __low2float(h), b1 = __high2float(h);
+        const float a0 = r8[2 * u] * sc, a1 = r8[2 * u + 1] * sc;
+        float b0, b1;
+        if constexpr (F16) {
+          const __half2 h = __floats2half2_rn(a0, a1);
+          b0 = __low2float(h);
+          b1 = __high2float(h);
+          w[u] = *reinterpret_cast<const uint32_t*>(&h);
+        } else {
+          const __nv_bfloat162 h = __floats2bfloat162_rn(a0, a1);
+          b0 = __low2float(h);
+          b1 = __high2float(h);
+          w[u] = *reinterpret_cast<const uint32_t*>(&h);
+        }
         e2 = fmaf(a0 - b0, a0 - b0, e2);
         e2 = fmaf(a1 - b1, a1 - b1, e2);
         n2 = fmaf(a0, a0, n2);
         n2 = fmaf(a1, a1, n2);
-        w[u] = *reinterpret_cast<const uint32_t*>(&h);
       }
       const int kb = kc >> 3, c16 = kc & 7;
       uint4* dst = reinterpret_cast<uint4*>(arow + kb * (kRows * 128) + ((c16 ^ (rin & 7)) << 4));
       *dst = make_uint4(w[0], w[1], w[2], w[3]);
     };
-    // twice the bound on |c~ - c|: bf16 rounding of r (Cauchy-Schwarz with
-    // the largest atom norm) plus slack for the accumulation order
-    auto band_of = [&](float e2, float n2) {
-      return 2.0f * dmax * sqrtf(e2) + 0.000244140625f * dmax * sqrtf(n2);
+    // row scale s of the A operand: exact, and for bf16 operands it keeps
+    // the products of a tiny residual out of the fp32 subnormal range
+    auto scale_of = [](float amax) { return pow2_scale(amax); };
+    // writes the A row from the fp32 residual in rres; returns the band
+    auto write_a_row = [&](float sc, float& n2_out) {
+      float e2 = 0.0f, n2 = 0.0f;
+#pragma unroll 1
+      for (int kc = 0; kc < D / 8; ++kc) {
+        float r8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) r8[u] = rres[(kc * 8 + u) * kTileRows];
+        write_a_chunk(kc, r8, sc, e2, n2);
+      }
+      n2_out = n2;
+      // twice the bound on |c~ - s c| (scaled units): rounding of s r
+      // (Cauchy-Schwarz with the largest operand atom norm), conversion of
+      // the dictionary to the operand type, and slack for the accumulation
+      const float econv = F16 ? __ldg(p.dmax + 1) : 0.0f;
+      const float dmax = __ldg(p.dmax) * tdict_of() + econv;
+      const float rn = sqrtf(n2);
+      return 2.0f * dmax * sqrtf(e2) + 2.0f * econv * rn + 0.000244140625f * dmax * rn;
     };
     // fp32 correlation in k order (the CUDA-core encoder's arithmetic)
     auto dot_atom = [&](uint32_t i) {
@@ -453,8 +533,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t grow = (int64_t)tile * kTileRows + row;
       const bool valid = grow < p.n_vec;
       if (lead && !*s_abort) {
-        // residual <- x; A <- bf16(x)
-        float e2 = 0.0f, n2 = 0.0f;
+        // residual <- x; A <- operand(scale * x)
+        float amax = 0.0f;
 #pragma unroll 1
         for (int kc = 0; kc < D / 8; ++kc) {
           float r8[8];
@@ -480,10 +560,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int u = 0; u < 8; ++u) r8[u] = 0.0f;
           }
 #pragma unroll
-          for (int u = 0; u < 8; ++u) rres[(kc * 8 + u) * kTileRows] = r8[u];
-          write_a_chunk(kc, r8, e2, n2);
+          for (int u = 0; u < 8; ++u) {
+            rres[(kc * 8 + u) * kTileRows] = r8[u];
+            amax = fmaxf(amax, fabsf(r8[u]));
+          }
         }
-        s_band[row] = band_of(e2, n2);
+        const float sc = scale_of(amax);
+        float n2;
+        s_band[row] = write_a_row(sc, n2);
+        s_scl[row] = sc;
         s_act[row] = (valid && n2 > 0.0f) ? 1u : 0u;
         fence_proxy_async();
         __syncwarp();
@@ -493,8 +578,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       float band = s_band[row];
       bool active = s_act[row] != 0u;
 
+      float best_next = -INFINITY;   // lower bound on the next step's max
       for (int j = 0; j < steps_total; ++j) {
-        float best = -INFINITY, thr = -INFINITY;
+        float best = best_next, thr = best_next - band;
+        best_next = -INFINITY;
         int cnt = 0;
         bool ovf = false;
 #pragma unroll 1
@@ -513,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + tbuf * (kSets * kAtomTile) +
                                  rs * kAtomTile + half * 64;
           // two 32-column halves: 32 accumulator registers live at a time
-#pragma unroll 1
+#pragma unroll
           for (int c = 0; c < 2; ++c) {
             uint32_t v[32];
             __syncwarp();  // reconverge (the previous half may have diverged)
@@ -531,67 +618,79 @@ __global__ void __launch_bounds__(kThreads, 1)
               float t8[8];
 #pragma unroll
               for (int i = 0; i < 8; ++i)
-                t8[i] = fmaxf(fabsf(__uint_as_float(v[g * 16 + i])),
-                              fabsf(__uint_as_float(v[g * 16 + i + 8])));
+                t8[i] = absmax2(__uint_as_float(v[g * 16 + i]), __uint_as_float(v[g * 16 + i + 8]));
 #pragma unroll
-              for (int i = 0; i < 4; ++i) t8[i] = fmaxf(t8[i], t8[i + 4]);
-              m16[g] = fmaxf(fmaxf(t8[0], t8[2]), fmaxf(t8[1], t8[3]));
+              for (int i = 0; i < 4; ++i) t8[i] = absmax2(t8[i], t8[i + 4]);
+              m16[g] = fabsf(absmax2(absmax2(t8[0], t8[2]), absmax2(t8[1], t8[3])));
             }
             const float mt = fmaxf(m16[0], m16[1]);
-            if (active && mt >= thr) {
+            const bool trig = active && mt >= thr;
+            if (trig) {
               best = fmaxf(best, mt);
               thr = best - band;
             }
             // Candidates: every column within `band` of the running maximum.
-            // A triggering lane stages its 16-column group in shared memory
-            // and 16 lanes of the warp test and append them to that lane's
-            // list together (cost per trigger independent of group width).
+            // Triggering lanes stage their raw 16-column groups in shared
+            // memory, two at a time; each half-warp tests and appends one
+            // staged group to its owner's list.
+            if (__ballot_sync(0xffffffffu, trig) == 0u) continue;
             const int col0 = a * kAtomTile + half * 64 + c * 32;
 #pragma unroll
             for (int g = 0; g < 2; ++g) {
-              unsigned tm = __ballot_sync(0xffffffffu, active && m16[g] >= thr);
+              unsigned tm = __ballot_sync(0xffffffffu, trig && m16[g] >= thr);
               while (tm != 0u) {
-                const int L = __ffs(tm) - 1;
+                const int L1 = __ffs(tm) - 1;
                 tm &= tm - 1u;
-                if (lane == L) {
-                  float4* s4 = reinterpret_cast<float4*>(stg);
+                const int L2 = tm != 0u ? __ffs(tm) - 1 : -1;
+                if (L2 >= 0) tm &= tm - 1u;
+                if (lane == L1 || lane == L2) {
+                  uint4* s4 = reinterpret_cast<uint4*>(stg + (lane == L1 ? 0 : 16));
 #pragma unroll
                   for (int i = 0; i < 4; ++i)
-                    s4[i] = make_float4(fabsf(__uint_as_float(v[g * 16 + 4 * i])),
-                                        fabsf(__uint_as_float(v[g * 16 + 4 * i + 1])),
-                                        fabsf(__uint_as_float(v[g * 16 + 4 * i + 2])),
-                                        fabsf(__uint_as_float(v[g * 16 + 4 * i + 3])));
+                    s4[i] = make_uint4(v[g * 16 + 4 * i], v[g * 16 + 4 * i + 1],
+                                       v[g * 16 + 4 * i + 2], v[g * 16 + 4 * i + 3]);
                 }
                 __syncwarp();
-                const float thrL = __shfl_sync(0xffffffffu, thr, L);
-                const float av = lane < 16 ? stg[lane] : 0.0f;
-                const int col = col0 + g * 16 + lane;
-                const bool take = lane < 16 && av >= thrL && col < p.n;
+                const int hl = lane >> 4;                    // half-warp -> owner
+                const int L = hl == 0 ? L1 : L2;
+                const int Ls = L < 0 ? L1 : L;               // valid shuffle source
+                const float thrL = __shfl_sync(0xffffffffu, thr, Ls);
+                const int cntL0 = __shfl_sync(0xffffffffu, cnt, Ls);
+                const float av = fabsf(stg[lane]);
+                const int col = col0 + g * 16 + (lane & 15);
+                const bool take = L >= 0 && av >= thrL && col < p.n;
                 const unsigned pm = __ballot_sync(0xffffffffu, take);
-                const int np = __popc(pm);
-                int cntL = __shfl_sync(0xffffffffu, cnt, L);
-                if (cntL + np > kCand) {
-                  // make room: drop the owner's stale candidates
-                  if (lane == L) {
+                const unsigned pmh = hl == 0 ? (pm & 0xFFFFu) : (pm >> 16);
+                const int np = __popc(pmh);
+                int cntL = cntL0;
+                const bool full = L >= 0 && cntL + np > kCand;
+                if (__ballot_sync(0xffffffffu, full) != 0u) {
+                  // make room: owners drop their stale candidates
+                  if (lane == L1 || lane == L2) {
                     int w = 0;
                     for (int t = 0; t < cnt; ++t)
                       if (cand_val(cw[t]) >= thr) cw[w++] = cw[t];
                     cnt = w;
                   }
                   __syncwarp();
-                  cntL = __shfl_sync(0xffffffffu, cnt, L);
+                  cntL = __shfl_sync(0xffffffffu, cnt, Ls);
                 }
                 if (take) {
-                  const int pos = cntL + __popc(pm & lt);
+                  const int pos = cntL + __popc(pmh & ((1u << (lane & 15)) - 1u));
                   const uint32_t ab = __float_as_uint(av);
                   if (pos < kCand)
                     s_cw[(e * 32 + L) * kCand + pos] =
                         (((ab + 0xFFFFu) >> 16) << 16) | (uint32_t)col;
                 }
-                if (lane == L) {
-                  const int nc = cntL + np;
-                  ovf |= nc > kCand;
-                  cnt = nc < kCand ? nc : kCand;
+                const int np1 = __popc(pm & 0xFFFFu), np2 = __popc(pm >> 16);
+                const int cn1 = __shfl_sync(0xffffffffu, cntL, 0);
+                const int cn2 = __shfl_sync(0xffffffffu, cntL, 16);
+                if (lane == L1) {
+                  ovf |= cn1 + np1 > kCand;
+                  cnt = min(cn1 + np1, kCand);
+                } else if (lane == L2) {
+                  ovf |= cn2 + np2 > kCand;
+                  cnt = min(cn2 + np2, kCand);
                 }
                 __syncwarp();
               }
@@ -607,14 +706,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         epi_sync();
         const float pbest = s_best[tix ^ 128];
         const uint32_t pcw_cnt = s_cnt[tix ^ 128];
+        uint32_t sidx = 0xFFFFFFFFu, own_best = 0xFFFFFFFFu;   // own top-2 candidates
         const bool anyovf = ovf || (pcw_cnt >> 31) != 0u;
         {
           // each thread re-scores its own candidates that survive the row's
           // threshold; the chunk-outer loop reads the fp32 residual once for
           // all of them and keeps every dot in k order
           const float gthr = fmaxf(best, pbest) - band;
-          float babs = -1.0f, bcoef = 0.0f;
+          float babs = -1.0f, bcoef = 0.0f, sabs = -1.0f;
           uint32_t bidx = 0xFFFFFFFFu;
+          sidx = 0xFFFFFFFFu;
           if (active && !anyovf && !*s_abort) {
             bool ok_e[kCand];
             uint32_t ix[kCand];
@@ -653,12 +754,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!ok_e[e2]) continue;
               const float aa = fabsf(acc[e2]);
               if (aa > babs || (aa == babs && ix[e2] < bidx)) {
+                sabs = babs;
+                sidx = bidx;
                 babs = aa;
                 bcoef = acc[e2];
                 bidx = ix[e2];
+              } else if (aa > sabs || (aa == sabs && ix[e2] < sidx)) {
+                sabs = aa;
+                sidx = ix[e2];
               }
             }
           }
+          own_best = bidx;
           s_rabs[tix] = babs;
           s_ridx[tix] = bidx;
           s_rcoef[tix] = bcoef;
@@ -679,7 +786,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               bidx = oidx;
               coef = s_rcoef[tix ^ 128];
             }
-            pick = bidx;
+            s_ridx[tix] = bidx;   // the row's pick, read by the partner after the barrier
+            if (bidx < (uint32_t)p.n) {
+              pick = bidx;
+            } else {
+              // no candidate survived (only possible with non-finite
+              // correlations): keep atom 0 with coefficient 0 and report it
+              record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x43000000u | (uint32_t)j);
+              pick = 0u;
+              coef = 0.0f;
+            }
           }
           // rows whose candidate list overflowed: exact fp32 scan of every
           // atom shared by the warp, one such row at a time
@@ -736,30 +852,37 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncwarp();
           }
+          if (pick >= (uint32_t)p.n) {
+            record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x44000000u | pick);
+            pick = 0u;
+            coef = 0.0f;
+          }
           if (valid) p.codes[grow * p.k_atoms + j] = make_word(coef, pick);
 
           // residual update r -= coef * d_pick; next A operand
           if (active) {
-            float e2 = 0.0f, n2 = 0.0f;
+            float amax = 0.0f;
             const uint4* dp = reinterpret_cast<const uint4*>(p.dict + (int64_t)pick * D);
 #pragma unroll 1
             for (int kc = 0; kc < D / 8; ++kc) {
               const uint4 dv = __ldg(dp + kc);
               const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
-              float r8[8];
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
                 float* r0 = rres + (kc * 8 + 2 * u) * kTileRows;
                 float* r1 = rres + (kc * 8 + 2 * u + 1) * kTileRows;
-                r8[2 * u] = fmaf(-coef, bf16_lo(dw[u]), *r0);
-                r8[2 * u + 1] = fmaf(-coef, bf16_hi(dw[u]), *r1);
-                *r0 = r8[2 * u];
-                *r1 = r8[2 * u + 1];
+                const float n0 = fmaf(-coef, bf16_lo(dw[u]), *r0);
+                const float n1 = fmaf(-coef, bf16_hi(dw[u]), *r1);
+                *r0 = n0;
+                *r1 = n1;
+                amax = fmaxf(amax, fmaxf(fabsf(n0), fabsf(n1)));
               }
-              if (j + 1 < steps_total) write_a_chunk(kc, r8, e2, n2);
             }
             if (j + 1 < steps_total) {
-              s_band[row] = band_of(e2, n2);
+              const float sc = scale_of(amax);
+              float n2;
+              s_band[row] = write_a_row(sc, n2);
+              s_scl[row] = sc;
               s_act[row] = n2 > 0.0f ? 1u : 0u;
             }
           }
@@ -772,6 +895,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         epi_sync();
         band = s_band[row];
         active = s_act[row] != 0u;
+        // lower bound for the next step: the fp32 correlation of the new
+        // residual with this thread's best candidate that was not picked;
+        // |c'| - band/2 never exceeds that atom's tensor-core value, hence
+        // the next step's maximum (band/2 covers the rounding and
+        // accumulation errors)
+        if (active && !anyovf && j + 1 < steps_total && !*s_abort) {
+          const uint32_t pick_row = s_ridx[lead ? tix : (tix ^ 128)];
+          const uint32_t ru = own_best != pick_row ? own_best : sidx;
+          if (ru < (uint32_t)p.n) best_next = fabsf(dot_atom(ru)) * s_scl[row] * tdict_of() - 0.5f * band;
+        }
       }
       if (lead && valid && p.rsq != nullptr && !*s_abort) {
         float sq = 0.0f;
@@ -795,12 +928,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// max_i ||d_i|| (one thread per atom, 16-byte loads); *out must be zero
-// before the launch
+// Dictionary statistics, one thread per atom (16-byte loads): st[0] =
+// max_i ||d_i||, st[2] = max_ij |d_ij| (float bits; both maxima via integer
+// atomicMax, valid for non-negative floats).  st must be zero before the
+// launch.
 template <int D>
-__global__ void __launch_bounds__(128) dict_norm_kernel(const uint16_t* dict, int n, float* out) {
+__global__ void __launch_bounds__(128) dict_stats_kernel(const uint16_t* dict, int n, float* st) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  float s = 0.0f;
+  float s = 0.0f, am = 0.0f;
   if (i < n) {
     const uint4* dp = reinterpret_cast<const uint4*>(dict + (int64_t)i * D);
 #pragma unroll
@@ -809,15 +944,68 @@ __global__ void __launch_bounds__(128) dict_norm_kernel(const uint16_t* dict, in
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        s = fmaf(bf16_lo(w[u]), bf16_lo(w[u]), s);
-        s = fmaf(bf16_hi(w[u]), bf16_hi(w[u]), s);
+        const float lo = bf16_lo(w[u]), hi = bf16_hi(w[u]);
+        s = fmaf(lo, lo, s);
+        s = fmaf(hi, hi, s);
+        am = fmaxf(am, fmaxf(fabsf(lo), fabsf(hi)));
       }
     }
   }
   float m = sqrtf(s);
 #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  }
+  if ((threadIdx.x & 31) == 0) {
+    if (m > 0.0f) atomicMax(reinterpret_cast<int*>(st), __float_as_int(m));
+    if (am > 0.0f) atomicMax(reinterpret_cast<int*>(st) + 2, __float_as_int(am));
+  }
+}
+
+// fp16 operand copy of the dictionary: out = fp16(t d) with t from st[2];
+// st[1] = max_i ||t d_i - fp16(t d_i)|| (zero before the launch)
+template <int D>
+__global__ void __launch_bounds__(128) dict_f16_kernel(const uint16_t* dict, int n, float* st,
+                                                       __half* out) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const float t = pow2_scale(__int_as_float(reinterpret_cast<const int*>(st)[2]));
+  float e = 0.0f;
+  if (i < n) {
+    const uint4* dp = reinterpret_cast<const uint4*>(dict + (int64_t)i * D);
+    uint4* op = reinterpret_cast<uint4*>(out + (int64_t)i * D);
+#pragma unroll
+    for (int kc = 0; kc < D / 8; ++kc) {
+      const uint4 v = __ldg(dp + kc);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float lo = bf16_lo(w[u]) * t, hi = bf16_hi(w[u]) * t;
+        const __half2 h = __floats2half2_rn(lo, hi);
+        const float dl = lo - __low2float(h), dh = hi - __high2float(h);
+        e = fmaf(dl, dl, e);
+        e = fmaf(dh, dh, e);
+        o[u] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      op[kc] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+  float m = sqrtf(e);
+#pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((threadIdx.x & 31) == 0 && m > 0.0f) atomicMax(reinterpret_cast<int*>(out), __float_as_int(m));
+  if ((threadIdx.x & 31) == 0 && m > 0.0f) atomicMax(reinterpret_cast<int*>(st) + 1, __float_as_int(m));
+}
+
+// operand type of the tensor-core encoder: fp16 (default) or bf16 when the
+// environment variable SDK_ENCODE_OPERANDS is "bf16"
+bool operands_f16() {
+  static int mode = -1;
+  if (mode < 0) {
+    const char* v = getenv("SDK_ENCODE_OPERANDS");
+    mode = (v != nullptr && strcmp(v, "bf16") == 0) ? 0 : 1;
+  }
+  return mode == 1;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -835,12 +1023,17 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 }  // namespace tc
 
+// scratch: 256 B of dictionary statistics, the fp16 operand copy of the
+// dictionary (256-byte aligned), then one fp32 residual tile per CTA
+static size_t dict_copy_bytes(int head_dim, int n_atoms) {
+  return ((size_t)n_atoms * head_dim * 2 + 255) & ~(size_t)255;
+}
+
 size_t encode_tc_scratch_bytes(int64_t n_vec, int head_dim, int n_atoms) {
-  (void)n_atoms;
-  if (head_dim != 64 && head_dim != 128) return 256;
+  if ((head_dim != 64 && head_dim != 128) || n_vec <= 0) return 256;
   int64_t tiles = (n_vec + tc::kTileRows - 1) / tc::kTileRows;
   if (tiles > tc::kMaxCtas) tiles = tc::kMaxCtas;
-  return 256 + (size_t)tiles * head_dim * tc::kTileRows * 4;
+  return 256 + dict_copy_bytes(head_dim, n_atoms) + (size_t)tiles * head_dim * tc::kTileRows * 4;
 }
 
 sdk_status launch_encode_tc(const EncodeParams& p, int head_dim, void* scratch,
@@ -857,26 +1050,35 @@ sdk_status launch_encode_tc(const EncodeParams& p, int head_dim, void* scratch,
   const int sms = num_sms();
   if (grid > sms) grid = sms;
   if (grid > tc::kMaxCtas) grid = tc::kMaxCtas;
+  const bool f16 = tc::operands_f16();
   const size_t per_cta = (size_t)head_dim * tc::kTileRows * 4;
-  if (scratch_bytes < 256 + (size_t)grid * per_cta) return SDK_ERR_CAPACITY;
+  const size_t dict_bytes = dict_copy_bytes(head_dim, p.n);
+  if (scratch_bytes < 256 + dict_bytes + (size_t)grid * per_cta) return SDK_ERR_CAPACITY;
+  float* stats = reinterpret_cast<float*>(scratch);
+  __half* dict16 = reinterpret_cast<__half*>(reinterpret_cast<char*>(scratch) + 256);
 
   CUtensorMap map;
   const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)p.n};
   const cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
   const cuuint32_t box[2] = {64u, (cuuint32_t)tc::kAtomTile};
   const cuuint32_t estr[2] = {1u, 1u};
-  CUresult cr = fn(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(p.dict), dims,
-                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  void* base = f16 ? static_cast<void*>(dict16) : const_cast<uint16_t*>(p.dict);
+  CUresult cr = fn(&map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return SDK_ERR_INVALID_ARG;
   *taken = true;
 
-  float* dmax = reinterpret_cast<float*>(scratch);
-  if (cudaMemsetAsync(dmax, 0, sizeof(float), stream) != cudaSuccess) return SDK_ERR_CUDA;
-  if (head_dim == 128)
-    tc::dict_norm_kernel<128><<<(p.n + 127) / 128, 128, 0, stream>>>(p.dict, p.n, dmax);
-  else
-    tc::dict_norm_kernel<64><<<(p.n + 127) / 128, 128, 0, stream>>>(p.dict, p.n, dmax);
+  if (cudaMemsetAsync(stats, 0, 4 * sizeof(float), stream) != cudaSuccess) return SDK_ERR_CUDA;
+  const unsigned dgrid = (unsigned)((p.n + 127) / 128);
+  if (head_dim == 128) {
+    tc::dict_stats_kernel<128><<<dgrid, 128, 0, stream>>>(p.dict, p.n, stats);
+    if (f16) tc::dict_f16_kernel<128><<<dgrid, 128, 0, stream>>>(p.dict, p.n, stats, dict16);
+  } else {
+    tc::dict_stats_kernel<64><<<dgrid, 128, 0, stream>>>(p.dict, p.n, stats);
+    if (f16) tc::dict_f16_kernel<64><<<dgrid, 128, 0, stream>>>(p.dict, p.n, stats, dict16);
+  }
 
   tc::TcParams tp;
   tp.x = p.x;
@@ -888,23 +1090,35 @@ sdk_status launch_encode_tc(const EncodeParams& p, int head_dim, void* scratch,
   tp.codes = p.codes;
   tp.rsq = p.rsq;
   tp.hdr = p.hdr;
-  tp.resid = reinterpret_cast<float*>(reinterpret_cast<char*>(scratch) + 256);
-  tp.dmax = dmax;
+  tp.resid = reinterpret_cast<float*>(reinterpret_cast<char*>(scratch) + 256 + dict_bytes);
+  tp.dmax = stats;
   tp.n_tiles = (int)tiles;
   tp.n_atom_tiles = (p.n + tc::kAtomTile - 1) / tc::kAtomTile;
 
   static bool attr = false;
   if (!attr) {
-    cudaFuncSetAttribute(tc::encode_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         tc::Cfg<128>::kSmem);
-    cudaFuncSetAttribute(tc::encode_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         tc::Cfg<64>::kSmem);
+    cudaFuncSetAttribute(tc::encode_tc_kernel<128, true>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Cfg<128>::kSmem);
+    cudaFuncSetAttribute(tc::encode_tc_kernel<64, true>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Cfg<64>::kSmem);
+    cudaFuncSetAttribute(tc::encode_tc_kernel<128, false>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Cfg<128>::kSmem);
+    cudaFuncSetAttribute(tc::encode_tc_kernel<64, false>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Cfg<64>::kSmem);
     attr = true;
   }
-  if (head_dim == 128)
-    tc::encode_tc_kernel<128><<<(unsigned)grid, tc::kThreads, tc::Cfg<128>::kSmem, stream>>>(map, tp);
-  else
-    tc::encode_tc_kernel<64><<<(unsigned)grid, tc::kThreads, tc::Cfg<64>::kSmem, stream>>>(map, tp);
+  const dim3 g((unsigned)grid);
+  if (head_dim == 128) {
+    if (f16)
+      tc::encode_tc_kernel<128, true><<<g, tc::kThreads, tc::Cfg<128>::kSmem, stream>>>(map, tp);
+    else
+      tc::encode_tc_kernel<128, false><<<g, tc::kThreads, tc::Cfg<128>::kSmem, stream>>>(map, tp);
+  } else {
+    if (f16)
+      tc::encode_tc_kernel<64, true><<<g, tc::kThreads, tc::Cfg<64>::kSmem, stream>>>(map, tp);
+    else
+      tc::encode_tc_kernel<64, false><<<g, tc::kThreads, tc::Cfg<64>::kSmem, stream>>>(map, tp);
+  }
   return cudaGetLastError() == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
 }
 

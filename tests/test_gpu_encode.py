@@ -1,6 +1,10 @@
 """GPU parity of the greedy-pursuit encoder (sdk_encode / sdk_encode_simt
 through the C ABI) and of sdk_append against the fp64 oracle."""
 
+import os
+import subprocess
+import sys
+
 import numpy as np
 import pytest
 import torch
@@ -22,7 +26,7 @@ def _enc(fn, x, D, k=16, rsq=False):
                            workspace=ws)
     torch.cuda.synchronize()
     rc, hdr = sdk.sdk_check_status(ws)
-    assert rc == 0
+    assert rc == 0, (rc, [hex(h) for h in hdr])
     return res, hdr
 
 
@@ -83,8 +87,10 @@ def test_prefill_sampled_vectors_and_certificate(fn):
 @pytest.mark.parametrize("fn", ENCODERS)
 def test_edge_cases(fn):
     """Ragged vector count, a zero vector (atom 0, coefficient 0 at every
-    step), a scaled atom (exact first pick, then zero residual), bf16
-    input, fewer picks, and a dictionary size that fills no tile."""
+    step), a scaled atom (exact first pick; the residual then shrinks by
+    about 2^-10 per step towards the fp32 subnormal range, which the
+    operand scaling must survive), bf16 input, fewer picks, and a
+    dictionary size that fills no tile."""
     g = workloads.make_gen(21)
     n, d = 1000, 128
     D = workloads.gaussian_dictionary(n, d, g)
@@ -170,3 +176,36 @@ def test_append_writes_the_layout():
     with pytest.raises(sdk.SdkError):
         sdk.sdk_append(store, torch.randn(B, Hkv, 50, d).cuda(),
                        torch.randn(B, Hkv, 50, d).cuda(), DK, DV)
+
+
+_BF16_OPERANDS = r"""
+import sys, torch
+sys.path.insert(0, sys.argv[1])
+import workloads, sparse_dictionary_coded_b200 as sdk
+w = workloads.layer4k()
+p = workloads.prefill(n_tokens=256)
+for x, D in ((w["xv"].reshape(-1, 128)[:4096], w["DV"]),
+             (p["xk"].reshape(-1, 128), p["DK"])):
+    x, D = x.cuda(), D.cuda()
+    out = []
+    for fn in (sdk.sdk_encode, sdk.sdk_encode_simt):
+        ws = sdk.new_workspace(sdk.sdk_encode_workspace_bytes(x.shape[0], 128, D.shape[0]))
+        c, r = fn(x, D, resid_sqnorm=True, workspace=ws)
+        torch.cuda.synchronize()
+        assert sdk.sdk_check_status(ws)[0] == 0
+        out.append((c.cpu(), r.cpu()))
+    assert torch.equal(out[0][0], out[1][0]) and torch.equal(out[0][1], out[1][1])
+print("bf16 operands: identical")
+"""
+
+
+def test_bf16_operands_agree_exactly():
+    """The tensor-core encoder with bf16 operands (SDK_ENCODE_OPERANDS=bf16,
+    read once per process, hence a child process) gives the same words and
+    residual energies as the CUDA-core encoder."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, SDK_ENCODE_OPERANDS="bf16")
+    r = subprocess.run([sys.executable, "-c", _BF16_OPERANDS, root], env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "identical" in r.stdout
