@@ -19,7 +19,7 @@ key and value vectors first and then applies textbook attention:
   5. V^_t   = sum_{j<16} c^V_tj D_V[idx^V_tj];  out = sum_t p_t V^_t
 Query head h reads KV head h // (Hq / Hkv).
 
-Readings where the pages are silent (listed in DESIGN.md): "first Klow
+Readings where the pages are silent: "first Klow
 atoms" are the first three in greedy pick order; k uses ceil; ties in the
 selection go to the lower token index; the logit scale is 1/sqrt(d) unless
 given; selection is per query head; the full-softmax flag only widens the

@@ -12,7 +12,7 @@ FAQ "What is the 15x KV cache compression ..."; authors' abstract):
   * the encoder is a projection-based greedy pursuit that replaces OMP so
     that no least-squares refit is done.
 
-Readings where the pages are silent (each one is listed in the design doc):
+Readings where the pages are silent:
   * a step picks the atom that maximises |<r, d_i>|; ties go to the lowest
     atom index (np.argmax returns the first occurrence);
   * the coefficient is the projection <r, d_i*> itself, unrounded, and the

@@ -29,7 +29,7 @@ N_ATOMS = 32768
 K_ATOMS = 16
 KLOW_PLANES = 3
 
-# The five workloads (one per entry of the benchmark's config list).
+# The five workloads.
 WORKLOADS = {
     "tiny": dict(
         index=0, d=64, n_atoms=1024, n_tokens=256, B=1, Hq=4, Hkv=1, L=1,
