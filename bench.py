@@ -172,12 +172,15 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The largest x over all ranks (every rank gets it)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
     return float(t.item())
 
 
@@ -543,7 +546,7 @@ def reference_arm(args):
     name = args.workload
     vals = []
     for _ in range(args.warmup):
-        pass
+        cpu_baseline(name, budget_s=0.5)
     t0 = time.perf_counter()
     for _ in range(max(1, args.steps)):
         vals.append(cpu_baseline(name, budget_s=min(20.0, 120.0 / max(1, args.steps))))
