@@ -193,6 +193,48 @@ SDK_API sdk_status sdk_decode_attn(const float* q, int32_t B, int32_t Hq, int32_
 SDK_API size_t sdk_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t head_dim,
                                   int32_t n_atoms, int64_t max_len);
 
+/* ------------------------------------------------- decode, no workspace
+ * sdk_decode_attn_static -- sdk_decode_attn with its workspace in a fixed
+ * array of SDK_DECODE_STATIC_WS_BYTES (16 MiB) of the library's own device
+ * memory, one per device, so that the call allocates nothing and takes no
+ * workspace.  The paper has no counterpart: this is a calling convention
+ * for hosts that cannot allocate device memory where they decode (a
+ * serving loop whose memory is budgeted before the first request, a plain
+ * C host without a device allocator of its own).
+ *
+ *   arguments  as sdk_decode_attn, without workspace/ws_bytes;
+ *   status_out device, uint32 [2], 4-byte aligned, nullable: after the
+ *              decode, the call copies in the first device-side failure
+ *              recorded since the last such copy (status, detail; {0, 0} if
+ *              none) and zeroes it in the array.  With NULL a failure stays
+ *              recorded until a later call passes status_out.
+ *   limit      sdk_decode_workspace_bytes(B, Hq, head_dim, n_atoms,
+ *              max_len) <= SDK_DECODE_STATIC_WS_BYTES, else SDK_ERR_CAPACITY
+ *              before anything is launched (for example one sequence with
+ *              32 query heads over 32768-atom dictionaries fits up to
+ *              about 11,000 tokens).
+ *   zeroing    the array's header words must start at zero: they are zero
+ *              when the module loads and status_out re-zeroes them; the
+ *              kernels write every other byte before reading it.
+ *   setup      the first call on a device looks up the array's address
+ *              (cudaGetSymbolAddress, which may load the module); make that
+ *              first call before any stream capture.
+ *   races      there is one array per device: calls that overlap in time
+ *              on a device (other streams, other host threads) race on it
+ *              and give undefined results; serialise them on one stream.
+ */
+#define SDK_DECODE_STATIC_WS_BYTES (16u << 20)
+SDK_API sdk_status sdk_decode_attn_static(const float* q, int32_t B, int32_t Hq,
+                           int32_t Hkv, int32_t head_dim,
+                           const void* dict_k, const void* dict_v,
+                           int32_t n_atoms, const uint32_t* k_lo,
+                           const uint32_t* k_full, const uint32_t* v_full,
+                           int64_t cap, const int32_t* lens_host,
+                           int32_t klow, int32_t khigh, int32_t top_num,
+                           int32_t top_den, int32_t full_softmax, float scale,
+                           float* out, uint32_t* status_out,
+                           sdk_stream_t stream);
+
 /* Byte offsets of the decode workspace regions, for inspection by tests
  * and tools after a call (contents are valid until the next call using the
  * same workspace).  R = B*Hq query heads, L = max_len. */

@@ -18,6 +18,7 @@ STATUS_NAMES = {
 }
 SDK_F32, SDK_BF16 = 0, 1
 MAX_ATOMS, K_ATOMS, KLOW_PLANES, MAX_BATCH, WS_ALIGN = 32768, 16, 3, 64, 256
+DECODE_STATIC_WS_BYTES = 16 << 20
 
 # every symbol include/sdk.h declares, with (restype, argtypes)
 _vp, _i32, _i64, _sz, _f32 = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64,
@@ -38,6 +39,11 @@ SIGNATURES = {
                                        _i32, _vp, _vp, _vp, _i64, _vp, _i32,
                                        _i32, _i32, _i32, _i32, _f32, _vp, _vp,
                                        _sz, _vp]),
+    "sdk_decode_attn_static": (ctypes.c_int, [_vp, _i32, _i32, _i32, _i32,
+                                              _vp, _vp, _i32, _vp, _vp, _vp,
+                                              _i64, _vp, _i32, _i32, _i32,
+                                              _i32, _i32, _f32, _vp, _vp,
+                                              _vp]),
     "sdk_decode_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i64]),
     "sdk_decode_layout_of": (ctypes.c_int, [_i32, _i32, _i32, _i32, _i64,
                                             _vp]),

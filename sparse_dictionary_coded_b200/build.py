@@ -15,7 +15,8 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsdk.so")
 
-SOURCES = ["api.cu", "decode.cu", "encode_simt.cu", "encode_tc.cu"]
+SOURCES = ["api.cu", "decode.cu", "decode_static.cu", "encode_simt.cu",
+           "encode_tc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
          "-Xcompiler", "-fvisibility=hidden", "-I", os.path.join(ROOT, "include")]
