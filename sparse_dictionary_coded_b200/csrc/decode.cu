@@ -17,16 +17,17 @@
 //   final_kernel     one CTA per head: last radix digit over the candidates,
 //                    the exact k-th key, tie handling by token index, and
 //                    the rest of the selected set.
-//   rescore_kernel   s_t = scale * sum_{j<khigh} c_tj QD[idx_tj] for the
-//                    selected tokens (64-byte k_full records).
-//   value_kernel     p_t = exp(s_t - max) / z and the scatter
-//                    w[idx^V_tj] += p_t c^V_tj (shared-memory fixed-point
-//                    atomics into a per-atom weight tile per CTA; a cluster
-//                    of CTAs per head sums its tiles through distributed
-//                    shared memory).
+//   attend_kernel    s_t = scale * sum_{j<khigh} c_tj QD[idx_tj] for the
+//                    selected tokens (64-byte k_full records), p = softmax,
+//                    and the scatter w[idx^V_tj] += p_t c^V_tj into a
+//                    shared-memory per-atom weight tile (fixed-point
+//                    atomics); one cluster of CTAs per head shares the
+//                    softmax statistics and sums its tiles through
+//                    distributed shared memory.
 //   out_kernel       out += w D_V over atom tiles (vector reductions into
 //                    `out`, zeroed by qd_kernel).
 #include <cooperative_groups.h>
+#include <type_traits>
 
 #include "sdk_internal.cuh"
 
@@ -102,21 +103,28 @@ __device__ void block_find_desc(const uint32_t* hist, uint32_t k,
   __syncthreads();
 }
 
+constexpr int kTable = 32768;   // shared QD / weight tables: every 15-bit index
+
 // ---------------------------------------------------------------- qd_kernel
-// QD[r][a] = sum_k q[r][k] D_K[a][k] on a 128-atom x 32-row tile.  The atom
-// tile is kept as bf16 in shared memory ([k][atom]); thread (ta, tr) owns
-// atoms 4ta..4ta+3 and rows 4tr..4tr+3 (16 accumulators, fp32 FMA chains in
-// k order).  48 KB of shared memory per CTA lets four CTAs share an SM.
+// QD[r][a] = sum_k q[r][k] D_K[a][k] on a 64-atom x 32-row tile per CTA of
+// two warps.  The atom tile is staged as bf16 [k][64] and the query rows as
+// fp32 [k][32] (groups of 4 rows XOR-swizzled by k, so the transposing
+// stores spread over the banks).  Lane (ta, tr) of warp w owns atoms
+// 32w + 4ta .. +3 and rows 8tr .. 8tr+7: per k, one 8-byte and two 16-byte
+// shared loads feed 32 FMAs (fp32, k order).  32 KB of shared memory.
 // The first kernel of a call also zeroes the per-head selection state, both
 // histograms and `out` (accumulated with reductions by out_kernel).
-constexpr int kQdThreads = 256;
+constexpr int kGvAtoms = 64;
+constexpr int kQdThreads = 64;
+
+__device__ __forceinline__ int qswz(int k, int r) { return (((r >> 2) ^ (k & 7)) << 2) | (r & 3); }
 
 template <int D>
 __global__ void __launch_bounds__(kQdThreads) qd_kernel(DecodeParams p) {
-  __shared__ __align__(16) uint16_t Ds[D][128];   // atom tile, k-major, bf16
-  __shared__ __align__(16) float Qs[D][32];       // query rows, k-major
+  __shared__ __align__(16) uint16_t Ds[D][kGvAtoms];
+  __shared__ __align__(16) float Qs[D][32];
   const int n = p.n, R = p.R, tid = threadIdx.x;
-  const int a0 = blockIdx.x * 128, r0 = blockIdx.y * 32;
+  const int a0 = blockIdx.x * kGvAtoms, r0 = blockIdx.y * 32;
   {
     const int64_t nthr = (int64_t)gridDim.x * gridDim.y * kQdThreads;
     const int64_t g0 = ((int64_t)blockIdx.y * gridDim.x + blockIdx.x) * kQdThreads + tid;
@@ -140,140 +148,217 @@ __global__ void __launch_bounds__(kQdThreads) qd_kernel(DecodeParams p) {
       p.st[e] = st;
     }
   }
-  for (int e = tid; e < 128 * (D / 8); e += kQdThreads) {
-    const int a = e & 127, c = e >> 7;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (a0 + a < n) v = __ldg(reinterpret_cast<const uint4*>(p.dk + (int64_t)(a0 + a) * D) + c);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  // atom tile: lanes take consecutive atoms; all loads of a thread are in
+  // flight before its first store
+  constexpr int kChunk = 8;   // loads in flight per thread while staging
+#pragma unroll 1
+  for (int u0 = 0; u0 < kGvAtoms * (D / 8) / kQdThreads; u0 += kChunk) {
+    uint4 v[kChunk];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      Ds[c * 8 + 2 * u][a] = (uint16_t)(w[u] & 0xFFFFu);
-      Ds[c * 8 + 2 * u + 1][a] = (uint16_t)(w[u] >> 16);
+    for (int u = 0; u < kChunk; ++u) {
+      const int e = tid + (u0 + u) * kQdThreads;
+      const int a = e % kGvAtoms, c = e / kGvAtoms;
+      v[u] = (a0 + a < n) ? __ldg(reinterpret_cast<const uint4*>(p.dk + (int64_t)(a0 + a) * D) + c)
+                          : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < kChunk; ++u) {
+      const int e = tid + (u0 + u) * kQdThreads;
+      const int a = e % kGvAtoms, c = e / kGvAtoms;
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        Ds[c * 8 + 2 * x][a] = (uint16_t)(w[x] & 0xFFFFu);
+        Ds[c * 8 + 2 * x + 1][a] = (uint16_t)(w[x] >> 16);
+      }
     }
   }
-  for (int e = tid; e < 32 * D; e += kQdThreads) {
-    const int r = e & 31, k = e >> 5;
-    Qs[k][r] = (r0 + r < R) ? __ldg(p.q + (int64_t)(r0 + r) * D + k) : 0.0f;
+  // query rows: 16-byte loads along k
+#pragma unroll 1
+  for (int u0 = 0; u0 < 32 * (D / 4) / kQdThreads; u0 += kChunk) {
+    float4 v[kChunk];
+#pragma unroll
+    for (int u = 0; u < kChunk; ++u) {
+      const int e = tid + (u0 + u) * kQdThreads;
+      const int k4 = e % (D / 4), r = e / (D / 4);
+      v[u] = (r0 + r < R) ? __ldg(reinterpret_cast<const float4*>(p.q + (int64_t)(r0 + r) * D) + k4)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kChunk; ++u) {
+      const int e = tid + (u0 + u) * kQdThreads;
+      const int k4 = e % (D / 4), r = e / (D / 4);
+      const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) Qs[4 * k4 + j][qswz(4 * k4 + j, r)] = x[j];
+    }
   }
   __syncthreads();
-  const int ta = tid & 31, tr = tid >> 5;
-  float acc[4][4];
+  const int lane = tid & 31, warp = tid >> 5;
+  const int ta = lane & 7, tr = lane >> 3;
+  const int ac = warp * 32 + 4 * ta;          // first atom column of the thread
+  float acc[8][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int u = 0; u < 4; ++u) acc[i][u] = 0.0f;
-#pragma unroll 8
+#pragma unroll 4
   for (int k = 0; k < D; ++k) {
-    const uint2 dv = *reinterpret_cast<const uint2*>(&Ds[k][4 * ta]);
-    const float4 qv = *reinterpret_cast<const float4*>(&Qs[k][4 * tr]);
+    const uint2 dv = *reinterpret_cast<const uint2*>(&Ds[k][ac]);
+    const float4 qa = *reinterpret_cast<const float4*>(&Qs[k][((2 * tr) ^ (k & 7)) << 2]);
+    const float4 qb = *reinterpret_cast<const float4*>(&Qs[k][((2 * tr + 1) ^ (k & 7)) << 2]);
     const float dd[4] = {bf16_lo(dv.x), bf16_hi(dv.x), bf16_lo(dv.y), bf16_hi(dv.y)};
-    const float qq[4] = {qv.x, qv.y, qv.z, qv.w};
+    const float qq[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
       for (int u = 0; u < 4; ++u) acc[i][u] = fmaf(qq[i], dd[u], acc[i][u]);
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = r0 + 4 * tr + i;
+  for (int i = 0; i < 8; ++i) {
+    const int r = r0 + 8 * tr + i;
     if (r >= R) continue;
-    float* dst = p.qd + (int64_t)r * n + a0 + 4 * ta;
-    if (a0 + 4 * ta + 3 < n && (n & 3) == 0) {
+    float* dst = p.qd + (int64_t)r * n + a0 + ac;
+    if (a0 + ac + 3 < n && (n & 3) == 0) {
       *reinterpret_cast<float4*>(dst) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
     } else {
 #pragma unroll
       for (int u = 0; u < 4; ++u)
-        if (a0 + 4 * ta + u < n) dst[u] = acc[i][u];
+        if (a0 + ac + u < n) dst[u] = acc[i][u];
     }
   }
 }
 
-// Stage QD[r] (n floats) into shared memory.
-__device__ __forceinline__ void stage_row(float* dst, const float* src, int n) {
-  if ((n & 3) == 0 && ((reinterpret_cast<uintptr_t>(src) & 15) == 0)) {
-    const float4* s4 = reinterpret_cast<const float4*>(src);
-    float4* d4 = reinterpret_cast<float4*>(dst);
-    for (int i = threadIdx.x; i < (n >> 2); i += blockDim.x) d4[i] = __ldg(s4 + i);
-  } else {
-    for (int i = threadIdx.x; i < n; i += blockDim.x) dst[i] = __ldg(src + i);
-  }
-}
-
 // -------------------------------------------------------------- klow_kernel
+// s_lo for every (query head, token): QD[r] staged in a 32768-entry shared
+// table (zero past n: every 15-bit index reads inside it, and an index >= n
+// is reported once per thread after the scan), the three k_lo planes read
+// four tokens at a time (16-byte loads when the planes are 16-byte
+// aligned), one gather and one FMA per word.  Writes the order-preserving
+// key of every token and the 12-bit histogram of key bits 31..20 of every
+// head (shared-memory atomics, flushed once per segment).
 constexpr int kScanThreads = 512;
 constexpr int kKlowThreads = 1024;
-constexpr int kKlowU = 4;   // tokens per thread per batch
 
-__global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p) {
+// QD row -> table[0..kTable), zero past n.  Eight 16-byte loads per thread
+// are issued before any is stored, so the staging costs about one L2 round
+// trip instead of eight.
+__device__ __forceinline__ void stage_table(float* table, const float* src, int n) {
+  const int nt = blockDim.x;
+  if ((n & 3) == 0 && ((reinterpret_cast<uintptr_t>(src) & 15) == 0)) {
+    const float4* s4 = reinterpret_cast<const float4*>(src);
+    float4* d4 = reinterpret_cast<float4*>(table);
+    const int n4 = n >> 2;
+    for (int i0 = threadIdx.x; i0 < n4; i0 += 8 * nt) {
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * nt;
+        v[u] = i < n4 ? __ldg(s4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * nt;
+        if (i < n4) d4[i] = v[u];
+      }
+    }
+  } else {
+    for (int i = threadIdx.x; i < n; i += nt) table[i] = __ldg(src + i);
+  }
+  for (int i = n + threadIdx.x; i < kTable; i += nt) table[i] = 0.0f;
+}
+
+__global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, int vec) {
   extern __shared__ float4 smem4[];
-  float* sq = reinterpret_cast<float*>(smem4);
-  uint32_t* sh = reinterpret_cast<uint32_t*>(sq + ((p.n + 3) & ~3));
+  float* table = reinterpret_cast<float*>(smem4);
+  uint32_t* sh = reinterpret_cast<uint32_t*>(table + kTable);
   const int n = p.n, tid = threadIdx.x;
   const int64_t total = p.tok_off[p.B];
   const int64_t G0 = total * blockIdx.x / gridDim.x;
   const int64_t G1 = total * (blockIdx.x + 1) / gridDim.x;
   const int nlo = min(p.klow, kLoPlanes);
+  uint32_t maxidx = 0u;
 
-  for_segments(p.tok_off, p.lens, p.B, G0, G1, [&](int b, int h, int64_t t0, int64_t t1) {
+  for_segments(p.tok_off, p.lens, p.B, G0, G1, [&](int b, int h, int64_t t0l, int64_t t1l) {
     const int r = b * p.Hq + h, kvh = h / p.g;
-    const float* qdr = p.qd + (int64_t)r * n;
-    const bool stage = (t1 - t0) * p.klow >= (int64_t)(n / 2);
-    if (stage) stage_row(sq, qdr, n);
+    const int t0 = (int)t0l, t1 = (int)t1l;    // token indices fit 31 bits
+    stage_table(table, p.qd + (int64_t)r * n, n);
     for (int i = tid; i < 4096; i += kKlowThreads) sh[i] = 0u;
     __syncthreads();
-    const float* src = stage ? sq : qdr;
     const int64_t head = (int64_t)b * p.Hkv + kvh;
     const uint32_t* plane = p.k_lo + head * kLoPlanes * p.cap;
     const uint32_t* rec = p.k_full + head * p.cap * kAtoms;
     uint32_t* keys = p.keys + (int64_t)r * p.L;
-    constexpr int64_t kBatch = (int64_t)kKlowU * kKlowThreads;
-    // register double buffer: the next batch's plane words are in flight
-    // while the current batch is scored
-    uint32_t wv[kKlowU][kLoPlanes], wn[kKlowU][kLoPlanes];
-    auto load_batch = [&](int64_t tb, uint32_t (&w)[kKlowU][kLoPlanes]) {
+    // quads of 4 tokens [4q, 4q+4); the segment's edge quads are masked
+    const int q0 = t0 >> 2, q1 = (t1 + 3) >> 2;
+    auto load_quad = [&](int q, uint32_t (&w)[kLoPlanes][4]) {
 #pragma unroll
-      for (int u = 0; u < kKlowU; ++u) {
-        const int64_t t = tb + tid + u * kKlowThreads;
+      for (int j = 0; j < kLoPlanes; ++j) {
+        if (j < nlo && q < q1) {
+          if (vec) {
+            const uint4 v = __ldcs(reinterpret_cast<const uint4*>(plane + j * p.cap) + q);
+            w[j][0] = v.x; w[j][1] = v.y; w[j][2] = v.z; w[j][3] = v.w;
+            if (4 * q < t0 || 4 * q + 4 > t1) {     // edge quad: words of other tokens
 #pragma unroll
-        for (int j = 0; j < kLoPlanes; ++j)
-          w[u][j] = (t < t1 && j < nlo) ? __ldcs(plane + j * p.cap + t) : 0u;
+              for (int u = 0; u < 4; ++u)
+                if (4 * q + u < t0 || 4 * q + u >= t1) w[j][u] = 0u;
+            }
+          } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int t = 4 * q + u;
+              w[j][u] = (t >= t0 && t < t1) ? __ldcs(plane + j * p.cap + t) : 0u;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) w[j][u] = 0u;
+        }
       }
     };
-    load_batch(t0, wv);
-    for (int64_t tb = t0; tb < t1; tb += kBatch) {
-      if (tb + kBatch < t1) load_batch(tb + kBatch, wn);
+    // plane lines two iterations ahead into L2 (one lane per 128-byte line)
+    auto prefetch = [&](int q) {
+      if (vec && q < q1 && (q & 7) == 0) {
 #pragma unroll
-      for (int u = 0; u < kKlowU; ++u) {
-        const int64_t t = tb + tid + u * kKlowThreads;
-        if (t >= t1) continue;
+        for (int j = 0; j < kLoPlanes; ++j)
+          if (j < nlo)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(
+                reinterpret_cast<const uint4*>(plane + j * p.cap) + q));
+      }
+    };
+    uint32_t wc[kLoPlanes][4], wn[kLoPlanes][4];
+    int q = q0 + tid;
+    load_quad(q, wc);
+    prefetch(q + kKlowThreads);
+    for (; q < q1; q += kKlowThreads) {
+      load_quad(q + kKlowThreads, wn);
+      prefetch(q + 2 * kKlowThreads);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int t = 4 * q + u;
         float s = 0.0f;
 #pragma unroll
         for (int j = 0; j < kLoPlanes; ++j) {
-          if (j >= nlo) break;
-          const uint32_t idx = word_idx(wv[u][j]);
-          if (idx >= (uint32_t)n) {
-            record_error(p.hdr, SDK_ERR_DEVICE_CHECK, idx);
-            continue;
-          }
-          s = fmaf(word_coef(wv[u][j]), src[idx], s);
+          const uint32_t idx = word_idx(wc[j][u]);
+          maxidx = max(maxidx, idx);
+          s = fmaf(word_coef(wc[j][u]), table[idx], s);
         }
-        for (int j = kLoPlanes; j < p.klow; ++j) {
-          const uint32_t wj = __ldg(rec + t * kAtoms + j);
+        for (int j = kLoPlanes; j < p.klow; ++j) {      // klow > 3: k_full words
+          const uint32_t wj = (t >= t0 && t < t1) ? __ldg(rec + (int64_t)t * kAtoms + j) : 0u;
           const uint32_t idx = word_idx(wj);
-          if (idx >= (uint32_t)n) {
-            record_error(p.hdr, SDK_ERR_DEVICE_CHECK, idx);
-            continue;
-          }
-          s = fmaf(word_coef(wj), src[idx], s);
+          maxidx = max(maxidx, idx);
+          s = fmaf(word_coef(wj), table[idx], s);
         }
-        const uint32_t key = score_key(s);
-        keys[t] = key;
-        atomicAdd(&sh[key >> 20], 1u);
+        if (t >= t0 && t < t1) {
+          const uint32_t key = score_key(s);
+          keys[t] = key;
+          atomicAdd(&sh[key >> 20], 1u);
+        }
       }
 #pragma unroll
-      for (int u = 0; u < kKlowU; ++u)
+      for (int j = 0; j < kLoPlanes; ++j)
 #pragma unroll
-        for (int j = 0; j < kLoPlanes; ++j) wv[u][j] = wn[u][j];
+        for (int u = 0; u < 4; ++u) wc[j][u] = wn[j][u];
     }
     __syncthreads();
     uint32_t* gh = p.hist1 + (int64_t)r * 4096;
@@ -281,22 +366,39 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p) {
       if (sh[i]) atomicAdd(&gh[i], sh[i]);
     __syncthreads();
   });
+  if (maxidx >= (uint32_t)n) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, maxidx);
 }
 
 // ------------------------------------------------------------- pass2_kernel
 // Tokens above the bucket of the k-th key are selected, tokens inside it
 // become candidates (with a histogram of key bits 19..8), the others go to
-// the complement.  Each warp compacts 128 tokens per iteration with ballots
-// and reserves its output slots with one atomic per category.
+// the complement (full-softmax flag only).  A segment is taken in rounds of
+// kSelBuf tokens; each warp takes 128 tokens per step (4 coalesced key
+// loads per lane) and appends its selected tokens to a shared-memory buffer
+// (shared atomics), which is copied out once per round behind one global
+// atomic.  Candidates (and their histogram) are buffered the same way; the
+// complement path (full-softmax flag) writes to global memory directly.
+// Both run only when a ballot finds some.
+constexpr int kSelBuf = 8192;
+constexpr int kCandBuf = 2048;
+constexpr int kPass2Smem = (kSelBuf + 2 * kCandBuf + 4096) * 4;
+
 __global__ void __launch_bounds__(kScanThreads, 2) pass2_kernel(DecodeParams p) {
   __shared__ uint32_t s_tmp[48];
+  __shared__ uint32_t s_nsel, s_base, s_ncand, s_cbase;
+  extern __shared__ uint32_t s_dyn[];   // kPass2Smem bytes
+  int32_t* s_sel = reinterpret_cast<int32_t*>(s_dyn);
+  int32_t* s_ct = s_sel + kSelBuf;
+  uint32_t* s_ck = reinterpret_cast<uint32_t*>(s_ct + kCandBuf);
+  uint32_t* s_h2 = s_ck + kCandBuf;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned lt = (1u << lane) - 1u;
   const int64_t total = p.tok_off[p.B];
   const int64_t G0 = total * blockIdx.x / gridDim.x;
   const int64_t G1 = total * (blockIdx.x + 1) / gridDim.x;
+  constexpr int kWarps = kScanThreads / 32;
 
-  for_segments(p.tok_off, p.lens, p.B, G0, G1, [&](int b, int h, int64_t t0, int64_t t1) {
+  for_segments(p.tok_off, p.lens, p.B, G0, G1, [&](int b, int h, int64_t t0l, int64_t t1l) {
     const int r = b * p.Hq + h;
     const int Nb = p.lens[b];
     sdk_select_state* st = p.st + r;
@@ -308,77 +410,121 @@ __global__ void __launch_bounds__(kScanThreads, 2) pass2_kernel(DecodeParams p) 
       if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x10000000u | r);
       return;
     }
-    if (t0 == 0 && tid == 0) st->n_above = above1;
+    if (t0l == 0 && tid == 0) st->n_above = above1;
     const uint32_t* keys = p.keys + (int64_t)r * p.L;
     int32_t* list = p.list + (int64_t)r * p.L;
     int32_t* ct = p.cand_t + (int64_t)r * p.L;
     uint32_t* ck = p.cand_key + (int64_t)r * p.L;
     uint32_t* h2 = p.hist2 + (int64_t)r * 4096;
+    const bool full = p.full != 0;
     uint32_t cmax = 0u;
-    const int nwarps = kScanThreads / 32;
-    constexpr int U = 4;                       // tokens per lane per batch
-    constexpr int64_t WB = 32 * U;             // tokens per warp batch
-    uint32_t kc[U], kn[U];
-    auto load_keys = [&](int64_t tb, uint32_t (&kk)[U]) {
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int64_t t = tb + lane + 32 * u;
-        kk[u] = t < t1 ? keys[t] : 0u;
+    for (int i = tid; i < 4096; i += kScanThreads) s_h2[i] = 0u;
+    for (int rt0 = (int)t0l; rt0 < (int)t1l; rt0 += kSelBuf) {
+      const int t1 = min((int)t1l, rt0 + kSelBuf);
+      if (tid == 0) {
+        s_nsel = 0u;
+        s_ncand = 0u;
       }
-    };
-    int64_t tb = t0 + (int64_t)warp * WB;
-    if (tb < t1) load_keys(tb, kc);
-    for (; tb < t1; tb += (int64_t)nwarps * WB) {
-      const int64_t tnext = tb + (int64_t)nwarps * WB;
-      if (tnext < t1) load_keys(tnext, kn);
-      unsigned ms[U], mc[U], mo[U];
-      uint32_t ns = 0, nc = 0, no = 0;
+      __syncthreads();
+      uint32_t kc[4], kn[4];
+      auto load = [&](int tb, uint32_t (&kk)[4]) {
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const bool valid = tb + lane + 32 * u < t1;
-        const uint32_t d1 = kc[u] >> 20;
-        ms[u] = __ballot_sync(0xffffffffu, valid && d1 > b1);
-        mc[u] = __ballot_sync(0xffffffffu, valid && d1 == b1);
-        mo[u] = __ballot_sync(0xffffffffu, valid && d1 < b1 && p.full);
-        ns += __popc(ms[u]);
-        nc += __popc(mc[u]);
-        no += __popc(mo[u]);
-      }
-      uint32_t bs = 0, bc = 0, bo = 0;
-      if (lane == 0) {
-        if (ns) bs = atomicAdd(&st->n_sel, ns);
-        if (nc) bc = atomicAdd(&st->n_cand, nc);
-        if (no) bo = atomicAdd(&st->n_comp, no);
-      }
-      bs = __shfl_sync(0xffffffffu, bs, 0);
-      bc = __shfl_sync(0xffffffffu, bc, 0);
-      bo = __shfl_sync(0xffffffffu, bo, 0);
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int64_t t = tb + lane + 32 * u;
-        if ((ms[u] >> lane) & 1u) {
-          const uint32_t pos = bs + __popc(ms[u] & lt);
-          if (pos < (uint32_t)Nb) list[pos] = (int32_t)t;
-        } else if ((mc[u] >> lane) & 1u) {
-          const uint32_t pos = bc + __popc(mc[u] & lt);
-          if (pos < (uint32_t)Nb) {
-            ct[pos] = (int32_t)t;
-            ck[pos] = kc[u];
-          }
-          atomicAdd(&h2[(kc[u] >> 8) & 0xFFFu], 1u);
-        } else if ((mo[u] >> lane) & 1u) {
-          const uint32_t pos = bo + __popc(mo[u] & lt);
-          if (pos < (uint32_t)Nb) list[Nb - 1 - (int64_t)pos] = (int32_t)t;
-          cmax = max(cmax, kc[u]);
+        for (int u = 0; u < 4; ++u) {
+          const int t = tb + lane + 32 * u;
+          kk[u] = t < t1 ? __ldcs(keys + t) : 0u;
         }
-        bs += __popc(ms[u]);
-        bc += __popc(mc[u]);
-        bo += __popc(mo[u]);
-      }
+      };
+      int tb = rt0 + warp * 128;
+      if (tb < t1) load(tb, kc);
+      for (; tb < t1; tb += kWarps * 128) {
+        const int tnext = tb + kWarps * 128;
+        if (tnext < t1) load(tnext, kn);
+        unsigned ms[4];
+        uint32_t ns = 0u;
+        bool anyc = false, anyo = false;
 #pragma unroll
-      for (int u = 0; u < U; ++u) kc[u] = kn[u];
+        for (int u = 0; u < 4; ++u) {
+          const bool valid = tb + lane + 32 * u < t1;
+          const uint32_t d1 = kc[u] >> 20;
+          ms[u] = __ballot_sync(0xffffffffu, valid && d1 > b1);
+          ns += __popc(ms[u]);
+          anyc |= valid && d1 == b1;
+          anyo |= valid && d1 < b1;
+        }
+        uint32_t bs = 0u;
+        if (lane == 0 && ns) bs = atomicAdd(&s_nsel, ns);
+        bs = __shfl_sync(0xffffffffu, bs, 0);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if ((ms[u] >> lane) & 1u) s_sel[bs + __popc(ms[u] & lt)] = tb + lane + 32 * u;
+          bs += __popc(ms[u]);
+        }
+        if (__any_sync(0xffffffffu, anyc)) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const bool c = tb + lane + 32 * u < t1 && (kc[u] >> 20) == b1;
+            const unsigned mc = __ballot_sync(0xffffffffu, c);
+            if (mc == 0u) continue;
+            uint32_t bc = 0u;
+            if (lane == 0) bc = atomicAdd(&s_ncand, (uint32_t)__popc(mc));
+            bc = __shfl_sync(0xffffffffu, bc, 0) + __popc(mc & lt);
+            // slots past the buffer go straight to global memory
+            const bool spill = c && bc >= (uint32_t)kCandBuf;
+            const unsigned mspill = __ballot_sync(0xffffffffu, spill);
+            uint32_t bg = 0u;
+            if (mspill && lane == 0) bg = atomicAdd(&st->n_cand, (uint32_t)__popc(mspill));
+            bg = __shfl_sync(0xffffffffu, bg, 0) + __popc(mspill & lt);
+            if (c) {
+              const int t = tb + lane + 32 * u;
+              if (!spill) {
+                s_ct[bc] = t;
+                s_ck[bc] = kc[u];
+              } else if (bg < (uint32_t)Nb) {
+                ct[bg] = t;
+                ck[bg] = kc[u];
+              }
+              atomicAdd(&s_h2[(kc[u] >> 8) & 0xFFFu], 1u);
+            }
+          }
+        }
+        if (full && __any_sync(0xffffffffu, anyo)) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const bool o = tb + lane + 32 * u < t1 && (kc[u] >> 20) < b1;
+            const unsigned mo = __ballot_sync(0xffffffffu, o);
+            if (mo == 0u) continue;
+            uint32_t bo = 0u;
+            if (lane == 0) bo = atomicAdd(&st->n_comp, (uint32_t)__popc(mo));
+            bo = __shfl_sync(0xffffffffu, bo, 0) + __popc(mo & lt);
+            if (o) {
+              if (bo < (uint32_t)Nb) list[Nb - 1 - (int)bo] = tb + lane + 32 * u;
+              cmax = max(cmax, kc[u]);
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) kc[u] = kn[u];
+      }
+      __syncthreads();
+      if (tid == 0) {
+        s_base = s_nsel ? atomicAdd(&st->n_sel, s_nsel) : 0u;
+        s_ncand = min(s_ncand, (uint32_t)kCandBuf);
+        s_cbase = s_ncand ? atomicAdd(&st->n_cand, s_ncand) : 0u;
+      }
+      __syncthreads();
+      const uint32_t nsel = s_nsel, base = s_base, ncand = s_ncand, cbase = s_cbase;
+      for (uint32_t i = tid; i < nsel; i += kScanThreads)
+        if (base + i < (uint32_t)Nb) list[base + i] = s_sel[i];
+      for (uint32_t i = tid; i < ncand; i += kScanThreads)
+        if (cbase + i < (uint32_t)Nb) {
+          ct[cbase + i] = s_ct[i];
+          ck[cbase + i] = s_ck[i];
+        }
+      __syncthreads();
     }
-    if (p.full) {
+    for (int i = tid; i < 4096; i += kScanThreads)
+      if (s_h2[i]) atomicAdd(&h2[i], s_h2[i]);
+    if (full) {
       cmax = warp_umax(cmax);
       if (lane == 0 && cmax) atomicMax(&st->max_comp, cmax);
     }
@@ -533,297 +679,361 @@ __global__ void __launch_bounds__(kScanThreads) final_kernel(DecodeParams p) {
   }
 }
 
-// ----------------------------------------------------------- rescore_kernel
-// s_t = scale * sum_{j<khigh} c_tj QD[idx_tj] for the selected tokens.  Four
-// lanes share a token: lane c of the group loads words 4c..4c+3 of the
-// 64-byte record (one coalesced 16-byte load; the group reads the record in
-// full), gathers their QD terms and the group sums its partials with two
-// shuffles.  A ring of kRing iterations keeps list entries and records in
-// flight ahead of the one being scored.
-constexpr int kRecThreads = 1024;
-constexpr int kRing = 4;
-
-__global__ void __launch_bounds__(kRecThreads, 1) rescore_kernel(DecodeParams p) {
-  extern __shared__ float4 smem4[];
-  float* sq = reinterpret_cast<float*>(smem4);
-  const int n = p.n, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int grp = lane >> 2, c = lane & 3;
-  constexpr int kWarps = kRecThreads / 32;
-  const int64_t total = p.sel_off[p.B];
-  const int64_t G0 = total * blockIdx.x / gridDim.x;
-  const int64_t G1 = total * (blockIdx.x + 1) / gridDim.x;
-
-  for_segments(p.sel_off, p.kcnt, p.B, G0, G1, [&](int b, int h, int64_t i0, int64_t i1) {
-    const int r = b * p.Hq + h, kvh = h / p.g;
-    const float* qdr = p.qd + (int64_t)r * n;
-    const bool stage = (i1 - i0) * p.khigh >= (int64_t)(n / 2);
-    if (stage) stage_row(sq, qdr, n);
-    __syncthreads();
-    const float* src = stage ? sq : qdr;
-    const uint4* rec = reinterpret_cast<const uint4*>(p.k_full +
-                                                      ((int64_t)b * p.Hkv + kvh) * p.cap * kAtoms);
-    const int32_t* list = p.list + (int64_t)r * p.L;
-    float* out = p.sel_score + (int64_t)r * p.L;
-    const int Nb = p.lens[b];
-    const int jmax = min(p.khigh - 4 * c, 4);   // words of this lane that count
-    auto entry = [&](int64_t it) { return i0 + (it * kWarps + warp) * 8 + grp; };
-    auto fetch = [&](int64_t it, int& t, uint4& w) {
-      const int64_t i = entry(it);
-      t = i < i1 ? list[i] : -1;
-      if (i < i1 && (t < 0 || t >= Nb)) {
-        if (c == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x30000000u | r);
-        t = -1;
-      }
-      w = t >= 0 ? __ldcs(rec + (int64_t)t * 4 + c) : make_uint4(0u, 0u, 0u, 0u);
-    };
-    int tq[kRing];
-    uint4 wq[kRing];
-#pragma unroll
-    for (int s2 = 0; s2 < kRing; ++s2) fetch(s2, tq[s2], wq[s2]);
-    float smax = -INFINITY;
-    for (int64_t it0 = 0; entry(it0) - grp < i1; it0 += kRing) {
-#pragma unroll
-      for (int s2 = 0; s2 < kRing; ++s2) {
-        const int64_t it = it0 + s2;
-        const int64_t i = entry(it);
-        const int t = tq[s2];
-        const uint4 w = wq[s2];
-        fetch(it + kRing, tq[s2], wq[s2]);
-        const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
-        float part = 0.0f;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (u >= jmax) break;
-          const uint32_t idx = word_idx(wd[u]);
-          if (t >= 0 && idx >= (uint32_t)n) {
-            record_error(p.hdr, SDK_ERR_DEVICE_CHECK, idx);
-            continue;
-          }
-          if (t >= 0) part = fmaf(word_coef(wd[u]), src[idx], part);
-        }
-        part += __shfl_xor_sync(0xffffffffu, part, 1);
-        part += __shfl_xor_sync(0xffffffffu, part, 2);
-        if (c == 0 && i < i1) {
-          const float sc = t >= 0 ? part * p.scale : -INFINITY;
-          out[i] = sc;
-          smax = fmaxf(smax, sc);
-        }
-      }
-    }
-    smax = warp_max(smax);
-    if (lane == 0 && smax > -INFINITY) atomicMax(&p.st[r].max_score, score_key(smax));
-    __syncthreads();
-  });
-}
-
-// ------------------------------------------------------------- value_kernel
-// One cluster of C CTAs per query head; CTA `rank` owns a contiguous share
-// of the head's softmax domain (the selected set, or every token with the
-// full-softmax flag).
-//   pass A  e_t = exp(logit_t - max); the cluster sums e_t into z
-//           (distributed shared memory).
-//   pass B  p_t = e_t / z; w[idx^V_tj] += p_t c^V_tj into a shared-memory
-//           tile of n bins, four lanes per token as in rescore_kernel.  The
-//           bins hold 2^-20 fixed point in int32 (native shared-memory
-//           integer atomics, exact and order-independent).  Since
-//           sum_t p_t = 1, a bin can leave the int32 range only if the
-//           CTA's sum of |p_t c_tj| reaches 2^10; a CTA that sees that
-//           re-runs pass B with fp32 atomics.
-//   reduce  each CTA sums its slice of the atoms over the cluster's tiles
-//           and writes w[r] (already normalised) with plain stores.
+// ------------------------------------------------------------ attend_kernel
+// Khigh rescore, softmax and value scatter of one query head, fused.  One
+// cluster of C CTAs per head; CTA `rank` owns the slice
+// [k*rank/C, k*(rank+1)/C) of the head's selected entries list[0..k-1] and,
+// with the full-softmax flag, a slice of the complement entries
+// list[k..N-1] (logit scale * s_lo).
+//   phase 1  QD[r] is staged in a 32768-entry shared table (zero past n, so
+//            every 15-bit index reads inside it; an index >= n adds 0 and is
+//            reported after the loop).  s_i = scale * sum_{j<khigh} c_tj
+//            QD[idx_tj] for the own selected entries, four lanes per
+//            64-byte record, written to sel_score; the cluster's maximum m
+//            through distributed shared memory (with the flag, also the
+//            largest complement logit).
+//   phase 2  z = sum of exp(logit - m) over the head's domain, summed over
+//            the cluster.
+//   phase 3  the table becomes the per-atom weight tile: w[idx^V] += p c^V
+//            with p = exp(logit - m) / z, in 2^-20 fixed point (native int32
+//            shared-memory atomics: exact and order-independent).  Since
+//            sum p = 1, a bin can leave the int32 range only if the CTA's
+//            sum of |p c| reaches 2^10; a CTA that sees that re-runs the
+//            phase with fp32 atomics.
+//   phase 4  each CTA sums its slice of the atoms over the cluster's tiles
+//            and writes the normalised w[r].
+// Records are read in warp batches of 32 entries (one coalesced load of 32
+// list entries, then four records per 4-lane group); the next batch's
+// records are in flight while the current batch is used.
+constexpr int kAttThreads = 768;
 constexpr float kFixScale = 1048576.0f;       // 2^20
 constexpr float kFixInv = 1.0f / 1048576.0f;
 
-__global__ void __launch_bounds__(kRecThreads, 1) value_kernel(DecodeParams p, int C) {
+// Calls f(i, t, w) for every entry i in [e0, e1) of `list`, from all 32
+// lanes of every warp; the 4-lane group (lane >> 2) of entry i holds its
+// record, lane c the words 4c..4c+3 in w.  t < 0 marks a padding slot or an
+// invalid token (reported).  Every lane calls f the same number of times.
+template <class F>
+__device__ __forceinline__ void for_records(const int32_t* list, int e0, int e1, const uint4* rec,
+                                            int Nb, WsHeader* hdr, uint32_t tag, F f) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int grp = lane >> 2, c = lane & 3;
+  constexpr int kStep = kAttThreads;          // entries per round of all warps
+  auto list_at = [&](int b) { return (b + lane < e1) ? __ldg(list + b + lane) : -1; };
+  auto fetch = [&](int b, int tl, int (&t)[4], uint4 (&w)[4]) {
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      int tt = __shfl_sync(0xffffffffu, tl, s * 8 + grp);
+      const int i = b + s * 8 + grp;
+      if (i >= e1) {
+        tt = -1;
+      } else if ((unsigned)tt >= (unsigned)Nb) {
+        if (c == 0) record_error(hdr, SDK_ERR_DEVICE_CHECK, tag);
+        tt = -1;
+      }
+      t[s] = tt;
+      w[s] = tt >= 0 ? __ldcs(rec + (int64_t)tt * 4 + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  // the record of a list entry, two batches ahead, into L2 (64 bytes)
+  auto prefetch = [&](int tl) {
+    if ((unsigned)tl < (unsigned)Nb) {
+      const uint4* a = rec + (int64_t)tl * 4;
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(a + 2));
+    }
+  };
+  int b = e0 + warp * 32;
+  if (b >= e1) return;
+  int tl1 = list_at(b + kStep);        // list entries of batch b + 1
+  int tl2 = list_at(b + 2 * kStep);    // and of batch b + 2
+  int tc[4];
+  uint4 wc[4];
+  fetch(b, list_at(b), tc, wc);
+  prefetch(tl1);
+  for (; b < e1; b += kStep) {
+    const int bn = b + kStep;
+    int tn[4];
+    uint4 wn[4];
+    const bool more = bn < e1;
+    if (more) {
+      fetch(bn, tl1, tn, wn);
+      prefetch(tl2);
+      tl1 = tl2;
+      tl2 = list_at(bn + 2 * kStep);
+    }
+#pragma unroll
+    for (int s = 0; s < 4; ++s) f(b + s * 8 + grp, tc[s], wc[s]);
+    if (more) {
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        tc[s] = tn[s];
+        wc[s] = wn[s];
+      }
+    }
+  }
+}
+
+// block-wide reduction of one float per thread into s_red[0] (max or sum)
+template <bool kMax>
+__device__ __forceinline__ float block_reduce(float v, float* s_red) {
+  v = kMax ? warp_max(v) : warp_sum(v);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) s_red[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    float x = lane < (int)(blockDim.x >> 5) ? s_red[lane] : (kMax ? -INFINITY : 0.0f);
+    x = kMax ? warp_max(x) : warp_sum(x);
+    if (lane == 0) s_red[32] = x;
+  }
+  __syncthreads();
+  return s_red[32];
+}
+
+__global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, int C) {
   extern __shared__ float4 smem4[];
+  float* table = reinterpret_cast<float*>(smem4);
   int* siw = reinterpret_cast<int*>(smem4);
-  float* sfw = reinterpret_cast<float*>(smem4);
-  __shared__ float s_red[kRecThreads / 32];
-  __shared__ float s_z;
+  __shared__ float s_red[33];
+  __shared__ float s_val;
   __shared__ int s_float;
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
-  const int n = p.n, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int grp = lane >> 2, c = lane & 3;
-  constexpr int kWarps = kRecThreads / 32;
+  const int n = p.n, tid = threadIdx.x;
+  const int c = threadIdx.x & 3;
   const int r = blockIdx.x / C;
   const int rank = (int)cluster.block_rank();
   const int b = r / p.Hq, h = r % p.Hq, kvh = h / p.g;
-  const int64_t Dr = p.dcnt[b];
-  const int64_t i0 = Dr * rank / C, i1 = Dr * (rank + 1) / C;
   const int k = p.kcnt[b];
+  const int Dr = p.dcnt[b];
   const int Nb = p.lens[b];
-  const sdk_select_state* st = p.st + r;
-  float m = key_score(st->max_score);
-  if (p.full && st->n_comp > 0u) m = fmaxf(m, p.scale * key_score(st->max_comp));
-  const uint4* rec = reinterpret_cast<const uint4*>(p.v_full +
-                                                    ((int64_t)b * p.Hkv + kvh) * p.cap * kAtoms);
+  const int s0 = (int)((int64_t)k * rank / C), s1 = (int)((int64_t)k * (rank + 1) / C);
+  const int c0 = k + (int)((int64_t)(Dr - k) * rank / C);
+  const int c1 = k + (int)((int64_t)(Dr - k) * (rank + 1) / C);
+  const int64_t head = (int64_t)b * p.Hkv + kvh;
+  const uint4* krec = reinterpret_cast<const uint4*>(p.k_full + head * p.cap * kAtoms);
+  const uint4* vrec = reinterpret_cast<const uint4*>(p.v_full + head * p.cap * kAtoms);
   const int32_t* list = p.list + (int64_t)r * p.L;
-  const float* ss = p.sel_score + (int64_t)r * p.L;
+  float* ss = p.sel_score + (int64_t)r * p.L;
   const uint32_t* keys = p.keys + (int64_t)r * p.L;
-  auto logit_of = [&](int64_t i, int64_t t) {
-    return (i < k) ? ss[i] : p.scale * key_score(keys[t]);
-  };
+  sdk_select_state* st = p.st + r;
+  uint32_t maxidx = 0u;
 
-  for (int i = tid; i < n; i += kRecThreads) siw[i] = 0;
-  // ---- pass A: z
-  float z = 0.0f;
-  for (int64_t i = i0 + tid; i < i1; i += kRecThreads) {
-    const int64_t t = i < k ? 0 : (int64_t)list[i];
-    if (t < 0 || t >= Nb) continue;
-    z += expf(logit_of(i, t) - m);
-  }
-  z = warp_sum(z);
-  if (lane == 0) s_red[warp] = z;
+  // ---- phase 1: stage QD[r], rescore the own selected entries
+  stage_table(table, p.qd + (int64_t)r * n, n);
   __syncthreads();
+  const int jmax = min(p.khigh - 4 * c, 4);   // words of this lane that count
+  float smax = -INFINITY;
+  for_records(list, s0, s1, krec, Nb, p.hdr, 0x30000000u | r,
+              [&](int i, int t, uint4 w) {
+                const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+                float part = 0.0f;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  if (u >= jmax) break;
+                  const uint32_t idx = word_idx(wd[u]);
+                  maxidx = max(maxidx, idx);
+                  part = fmaf(word_coef(wd[u]), table[idx], part);
+                }
+                part += __shfl_xor_sync(0xffffffffu, part, 1);
+                part += __shfl_xor_sync(0xffffffffu, part, 2);
+                if (t >= 0) {
+                  const float sc = part * p.scale;
+                  if (c == 0) ss[i] = sc;
+                  smax = fmaxf(smax, sc);
+                }
+              });
+  smax = block_reduce<true>(smax, s_red);
+  if (tid == 0) s_val = smax;
+  cluster.sync();
+  float m = -INFINITY;
+  for (int cc = 0; cc < C; ++cc) m = fmaxf(m, *cluster.map_shared_rank(&s_val, cc));
+  if (rank == 0 && tid == 0 && m > -INFINITY) st->max_score = score_key(m);
+  if (p.full && st->n_comp > 0u) m = fmaxf(m, p.scale * key_score(st->max_comp));
+
+  // ---- phase 2: z over the own slices of the domain
+  float z = 0.0f;
+#pragma unroll 4
+  for (int i = s0 + tid; i < s1; i += kAttThreads) z += expf(ss[i] - m);
+#pragma unroll 4
+  for (int i = c0 + tid; i < c1; i += kAttThreads) {
+    const int t = list[i];
+    if (t >= 0 && t < Nb) z += expf(p.scale * key_score(keys[t]) - m);
+  }
+  z = block_reduce<false>(z, s_red);
+  cluster.sync();   // every CTA has read s_val of phase 1
   if (tid == 0) {
-    float zz = 0.0f;
-    for (int i = 0; i < kWarps; ++i) zz += s_red[i];
-    s_z = zz;
+    s_val = z;
     s_float = 0;
   }
   cluster.sync();
   float ztot = 0.0f;
-  for (int cc = 0; cc < C; ++cc) ztot += *cluster.map_shared_rank(&s_z, cc);
+  for (int cc = 0; cc < C; ++cc) ztot += *cluster.map_shared_rank(&s_val, cc);
   const float invz = 1.0f / ztot;
 
-  // ---- pass B: scatter p_t c_tj (fixed point; fp32 atomics on re-run)
-  auto entry = [&](int64_t it) { return i0 + (it * kWarps + warp) * 8 + grp; };
-  auto fetch = [&](int64_t it, int& t, uint4& w) {
-    const int64_t i = entry(it);
-    t = i < i1 ? list[i] : -1;
-    if (i < i1 && (t < 0 || t >= Nb)) {
-      if (c == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x31000000u | r);
-      t = -1;
-    }
-    w = t >= 0 ? __ldcs(rec + (int64_t)t * 4 + c) : make_uint4(0u, 0u, 0u, 0u);
-  };
-  for (int pass = 0; pass < 2; ++pass) {
-    const bool use_float = pass == 1;
-    if (use_float) {
-      if (!s_float) break;
-      __syncthreads();
-      for (int i = tid; i < n; i += kRecThreads) sfw[i] = 0.0f;
+  // ---- phase 3: scatter p c^V into the weight tile
+  auto phase3 = [&](auto fl) {
+    constexpr bool kFloat = decltype(fl)::value;
+    {
+      uint4* t4 = reinterpret_cast<uint4*>(smem4);
+      for (int i = tid; i < kTable / 4; i += kAttThreads) t4[i] = make_uint4(0u, 0u, 0u, 0u);
     }
     __syncthreads();
     float absum = 0.0f;
-    int tq[kRing];
-    uint4 wq[kRing];
+    auto scatter = [&](float lg, int t, uint4 w) {
+      if (t < 0) return;
+      const float pt = expf(lg - m) * invz;
+      const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int s2 = 0; s2 < kRing; ++s2) fetch(s2, tq[s2], wq[s2]);
-    for (int64_t it0 = 0; entry(it0) - grp < i1; it0 += kRing) {
-#pragma unroll
-      for (int s2 = 0; s2 < kRing; ++s2) {
-        const int64_t it = it0 + s2;
-        const int64_t i = entry(it);
-        const int t = tq[s2];
-        const uint4 w = wq[s2];
-        fetch(it + kRing, tq[s2], wq[s2]);
-        if (t < 0) continue;
-        const float pt = expf(logit_of(i, t) - m) * invz;
-        const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint32_t idx = word_idx(wd[u]);
-          if (idx >= (uint32_t)n) {
-            record_error(p.hdr, SDK_ERR_DEVICE_CHECK, idx);
-            continue;
-          }
-          const float v = pt * word_coef(wd[u]);
-          if (use_float) {
-            atomicAdd(&sfw[idx], v);
-          } else {
-            absum += fabsf(v);
-            atomicAdd(&siw[idx], __float2int_rn(v * kFixScale));
-          }
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t idx = word_idx(wd[u]);
+        maxidx = max(maxidx, idx);
+        const float v = pt * word_coef(wd[u]);
+        if constexpr (kFloat) {
+          atomicAdd(&table[idx], v);
+        } else {
+          absum += fabsf(v);
+          atomicAdd(&siw[idx], __float2int_rn(v * kFixScale));
         }
       }
-    }
-    if (!use_float) {
-      // exact int32 range guard (see above); also catches NaN
-      if (!(absum < 1024.0f)) s_float = 1;
-      __syncthreads();
-      if (s_float) continue;
-      break;
-    }
-  }
+    };
+    for_records(list, s0, s1, vrec, Nb, p.hdr, 0x31000000u | r,
+                [&](int i, int t, uint4 w) { scatter(t >= 0 ? ss[i] : 0.0f, t, w); });
+    if (p.full)
+      for_records(list, c0, c1, vrec, Nb, p.hdr, 0x32000000u | r,
+                  [&](int i, int t, uint4 w) {
+                    scatter(t >= 0 ? p.scale * key_score(keys[t]) : 0.0f, t, w);
+                  });
+    if (!kFloat && !(absum < 1024.0f)) s_float = 1;   // also catches NaN
+    __syncthreads();
+  };
+  phase3(std::false_type{});
+  if (s_float) phase3(std::true_type{});
+  if (maxidx >= (uint32_t)n) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, maxidx);
+
+  // ---- phase 4: sum the cluster's tiles over this CTA's slice of atoms
   cluster.sync();
-  // reduce this CTA's slice of the atoms over the C tiles of the cluster
-  const int a0 = (int)((int64_t)n * rank / C), a1 = (int)((int64_t)n * (rank + 1) / C);
+  // slices of 4-atom groups; all C tiles' words of a group are loaded
+  // before any is summed
+  const int ng = (n + 3) >> 2;
+  const int g0 = (int)((int64_t)ng * rank / C), g1 = (int)((int64_t)ng * (rank + 1) / C);
   float* gw = p.w + (int64_t)r * n;
-  for (int a = a0 + tid; a < a1; a += kRecThreads) {
-    float sum = 0.0f;
-    for (int cc = 0; cc < C; ++cc) {
-      const bool f = *cluster.map_shared_rank(&s_float, cc) != 0;
-      const int* tile = cluster.map_shared_rank(siw, cc);
-      sum += f ? __int_as_float(tile[a]) : (float)tile[a] * kFixInv;
+  const int4* tiles[8];
+  bool isf[8];
+#pragma unroll
+  for (int cc = 0; cc < 8; ++cc) {
+    if (cc < C) {
+      tiles[cc] = reinterpret_cast<const int4*>(cluster.map_shared_rank(siw, cc));
+      isf[cc] = *cluster.map_shared_rank(&s_float, cc) != 0;
     }
-    gw[a] = sum;
   }
-  if (rank == 0 && tid == 0) p.st[r].z = ztot;
+  for (int g = g0 + tid; g < g1; g += kAttThreads) {
+    int4 v[8];
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc)
+      if (cc < C) v[cc] = tiles[cc][g];
+    float sum[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+      if (cc >= C) break;
+      const int vv[4] = {v[cc].x, v[cc].y, v[cc].z, v[cc].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) sum[u] += isf[cc] ? __int_as_float(vv[u]) : (float)vv[u] * kFixInv;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (4 * g + u < n) gw[4 * g + u] = sum[u];
+  }
+  if (rank == 0 && tid == 0) st->z = ztot;
   cluster.sync();
 }
 
 // --------------------------------------------------------------- out_kernel
-// out[r][k] += sum_{a in tile} w[r][a] D_V[a][k] over a 128-atom tile and a
-// 32-row block.  The atom tile stays bf16 in shared memory ([atom][k]);
-// thread (tk, tr) owns columns tk*C.. and rows 4tr..4tr+3; results are
-// added with vector reductions into `out` (zeroed by qd_kernel).
+// out[r][c] += sum_a w[r][a] D_V[a][c] over `tpc` consecutive 64-atom tiles
+// and a 32-row block, D/32 warps per CTA.  Per tile the value rows are
+// staged as fp32 [a][D] (converted from bf16) and the weights as fp32
+// [a][32] (4-row groups XOR-swizzled by a).  Lane (tc, tr) of warp w owns
+// columns 32w + 4tc .. +3 and rows 8tr .. 8tr+7 (32 accumulators over all
+// the CTA's tiles): per atom, three 16-byte shared loads feed 32 FMAs.  The
+// partial sums are added into `out` (zeroed by qd_kernel) with one vector
+// reduction per row.
 template <int D>
-__global__ void __launch_bounds__(kQdThreads) out_kernel(DecodeParams p) {
-  __shared__ __align__(16) uint16_t Ds[128][D];   // atom tile, bf16
-  __shared__ __align__(16) float Ws[128][32];     // w tile, [atom][row]
+__global__ void __launch_bounds__(D) out_kernel(DecodeParams p, int tpc) {
+  __shared__ __align__(16) float Vs[kGvAtoms][D];
+  __shared__ __align__(16) float Ws[kGvAtoms][32];
+  constexpr int kThreads = D;
   const int n = p.n, R = p.R, tid = threadIdx.x;
-  const int a0 = blockIdx.x * 128, r0 = blockIdx.y * 32;
-  for (int e = tid; e < 128 * (D / 8); e += kQdThreads) {
-    const int a = e / (D / 8), c = e % (D / 8);
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (a0 + a < n) v = __ldg(reinterpret_cast<const uint4*>(p.dv + (int64_t)(a0 + a) * D) + c);
-    *reinterpret_cast<uint4*>(&Ds[a][c * 8]) = v;
-  }
-  for (int e = tid; e < 128 * 32; e += kQdThreads) {
-    const int r = e & 31, a = e >> 5;
-    Ws[a][r] = (r0 + r < R && a0 + a < n) ? p.w[(int64_t)(r0 + r) * n + a0 + a] : 0.0f;
-  }
-  __syncthreads();
-  constexpr int C = D / 32;
-  const int tk = tid & 31, tr = tid >> 5;
-  float acc[4][C];
+  const int r0 = blockIdx.y * 32;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int tc = lane & 7, tr = lane >> 3;
+  const int cc = warp * 32 + 4 * tc;
+  float acc[8][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int cc = 0; cc < C; ++cc) acc[i][cc] = 0.0f;
-#pragma unroll 8
-  for (int a = 0; a < 128; ++a) {
-    float dv[C];
-    if constexpr (C == 4) {
-      const uint2 v = *reinterpret_cast<const uint2*>(&Ds[a][tk * 4]);
-      dv[0] = bf16_lo(v.x); dv[1] = bf16_hi(v.x); dv[2] = bf16_lo(v.y); dv[3] = bf16_hi(v.y);
-    } else {
-      const uint32_t v = *reinterpret_cast<const uint32_t*>(&Ds[a][tk * 2]);
-      dv[0] = bf16_lo(v); dv[1] = bf16_hi(v);
+    for (int u = 0; u < 4; ++u) acc[i][u] = 0.0f;
+  for (int tile = 0; tile < tpc; ++tile) {
+    const int a0 = (blockIdx.x * tpc + tile) * kGvAtoms;
+    if (a0 >= n) break;
+    if (tile) __syncthreads();
+    constexpr int kChunk = 8;   // loads in flight per thread while staging
+#pragma unroll 1
+    for (int u0 = 0; u0 < kGvAtoms * (D / 8) / kThreads; u0 += kChunk) {
+      uint4 v[kChunk];
+#pragma unroll
+      for (int u = 0; u < kChunk; ++u) {
+        const int e = tid + (u0 + u) * kThreads;
+        const int c = e % (D / 8), a = e / (D / 8);
+        v[u] = (a0 + a < n) ? __ldg(reinterpret_cast<const uint4*>(p.dv + (int64_t)(a0 + a) * D) + c)
+                            : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kChunk; ++u) {
+        const int e = tid + (u0 + u) * kThreads;
+        const int c = e % (D / 8), a = e / (D / 8);
+        float4* dst = reinterpret_cast<float4*>(&Vs[a][c * 8]);
+        dst[0] = make_float4(bf16_lo(v[u].x), bf16_hi(v[u].x), bf16_lo(v[u].y), bf16_hi(v[u].y));
+        dst[1] = make_float4(bf16_lo(v[u].z), bf16_hi(v[u].z), bf16_lo(v[u].w), bf16_hi(v[u].w));
+      }
     }
-    const float4 wv = *reinterpret_cast<const float4*>(&Ws[a][4 * tr]);
-    const float wr[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll 1
+    for (int u0 = 0; u0 < kGvAtoms * 32 / kThreads; u0 += kChunk) {
+      float v[kChunk];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+      for (int u = 0; u < kChunk; ++u) {
+        const int e = tid + (u0 + u) * kThreads;
+        const int a = e % kGvAtoms, r = e / kGvAtoms;
+        v[u] = (r0 + r < R && a0 + a < n) ? __ldg(p.w + (int64_t)(r0 + r) * n + a0 + a) : 0.0f;
+      }
 #pragma unroll
-      for (int cc = 0; cc < C; ++cc) acc[i][cc] = fmaf(wr[i], dv[cc], acc[i][cc]);
+      for (int u = 0; u < kChunk; ++u) {
+        const int e = tid + (u0 + u) * kThreads;
+        const int a = e % kGvAtoms, r = e / kGvAtoms;
+        Ws[a][qswz(a, r)] = v[u];
+      }
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int a = 0; a < kGvAtoms; ++a) {
+      const float4 vv = *reinterpret_cast<const float4*>(&Vs[a][cc]);
+      const float4 wa = *reinterpret_cast<const float4*>(&Ws[a][((2 * tr) ^ (a & 7)) << 2]);
+      const float4 wb = *reinterpret_cast<const float4*>(&Ws[a][((2 * tr + 1) ^ (a & 7)) << 2]);
+      const float dv[4] = {vv.x, vv.y, vv.z, vv.w};
+      const float wr[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) acc[i][u] = fmaf(wr[i], dv[u], acc[i][u]);
+    }
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = r0 + 4 * tr + i;
+  for (int i = 0; i < 8; ++i) {
+    const int r = r0 + 8 * tr + i;
     if (r >= R) continue;
-    float* dst = p.out + (int64_t)r * D + tk * C;
-    if constexpr (C == 4) {
-      asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(acc[i][0]),
-                   "f"(acc[i][1]), "f"(acc[i][2]), "f"(acc[i][3])
-                   : "memory");
-    } else {
-      asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(dst), "f"(acc[i][0]),
-                   "f"(acc[i][1])
-                   : "memory");
-    }
+    float* dst = p.out + (int64_t)r * D + cc;
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(acc[i][0]),
+                 "f"(acc[i][1]), "f"(acc[i][2]), "f"(acc[i][3])
+                 : "memory");
   }
 }
 
@@ -865,45 +1075,41 @@ static int grid_for(int64_t work, int64_t per_cta, int cap_ctas) {
 
 sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
   const int sms = num_sms();
-  const size_t qd_smem = (size_t)((p.n + 3) & ~3) * 4;
   static bool attr = false;
   if (!attr) {
-    cudaFuncSetAttribute(klow_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    cudaFuncSetAttribute(rescore_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    cudaFuncSetAttribute(klow_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kTable * 4 + 4096 * 4);
     cudaFuncSetAttribute(final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    cudaFuncSetAttribute(value_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    cudaFuncSetAttribute(value_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+    cudaFuncSetAttribute(pass2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPass2Smem);
+    cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTable * 4);
     attr = true;
   }
   {
-    dim3 grid((p.n + 127) / 128, (p.R + 31) / 32);
+    dim3 grid((p.n + kGvAtoms - 1) / kGvAtoms, (p.R + 31) / 32);
     if (p.d == 128) qd_kernel<128><<<grid, kQdThreads, 0, stream>>>(p);
     else qd_kernel<64><<<grid, kQdThreads, 0, stream>>>(p);
   }
   {
     const int g = grid_for(p.tok_off[p.B], 2048, sms);
-    klow_kernel<<<g, kKlowThreads, qd_smem + 4096 * 4, stream>>>(p);
+    const int vec = (p.cap % 4 == 0) && ((reinterpret_cast<uintptr_t>(p.k_lo) & 15u) == 0u);
+    klow_kernel<<<g, kKlowThreads, (size_t)kTable * 4 + 4096 * 4, stream>>>(p, vec);
   }
   {
     const int g = grid_for(p.tok_off[p.B], 8192, 2 * sms);
-    pass2_kernel<<<g, kScanThreads, 0, stream>>>(p);
+    pass2_kernel<<<g, kScanThreads, kPass2Smem, stream>>>(p);
   }
   final_kernel<<<p.R, kScanThreads, (size_t)2 * kFinalStage * 4, stream>>>(p);
   {
-    int64_t per = p.sel_off[p.B] / sms;
-    if (per < 1024) per = 1024;
-    const int g = grid_for(p.sel_off[p.B], per, sms);
-    rescore_kernel<<<g, kRecThreads, qd_smem, stream>>>(p);
-  }
-  {
+    // one cluster of C CTAs per query head, C a power of two <= 8 while the
+    // clusters fit the SMs and every CTA keeps >= 1024 entries
     int64_t dmax = 0;
     for (int b = 0; b < p.B; ++b) dmax = p.dcnt[b] > dmax ? p.dcnt[b] : dmax;
     int C = 1;
     while (C < 8 && (int64_t)p.R * C * 2 <= sms && dmax / (2 * C) >= 1024) C *= 2;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(p.R * C));
-    cfg.blockDim = dim3(kRecThreads);
-    cfg.dynamicSmemBytes = qd_smem;
+    cfg.blockDim = dim3(kAttThreads);
+    cfg.dynamicSmemBytes = (size_t)kTable * 4;
     cfg.stream = stream;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
@@ -912,12 +1118,17 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
     at[0].val.clusterDim.z = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, value_kernel, p, C) != cudaSuccess) return SDK_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, attend_kernel, p, C) != cudaSuccess) return SDK_ERR_CUDA;
   }
   {
-    dim3 grid((p.n + 127) / 128, (p.R + 31) / 32);
-    if (p.d == 128) out_kernel<128><<<grid, kQdThreads, 0, stream>>>(p);
-    else out_kernel<64><<<grid, kQdThreads, 0, stream>>>(p);
+    // atom tiles per CTA: enough CTAs for ~4 per SM, fewer reductions
+    const int tiles = (p.n + kGvAtoms - 1) / kGvAtoms;
+    const int rb = (p.R + 31) / 32;
+    int tpc = 1;
+    while (tpc < 8 && (int64_t)((tiles + 2 * tpc - 1) / (2 * tpc)) * rb >= 4 * sms) tpc *= 2;
+    dim3 grid((tiles + tpc - 1) / tpc, rb);
+    if (p.d == 128) out_kernel<128><<<grid, 128, 0, stream>>>(p, tpc);
+    else out_kernel<64><<<grid, 64, 0, stream>>>(p, tpc);
   }
   return cudaGetLastError() == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
 }
