@@ -42,6 +42,8 @@ def enc_flop_per_vector(n_atoms, head_dim):
 # kernels of one tensor-core encode call: dictionary statistics, fp16
 # dictionary copy, encoder
 ENC_KERNELS_PER_CALL = 3
+# kernels of one decode layer: qd, klow, pass2, final, attend, out
+DEC_KERNELS_PER_LAYER = 6
 ENC_DTYPE = ("f32 (residuals and re-scoring; tensor-core operands fp16 with "
              "fp32 accumulation; bf16 dictionaries; fp16 coefficients)")
 
@@ -234,8 +236,9 @@ def union_bytes(sdk, ws_list, lay, B, Hq, Hkv, N, k, full):
     total = 0
     usum = 0
     for ws in ws_list:
-        lst = ws[lay["list"]:lay["list"] + B * Hq * N * 4].view(torch.int32)
-        lst = lst.view(B, Hkv, g, N)[..., :k].long()
+        row = lay["row"]                 # per-head stride of the list
+        lst = ws[lay["list"]:lay["list"] + B * Hq * row * 4].view(torch.int32)
+        lst = lst.view(B, Hkv, g, row)[..., :k].long()
         mark = torch.zeros(B, Hkv, N, dtype=torch.bool, device=lst.device)
         mark.scatter_(2, lst.reshape(B, Hkv, g * k), True)
         U = int(mark.sum())
@@ -320,9 +323,9 @@ def bench_layer4k(args, world, rank, pk):
                          "per-step events)"},
         "dtype": ENC_DTYPE,
         # kernels per step: append = 2 x (dictionary statistics + fp16
-        # dictionary copy + encode + scatter); decode = 7 (qd, klow, pass2,
-        # final, rescore, value, out)
-        "gpu_launches": args.steps * (2 * ENC_KERNELS_PER_CALL + 2 + 7),
+        # dictionary copy + encode + scatter); decode = DEC_KERNELS_PER_LAYER
+        "gpu_launches": args.steps * (2 * ENC_KERNELS_PER_CALL + 2 +
+                                      DEC_KERNELS_PER_LAYER),
         "enc_fallback_rows": hdr[2],
     }
     if not args.no_e2e:
@@ -427,7 +430,7 @@ def bench_decode(args, world, rank, pk, name):
                    "l2": "flushed between steps; codes (%.1f GB) exceed L2"
                          % (L * B * Hkv * N * 140 / 1e9)},
         "dtype": "f32 (bf16 dictionaries, fp16 coefficients)",
-        "gpu_launches": args.steps * L * 7,
+        "gpu_launches": args.steps * L * DEC_KERNELS_PER_LAYER,
     }
 
 

@@ -237,7 +237,8 @@ SDK_API sdk_status sdk_decode_attn_static(const float* q, int32_t B, int32_t Hq,
 
 /* Byte offsets of the decode workspace regions, for inspection by tests
  * and tools after a call (contents are valid until the next call using the
- * same workspace).  R = B*Hq query heads, L = max_len. */
+ * same workspace).  R = B*Hq query heads, L = `row` (max_len rounded up to
+ * a multiple of 4). */
 typedef struct {
   size_t header;     /* 256-byte status header                            */
   size_t qd;         /* float  [R][n_atoms]   QD = D_K q                  */
@@ -254,6 +255,9 @@ typedef struct {
   size_t w;          /* float  [R][n_atoms] unnormalised per-atom weights */
   size_t part;       /* float  partial sums of w D_V                      */
   size_t total;      /* total bytes                                       */
+  size_t row;        /* elements per head in keys, list, cand_t, cand_key
+                        and sel_score: max_len rounded up to a multiple of
+                        4 (16-byte aligned rows)                          */
 } sdk_decode_layout;
 
 /* Per-head selection state in the decode workspace (region `state`).

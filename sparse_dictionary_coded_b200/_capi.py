@@ -55,7 +55,7 @@ SIGNATURES = {
 class DecodeLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "header", "qd", "keys", "hist1", "hist2", "state", "list", "cand_t",
-        "cand_key", "sel_score", "w", "part", "total")]
+        "cand_key", "sel_score", "w", "part", "total", "row")]
 
 
 SELECT_STATE_FIELDS = ("kth_key", "k", "n_above", "n_cand", "n_sel", "n_comp",

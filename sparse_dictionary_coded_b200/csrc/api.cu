@@ -298,7 +298,7 @@ sdk_status sdk_decode_attn(const float* q, int32_t B, int32_t Hq, int32_t Hkv, i
   p.w = reinterpret_cast<float*>(ws + l.w);
   p.part = reinterpret_cast<float*>(ws + l.part);
   p.cap = cap;
-  p.L = max_len;
+  p.L = (int64_t)l.row;   // row stride of the per-token regions
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;

@@ -235,8 +235,10 @@ __global__ void __launch_bounds__(kQdThreads) qd_kernel(DecodeParams p) {
 // is reported once per thread after the scan), the three k_lo planes read
 // four tokens at a time (16-byte loads when the planes are 16-byte
 // aligned), one gather and one FMA per word.  Writes the order-preserving
-// key of every token and the 12-bit histogram of key bits 31..20 of every
-// head (shared-memory atomics, flushed once per segment).
+// key of every token (one 16-byte store per quad; four 4-byte stores per
+// quad cost as much as the rest of the scan) and the 12-bit histogram of
+// key bits 31..20 of every head (shared-memory atomics, flushed once per
+// segment).
 constexpr int kScanThreads = 512;
 constexpr int kKlowThreads = 1024;
 
@@ -333,6 +335,7 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
     for (; q < q1; q += kKlowThreads) {
       load_quad(q + kKlowThreads, wn);
       prefetch(q + 2 * kKlowThreads);
+      uint32_t kq[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int t = 4 * q + u;
@@ -349,10 +352,21 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
           maxidx = max(maxidx, idx);
           s = fmaf(word_coef(wj), table[idx], s);
         }
-        if (t >= t0 && t < t1) {
-          const uint32_t key = score_key(s);
-          keys[t] = key;
-          atomicAdd(&sh[key >> 20], 1u);
+        kq[u] = score_key(s);
+      }
+      // keys: one 16-byte store per whole quad (rows are 16-byte aligned)
+      if (4 * q >= t0 && 4 * q + 4 <= t1) {
+        *reinterpret_cast<uint4*>(keys + 4 * q) = make_uint4(kq[0], kq[1], kq[2], kq[3]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) atomicAdd(&sh[kq[u] >> 20], 1u);
+      } else if (q < q1) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int t = 4 * q + u;
+          if (t >= t0 && t < t1) {
+            keys[t] = kq[u];
+            atomicAdd(&sh[kq[u] >> 20], 1u);
+          }
         }
       }
 #pragma unroll
@@ -372,27 +386,40 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
 // ------------------------------------------------------------- pass2_kernel
 // Tokens above the bucket of the k-th key are selected, tokens inside it
 // become candidates (with a histogram of key bits 19..8), the others go to
-// the complement (full-softmax flag only).  A segment is taken in rounds of
-// kSelBuf tokens; each warp takes 128 tokens per step (4 coalesced key
-// loads per lane) and appends its selected tokens to a shared-memory buffer
-// (shared atomics), which is copied out once per round behind one global
-// atomic.  Candidates (and their histogram) are buffered the same way; the
-// complement path (full-softmax flag) writes to global memory directly.
-// Both run only when a ballot finds some.
-constexpr int kSelBuf = 8192;
+// the complement (full-softmax flag only).  A warp takes 512 tokens per
+// step: each lane takes 16 consecutive keys (four 16-byte copies streamed
+// through a per-lane shared-memory ring three steps ahead, about 6 KB per
+// warp in flight), counts its tokens of each kind, and a warp scan gives
+// every lane its output slots behind one atomic per warp and kind.  Candidates and their
+// histogram go through shared memory (flushed once per segment; slots past
+// the buffer go straight to global memory).  The few tokens before the
+// first 16-byte boundary of a segment and after its last one take a scalar
+// path.
 constexpr int kCandBuf = 2048;
-constexpr int kPass2Smem = (kSelBuf + 2 * kCandBuf + 4096) * 4;
+constexpr int kP2Stages = 4;                            // key ring depth per lane
+constexpr int kP2RingOff = 2 * kCandBuf + 4096;         // in words
+constexpr int kPass2Smem = (kP2RingOff + kP2Stages * (kScanThreads / 32) * 128 * 4) * 4;
 
-__global__ void __launch_bounds__(kScanThreads, 2) pass2_kernel(DecodeParams p) {
+__device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v, uint32_t& total) {
+  const int lane = threadIdx.x & 31;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  total = __shfl_sync(0xffffffffu, x, 31);
+  return x - v;
+}
+
+__global__ void __launch_bounds__(kScanThreads, 1) pass2_kernel(DecodeParams p) {
   __shared__ uint32_t s_tmp[48];
-  __shared__ uint32_t s_nsel, s_base, s_ncand, s_cbase;
+  __shared__ uint32_t s_ncand, s_cbase;
   extern __shared__ uint32_t s_dyn[];   // kPass2Smem bytes
-  int32_t* s_sel = reinterpret_cast<int32_t*>(s_dyn);
-  int32_t* s_ct = s_sel + kSelBuf;
+  int32_t* s_ct = reinterpret_cast<int32_t*>(s_dyn);
   uint32_t* s_ck = reinterpret_cast<uint32_t*>(s_ct + kCandBuf);
   uint32_t* s_h2 = s_ck + kCandBuf;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const unsigned lt = (1u << lane) - 1u;
   const int64_t total = p.tok_off[p.B];
   const int64_t G0 = total * blockIdx.x / gridDim.x;
   const int64_t G1 = total * (blockIdx.x + 1) / gridDim.x;
@@ -401,127 +428,227 @@ __global__ void __launch_bounds__(kScanThreads, 2) pass2_kernel(DecodeParams p) 
   for_segments(p.tok_off, p.lens, p.B, G0, G1, [&](int b, int h, int64_t t0l, int64_t t1l) {
     const int r = b * p.Hq + h;
     const int Nb = p.lens[b];
+    const int t0 = (int)t0l, t1 = (int)t1l;
     sdk_select_state* st = p.st + r;
     uint32_t b1, above1, cnt1;
     bool bad;
+    for (int i = tid; i < 4096; i += kScanThreads) s_h2[i] = 0u;
+    if (tid == 0) s_ncand = 0u;
     block_find_desc<4096>(p.hist1 + (int64_t)r * 4096, (uint32_t)p.kcnt[b], s_tmp, b1, above1,
-                          cnt1, bad);
+                          cnt1, bad);   // ends with a barrier
     if (bad) {
       if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x10000000u | r);
       return;
     }
-    if (t0l == 0 && tid == 0) st->n_above = above1;
+    if (t0 == 0 && tid == 0) st->n_above = above1;
+    const uint32_t kLo = b1 << 20, kHi = kLo | 0xFFFFFu;   // the k-th key's bucket
     const uint32_t* keys = p.keys + (int64_t)r * p.L;
     int32_t* list = p.list + (int64_t)r * p.L;
     int32_t* ct = p.cand_t + (int64_t)r * p.L;
     uint32_t* ck = p.cand_key + (int64_t)r * p.L;
-    uint32_t* h2 = p.hist2 + (int64_t)r * 4096;
     const bool full = p.full != 0;
     uint32_t cmax = 0u;
-    for (int i = tid; i < 4096; i += kScanThreads) s_h2[i] = 0u;
-    for (int rt0 = (int)t0l; rt0 < (int)t1l; rt0 += kSelBuf) {
-      const int t1 = min((int)t1l, rt0 + kSelBuf);
-      if (tid == 0) {
-        s_nsel = 0u;
-        s_ncand = 0u;
+
+    // one warp-wide step over up to 16 tokens per lane: tt(j) gives the
+    // token of key j of this lane, kk[j] its key (valid when ok(j))
+    auto step = [&](const uint32_t (&kk)[16], auto tt, auto ok) {
+      uint32_t ns = 0u, nc = 0u, no = 0u;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (!ok(j)) continue;
+        const uint32_t d1 = kk[j] >> 20;
+        ns += d1 > b1 ? 1u : 0u;
+        nc += d1 == b1 ? 1u : 0u;
+        no += d1 < b1 ? 1u : 0u;
       }
-      __syncthreads();
-      uint32_t kc[4], kn[4];
-      auto load = [&](int tb, uint32_t (&kk)[4]) {
+      uint32_t tot;
+      uint32_t pos = warp_excl_scan(ns, tot);
+      if (tot) {
+        uint32_t base = 0u;
+        if (lane == 0) base = atomicAdd(&st->n_sel, tot);
+        pos += __shfl_sync(0xffffffffu, base, 0);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int t = tb + lane + 32 * u;
-          kk[u] = t < t1 ? __ldcs(keys + t) : 0u;
-        }
-      };
-      int tb = rt0 + warp * 128;
-      if (tb < t1) load(tb, kc);
-      for (; tb < t1; tb += kWarps * 128) {
-        const int tnext = tb + kWarps * 128;
-        if (tnext < t1) load(tnext, kn);
-        unsigned ms[4];
-        uint32_t ns = 0u;
-        bool anyc = false, anyo = false;
+        for (int j = 0; j < 16; ++j)
+          if (ok(j) && (kk[j] >> 20) > b1) {
+            if (pos < (uint32_t)Nb) list[pos] = tt(j);
+            ++pos;
+          }
+      }
+      if (__any_sync(0xffffffffu, nc != 0u)) {
+        uint32_t cpos = warp_excl_scan(nc, tot);
+        uint32_t base = 0u;
+        if (lane == 0) base = atomicAdd(&s_ncand, tot);
+        cpos += __shfl_sync(0xffffffffu, base, 0);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const bool valid = tb + lane + 32 * u < t1;
-          const uint32_t d1 = kc[u] >> 20;
-          ms[u] = __ballot_sync(0xffffffffu, valid && d1 > b1);
-          ns += __popc(ms[u]);
-          anyc |= valid && d1 == b1;
-          anyo |= valid && d1 < b1;
-        }
-        uint32_t bs = 0u;
-        if (lane == 0 && ns) bs = atomicAdd(&s_nsel, ns);
-        bs = __shfl_sync(0xffffffffu, bs, 0);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if ((ms[u] >> lane) & 1u) s_sel[bs + __popc(ms[u] & lt)] = tb + lane + 32 * u;
-          bs += __popc(ms[u]);
-        }
-        if (__any_sync(0xffffffffu, anyc)) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const bool c = tb + lane + 32 * u < t1 && (kc[u] >> 20) == b1;
-            const unsigned mc = __ballot_sync(0xffffffffu, c);
-            if (mc == 0u) continue;
-            uint32_t bc = 0u;
-            if (lane == 0) bc = atomicAdd(&s_ncand, (uint32_t)__popc(mc));
-            bc = __shfl_sync(0xffffffffu, bc, 0) + __popc(mc & lt);
-            // slots past the buffer go straight to global memory
-            const bool spill = c && bc >= (uint32_t)kCandBuf;
-            const unsigned mspill = __ballot_sync(0xffffffffu, spill);
-            uint32_t bg = 0u;
-            if (mspill && lane == 0) bg = atomicAdd(&st->n_cand, (uint32_t)__popc(mspill));
-            bg = __shfl_sync(0xffffffffu, bg, 0) + __popc(mspill & lt);
-            if (c) {
-              const int t = tb + lane + 32 * u;
-              if (!spill) {
-                s_ct[bc] = t;
-                s_ck[bc] = kc[u];
-              } else if (bg < (uint32_t)Nb) {
-                ct[bg] = t;
-                ck[bg] = kc[u];
+        for (int j = 0; j < 16; ++j)
+          if (ok(j) && (kk[j] >> 20) == b1) {
+            if (cpos < (uint32_t)kCandBuf) {
+              s_ct[cpos] = tt(j);
+              s_ck[cpos] = kk[j];
+            } else {
+              const uint32_t g = atomicAdd(&st->n_cand, 1u);   // rare overflow
+              if (g < (uint32_t)Nb) {
+                ct[g] = tt(j);
+                ck[g] = kk[j];
               }
-              atomicAdd(&s_h2[(kc[u] >> 8) & 0xFFFu], 1u);
             }
+            atomicAdd(&s_h2[(kk[j] >> 8) & 0xFFFu], 1u);
+            ++cpos;
           }
-        }
-        if (full && __any_sync(0xffffffffu, anyo)) {
+      }
+      if (full && __any_sync(0xffffffffu, no != 0u)) {
+        uint32_t opos = warp_excl_scan(no, tot);
+        uint32_t base = 0u;
+        if (lane == 0) base = atomicAdd(&st->n_comp, tot);
+        opos += __shfl_sync(0xffffffffu, base, 0);
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const bool o = tb + lane + 32 * u < t1 && (kc[u] >> 20) < b1;
-            const unsigned mo = __ballot_sync(0xffffffffu, o);
-            if (mo == 0u) continue;
-            uint32_t bo = 0u;
-            if (lane == 0) bo = atomicAdd(&st->n_comp, (uint32_t)__popc(mo));
-            bo = __shfl_sync(0xffffffffu, bo, 0) + __popc(mo & lt);
-            if (o) {
-              if (bo < (uint32_t)Nb) list[Nb - 1 - (int)bo] = tb + lane + 32 * u;
-              cmax = max(cmax, kc[u]);
-            }
+        for (int j = 0; j < 16; ++j)
+          if (ok(j) && (kk[j] >> 20) < b1) {
+            if (opos < (uint32_t)Nb) list[Nb - 1 - (int)opos] = tt(j);
+            cmax = max(cmax, kk[j]);
+            ++opos;
           }
-        }
+      }
+    };
+
+    // scalar edges: tokens before the first 16-byte boundary and after the
+    // last one (at most 3 + 3), taken by warp 0
+    const int lead = (int)((4u - (uint32_t)((reinterpret_cast<uintptr_t>(keys + t0) >> 2) & 3u)) & 3u);
+    const int ta = min(t1, t0 + lead);
+    const int tb = ta + ((t1 - ta) & ~3);
+    if (warp == 0) {
+      uint32_t kk[16];
+      const int ne = (ta - t0) + (t1 - tb);
+      auto edge_t = [&](int j) { return j < ta - t0 ? t0 + j : tb + (j - (ta - t0)); };
 #pragma unroll
-        for (int u = 0; u < 4; ++u) kc[u] = kn[u];
+      for (int j = 0; j < 16; ++j) kk[j] = 0u;
+      if (lane == 0) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j < ne) kk[j] = keys[edge_t(j)];
       }
-      __syncthreads();
-      if (tid == 0) {
-        s_base = s_nsel ? atomicAdd(&st->n_sel, s_nsel) : 0u;
-        s_ncand = min(s_ncand, (uint32_t)kCandBuf);
-        s_cbase = s_ncand ? atomicAdd(&st->n_cand, s_ncand) : 0u;
-      }
-      __syncthreads();
-      const uint32_t nsel = s_nsel, base = s_base, ncand = s_ncand, cbase = s_cbase;
-      for (uint32_t i = tid; i < nsel; i += kScanThreads)
-        if (base + i < (uint32_t)Nb) list[base + i] = s_sel[i];
-      for (uint32_t i = tid; i < ncand; i += kScanThreads)
-        if (cbase + i < (uint32_t)Nb) {
-          ct[cbase + i] = s_ct[i];
-          ck[cbase + i] = s_ck[i];
-        }
-      __syncthreads();
+      step(kk, edge_t, [&](int j) { return lane == 0 && j < ne; });
     }
+    // body: whole quads [ta, tb) (keys + ta is 16-byte aligned), 512
+    // tokens per warp step; quad q holds tokens ta + 4q .. ta + 4q + 3.  Each
+    // lane streams its four quads per step through a kP2Stages-deep ring in
+    // shared memory (cp.async), so kP2Stages - 1 steps are in flight.
+    const int q1 = (tb - ta) >> 2;
+    const uint4* kq = reinterpret_cast<const uint4*>(keys + ta);
+    uint4* ring = reinterpret_cast<uint4*>(s_dyn + kP2RingOff) + warp * (kP2Stages * 128);
+    auto issue = [&](int qb, int slot) {
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int q = qb + lane + 32 * v;
+        cp_async16(ring + slot * 128 + 32 * v + lane, q < q1 ? kq + q : kq, q < q1);
+      }
+      cp_async_commit();
+    };
+    constexpr int kStride = kWarps * 128;
+    const int qfirst = warp * 128;
+    // selected tokens of the previous step, written once its slots are known
+    uint32_t pend_msel = 0u, pend_pos = 0u, pend_rsv = 0u;
+    int pend_qb = 0;
+    auto write_sel = [&]() {
+      const uint32_t base = __shfl_sync(0xffffffffu, pend_rsv, 0);
+      uint32_t pos = base + pend_pos;
+      for (uint32_t m = pend_msel; m; m &= m - 1u, ++pos) {
+        const int j = __ffs(m) - 1;
+        if (pos < (uint32_t)Nb) list[pos] = ta + 4 * (pend_qb + lane + 32 * (j >> 2)) + (j & 3);
+      }
+    };
+#pragma unroll
+    for (int s2 = 0; s2 < kP2Stages - 1; ++s2) issue(qfirst + s2 * kStride, s2);
+    int slot = 0;
+    for (int qb = qfirst; qb < q1; qb += kStride) {
+      issue(qb + (kP2Stages - 1) * kStride, (slot + kP2Stages - 1) % kP2Stages);
+      cp_async_wait<kP2Stages - 1>();
+      // classify the lane's 16 keys into bit masks (bit j = key j), then
+      // walk only the set bits
+      const uint4* rs = ring + slot * 128 + lane;
+      uint32_t msel = 0u, mcand = 0u, mval = 0u;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 x = rs[32 * v];
+        const uint32_t kv[4] = {x.x, x.y, x.z, x.w};
+        if (qb + lane + 32 * v < q1) mval |= 0xFu << (4 * v);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (kv[u] > kHi) msel |= 1u << (4 * v + u);
+          if (kv[u] >= kLo) mcand |= 1u << (4 * v + u);
+        }
+      }
+      msel &= mval;
+      mcand &= mval & ~msel;
+      auto tok = [&](int j) { return ta + 4 * (qb + lane + 32 * (j >> 2)) + (j & 3); };
+      auto key_at = [&](int j) {
+        const uint4 x = rs[32 * (j >> 2)];
+        const int u = j & 3;
+        return u == 0 ? x.x : u == 1 ? x.y : u == 2 ? x.z : x.w;
+      };
+      uint32_t tot;
+      // the slots of this step's selected tokens are reserved now and
+      // written one step later, so the atomic's round trip overlaps a step
+      const uint32_t pos = warp_excl_scan((uint32_t)__popc(msel), tot);
+      const uint32_t rsv = (lane == 0 && tot) ? atomicAdd(&st->n_sel, tot) : 0u;
+      write_sel();
+      pend_msel = msel;
+      pend_pos = pos;
+      pend_rsv = rsv;
+      pend_qb = qb;
+      if (__any_sync(0xffffffffu, mcand != 0u)) {
+        uint32_t cpos = warp_excl_scan((uint32_t)__popc(mcand), tot);
+        uint32_t base = 0u;
+        if (lane == 0) base = atomicAdd(&s_ncand, tot);
+        cpos += __shfl_sync(0xffffffffu, base, 0);
+        for (uint32_t m = mcand; m; m &= m - 1u, ++cpos) {
+          const int j = __ffs(m) - 1;
+          const uint32_t key = key_at(j);
+          if (cpos < (uint32_t)kCandBuf) {
+            s_ct[cpos] = tok(j);
+            s_ck[cpos] = key;
+          } else {
+            const uint32_t g = atomicAdd(&st->n_cand, 1u);   // rare overflow
+            if (g < (uint32_t)Nb) {
+              ct[g] = tok(j);
+              ck[g] = key;
+            }
+          }
+          atomicAdd(&s_h2[(key >> 8) & 0xFFFu], 1u);
+        }
+      }
+      if (full) {
+        const uint32_t mo = mval & ~msel & ~mcand;
+        uint32_t opos = warp_excl_scan((uint32_t)__popc(mo), tot);
+        if (tot) {
+          uint32_t base = 0u;
+          if (lane == 0) base = atomicAdd(&st->n_comp, tot);
+          opos += __shfl_sync(0xffffffffu, base, 0);
+          for (uint32_t m = mo; m; m &= m - 1u, ++opos) {
+            const int j = __ffs(m) - 1;
+            if (opos < (uint32_t)Nb) list[Nb - 1 - (int)opos] = tok(j);
+            cmax = max(cmax, key_at(j));
+          }
+        }
+      }
+      slot = slot + 1 == kP2Stages ? 0 : slot + 1;
+    }
+    write_sel();
+    cp_async_wait<0>();   // drain the copies issued past the end
+    __syncthreads();
+    // flush the candidates and the histogram of this segment
+    if (tid == 0) {
+      s_ncand = min(s_ncand, (uint32_t)kCandBuf);
+      s_cbase = s_ncand ? atomicAdd(&st->n_cand, s_ncand) : 0u;
+    }
+    __syncthreads();
+    const uint32_t ncand = s_ncand, cbase = s_cbase;
+    for (uint32_t i = tid; i < ncand; i += kScanThreads)
+      if (cbase + i < (uint32_t)Nb) {
+        ct[cbase + i] = s_ct[i];
+        ck[cbase + i] = s_ck[i];
+      }
+    uint32_t* h2 = p.hist2 + (int64_t)r * 4096;
     for (int i = tid; i < 4096; i += kScanThreads)
       if (s_h2[i]) atomicAdd(&h2[i], s_h2[i]);
     if (full) {
@@ -684,94 +811,89 @@ __global__ void __launch_bounds__(kScanThreads) final_kernel(DecodeParams p) {
 // cluster of C CTAs per head; CTA `rank` owns the slice
 // [k*rank/C, k*(rank+1)/C) of the head's selected entries list[0..k-1] and,
 // with the full-softmax flag, a slice of the complement entries
-// list[k..N-1] (logit scale * s_lo).
+// list[k..N-1] (logit scale * s_lo).  One thread per entry: it loads the
+// whole 64-byte record (four 16-byte loads) and walks its 16 words.
 //   phase 1  QD[r] is staged in a 32768-entry shared table (zero past n, so
-//            every 15-bit index reads inside it; an index >= n adds 0 and is
-//            reported after the loop).  s_i = scale * sum_{j<khigh} c_tj
-//            QD[idx_tj] for the own selected entries, four lanes per
-//            64-byte record, written to sel_score; the cluster's maximum m
-//            through distributed shared memory (with the flag, also the
-//            largest complement logit).
-//   phase 2  z = sum of exp(logit - m) over the head's domain, summed over
-//            the cluster.
-//   phase 3  the table becomes the per-atom weight tile: w[idx^V] += p c^V
+//            every 15-bit index reads inside it; with n < 32768 an index >= n
+//            adds 0 and is reported after the loop).  s_i = scale *
+//            sum_{j<khigh} c_tj QD[idx_tj] for the own selected entries,
+//            written to sel_score, with a running maximum and a running
+//            sum of exp(s - running max) per thread (online softmax).  The
+//            cluster's maximum m comes through distributed shared memory
+//            (with the flag, also the largest complement logit), then z.
+//   phase 2  the table becomes the per-atom weight tile: w[idx^V] += p c^V
 //            with p = exp(logit - m) / z, in 2^-20 fixed point (native int32
 //            shared-memory atomics: exact and order-independent).  Since
 //            sum p = 1, a bin can leave the int32 range only if the CTA's
 //            sum of |p c| reaches 2^10; a CTA that sees that re-runs the
 //            phase with fp32 atomics.
-//   phase 4  each CTA sums its slice of the atoms over the cluster's tiles
+//   phase 3  each CTA sums its slice of the atoms over the cluster's tiles
 //            and writes the normalised w[r].
-// Records are read in warp batches of 32 entries (one coalesced load of 32
-// list entries, then four records per 4-lane group); the next batch's
-// records are in flight while the current batch is used.
 constexpr int kAttThreads = 768;
+// shared memory: the QD / weight table, then a two-slot record ring
+constexpr int kAttSmem = kTable * 4 + 2 * kAttThreads * 64;
 constexpr float kFixScale = 1048576.0f;       // 2^20
 constexpr float kFixInv = 1.0f / 1048576.0f;
 
-// Calls f(i, t, w) for every entry i in [e0, e1) of `list`, from all 32
-// lanes of every warp; the 4-lane group (lane >> 2) of entry i holds its
-// record, lane c the words 4c..4c+3 in w.  t < 0 marks a padding slot or an
-// invalid token (reported).  Every lane calls f the same number of times.
+// Calls f(i, t, w) for every entry i in [e0, e1) of `list` owned by this
+// thread (i = e0 + tid + j*T); w holds the 16 words of token t's record.
+// Entries naming a token outside [0, Nb) are reported and skipped.  Records
+// stream through a two-slot ring per thread in shared memory (cp.async; the
+// four 16-byte chunks of a slot are XOR-swizzled by thread so the reads are
+// free of bank conflicts): entries i + T and i + 2T are in flight while i
+// is used, and the record of i + 3T is prefetched into L2.
 template <class F>
 __device__ __forceinline__ void for_records(const int32_t* list, int e0, int e1, const uint4* rec,
-                                            int Nb, WsHeader* hdr, uint32_t tag, F f) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int grp = lane >> 2, c = lane & 3;
-  constexpr int kStep = kAttThreads;          // entries per round of all warps
-  auto list_at = [&](int b) { return (b + lane < e1) ? __ldg(list + b + lane) : -1; };
-  auto fetch = [&](int b, int tl, int (&t)[4], uint4 (&w)[4]) {
+                                            int Nb, WsHeader* hdr, uint32_t tag, uint4* ring,
+                                            F f) {
+  constexpr int T = kAttThreads;
+  const int tid = threadIdx.x;
+  const int sw = (tid >> 1) & 3;
+  // raw list entries: nothing waits on these loads until they are used
+  // (two and four iterations later); out-of-range tokens are caught there
+  auto list_at = [&](int i) -> int { return i < e1 ? __ldg(list + i) : -1; };
+  auto ok = [&](int t) { return (unsigned)t < (unsigned)Nb; };
+  auto issue = [&](int t, int slot) {
+    const bool v = ok(t);
+    const uint4* a = rec + (int64_t)(v ? t : 0) * 4;
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      int tt = __shfl_sync(0xffffffffu, tl, s * 8 + grp);
-      const int i = b + s * 8 + grp;
-      if (i >= e1) {
-        tt = -1;
-      } else if ((unsigned)tt >= (unsigned)Nb) {
-        if (c == 0) record_error(hdr, SDK_ERR_DEVICE_CHECK, tag);
-        tt = -1;
-      }
-      t[s] = tt;
-      w[s] = tt >= 0 ? __ldcs(rec + (int64_t)tt * 4 + c) : make_uint4(0u, 0u, 0u, 0u);
-    }
+    for (int u = 0; u < 4; ++u) cp_async16(ring + (slot * T + tid) * 4 + (u ^ sw), a + u, v);
+    cp_async_commit();
   };
-  // the record of a list entry, two batches ahead, into L2 (64 bytes)
-  auto prefetch = [&](int tl) {
-    if ((unsigned)tl < (unsigned)Nb) {
-      const uint4* a = rec + (int64_t)tl * 4;
+  auto prefetch = [&](int t) {
+    if (ok(t)) {
+      const uint4* a = rec + (int64_t)t * 4;
       asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
       asm volatile("prefetch.global.L2 [%0];" ::"l"(a + 2));
     }
   };
-  int b = e0 + warp * 32;
-  if (b >= e1) return;
-  int tl1 = list_at(b + kStep);        // list entries of batch b + 1
-  int tl2 = list_at(b + 2 * kStep);    // and of batch b + 2
-  int tc[4];
-  uint4 wc[4];
-  fetch(b, list_at(b), tc, wc);
-  prefetch(tl1);
-  for (; b < e1; b += kStep) {
-    const int bn = b + kStep;
-    int tn[4];
-    uint4 wn[4];
-    const bool more = bn < e1;
-    if (more) {
-      fetch(bn, tl1, tn, wn);
-      prefetch(tl2);
-      tl1 = tl2;
-      tl2 = list_at(bn + 2 * kStep);
-    }
+  int i = e0 + tid;
+  if (i >= e1) return;
+  int t0 = list_at(i), t1 = list_at(i + T), t2 = list_at(i + 2 * T);
+  issue(t0, 0);
+  issue(t1, 1);
+  int t3 = list_at(i + 3 * T);
+  int slot = 0;
+  for (; i < e1; i += T) {
+    cp_async_wait<1>();               // the slot of entry i has landed
+    uint4 w[4];
 #pragma unroll
-    for (int s = 0; s < 4; ++s) f(b + s * 8 + grp, tc[s], wc[s]);
-    if (more) {
-#pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        tc[s] = tn[s];
-        wc[s] = wn[s];
-      }
-    }
+    for (int u = 0; u < 4; ++u) w[u] = ring[(slot * T + tid) * 4 + (u ^ sw)];
+    // the slot's words are in registers before the next copy may land in it
+    asm volatile("" ::"r"(w[0].x), "r"(w[0].y), "r"(w[0].z), "r"(w[0].w), "r"(w[1].x),
+                 "r"(w[1].y), "r"(w[1].z), "r"(w[1].w), "r"(w[2].x), "r"(w[2].y), "r"(w[2].z),
+                 "r"(w[2].w), "r"(w[3].x), "r"(w[3].y), "r"(w[3].z), "r"(w[3].w));
+    issue(t2, slot);                  // entry i + 2T into the freed slot
+    prefetch(t3);
+    if (ok(t0)) f(i, t0, w);
+    else record_error(hdr, SDK_ERR_DEVICE_CHECK, tag);
+    t0 = t1;
+    t1 = t2;
+    t2 = t3;
+    t3 = list_at(i + 4 * T);
+    slot ^= 1;
   }
+  cp_async_wait<0>();
 }
 
 // block-wide reduction of one float per thread into s_red[0] (max or sum)
@@ -787,20 +909,23 @@ __device__ __forceinline__ float block_reduce(float v, float* s_red) {
     if (lane == 0) s_red[32] = x;
   }
   __syncthreads();
-  return s_red[32];
+  const float r = s_red[32];
+  __syncthreads();   // s_red may be reused right away
+  return r;
 }
 
+template <bool kAll16, bool kCheck>
 __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, int C) {
   extern __shared__ float4 smem4[];
   float* table = reinterpret_cast<float*>(smem4);
   int* siw = reinterpret_cast<int*>(smem4);
+  uint4* ring = reinterpret_cast<uint4*>(smem4 + kTable / 4);   // 2 slots x T records
   __shared__ float s_red[33];
   __shared__ float s_val;
   __shared__ int s_float;
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   const int n = p.n, tid = threadIdx.x;
-  const int c = threadIdx.x & 3;
   const int r = blockIdx.x / C;
   const int rank = (int)cluster.block_rank();
   const int b = r / p.Hq, h = r % p.Hq, kvh = h / p.g;
@@ -817,48 +942,49 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
   float* ss = p.sel_score + (int64_t)r * p.L;
   const uint32_t* keys = p.keys + (int64_t)r * p.L;
   sdk_select_state* st = p.st + r;
+  const float scale = p.scale;
+  const int khigh = p.khigh;
   uint32_t maxidx = 0u;
 
   // ---- phase 1: stage QD[r], rescore the own selected entries
   stage_table(table, p.qd + (int64_t)r * n, n);
   __syncthreads();
-  const int jmax = min(p.khigh - 4 * c, 4);   // words of this lane that count
-  float smax = -INFINITY;
-  for_records(list, s0, s1, krec, Nb, p.hdr, 0x30000000u | r,
-              [&](int i, int t, uint4 w) {
-                const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
-                float part = 0.0f;
+  float smax = -INFINITY, zrun = 0.0f;     // online softmax of this thread
+  for_records(list, s0, s1, krec, Nb, p.hdr, 0x30000000u | r, ring,
+              [&](int i, int t, const uint4 (&w)[4]) {
+                float s = 0.0f;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                  if (u >= jmax) break;
-                  const uint32_t idx = word_idx(wd[u]);
-                  maxidx = max(maxidx, idx);
-                  part = fmaf(word_coef(wd[u]), table[idx], part);
+                for (int u = 0; u < 16; ++u) {
+                  if (!kAll16 && u >= khigh) break;
+                  const uint32_t wd = (u & 3) == 0 ? w[u >> 2].x : (u & 3) == 1 ? w[u >> 2].y
+                                    : (u & 3) == 2 ? w[u >> 2].z : w[u >> 2].w;
+                  const uint32_t idx = word_idx(wd);
+                  if (kCheck) maxidx = max(maxidx, idx);
+                  s = fmaf(word_coef(wd), table[idx], s);
                 }
-                part += __shfl_xor_sync(0xffffffffu, part, 1);
-                part += __shfl_xor_sync(0xffffffffu, part, 2);
-                if (t >= 0) {
-                  const float sc = part * p.scale;
-                  if (c == 0) ss[i] = sc;
-                  smax = fmaxf(smax, sc);
+                s *= scale;
+                ss[i] = s;
+                if (s > smax) {
+                  zrun = zrun * expf(smax - s) + 1.0f;
+                  smax = s;
+                } else {
+                  zrun += expf(s - smax);
                 }
               });
-  smax = block_reduce<true>(smax, s_red);
-  if (tid == 0) s_val = smax;
+  float m = block_reduce<true>(smax, s_red);
+  if (tid == 0) s_val = m;
   cluster.sync();
-  float m = -INFINITY;
+  m = -INFINITY;
   for (int cc = 0; cc < C; ++cc) m = fmaxf(m, *cluster.map_shared_rank(&s_val, cc));
   if (rank == 0 && tid == 0 && m > -INFINITY) st->max_score = score_key(m);
-  if (p.full && st->n_comp > 0u) m = fmaxf(m, p.scale * key_score(st->max_comp));
+  if (p.full && st->n_comp > 0u) m = fmaxf(m, scale * key_score(st->max_comp));
 
-  // ---- phase 2: z over the own slices of the domain
-  float z = 0.0f;
-#pragma unroll 4
-  for (int i = s0 + tid; i < s1; i += kAttThreads) z += expf(ss[i] - m);
+  // z: the own selected entries (rescaled to m) and complement entries
+  float z = smax > -INFINITY ? zrun * expf(smax - m) : 0.0f;
 #pragma unroll 4
   for (int i = c0 + tid; i < c1; i += kAttThreads) {
     const int t = list[i];
-    if (t >= 0 && t < Nb) z += expf(p.scale * key_score(keys[t]) - m);
+    if ((unsigned)t < (unsigned)Nb) z += expf(scale * key_score(keys[t]) - m);
   }
   z = block_reduce<false>(z, s_red);
   cluster.sync();   // every CTA has read s_val of phase 1
@@ -871,50 +997,53 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
   for (int cc = 0; cc < C; ++cc) ztot += *cluster.map_shared_rank(&s_val, cc);
   const float invz = 1.0f / ztot;
 
-  // ---- phase 3: scatter p c^V into the weight tile
-  auto phase3 = [&](auto fl) {
+  // ---- phase 2: scatter p c^V into the weight tile
+  auto phase2 = [&](auto fl) {
     constexpr bool kFloat = decltype(fl)::value;
     {
       uint4* t4 = reinterpret_cast<uint4*>(smem4);
       for (int i = tid; i < kTable / 4; i += kAttThreads) t4[i] = make_uint4(0u, 0u, 0u, 0u);
     }
     __syncthreads();
+    // fixed point: p already carries the 2^20 scale
+    const float pscale = kFloat ? invz : invz * kFixScale;
     float absum = 0.0f;
-    auto scatter = [&](float lg, int t, uint4 w) {
-      if (t < 0) return;
-      const float pt = expf(lg - m) * invz;
-      const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+    auto scatter = [&](float lg, const uint4 (&w)[4]) {
+      const float pt = expf(lg - m) * pscale;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const uint32_t idx = word_idx(wd[u]);
-        maxidx = max(maxidx, idx);
-        const float v = pt * word_coef(wd[u]);
+      for (int u = 0; u < 16; ++u) {
+        const uint32_t wd = (u & 3) == 0 ? w[u >> 2].x : (u & 3) == 1 ? w[u >> 2].y
+                          : (u & 3) == 2 ? w[u >> 2].z : w[u >> 2].w;
+        const uint32_t idx = word_idx(wd);
+        if (kCheck) maxidx = max(maxidx, idx);
+        const float v = pt * word_coef(wd);
         if constexpr (kFloat) {
           atomicAdd(&table[idx], v);
         } else {
           absum += fabsf(v);
-          atomicAdd(&siw[idx], __float2int_rn(v * kFixScale));
+          atomicAdd(&siw[idx], __float2int_rn(v));
         }
       }
     };
-    for_records(list, s0, s1, vrec, Nb, p.hdr, 0x31000000u | r,
-                [&](int i, int t, uint4 w) { scatter(t >= 0 ? ss[i] : 0.0f, t, w); });
+    for_records(list, s0, s1, vrec, Nb, p.hdr, 0x31000000u | r, ring,
+                [&](int i, int t, const uint4 (&w)[4]) { scatter(ss[i], w); });
     if (p.full)
-      for_records(list, c0, c1, vrec, Nb, p.hdr, 0x32000000u | r,
-                  [&](int i, int t, uint4 w) {
-                    scatter(t >= 0 ? p.scale * key_score(keys[t]) : 0.0f, t, w);
+      for_records(list, c0, c1, vrec, Nb, p.hdr, 0x32000000u | r, ring,
+                  [&](int i, int t, const uint4 (&w)[4]) {
+                    scatter(scale * key_score(keys[t]), w);
                   });
-    if (!kFloat && !(absum < 1024.0f)) s_float = 1;   // also catches NaN
+    // int32 range guard (also catches NaN): sum |p c| * 2^20 < 2^30
+    if (!kFloat && !(absum < 1073741824.0f)) s_float = 1;
     __syncthreads();
   };
-  phase3(std::false_type{});
-  if (s_float) phase3(std::true_type{});
-  if (maxidx >= (uint32_t)n) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, maxidx);
+  phase2(std::false_type{});
+  if (s_float) phase2(std::true_type{});
+  if (kCheck && maxidx >= (uint32_t)n) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, maxidx);
 
-  // ---- phase 4: sum the cluster's tiles over this CTA's slice of atoms
-  cluster.sync();
-  // slices of 4-atom groups; all C tiles' words of a group are loaded
+  // ---- phase 3: sum the cluster's tiles over this CTA's slice of atoms,
+  // in groups of 4 atoms; a group's loads from all C tiles are in flight
   // before any is summed
+  cluster.sync();
   const int ng = (n + 3) >> 2;
   const int g0 = (int)((int64_t)ng * rank / C), g1 = (int)((int64_t)ng * (rank + 1) / C);
   float* gw = p.w + (int64_t)r * n;
@@ -1050,6 +1179,8 @@ sdk_decode_layout decode_layout(int B, int Hq, int d, int n, int64_t L) {
     return o;
   };
   (void)d;
+  L = (L + 3) & ~(int64_t)3;   // 16-byte aligned rows
+  l.row = (size_t)L;
   l.header = take(sizeof(WsHeader));
   l.qd = take(R * n * 4);
   l.keys = take(R * L * 4);
@@ -1081,7 +1212,14 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
                          kTable * 4 + 4096 * 4);
     cudaFuncSetAttribute(final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     cudaFuncSetAttribute(pass2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPass2Smem);
-    cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTable * 4);
+    cudaFuncSetAttribute(attend_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kAttSmem);
+    cudaFuncSetAttribute(attend_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kAttSmem);
+    cudaFuncSetAttribute(attend_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kAttSmem);
+    cudaFuncSetAttribute(attend_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kAttSmem);
     attr = true;
   }
   {
@@ -1095,7 +1233,7 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
     klow_kernel<<<g, kKlowThreads, (size_t)kTable * 4 + 4096 * 4, stream>>>(p, vec);
   }
   {
-    const int g = grid_for(p.tok_off[p.B], 8192, 2 * sms);
+    const int g = grid_for(p.tok_off[p.B], 8192, sms);
     pass2_kernel<<<g, kScanThreads, kPass2Smem, stream>>>(p);
   }
   final_kernel<<<p.R, kScanThreads, (size_t)2 * kFinalStage * 4, stream>>>(p);
@@ -1109,7 +1247,7 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(p.R * C));
     cfg.blockDim = dim3(kAttThreads);
-    cfg.dynamicSmemBytes = (size_t)kTable * 4;
+    cfg.dynamicSmemBytes = kAttSmem;
     cfg.stream = stream;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
@@ -1118,7 +1256,10 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
     at[0].val.clusterDim.z = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, attend_kernel, p, C) != cudaSuccess) return SDK_ERR_CUDA;
+    const bool all16 = p.khigh == kAtoms, check = p.n < kTable;
+    auto kern = all16 ? (check ? attend_kernel<true, true> : attend_kernel<true, false>)
+                      : (check ? attend_kernel<false, true> : attend_kernel<false, false>);
+    if (cudaLaunchKernelEx(&cfg, kern, p, C) != cudaSuccess) return SDK_ERR_CUDA;
   }
   {
     // atom tiles per CTA: enough CTAs for ~4 per SM, fewer reductions

@@ -54,6 +54,10 @@ def test_workspace_sizes(lib):
     assert all(o % 256 == 0 for o in offs)
     assert lay["keys"] - lay["qd"] >= 32 * 32768 * 4
     assert lib.sdk_decode_workspace_bytes(1, 32, 128, 32768, 4096) == lay["total"]
+    # per-token regions: rows of max_len rounded up to a multiple of 4
+    assert lay["row"] == 4096
+    assert sdk.sdk_decode_layout_of(2, 8, 64, 1000, 4097)["row"] == 4100
+    assert lay["list"] - lay["state"] >= 0 and lay["cand_t"] - lay["list"] >= 32 * 4096 * 4
     assert lib.sdk_decode_workspace_bytes(0, 32, 128, 32768, 4096) == 0
     assert lib.sdk_decode_workspace_bytes(1, 32, 96, 32768, 4096) == 0
     assert lib.sdk_encode_workspace_bytes(1000, 128, 32768) >= 256

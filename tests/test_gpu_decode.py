@@ -42,14 +42,16 @@ def _run(q, DK, DV, store, **kw):
 
 
 def _gpu_sets(ws, lay, R, L, ks):
-    lst = ws[lay["list"]:lay["list"] + R * L * 4].view(torch.int32)
-    lst = lst.view(R, L).cpu().numpy()
+    row = lay["row"]                     # per-head stride (>= L, multiple of 4)
+    lst = ws[lay["list"]:lay["list"] + R * row * 4].view(torch.int32)
+    lst = lst.view(R, row).cpu().numpy()
     return [lst[r, :ks[r]] for r in range(R)]
 
 
 def _gpu_keys(ws, lay, R, L):
-    k = ws[lay["keys"]:lay["keys"] + R * L * 4].view(torch.int32)
-    return k.view(R, L).cpu().numpy().view(np.uint32)
+    row = lay["row"]
+    k = ws[lay["keys"]:lay["keys"] + R * row * 4].view(torch.int32)
+    return k.view(R, row)[:, :L].cpu().numpy().view(np.uint32)
 
 
 def _key_to_float(keys):
