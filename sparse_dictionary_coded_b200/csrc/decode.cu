@@ -14,9 +14,9 @@
 //                    above it are selected, tokens inside it become
 //                    candidates (compacted, with a second 12-bit histogram),
 //                    tokens below go to the complement.
-//   final_kernel     one CTA per head: last radix digit over the candidates,
-//                    the exact k-th key, tie handling by token index, and
-//                    the rest of the selected set.
+//   final_kernel     one CTA per head: last radix digits over the
+//                    candidates, the exact k-th key, tie handling by token
+//                    index, and the rest of the selected set.
 //   attend_kernel    s_t = scale * sum_{j<khigh} c_tj QD[idx_tj] for the
 //                    selected tokens (64-byte k_full records), p = softmax,
 //                    and the scatter w[idx^V_tj] += p_t c^V_tj into a
@@ -59,7 +59,7 @@ __device__ __forceinline__ void for_segments(const int64_t* off, const int* cnt,
 // the bin holding the k-th element (1-based), the count in higher bins and
 // the count in that bin.  s_tmp: >= 40 words of shared memory.  Sets
 // *bad when k is 0 or exceeds the histogram total.
-template <int NB>
+template <int NB, bool kL2 = false>   // kL2: hist is global memory written by other CTAs
 __device__ void block_find_desc(const uint32_t* hist, uint32_t k,
                                 uint32_t* s_tmp, uint32_t& bin,
                                 uint32_t& above, uint32_t& cnt, bool& bad) {
@@ -76,7 +76,7 @@ __device__ void block_find_desc(const uint32_t* hist, uint32_t k,
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
     const int rb = tid * PER + u;
-    c[u] = rb < NB ? hist[NB - 1 - rb] : 0u;
+    c[u] = rb < NB ? (kL2 ? __ldcg(hist + NB - 1 - rb) : hist[NB - 1 - rb]) : 0u;
     sum += c[u];
   }
   uint32_t tot;
@@ -106,28 +106,45 @@ __device__ void block_find_desc(const uint32_t* hist, uint32_t k,
 constexpr int kTable = 32768;   // shared QD / weight tables: every 15-bit index
 
 // ---------------------------------------------------------------- qd_kernel
-// QD[r][a] = sum_k q[r][k] D_K[a][k] on a 64-atom x 32-row tile per CTA of
-// two warps.  The atom tile is staged as bf16 [k][64] and the query rows as
-// fp32 [k][32] (groups of 4 rows XOR-swizzled by k, so the transposing
-// stores spread over the banks).  Lane (ta, tr) of warp w owns atoms
-// 32w + 4ta .. +3 and rows 8tr .. 8tr+7: per k, one 8-byte and two 16-byte
-// shared loads feed 32 FMAs (fp32, k order).  32 KB of shared memory.
+// QD[r][a] = sum_k q[r][k] D_K[a][k].  A CTA takes kGvTiles atom tiles of
+// kGvAtoms atoms and RB row blocks of 32 query rows (1 x 1 for up to 32
+// rows, 4 x 2 above); two warps per (tile, row block).  Every atom tile of the CTA is requested at once with
+// cp.async (bf16 [atom][D], the 16-byte chunks of atom a XOR-swizzled by
+// a & 7), so the CTA's whole share of the dictionary is in flight before the
+// first FMA; the query rows are staged fp32 [k][32] (4-row groups
+// XOR-swizzled by k).  Lane (ta, tr) of warp w of a pair owns atoms
+// 32w + ta + 8x (x = 0..3) and rows 8tr .. 8tr+7: per 8 values of k, four
+// 16-byte atom loads (conflict-free through the swizzle) and sixteen
+// broadcast row loads feed 256 FMAs (fp32, k order).
 // The first kernel of a call also zeroes the per-head selection state, both
 // histograms and `out` (accumulated with reductions by out_kernel).
 constexpr int kGvAtoms = 64;
-constexpr int kQdThreads = 64;
 
 __device__ __forceinline__ int qswz(int k, int r) { return (((r >> 2) ^ (k & 7)) << 2) | (r & 3); }
 
-template <int D>
-__global__ void __launch_bounds__(kQdThreads) qd_kernel(DecodeParams p) {
-  __shared__ __align__(16) uint16_t Ds[D][kGvAtoms];
-  __shared__ __align__(16) float Qs[D][32];
+constexpr int qd_smem_bytes(int d, int rb, int tiles) { return tiles * kGvAtoms * d * 2 + rb * d * 32 * 4; }
+
+template <int D, int RB, int kGvTiles>
+__global__ void __launch_bounds__(64 * kGvTiles * RB, (RB > 1 ? 2 : 1)) qd_kernel(DecodeParams p) {
+  constexpr int kThreads = 64 * kGvTiles * RB;
+  constexpr int kChunks = D / 8;                  // 16-byte chunks per atom row
+  extern __shared__ uint4 qd_smem[];
+  uint4* Dt = qd_smem;                            // [tile][atom][chunk]
+  float* Qs = reinterpret_cast<float*>(qd_smem + kGvTiles * kGvAtoms * kChunks);  // [rb][k][32]
   const int n = p.n, R = p.R, tid = threadIdx.x;
-  const int a0 = blockIdx.x * kGvAtoms, r0 = blockIdx.y * 32;
+  const int a0 = blockIdx.x * (kGvTiles * kGvAtoms);
+  const int r0 = blockIdx.y * (32 * RB);
+  // dictionary tiles: every chunk of the CTA in flight at once
+  for (int e = tid; e < kGvTiles * kGvAtoms * kChunks; e += kThreads) {
+    const int a = e / kChunks, c = e % kChunks;   // a: atom within the CTA
+    const bool v = a0 + a < n;
+    const uint4* src = reinterpret_cast<const uint4*>(p.dk + (int64_t)(v ? a0 + a : 0) * D) + c;
+    cp_async16(Dt + a * kChunks + (c ^ (a & 7)), src, v);
+  }
+  cp_async_commit();
   {
-    const int64_t nthr = (int64_t)gridDim.x * gridDim.y * kQdThreads;
-    const int64_t g0 = ((int64_t)blockIdx.y * gridDim.x + blockIdx.x) * kQdThreads + tid;
+    const int64_t nthr = (int64_t)gridDim.x * gridDim.y * kThreads;
+    const int64_t g0 = ((int64_t)blockIdx.y * gridDim.x + blockIdx.x) * kThreads + tid;
     const int64_t hwords = (int64_t)R * 4096;
     for (int64_t e = g0; e < hwords; e += nthr) {
       p.hist1[e] = 0u;
@@ -148,84 +165,78 @@ __global__ void __launch_bounds__(kQdThreads) qd_kernel(DecodeParams p) {
       p.st[e] = st;
     }
   }
-  // atom tile: lanes take consecutive atoms; all loads of a thread are in
-  // flight before its first store
-  constexpr int kChunk = 8;   // loads in flight per thread while staging
-#pragma unroll 1
-  for (int u0 = 0; u0 < kGvAtoms * (D / 8) / kQdThreads; u0 += kChunk) {
-    uint4 v[kChunk];
+  // query rows (16-byte loads along k, all of a thread's loads in flight
+  // before its first store)
+  constexpr int kQ4 = RB * 32 * (D / 4);
+  constexpr int kQPer = (kQ4 + kThreads - 1) / kThreads;
+  for (int e0 = tid; e0 < kQ4; e0 += kQPer * kThreads) {
+    float4 v[kQPer];
 #pragma unroll
-    for (int u = 0; u < kChunk; ++u) {
-      const int e = tid + (u0 + u) * kQdThreads;
-      const int a = e % kGvAtoms, c = e / kGvAtoms;
-      v[u] = (a0 + a < n) ? __ldg(reinterpret_cast<const uint4*>(p.dk + (int64_t)(a0 + a) * D) + c)
-                          : make_uint4(0u, 0u, 0u, 0u);
+    for (int u = 0; u < kQPer; ++u) {
+      const int e = e0 + u * kThreads;
+      const int k4 = e % (D / 4), rr = e / (D / 4);
+      v[u] = (e < kQ4 && r0 + rr < R)
+                 ? __ldg(reinterpret_cast<const float4*>(p.q + (int64_t)(r0 + rr) * D) + k4)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int u = 0; u < kChunk; ++u) {
-      const int e = tid + (u0 + u) * kQdThreads;
-      const int a = e % kGvAtoms, c = e / kGvAtoms;
-      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        Ds[c * 8 + 2 * x][a] = (uint16_t)(w[x] & 0xFFFFu);
-        Ds[c * 8 + 2 * x + 1][a] = (uint16_t)(w[x] >> 16);
-      }
-    }
-  }
-  // query rows: 16-byte loads along k
-#pragma unroll 1
-  for (int u0 = 0; u0 < 32 * (D / 4) / kQdThreads; u0 += kChunk) {
-    float4 v[kChunk];
-#pragma unroll
-    for (int u = 0; u < kChunk; ++u) {
-      const int e = tid + (u0 + u) * kQdThreads;
-      const int k4 = e % (D / 4), r = e / (D / 4);
-      v[u] = (r0 + r < R) ? __ldg(reinterpret_cast<const float4*>(p.q + (int64_t)(r0 + r) * D) + k4)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < kChunk; ++u) {
-      const int e = tid + (u0 + u) * kQdThreads;
-      const int k4 = e % (D / 4), r = e / (D / 4);
+    for (int u = 0; u < kQPer; ++u) {
+      const int e = e0 + u * kThreads;
+      if (e >= kQ4) break;
+      const int k4 = e % (D / 4), rr = e / (D / 4);
+      const int rb = rr >> 5, r = rr & 31;
+      float* qb = Qs + rb * D * 32;
       const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
-      for (int j = 0; j < 4; ++j) Qs[4 * k4 + j][qswz(4 * k4 + j, r)] = x[j];
+      for (int j = 0; j < 4; ++j) qb[(4 * k4 + j) * 32 + qswz(4 * k4 + j, r)] = x[j];
     }
   }
+  cp_async_wait<0>();
   __syncthreads();
   const int lane = tid & 31, warp = tid >> 5;
+  const int pair = warp >> 1, wp = warp & 1;
+  const int tile = pair % kGvTiles, rb = pair / kGvTiles;
   const int ta = lane & 7, tr = lane >> 3;
-  const int ac = warp * 32 + 4 * ta;          // first atom column of the thread
+  const uint4* Dtile = Dt + tile * kGvAtoms * kChunks;
+  const float* Qb = Qs + rb * D * 32;
   float acc[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int u = 0; u < 4; ++u) acc[i][u] = 0.0f;
-#pragma unroll 4
-  for (int k = 0; k < D; ++k) {
-    const uint2 dv = *reinterpret_cast<const uint2*>(&Ds[k][ac]);
-    const float4 qa = *reinterpret_cast<const float4*>(&Qs[k][((2 * tr) ^ (k & 7)) << 2]);
-    const float4 qb = *reinterpret_cast<const float4*>(&Qs[k][((2 * tr + 1) ^ (k & 7)) << 2]);
-    const float dd[4] = {bf16_lo(dv.x), bf16_hi(dv.x), bf16_lo(dv.y), bf16_hi(dv.y)};
-    const float qq[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+    for (int x = 0; x < 4; ++x) acc[i][x] = 0.0f;
+#pragma unroll 1
+  for (int kc = 0; kc < kChunks; ++kc) {
+    uint4 dv[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int x = 0; x < 4; ++x) {
+      const int a = 32 * wp + ta + 8 * x;
+      dv[x] = Dtile[a * kChunks + (kc ^ (a & 7))];
+    }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) acc[i][u] = fmaf(qq[i], dd[u], acc[i][u]);
+    for (int kk = 0; kk < 8; ++kk) {
+      const float* qk = Qb + (8 * kc + kk) * 32;
+      const float4 qa = *reinterpret_cast<const float4*>(qk + (((2 * tr) ^ kk) << 2));
+      const float4 qb = *reinterpret_cast<const float4*>(qk + (((2 * tr + 1) ^ kk) << 2));
+      const float qq[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const uint32_t wv = (kk >> 1) == 0 ? dv[x].x : (kk >> 1) == 1 ? dv[x].y
+                          : (kk >> 1) == 2 ? dv[x].z : dv[x].w;
+        const float d = (kk & 1) ? bf16_hi(wv) : bf16_lo(wv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i][x] = fmaf(qq[i], d, acc[i][x]);
+      }
+    }
   }
+  const int abase = a0 + tile * kGvAtoms + 32 * wp + ta;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int r = r0 + 8 * tr + i;
+    const int r = r0 + rb * 32 + 8 * tr + i;
     if (r >= R) continue;
-    float* dst = p.qd + (int64_t)r * n + a0 + ac;
-    if (a0 + ac + 3 < n && (n & 3) == 0) {
-      *reinterpret_cast<float4*>(dst) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-    } else {
+    float* dst = p.qd + (int64_t)r * n;
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (a0 + ac + u < n) dst[u] = acc[i][u];
-    }
+    for (int x = 0; x < 4; ++x)
+      if (abase + 8 * x < n) dst[abase + 8 * x] = acc[i][x];
   }
 }
 
@@ -381,6 +392,175 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
     __syncthreads();
   });
   if (maxidx >= (uint32_t)n) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, maxidx);
+}
+
+// ------------------------------------------------------- final selection
+constexpr int kFinalStage = 12288;   // candidates staged in shared memory
+// The last two radix digits of one query head over its candidates, the
+// exact k-th key, the tie rule (lower token index first) and the rest of the
+// selected set (inputs written by pass2_kernel, read through L2).
+// s_cand: 2 * kFinalStage words of shared memory; sh: 2048 words.
+__device__ void final_head(const DecodeParams& p, int r, uint32_t* s_cand, uint32_t* s_tmp,
+                           uint32_t* sh, uint32_t* s_cnt) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned lt = (1u << lane) - 1u;
+  const int b = r / p.Hq;
+  const int Nb = p.lens[b];
+  const uint32_t k = (uint32_t)p.kcnt[b];
+  sdk_select_state* st = p.st + r;
+  const uint32_t n_cand = __ldcg(&st->n_cand);
+  const uint32_t n_above = __ldcg(&st->n_above);
+  if (__ldcg(&st->n_sel) != n_above || n_above >= k || n_cand == 0u || n_cand > (uint32_t)Nb) {
+    if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x20000000u | r);
+    return;
+  }
+  const uint32_t* ck = p.cand_key + (int64_t)r * p.L;
+  const int32_t* ct = p.cand_t + (int64_t)r * p.L;
+  int32_t* list = p.list + (int64_t)r * p.L;
+  const uint32_t k1 = k - n_above;
+  // candidates in shared memory when they fit (one coalesced pass over the
+  // global copy; the passes below then read shared memory).  Otherwise the
+  // passes read global memory that no CTA of this SM has loaded before.
+  if (n_cand <= (uint32_t)kFinalStage) {
+    // eight loads of each array in flight per thread before any store
+    for (uint32_t i0 = tid; i0 < n_cand; i0 += 8 * kScanThreads) {
+      uint32_t kv[8], tv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t i = i0 + u * kScanThreads;
+        kv[u] = i < n_cand ? __ldcg(ck + i) : 0u;
+        tv[u] = i < n_cand ? (uint32_t)__ldcg(ct + i) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t i = i0 + u * kScanThreads;
+        if (i < n_cand) {
+          s_cand[i] = kv[u];
+          s_cand[kFinalStage + i] = tv[u];
+        }
+      }
+    }
+    __syncthreads();
+    ck = s_cand;
+    ct = reinterpret_cast<const int32_t*>(s_cand + kFinalStage);
+  }
+
+  uint32_t b2, above2, cnt2, b3, above3, cnt3;
+  bool bad;
+  block_find_desc<4096, true>(p.hist2 + (int64_t)r * 4096, k1, s_tmp, b2, above2, cnt2, bad);
+  if (bad) {
+    if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x21000000u | r);
+    return;
+  }
+  const uint32_t k2 = k1 - above2;
+  for (int i = tid; i < 256; i += kScanThreads) sh[i] = 0u;
+  __syncthreads();
+  for (uint32_t i = tid; i < n_cand; i += kScanThreads) {
+    const uint32_t key = ck[i];
+    if (((key >> 8) & 0xFFFu) == b2) atomicAdd(&sh[key & 0xFFu], 1u);
+  }
+  __syncthreads();
+  block_find_desc<256>(sh, k2, s_tmp, b3, above3, cnt3, bad);
+  if (bad) {
+    if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x22000000u | r);
+    return;
+  }
+  const uint32_t b1 = ck[0] >> 20;
+  const uint32_t T = (b1 << 20) | (b2 << 8) | b3;
+  const uint32_t eq_take = k2 - above3;
+  const uint32_t eq_total = cnt3;
+
+  // more ties than places: the eq_take-th smallest token index among the
+  // ties, by radix select over index digits 31..21, 20..10, 9..0 (bins kept
+  // in reverse so the descending search walks ascending indices)
+  uint32_t t_cut = 0xFFFFFFFFu;
+  if (eq_total > eq_take) {
+    uint32_t prefix = 0u, rank = eq_take;
+    for (int ps = 0; ps < 3; ++ps) {
+      const int sh_lo = ps == 0 ? 21 : (ps == 1 ? 10 : 0);
+      const int wbits = ps == 2 ? 10 : 11;
+      const uint32_t nb = 1u << wbits;
+      for (int i = tid; i < 2048; i += kScanThreads) sh[i] = 0u;
+      __syncthreads();
+      for (uint32_t i = tid; i < n_cand; i += kScanThreads) {
+        if (ck[i] != T) continue;
+        const uint32_t t = (uint32_t)ct[i];
+        const uint32_t hi = (ps == 0) ? 0u : (t >> (sh_lo + wbits));
+        if (hi != prefix) continue;
+        atomicAdd(&sh[2047u - ((t >> sh_lo) & (nb - 1u))], 1u);
+      }
+      __syncthreads();
+      uint32_t bin, above, cnt;
+      block_find_desc<2048>(sh, rank, s_tmp, bin, above, cnt, bad);
+      if (bad) {
+        if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x23000000u | r);
+        return;
+      }
+      prefix = (prefix << wbits) | (2047u - bin);
+      rank -= above;
+    }
+    t_cut = prefix;
+  }
+
+  if (tid == 0) {
+    s_cnt[0] = n_above;
+    s_cnt[1] = __ldcg(&st->n_comp);
+  }
+  __syncthreads();
+  uint32_t cmax = 0u;
+  for (uint32_t i0 = (uint32_t)warp * 32; i0 < n_cand; i0 += kScanThreads) {
+    const uint32_t i = i0 + lane;
+    uint32_t key = 0u, t = 0u;
+    bool sel = false, comp = false;
+    if (i < n_cand) {
+      key = ck[i];
+      t = (uint32_t)ct[i];
+      sel = key > T || (key == T && t <= t_cut);
+      comp = !sel && p.full;
+    }
+    const unsigned msel = __ballot_sync(0xffffffffu, sel);
+    const unsigned mcomp = __ballot_sync(0xffffffffu, comp);
+    uint32_t bs = 0, bo = 0;
+    if (lane == 0) {
+      if (msel) bs = atomicAdd(&s_cnt[0], (uint32_t)__popc(msel));
+      if (mcomp) bo = atomicAdd(&s_cnt[1], (uint32_t)__popc(mcomp));
+    }
+    bs = __shfl_sync(0xffffffffu, bs, 0) + __popc(msel & lt);
+    bo = __shfl_sync(0xffffffffu, bo, 0) + __popc(mcomp & lt);
+    if (sel) {
+      if (bs < k) list[bs] = (int32_t)t;
+      else record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x26000000u | r);
+    }
+    if (comp) {
+      if (bo < (uint32_t)Nb) list[Nb - 1 - (int64_t)bo] = (int32_t)t;
+      else record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x27000000u | r);
+      cmax = max(cmax, key);
+    }
+  }
+  if (p.full) {
+    cmax = warp_umax(cmax);
+    if (lane == 0 && cmax) atomicMax(&st->max_comp, cmax);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    st->kth_key = T;
+    st->eq_total = eq_total;
+    st->eq_taken = eq_take;
+    st->n_sel = s_cnt[0];
+    st->n_comp = s_cnt[1];
+    if (s_cnt[0] != k) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x24000000u | r);
+    if (p.full && s_cnt[0] + s_cnt[1] != (uint32_t)Nb)
+      record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x25000000u | r);
+  }
+}
+
+// One CTA per query head runs the final selection.
+__global__ void __launch_bounds__(kScanThreads) final_kernel(DecodeParams p) {
+  __shared__ uint32_t s_tmp[48];
+  __shared__ uint32_t sh[2048];
+  __shared__ uint32_t s_cnt[2];
+  extern __shared__ uint32_t s_cand[];   // 2 * kFinalStage words
+  final_head(p, blockIdx.x, s_cand, s_tmp, sh, s_cnt);
 }
 
 // ------------------------------------------------------------- pass2_kernel
@@ -659,153 +839,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) pass2_kernel(DecodeParams p) 
   });
 }
 
-// ------------------------------------------------------------- final_kernel
-constexpr int kFinalStage = 12288;   // candidates staged in shared memory
-// One CTA per query head: the last two radix digits over the candidates, the
-// exact k-th key, the tie rule (lower token index first) and the rest of the
-// selected set.
-__global__ void __launch_bounds__(kScanThreads) final_kernel(DecodeParams p) {
-  __shared__ uint32_t s_tmp[48];
-  __shared__ uint32_t sh[2048];
-  __shared__ uint32_t s_cnt[2];
-  const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const unsigned lt = (1u << lane) - 1u;
-  const int b = r / p.Hq;
-  const int Nb = p.lens[b];
-  const uint32_t k = (uint32_t)p.kcnt[b];
-  sdk_select_state* st = p.st + r;
-  const uint32_t n_cand = st->n_cand;
-  const uint32_t n_above = st->n_above;
-  if (st->n_sel != n_above || n_above >= k || n_cand == 0u || n_cand > (uint32_t)Nb) {
-    if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x20000000u | r);
-    return;
-  }
-  const uint32_t* ck = p.cand_key + (int64_t)r * p.L;
-  const int32_t* ct = p.cand_t + (int64_t)r * p.L;
-  int32_t* list = p.list + (int64_t)r * p.L;
-  const uint32_t k1 = k - n_above;
-  // candidates in shared memory when they fit (one coalesced pass over the
-  // global copy; the passes below then read shared memory)
-  extern __shared__ uint32_t s_cand[];
-  if (n_cand <= (uint32_t)kFinalStage) {
-    for (uint32_t i = tid; i < n_cand; i += kScanThreads) {
-      s_cand[i] = ck[i];
-      s_cand[kFinalStage + i] = (uint32_t)ct[i];
-    }
-    __syncthreads();
-    ck = s_cand;
-    ct = reinterpret_cast<const int32_t*>(s_cand + kFinalStage);
-  }
-
-  uint32_t b2, above2, cnt2, b3, above3, cnt3;
-  bool bad;
-  block_find_desc<4096>(p.hist2 + (int64_t)r * 4096, k1, s_tmp, b2, above2, cnt2, bad);
-  if (bad) {
-    if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x21000000u | r);
-    return;
-  }
-  const uint32_t k2 = k1 - above2;
-  for (int i = tid; i < 256; i += kScanThreads) sh[i] = 0u;
-  __syncthreads();
-  for (uint32_t i = tid; i < n_cand; i += kScanThreads) {
-    const uint32_t key = ck[i];
-    if (((key >> 8) & 0xFFFu) == b2) atomicAdd(&sh[key & 0xFFu], 1u);
-  }
-  __syncthreads();
-  block_find_desc<256>(sh, k2, s_tmp, b3, above3, cnt3, bad);
-  if (bad) {
-    if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x22000000u | r);
-    return;
-  }
-  const uint32_t b1 = ck[0] >> 20;
-  const uint32_t T = (b1 << 20) | (b2 << 8) | b3;
-  const uint32_t eq_take = k2 - above3;
-  const uint32_t eq_total = cnt3;
-
-  // more ties than places: the eq_take-th smallest token index among the
-  // ties, by radix select over index digits 31..21, 20..10, 9..0 (bins kept
-  // in reverse so the descending search walks ascending indices)
-  uint32_t t_cut = 0xFFFFFFFFu;
-  if (eq_total > eq_take) {
-    uint32_t prefix = 0u, rank = eq_take;
-    for (int ps = 0; ps < 3; ++ps) {
-      const int sh_lo = ps == 0 ? 21 : (ps == 1 ? 10 : 0);
-      const int wbits = ps == 2 ? 10 : 11;
-      const uint32_t nb = 1u << wbits;
-      for (int i = tid; i < 2048; i += kScanThreads) sh[i] = 0u;
-      __syncthreads();
-      for (uint32_t i = tid; i < n_cand; i += kScanThreads) {
-        if (ck[i] != T) continue;
-        const uint32_t t = (uint32_t)ct[i];
-        const uint32_t hi = (ps == 0) ? 0u : (t >> (sh_lo + wbits));
-        if (hi != prefix) continue;
-        atomicAdd(&sh[2047u - ((t >> sh_lo) & (nb - 1u))], 1u);
-      }
-      __syncthreads();
-      uint32_t bin, above, cnt;
-      block_find_desc<2048>(sh, rank, s_tmp, bin, above, cnt, bad);
-      if (bad) {
-        if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x23000000u | r);
-        return;
-      }
-      prefix = (prefix << wbits) | (2047u - bin);
-      rank -= above;
-    }
-    t_cut = prefix;
-  }
-
-  if (tid == 0) {
-    s_cnt[0] = n_above;
-    s_cnt[1] = st->n_comp;
-  }
-  __syncthreads();
-  uint32_t cmax = 0u;
-  for (uint32_t i0 = (uint32_t)warp * 32; i0 < n_cand; i0 += kScanThreads) {
-    const uint32_t i = i0 + lane;
-    uint32_t key = 0u, t = 0u;
-    bool sel = false, comp = false;
-    if (i < n_cand) {
-      key = ck[i];
-      t = (uint32_t)ct[i];
-      sel = key > T || (key == T && t <= t_cut);
-      comp = !sel && p.full;
-    }
-    const unsigned msel = __ballot_sync(0xffffffffu, sel);
-    const unsigned mcomp = __ballot_sync(0xffffffffu, comp);
-    uint32_t bs = 0, bo = 0;
-    if (lane == 0) {
-      if (msel) bs = atomicAdd(&s_cnt[0], (uint32_t)__popc(msel));
-      if (mcomp) bo = atomicAdd(&s_cnt[1], (uint32_t)__popc(mcomp));
-    }
-    bs = __shfl_sync(0xffffffffu, bs, 0) + __popc(msel & lt);
-    bo = __shfl_sync(0xffffffffu, bo, 0) + __popc(mcomp & lt);
-    if (sel) {
-      if (bs < k) list[bs] = (int32_t)t;
-      else record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x26000000u | r);
-    }
-    if (comp) {
-      if (bo < (uint32_t)Nb) list[Nb - 1 - (int64_t)bo] = (int32_t)t;
-      else record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x27000000u | r);
-      cmax = max(cmax, key);
-    }
-  }
-  if (p.full) {
-    cmax = warp_umax(cmax);
-    if (lane == 0 && cmax) atomicMax(&st->max_comp, cmax);
-  }
-  __syncthreads();
-  if (tid == 0) {
-    st->kth_key = T;
-    st->eq_total = eq_total;
-    st->eq_taken = eq_take;
-    st->n_sel = s_cnt[0];
-    st->n_comp = s_cnt[1];
-    if (s_cnt[0] != k) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x24000000u | r);
-    if (p.full && s_cnt[0] + s_cnt[1] != (uint32_t)Nb)
-      record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x25000000u | r);
-  }
-}
-
 // ------------------------------------------------------------ attend_kernel
 // Khigh rescore, softmax and value scatter of one query head, fused.  One
 // cluster of C CTAs per head; CTA `rank` owns the slice
@@ -1078,76 +1111,80 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
 }
 
 // --------------------------------------------------------------- out_kernel
-// out[r][c] += sum_a w[r][a] D_V[a][c] over `tpc` consecutive 64-atom tiles
-// and a 32-row block, D/32 warps per CTA.  Per tile the value rows are
-// staged as fp32 [a][D] (converted from bf16) and the weights as fp32
-// [a][32] (4-row groups XOR-swizzled by a).  Lane (tc, tr) of warp w owns
-// columns 32w + 4tc .. +3 and rows 8tr .. 8tr+7 (32 accumulators over all
-// the CTA's tiles): per atom, three 16-byte shared loads feed 32 FMAs.  The
-// partial sums are added into `out` (zeroed by qd_kernel) with one vector
-// reduction per row.
-template <int D>
-__global__ void __launch_bounds__(D) out_kernel(DecodeParams p, int tpc) {
-  __shared__ __align__(16) float Vs[kGvAtoms][D];
-  __shared__ __align__(16) float Ws[kGvAtoms][32];
-  constexpr int kThreads = D;
+// out[r][c] += sum_a w[r][a] D_V[a][c] over kGvTiles consecutive atom tiles
+// of kGvAtoms atoms and RB row blocks of 32 rows.  All value tiles of the
+// CTA are requested at once with cp.async (bf16 [atom][D], natural layout:
+// the column loads below are contiguous); each tile's weights are staged
+// fp32 [a][32] (4-row groups XOR-swizzled by a).  Lane (tc, tr) of warp w
+// of a row block owns columns 32w + 4tc .. +3 and rows 8tr .. 8tr+7 (32
+// accumulators over the CTA's atoms): per atom one 8-byte value load and two
+// broadcast weight loads feed 32 FMAs.  The partial sums are added into
+// `out` (zeroed by qd_kernel) with one vector reduction per row.
+constexpr int out_smem_bytes(int d, int rb, int tiles) {
+  return tiles * kGvAtoms * d * 2 + rb * kGvAtoms * 32 * 4;
+}
+
+template <int D, int RB, int kGvTiles>
+__global__ void __launch_bounds__(D * RB) out_kernel(DecodeParams p) {
+  constexpr int kThreads = D * RB;                // D/32 warps per row block
+  constexpr int kChunks = D / 8;
+  extern __shared__ uint4 out_smem[];
+  uint4* Vt = out_smem;                           // [atom][chunk], kGvTiles tiles
+  float* Ws = reinterpret_cast<float*>(out_smem + kGvTiles * kGvAtoms * kChunks);  // [rb][a][32]
   const int n = p.n, R = p.R, tid = threadIdx.x;
-  const int r0 = blockIdx.y * 32;
+  const int a0 = blockIdx.x * (kGvTiles * kGvAtoms);
+  const int r0 = blockIdx.y * (32 * RB);
+  for (int e = tid; e < kGvTiles * kGvAtoms * kChunks; e += kThreads) {
+    const int a = e / kChunks, c = e % kChunks;
+    const bool v = a0 + a < n;
+    const uint4* src = reinterpret_cast<const uint4*>(p.dv + (int64_t)(v ? a0 + a : 0) * D) + c;
+    cp_async16(Vt + a * kChunks + c, src, v);
+  }
+  cp_async_commit();
   const int lane = tid & 31, warp = tid >> 5;
+  const int rb = warp / (D / 32), wc = warp % (D / 32);
   const int tc = lane & 7, tr = lane >> 3;
-  const int cc = warp * 32 + 4 * tc;
+  const int cc = 32 * wc + 4 * tc;
   float acc[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int u = 0; u < 4; ++u) acc[i][u] = 0.0f;
-  for (int tile = 0; tile < tpc; ++tile) {
-    const int a0 = (blockIdx.x * tpc + tile) * kGvAtoms;
-    if (a0 >= n) break;
-    if (tile) __syncthreads();
-    constexpr int kChunk = 8;   // loads in flight per thread while staging
-#pragma unroll 1
-    for (int u0 = 0; u0 < kGvAtoms * (D / 8) / kThreads; u0 += kChunk) {
-      uint4 v[kChunk];
+  for (int tile = 0; tile < kGvTiles; ++tile) {
+    const int ta0 = a0 + tile * kGvAtoms;
+    if (ta0 >= n) break;
+    if (tile) __syncthreads();                    // previous weights consumed
+    // weights of this tile: lanes along atoms (coalesced), all of a
+    // thread's loads in flight before its first store
+    constexpr int kW = RB * kGvAtoms * 32;
+    constexpr int kWPer = (kW + kThreads - 1) / kThreads;
+    for (int e0 = tid; e0 < kW; e0 += kWPer * kThreads) {
+      float v[kWPer];
 #pragma unroll
-      for (int u = 0; u < kChunk; ++u) {
-        const int e = tid + (u0 + u) * kThreads;
-        const int c = e % (D / 8), a = e / (D / 8);
-        v[u] = (a0 + a < n) ? __ldg(reinterpret_cast<const uint4*>(p.dv + (int64_t)(a0 + a) * D) + c)
-                            : make_uint4(0u, 0u, 0u, 0u);
+      for (int u = 0; u < kWPer; ++u) {
+        const int e = e0 + u * kThreads;
+        const int a = e % kGvAtoms, rr = e / kGvAtoms;
+        v[u] = (e < kW && r0 + rr < R && ta0 + a < n) ? __ldg(p.w + (int64_t)(r0 + rr) * n + ta0 + a)
+                                                        : 0.0f;
       }
 #pragma unroll
-      for (int u = 0; u < kChunk; ++u) {
-        const int e = tid + (u0 + u) * kThreads;
-        const int c = e % (D / 8), a = e / (D / 8);
-        float4* dst = reinterpret_cast<float4*>(&Vs[a][c * 8]);
-        dst[0] = make_float4(bf16_lo(v[u].x), bf16_hi(v[u].x), bf16_lo(v[u].y), bf16_hi(v[u].y));
-        dst[1] = make_float4(bf16_lo(v[u].z), bf16_hi(v[u].z), bf16_lo(v[u].w), bf16_hi(v[u].w));
-      }
-    }
-#pragma unroll 1
-    for (int u0 = 0; u0 < kGvAtoms * 32 / kThreads; u0 += kChunk) {
-      float v[kChunk];
-#pragma unroll
-      for (int u = 0; u < kChunk; ++u) {
-        const int e = tid + (u0 + u) * kThreads;
-        const int a = e % kGvAtoms, r = e / kGvAtoms;
-        v[u] = (r0 + r < R && a0 + a < n) ? __ldg(p.w + (int64_t)(r0 + r) * n + a0 + a) : 0.0f;
-      }
-#pragma unroll
-      for (int u = 0; u < kChunk; ++u) {
-        const int e = tid + (u0 + u) * kThreads;
-        const int a = e % kGvAtoms, r = e / kGvAtoms;
-        Ws[a][qswz(a, r)] = v[u];
+      for (int u = 0; u < kWPer; ++u) {
+        const int e = e0 + u * kThreads;
+        if (e >= kW) break;
+        const int a = e % kGvAtoms, rr = e / kGvAtoms;
+        Ws[((rr >> 5) * kGvAtoms + a) * 32 + qswz(a, rr & 31)] = v[u];
       }
     }
+    if (tile == 0) cp_async_wait<0>();
     __syncthreads();
+    const uint4* Vtile = Vt + tile * kGvAtoms * kChunks;
+    const float* Wb = Ws + rb * kGvAtoms * 32;
 #pragma unroll 4
     for (int a = 0; a < kGvAtoms; ++a) {
-      const float4 vv = *reinterpret_cast<const float4*>(&Vs[a][cc]);
-      const float4 wa = *reinterpret_cast<const float4*>(&Ws[a][((2 * tr) ^ (a & 7)) << 2]);
-      const float4 wb = *reinterpret_cast<const float4*>(&Ws[a][((2 * tr + 1) ^ (a & 7)) << 2]);
-      const float dv[4] = {vv.x, vv.y, vv.z, vv.w};
+      const uint2 vv = reinterpret_cast<const uint2*>(Vtile + a * kChunks)[cc >> 2];
+      const float4 wa = *reinterpret_cast<const float4*>(Wb + a * 32 + (((2 * tr) ^ (a & 7)) << 2));
+      const float4 wb = *reinterpret_cast<const float4*>(Wb + a * 32 + (((2 * tr + 1) ^ (a & 7)) << 2));
+      const float dv[4] = {bf16_lo(vv.x), bf16_hi(vv.x), bf16_lo(vv.y), bf16_hi(vv.y)};
       const float wr[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
       for (int i = 0; i < 8; ++i)
@@ -1157,7 +1194,7 @@ __global__ void __launch_bounds__(D) out_kernel(DecodeParams p, int tpc) {
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int r = r0 + 8 * tr + i;
+    const int r = r0 + rb * 32 + 8 * tr + i;
     if (r >= R) continue;
     float* dst = p.out + (int64_t)r * D + cc;
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(acc[i][0]),
@@ -1210,8 +1247,17 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
   if (!attr) {
     cudaFuncSetAttribute(klow_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kTable * 4 + 4096 * 4);
-    cudaFuncSetAttribute(final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     cudaFuncSetAttribute(pass2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPass2Smem);
+    cudaFuncSetAttribute(final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         2 * kFinalStage * 4);
+    cudaFuncSetAttribute(qd_kernel<128, 2, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         qd_smem_bytes(128, 2, 4));
+    cudaFuncSetAttribute(qd_kernel<64, 2, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         qd_smem_bytes(64, 2, 4));
+    cudaFuncSetAttribute(out_kernel<128, 2, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         out_smem_bytes(128, 2, 4));
+    cudaFuncSetAttribute(out_kernel<64, 2, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         out_smem_bytes(64, 2, 4));
     cudaFuncSetAttribute(attend_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kAttSmem);
     cudaFuncSetAttribute(attend_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1222,10 +1268,22 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
                          kAttSmem);
     attr = true;
   }
+  // GEMV shapes: up to 32 query rows one tile x one row block per CTA,
+  // above that four tiles x two row blocks (the staged rows are reused)
+  const bool wide = p.R > 32;
+  const int gv_tiles = wide ? 4 : 1, gv_rb = wide ? 2 : 1;
+  const dim3 gv_grid((p.n + gv_tiles * kGvAtoms - 1) / (gv_tiles * kGvAtoms),
+                     (p.R + 32 * gv_rb - 1) / (32 * gv_rb));
   {
-    dim3 grid((p.n + kGvAtoms - 1) / kGvAtoms, (p.R + 31) / 32);
-    if (p.d == 128) qd_kernel<128><<<grid, kQdThreads, 0, stream>>>(p);
-    else qd_kernel<64><<<grid, kQdThreads, 0, stream>>>(p);
+    const size_t sm = qd_smem_bytes(p.d, gv_rb, gv_tiles);
+    const unsigned th = 64 * gv_tiles * gv_rb;
+    if (p.d == 128) {
+      if (wide) qd_kernel<128, 2, 4><<<gv_grid, th, sm, stream>>>(p);
+      else qd_kernel<128, 1, 1><<<gv_grid, th, sm, stream>>>(p);
+    } else {
+      if (wide) qd_kernel<64, 2, 4><<<gv_grid, th, sm, stream>>>(p);
+      else qd_kernel<64, 1, 1><<<gv_grid, th, sm, stream>>>(p);
+    }
   }
   {
     const int g = grid_for(p.tok_off[p.B], 2048, sms);
@@ -1262,14 +1320,14 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
     if (cudaLaunchKernelEx(&cfg, kern, p, C) != cudaSuccess) return SDK_ERR_CUDA;
   }
   {
-    // atom tiles per CTA: enough CTAs for ~4 per SM, fewer reductions
-    const int tiles = (p.n + kGvAtoms - 1) / kGvAtoms;
-    const int rb = (p.R + 31) / 32;
-    int tpc = 1;
-    while (tpc < 8 && (int64_t)((tiles + 2 * tpc - 1) / (2 * tpc)) * rb >= 4 * sms) tpc *= 2;
-    dim3 grid((tiles + tpc - 1) / tpc, rb);
-    if (p.d == 128) out_kernel<128><<<grid, 128, 0, stream>>>(p, tpc);
-    else out_kernel<64><<<grid, 64, 0, stream>>>(p, tpc);
+    const size_t sm = out_smem_bytes(p.d, gv_rb, gv_tiles);
+    if (p.d == 128) {
+      if (wide) out_kernel<128, 2, 4><<<gv_grid, 128 * 2, sm, stream>>>(p);
+      else out_kernel<128, 1, 1><<<gv_grid, 128, sm, stream>>>(p);
+    } else {
+      if (wide) out_kernel<64, 2, 4><<<gv_grid, 64 * 2, sm, stream>>>(p);
+      else out_kernel<64, 1, 1><<<gv_grid, 64, sm, stream>>>(p);
+    }
   }
   return cudaGetLastError() == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
 }
