@@ -27,6 +27,7 @@
 //   out_kernel       out += w D_V over atom tiles (vector reductions into
 //                    `out`, zeroed by qd_kernel).
 #include <cooperative_groups.h>
+#include <stdlib.h>
 #include <type_traits>
 
 #include "sdk_internal.cuh"
@@ -126,6 +127,8 @@ constexpr int qd_smem_bytes(int d, int rb, int tiles) { return tiles * kGvAtoms 
 
 template <int D, int RB, int kGvTiles>
 __global__ void __launch_bounds__(64 * kGvTiles * RB, (RB > 1 ? 2 : 1)) qd_kernel(DecodeParams p) {
+  pdl_wait();     // nothing global is touched before the previous kernel is done
+  pdl_launch();
   constexpr int kThreads = 64 * kGvTiles * RB;
   constexpr int kChunks = D / 8;                  // 16-byte chunks per atom row
   extern __shared__ uint4 qd_smem[];
@@ -282,6 +285,8 @@ __device__ __forceinline__ void stage_table(float* table, const float* src, int 
 }
 
 __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, int vec) {
+  pdl_wait();     // nothing global is touched before the previous kernel is done
+  pdl_launch();
   extern __shared__ float4 smem4[];
   float* table = reinterpret_cast<float*>(smem4);
   uint32_t* sh = reinterpret_cast<uint32_t*>(table + kTable);
@@ -556,6 +561,8 @@ __device__ void final_head(const DecodeParams& p, int r, uint32_t* s_cand, uint3
 
 // One CTA per query head runs the final selection.
 __global__ void __launch_bounds__(kScanThreads) final_kernel(DecodeParams p) {
+  pdl_wait();     // nothing global is touched before the previous kernel is done
+  pdl_launch();
   __shared__ uint32_t s_tmp[48];
   __shared__ uint32_t sh[2048];
   __shared__ uint32_t s_cnt[2];
@@ -593,6 +600,8 @@ __device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v, uint32_t& total) 
 }
 
 __global__ void __launch_bounds__(kScanThreads, 1) pass2_kernel(DecodeParams p) {
+  pdl_wait();     // nothing global is touched before the previous kernel is done
+  pdl_launch();
   __shared__ uint32_t s_tmp[48];
   __shared__ uint32_t s_ncand, s_cbase;
   extern __shared__ uint32_t s_dyn[];   // kPass2Smem bytes
@@ -949,6 +958,8 @@ __device__ __forceinline__ float block_reduce(float v, float* s_red) {
 
 template <bool kAll16, bool kCheck>
 __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, int C) {
+  pdl_wait();     // nothing global is touched before the previous kernel is done
+  pdl_launch();
   extern __shared__ float4 smem4[];
   float* table = reinterpret_cast<float*>(smem4);
   int* siw = reinterpret_cast<int*>(smem4);
@@ -1126,6 +1137,8 @@ constexpr int out_smem_bytes(int d, int rb, int tiles) {
 
 template <int D, int RB, int kGvTiles>
 __global__ void __launch_bounds__(D * RB) out_kernel(DecodeParams p) {
+  pdl_wait();     // nothing global is touched before the previous kernel is done
+  pdl_launch();
   constexpr int kThreads = D * RB;                // D/32 warps per row block
   constexpr int kChunks = D / 8;
   extern __shared__ uint4 out_smem[];
@@ -1241,6 +1254,47 @@ static int grid_for(int64_t work, int64_t per_cta, int cap_ctas) {
   return (int)g;
 }
 
+// Optional launch with programmatic stream serialization (the kernel may
+// start while the previous one drains; every decode kernel waits for it
+// before touching memory).  Off by default: measured on B200 it made the
+// 32-layer 256K-token step slower (early-resident CTAs of the next kernel
+// hold SM resources); SDK_DECODE_PDL=1 in the environment turns it on.
+static bool pdl_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* v = getenv("SDK_DECODE_PDL");
+    on = (v != nullptr && v[0] == '1') ? 1 : 0;
+  }
+  return on == 1;
+}
+
+template <class... KArgs, class... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, unsigned cluster, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[2];
+  int na = 0;
+  if (pdl_enabled()) {
+    at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (cluster > 1) {
+    at[na].id = cudaLaunchAttributeClusterDimension;
+    at[na].val.clusterDim.x = cluster;
+    at[na].val.clusterDim.y = 1;
+    at[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
   const int sms = num_sms();
   static bool attr = false;
@@ -1268,6 +1322,7 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
                          kAttSmem);
     attr = true;
   }
+  cudaError_t e = cudaSuccess;
   // GEMV shapes: up to 32 query rows one tile x one row block per CTA,
   // above that four tiles x two row blocks (the staged rows are reused)
   const bool wide = p.R > 32;
@@ -1278,23 +1333,29 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
     const size_t sm = qd_smem_bytes(p.d, gv_rb, gv_tiles);
     const unsigned th = 64 * gv_tiles * gv_rb;
     if (p.d == 128) {
-      if (wide) qd_kernel<128, 2, 4><<<gv_grid, th, sm, stream>>>(p);
-      else qd_kernel<128, 1, 1><<<gv_grid, th, sm, stream>>>(p);
+      e = wide ? launch_pdl(qd_kernel<128, 2, 4>, gv_grid, dim3(th), sm, stream, 1, p)
+               : launch_pdl(qd_kernel<128, 1, 1>, gv_grid, dim3(th), sm, stream, 1, p);
     } else {
-      if (wide) qd_kernel<64, 2, 4><<<gv_grid, th, sm, stream>>>(p);
-      else qd_kernel<64, 1, 1><<<gv_grid, th, sm, stream>>>(p);
+      e = wide ? launch_pdl(qd_kernel<64, 2, 4>, gv_grid, dim3(th), sm, stream, 1, p)
+               : launch_pdl(qd_kernel<64, 1, 1>, gv_grid, dim3(th), sm, stream, 1, p);
     }
+    if (e != cudaSuccess) return SDK_ERR_CUDA;
   }
   {
     const int g = grid_for(p.tok_off[p.B], 2048, sms);
     const int vec = (p.cap % 4 == 0) && ((reinterpret_cast<uintptr_t>(p.k_lo) & 15u) == 0u);
-    klow_kernel<<<g, kKlowThreads, (size_t)kTable * 4 + 4096 * 4, stream>>>(p, vec);
+    e = launch_pdl(klow_kernel, dim3(g), dim3(kKlowThreads), (size_t)kTable * 4 + 4096 * 4, stream,
+                   1, p, vec);
+    if (e != cudaSuccess) return SDK_ERR_CUDA;
   }
   {
     const int g = grid_for(p.tok_off[p.B], 8192, sms);
-    pass2_kernel<<<g, kScanThreads, kPass2Smem, stream>>>(p);
+    e = launch_pdl(pass2_kernel, dim3(g), dim3(kScanThreads), (size_t)kPass2Smem, stream, 1, p);
+    if (e != cudaSuccess) return SDK_ERR_CUDA;
   }
-  final_kernel<<<p.R, kScanThreads, (size_t)2 * kFinalStage * 4, stream>>>(p);
+  e = launch_pdl(final_kernel, dim3(p.R), dim3(kScanThreads), (size_t)2 * kFinalStage * 4, stream, 1,
+                 p);
+  if (e != cudaSuccess) return SDK_ERR_CUDA;
   {
     // one cluster of C CTAs per query head, C a power of two <= 8 while the
     // clusters fit the SMs and every CTA keeps >= 1024 entries
@@ -1302,32 +1363,23 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
     for (int b = 0; b < p.B; ++b) dmax = p.dcnt[b] > dmax ? p.dcnt[b] : dmax;
     int C = 1;
     while (C < 8 && (int64_t)p.R * C * 2 <= sms && dmax / (2 * C) >= 1024) C *= 2;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(p.R * C));
-    cfg.blockDim = dim3(kAttThreads);
-    cfg.dynamicSmemBytes = kAttSmem;
-    cfg.stream = stream;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = (unsigned)C;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
     const bool all16 = p.khigh == kAtoms, check = p.n < kTable;
     auto kern = all16 ? (check ? attend_kernel<true, true> : attend_kernel<true, false>)
                       : (check ? attend_kernel<false, true> : attend_kernel<false, false>);
-    if (cudaLaunchKernelEx(&cfg, kern, p, C) != cudaSuccess) return SDK_ERR_CUDA;
+    e = launch_pdl(kern, dim3((unsigned)(p.R * C)), dim3(kAttThreads), (size_t)kAttSmem, stream,
+                   (unsigned)C, p, C);
+    if (e != cudaSuccess) return SDK_ERR_CUDA;
   }
   {
     const size_t sm = out_smem_bytes(p.d, gv_rb, gv_tiles);
     if (p.d == 128) {
-      if (wide) out_kernel<128, 2, 4><<<gv_grid, 128 * 2, sm, stream>>>(p);
-      else out_kernel<128, 1, 1><<<gv_grid, 128, sm, stream>>>(p);
+      e = wide ? launch_pdl(out_kernel<128, 2, 4>, gv_grid, dim3(256), sm, stream, 1, p)
+               : launch_pdl(out_kernel<128, 1, 1>, gv_grid, dim3(128), sm, stream, 1, p);
     } else {
-      if (wide) out_kernel<64, 2, 4><<<gv_grid, 64 * 2, sm, stream>>>(p);
-      else out_kernel<64, 1, 1><<<gv_grid, 64, sm, stream>>>(p);
+      e = wide ? launch_pdl(out_kernel<64, 2, 4>, gv_grid, dim3(128), sm, stream, 1, p)
+               : launch_pdl(out_kernel<64, 1, 1>, gv_grid, dim3(64), sm, stream, 1, p);
     }
+    if (e != cudaSuccess) return SDK_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
 }

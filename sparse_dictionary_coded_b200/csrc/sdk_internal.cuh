@@ -96,6 +96,16 @@ __device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, uint32_t* s_warp
   return base + v;
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel of the stream drains;
+// pdl_wait() blocks until that kernel has completed and its memory is
+// visible (a no-op for an ordinary launch).  pdl_launch() lets the next
+// kernel of the stream start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // 16-byte asynchronous global -> shared copy (L2 only, no registers); with
 // valid == false nothing is read and the 16 bytes are zero-filled (the
 // source operand is then only a placeholder address).
