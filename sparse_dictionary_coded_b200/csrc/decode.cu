@@ -1268,6 +1268,16 @@ static bool pdl_enabled() {
   return on == 1;
 }
 
+// QD on the tensor cores (three bf16 parts of q) unless SDK_DECODE_QD_TC=0.
+static bool qd_tensor_cores() {
+  static int on = -1;
+  if (on < 0) {
+    const char* v = getenv("SDK_DECODE_QD_TC");
+    on = (v != nullptr && v[0] == '0') ? 0 : 1;
+  }
+  return on == 1;
+}
+
 template <class... KArgs, class... Args>
 static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
                               cudaStream_t stream, unsigned cluster, Args... args) {
@@ -1329,7 +1339,12 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
   const int gv_tiles = wide ? 4 : 1, gv_rb = wide ? 2 : 1;
   const dim3 gv_grid((p.n + gv_tiles * kGvAtoms - 1) / (gv_tiles * kGvAtoms),
                      (p.R + 32 * gv_rb - 1) / (32 * gv_rb));
-  {
+  bool qd_tc = false;
+  if (qd_tensor_cores()) {
+    const sdk_status st = launch_qd_tc(p, stream, &qd_tc);
+    if (st != SDK_OK) return st;
+  }
+  if (!qd_tc) {
     const size_t sm = qd_smem_bytes(p.d, gv_rb, gv_tiles);
     const unsigned th = 64 * gv_tiles * gv_rb;
     if (p.d == 128) {

@@ -266,3 +266,54 @@ def test_full_size_layer_sampled_heads(name):
             ref = oracle.decode_head_ref(qn[b, h], kwn, vwn, DKn, DVn,
                                          force_set=sets[r])
         assert np.max(np.abs(outn[b, h] - ref["out"])) <= OUT_TOL
+
+
+_QD_PATH_CASE = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+sys.path.insert(0, sys.argv[1] + "/tests")
+import workloads, sparse_dictionary_coded_b200 as sdk
+from test_gpu_decode import _random_case, _store
+for name, args in (("b1", (81, 1, 32, 8, 2000, 128, 32768)),
+                   ("b4", (82, 4, 32, 8, 600, 128, 4096))):
+    q, DK, DV, kw, vw, lens = _random_case(*args)
+    B, Hq, d = q.shape
+    store = _store(kw, vw, lens)
+    n = DK.shape[0]
+    ws = sdk.new_workspace(sdk.sdk_decode_workspace_bytes(B, Hq, d, n, max(lens)))
+    out = sdk.sdk_decode_attn(q.cuda(), DK.cuda(), DV.cuda(), store, workspace=ws)
+    torch.cuda.synchronize()
+    assert sdk.sdk_check_status(ws)[0] == 0
+    lay = sdk.sdk_decode_layout_of(B, Hq, d, n, max(lens))
+    qd = ws[lay["qd"]:lay["qd"] + B * Hq * n * 4].view(torch.float32).cpu().numpy()
+    np.save(sys.argv[2] + "/qd_" + name + ".npy", qd)
+    np.save(sys.argv[2] + "/out_" + name + ".npy", out.cpu().numpy())
+print("saved")
+"""
+
+
+def test_qd_on_cuda_cores_matches_tensor_cores(tmp_path):
+    """D1 runs on the tensor cores (q split into three bf16 parts) unless
+    SDK_DECODE_QD_TC=0 selects the fp32 CUDA-core kernel (read once per
+    process, hence child processes): both give QD within fp32 rounding of
+    each other and the same outputs, at 32 and at 128 query rows."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    res = {}
+    for mode in ("1", "0"):
+        d = tmp_path / mode
+        d.mkdir()
+        env = dict(os.environ, SDK_DECODE_QD_TC=mode)
+        r = subprocess.run([sys.executable, "-c", _QD_PATH_CASE, root, str(d)],
+                           env=env, capture_output=True, text=True, timeout=600)
+        assert r.returncode == 0, r.stdout + r.stderr
+        res[mode] = d
+    for name in ("b1", "b4"):
+        qa = np.load(res["1"] / ("qd_" + name + ".npy"))
+        qb = np.load(res["0"] / ("qd_" + name + ".npy"))
+        assert np.max(np.abs(qa - qb)) <= 2e-6 * np.max(np.abs(qb))
+        oa = np.load(res["1"] / ("out_" + name + ".npy"))
+        ob = np.load(res["0"] / ("out_" + name + ".npy"))
+        assert np.max(np.abs(oa - ob)) <= OUT_TOL
