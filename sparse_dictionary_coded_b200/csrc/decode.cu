@@ -1278,6 +1278,16 @@ static bool qd_tensor_cores() {
   return on == 1;
 }
 
+// w D_V on the tensor cores (three bf16 parts of w) unless SDK_DECODE_OUT_TC=0.
+static bool out_tensor_cores() {
+  static int on = -1;
+  if (on < 0) {
+    const char* v = getenv("SDK_DECODE_OUT_TC");
+    on = (v != nullptr && v[0] == '0') ? 0 : 1;
+  }
+  return on == 1;
+}
+
 template <class... KArgs, class... Args>
 static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
                               cudaStream_t stream, unsigned cluster, Args... args) {
@@ -1385,7 +1395,14 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
                    (unsigned)C, p, C);
     if (e != cudaSuccess) return SDK_ERR_CUDA;
   }
-  {
+  // w D_V: tensor cores above 32 query rows; at 32 or fewer the CUDA-core
+  // kernel was measured faster (the tensor-core CTAs are latency-bound)
+  bool out_tc = false;
+  if (out_tensor_cores() && p.R > 32) {
+    const sdk_status st = launch_out_tc(p, stream, &out_tc);
+    if (st != SDK_OK) return st;
+  }
+  if (!out_tc) {
     const size_t sm = out_smem_bytes(p.d, gv_rb, gv_tiles);
     if (p.d == 128) {
       e = wide ? launch_pdl(out_kernel<128, 2, 4>, gv_grid, dim3(256), sm, stream, 1, p)

@@ -194,6 +194,8 @@ int num_sms();  // cached multiprocessor count of the current device
 
 // QD on the tensor cores (taken = false: not available, use the CUDA cores)
 sdk_status launch_qd_tc(const DecodeParams& p, cudaStream_t stream, bool* taken);
+// out += w D_V on the tensor cores (taken = false: use the CUDA cores)
+sdk_status launch_out_tc(const DecodeParams& p, cudaStream_t stream, bool* taken);
 sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream);
 sdk_decode_layout decode_layout(int B, int Hq, int d, int n, int64_t L);
 sdk_status launch_encode_simt(const EncodeParams& p, int head_dim, cudaStream_t stream);

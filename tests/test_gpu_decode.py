@@ -275,6 +275,7 @@ sys.path.insert(0, sys.argv[1] + "/tests")
 import workloads, sparse_dictionary_coded_b200 as sdk
 from test_gpu_decode import _random_case, _store
 for name, args in (("b1", (81, 1, 32, 8, 2000, 128, 32768)),
+                   ("b2", (83, 2, 32, 8, 900, 64, 2048)),
                    ("b4", (82, 4, 32, 8, 600, 128, 4096))):
     q, DK, DV, kw, vw, lens = _random_case(*args)
     B, Hq, d = q.shape
@@ -292,11 +293,12 @@ print("saved")
 """
 
 
-def test_qd_on_cuda_cores_matches_tensor_cores(tmp_path):
-    """D1 runs on the tensor cores (q split into three bf16 parts) unless
-    SDK_DECODE_QD_TC=0 selects the fp32 CUDA-core kernel (read once per
-    process, hence child processes): both give QD within fp32 rounding of
-    each other and the same outputs, at 32 and at 128 query rows."""
+def test_gemvs_on_cuda_cores_match_tensor_cores(tmp_path):
+    """D1 and D6 run on the tensor cores (q and w split into three bf16
+    parts) unless SDK_DECODE_QD_TC=0 / SDK_DECODE_OUT_TC=0 select the fp32
+    CUDA-core kernels (read once per process, hence child processes): both
+    give QD within fp32 rounding of each other and the same outputs, at 32,
+    64 (head_dim 64) and 128 query rows."""
     import os
     import subprocess
     import sys
@@ -305,15 +307,15 @@ def test_qd_on_cuda_cores_matches_tensor_cores(tmp_path):
     for mode in ("1", "0"):
         d = tmp_path / mode
         d.mkdir()
-        env = dict(os.environ, SDK_DECODE_QD_TC=mode)
+        env = dict(os.environ, SDK_DECODE_QD_TC=mode, SDK_DECODE_OUT_TC=mode)
         r = subprocess.run([sys.executable, "-c", _QD_PATH_CASE, root, str(d)],
                            env=env, capture_output=True, text=True, timeout=600)
         assert r.returncode == 0, r.stdout + r.stderr
         res[mode] = d
-    for name in ("b1", "b4"):
+    for name in ("b1", "b2", "b4"):
         qa = np.load(res["1"] / ("qd_" + name + ".npy"))
         qb = np.load(res["0"] / ("qd_" + name + ".npy"))
         assert np.max(np.abs(qa - qb)) <= 2e-6 * np.max(np.abs(qb))
         oa = np.load(res["1"] / ("out_" + name + ".npy"))
         ob = np.load(res["0"] / ("out_" + name + ".npy"))
-        assert np.max(np.abs(oa - ob)) <= OUT_TOL
+        assert np.max(np.abs(oa - ob)) <= 1e-5 * max(1.0, np.max(np.abs(ob)))
