@@ -9,7 +9,8 @@ step is the whole hot path on that layer -- greedy-pursuit encode of all
 4096 x 8 x 2 = 65,536 K/V vectors written into the code store (sdk_append),
 then one decode-attention step over the 4096 tokens (sdk_decode_attn).
 'decode256k' / 'decode32k_b4' time a 32-layer decode step, 'prefill256k_vec'
-the encode of 262,144 vectors.
+the encode of 262,144 vectors, 'append_token_b1' / 'append_token_b4' the
+append of one generated token to all 32 layers (batch 1 / batch 4).
 
 Timing: W untimed warm-up steps, then K steps, each timed with CUDA events on
 the launching stream; the L2 is flushed (256 MiB memset) between steps,
@@ -68,7 +69,8 @@ def parse():
     ap.add_argument("--impl", default="sdk", choices=["sdk", "reference"])
     ap.add_argument("--workload", default="layer4k",
                     choices=["layer4k", "decode256k", "decode32k_b4",
-                             "prefill256k_vec"])
+                             "prefill256k_vec", "append_token_b1",
+                             "append_token_b4"])
     ap.add_argument("--layers", type=int, default=None,
                     help="decode workloads: layers to instantiate (default: "
                          "the workload's 32); fewer layers make small ncu "
@@ -476,6 +478,98 @@ def bench_prefill(args, world, rank, pk):
     }
 
 
+APPEND_WORKLOADS = {"append_token_b1": "decode256k",
+                    "append_token_b4": "decode32k_b4"}
+
+
+def bench_append(args, world, rank, pk, name):
+    """One generated token's append over all layers of a 32-layer decode
+    workload: per layer, B x 8 new K and 8 new V vectors encoded against
+    that layer's own dictionaries and written into its code store
+    (sdk_append with n_new = 1, one call per layer)."""
+    import torch
+    import workloads
+    import sparse_dictionary_coded_b200 as sdk
+    base = APPEND_WORKLOADS[name]
+    W = workloads.WORKLOADS[base]
+    L, B, Hkv, d, n = W["L"], W["B"], W["Hkv"], W["d"], W["n_atoms"]
+    if args.layers is not None:
+        L = max(1, min(L, args.layers))
+    cap = 4
+    layers = []
+    for l in range(L):
+        a = workloads.append_token(base, l + 1000 * rank, device="cuda")
+        layers.append(dict(DK=a["DK"], DV=a["DV"], xk=a["xk"].contiguous(),
+                           xv=a["xv"].contiguous(),
+                           store=sdk.CodeStore(B, Hkv, cap)))
+    aws = sdk.new_workspace(sdk.sdk_append_workspace_bytes(B, Hkv, 1, d, n))
+    n_vec = L * 2 * B * Hkv
+    torch.cuda.synchronize()
+
+    def step():
+        for ly in layers:
+            ly["store"].lens = [cap - 1] * B
+            sdk.sdk_append(ly["store"], ly["xk"], ly["xv"], ly["DK"], ly["DV"],
+                           workspace=aws)
+
+    flush = make_flush()
+    clocks = Clocks(torch.cuda.current_device())
+    ms, ck = timed_steps(step, args.steps, args.warmup, flush, world, clocks)
+    rc, _ = sdk.sdk_check_status(aws)
+    assert rc == 0, "device check failed in append"
+    step_ms = max_over_ranks(statistics.mean(ms), world)
+    flops = n_vec * enc_flop_per_vector(n, d)
+    tfl = flops / (step_ms * 1e-3) / 1e12
+    res = {
+        "value": world * n_vec / (step_ms * 1e-3),
+        "unit": "encoded KV vecs/s (one token appended to all %d layers)" % L,
+        "ms_per_step": step_ms,
+        "us_per_token": step_ms * 1e3,
+        "us_per_layer": step_ms * 1e3 / L,
+        # the correlation GEMM runs on the tensor cores; a call is 16
+        # dependent greedy steps, each ending in a grid-wide exchange, so the
+        # fraction is small: the step latency, not the FLOP rate, bounds it
+        "roofline": dict(tensor_roofline(tfl, pk, "encode_small_kernel (%d "
+                                         "launches)" % L),
+                         note="latency-bound: 16 dependent steps per call, "
+                              "%.1f us per step" % (step_ms * 1e3 / L / 16),
+                         hbm_floor_us=L * 2 * n * d * 2 / (pk["hbm"] * 1e9) * 1e6),
+        "clocks": ck,
+        "config": {"workload": name, "layers": L, "B": B, "Hkv": Hkv,
+                   "head_dim": d, "n_atoms": n, "k_atoms": 16, "n_new": 1,
+                   "l2": "flushed between steps; the %d layers' dictionaries "
+                         "(%.0f MB) exceed L2" % (L, L * 2 * n * d * 2 / 1e6)},
+        "dtype": ("f32 (residuals, exact re-scoring; tensor-core operands "
+                  "bf16 with fp32 accumulation; fp16 coefficients)"),
+        # per layer one kernel (the exchange words are cleared by a runtime
+        # memset, not counted)
+        "gpu_launches": args.steps * L,
+    }
+    if not args.no_e2e:
+        hx = [(ly["xk"].cpu().pin_memory(), ly["xv"].cpu().pin_memory())
+              for ly in layers]
+        hout = torch.empty(L, 2, B, Hkv, 16, dtype=torch.int32).pin_memory()
+
+        def e2e_step():
+            for l, ly in enumerate(layers):
+                ly["xk"].copy_(hx[l][0], non_blocking=True)
+                ly["xv"].copy_(hx[l][1], non_blocking=True)
+                ly["store"].lens = [cap - 1] * B
+                sdk.sdk_append(ly["store"], ly["xk"], ly["xv"], ly["DK"],
+                               ly["DV"], workspace=aws)
+                hout[l, 0].copy_(ly["store"].k_full[:, :, cap - 1], non_blocking=True)
+                hout[l, 1].copy_(ly["store"].v_full[:, :, cap - 1], non_blocking=True)
+
+        ms_e, _ = timed_steps(e2e_step, max(2, args.steps // 2), 1, flush, world)
+        t = max_over_ranks(statistics.mean(ms_e), world)
+        res["e2e"] = {"value": world * n_vec / (t * 1e-3),
+                      "unit": "encoded KV vecs/s", "ms_per_step": t,
+                      "h2d_bytes_per_step": sum(a.numel() * 4 + b.numel() * 4
+                                                for a, b in hx),
+                      "d2h_bytes_per_step": hout.numel() * 4}
+    return res
+
+
 # ------------------------------------------------------ oracle timings
 
 def cpu_baseline(name, budget_s=15.0):
@@ -487,6 +581,23 @@ def cpu_baseline(name, budget_s=15.0):
     import workloads
     cores = len(os.sched_getaffinity(0))
     torch.set_num_threads(cores)
+    if name in APPEND_WORKLOADS:
+        base = APPEND_WORKLOADS[name]
+        W = workloads.WORKLOADS[base]
+        a = workloads.append_token(base, 0)
+        xs = a["xk"].reshape(-1, a["d"]).double().numpy()
+        Dn = a["DK"].float().double().numpy()
+        t0 = time.perf_counter()
+        nvec = 0
+        while time.perf_counter() - t0 < budget_s * 0.8 and nvec < xs.shape[0]:
+            oracle.encode_ref(xs[nvec:nvec + 4], Dn)
+            nvec += 4
+        t_vec = (time.perf_counter() - t0) / nvec
+        per_step = W["L"] * 2 * W["B"] * W["Hkv"]
+        return {"value": 1.0 / t_vec, "unit": "encoded KV vecs/s",
+                "cores": cores, "kind": "oracle",
+                "sample": "%d of the %d vectors of one token's append encoded "
+                          "by the oracle" % (nvec, per_step)}
     if name in ("layer4k", "prefill256k_vec"):
         if name == "layer4k":
             w = workloads.layer4k()
@@ -582,6 +693,8 @@ def main():
         res = bench_layer4k(args, world, rank, pk)
     elif args.workload == "prefill256k_vec":
         res = bench_prefill(args, world, rank, pk)
+    elif args.workload in APPEND_WORKLOADS:
+        res = bench_append(args, world, rank, pk, args.workload)
     else:
         res = bench_decode(args, world, rank, pk, args.workload)
     if rank == 0:

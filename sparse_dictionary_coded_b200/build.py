@@ -15,7 +15,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsdk.so")
 
-SOURCES = ["api.cu", "decode.cu", "decode_static.cu", "encode_simt.cu",
+SOURCES = ["api.cu", "decode.cu", "decode_static.cu", "encode_simt.cu", "encode_small.cu",
            "encode_tc.cu", "out_tc.cu", "qd_tc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",

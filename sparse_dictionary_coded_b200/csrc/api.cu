@@ -72,8 +72,10 @@ int32_t sdk_version(void) { return 1; }
 
 size_t sdk_encode_workspace_bytes(int64_t n_vec, int32_t head_dim, int32_t n_atoms) {
   if (n_vec < 0) n_vec = 0;
-  return align_up(sizeof(WsHeader), 256) +
-         align_up(encode_tc_scratch_bytes(n_vec, head_dim, n_atoms), 256);
+  size_t scratch = encode_tc_scratch_bytes(n_vec, head_dim, n_atoms);
+  if (n_vec >= 1 && n_vec <= kSmallEncodeRows && encode_small_scratch_bytes() > scratch)
+    scratch = encode_small_scratch_bytes();
+  return align_up(sizeof(WsHeader), 256) + align_up(scratch, 256);
 }
 
 // Runs the encoder with an explicit header and scratch area (the scratch is
@@ -81,6 +83,16 @@ size_t sdk_encode_workspace_bytes(int64_t n_vec, int32_t head_dim, int32_t n_ato
 static sdk_status encode_core(bool allow_tc, const EncodeParams& p, int head_dim, void* scratch,
                               size_t scratch_bytes, cudaStream_t st) {
   if (p.n_vec == 0) return SDK_OK;
+  if (allow_tc && p.n_vec <= kSmallEncodeRows) {
+    SmallEncode e;
+    memset(&e, 0, sizeof(e));
+    e.p[0] = p;
+    e.streams = 1;
+    e.head_dim = head_dim;
+    bool taken = false;
+    sdk_status s = launch_encode_small(e, scratch, scratch_bytes, st, &taken);
+    if (taken) return s;
+  }
   if (allow_tc) {
     bool taken = false;
     sdk_status s = launch_encode_tc(p, head_dim, scratch, scratch_bytes, st, &taken);
@@ -197,6 +209,48 @@ sdk_status sdk_append(const void* xk, const void* xv, int32_t x_dtype, int32_t B
   char* scratch = ws + hb + align_up((size_t)nv * kAtoms * 4, 256);
   const size_t scratch_bytes = sdk_encode_workspace_bytes(nv, head_dim, n_atoms) - hb;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // a few vectors: the atom-parallel encoder writes straight into the store,
+  // K and V in one launch when both fit
+  if (nv <= kSmallEncodeRows) {
+    SmallEncode e;
+    memset(&e, 0, sizeof(e));
+    for (int s = 0; s < 2; ++s) {
+      EncodeParams& p = e.p[s];
+      p.x = s == 0 ? xk : xv;
+      p.x_dtype = x_dtype;
+      p.n_vec = nv;
+      p.dict = reinterpret_cast<const uint16_t*>(s == 0 ? dict_k : dict_v);
+      p.n = n_atoms;
+      p.k_atoms = kAtoms;
+      p.codes = s == 0 ? k_full : v_full;
+      p.rsq = nullptr;
+      p.hdr = reinterpret_cast<WsHeader*>(ws);
+    }
+    e.head_dim = head_dim;
+    e.append = true;
+    e.lo[0] = k_lo;
+    e.lo[1] = nullptr;
+    e.cap = cap;
+    e.B = B;
+    e.Hkv = Hkv;
+    e.n_new = n_new;
+    e.lens = lens_host;
+    e.streams = 2;
+    bool taken = false;
+    sdk_status rc = launch_encode_small(e, scratch, scratch_bytes, st, &taken);
+    if (taken) return rc;
+    SmallEncode one = e;
+    one.streams = 1;
+    rc = launch_encode_small(one, scratch, scratch_bytes, st, &taken);
+    if (taken) {
+      if (rc != SDK_OK) return rc;
+      one.p[0] = e.p[1];
+      one.lo[0] = nullptr;
+      rc = launch_encode_small(one, scratch, scratch_bytes, st, &taken);
+      if (!taken) return SDK_ERR_CUDA;  // the same shape was taken just before
+      return rc;
+    }
+  }
   for (int s = 0; s < 2; ++s) {
     EncodeParams p;
     p.x = s == 0 ? xk : xv;

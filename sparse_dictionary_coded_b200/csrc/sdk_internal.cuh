@@ -205,4 +205,25 @@ sdk_status launch_encode_tc(const EncodeParams& p, int head_dim, void* scratch,
                             size_t scratch_bytes, cudaStream_t stream, bool* taken);
 size_t encode_tc_scratch_bytes(int64_t n_vec, int head_dim, int n_atoms);
 
+// Atom-parallel encoder for a few vectors of one or two streams (rows per
+// call: 64 in total, the second stream starting at an even slot).  In
+// append mode p[s].codes is the code store (full words) and lo[s] the
+// first-3 planes (or null); words land at token lens[b] + i.
+struct SmallEncode {
+  EncodeParams p[2];
+  int streams;
+  int head_dim;
+  bool append;
+  uint32_t* lo[2];
+  int64_t cap;
+  int B, Hkv, n_new;
+  const int32_t* lens;  // host, [B]
+};
+// Sets *taken = false when it does not handle the call (too many rows,
+// dictionary too large for one wave, switched off by SDK_ENCODE_SMALL=0).
+sdk_status launch_encode_small(const SmallEncode& e, void* scratch, size_t scratch_bytes,
+                               cudaStream_t stream, bool* taken);
+size_t encode_small_scratch_bytes();
+constexpr int64_t kSmallEncodeRows = 64;
+
 }  // namespace sdk

@@ -209,3 +209,144 @@ def test_bf16_operands_agree_exactly():
                        capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "identical" in r.stdout
+
+
+SMALL_CASES = [
+    # (n_vec, head_dim, n_atoms, x dtype, k_atoms)
+    (1, 128, 32768, torch.float32, 16),
+    (7, 64, 1000, torch.bfloat16, 16),
+    (33, 128, 4097, torch.float32, 5),
+    (64, 128, 32768, torch.float32, 16),
+    (64, 64, 3, torch.float32, 16),
+    (2, 128, 1, torch.float32, 4),
+]
+
+
+@pytest.mark.parametrize("case", SMALL_CASES, ids=lambda c: "m%d_d%d_n%d" % c[:3])
+def test_small_batch_encoder_matches_simt_exactly(case):
+    """At most 64 vectors go to the atom-parallel encoder (the dictionary
+    spread over all SMs, one grid barrier per greedy step).  It keeps the
+    CUDA-core encoder's fp32 arithmetic, so words and residual energies are
+    bit-identical to sdk_encode_simt; the picks also pass the oracle walk.
+    Cases: one vector, ragged counts, a full 64-row call, dictionaries of
+    1 and 3 atoms (an atom picked again and again), bf16 input, k < 16."""
+    m, d, n, dt, k = case
+    g = workloads.make_gen(61 + m + n)
+    D = workloads.gaussian_dictionary(n, d, g)
+    if n >= 16:
+        x, _, _ = workloads.planted_vectors(D, m, g, noise_rel=0.05)
+    else:
+        x = torch.randn(m, d, generator=g)
+    x = x.to(dt)
+    (a, ra), _ = _enc("sdk_encode", x, D, k=k, rsq=True)
+    (b, rb), _ = _enc("sdk_encode_simt", x, D, k=k, rsq=True)
+    assert torch.equal(a.cpu(), b.cpu())
+    assert torch.equal(ra.cpu(), rb.cpu())
+    # with fewer atoms than picks the greedy coefficients shrink
+    # geometrically once every atom has been taken, down to the rounding
+    # noise of an fp32 dot product on either side; the oracle walk covers
+    # the first min(n, k) steps there
+    k_or = min(k, n)
+    ref = _oracle(x.float(), D, k_or)
+    check_encode(words_np(a)[:, :k_or], ref)
+
+
+def test_small_batch_encoder_edge_vectors():
+    """Zero vector (atom 0 with coefficient 0 at every step, as the
+    CUDA-core scan leaves it), a scaled atom (exact first pick), and
+    identical atoms tied for the pick (the lowest index wins) in one call."""
+    g = workloads.make_gen(71)
+    n, d = 32768, 128
+    D = workloads.gaussian_dictionary(n, d, g)
+    D[20000:20012] = D[31000]
+    x = torch.randn(5, d, generator=g)
+    x[0] = 0.0
+    x[1] = 2.5 * D[417].float()
+    x[2] = 3.0 * D[31000].float() + 0.01 * torch.randn(d, generator=g)
+    (a, ra), _ = _enc("sdk_encode", x, D, rsq=True)
+    (b, rb), _ = _enc("sdk_encode_simt", x, D, rsq=True)
+    assert torch.equal(a.cpu(), b.cpu()) and torch.equal(ra.cpu(), rb.cpu())
+    idx, coef = oracle.unpack_words(words_np(a))
+    assert np.all(idx[0] == 0) and np.all(coef[0] == 0.0)
+    assert idx[1, 0] == 417 and abs(coef[1, 0] - 2.5) < 2e-3
+    assert idx[2, 0] == 20000
+
+
+APPEND_CASES = [
+    # (B, Hkv, n_new, x dtype): K and V in one launch up to 32 vectors each,
+    # two launches up to 64, the tensor-core encoder beyond
+    (1, 8, 1, torch.float32),
+    (4, 8, 1, torch.bfloat16),
+    (3, 3, 3, torch.float32),
+    (5, 8, 1, torch.float32),
+    (2, 8, 5, torch.float32),
+]
+
+
+@pytest.mark.parametrize("case", APPEND_CASES, ids=lambda c: "B%d_H%d_n%d" % c[:3])
+def test_token_append_writes_exact_codes(case):
+    """Per-token append (the decode loop's shape): the encoder writes the
+    words straight into the code store at lens[b]..lens[b]+n_new-1, the
+    first 3 key words also into the k_lo planes; every word equals the
+    CUDA-core encoder's and nothing else in the store changes."""
+    B, Hkv, n_new, dt = case
+    g = workloads.make_gen(81 + B * Hkv * n_new)
+    n, d, cap = 32768, 128, 40
+    DK = workloads.gaussian_dictionary(n, d, g).cuda()
+    DV = workloads.gaussian_dictionary(n, d, g).cuda()
+    store = sdk.CodeStore(B, Hkv, cap)
+    lens0 = [int(v) for v in torch.randint(0, cap - n_new + 1, (B,), generator=g)]
+    store.lens = list(lens0)
+    for t in (store.k_lo, store.k_full, store.v_full):
+        t.fill_(0x12345)
+    xk = torch.randn(B, Hkv, n_new, d, generator=g).to(dt).cuda()
+    xv = torch.randn(B, Hkv, n_new, d, generator=g).to(dt).cuda()
+    ws = sdk.sdk_append(store, xk, xv, DK, DV)
+    torch.cuda.synchronize()
+    assert sdk.sdk_check_status(ws)[0] == 0
+    assert store.lens == [l + n_new for l in lens0]
+    ck = sdk.sdk_encode_simt(xk, DK).view(B, Hkv, n_new, 16)
+    cv = sdk.sdk_encode_simt(xv, DV).view(B, Hkv, n_new, 16)
+    for b, l0 in enumerate(lens0):
+        assert torch.equal(store.k_full[b, :, l0:l0 + n_new], ck[b])
+        assert torch.equal(store.v_full[b, :, l0:l0 + n_new], cv[b])
+        assert torch.equal(store.k_lo[b, :, :, l0:l0 + n_new],
+                           ck[b, :, :, :3].transpose(-1, -2))
+        for t in (store.k_full, store.v_full):
+            assert torch.all(t[b, :, :l0] == 0x12345)
+            assert torch.all(t[b, :, l0 + n_new:] == 0x12345)
+        assert torch.all(store.k_lo[b, :, :, :l0] == 0x12345)
+        assert torch.all(store.k_lo[b, :, :, l0 + n_new:] == 0x12345)
+    ref = _oracle(xk.float().cpu(), DK.cpu())
+    check_encode(words_np(ck.reshape(-1, 16)), ref)
+
+
+_SMALL_OFF = r"""
+import sys, torch
+sys.path.insert(0, sys.argv[1])
+import workloads, sparse_dictionary_coded_b200 as sdk
+g = workloads.make_gen(91)
+D = workloads.gaussian_dictionary(32768, 128, g).cuda()
+x = torch.randn(24, 128, generator=g).cuda()
+out = []
+for fn in (sdk.sdk_encode, sdk.sdk_encode_simt):
+    ws = sdk.new_workspace(sdk.sdk_encode_workspace_bytes(24, 128, 32768))
+    c, r = fn(x, D, resid_sqnorm=True, workspace=ws)
+    torch.cuda.synchronize()
+    assert sdk.sdk_check_status(ws)[0] == 0
+    out.append((c.cpu(), r.cpu()))
+assert torch.equal(out[0][0], out[1][0]) and torch.equal(out[0][1], out[1][1])
+print("small encoder off: identical")
+"""
+
+
+def test_small_batch_switch_off_uses_tensor_core_encoder():
+    """With SDK_ENCODE_SMALL=0 (read once per process, hence a child
+    process) a 24-vector call runs the tensor-core encoder; its words still
+    equal the CUDA-core encoder's."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, SDK_ENCODE_SMALL="0")
+    r = subprocess.run([sys.executable, "-c", _SMALL_OFF, root], env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "identical" in r.stdout

@@ -241,6 +241,24 @@ def decode_layer(name, layer, device="cpu", n_tokens=None, B=None):
                 Hq=Hq, Hkv=Hkv, d=d, n_atoms=n, n_tokens=N)
 
 
+def append_token(name, layer, device="cpu"):
+    """One generated token of a 32-layer decode workload ('decode32k_b4',
+    'decode256k'): the new K and V vectors of every KV head of its B
+    sequences in one layer ([B, Hkv, 1, d], planted 16-sparse + noise of
+    norm 0.05||x||) and that layer's own dictionaries.  Seed stream apart
+    from decode_layer's, so no context codes are drawn."""
+    w = WORKLOADS[name]
+    gen = make_gen(seed_of(name) * 1000 + 500 + layer, device)
+    d, n, Hkv, B = w["d"], w["n_atoms"], w["Hkv"], w["B"]
+    DK = gaussian_dictionary(n, d, gen, device)
+    DV = gaussian_dictionary(n, d, gen, device)
+    xk, _, _ = planted_vectors(DK, B * Hkv, gen, noise_rel=0.05)
+    xv, _, _ = planted_vectors(DV, B * Hkv, gen, noise_rel=0.05)
+    return dict(DK=DK, DV=DV, xk=xk.view(B, Hkv, 1, d),
+                xv=xv.view(B, Hkv, 1, d), L=w["L"], B=B, Hkv=Hkv, d=d,
+                n_atoms=n)
+
+
 def prefill(device="cpu", n_tokens=None):
     """Workload 'prefill256k_vec': dense Student-t K and V vectors and the
     correlated K and V dictionaries of one layer."""
