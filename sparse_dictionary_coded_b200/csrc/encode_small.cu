@@ -121,6 +121,67 @@ __device__ __forceinline__ ulonglong2 ld_relaxed_v2(const unsigned long long* p)
   return v;
 }
 
+// Maximum over the words of one slot pair from CTAs c0, c0 + cstep, ...:
+// all loads issued at once, each word polled until it carries `tag`
+// (bounded by 1 s and the CTA's abort flag).  False on timeout.
+template <int B>
+__device__ __forceinline__ bool gather_words(const unsigned long long* wb, int c0, int cstep, int G,
+                                             int vr, bool v1, uint32_t tag,
+                                             volatile uint32_t* abort_flag, unsigned long long& mx0,
+                                             unsigned long long& mx1) {
+  for (int cb = c0; cb < G; cb += cstep * B) {
+    ulonglong2 w[B];
+#pragma unroll
+    for (int u = 0; u < B; ++u) {
+      const int c = cb + u * cstep;
+      if (c < G) w[u] = ld_relaxed_v2(wb + (size_t)c * 64 + vr);
+    }
+#pragma unroll
+    for (int u = 0; u < B; ++u) {
+      const int c = cb + u * cstep;
+      if (c >= G) break;
+      ulonglong2 x = w[u];
+      if (word_tag(x.x) != tag || (v1 && word_tag(x.y) != tag)) {
+        const uint64_t t0 = tc::globaltimer();
+        while (true) {
+          x = ld_relaxed_v2(wb + (size_t)c * 64 + vr);
+          if (word_tag(x.x) == tag && (!v1 || word_tag(x.y) == tag)) break;
+          if (*abort_flag || tc::globaltimer() - t0 > tc::kWaitNs) return false;
+          __nanosleep(20);
+        }
+      }
+      mx0 = max(mx0, x.x & ~0xFFFEull);
+      if (v1) mx1 = max(mx1, x.y & ~0xFFFEull);
+    }
+  }
+  return true;
+}
+
+// <r, d> as the CUDA-core encoder computes it: an fp32 FMA chain over
+// k = 0..D-1.  d is atom ai of a 128-atom tile in the swizzled K-major
+// operand layout, r a residual row in shared memory.
+template <int D>
+__device__ __forceinline__ float exact_chain(const uint8_t* base, int ai, const float4* rr) {
+  const uint8_t* row = base + ai * 128;
+  const int sw = ai & 7;
+  float c = 0.0f;
+#pragma unroll
+  for (int kc = 0; kc < D / 8; ++kc) {
+    const uint4 w = *reinterpret_cast<const uint4*>(row + (kc >> 3) * (128 * 128) +
+                                                    (((kc & 7) ^ sw) << 4));
+    const float4 a = rr[2 * kc], b = rr[2 * kc + 1];
+    c = fmaf(a.x, bf16_lo(w.x), c);
+    c = fmaf(a.y, bf16_hi(w.x), c);
+    c = fmaf(a.z, bf16_lo(w.y), c);
+    c = fmaf(a.w, bf16_hi(w.y), c);
+    c = fmaf(b.x, bf16_lo(w.z), c);
+    c = fmaf(b.y, bf16_hi(w.z), c);
+    c = fmaf(b.z, bf16_lo(w.w), c);
+    c = fmaf(b.w, bf16_hi(w.w), c);
+  }
+  return c;
+}
+
 // 2^(127 - e) for the exponent e of max |r| (clamped so the scale and the
 // scaled maximum stay normal): max |r s| in [1, 2) for normal maxima.
 __device__ __forceinline__ float row_scale(uint32_t maxbits) {
@@ -135,8 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap map1, SmallParams p) {
   using C = SCfg<D>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1k(smem_raw);
   float* rT = reinterpret_cast<float*>(smem + C::kOffR);           // [64][D + 4] residual rows
   uint32_t* cand = reinterpret_cast<uint32_t*>(smem + C::kOffCand);
   uint8_t* misc = smem + C::kOffMisc;
@@ -144,10 +204,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned long long* s_best = s_key + kSlots;                                       // 64
   uint64_t* bars = reinterpret_cast<uint64_t*>(s_best + kSlots);                     // 2
   float* s_rn = reinterpret_cast<float*>(bars + 2);                                  // 64
-  uint32_t* s_rmax = reinterpret_cast<uint32_t*>(s_rn + kSlots);                     // 64
-  int* s_pick = reinterpret_cast<int*>(s_rmax + kSlots);                             // 64
-  float* s_coef = reinterpret_cast<float*>(s_pick + kSlots);                         // 64
-  float* s_band = s_coef + kSlots;                                                   // 64
+  uint32_t* s_rmax = reinterpret_cast<uint32_t*>(s_rn + kSlots);                     // 2 x 64
+  float* s_band = reinterpret_cast<float*>(s_rmax + 2 * kSlots);                     // 64
   uint32_t* s_dmax = reinterpret_cast<uint32_t*>(s_band + kSlots);                   // 2
   volatile uint32_t* s_abort = s_dmax + 2;
   volatile uint32_t* s_tmem = s_dmax + 3;
@@ -190,6 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     s_best[tid] = 0ull;
     s_rn[tid] = 0.0f;
     s_rmax[tid] = 0u;
+    s_rmax[kSlots + tid] = 0u;
   }
   __syncthreads();
   tc_fence_after();
@@ -270,43 +329,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // exact correlation of residual row vr with slice atom al: the CUDA-core
   // encoder's fp32 FMA chain over k = 0..D-1
   auto chain = [&](int vr, int al) -> float {
-    const uint8_t* base = tile_addr(vr_stream(vr), al / kTileAtoms);
-    const int ai = al % kTileAtoms;
-    const float4* rr = reinterpret_cast<const float4*>(rT + vr * C::kRStride);
-    auto dchunk = [&](int kc) {
-      return *reinterpret_cast<const uint4*>(base + (kc >> 3) * (kTileAtoms * 128) + ai * 128 +
-                                             (((kc & 7) ^ (ai & 7)) << 4));
-    };
-    // loads run two 8-element chunks ahead of the FMA chain, so only the
-    // chain's own latency remains
-    uint4 w0 = dchunk(0), w1 = dchunk(1);
-    float4 p0 = rr[0], q0 = rr[1], p1 = rr[2], q1 = rr[3];
-    float c = 0.0f;
-#pragma unroll
-    for (int kc = 0; kc < D / 8; ++kc) {
-      uint4 w2 = w1;
-      float4 p2 = p1, q2 = q1;
-      if (kc + 2 < D / 8) {
-        w2 = dchunk(kc + 2);
-        p2 = rr[2 * kc + 4];
-        q2 = rr[2 * kc + 5];
-      }
-      c = fmaf(p0.x, bf16_lo(w0.x), c);
-      c = fmaf(p0.y, bf16_hi(w0.x), c);
-      c = fmaf(p0.z, bf16_lo(w0.y), c);
-      c = fmaf(p0.w, bf16_hi(w0.y), c);
-      c = fmaf(q0.x, bf16_lo(w0.z), c);
-      c = fmaf(q0.y, bf16_hi(w0.z), c);
-      c = fmaf(q0.z, bf16_lo(w0.w), c);
-      c = fmaf(q0.w, bf16_hi(w0.w), c);
-      w0 = w1;
-      p0 = p1;
-      q0 = q1;
-      w1 = w2;
-      p1 = p2;
-      q1 = q2;
-    }
-    return c;
+    return exact_chain<D>(tile_addr(vr_stream(vr), al / kTileAtoms), al % kTileAtoms,
+                          reinterpret_cast<const float4*>(rT + vr * C::kRStride));
   };
   // word pairs (two adjacent slots) per CTA that hold valid rows
   const int np0 = (p.m[0] + 1) >> 1, np1 = dual ? (p.m[1] + 1) >> 1 : 0;
@@ -316,58 +340,66 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int np_pad = 1 << lg_np;   // <= 32
   const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + tw * 64;
 
+  // bf16(r s) of 8 residual components into row vr's B operand; returns
+  // their sum of squares
+  auto put_b = [&](int vr, int c, const float4& x0, const float4& x1, float sc) -> float {
+    const float v[8] = {x0.x * sc, x0.y * sc, x0.z * sc, x0.w * sc,
+                        x1.x * sc, x1.y * sc, x1.z * sc, x1.w * sc};
+    uint32_t w[4];
+    float sq = 0.0f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * u], v[2 * u + 1]);
+      w[u] = *reinterpret_cast<const uint32_t*>(&h);
+      sq = fmaf(v[2 * u], v[2 * u], sq);
+      sq = fmaf(v[2 * u + 1], v[2 * u + 1], sq);
+    }
+    const int s = vr_stream(vr), row = vr_row(vr);
+    const int kb = c >> 3, c16 = c & 7;
+    *reinterpret_cast<uint4*>(smem + C::kOffB + s * C::kBBytes + kb * (kSlots * 128) + row * 128 +
+                              ((c16 ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+    return sq;
+  };
+  // step 0's B operand: r = x, scale from max |x|
+  for (int e = tid; e < (D / 8) << lg_nv; e += kThreads) {
+    const int vi = e & (nv_pad - 1), c = e >> lg_nv;
+    if (vi >= nvalid) continue;
+    const int vr = slot_of(vi);
+    const float4* r4 = reinterpret_cast<const float4*>(rT + vr * C::kRStride + 8 * c);
+    atomicAdd(&s_rn[vr], put_b(vr, c, r4[0], r4[1], row_scale(s_rmax[vr])));
+  }
+  fence_proxy_async();
+  __syncthreads();
+
+  // Per step j: s_rmax[j & 1] = max |r_j| (r_j's zero test; the scale of
+  // r_{j+1}'s operand), s_rn = ||r_j s||^2 of the operand in B.
   for (int j = 0; j < p.k_atoms && !*s_abort; ++j) {
     const int buf = j & 1;
     const uint32_t tag = (uint32_t)(j + 1);
-    // 1. B operand: bf16(r s) per valid row; ||r s||^2
-    for (int e = tid; e < (D / 8) << lg_nv; e += kThreads) {
-      const int vi = e & (nv_pad - 1), c = e >> lg_nv;
-      if (vi >= nvalid) continue;
-      const int vr = slot_of(vi);
-      const float sc = row_scale(s_rmax[vr]);
-      const float4 x0 = *reinterpret_cast<const float4*>(rT + vr * C::kRStride + 8 * c);
-      const float4 x1 = *reinterpret_cast<const float4*>(rT + vr * C::kRStride + 8 * c + 4);
-      const float v[8] = {x0.x * sc, x0.y * sc, x0.z * sc, x0.w * sc,
-                          x1.x * sc, x1.y * sc, x1.z * sc, x1.w * sc};
-      uint32_t w[4];
-      float sq = 0.0f;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * u], v[2 * u + 1]);
-        w[u] = *reinterpret_cast<const uint32_t*>(&h);
-        sq = fmaf(v[2 * u], v[2 * u], sq);
-        sq = fmaf(v[2 * u + 1], v[2 * u + 1], sq);
-      }
-      const int s = vr_stream(vr), row = vr_row(vr);
-      const int kb = c >> 3, c16 = c & 7;
-      *reinterpret_cast<uint4*>(smem + C::kOffB + s * C::kBBytes + kb * (kSlots * 128) + row * 128 +
-                                ((c16 ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-      atomicAdd(&s_rn[vr], sq);
-    }
-    fence_proxy_async();
-    __syncthreads();
-    // 2. correlations of the slice with all rows
+    const uint32_t* rmax = s_rmax + buf * kSlots;
+    uint32_t* rmax_next = s_rmax + (buf ^ 1) * kSlots;
+    // 1. correlations of the slice with all rows; meanwhile each row's band
     if (tid == 0) {
       tc_fence_after();
       for (int s = 0; s < ns; ++s) {
         const int N = s == 0 ? N0 : N1;
         const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
                                ((uint32_t)(kTileAtoms >> 4) << 24);
-        const uint32_t bbase = smem_u32(smem + C::kOffB + s * C::kBBytes);
+        const uint64_t bdesc = smem_desc(smem_u32(smem + C::kOffB + s * C::kBBytes));
         for (int t = 0; t < tiles; ++t) {
-          const uint32_t abase = smem_u32(tile_addr(s, t));
+          const uint64_t adesc = smem_desc(smem_u32(tile_addr(s, t)));
 #pragma unroll
           for (int ks = 0; ks < C::KSTEPS; ++ks) {
+            // descriptor start addresses advance in 16-byte units
             const uint32_t aoff = (ks >> 2) * (kTileAtoms * 128) + (ks & 3) * 32;
             const uint32_t boff = (ks >> 2) * (kSlots * 128) + (ks & 3) * 32;
-            tc_mma(tmem + t * 64 + s * 32, smem_desc(abase + aoff), smem_desc(bbase + boff), idesc,
+            tc_mma(tmem + t * 64 + s * 32, adesc + (aoff >> 4), bdesc + (boff >> 4), idesc,
                    ks > 0 ? 1u : 0u);
           }
         }
       }
       tc_commit(bar_mma);
     }
-    // the candidate band of every row (while the MMAs run)
     if (tid < kSlots && vr_valid(tid))
       s_band[tid] = 0.0078125f * sqrtf(s_rn[tid]) * __uint_as_float(s_dmax[vr_stream(tid)]) * 1.01f +
                     7.7e-34f;
@@ -378,7 +410,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (*s_abort) break;
     tc_fence_after();
-    // 3. per warp (32 atoms, one per lane) and row: the largest |c~|, every
+    // state for the exchange and the fused update of this step
+    if (tid < kSlots) {
+      s_best[tid] = 0ull;
+      s_rn[tid] = 0.0f;
+      rmax_next[tid] = 0u;
+    }
+    // 2. per warp (32 atoms, one per lane) and row: the largest |c~|, every
     // atom not provably below it (|c~| >= max - band) into the warp's list,
     // then the list re-scored exactly, one entry per lane.  Rows are taken 16
     // accumulator columns at a time.
@@ -392,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // rows of the group to scan (valid and not zero) and their bands,
         // lane u holding row u's
         const int vr_l = cg * 16 + (lane & 15);
-        const bool row_l = vr_valid(vr_l) && s_rmax[vr_l] != 0u;
+        const bool row_l = vr_valid(vr_l) && rmax[vr_l] != 0u;
         const float band_l = s_band[vr_l];
         const uint32_t rows = __ballot_sync(0xffffffffu, row_l) & 0xFFFFu;
         int cnt = 0;
@@ -422,10 +460,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc_fence_before();
     // a zero row: every chain gives +0, the slice's first atom wins
-    if (tid < kSlots && vr_valid(tid) && s_rmax[tid] == 0u)
+    if (tid < kSlots && vr_valid(tid) && rmax[tid] == 0u)
       atomicMax(&s_key[tid], win_word(0.0f, (uint32_t)a0));
     __syncthreads();
-    // 4. publish the slice winners, then take the maximum over all slices:
+    // 3. publish the slice winners, then take the maximum over all slices:
     // 16-byte loads of two adjacent slots' words, polled until every valid
     // one carries this step's tag
     unsigned long long* wb = p.words + (size_t)buf * G * kSlots;
@@ -440,36 +478,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int vr = pr < np0 ? 2 * pr : 32 + 2 * (pr - np0);
         const bool v1 = vr_valid(vr + 1);
         const int cstep = kThreads >> lg_np;
+        const int c0 = tid >> lg_np;
         unsigned long long mx0 = 0ull, mx1 = 0ull;
-        for (int c0 = tid >> lg_np; ok && c0 < G; c0 += cstep * kBatch) {
-          ulonglong2 w[kBatch];
-#pragma unroll
-          for (int u = 0; u < kBatch; ++u) {
-            const int c = c0 + u * cstep;
-            if (c < G) w[u] = ld_relaxed_v2(wb + (size_t)c * kSlots + vr);
-          }
-#pragma unroll
-          for (int u = 0; u < kBatch; ++u) {
-            const int c = c0 + u * cstep;
-            if (c >= G) break;
-            ulonglong2 x = w[u];
-            if (word_tag(x.x) != tag || (v1 && word_tag(x.y) != tag)) {
-              const uint64_t t0 = globaltimer();
-              while (true) {
-                x = ld_relaxed_v2(wb + (size_t)c * kSlots + vr);
-                if (word_tag(x.x) == tag && (!v1 || word_tag(x.y) == tag)) break;
-                if (*s_abort || globaltimer() - t0 > kWaitNs) {
-                  ok = false;
-                  break;
-                }
-                __nanosleep(20);
-              }
-              if (!ok) break;
-            }
-            mx0 = max(mx0, x.x & ~0xFFFEull);
-            if (v1) mx1 = max(mx1, x.y & ~0xFFFEull);
-          }
-        }
+        if (cstep * 4 >= G)
+          ok = gather_words<4>(wb, c0, cstep, G, vr, v1, tag, s_abort, mx0, mx1);
+        else
+          ok = gather_words<kBatch>(wb, c0, cstep, G, vr, v1, tag, s_abort, mx0, mx1);
         if (mx0) atomicMax(&s_best[vr], mx0);
         if (mx1) atomicMax(&s_best[vr + 1], mx1);
       }
@@ -480,65 +494,57 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
     if (*s_abort) break;
-    // pick and coefficient; per-step state back to zero
-    if (tid < kSlots) {
-      const unsigned long long w = s_best[tid];
-      if (vr_valid(tid)) {
-        if (w & 1ull) {
-          s_pick[tid] = (int)(0x7FFFu - (uint32_t)((w >> 17) & 0x7FFFu));
-          const float a = __uint_as_float((uint32_t)(w >> 32));
-          s_coef[tid] = ((w >> 16) & 1ull) ? -a : a;
-        } else {
-          // every |c| NaN: atom 0 with coefficient 0, as the CUDA-core scan
-          s_pick[tid] = 0;
-          s_coef[tid] = 0.0f;
-        }
-      }
-      s_key[tid] = 0ull;
-      s_rn[tid] = 0.0f;
-      s_rmax[tid] = 0u;
-    }
-    __syncthreads();
-    if (tid < kSlots) s_best[tid] = 0ull;
-    // 5. residual update (identical in every CTA): 8 components per thread
+    // 4. pick and coefficient of every row (read by every thread of the row
+    // from the maximum word), r_{j+1} = fmaf(-coef, d, r_j) in fp32 (the
+    // same in every CTA), and r_{j+1}'s operand scaled as r_j's maximum
+    // asks (|r_{j+1} s| <= ||r_j s|| <= 2 sqrt(D): no overflow)
+    if (tid < kSlots) s_key[tid] = 0ull;
     for (int e = tid; e < (D / 8) << lg_nv; e += kThreads) {
       const int vi = e & (nv_pad - 1), c = e >> lg_nv;
       if (vi >= nvalid) continue;
       const int vr = slot_of(vi);
       const int s = vr_stream(vr);
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(p.dict[s] + (int64_t)s_pick[vr] * D) + c);
-      const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-      const float cf = s_coef[vr];
+      const unsigned long long bw = s_best[vr];
+      int pick = 0;
+      float cf = 0.0f;   // every |c| NaN: atom 0 with coefficient 0, as the CUDA-core scan
+      if (bw & 1ull) {
+        pick = (int)(0x7FFFu - (uint32_t)((bw >> 17) & 0x7FFFu));
+        const float a = __uint_as_float((uint32_t)(bw >> 32));
+        cf = ((bw >> 16) & 1ull) ? -a : a;
+      }
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(p.dict[s] + (int64_t)pick * D) + c);
       float4* r4 = reinterpret_cast<float4*>(rT + vr * C::kRStride + 8 * c);
       float4 x0 = r4[0], x1 = r4[1];
-      x0.x = fmaf(-cf, bf16_lo(wv[0]), x0.x);
-      x0.y = fmaf(-cf, bf16_hi(wv[0]), x0.y);
-      x0.z = fmaf(-cf, bf16_lo(wv[1]), x0.z);
-      x0.w = fmaf(-cf, bf16_hi(wv[1]), x0.w);
-      x1.x = fmaf(-cf, bf16_lo(wv[2]), x1.x);
-      x1.y = fmaf(-cf, bf16_hi(wv[2]), x1.y);
-      x1.z = fmaf(-cf, bf16_lo(wv[3]), x1.z);
-      x1.w = fmaf(-cf, bf16_hi(wv[3]), x1.w);
+      x0.x = fmaf(-cf, bf16_lo(w.x), x0.x);
+      x0.y = fmaf(-cf, bf16_hi(w.x), x0.y);
+      x0.z = fmaf(-cf, bf16_lo(w.y), x0.z);
+      x0.w = fmaf(-cf, bf16_hi(w.y), x0.w);
+      x1.x = fmaf(-cf, bf16_lo(w.z), x1.x);
+      x1.y = fmaf(-cf, bf16_hi(w.z), x1.y);
+      x1.z = fmaf(-cf, bf16_lo(w.w), x1.z);
+      x1.w = fmaf(-cf, bf16_hi(w.w), x1.w);
       r4[0] = x0;
       r4[1] = x1;
       const float m8 = fmaxf(fmaxf(fmaxf(fabsf(x0.x), fabsf(x0.y)), fmaxf(fabsf(x0.z), fabsf(x0.w))),
                              fmaxf(fmaxf(fabsf(x1.x), fabsf(x1.y)), fmaxf(fabsf(x1.z), fabsf(x1.w))));
-      // NaN components: the row is degenerate; keep the scale of the rest
-      if (m8 > 0.0f) atomicMax(&s_rmax[vr], __float_as_uint(m8));
-    }
-    if (g == 0 && tid < kSlots && vr_valid(tid)) {
-      const int s = vr_stream(tid), i = vr_row(tid);
-      const uint32_t word = make_word(s_coef[tid], (uint32_t)s_pick[tid]);
-      if (!p.append) {
-        p.codes[s][(int64_t)i * p.k_atoms + j] = word;
-      } else {
-        const int bk = i / p.n_new;
-        const int64_t t = (int64_t)p.lens[bk / p.Hkv] + i % p.n_new;
-        p.codes[s][((int64_t)bk * p.cap + t) * kAtoms + j] = word;
-        if (p.lo[s] != nullptr && j < kLoPlanes)
-          p.lo[s][((int64_t)bk * kLoPlanes + j) * p.cap + t] = word;
+      // NaN components: the row is degenerate; the rest sets the scale
+      if (m8 > 0.0f) atomicMax(&rmax_next[vr], __float_as_uint(m8));
+      atomicAdd(&s_rn[vr], put_b(vr, c, x0, x1, row_scale(rmax[vr])));
+      if (c == 0 && g == 0) {
+        const int i = vr_row(vr);
+        const uint32_t word = make_word(cf, (uint32_t)pick);
+        if (!p.append) {
+          p.codes[s][(int64_t)i * p.k_atoms + j] = word;
+        } else {
+          const int bk = i / p.n_new;
+          const int64_t t = (int64_t)p.lens[bk / p.Hkv] + i % p.n_new;
+          p.codes[s][((int64_t)bk * p.cap + t) * kAtoms + j] = word;
+          if (p.lo[s] != nullptr && j < kLoPlanes)
+            p.lo[s][((int64_t)bk * kLoPlanes + j) * p.cap + t] = word;
+        }
       }
     }
+    fence_proxy_async();
     __syncthreads();
   }
   if (g == 0 && !*s_abort && tid < kSlots && vr_valid(tid)) {

@@ -152,8 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     encode_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1k(smem_raw);
   uint32_t* s_cw = reinterpret_cast<uint32_t*>(smem + C::kOffCw);
   float* s_best = reinterpret_cast<float*>(smem + C::kOffBest);
   uint32_t* s_cnt = reinterpret_cast<uint32_t*>(smem + C::kOffCnt);

@@ -56,8 +56,7 @@ template <int D>
 __global__ void __launch_bounds__(kOThreads, 1) out_tc_kernel(DecodeParams p) {
   using C = OCfg<D>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1k(smem_raw);
   const uint32_t bar = smem_u32(smem + C::kOffBar);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile uint32_t* s_tmem = misc;

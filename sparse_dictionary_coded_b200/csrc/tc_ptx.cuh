@@ -14,6 +14,13 @@ constexpr unsigned long long kWaitNs = 1000000000ull;   // bounded waits: 1 s
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+// First 1024-byte aligned byte of a dynamic shared-memory array (the
+// 128-byte swizzle atoms need it).  Computed as an offset added to the array
+// itself, so the compiler still knows every access through the result is a
+// shared-memory access (casting through an integer would make them generic).
+__device__ __forceinline__ uint8_t* align_smem_1k(uint8_t* raw) {
+  return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

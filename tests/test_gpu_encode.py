@@ -129,17 +129,18 @@ def test_tensor_core_and_simt_agree_exactly():
 def test_candidate_overflow_falls_back_to_exact_scan():
     """Twelve identical atoms tie for the first pick: the tensor-core
     encoder's candidate list overflows, the row is re-scanned exactly, and
-    the pick is the lowest of the tied indices (counted in the header)."""
+    the pick is the lowest of the tied indices (counted in the header).
+    80 vectors: more than the small-batch encoder takes."""
     g = workloads.make_gen(41)
     n, d = 512, 64
     D = workloads.gaussian_dictionary(n, d, g)
     D[20:32] = D[300]
-    x = 3.0 * D[300].float()[None, :].repeat(40, 1)
-    x += 0.01 * torch.randn(40, d, generator=g)
+    x = 3.0 * D[300].float()[None, :].repeat(80, 1)
+    x += 0.01 * torch.randn(80, d, generator=g)
     (codes, _), hdr = _enc("sdk_encode", x, D, rsq=True)
     idx, _ = oracle.unpack_words(words_np(codes))
     assert np.all(idx[:, 0] == 20)
-    assert hdr[2] >= 40                 # rows re-scanned exactly
+    assert hdr[2] >= 80                 # rows re-scanned exactly
     ref = _oracle(x, D)
     check_encode(words_np(codes), ref)
     b = _enc("sdk_encode_simt", x, D)[0]
