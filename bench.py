@@ -405,6 +405,27 @@ def bench_decode(args, world, rank, pk, name):
     ms, ck = timed_steps(g.replay, args.steps, args.warmup, flush, world, clocks)
     # serialised-layer variant without the graph, for reference
     ms_nog, _ = timed_steps(step, max(2, args.steps // 2), 1, flush, world)
+    e2e = None
+    if not args.no_e2e:
+        # through the public API with host buffers: every layer's queries
+        # copied in from pinned memory, the step replayed, every layer's
+        # output read back
+        hq = [ly["q"].cpu().pin_memory() for ly in layers]
+        hout = torch.empty(len(layers), B, Hq, d).pin_memory()
+
+        def e2e_step():
+            for ly, h in zip(layers, hq):
+                ly["q"].copy_(h, non_blocking=True)
+            g.replay()
+            for l, ly in enumerate(layers):
+                hout[l].copy_(ly["out"], non_blocking=True)
+
+        ms_e, _ = timed_steps(e2e_step, max(2, args.steps // 2), 1, flush, world)
+        t = max_over_ranks(statistics.mean(ms_e), world)
+        e2e = {"value": world * B * N / (t * 1e-3), "unit": "ctx tokens/s/step",
+               "ms_per_step": t,
+               "h2d_bytes_per_step": sum(h.numel() * 4 for h in hq),
+               "d2h_bytes_per_step": hout.numel() * 4}
     for ly in layers:
         rc, _ = sdk.sdk_check_status(ly["ws"])
         assert rc == 0, "device check failed in decode"
@@ -433,6 +454,7 @@ def bench_decode(args, world, rank, pk, name):
                          % (L * B * Hkv * N * 140 / 1e9)},
         "dtype": "f32 (bf16 dictionaries, fp16 coefficients)",
         "gpu_launches": args.steps * L * DEC_KERNELS_PER_LAYER,
+        **({"e2e": e2e} if e2e else {}),
     }
 
 
@@ -461,6 +483,28 @@ def bench_prefill(args, world, rank, pk):
     rc, hdr = sdk.sdk_check_status(ws)
     assert rc == 0
     step_ms = max_over_ranks(statistics.mean(ms), world)
+    e2e = None
+    if not args.no_e2e:
+        # host vectors in (pinned), codes back out, every step
+        hxk, hxv = xk.cpu().pin_memory(), xv.cpu().pin_memory()
+        hck = torch.empty(ck_.shape, dtype=ck_.dtype).pin_memory()
+        hcv = torch.empty(cv_.shape, dtype=cv_.dtype).pin_memory()
+        dxk, dxv = torch.empty_like(xk), torch.empty_like(xv)
+
+        def e2e_step():
+            dxk.copy_(hxk, non_blocking=True)
+            dxv.copy_(hxv, non_blocking=True)
+            sdk.sdk_encode(dxk, w["DK"], codes=ck_, workspace=ws)
+            sdk.sdk_encode(dxv, w["DV"], codes=cv_, workspace=ws)
+            hck.copy_(ck_, non_blocking=True)
+            hcv.copy_(cv_, non_blocking=True)
+
+        ms_e, _ = timed_steps(e2e_step, max(2, args.steps // 2), 1, flush, world)
+        t = max_over_ranks(statistics.mean(ms_e), world)
+        e2e = {"value": world * 2 * nv / (t * 1e-3), "unit": "encoded KV vecs/s",
+               "ms_per_step": t,
+               "h2d_bytes_per_step": (hxk.numel() + hxv.numel()) * 4,
+               "d2h_bytes_per_step": (hck.numel() + hcv.numel()) * 4}
     flops = 2 * nv * enc_flop_per_vector(n, d)
     tfl = flops / (step_ms * 1e-3) / 1e12
     return {
@@ -475,6 +519,7 @@ def bench_prefill(args, world, rank, pk):
         "dtype": ENC_DTYPE,
         "gpu_launches": args.steps * 2 * ENC_KERNELS_PER_CALL,
         "enc_fallback_rows": hdr[2],
+        **({"e2e": e2e} if e2e else {}),
     }
 
 
