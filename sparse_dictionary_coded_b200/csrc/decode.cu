@@ -895,18 +895,19 @@ __device__ __forceinline__ void for_records(const int32_t* list, int e0, int e1,
   // (two and four iterations later); out-of-range tokens are caught there
   auto list_at = [&](int i) -> int { return i < e1 ? __ldg(list + i) : -1; };
   auto ok = [&](int t) { return (unsigned)t < (unsigned)Nb; };
+  // records sit at random token positions: both the copies and the L2
+  // prefetch ask for exactly the record's 64 bytes, not its 128-byte line
   auto issue = [&](int t, int slot) {
     const bool v = ok(t);
     const uint4* a = rec + (int64_t)(v ? t : 0) * 4;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) cp_async16(ring + (slot * T + tid) * 4 + (u ^ sw), a + u, v);
+    for (int u = 0; u < 4; ++u) cp_async16_64B(ring + (slot * T + tid) * 4 + (u ^ sw), a + u, v);
     cp_async_commit();
   };
   auto prefetch = [&](int t) {
     if (ok(t)) {
       const uint4* a = rec + (int64_t)t * 4;
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(a + 2));
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], 64;" ::"l"(a) : "memory");
     }
   };
   int i = e0 + tid;
@@ -1332,6 +1333,7 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
                          out_smem_bytes(128, 2, 4));
     cudaFuncSetAttribute(out_kernel<64, 2, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          out_smem_bytes(64, 2, 4));
+
     cudaFuncSetAttribute(attend_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kAttSmem);
     cudaFuncSetAttribute(attend_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1403,13 +1405,15 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
     if (st != SDK_OK) return st;
   }
   if (!out_tc) {
-    const size_t sm = out_smem_bytes(p.d, gv_rb, gv_tiles);
-    if (p.d == 128) {
-      e = wide ? launch_pdl(out_kernel<128, 2, 4>, gv_grid, dim3(256), sm, stream, 1, p)
-               : launch_pdl(out_kernel<128, 1, 1>, gv_grid, dim3(128), sm, stream, 1, p);
+    if (wide) {
+      const size_t sm = out_smem_bytes(p.d, gv_rb, gv_tiles);
+      e = p.d == 128 ? launch_pdl(out_kernel<128, 2, 4>, gv_grid, dim3(256), sm, stream, 1, p)
+                     : launch_pdl(out_kernel<64, 2, 4>, gv_grid, dim3(128), sm, stream, 1, p);
     } else {
-      e = wide ? launch_pdl(out_kernel<64, 2, 4>, gv_grid, dim3(128), sm, stream, 1, p)
-               : launch_pdl(out_kernel<64, 1, 1>, gv_grid, dim3(64), sm, stream, 1, p);
+      // up to 32 rows: 64 atoms per CTA (measured faster than 128 or 256)
+      const size_t sm = out_smem_bytes(p.d, 1, 1);
+      e = p.d == 128 ? launch_pdl(out_kernel<128, 1, 1>, gv_grid, dim3(128), sm, stream, 1, p)
+                     : launch_pdl(out_kernel<64, 1, 1>, gv_grid, dim3(64), sm, stream, 1, p);
     }
     if (e != cudaSuccess) return SDK_ERR_CUDA;
   }

@@ -115,6 +115,14 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, boo
                "r"(valid ? 16 : 0)
                : "memory");
 }
+// The same with the L2 prefetch size limited to 64 bytes (for 64-byte
+// records at scattered addresses).
+__device__ __forceinline__ void cp_async16_64B(void* smem_dst, const void* gsrc, bool valid) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(smem_dst);
+  asm volatile("cp.async.cg.shared.global.L2::64B [%0], [%1], 16, %2;" ::"r"(d), "l"(gsrc),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
