@@ -19,6 +19,9 @@ encode   greedy pursuit (the projection-based replacement for OMP), the
 decode   decode attention with query-aware hierarchical sparsity, written
          as the plain definition over decoded key/value vectors.
 certify  replay of someone else's codes in fp64: checks every greedy pick.
+omp      orthogonal matching pursuit (least-squares refit at every step), the
+         encoder the pages replace; only for measuring what the greedy
+         pursuit gives up (``python -m oracle.compare_omp``).
 
 Pins: every function here is checked in ``tests/test_oracle_*.py`` against
 facts fixed by the pages or by mathematics (brute force on tiny inputs,
@@ -32,9 +35,11 @@ from .encode import (FP16_MAX, greedy_pursuit, encode_ref, store_coef_fp16,
 from .decode import (topk_count, select_top, decode_attn_ref,
                      decode_head_ref, decode_vectors)
 from .certify import certify_codes
+from .omp import omp, omp_ref
 
 __all__ = [
     "FP16_MAX", "greedy_pursuit", "encode_ref", "store_coef_fp16",
     "pack_words", "unpack_words", "topk_count", "select_top",
     "decode_attn_ref", "decode_head_ref", "decode_vectors", "certify_codes",
+    "omp", "omp_ref",
 ]
