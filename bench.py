@@ -75,6 +75,11 @@ def parse():
                     help="decode workloads: layers to instantiate (default: "
                          "the workload's 32); fewer layers make small ncu "
                          "captures and are recorded in config.layers")
+    ap.add_argument("--int-softmax", action="store_true",
+                    help="decode workloads: integer softmax (token-wise INT16 "
+                         "logits, integer exponential); recorded in config")
+    ap.add_argument("--full-softmax", action="store_true",
+                    help="decode workloads: softmax over every token")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -388,7 +393,9 @@ def bench_decode(args, world, rank, pk, name):
     def step():
         for ly in layers:
             sdk.sdk_decode_attn(ly["q"], ly["DK"], ly["DV"], ly["store"],
-                                out=ly["out"], workspace=ly["ws"])
+                                out=ly["out"], workspace=ly["ws"],
+                                full_softmax=args.full_softmax,
+                                int_softmax=args.int_softmax)
 
     # capture the 32 layer calls in one CUDA graph
     s = torch.cuda.Stream()
@@ -433,7 +440,7 @@ def bench_decode(args, world, rank, pk, name):
     lay = sdk.sdk_decode_layout_of(B, Hq, d, n, N)
     k = (N + 9) // 10
     code_bytes, U = union_bytes(sdk, [ly["ws"] for ly in layers], lay, B, Hq,
-                                Hkv, N, k, False)
+                                Hkv, N, k, args.full_softmax)
     alg = code_bytes + L * 2 * n * d * 2
     gbs = alg / (step_ms * 1e-3) / 1e9
     return {
@@ -450,6 +457,9 @@ def bench_decode(args, world, rank, pk, name):
         "config": {"workload": name, "layers": L, "B": B, "Hq": Hq,
                    "Hkv": Hkv, "head_dim": d, "n_atoms": n, "n_tokens": N,
                    "klow": 3, "khigh": 16, "top": "1/10",
+                   "softmax": ("integer (INT16 logits)" if args.int_softmax
+                               else "fp32") + (", all tokens" if args.full_softmax
+                                               else ", selected set"),
                    "l2": "flushed between steps; codes (%.1f GB) exceed L2"
                          % (L * B * Hkv * N * 140 / 1e9)},
         "dtype": "f32 (bf16 dictionaries, fp16 coefficients)",

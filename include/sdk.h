@@ -153,6 +153,10 @@ SDK_API sdk_status sdk_append(const void* xk, const void* xv, int32_t x_dtype,
 SDK_API size_t sdk_append_workspace_bytes(int32_t B, int32_t Hkv, int32_t n_new,
                                   int32_t head_dim, int32_t n_atoms);
 
+/* decode flags */
+#define SDK_DECODE_FULL_SOFTMAX 1   /* softmax over every token, not only S   */
+#define SDK_DECODE_INT_SOFTMAX 2    /* integer softmax (see sdk_decode_attn)  */
+
 /* ------------------------------------------------------------ decode attn
  * One layer of decode attention for B sequences over their code stores
  * (review Summary: score all tokens at Klow=3, refine the top 10% at
@@ -162,8 +166,18 @@ SDK_API size_t sdk_append_workspace_bytes(int32_t B, int32_t Hkv, int32_t n_new,
  *   S       = the k = ceil(top_num*N/top_den) tokens with the largest s_lo
  *             (ties: lower token index)
  *   s_t     = scale * sum_{j<khigh} c_tj QD[idx_tj]  for t in S
- *   p       = softmax of s over S; with full_softmax != 0 the softmax runs
- *             over all N tokens, t outside S using scale * s_lo_t
+ *   p       = softmax of s over S; with flags & SDK_DECODE_FULL_SOFTMAX the
+ *             softmax runs over all N tokens, t outside S using
+ *             scale * s_lo_t.  With flags & SDK_DECODE_INT_SOFTMAX the
+ *             softmax is integer (review Summary: integer polynomial
+ *             Softmax on token-wise INT16 requantised inputs, bit-shift
+ *             guards against INT32 overflow, fixed-point reciprocals):
+ *             the head's fp32 logits l are requantised to q = rint(l / S),
+ *             S = max|l| / 32767; e = I-BERT's integer exponential of
+ *             (q - max q) >> sh (second-order polynomial on (-ln 2, 0] and
+ *             a shift by the whole multiples of ln 2; sh the smallest shift
+ *             keeping its squares below 2^31); P = (e * floor(2^61 / sum e))
+ *             >> 31, probabilities in Q30.  `state` records sum e and sh.
  *   w[a]    = sum_t p_t sum_j c^V_tj [idx^V_tj == a] (over the softmax domain)
  *   out     = w D_V
  *
@@ -172,6 +186,8 @@ SDK_API size_t sdk_append_workspace_bytes(int32_t B, int32_t Hkv, int32_t n_new,
  *   lens_host  host, int32 [B], 1 <= lens[b] <= cap
  *   klow       1 .. khigh;  khigh  klow .. 16
  *   top_num, top_den   0 < top_num <= top_den
+ *   flags      0, or a combination of SDK_DECODE_FULL_SOFTMAX and
+ *              SDK_DECODE_INT_SOFTMAX (other bits: SDK_ERR_INVALID_ARG)
  *   scale      logit scale (1/sqrt(head_dim) for standard attention)
  *   out        device, float [B][Hq][head_dim], 16-byte aligned
  *   workspace  device, >= sdk_decode_workspace_bytes(B, Hq, head_dim,
@@ -186,7 +202,7 @@ SDK_API sdk_status sdk_decode_attn(const float* q, int32_t B, int32_t Hq, int32_
                            const uint32_t* v_full, int64_t cap,
                            const int32_t* lens_host, int32_t klow,
                            int32_t khigh, int32_t top_num, int32_t top_den,
-                           int32_t full_softmax, float scale, float* out,
+                           int32_t flags, float scale, float* out,
                            void* workspace, size_t ws_bytes,
                            sdk_stream_t stream);
 
@@ -231,7 +247,7 @@ SDK_API sdk_status sdk_decode_attn_static(const float* q, int32_t B, int32_t Hq,
                            const uint32_t* k_full, const uint32_t* v_full,
                            int64_t cap, const int32_t* lens_host,
                            int32_t klow, int32_t khigh, int32_t top_num,
-                           int32_t top_den, int32_t full_softmax, float scale,
+                           int32_t top_den, int32_t flags, float scale,
                            float* out, uint32_t* status_out,
                            sdk_stream_t stream);
 
@@ -247,7 +263,7 @@ typedef struct {
   size_t hist2;      /* uint32 [R][4096] bits 19..8 inside the bucket     */
   size_t state;      /* sdk_select_state [R]                              */
   size_t list;       /* int32  [R][L]  the selected tokens at the front
-                        (unordered); with full_softmax the other tokens
+                        (unordered); with SDK_DECODE_FULL_SOFTMAX the other tokens
                         fill the back                                     */
   size_t cand_t;     /* int32  [R][L]  tokens inside the pass-1 bucket    */
   size_t cand_key;   /* uint32 [R][L]  their keys                         */
@@ -274,8 +290,11 @@ typedef struct {
   uint32_t eq_taken;   /* how many of those are in the selected set        */
   uint32_t max_score;  /* key of max s_t over the selected set             */
   uint32_t max_comp;   /* key of the largest s_lo outside it (0 = none)    */
-  float z;             /* softmax denominator                              */
-  uint32_t pad[5];
+  float z;             /* softmax denominator (integer softmax: E, rounded) */
+  uint32_t isoft_sum[2];  /* integer softmax: E = sum of the integer
+                             exponentials, low and high words              */
+  uint32_t isoft_shift;   /* integer softmax: the overflow guard's shift   */
+  uint32_t pad[2];
 } sdk_select_state;
 
 SDK_API sdk_status sdk_decode_layout_of(int32_t B, int32_t Hq, int32_t head_dim,

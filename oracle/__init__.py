@@ -17,7 +17,8 @@ Modules
 encode   greedy pursuit (the projection-based replacement for OMP), the
          fp16 coefficient storage rule and the 32-bit code word format.
 decode   decode attention with query-aware hierarchical sparsity, written
-         as the plain definition over decoded key/value vectors.
+         as the plain definition over decoded key/value vectors; optional
+         integer softmax (token-wise INT16 logits, integer exponential).
 certify  replay of someone else's codes in fp64: checks every greedy pick.
 omp      orthogonal matching pursuit (least-squares refit at every step), the
          encoder the pages replace; only for measuring what the greedy
@@ -33,7 +34,7 @@ figure, whose code bit widths the pages do not give.
 from .encode import (FP16_MAX, greedy_pursuit, encode_ref, store_coef_fp16,
                      pack_words, unpack_words)
 from .decode import (topk_count, select_top, decode_attn_ref,
-                     decode_head_ref, decode_vectors)
+                     decode_head_ref, decode_vectors, integer_softmax)
 from .certify import certify_codes
 from .omp import omp, omp_ref
 
@@ -41,5 +42,5 @@ __all__ = [
     "FP16_MAX", "greedy_pursuit", "encode_ref", "store_coef_fp16",
     "pack_words", "unpack_words", "topk_count", "select_top",
     "decode_attn_ref", "decode_head_ref", "decode_vectors", "certify_codes",
-    "omp", "omp_ref",
+    "omp", "omp_ref", "integer_softmax",
 ]

@@ -24,11 +24,77 @@ atoms" are the first three in greedy pick order; k uses ceil; ties in the
 selection go to the lower token index; the logit scale is 1/sqrt(d) unless
 given; selection is per query head; the full-softmax flag only widens the
 softmax domain.
+
+Integer softmax (optional, ``int_softmax=True``; ``integer_softmax``).  The review's Summary
+says the paper runs Softmax as an integer polynomial approximation on
+inputs requantised to token-wise INT16, with bit-shift guards against INT32
+overflow and fixed-point reciprocals for the divisions; the polynomial is
+not given.  Reading: I-BERT's integer exponential (Kim et al., 2021,
+"I-BERT: Integer-only BERT Quantization"), the published second-order
+polynomial exp(p) ~ 0.3585 (p + 1.353)^2 + 0.344 on p in (-ln 2, 0] with
+exp(x) = 2^-z exp(p), x = p - z ln 2.  Steps for the logits l of one query
+head (fp32, the precision the kernel holds them in):
+  a. S = fp32(max |l|) / 32767 in fp32 (S = 1 if every l is 0);
+     q_t = rint(l_t / S) in fp64, clipped to [-32767, 32767] (a NaN logit
+     maps to -32767): token-wise INT16;
+  b. x_t = (q_t - max q) >> sh (arithmetic shift), sh the smallest shift
+     with q_b^2 + q_c < 2^31 at the scale Sw = S 2^sh (the overflow guard),
+     where q_ln2 = floor(ln 2 / Sw) (at least 1), q_b = floor(1.353 / Sw),
+     q_c = floor(0.344 / (0.3585 Sw^2)), all in fp64;
+  c. z_t = floor(-x_t / q_ln2), p_t = x_t + z_t q_ln2,
+     e_t = ((p_t + q_b)^2 + q_c) >> z_t   (0 when z_t >= 31);
+  d. E = sum_t e_t (int64), recip = floor(2^61 / E),
+     P_t = (e_t recip) >> 31: probabilities in Q30 (P_t / 2^30).
 """
+
+import math
 
 import numpy as np
 
 from .encode import unpack_words
+
+ISOFT_A, ISOFT_B, ISOFT_C = 0.3585, 1.353, 0.344
+LN2 = math.log(2.0)
+
+
+def integer_softmax(logits):
+    """The integer softmax above for one query head's logits (any float
+    array; taken as fp32).  Returns (P int64 Q30 probabilities, E int, sh
+    int)."""
+    l32 = np.asarray(logits, dtype=np.float32)
+    if l32.size == 0:
+        return np.zeros(0, dtype=np.int64), 0, 0
+    finite = l32[np.isfinite(l32)]
+    lmax = np.float32(np.max(np.abs(finite))) if finite.size else np.float32(0.0)
+    S = np.float32(lmax / np.float32(32767.0)) if lmax > 0 else np.float32(1.0)
+    q = np.empty(l32.shape, dtype=np.int64)
+    for t, v in enumerate(l32.tolist()):
+        if v != v:
+            q[t] = -32767
+        else:
+            q[t] = int(min(max(np.rint(float(v) / float(S)), -32767.0), 32767.0))
+    qmax = int(q.max())
+    sh = 0
+    while True:
+        Sw = float(S) * 2.0 ** sh
+        q_ln2 = max(1, int(math.floor(LN2 / Sw)))
+        q_b = int(math.floor(ISOFT_B / Sw))
+        q_c = int(math.floor(ISOFT_C / (ISOFT_A * Sw * Sw)))
+        if q_b * q_b + q_c < 2 ** 31:
+            break
+        sh += 1
+    e = np.zeros(q.shape, dtype=np.int64)
+    for t in range(q.size):
+        x = (int(q[t]) - qmax) >> sh          # Python >> floors, as an arithmetic shift
+        z = (-x) // q_ln2
+        pp = x + z * q_ln2
+        L = (pp + q_b) * (pp + q_b) + q_c
+        assert 0 <= L < 2 ** 31
+        e[t] = L >> z if z < 31 else 0
+    E = int(e.sum())
+    recip = (1 << 61) // E
+    P = np.array([(int(v) * recip) >> 31 for v in e.tolist()], dtype=np.int64)
+    return P, E, sh
 
 
 def topk_count(n_tokens, top_num, top_den):
@@ -76,7 +142,7 @@ def _softmax(z):
 
 def decode_head_ref(q, kwords, vwords, DK, DV, klow=3, khigh=16,
                     top_num=1, top_den=10, full_softmax=False, scale=None,
-                    force_set=None):
+                    force_set=None, int_softmax=False):
     """One query head over one sequence.
 
     q [d]; kwords, vwords [N, 16] uint32 words; DK, DV [n, d].
@@ -110,7 +176,11 @@ def decode_head_ref(q, kwords, vwords, DK, DV, klow=3, khigh=16,
     else:
         logits = s_sel
         domain = sel
-    p = _softmax(logits)
+    if int_softmax:
+        P, E, _ = integer_softmax(logits)
+        p = P.astype(np.float64) / float(1 << 30)
+    else:
+        p = _softmax(logits)
     v_hat = decode_vectors(vwords[domain], DV, 16)
     out = p @ v_hat
     return {"out": out, "s_lo": s_lo, "sel": sel, "p": p, "domain": domain,
@@ -118,7 +188,8 @@ def decode_head_ref(q, kwords, vwords, DK, DV, klow=3, khigh=16,
 
 
 def decode_attn_ref(q, kwords, vwords, DK, DV, lens=None, klow=3, khigh=16,
-                    top_num=1, top_den=10, full_softmax=False, scale=None):
+                    top_num=1, top_den=10, full_softmax=False, scale=None,
+                    int_softmax=False):
     """One layer of decode attention for B sequences.
 
     q [B, Hq, d]; kwords, vwords [B, Hkv, N_max, 16] uint32 (only the first
@@ -141,7 +212,8 @@ def decode_attn_ref(q, kwords, vwords, DK, DV, lens=None, klow=3, khigh=16,
             kvh = h // g
             r = decode_head_ref(q[b, h], kwords[b, kvh, :n_b],
                                 vwords[b, kvh, :n_b], DK, DV, klow, khigh,
-                                top_num, top_den, full_softmax, scale)
+                                top_num, top_den, full_softmax, scale,
+                                int_softmax=int_softmax)
             out[b, h] = r["out"]
             details[(b, h)] = r
     return out, details

@@ -17,7 +17,8 @@ import torch
 
 from . import _capi
 from ._capi import (SDK_OK, SDK_F32, SDK_BF16, MAX_ATOMS, K_ATOMS,
-                    KLOW_PLANES, MAX_BATCH, DecodeLayout, load)
+                    KLOW_PLANES, MAX_BATCH, SDK_DECODE_FULL_SOFTMAX,
+                    SDK_DECODE_INT_SOFTMAX, DecodeLayout, load)
 
 __all__ = [
     "SdkError", "load", "sdk_encode", "sdk_encode_simt", "sdk_append",
@@ -119,6 +120,8 @@ def read_select_state(ws, layout, R):
         col = raw[:, i].clone()
         out[f] = col.view(torch.float32) if f == "z" else (
             col.to(torch.int64) & 0xFFFFFFFF)
+    # integer softmax: the sum of the integer exponentials (int64)
+    out["isoft_sum"] = out["isoft_sum_lo"] | (out["isoft_sum_hi"] << 32)
     return out
 
 
@@ -217,10 +220,11 @@ def sdk_append(store, xk, xv, dict_k, dict_v, workspace=None, stream=None):
 
 def sdk_decode_attn(q, dict_k, dict_v, store, klow=3, khigh=16, top_num=1,
                     top_den=10, full_softmax=False, scale=None, out=None,
-                    workspace=None, stream=None):
+                    workspace=None, stream=None, int_softmax=False):
     """One layer of decode attention.  q [B, Hq, head_dim] fp32.  Returns
     out [B, Hq, head_dim] fp32 (and leaves the intermediate results in the
-    workspace)."""
+    workspace).  full_softmax / int_softmax set SDK_DECODE_FULL_SOFTMAX /
+    SDK_DECODE_INT_SOFTMAX."""
     lib = load()
     q = _cuda_contig(q, "q", (torch.float32,))
     dk = _cuda_contig(dict_k, "dict_k", (torch.bfloat16,))
@@ -240,7 +244,9 @@ def sdk_decode_attn(q, dict_k, dict_v, store, klow=3, khigh=16, top_num=1,
     rc = lib.sdk_decode_attn(_ptr(q), B, Hq, store.Hkv, d, _ptr(dk), _ptr(dv),
                              n_atoms, _ptr(store.k_lo), _ptr(store.k_full),
                              _ptr(store.v_full), store.cap, lens, klow, khigh,
-                             top_num, top_den, 1 if full_softmax else 0,
+                             top_num, top_den,
+                             (SDK_DECODE_FULL_SOFTMAX if full_softmax else 0) |
+                             (SDK_DECODE_INT_SOFTMAX if int_softmax else 0),
                              float(scale), _ptr(out), _ptr(workspace),
                              workspace.numel(), _stream(stream))
     _check(rc, "sdk_decode_attn")

@@ -17,6 +17,7 @@ STATUS_NAMES = {
     6: "SDK_ERR_DEVICE_CHECK",
 }
 SDK_F32, SDK_BF16 = 0, 1
+SDK_DECODE_FULL_SOFTMAX, SDK_DECODE_INT_SOFTMAX = 1, 2
 MAX_ATOMS, K_ATOMS, KLOW_PLANES, MAX_BATCH, WS_ALIGN = 32768, 16, 3, 64, 256
 DECODE_STATIC_WS_BYTES = 16 << 20
 
@@ -59,7 +60,8 @@ class DecodeLayout(ctypes.Structure):
 
 
 SELECT_STATE_FIELDS = ("kth_key", "k", "n_above", "n_cand", "n_sel", "n_comp",
-                       "eq_total", "eq_taken", "max_score", "max_comp", "z")
+                       "eq_total", "eq_taken", "max_score", "max_comp", "z",
+                       "isoft_sum_lo", "isoft_sum_hi", "isoft_shift")
 SELECT_STATE_WORDS = 16
 
 _lib = None

@@ -306,7 +306,7 @@ sdk_status sdk_decode_attn(const float* q, int32_t B, int32_t Hq, int32_t Hkv, i
                            const void* dict_k, const void* dict_v, int32_t n_atoms,
                            const uint32_t* k_lo, const uint32_t* k_full, const uint32_t* v_full,
                            int64_t cap, const int32_t* lens_host, int32_t klow, int32_t khigh,
-                           int32_t top_num, int32_t top_den, int32_t full_softmax, float scale,
+                           int32_t top_num, int32_t top_den, int32_t flags, float scale,
                            float* out, void* workspace, size_t ws_bytes, sdk_stream_t stream) {
   if (B < 1 || B > SDK_MAX_BATCH || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return SDK_ERR_INVALID_ARG;
   if ((int64_t)B * Hq > 2048) return SDK_ERR_INVALID_ARG;
@@ -315,6 +315,7 @@ sdk_status sdk_decode_attn(const float* q, int32_t B, int32_t Hq, int32_t Hkv, i
   if (klow < 1 || khigh < klow || khigh > SDK_K_ATOMS) return SDK_ERR_INVALID_ARG;
   if (top_num < 1 || top_den < 1 || top_num > top_den) return SDK_ERR_INVALID_ARG;
   if (!(scale > 0.0f) || !std::isfinite(scale)) return SDK_ERR_INVALID_ARG;
+  if (flags & ~(SDK_DECODE_FULL_SOFTMAX | SDK_DECODE_INT_SOFTMAX)) return SDK_ERR_INVALID_ARG;
   if (!q || !dict_k || !dict_v || !k_lo || !k_full || !v_full || !out || !lens_host || !workspace)
     return SDK_ERR_INVALID_ARG;
   if (!aligned(workspace, SDK_WS_ALIGN) || !aligned(dict_k, 16) || !aligned(dict_v, 16) ||
@@ -361,7 +362,8 @@ sdk_status sdk_decode_attn(const float* q, int32_t B, int32_t Hq, int32_t Hkv, i
   p.n = n_atoms;
   p.klow = klow;
   p.khigh = khigh;
-  p.full = full_softmax ? 1 : 0;
+  p.full = (flags & SDK_DECODE_FULL_SOFTMAX) ? 1 : 0;
+  p.isoft = (flags & SDK_DECODE_INT_SOFTMAX) ? 1 : 0;
   p.R = B * Hq;
   p.n_out_tiles = (n_atoms + 127) / 128;
   p.scale = scale;

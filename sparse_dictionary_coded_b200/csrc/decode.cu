@@ -163,8 +163,8 @@ __global__ void __launch_bounds__(64 * kGvTiles * RB, (RB > 1 ? 2 : 1)) qd_kerne
       st.max_score = 0u;
       st.max_comp = 0u;
       st.z = 0.0f;
-#pragma unroll
-      for (int u = 0; u < 5; ++u) st.pad[u] = 0u;
+      st.isoft_sum[0] = st.isoft_sum[1] = st.isoft_shift = 0u;
+      st.pad[0] = st.pad[1] = 0u;
       p.st[e] = st;
     }
   }
@@ -957,6 +957,78 @@ __device__ __forceinline__ float block_reduce(float v, float* s_red) {
   return r;
 }
 
+// ---- integer softmax (flag SDK_DECODE_INT_SOFTMAX) ------------------------
+// Logits of one query head requantised to token-wise INT16 (scale S =
+// max |l| / 32767), an integer exponential by I-BERT's second-order
+// polynomial exp(p) ~ 0.3585 (p + 1.353)^2 + 0.344 on (-ln 2, 0] with
+// exp(x) = 2^-z exp(p), a bit-shift guard that keeps the squares inside
+// INT32, an int64 sum and a fixed-point reciprocal (review of "LLM
+// Inference in a Flash!", Summary: integer polynomial Softmax on INT16
+// requantised inputs with bit-shift overflow guards and fixed-point
+// reciprocals; the polynomial is I-BERT's published one).
+struct ISoft {
+  float S;        // INT16 step of the logits
+  int qmax;       // INT16 value of the largest logit
+  int sh;         // right shift of q - qmax (overflow guard)
+  int q_ln2, q_b, q_c;
+};
+
+__device__ __forceinline__ int isoft_q(float l, float S) {
+  if (l != l) return -32767;   // NaN: the lowest INT16 value
+  const double v = rint((double)l / (double)S);
+  return (int)fmin(fmax(v, -32767.0), 32767.0);
+}
+
+// constants for logits whose largest magnitude is lmax and largest value lhi
+__device__ __forceinline__ ISoft isoft_setup(float lmax, float lhi) {
+  ISoft c;
+  c.S = lmax > 0.0f ? lmax / 32767.0f : 1.0f;
+  c.qmax = isoft_q(lhi, c.S);
+  // the smallest shift whose constants keep (p + q_b)^2 + q_c below 2^31
+  // (all in fp64; converted to int only once they fit)
+  for (c.sh = 0;; ++c.sh) {
+    const double sw = ldexp((double)c.S, c.sh);
+    const double qb = floor(1.353 / sw);
+    const double qc = floor(0.344 / (0.3585 * sw * sw));
+    if (qb * qb + qc < 2147483648.0) {
+      const double qln2 = floor(0.6931471805599453 / sw);
+      c.q_ln2 = qln2 < 1.0 ? 1 : (int)qln2;
+      c.q_b = (int)qb;
+      c.q_c = (int)qc;
+      break;
+    }
+  }
+  return c;
+}
+
+// integer exponential of one logit (relative to the largest), < 2^31
+__device__ __forceinline__ uint32_t isoft_exp(float l, const ISoft& c) {
+  const int x = (isoft_q(l, c.S) - c.qmax) >> c.sh;   // <= 0, arithmetic shift
+  const int z = (-x) / c.q_ln2;
+  const int pp = x + z * c.q_ln2;
+  const long long L = (long long)(pp + c.q_b) * (pp + c.q_b) + c.q_c;
+  return z < 31 ? (uint32_t)(L >> z) : 0u;
+}
+
+__device__ __forceinline__ unsigned long long block_sum_u64(unsigned long long v,
+                                                            unsigned long long* s_red64) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) s_red64[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    unsigned long long x = lane < (int)(blockDim.x >> 5) ? s_red64[lane] : 0ull;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    if (lane == 0) s_red64[32] = x;
+  }
+  __syncthreads();
+  const unsigned long long r = s_red64[32];
+  __syncthreads();
+  return r;
+}
+
 template <bool kAll16, bool kCheck>
 __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, int C) {
   pdl_wait();     // nothing global is touched before the previous kernel is done
@@ -967,6 +1039,9 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
   uint4* ring = reinterpret_cast<uint4*>(smem4 + kTable / 4);   // 2 slots x T records
   __shared__ float s_red[33];
   __shared__ float s_val;
+  __shared__ float s_val2;
+  __shared__ unsigned long long s_red64[33];
+  __shared__ unsigned long long s_sum64;
   __shared__ int s_float;
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
@@ -995,6 +1070,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
   stage_table(table, p.qd + (int64_t)r * n, n);
   __syncthreads();
   float smax = -INFINITY, zrun = 0.0f;     // online softmax of this thread
+  float smin = INFINITY;                   // for the integer softmax's scale
   for_records(list, s0, s1, krec, Nb, p.hdr, 0x30000000u | r, ring,
               [&](int i, int t, const uint4 (&w)[4]) {
                 float s = 0.0f;
@@ -1009,6 +1085,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
                 }
                 s *= scale;
                 ss[i] = s;
+                smin = fminf(smin, s);
                 if (s > smax) {
                   zrun = zrun * expf(smax - s) + 1.0f;
                   smax = s;
@@ -1024,22 +1101,60 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
   if (rank == 0 && tid == 0 && m > -INFINITY) st->max_score = score_key(m);
   if (p.full && st->n_comp > 0u) m = fmaxf(m, scale * key_score(st->max_comp));
 
-  // z: the own selected entries (rescaled to m) and complement entries
-  float z = smax > -INFINITY ? zrun * expf(smax - m) : 0.0f;
-#pragma unroll 4
-  for (int i = c0 + tid; i < c1; i += kAttThreads) {
-    const int t = list[i];
-    if ((unsigned)t < (unsigned)Nb) z += expf(scale * key_score(keys[t]) - m);
-  }
-  z = block_reduce<false>(z, s_red);
-  cluster.sync();   // every CTA has read s_val of phase 1
-  if (tid == 0) {
-    s_val = z;
-    s_float = 0;
-  }
-  cluster.sync();
+  const bool isoft = p.isoft != 0;
+  ISoft ic;
+  unsigned long long recip = 0ull, etot = 0ull;
   float ztot = 0.0f;
-  for (int cc = 0; cc < C; ++cc) ztot += *cluster.map_shared_rank(&s_val, cc);
+  if (!isoft) {
+    // z: the own selected entries (rescaled to m) and complement entries
+    float z = smax > -INFINITY ? zrun * expf(smax - m) : 0.0f;
+#pragma unroll 4
+    for (int i = c0 + tid; i < c1; i += kAttThreads) {
+      const int t = list[i];
+      if ((unsigned)t < (unsigned)Nb) z += expf(scale * key_score(keys[t]) - m);
+    }
+    z = block_reduce<false>(z, s_red);
+    cluster.sync();   // every CTA has read s_val of phase 1
+    if (tid == 0) {
+      s_val = z;
+      s_float = 0;
+    }
+    cluster.sync();
+    for (int cc = 0; cc < C; ++cc) ztot += *cluster.map_shared_rank(&s_val, cc);
+  } else {
+    // the smallest logit of the domain (own selected and complement
+    // entries), then the INT16 scale, the integer exponentials and their sum
+#pragma unroll 4
+    for (int i = c0 + tid; i < c1; i += kAttThreads) {
+      const int t = list[i];
+      if ((unsigned)t < (unsigned)Nb) smin = fminf(smin, scale * key_score(keys[t]));
+    }
+    const float mn = -block_reduce<true>(-smin, s_red);
+    cluster.sync();   // every CTA has read s_val of phase 1
+    if (tid == 0) s_val2 = mn;
+    cluster.sync();
+    float lo = INFINITY;
+    for (int cc = 0; cc < C; ++cc) lo = fminf(lo, *cluster.map_shared_rank(&s_val2, cc));
+    const float hi_abs = m > -INFINITY ? fabsf(m) : 0.0f;
+    const float lo_abs = lo < INFINITY ? fabsf(lo) : 0.0f;
+    ic = isoft_setup(fmaxf(hi_abs, lo_abs), m > -INFINITY ? m : 0.0f);
+    unsigned long long e = 0ull;
+    for (int i = s0 + tid; i < s1; i += kAttThreads) e += isoft_exp(ss[i], ic);
+#pragma unroll 4
+    for (int i = c0 + tid; i < c1; i += kAttThreads) {
+      const int t = list[i];
+      if ((unsigned)t < (unsigned)Nb) e += isoft_exp(scale * key_score(keys[t]), ic);
+    }
+    e = block_sum_u64(e, s_red64);
+    if (tid == 0) {
+      s_sum64 = e;
+      s_float = 0;
+    }
+    cluster.sync();
+    for (int cc = 0; cc < C; ++cc) etot += *cluster.map_shared_rank(&s_sum64, cc);
+    recip = etot > 0ull ? (1ull << 61) / etot : 0ull;
+    ztot = (float)etot;
+  }
   const float invz = 1.0f / ztot;
 
   // ---- phase 2: scatter p c^V into the weight tile
@@ -1053,8 +1168,13 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
     // fixed point: p already carries the 2^20 scale
     const float pscale = kFloat ? invz : invz * kFixScale;
     float absum = 0.0f;
+    // integer softmax: P in Q30 from the integer exponential and the
+    // fixed-point reciprocal, then the tile's scale (2^20 or 1)
+    const float qscale = kFloat ? 9.313225746154785e-10f : 9.765625e-4f;   // 2^-30, 2^-10
     auto scatter = [&](float lg, const uint4 (&w)[4]) {
-      const float pt = expf(lg - m) * pscale;
+      const float pt =
+          isoft ? (float)(((unsigned long long)isoft_exp(lg, ic) * recip) >> 31) * qscale
+                : expf(lg - m) * pscale;
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         const uint32_t wd = (u & 3) == 0 ? w[u >> 2].x : (u & 3) == 1 ? w[u >> 2].y
@@ -1118,7 +1238,14 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
     for (int u = 0; u < 4; ++u)
       if (4 * g + u < n) gw[4 * g + u] = sum[u];
   }
-  if (rank == 0 && tid == 0) st->z = ztot;
+  if (rank == 0 && tid == 0) {
+    st->z = ztot;
+    if (isoft) {
+      st->isoft_sum[0] = (uint32_t)etot;
+      st->isoft_sum[1] = (uint32_t)(etot >> 32);
+      st->isoft_shift = (uint32_t)ic.sh;
+    }
+  }
   cluster.sync();
 }
 

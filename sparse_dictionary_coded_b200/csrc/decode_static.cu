@@ -58,7 +58,7 @@ sdk_status sdk_decode_attn_static(const float* q, int32_t B, int32_t Hq, int32_t
                                   int32_t n_atoms, const uint32_t* k_lo, const uint32_t* k_full,
                                   const uint32_t* v_full, int64_t cap, const int32_t* lens_host,
                                   int32_t klow, int32_t khigh, int32_t top_num, int32_t top_den,
-                                  int32_t full_softmax, float scale, float* out,
+                                  int32_t flags, float scale, float* out,
                                   uint32_t* status_out, sdk_stream_t stream) {
   // the lengths decide the workspace size, so they are checked first
   if (lens_host == nullptr || B < 1 || B > SDK_MAX_BATCH || cap < 1) return SDK_ERR_INVALID_ARG;
@@ -76,7 +76,7 @@ sdk_status sdk_decode_attn_static(const float* q, int32_t B, int32_t Hq, int32_t
   sdk_status s = static_workspace(&ws);
   if (s != SDK_OK) return s;
   s = sdk_decode_attn(q, B, Hq, Hkv, head_dim, dict_k, dict_v, n_atoms, k_lo, k_full, v_full, cap,
-                      lens_host, klow, khigh, top_num, top_den, full_softmax, scale, out, ws,
+                      lens_host, klow, khigh, top_num, top_den, flags, scale, out, ws,
                       (size_t)SDK_DECODE_STATIC_WS_BYTES, stream);
   if (s != SDK_OK || status_out == nullptr) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

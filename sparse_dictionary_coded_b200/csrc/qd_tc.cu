@@ -89,8 +89,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
       st.max_score = 0u;
       st.max_comp = 0u;
       st.z = 0.0f;
-#pragma unroll
-      for (int u = 0; u < 5; ++u) st.pad[u] = 0u;
+      st.isoft_sum[0] = st.isoft_sum[1] = st.isoft_shift = 0u;
+      st.pad[0] = st.pad[1] = 0u;
       p.st[e] = st;
     }
   }

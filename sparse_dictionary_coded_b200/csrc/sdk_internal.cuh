@@ -175,7 +175,7 @@ struct DecodeParams {
   WsHeader* hdr;
   int64_t cap;
   int64_t L;
-  int B, Hq, Hkv, g, d, n, klow, khigh, full, R, n_out_tiles;
+  int B, Hq, Hkv, g, d, n, klow, khigh, full, isoft, R, n_out_tiles;
   float scale;
   int lens[kMaxBatch];
   int kcnt[kMaxBatch];

@@ -61,15 +61,33 @@ def _key_to_float(keys):
     return b.view(np.float32)
 
 
+def _isoft_logits(ws, lay, r, k, n_b, full, keys_r, scale):
+    """The fp32 logits the kernel fed its integer softmax for head r: the
+    rescored selected entries (sel_score) and, with the full flag, scale *
+    s_lo of the others (from their keys, in fp32 like the kernel)."""
+    row = lay["row"]
+    ss = ws[lay["sel_score"]:lay["sel_score"] + (r + 1) * row * 4].view(torch.float32)
+    sel = ss.view(r + 1, row)[r, :k].cpu().numpy()
+    if not full:
+        return sel
+    lst = ws[lay["list"]:lay["list"] + (r + 1) * row * 4].view(torch.int32)
+    lst = lst.view(r + 1, row)[r].cpu().numpy()
+    comp = lst[k:n_b]                                # the back of the list
+    lo = _key_to_float(keys_r[comp])
+    return np.concatenate([sel, np.float32(scale) * lo])
+
+
 def _compare(q, DK, DV, kw, vw, lens, klow=3, khigh=16, top_num=1, top_den=10,
-             full=False, heads=None):
+             full=False, heads=None, isoft=False):
     """Runs GPU decode and checks sets, s_lo and outputs against the oracle
-    for the given (b, h) heads (all if None)."""
+    for the given (b, h) heads (all if None).  isoft: integer softmax on
+    both sides, and the kernel's integer sum and guard shift recomputed
+    exactly from its own fp32 logits."""
     B, Hq, d = q.shape
     store = _store(kw, vw, lens)
     out, ws, lay, rc = _run(q, DK, DV, store, klow=klow, khigh=khigh,
                             top_num=top_num, top_den=top_den,
-                            full_softmax=full)
+                            full_softmax=full, int_softmax=isoft)
     assert rc == 0, "device check failed"
     L = max(lens)
     R = B * Hq
@@ -92,7 +110,13 @@ def _compare(q, DK, DV, kw, vw, lens, klow=3, khigh=16, top_num=1, top_den=10,
         assert int(st["n_sel"][r]) == ks[r]
         ref = oracle.decode_head_ref(qn[b, h], kwn[b, kvh, :n_b],
                                      vwn[b, kvh, :n_b], DKn, DVn, klow, khigh,
-                                     top_num, top_den, full)
+                                     top_num, top_den, full, int_softmax=isoft)
+        if isoft:
+            lg = _isoft_logits(ws, lay, r, ks[r], n_b, full, keys[r],
+                               1.0 / math.sqrt(d))
+            _, E, sh = oracle.integer_softmax(lg)
+            assert int(st["isoft_sum"][r]) == E, (r, int(st["isoft_sum"][r]), E)
+            assert int(st["isoft_shift"][r]) == sh
         # s_lo of the GPU within fp32 rounding of the oracle's
         s_gpu = _key_to_float(keys[r, :n_b]).astype(np.float64)
         scale_lo = np.max(np.abs(ref["s_lo"])) + 1e-30
@@ -103,7 +127,7 @@ def _compare(q, DK, DV, kw, vw, lens, klow=3, khigh=16, top_num=1, top_den=10,
             ref = oracle.decode_head_ref(qn[b, h], kwn[b, kvh, :n_b],
                                          vwn[b, kvh, :n_b], DKn, DVn, klow,
                                          khigh, top_num, top_den, full,
-                                         force_set=sets[r])
+                                         force_set=sets[r], int_softmax=isoft)
         err = np.max(np.abs(out[b, h] - ref["out"]))
         assert err <= OUT_TOL, (b, h, err)
         if full:
@@ -213,6 +237,56 @@ def test_klow_and_khigh_variants():
     q, DK, DV, kw, vw, lens = _random_case(12, 2, 8, 4, 700, 128, 4096)
     _compare(q, DK, DV, kw, vw, lens, klow=1, khigh=8, top_num=1, top_den=4)
     _compare(q, DK, DV, kw, vw, lens, klow=5, khigh=16, top_num=3, top_den=10)
+
+
+@pytest.mark.parametrize("full", [False, True])
+def test_integer_softmax(full):
+    """SDK_DECODE_INT_SOFTMAX: token-wise INT16 logits, I-BERT's integer
+    exponential with the overflow guard, fixed-point reciprocal.  Outputs
+    against the oracle's integer softmax; the kernel's integer sum and
+    guard shift equal the oracle's on the kernel's own fp32 logits.  Cases:
+    the tiny workload's oracle-encoded codes, the layer4k shape, a ragged
+    batch, and all tokens tied."""
+    w = workloads.tiny()
+    d, N = w["d"], w["n_tokens"]
+    DKn, DVn = w["DK"].float().double().numpy(), w["DV"].float().double().numpy()
+    rk = oracle.encode_ref(w["xk"].reshape(N, d).double().numpy(), DKn)
+    rv = oracle.encode_ref(w["xv"].reshape(N, d).double().numpy(), DVn)
+    kw = torch.from_numpy(oracle.pack_words(rk["idx"], oracle.store_coef_fp16(rk["coef"]))
+                          .view(np.int32)).view(1, 1, N, 16)
+    vw = torch.from_numpy(oracle.pack_words(rv["idx"], oracle.store_coef_fp16(rv["coef"]))
+                          .view(np.int32)).view(1, 1, N, 16)
+    _compare(_unit(w["q"]), w["DK"], w["DV"], kw, vw, [N], full=full, isoft=True)
+    q, DK, DV, kw, vw, lens = _random_case(78, 1, 32, 8, 4096, 128, 32768)
+    _compare(q, DK, DV, kw, vw, lens, full=full, isoft=True,
+             heads=[(0, h) for h in range(0, 32, 5)])
+    q, DK, DV, kw, vw, _ = _random_case(15, 3, 6, 2, 333, 64, 1000)
+    _compare(q, DK, DV, kw, vw, [1, 5, 333], full=full, isoft=True)
+    g = workloads.make_gen(16)
+    DK = workloads.gaussian_dictionary(512, 64, g)
+    DV = workloads.gaussian_dictionary(512, 64, g)
+    kw = workloads.random_codes((1, 1, 1), 512, g).expand(1, 1, 500, 16).contiguous()
+    vw = workloads.random_codes((1, 1, 500), 512, g)
+    _compare(_unit(workloads.queries(1, 2, 64, g)), DK, DV, kw, vw, [500], full=full,
+             isoft=True)
+
+
+def test_decode_flags_are_checked():
+    """Flag bits other than the two defined ones are rejected before any
+    launch."""
+    q, DK, DV, kw, vw, lens = _random_case(17, 1, 2, 1, 64, 64, 1000)
+    store = _store(kw, vw)
+    lib = sdk.load()
+    import ctypes
+    ws = sdk.new_workspace(sdk.sdk_decode_workspace_bytes(1, 2, 64, 1000, 64))
+    out = torch.empty(1, 2, 64, device="cuda")
+    qd, DKd, DVd = q.cuda(), DK.cuda(), DV.cuda()
+    lens_c = (ctypes.c_int32 * 1)(64)
+    rc = lib.sdk_decode_attn(qd.data_ptr(), 1, 2, 1, 64, DKd.data_ptr(), DVd.data_ptr(), 1000,
+                             store.k_lo.data_ptr(), store.k_full.data_ptr(),
+                             store.v_full.data_ptr(), store.cap, lens_c, 3, 16, 1, 10, 4,
+                             0.125, out.data_ptr(), ws.data_ptr(), ws.numel(), None)
+    assert rc == 1
 
 
 def test_bad_atom_index_is_reported_not_trapped():

@@ -190,3 +190,64 @@ def test_tiny_workload_runs():
     assert w["DK"].dtype == torch.bfloat16
     norms = w["DK"].float().norm(dim=1)
     assert torch.all((norms - 1).abs() < 1e-2)
+
+
+# ---------------------------------------------------------------- integer softmax
+# Pins of oracle.integer_softmax (token-wise INT16 logits, I-BERT's integer
+# exponential, fixed-point reciprocal): against the fp64 softmax, closed
+# forms and the integer invariants.
+
+def _softmax64(x):
+    x = np.asarray(x, dtype=np.float64)
+    e = np.exp(x - x.max())
+    return e / e.sum()
+
+
+def test_integer_softmax_uniform_and_single():
+    for n in (1, 2, 7, 300):
+        for v in (0.0, 3.5, -2.0):
+            P, E, sh = oracle.integer_softmax(np.full(n, v, dtype=np.float32))
+            assert np.all(P == P[0])
+            # each floor loses < 1, the reciprocal's floor < E / 2^31 < n
+            assert (1 << 30) - 2 * n <= int(P.sum()) <= (1 << 30)
+    P, _, _ = oracle.integer_softmax(np.array([1.25], dtype=np.float32))
+    assert (1 << 30) - 1 <= int(P[0]) <= (1 << 30)
+
+
+def test_integer_softmax_close_to_softmax():
+    """The second-order polynomial is within 0.7 % of exp on (-ln 2, 0], so
+    every probability is within about 1.5 % of the fp64 softmax (plus the
+    INT16 rounding of the logits)."""
+    rng = np.random.default_rng(11)
+    for sigma in (0.05, 0.5, 2.0, 8.0):
+        for n in (3, 50, 2000):
+            x = (sigma * rng.standard_normal(n)).astype(np.float32)
+            P, E, sh = oracle.integer_softmax(x)
+            p = P / float(1 << 30)
+            ref = _softmax64(x.astype(np.float64))
+            assert np.all(np.abs(p - ref) <= 0.015 * ref + 2.0 ** -28 + 2e-5 * ref.max())
+            assert abs(p.sum() - 1.0) <= 2 * n * 2.0 ** -30 + 1e-12
+
+
+def test_integer_softmax_two_tokens_ratio():
+    for t in (0.05, 0.3, 1.0, 2.5, 5.0):
+        P, _, _ = oracle.integer_softmax(np.array([0.0, -t], dtype=np.float32))
+        assert abs(P[1] / P[0] / np.exp(-t) - 1.0) <= 0.012
+
+
+def test_integer_softmax_monotone_and_guard():
+    rng = np.random.default_rng(12)
+    x = np.sort(rng.standard_normal(500)).astype(np.float32)
+    P, _, sh = oracle.integer_softmax(x)
+    assert np.all(np.diff(P) >= 0)
+    # small logit ranges engage the bit-shift guard (S = max|l| / 32767 too
+    # fine for INT32 squares); large ones do not
+    assert oracle.integer_softmax(np.array([1e-4, -2e-4], dtype=np.float32))[2] > 0
+    assert oracle.integer_softmax(np.array([3.0, -20.0], dtype=np.float32))[2] == 0
+
+
+def test_integer_softmax_nan_is_lowest():
+    P, _, _ = oracle.integer_softmax(np.array([0.5, np.nan, -0.5], dtype=np.float32))
+    Q, _, _ = oracle.integer_softmax(np.array([0.5, -0.5, -0.5], dtype=np.float32))
+    assert P[1] <= P[2]
+    assert abs(int(P[0]) - int(Q[0])) <= int(Q[0]) // 50
