@@ -422,6 +422,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // accumulator columns at a time.
     if (tw < tiles) {
       uint32_t* wl = cand + warp * kWarpCand;
+      int cnt = 0;
+      // re-score the listed candidates, one entry per lane
+      auto flush = [&]() {
+        __syncwarp();
+        for (int i = lane; i < cnt; i += 32) {
+          const uint32_t cw = wl[i];
+          const int vr = (int)(cw >> 16), al = (int)(cw & 0xFFFFu);
+          const unsigned long long key = win_word(chain(vr, al), (uint32_t)(a0 + al));
+          if (key) atomicMax(&s_key[vr], key);
+        }
+        __syncwarp();
+        cnt = 0;
+      };
       for (int cg = 0; cg < 4; ++cg) {
         if (!group_valid(cg)) continue;
         uint32_t v[16];
@@ -433,7 +446,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool row_l = vr_valid(vr_l) && rmax[vr_l] != 0u;
         const float band_l = s_band[vr_l];
         const uint32_t rows = __ballot_sync(0xffffffffu, row_l) & 0xFFFFu;
-        int cnt = 0;
+        uint32_t bal[16];
+        int gcnt = 0;
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
           const bool row = (rows >> u) & 1u;
@@ -441,22 +455,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b = (row && atom_ok && a == a) ? __float_as_uint(a) : 0u;
           const float wmax = __uint_as_float(__reduce_max_sync(0xffffffffu, b));
           const float band = __shfl_sync(0xffffffffu, band_l, u);
-          const bool is_c = row && atom_ok && !(a < wmax - band);
-          const uint32_t bal = __ballot_sync(0xffffffffu, is_c);
-          if (is_c)
-            wl[cnt + __popc(bal & ((1u << lane) - 1u))] =
+          bal[u] = __ballot_sync(0xffffffffu, row && atom_ok && !(a < wmax - band));
+          gcnt += __popc(bal[u]);
+        }
+        // the candidates of all groups go through one round of re-scoring,
+        // unless the list would overflow first
+        if (cnt + gcnt > kWarpCand) flush();
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          if ((bal[u] >> lane) & 1u)
+            wl[cnt + __popc(bal[u] & ((1u << lane) - 1u))] =
                 ((uint32_t)(cg * 16 + u) << 16) | (uint32_t)a_loc;
-          cnt += __popc(bal);
+          cnt += __popc(bal[u]);
         }
-        __syncwarp();
-        for (int i = lane; i < cnt; i += 32) {
-          const uint32_t cw = wl[i];
-          const int vr = (int)(cw >> 16), al = (int)(cw & 0xFFFFu);
-          const unsigned long long key = win_word(chain(vr, al), (uint32_t)(a0 + al));
-          if (key) atomicMax(&s_key[vr], key);
-        }
-        __syncwarp();
       }
+      flush();
     }
     tc_fence_before();
     // a zero row: every chain gives +0, the slice's first atom wins
