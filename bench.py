@@ -80,6 +80,11 @@ def parse():
                          "logits, integer exponential); recorded in config")
     ap.add_argument("--full-softmax", action="store_true",
                     help="decode workloads: softmax over every token")
+    ap.add_argument("--context-shard", action="store_true",
+                    help="decode workloads: split every sequence's context "
+                         "over the ranks (sdk_decode_attn_shard with NCCL "
+                         "exchanges; strong scaling of one context) instead "
+                         "of running one independent copy per rank")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -367,6 +372,78 @@ def e2e_layer4k(args, sdk, store, aws, dws, xk, xv, q, DK, DV, out, world,
     return {"value": world * n_vec / (t * 1e-3), "unit": "encoded KV vecs/s",
             "h2d_bytes_per_step": hxk.numel() * 4 + hxv.numel() * 4 + hq.numel() * 4,
             "d2h_bytes_per_step": hout.numel() * 4, "ms_per_step": t}
+
+
+def bench_decode_sharded(args, world, rank, pk, name):
+    """One decode step whose every sequence is split over the ranks (rank r
+    holds tokens [r N / world, (r + 1) N / world)); the exchanges between
+    the stages are NCCL collectives.  Layers run one after the other (no
+    CUDA graph)."""
+    import torch
+    import workloads
+    import sparse_dictionary_coded_b200 as sdk
+    from sparse_dictionary_coded_b200 import sharded
+    W = workloads.WORKLOADS[name]
+    L, B, Hq, Hkv, d, n, N = (W["L"], W["B"], W["Hq"], W["Hkv"], W["d"],
+                              W["n_atoms"], W["n_tokens"])
+    if args.layers is not None:
+        L = max(1, min(L, args.layers))
+    lo, hi = N * rank // world, N * (rank + 1) // world
+    plans = []
+    for l in range(L):
+        lay = workloads.decode_layer(name, l, device="cuda")
+        k_lo, k_full, v_full = workloads.layout(lay["kwords"][:, :, lo:hi].contiguous(),
+                                                lay["vwords"][:, :, lo:hi].contiguous())
+        del lay["kwords"], lay["vwords"]
+        store = sdk.CodeStore.from_tensors(k_lo, k_full, v_full, [hi - lo] * B)
+        q = (lay["q"] / lay["q"].norm(dim=-1, keepdim=True)).contiguous()
+        plans.append(sharded.ShardPlan(q, lay["DK"], lay["DV"], store, [N] * B, rank, world))
+    torch.cuda.synchronize()
+
+    def step():
+        for plan in plans:
+            gen = sharded.shard_stages(plan)
+            if world > 1:
+                sharded.run_exchanges(gen)
+            else:
+                for _ in gen:
+                    pass
+
+    flush = make_flush()
+    clocks = Clocks(torch.cuda.current_device())
+    ms, ck = timed_steps(step, args.steps, args.warmup, flush, world, clocks)
+    for plan in plans:
+        rc, _ = sdk.sdk_check_status(plan.ws)
+        assert rc == 0, "device check failed in sharded decode"
+    step_ms = max_over_ranks(statistics.mean(ms), world)
+    k = (N + 9) // 10
+    # algorithmic bytes of the whole step (all ranks): 12 B per token per KV
+    # head, 116 B per selected (token, query head) record pair, and every
+    # rank reads both dictionaries
+    alg = L * (12 * N * B * Hkv + 116 * k * B * Hq + world * 2 * n * d * 2)
+    gbs = alg / (step_ms * 1e-3) / 1e9
+    return {
+        "value": B * N / (step_ms * 1e-3),
+        "unit": "ctx tokens/s/step (%d layers, context split over %d GPUs)" % (L, world),
+        "ms_per_step": step_ms,
+        "scaling": "strong",
+        "roofline": {"bound": "hbm", "kernel": "context-sharded decode step "
+                     "(all stages, %d layers)" % L, "achieved": gbs,
+                     "peak": world * pk["hbm"], "unit": "GB/s",
+                     "frac": gbs / (world * pk["hbm"]), "traffic": None,
+                     "alg_bytes_per_step": alg,
+                     "note": "selected records counted per query head (no "
+                             "union); peak = ranks x measured HBM copy"},
+        "clocks": ck,
+        "config": {"workload": name, "layers": L, "B": B, "Hq": Hq,
+                   "Hkv": Hkv, "head_dim": d, "n_atoms": n, "n_tokens": N,
+                   "klow": 3, "khigh": 16, "top": "1/10",
+                   "parallelism": "context split over %d ranks" % world,
+                   "l2": "flushed between steps"},
+        "dtype": "f32 (bf16 dictionaries, fp16 coefficients)",
+        # per layer: qd, klow, pass2, 3 selection stages, attend x2, out
+        "gpu_launches": args.steps * L * 9,
+    }
 
 
 def bench_decode(args, world, rank, pk, name):
@@ -750,13 +827,15 @@ def main():
         res = bench_prefill(args, world, rank, pk)
     elif args.workload in APPEND_WORKLOADS:
         res = bench_append(args, world, rank, pk, args.workload)
+    elif args.context_shard:
+        res = bench_decode_sharded(args, world, rank, pk, args.workload)
     else:
         res = bench_decode(args, world, rank, pk, args.workload)
     if rank == 0:
         line = {"metric": METRIC, "value": res.pop("value"),
                 "unit": res.pop("unit"), "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": res.pop("ms_per_step"),
-                "higher_is_better": True, "scaling": "weak",
+                "higher_is_better": True, "scaling": res.pop("scaling", "weak"),
                 "vs_baseline": None, "dtype": res.pop("dtype"),
                 "data": "synthetic (seeded; shapes of the Llama-3.1-8B KV "
                         "workloads, no model or dataset)"}

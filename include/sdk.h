@@ -209,6 +209,51 @@ SDK_API sdk_status sdk_decode_attn(const float* q, int32_t B, int32_t Hq, int32_
 SDK_API size_t sdk_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t head_dim,
                                   int32_t n_atoms, int64_t max_len);
 
+/* ----------------------------------------- context-sharded decode attn
+ * The same computation as sdk_decode_attn (flags 0: fp32 softmax over the
+ * selected set) when every sequence's context is split over `world` ranks,
+ * rank r holding a contiguous token range (ranks in token order, every
+ * rank at least one token of every sequence).  Each rank runs stages 1..6
+ * in order on its own shard and workspace; between stages the ranks
+ * combine workspace regions (byte offsets from sdk_decode_layout_of for the
+ * rank's own lens; R = B*Hq):
+ *   after 1: sum over ranks, uint32 [R][4096] at `hist1` (the first-digit
+ *            histograms of the keys);
+ *   after 2: sum, uint32 [R][4096] at `hist2` (second digit, in the bucket);
+ *   after 3: sum, uint32 [R][256] at `hist1` (third digit);
+ *   after 4: all-gather the uint32 [R] at `hist2` (each rank's ties of the
+ *            k-th key) into a device array [world][R], passed to stage 5;
+ *   after 5: all-gather the float [R][2] at `hist2` + 4R bytes (each rank's
+ *            largest logit and sum of exp(logit - largest) per head) into a
+ *            device array [world][R][2], passed to stage 6;
+ *   after 6: sum `out` over ranks.
+ * The selected set is the exact global top k (k from glens, ties to the
+ * lower global token index); the result equals sdk_decode_attn over the
+ * whole context up to the order of fp32 additions.
+ *   stage      1 .. 6
+ *   rank, world   this rank, number of ranks
+ *   gathered   device: stage 5 the [world][R] tie counts, stage 6 the
+ *              [world][R][2] statistics (8-byte aligned); NULL otherwise
+ *   lens_host  host, int32 [B], this rank's tokens of each sequence (>= 1);
+ *              the code store holds them at positions 0 .. lens[b]-1
+ *   glens_host host, int32 [B], every sequence's whole length
+ *   others     as sdk_decode_attn; flags must be 0 (SDK_ERR_UNSUPPORTED)
+ * The paper has no multi-device design; this follows the exchange the
+ * decomposition of the selection and of the softmax needs.
+ */
+SDK_API sdk_status sdk_decode_attn_shard(int32_t stage, int32_t rank, int32_t world,
+                           const void* gathered, const float* q, int32_t B,
+                           int32_t Hq, int32_t Hkv, int32_t head_dim,
+                           const void* dict_k, const void* dict_v,
+                           int32_t n_atoms, const uint32_t* k_lo,
+                           const uint32_t* k_full, const uint32_t* v_full,
+                           int64_t cap, const int32_t* lens_host,
+                           const int32_t* glens_host, int32_t klow,
+                           int32_t khigh, int32_t top_num, int32_t top_den,
+                           int32_t flags, float scale, float* out,
+                           void* workspace, size_t ws_bytes,
+                           sdk_stream_t stream);
+
 /* ------------------------------------------------- decode, no workspace
  * sdk_decode_attn_static -- sdk_decode_attn with its workspace in a fixed
  * array of SDK_DECODE_STATIC_WS_BYTES (16 MiB) of the library's own device

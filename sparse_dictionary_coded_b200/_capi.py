@@ -45,6 +45,11 @@ SIGNATURES = {
                                               _i64, _vp, _i32, _i32, _i32,
                                               _i32, _i32, _f32, _vp, _vp,
                                               _vp]),
+    "sdk_decode_attn_shard": (ctypes.c_int, [_i32, _i32, _i32, _vp, _vp, _i32,
+                                             _i32, _i32, _i32, _vp, _vp, _i32,
+                                             _vp, _vp, _vp, _i64, _vp, _vp,
+                                             _i32, _i32, _i32, _i32, _i32, _f32,
+                                             _vp, _vp, _sz, _vp]),
     "sdk_decode_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i64]),
     "sdk_decode_layout_of": (ctypes.c_int, [_i32, _i32, _i32, _i32, _i64,
                                             _vp]),

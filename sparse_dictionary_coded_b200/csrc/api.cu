@@ -302,12 +302,19 @@ sdk_status sdk_decode_layout_of(int32_t B, int32_t Hq, int32_t head_dim, int32_t
   return SDK_OK;
 }
 
-sdk_status sdk_decode_attn(const float* q, int32_t B, int32_t Hq, int32_t Hkv, int32_t head_dim,
-                           const void* dict_k, const void* dict_v, int32_t n_atoms,
-                           const uint32_t* k_lo, const uint32_t* k_full, const uint32_t* v_full,
-                           int64_t cap, const int32_t* lens_host, int32_t klow, int32_t khigh,
-                           int32_t top_num, int32_t top_den, int32_t flags, float scale,
-                           float* out, void* workspace, size_t ws_bytes, sdk_stream_t stream) {
+}  // extern "C"
+
+// Checks the decode arguments and fills the kernel parameter block.  With
+// glens (the sequences' whole lengths; context-sharded decode) the selected
+// set size k comes from glens[b] and lens_host holds this rank's shard.
+static sdk_status build_decode_params(const float* q, int32_t B, int32_t Hq, int32_t Hkv,
+                                      int32_t head_dim, const void* dict_k, const void* dict_v,
+                                      int32_t n_atoms, const uint32_t* k_lo,
+                                      const uint32_t* k_full, const uint32_t* v_full, int64_t cap,
+                                      const int32_t* lens_host, const int32_t* glens,
+                                      int32_t klow, int32_t khigh, int32_t top_num,
+                                      int32_t top_den, int32_t flags, float scale, float* out,
+                                      void* workspace, size_t ws_bytes, DecodeParams& p) {
   if (B < 1 || B > SDK_MAX_BATCH || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return SDK_ERR_INVALID_ARG;
   if ((int64_t)B * Hq > 2048) return SDK_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return SDK_ERR_UNSUPPORTED;
@@ -325,12 +332,12 @@ sdk_status sdk_decode_attn(const float* q, int32_t B, int32_t Hq, int32_t Hkv, i
   int64_t max_len = 0;
   for (int b = 0; b < B; ++b) {
     if (lens_host[b] < 1 || lens_host[b] > cap) return SDK_ERR_INVALID_ARG;
+    if (glens != nullptr && glens[b] < lens_host[b]) return SDK_ERR_INVALID_ARG;
     if (lens_host[b] > max_len) max_len = lens_host[b];
   }
   const sdk_decode_layout l = decode_layout(B, Hq, head_dim, n_atoms, max_len);
   if (ws_bytes < l.total) return SDK_ERR_CAPACITY;
 
-  DecodeParams p;
   std::memset(&p, 0, sizeof(p));
   char* ws = reinterpret_cast<char*>(workspace);
   p.q = q;
@@ -367,12 +374,14 @@ sdk_status sdk_decode_attn(const float* q, int32_t B, int32_t Hq, int32_t Hkv, i
   p.R = B * Hq;
   p.n_out_tiles = (n_atoms + 127) / 128;
   p.scale = scale;
+  p.world = 1;
   p.tok_off[0] = p.sel_off[0] = p.dom_off[0] = 0;
   for (int b = 0; b < B; ++b) {
     const int64_t N = lens_host[b];
-    int64_t k = ((int64_t)top_num * N + top_den - 1) / top_den;
+    const int64_t G = glens != nullptr ? glens[b] : N;
+    int64_t k = ((int64_t)top_num * G + top_den - 1) / top_den;
     if (k < 1) k = 1;
-    if (k > N) k = N;
+    if (k > G) k = G;
     p.lens[b] = (int)N;
     p.kcnt[b] = (int)k;
     p.dcnt[b] = p.full ? (int)N : (int)k;
@@ -380,7 +389,49 @@ sdk_status sdk_decode_attn(const float* q, int32_t B, int32_t Hq, int32_t Hkv, i
     p.sel_off[b + 1] = p.sel_off[b] + (int64_t)Hq * k;
     p.dom_off[b + 1] = p.dom_off[b] + (int64_t)Hq * p.dcnt[b];
   }
+  return SDK_OK;
+}
+
+extern "C" {
+
+sdk_status sdk_decode_attn(const float* q, int32_t B, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                           const void* dict_k, const void* dict_v, int32_t n_atoms,
+                           const uint32_t* k_lo, const uint32_t* k_full, const uint32_t* v_full,
+                           int64_t cap, const int32_t* lens_host, int32_t klow, int32_t khigh,
+                           int32_t top_num, int32_t top_den, int32_t flags, float scale,
+                           float* out, void* workspace, size_t ws_bytes, sdk_stream_t stream) {
+  DecodeParams p;
+  const sdk_status s = build_decode_params(q, B, Hq, Hkv, head_dim, dict_k, dict_v, n_atoms, k_lo,
+                                           k_full, v_full, cap, lens_host, nullptr, klow, khigh,
+                                           top_num, top_den, flags, scale, out, workspace,
+                                           ws_bytes, p);
+  if (s != SDK_OK) return s;
   return launch_decode(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sdk_status sdk_decode_attn_shard(int32_t stage, int32_t rank, int32_t world, const void* gathered,
+                                 const float* q, int32_t B, int32_t Hq, int32_t Hkv,
+                                 int32_t head_dim, const void* dict_k, const void* dict_v,
+                                 int32_t n_atoms, const uint32_t* k_lo, const uint32_t* k_full,
+                                 const uint32_t* v_full, int64_t cap, const int32_t* lens_host,
+                                 const int32_t* glens_host, int32_t klow, int32_t khigh,
+                                 int32_t top_num, int32_t top_den, int32_t flags, float scale,
+                                 float* out, void* workspace, size_t ws_bytes,
+                                 sdk_stream_t stream) {
+  if (stage < 1 || stage > 6 || world < 1 || rank < 0 || rank >= world) return SDK_ERR_INVALID_ARG;
+  if (flags != 0) return SDK_ERR_UNSUPPORTED;   // selected-set fp32 softmax only
+  if (glens_host == nullptr) return SDK_ERR_INVALID_ARG;
+  if ((stage == 5 || stage == 6) && (gathered == nullptr || !aligned(gathered, 8)))
+    return SDK_ERR_INVALID_ARG;
+  DecodeParams p;
+  const sdk_status s = build_decode_params(q, B, Hq, Hkv, head_dim, dict_k, dict_v, n_atoms, k_lo,
+                                           k_full, v_full, cap, lens_host, glens_host, klow, khigh,
+                                           top_num, top_den, flags, scale, out, workspace,
+                                           ws_bytes, p);
+  if (s != SDK_OK) return s;
+  p.world = world;
+  p.shard_in = gathered;
+  return launch_decode(p, reinterpret_cast<cudaStream_t>(stream), stage, rank);
 }
 
 sdk_status sdk_workspace_init(void* workspace, size_t ws_bytes, sdk_stream_t stream) {

@@ -401,6 +401,38 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
 
 // ------------------------------------------------------- final selection
 constexpr int kFinalStage = 12288;   // candidates staged in shared memory
+
+// The rank-th smallest token index (1-based) among the candidates whose key
+// equals T, by radix select over index digits 31..21, 20..10, 9..0 (bins
+// kept in reverse so the descending search walks ascending indices).  sh:
+// 2048 words of shared memory.  Sets bad when rank exceeds the ties.
+__device__ uint32_t tie_cut(const uint32_t* ck, const int32_t* ct, uint32_t n_cand, uint32_t T,
+                            uint32_t rank, uint32_t* s_tmp, uint32_t* sh, bool& bad) {
+  const int tid = threadIdx.x;
+  uint32_t prefix = 0u;
+  bad = false;
+  for (int ps = 0; ps < 3; ++ps) {
+    const int sh_lo = ps == 0 ? 21 : (ps == 1 ? 10 : 0);
+    const int wbits = ps == 2 ? 10 : 11;
+    const uint32_t nb = 1u << wbits;
+    for (int i = tid; i < 2048; i += blockDim.x) sh[i] = 0u;
+    __syncthreads();
+    for (uint32_t i = tid; i < n_cand; i += blockDim.x) {
+      if (ck[i] != T) continue;
+      const uint32_t t = (uint32_t)ct[i];
+      const uint32_t hi = (ps == 0) ? 0u : (t >> (sh_lo + wbits));
+      if (hi != prefix) continue;
+      atomicAdd(&sh[2047u - ((t >> sh_lo) & (nb - 1u))], 1u);
+    }
+    __syncthreads();
+    uint32_t bin, above, cnt;
+    block_find_desc<2048>(sh, rank, s_tmp, bin, above, cnt, bad);
+    if (bad) return 0u;
+    prefix = (prefix << wbits) | (2047u - bin);
+    rank -= above;
+  }
+  return prefix;
+}
 // The last two radix digits of one query head over its candidates, the
 // exact k-th key, the tie rule (lower token index first) and the rest of the
 // selected set (inputs written by pass2_kernel, read through L2).
@@ -476,35 +508,14 @@ __device__ void final_head(const DecodeParams& p, int r, uint32_t* s_cand, uint3
   const uint32_t eq_total = cnt3;
 
   // more ties than places: the eq_take-th smallest token index among the
-  // ties, by radix select over index digits 31..21, 20..10, 9..0 (bins kept
-  // in reverse so the descending search walks ascending indices)
+  // ties (tie_cut)
   uint32_t t_cut = 0xFFFFFFFFu;
   if (eq_total > eq_take) {
-    uint32_t prefix = 0u, rank = eq_take;
-    for (int ps = 0; ps < 3; ++ps) {
-      const int sh_lo = ps == 0 ? 21 : (ps == 1 ? 10 : 0);
-      const int wbits = ps == 2 ? 10 : 11;
-      const uint32_t nb = 1u << wbits;
-      for (int i = tid; i < 2048; i += kScanThreads) sh[i] = 0u;
-      __syncthreads();
-      for (uint32_t i = tid; i < n_cand; i += kScanThreads) {
-        if (ck[i] != T) continue;
-        const uint32_t t = (uint32_t)ct[i];
-        const uint32_t hi = (ps == 0) ? 0u : (t >> (sh_lo + wbits));
-        if (hi != prefix) continue;
-        atomicAdd(&sh[2047u - ((t >> sh_lo) & (nb - 1u))], 1u);
-      }
-      __syncthreads();
-      uint32_t bin, above, cnt;
-      block_find_desc<2048>(sh, rank, s_tmp, bin, above, cnt, bad);
-      if (bad) {
-        if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x23000000u | r);
-        return;
-      }
-      prefix = (prefix << wbits) | (2047u - bin);
-      rank -= above;
+    t_cut = tie_cut(ck, ct, n_cand, T, eq_take, s_tmp, sh, bad);
+    if (bad) {
+      if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x23000000u | r);
+      return;
     }
-    t_cut = prefix;
   }
 
   if (tid == 0) {
@@ -570,6 +581,152 @@ __global__ void __launch_bounds__(kScanThreads) final_kernel(DecodeParams p) {
   final_head(p, blockIdx.x, s_cand, s_tmp, sh, s_cnt);
 }
 
+// ------------------------------------------- context-sharded final stages
+// A rank holds a contiguous token range of every sequence (ranks in token
+// order).  After klow the ranks sum hist1, so pass2 finds the global bucket
+// of the k-th key; the last two digits and the ties follow here in three
+// stages, with the ranks combining, between them, the regions that the
+// unsharded path has finished with:
+//   stage 3 writes hist3 [R][256] (third digit over the local candidates)
+//           at the start of hist1; the ranks sum it;
+//   stage 4 writes the local tie count [R] at the start of hist2; the ranks
+//           gather it into ties[world][R];
+//   stage 5 selects the local candidates above the k-th key and the rank's
+//           share of the ties (ties are taken in global token order, i.e.
+//           lower ranks first), completing the local selected list.
+// State carried in sdk_select_state: kth_key (b1 << 20 from pass2, then
+// with b2, then the key T), eq_taken (k2, then the ties to take over all
+// ranks), eq_total (all ties), n_sel (the local selected count).
+__device__ __forceinline__ bool shard_head_ok(const DecodeParams& p, int r,
+                                              const sdk_select_state* st) {
+  const uint32_t k = (uint32_t)p.kcnt[r / p.Hq];
+  const uint32_t n_above = __ldcg(&st->n_above);
+  return n_above < k && __ldcg(&st->n_cand) <= (uint32_t)p.lens[r / p.Hq];
+}
+
+__global__ void __launch_bounds__(kScanThreads) shard_digit3_kernel(DecodeParams p) {
+  __shared__ uint32_t s_tmp[48];
+  __shared__ uint32_t sh[256];
+  const int r = blockIdx.x, tid = threadIdx.x;
+  sdk_select_state* st = p.st + r;
+  if (!shard_head_ok(p, r, st)) {
+    if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x28000000u | r);
+    return;
+  }
+  const uint32_t k1 = (uint32_t)p.kcnt[r / p.Hq] - __ldcg(&st->n_above);
+  uint32_t b2, above2, cnt2;
+  bool bad;
+  block_find_desc<4096, true>(p.hist2 + (int64_t)r * 4096, k1, s_tmp, b2, above2, cnt2, bad);
+  if (bad) {
+    if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x29000000u | r);
+    return;
+  }
+  for (int i = tid; i < 256; i += kScanThreads) sh[i] = 0u;
+  __syncthreads();
+  const uint32_t n_cand = __ldcg(&st->n_cand);
+  const uint32_t* ck = p.cand_key + (int64_t)r * p.L;
+  for (uint32_t i = tid; i < n_cand; i += kScanThreads) {
+    const uint32_t key = __ldcg(ck + i);
+    if (((key >> 8) & 0xFFFu) == b2) atomicAdd(&sh[key & 0xFFu], 1u);
+  }
+  __syncthreads();
+  for (int i = tid; i < 256; i += kScanThreads) p.hist1[(int64_t)r * 256 + i] = sh[i];
+  if (tid == 0) {
+    st->kth_key = __ldcg(&st->kth_key) | (b2 << 8);
+    st->eq_taken = k1 - above2;   // k2
+  }
+}
+
+__global__ void __launch_bounds__(kScanThreads) shard_ties_kernel(DecodeParams p) {
+  __shared__ uint32_t s_tmp[48];
+  __shared__ uint32_t s_cnt;
+  const int r = blockIdx.x, tid = threadIdx.x;
+  sdk_select_state* st = p.st + r;
+  if (!shard_head_ok(p, r, st)) return;   // reported by the previous stage
+  const uint32_t k2 = __ldcg(&st->eq_taken);
+  uint32_t b3, above3, cnt3;
+  bool bad;
+  block_find_desc<256, true>(p.hist1 + (int64_t)r * 256, k2, s_tmp, b3, above3, cnt3, bad);
+  if (bad) {
+    if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x2A000000u | r);
+    return;
+  }
+  const uint32_t T = __ldcg(&st->kth_key) | b3;
+  if (tid == 0) s_cnt = 0u;
+  __syncthreads();
+  const uint32_t n_cand = __ldcg(&st->n_cand);
+  const uint32_t* ck = p.cand_key + (int64_t)r * p.L;
+  uint32_t c = 0u;
+  for (uint32_t i = tid; i < n_cand; i += kScanThreads) c += __ldcg(ck + i) == T ? 1u : 0u;
+  c = __reduce_add_sync(0xffffffffu, c);
+  if ((tid & 31) == 0 && c) atomicAdd(&s_cnt, c);
+  __syncthreads();
+  if (tid == 0) {
+    p.hist2[r] = s_cnt;          // the local ties, gathered over the ranks
+    st->kth_key = T;
+    st->eq_taken = k2 - above3;  // ties to take over all ranks
+    st->eq_total = cnt3;
+  }
+}
+
+// ties: device, uint32 [world][R], every rank's local tie count
+__global__ void __launch_bounds__(kScanThreads) shard_select_kernel(DecodeParams p,
+                                                                    const uint32_t* ties,
+                                                                    int rank_id) {
+  __shared__ uint32_t s_tmp[48];
+  __shared__ uint32_t sh[2048];
+  __shared__ uint32_t s_cnt;
+  const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned lt = (1u << lane) - 1u;
+  sdk_select_state* st = p.st + r;
+  if (!shard_head_ok(p, r, st)) return;
+  const int b = r / p.Hq;
+  const int Nb = p.lens[b];
+  const uint32_t T = __ldcg(&st->kth_key);
+  const uint32_t take_all = __ldcg(&st->eq_taken);
+  uint32_t before = 0u;
+  for (int w = 0; w < rank_id; ++w) before += __ldcg(ties + (int64_t)w * p.R + r);
+  const uint32_t mine = __ldcg(ties + (int64_t)rank_id * p.R + r);
+  const uint32_t quota = take_all > before ? min(take_all - before, mine) : 0u;
+  const uint32_t n_cand = __ldcg(&st->n_cand);
+  const uint32_t* ck = p.cand_key + (int64_t)r * p.L;
+  const int32_t* ct = p.cand_t + (int64_t)r * p.L;
+  int32_t* list = p.list + (int64_t)r * p.L;
+  // ties to take here: none, all, or the quota smallest indices
+  bool take_ties = quota > 0u;
+  uint32_t t_cut = 0xFFFFFFFFu;
+  if (take_ties && quota < mine) {
+    bool bad;
+    t_cut = tie_cut(ck, ct, n_cand, T, quota, s_tmp, sh, bad);
+    if (bad) {
+      if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x2B000000u | r);
+      return;
+    }
+  }
+  if (tid == 0) s_cnt = __ldcg(&st->n_sel);   // the local tokens above the bucket
+  __syncthreads();
+  for (uint32_t i0 = (uint32_t)warp * 32; i0 < n_cand; i0 += kScanThreads) {
+    const uint32_t i = i0 + lane;
+    bool sel = false;
+    uint32_t t = 0u;
+    if (i < n_cand) {
+      const uint32_t key = __ldcg(ck + i);
+      t = (uint32_t)__ldcg(ct + i);
+      sel = key > T || (key == T && take_ties && t <= t_cut);
+    }
+    const unsigned msel = __ballot_sync(0xffffffffu, sel);
+    uint32_t bs = 0;
+    if (lane == 0 && msel) bs = atomicAdd(&s_cnt, (uint32_t)__popc(msel));
+    bs = __shfl_sync(0xffffffffu, bs, 0) + __popc(msel & lt);
+    if (sel) {
+      if (bs < (uint32_t)Nb) list[bs] = (int32_t)t;
+      else record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x2C000000u | r);
+    }
+  }
+  __syncthreads();
+  if (tid == 0) st->n_sel = s_cnt;
+}
+
 // ------------------------------------------------------------- pass2_kernel
 // Tokens above the bucket of the k-th key are selected, tokens inside it
 // become candidates (with a histogram of key bits 19..8), the others go to
@@ -629,7 +786,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) pass2_kernel(DecodeParams p) 
       if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x10000000u | r);
       return;
     }
-    if (t0 == 0 && tid == 0) st->n_above = above1;
+    if (t0 == 0 && tid == 0) {
+      st->n_above = above1;
+      st->kth_key = b1 << 20;   // the first digit (the final stage completes the key)
+    }
     const uint32_t kLo = b1 << 20, kHi = kLo | 0xFFFFFu;   // the k-th key's bucket
     const uint32_t* keys = p.keys + (int64_t)r * p.L;
     int32_t* list = p.list + (int64_t)r * p.L;
@@ -1049,9 +1209,12 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
   const int r = blockIdx.x / C;
   const int rank = (int)cluster.block_rank();
   const int b = r / p.Hq, h = r % p.Hq, kvh = h / p.g;
-  const int k = p.kcnt[b];
-  const int Dr = p.dcnt[b];
+  sdk_select_state* st = p.st + r;
+  // context-sharded stages take the head's local selected count from the
+  // state (the rest of the selection is on the other ranks)
   const int Nb = p.lens[b];
+  const int k = p.att_mode ? (int)min(__ldcg(&st->n_sel), (uint32_t)Nb) : p.kcnt[b];
+  const int Dr = p.att_mode ? k : p.dcnt[b];
   const int s0 = (int)((int64_t)k * rank / C), s1 = (int)((int64_t)k * (rank + 1) / C);
   const int c0 = k + (int)((int64_t)(Dr - k) * rank / C);
   const int c1 = k + (int)((int64_t)(Dr - k) * (rank + 1) / C);
@@ -1061,11 +1224,29 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
   const int32_t* list = p.list + (int64_t)r * p.L;
   float* ss = p.sel_score + (int64_t)r * p.L;
   const uint32_t* keys = p.keys + (int64_t)r * p.L;
-  sdk_select_state* st = p.st + r;
   const float scale = p.scale;
   const int khigh = p.khigh;
   uint32_t maxidx = 0u;
 
+  float m = -INFINITY;
+  const bool isoft = p.isoft != 0;
+  ISoft ic;
+  unsigned long long recip = 0ull, etot = 0ull;
+  float ztot = 0.0f;
+  if (p.att_mode == 2) {
+    // context-sharded, second half: the softmax statistics of every rank
+    // (mz [world][R][2]: the rank's largest logit and its sum of
+    // exp(s - that) for this head) give this head's m and z
+    const float* mz = reinterpret_cast<const float*>(p.shard_in);
+    for (int w = 0; w < p.world; ++w) m = fmaxf(m, __ldcg(mz + ((int64_t)w * p.R + r) * 2));
+    for (int w = 0; w < p.world; ++w) {
+      const float mw = __ldcg(mz + ((int64_t)w * p.R + r) * 2);
+      const float zw = __ldcg(mz + ((int64_t)w * p.R + r) * 2 + 1);
+      if (mw > -INFINITY && zw > 0.0f) ztot += zw * expf(mw - m);
+    }
+    if (tid == 0) s_float = 0;
+    cluster.sync();
+  } else {
   // ---- phase 1: stage QD[r], rescore the own selected entries
   stage_table(table, p.qd + (int64_t)r * n, n);
   __syncthreads();
@@ -1093,7 +1274,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
                   zrun += expf(s - smax);
                 }
               });
-  float m = block_reduce<true>(smax, s_red);
+  m = block_reduce<true>(smax, s_red);
   if (tid == 0) s_val = m;
   cluster.sync();
   m = -INFINITY;
@@ -1101,10 +1282,6 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
   if (rank == 0 && tid == 0 && m > -INFINITY) st->max_score = score_key(m);
   if (p.full && st->n_comp > 0u) m = fmaxf(m, scale * key_score(st->max_comp));
 
-  const bool isoft = p.isoft != 0;
-  ISoft ic;
-  unsigned long long recip = 0ull, etot = 0ull;
-  float ztot = 0.0f;
   if (!isoft) {
     // z: the own selected entries (rescaled to m) and complement entries
     float z = smax > -INFINITY ? zrun * expf(smax - m) : 0.0f;
@@ -1155,6 +1332,20 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
     recip = etot > 0ull ? (1ull << 61) / etot : 0ull;
     ztot = (float)etot;
   }
+  if (p.att_mode == 1) {
+    // context-sharded, first half: this rank's statistics of the head go to
+    // mz [R][2] (gathered over the ranks); the cluster's shared memory stays
+    // until every CTA has read it
+    if (kCheck && maxidx >= (uint32_t)n) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, maxidx);
+    if (rank == 0 && tid == 0) {
+      float* mz = reinterpret_cast<float*>(p.hist2) + p.R + 2 * r;
+      mz[0] = m;
+      mz[1] = ztot;
+    }
+    cluster.sync();
+    return;
+  }
+  }   // phase 1
   const float invz = 1.0f / ztot;
 
   // ---- phase 2: scatter p c^V into the weight tile
@@ -1443,7 +1634,7 @@ static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
+sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, int rank_id) {
   const int sms = num_sms();
   static bool attr = false;
   if (!attr) {
@@ -1478,6 +1669,9 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
   const int gv_tiles = wide ? 4 : 1, gv_rb = wide ? 2 : 1;
   const dim3 gv_grid((p.n + gv_tiles * kGvAtoms - 1) / (gv_tiles * kGvAtoms),
                      (p.R + 32 * gv_rb - 1) / (32 * gv_rb));
+  auto run = [&](int part) -> sdk_status {
+  switch (part) {
+  case 0: {   // QD and the Klow scan
   bool qd_tc = false;
   if (qd_tensor_cores()) {
     const sdk_status st = launch_qd_tc(p, stream, &qd_tc);
@@ -1502,14 +1696,18 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
                    1, p, vec);
     if (e != cudaSuccess) return SDK_ERR_CUDA;
   }
-  {
+  return SDK_OK;
+  }
+  case 1: {   // pass 2 of the selection
     const int g = grid_for(p.tok_off[p.B], 8192, sms);
     e = launch_pdl(pass2_kernel, dim3(g), dim3(kScanThreads), (size_t)kPass2Smem, stream, 1, p);
-    if (e != cudaSuccess) return SDK_ERR_CUDA;
+    return e == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
   }
-  e = launch_pdl(final_kernel, dim3(p.R), dim3(kScanThreads), (size_t)2 * kFinalStage * 4, stream, 1,
-                 p);
-  if (e != cudaSuccess) return SDK_ERR_CUDA;
+  case 2:     // the final selection (whole context)
+    e = launch_pdl(final_kernel, dim3(p.R), dim3(kScanThreads), (size_t)2 * kFinalStage * 4, stream,
+                   1, p);
+    return e == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
+  case 3: {   // attend
   {
     // one cluster of C CTAs per query head, C a power of two <= 8 while the
     // clusters fit the SMs and every CTA keeps >= 1024 entries
@@ -1524,6 +1722,9 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
                    (unsigned)C, p, C);
     if (e != cudaSuccess) return SDK_ERR_CUDA;
   }
+  return SDK_OK;
+  }
+  default: {  // w D_V
   // w D_V: tensor cores above 32 query rows; at 32 or fewer the CUDA-core
   // kernel was measured faster (the tensor-core CTAs are latency-bound)
   bool out_tc = false;
@@ -1543,6 +1744,49 @@ sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream) {
                      : launch_pdl(out_kernel<64, 1, 1>, gv_grid, dim3(64), sm, stream, 1, p);
     }
     if (e != cudaSuccess) return SDK_ERR_CUDA;
+  }
+  return SDK_OK;
+  }
+  }
+  };
+  if (shard_stage == 0) {
+    for (int part = 0; part < 5; ++part) {
+      const sdk_status st = run(part);
+      if (st != SDK_OK) return st;
+    }
+  } else {
+    // context-sharded stages (sdk_decode_attn_shard): 1 QD + Klow scan;
+    // 2 pass 2; 3 third digit; 4 key and ties; 5 local selection and
+    // attend's first half; 6 attend's second half and w D_V
+    sdk_status st = SDK_OK;
+    switch (shard_stage) {
+      case 1: st = run(0); break;
+      case 2: st = run(1); break;
+      case 3:
+        e = launch_pdl(shard_digit3_kernel, dim3(p.R), dim3(kScanThreads), 0, stream, 1, p);
+        st = e == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
+        break;
+      case 4:
+        e = launch_pdl(shard_ties_kernel, dim3(p.R), dim3(kScanThreads), 0, stream, 1, p);
+        st = e == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
+        break;
+      case 5:
+        e = launch_pdl(shard_select_kernel, dim3(p.R), dim3(kScanThreads), 0, stream, 1, p,
+                       reinterpret_cast<const uint32_t*>(p.shard_in), rank_id);
+        if (e != cudaSuccess) return SDK_ERR_CUDA;
+        p.att_mode = 1;
+        st = run(3);
+        p.att_mode = 0;
+        break;
+      case 6:
+        p.att_mode = 2;
+        st = run(3);
+        p.att_mode = 0;
+        if (st == SDK_OK) st = run(4);
+        break;
+      default: return SDK_ERR_INVALID_ARG;
+    }
+    if (st != SDK_OK) return st;
   }
   return cudaGetLastError() == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
 }

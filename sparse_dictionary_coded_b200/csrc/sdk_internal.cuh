@@ -176,6 +176,10 @@ struct DecodeParams {
   int64_t cap;
   int64_t L;
   int B, Hq, Hkv, g, d, n, klow, khigh, full, isoft, R, n_out_tiles;
+  // context-sharded decode: 0 = whole decode; 1 / 2 = attend's first /
+  // second half (shard_in: the gathered softmax statistics); world ranks
+  int att_mode, world;
+  const void* shard_in;
   float scale;
   int lens[kMaxBatch];
   int kcnt[kMaxBatch];
@@ -204,7 +208,10 @@ int num_sms();  // cached multiprocessor count of the current device
 sdk_status launch_qd_tc(const DecodeParams& p, cudaStream_t stream, bool* taken);
 // out += w D_V on the tensor cores (taken = false: use the CUDA cores)
 sdk_status launch_out_tc(const DecodeParams& p, cudaStream_t stream, bool* taken);
-sdk_status launch_decode(const DecodeParams& p, cudaStream_t stream);
+// shard_stage 0: the whole decode; 1..6: one stage of the context-sharded
+// decode for rank rank_id (sdk_decode_attn_shard)
+sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage = 0,
+                         int rank_id = 0);
 sdk_decode_layout decode_layout(int B, int Hq, int d, int n, int64_t L);
 sdk_status launch_encode_simt(const EncodeParams& p, int head_dim, cudaStream_t stream);
 // Tensor-core encoder; sets *taken = false when it does not handle the
