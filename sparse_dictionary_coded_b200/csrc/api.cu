@@ -22,6 +22,21 @@ int num_sms() {
   return cache[dev];
 }
 
+static unsigned long long device_bit() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0ull;
+  return 1ull << dev;
+}
+
+bool device_needs_setup(const unsigned long long* flags) {
+  const unsigned long long bit = device_bit();
+  return bit == 0ull || (__atomic_load_n(flags, __ATOMIC_ACQUIRE) & bit) == 0ull;
+}
+
+void device_setup_done(unsigned long long* flags) {
+  __atomic_fetch_or(flags, device_bit(), __ATOMIC_RELEASE);
+}
+
 }  // namespace sdk
 
 using namespace sdk;

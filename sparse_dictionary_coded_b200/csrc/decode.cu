@@ -1636,8 +1636,8 @@ static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 
 sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, int rank_id) {
   const int sms = num_sms();
-  static bool attr = false;
-  if (!attr) {
+  static unsigned long long attr_set = 0ull;
+  if (device_needs_setup(&attr_set)) {
     cudaFuncSetAttribute(klow_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kTable * 4 + 4096 * 4);
     cudaFuncSetAttribute(pass2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPass2Smem);
@@ -1660,7 +1660,7 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
                          kAttSmem);
     cudaFuncSetAttribute(attend_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kAttSmem);
-    attr = true;
+    device_setup_done(&attr_set);
   }
   cudaError_t e = cudaSuccess;
   // GEMV shapes: up to 32 query rows one tile x one row block per CTA,

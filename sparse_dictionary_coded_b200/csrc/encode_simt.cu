@@ -139,13 +139,13 @@ sdk_status launch_encode_simt(const EncodeParams& p, int head_dim, cudaStream_t 
   if (p.n_vec == 0) return SDK_OK;
   const unsigned grid = (unsigned)((p.n_vec + kSimtVecs - 1) / kSimtVecs);
   const size_t smem = (size_t)2 * head_dim * kSimtVecs * 4;
-  static bool attr = false;
-  if (!attr) {
+  static unsigned long long attr_set = 0ull;
+  if (device_needs_setup(&attr_set)) {
     cudaFuncSetAttribute(encode_simt_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)(2 * 128 * kSimtVecs * 4));
     cudaFuncSetAttribute(encode_simt_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)(2 * 64 * kSimtVecs * 4));
-    attr = true;
+    device_setup_done(&attr_set);
   }
   if (head_dim == 128) encode_simt_kernel<128><<<grid, 256, smem, stream>>>(p);
   else encode_simt_kernel<64><<<grid, 256, smem, stream>>>(p);

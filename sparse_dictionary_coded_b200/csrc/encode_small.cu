@@ -636,13 +636,13 @@ sdk_status launch_encode_small(const SmallEncode& e, void* scratch, size_t scrat
   if (e.streams == 1) maps[1] = maps[0];
   const void* fn = D == 128 ? (const void*)encode_small_kernel<128> : (const void*)encode_small_kernel<64>;
   const int smem = D == 128 ? SCfg<128>::kSmem : SCfg<64>::kSmem;
-  static bool attr = false;
-  if (!attr) {
+  static unsigned long long attr_set = 0ull;
+  if (device_needs_setup(&attr_set)) {
     cudaFuncSetAttribute(encode_small_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          SCfg<128>::kSmem);
     cudaFuncSetAttribute(encode_small_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          SCfg<64>::kSmem);
-    attr = true;
+    device_setup_done(&attr_set);
   }
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem) != cudaSuccess)

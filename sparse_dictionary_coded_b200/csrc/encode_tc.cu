@@ -969,8 +969,8 @@ sdk_status launch_encode_tc(const EncodeParams& p, int head_dim, void* scratch,
   tp.n_tiles = (int)tiles;
   tp.n_atom_tiles = (p.n + tc::kAtomTile - 1) / tc::kAtomTile;
 
-  static bool attr = false;
-  if (!attr) {
+  static unsigned long long attr_set = 0ull;
+  if (device_needs_setup(&attr_set)) {
     cudaFuncSetAttribute(tc::encode_tc_kernel<128, true>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Cfg<128>::kSmem);
     cudaFuncSetAttribute(tc::encode_tc_kernel<64, true>,
@@ -979,7 +979,7 @@ sdk_status launch_encode_tc(const EncodeParams& p, int head_dim, void* scratch,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Cfg<128>::kSmem);
     cudaFuncSetAttribute(tc::encode_tc_kernel<64, false>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Cfg<64>::kSmem);
-    attr = true;
+    device_setup_done(&attr_set);
   }
   const dim3 g((unsigned)grid);
   if (head_dim == 128) {

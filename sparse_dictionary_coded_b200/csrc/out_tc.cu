@@ -201,13 +201,13 @@ sdk_status launch_out_tc(const DecodeParams& p, cudaStream_t stream, bool* taken
   // 16-byte weight copies need rows of a multiple of 4 atoms
   if ((p.d != 64 && p.d != 128) || (p.n & 3) != 0) return SDK_OK;
   *taken = true;
-  static bool attr = false;
-  if (!attr) {
+  static unsigned long long attr_set = 0ull;
+  if (device_needs_setup(&attr_set)) {
     cudaFuncSetAttribute(tc::out_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          tc::OCfg<128>::kSmem);
     cudaFuncSetAttribute(tc::out_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          tc::OCfg<64>::kSmem);
-    attr = true;
+    device_setup_done(&attr_set);
   }
   const dim3 grid((unsigned)((p.n + tc::kOAtoms - 1) / tc::kOAtoms),
                   (unsigned)((p.R + tc::kORows - 1) / tc::kORows));

@@ -313,13 +313,13 @@ sdk_status launch_qd_tc(const DecodeParams& p, cudaStream_t stream, bool* taken)
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return SDK_OK;   // fall back to the CUDA-core kernel
   *taken = true;
-  static bool attr = false;
-  if (!attr) {
+  static unsigned long long attr_set = 0ull;
+  if (device_needs_setup(&attr_set)) {
     cudaFuncSetAttribute(tc::qd_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          tc::QCfg<128>::kSmem);
     cudaFuncSetAttribute(tc::qd_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          tc::QCfg<64>::kSmem);
-    attr = true;
+    device_setup_done(&attr_set);
   }
   const int tiles = (p.n + tc::kQAtoms - 1) / tc::kQAtoms;
   int gx = num_sms();

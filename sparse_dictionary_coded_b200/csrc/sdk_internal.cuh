@@ -204,6 +204,14 @@ struct EncodeParams {
 
 int num_sms();  // cached multiprocessor count of the current device
 
+// Kernel attributes (the dynamic shared-memory limits) are set per device:
+// device_needs_setup tells whether the current device's bit in `flags` is
+// still clear, device_setup_done sets it once the attributes are set.
+// Concurrent first calls may both set the attributes, which is harmless;
+// none launches before its own setup is complete.
+bool device_needs_setup(const unsigned long long* flags);
+void device_setup_done(unsigned long long* flags);
+
 // QD on the tensor cores (taken = false: not available, use the CUDA cores)
 sdk_status launch_qd_tc(const DecodeParams& p, cudaStream_t stream, bool* taken);
 // out += w D_V on the tensor cores (taken = false: use the CUDA cores)
