@@ -10,9 +10,15 @@
 //     remainder below 2^-24 |w| for normal values) forming three A operands;
 //   * one thread issues 3 x 8 tcgen05.mma (M=128, N=head_dim, K=16) into one
 //     TMEM accumulator (fp32);
-//   * four warps read it back (one row per thread) and add it into `out`
-//     (zeroed by the QD kernel of the call) with vector reductions.
+//   * four warps read it back (one row per thread) into shared memory;
+//   * CTAs run in clusters of kOCluster adjacent atom slices: CTA k of a
+//     cluster sums rows [k 128/kOCluster, (k+1) 128/kOCluster) over the
+//     cluster's partial tiles (distributed shared memory) and adds them into
+//     `out` (zeroed by the QD kernel of the call) with vector reductions, so
+//     every output element takes n / (128 kOCluster) global reductions.
 // The single wait on the MMA completion is bounded (1 s; SDK_ERR_TIMEOUT).
+#include <cooperative_groups.h>
+
 #include "tc_ptx.cuh"
 
 namespace sdk {
@@ -22,6 +28,7 @@ constexpr int kORows = 128;    // MMA M
 constexpr int kOAtoms = 128;   // K per CTA
 constexpr int kOThreads = 128;
 constexpr int kOSplit = 3;
+constexpr int kOCluster = 4;   // CTAs (atom slices) summed on chip per reduction
 
 template <int D>
 struct OCfg {
@@ -33,6 +40,9 @@ struct OCfg {
   static constexpr int kOffA = kOffB + kBBytes;
   static constexpr int kOffV = kOffA + kOSplit * kABytes;
   static constexpr int kOffW = kOffV + kVBytes;
+  // the partial tile fp32 [128][D + 4] reuses the value and weight staging
+  static constexpr int kPStride = D + 4;
+  static_assert(kORows * kPStride * 4 <= kVBytes + kWBytes, "partial tile must fit");
   static constexpr int kOffBar = kOffW + kWBytes;
   static constexpr int kOffMisc = kOffBar + 8;
   static constexpr int kSmem = kOffMisc + 16 + 1024;     // + 1024-byte alignment slack
@@ -166,25 +176,57 @@ __global__ void __launch_bounds__(kOThreads, 1) out_tc_kernel(DecodeParams p) {
   const bool ok = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
   if (!ok && lane == 0) record_error(p.hdr, SDK_ERR_TIMEOUT, 0x53000000u | blockIdx.x);
   tc_fence_after();
-  const int row = r0 + warp * 32 + lane;
-  if (ok) {
+  // the accumulator into shared memory, one row per thread (zeros if the
+  // MMAs timed out: the error is recorded, the cluster still completes)
+  float* part = reinterpret_cast<float*>(smem + C::kOffV);
+  {
+    const int i = warp * 32 + lane;
 #pragma unroll
     for (int c0 = 0; c0 < D; c0 += 32) {
       uint32_t v[32];
-      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c0, v);
-      tmem_ld_wait();
-      if (row < R) {
-        float* dst = p.out + (int64_t)row * D + c0;
+      if (ok) {
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c0, v);
+        tmem_ld_wait();
+      } else {
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-          asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 4 * u),
-                       "f"(__uint_as_float(v[4 * u])), "f"(__uint_as_float(v[4 * u + 1])),
-                       "f"(__uint_as_float(v[4 * u + 2])), "f"(__uint_as_float(v[4 * u + 3]))
-                       : "memory");
+        for (int u = 0; u < 32; ++u) v[u] = 0u;
       }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        *reinterpret_cast<uint4*>(part + i * C::kPStride + c0 + 4 * u) =
+            make_uint4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
     }
   }
   tc_fence_before();
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  cluster.sync();
+  // this CTA's rows of the cluster's sum, into `out`
+  {
+    const int cr = (int)cluster.block_rank();
+    constexpr int kRowsPer = kORows / kOCluster;
+    const float* parts[kOCluster];
+#pragma unroll
+    for (int k = 0; k < kOCluster; ++k) parts[k] = cluster.map_shared_rank(part, k);
+    for (int e = tid; e < kRowsPer * (D / 4); e += kOThreads) {
+      const int i = cr * kRowsPer + e / (D / 4), c4 = e % (D / 4);
+      if (r0 + i >= R) continue;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k = 0; k < kOCluster; ++k) {
+        const float4 x = *reinterpret_cast<const float4*>(parts[k] + i * C::kPStride + 4 * c4);
+        acc.x += x.x;
+        acc.y += x.y;
+        acc.z += x.z;
+        acc.w += x.w;
+      }
+      float* dst = p.out + (int64_t)(r0 + i) * D + 4 * c4;
+      asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(acc.x),
+                   "f"(acc.y), "f"(acc.z), "f"(acc.w)
+                   : "memory");
+    }
+  }
+  cluster.sync();   // the peers' tiles are read before any CTA leaves
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
@@ -209,13 +251,24 @@ sdk_status launch_out_tc(const DecodeParams& p, cudaStream_t stream, bool* taken
                          tc::OCfg<64>::kSmem);
     device_setup_done(&attr_set);
   }
-  const dim3 grid((unsigned)((p.n + tc::kOAtoms - 1) / tc::kOAtoms),
-                  (unsigned)((p.R + tc::kORows - 1) / tc::kORows));
-  if (p.d == 128)
-    tc::out_tc_kernel<128><<<grid, tc::kOThreads, tc::OCfg<128>::kSmem, stream>>>(p);
-  else
-    tc::out_tc_kernel<64><<<grid, tc::kOThreads, tc::OCfg<64>::kSmem, stream>>>(p);
-  return cudaGetLastError() == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
+  // atom slices rounded up to whole clusters (slices past n are zero)
+  int slices = (p.n + tc::kOAtoms - 1) / tc::kOAtoms;
+  slices = (slices + tc::kOCluster - 1) / tc::kOCluster * tc::kOCluster;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)slices, (unsigned)((p.R + tc::kORows - 1) / tc::kORows));
+  cfg.blockDim = dim3(tc::kOThreads);
+  cfg.dynamicSmemBytes = p.d == 128 ? tc::OCfg<128>::kSmem : tc::OCfg<64>::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = tc::kOCluster;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  const cudaError_t e = p.d == 128 ? cudaLaunchKernelEx(&cfg, tc::out_tc_kernel<128>, p)
+                                   : cudaLaunchKernelEx(&cfg, tc::out_tc_kernel<64>, p);
+  return e == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
 }
 
 }  // namespace sdk

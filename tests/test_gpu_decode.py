@@ -350,7 +350,8 @@ import workloads, sparse_dictionary_coded_b200 as sdk
 from test_gpu_decode import _random_case, _store
 for name, args in (("b1", (81, 1, 32, 8, 2000, 128, 32768)),
                    ("b2", (83, 2, 32, 8, 900, 64, 2048)),
-                   ("b4", (82, 4, 32, 8, 600, 128, 4096))):
+                   ("b4", (82, 4, 32, 8, 600, 128, 4096)),
+                   ("b2-640", (84, 2, 32, 8, 700, 128, 640))):
     q, DK, DV, kw, vw, lens = _random_case(*args)
     B, Hq, d = q.shape
     store = _store(kw, vw, lens)
@@ -372,7 +373,9 @@ def test_gemvs_on_cuda_cores_match_tensor_cores(tmp_path):
     parts) unless SDK_DECODE_QD_TC=0 / SDK_DECODE_OUT_TC=0 select the fp32
     CUDA-core kernels (read once per process, hence child processes): both
     give QD within fp32 rounding of each other and the same outputs, at 32,
-    64 (head_dim 64) and 128 query rows."""
+    64 (head_dim 64) and 128 query rows, and with 640 atoms (five atom
+    slices: the tensor-core w D_V runs clusters of four, three of them
+    empty)."""
     import os
     import subprocess
     import sys
@@ -386,7 +389,7 @@ def test_gemvs_on_cuda_cores_match_tensor_cores(tmp_path):
                            env=env, capture_output=True, text=True, timeout=600)
         assert r.returncode == 0, r.stdout + r.stderr
         res[mode] = d
-    for name in ("b1", "b2", "b4"):
+    for name in ("b1", "b2", "b4", "b2-640"):
         qa = np.load(res["1"] / ("qd_" + name + ".npy"))
         qb = np.load(res["0"] / ("qd_" + name + ".npy"))
         assert np.max(np.abs(qa - qb)) <= 2e-6 * np.max(np.abs(qb))
