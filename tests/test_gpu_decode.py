@@ -301,11 +301,14 @@ def test_bad_atom_index_is_reported_not_trapped():
     assert rc2 == 0                      # cleared by the first read
 
 
-@pytest.mark.parametrize("name", ["decode32k_b4", "decode256k"])
-def test_full_size_layer_sampled_heads(name):
+@pytest.mark.parametrize("name,isoft", [("decode32k_b4", False), ("decode256k", False),
+                                        ("decode256k", True)],
+                         ids=["decode32k_b4", "decode256k", "decode256k-int-softmax"])
+def test_full_size_layer_sampled_heads(name, isoft):
     """One layer of the full-size decode workloads in the bench's launch
-    configuration; the oracle checks two sampled heads one by one and every
-    head's set size and softmax mass."""
+    configuration (and with the integer softmax at 256K); the oracle checks
+    two sampled heads one by one and every head's set size and softmax
+    mass."""
     lay = workloads.decode_layer(name, 0, device="cuda")
     B, Hq = lay["B"], lay["Hq"]
     N = lay["n_tokens"]
@@ -314,7 +317,8 @@ def test_full_size_layer_sampled_heads(name):
     store = sdk.CodeStore.from_tensors(k_lo, k_full, v_full, [N] * B)
     ws = sdk.new_workspace(sdk.sdk_decode_workspace_bytes(
         B, Hq, 128, 32768, N))
-    out = sdk.sdk_decode_attn(q, lay["DK"], lay["DV"], store, workspace=ws)
+    out = sdk.sdk_decode_attn(q, lay["DK"], lay["DV"], store, workspace=ws,
+                              int_softmax=isoft)
     torch.cuda.synchronize()
     rc, _ = sdk.sdk_check_status(ws)
     assert rc == 0
@@ -322,7 +326,7 @@ def test_full_size_layer_sampled_heads(name):
     st = sdk.read_select_state(ws, layd, B * Hq)
     k = oracle.topk_count(N, 1, 10)
     assert torch.all(st["n_sel"] == k)
-    assert torch.all(st["z"] >= 1.0)          # the max term contributes 1
+    assert torch.all(st["z"] >= 1.0)          # the max term contributes 1 (or its INT16 exp)
     assert torch.isfinite(out).all()
     R = B * Hq
     sets = _gpu_sets(ws, layd, R, N, [k] * R)
@@ -334,11 +338,11 @@ def test_full_size_layer_sampled_heads(name):
         kvh = h // (Hq // lay["Hkv"])
         kwn = words_np(lay["kwords"][b, kvh])
         vwn = words_np(lay["vwords"][b, kvh])
-        ref = oracle.decode_head_ref(qn[b, h], kwn, vwn, DKn, DVn)
+        ref = oracle.decode_head_ref(qn[b, h], kwn, vwn, DKn, DVn, int_softmax=isoft)
         r = b * Hq + h
         if check_selection(sets[r], ref["s_lo"], k):
             ref = oracle.decode_head_ref(qn[b, h], kwn, vwn, DKn, DVn,
-                                         force_set=sets[r])
+                                         force_set=sets[r], int_softmax=isoft)
         assert np.max(np.abs(outn[b, h] - ref["out"])) <= OUT_TOL
 
 

@@ -165,3 +165,15 @@ def test_ties_across_shards(world):
     kw = workloads.random_codes((1, 1, N), n, g)
     kw[0, 0, 1::2] = kw[0, 0, 7]
     _check(q, DK, DV, kw, vw, [N], [[0], [333], [700]][:world])
+
+
+def test_full_size_decode256k_two_ranks():
+    """One layer of the 256K workload (32 q / 8 KV heads, 262,144 tokens)
+    split over two ranks at an uneven cut: every head's selected set equals
+    the whole-context one; outputs against the whole-context decode, and
+    two sampled heads against the oracle."""
+    lay = workloads.decode_layer("decode256k", 0)
+    q = _unit(lay["q"])
+    N = lay["n_tokens"]
+    _check(q, lay["DK"], lay["DV"], lay["kwords"], lay["vwords"], [N],
+           [[0], [100_003]], oracle_heads=2)
