@@ -1037,22 +1037,23 @@ constexpr int kAttSmem = kTable * 4 + 2 * kAttThreads * 64;
 constexpr float kFixScale = 1048576.0f;       // 2^20
 constexpr float kFixInv = 1.0f / 1048576.0f;
 
-// Calls f(i, t, w) for every entry i in [e0, e1) of `list` owned by this
-// thread (i = e0 + tid + j*T); w holds the 16 words of token t's record.
-// Entries naming a token outside [0, Nb) are reported and skipped.  Records
-// stream through a two-slot ring per thread in shared memory (cp.async; the
-// four 16-byte chunks of a slot are XOR-swizzled by thread so the reads are
-// free of bank conflicts): entries i + T and i + 2T are in flight while i
-// is used, and the record of i + 3T is prefetched into L2.
-template <class F>
+// Calls f(i, t, w, x) for every entry i in [e0, e1) of `list` owned by this
+// thread (i = e0 + tid + j*T); w holds the 16 words of token t's record and
+// x = pay(i, t), a per-entry value whose load is issued together with the
+// record's copy.  Entries naming a token outside [0, Nb) are reported and
+// skipped.  Records stream through a two-slot ring per thread in shared
+// memory (cp.async; the four 16-byte chunks of a slot are XOR-swizzled by
+// thread so the reads are free of bank conflicts): entries i + T and i + 2T
+// are in flight while i is used and the record of i + 3T is prefetched into
+// L2.  The list entries themselves are loaded six iterations ahead, so no
+// iteration waits on a list load.
+template <class Pay, class F>
 __device__ __forceinline__ void for_records(const int32_t* list, int e0, int e1, const uint4* rec,
                                             int Nb, WsHeader* hdr, uint32_t tag, uint4* ring,
-                                            F f) {
+                                            Pay pay, F f) {
   constexpr int T = kAttThreads;
   const int tid = threadIdx.x;
   const int sw = (tid >> 1) & 3;
-  // raw list entries: nothing waits on these loads until they are used
-  // (two and four iterations later); out-of-range tokens are caught there
   auto list_at = [&](int i) -> int { return i < e1 ? __ldg(list + i) : -1; };
   auto ok = [&](int t) { return (unsigned)t < (unsigned)Nb; };
   // records sit at random token positions: both the copies and the L2
@@ -1072,10 +1073,13 @@ __device__ __forceinline__ void for_records(const int32_t* list, int e0, int e1,
   };
   int i = e0 + tid;
   if (i >= e1) return;
-  int t0 = list_at(i), t1 = list_at(i + T), t2 = list_at(i + 2 * T);
-  issue(t0, 0);
-  issue(t1, 1);
-  int t3 = list_at(i + 3 * T);
+  // q0..q5: the list entries i, i + T, ..., i + 5T
+  int q0 = list_at(i), q1 = list_at(i + T), q2 = list_at(i + 2 * T);
+  int q3 = list_at(i + 3 * T), q4 = list_at(i + 4 * T), q5 = list_at(i + 5 * T);
+  issue(q0, 0);
+  float x0 = ok(q0) ? pay(i, q0) : 0.0f;
+  issue(q1, 1);
+  float x1 = ok(q1) ? pay(i + T, q1) : 0.0f;
   int slot = 0;
   for (; i < e1; i += T) {
     cp_async_wait<1>();               // the slot of entry i has landed
@@ -1086,18 +1090,25 @@ __device__ __forceinline__ void for_records(const int32_t* list, int e0, int e1,
     asm volatile("" ::"r"(w[0].x), "r"(w[0].y), "r"(w[0].z), "r"(w[0].w), "r"(w[1].x),
                  "r"(w[1].y), "r"(w[1].z), "r"(w[1].w), "r"(w[2].x), "r"(w[2].y), "r"(w[2].z),
                  "r"(w[2].w), "r"(w[3].x), "r"(w[3].y), "r"(w[3].z), "r"(w[3].w));
-    issue(t2, slot);                  // entry i + 2T into the freed slot
-    prefetch(t3);
-    if (ok(t0)) f(i, t0, w);
+    issue(q2, slot);                  // entry i + 2T into the freed slot
+    const float x2 = ok(q2) ? pay(i + 2 * T, q2) : 0.0f;
+    prefetch(q3);
+    if (ok(q0)) f(i, q0, w, x0);
     else record_error(hdr, SDK_ERR_DEVICE_CHECK, tag);
-    t0 = t1;
-    t1 = t2;
-    t2 = t3;
-    t3 = list_at(i + 4 * T);
+    q0 = q1;
+    q1 = q2;
+    q2 = q3;
+    q3 = q4;
+    q4 = q5;
+    q5 = list_at(i + 6 * T);
+    x0 = x1;
+    x1 = x2;
     slot ^= 1;
   }
   cp_async_wait<0>();
 }
+// for_records without a per-entry value
+__device__ __forceinline__ float no_pay(int, int) { return 0.0f; }
 
 // block-wide reduction of one float per thread into s_red[0] (max or sum)
 template <bool kMax>
@@ -1252,8 +1263,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
   __syncthreads();
   float smax = -INFINITY, zrun = 0.0f;     // online softmax of this thread
   float smin = INFINITY;                   // for the integer softmax's scale
-  for_records(list, s0, s1, krec, Nb, p.hdr, 0x30000000u | r, ring,
-              [&](int i, int t, const uint4 (&w)[4]) {
+  for_records(list, s0, s1, krec, Nb, p.hdr, 0x30000000u | r, ring, no_pay,
+              [&](int i, int t, const uint4 (&w)[4], float) {
                 float s = 0.0f;
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
@@ -1381,13 +1392,15 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
         }
       }
     };
+    // the logits load with the records: the rescored ones, and with the
+    // flag the complement's scale * s_lo
     for_records(list, s0, s1, vrec, Nb, p.hdr, 0x31000000u | r, ring,
-                [&](int i, int t, const uint4 (&w)[4]) { scatter(ss[i], w); });
+                [&](int i, int) { return ss[i]; },
+                [&](int, int, const uint4 (&w)[4], float lg) { scatter(lg, w); });
     if (p.full)
       for_records(list, c0, c1, vrec, Nb, p.hdr, 0x32000000u | r, ring,
-                  [&](int i, int t, const uint4 (&w)[4]) {
-                    scatter(scale * key_score(keys[t]), w);
-                  });
+                  [&](int, int t) { return scale * key_score(keys[t]); },
+                  [&](int, int, const uint4 (&w)[4], float lg) { scatter(lg, w); });
     // int32 range guard (also catches NaN): sum |p c| * 2^20 < 2^30
     if (!kFloat && !(absum < 1073741824.0f)) s_float = 1;
     __syncthreads();
