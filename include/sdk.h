@@ -313,8 +313,11 @@ typedef struct {
   size_t cand_t;     /* int32  [R][L]  tokens inside the pass-1 bucket    */
   size_t cand_key;   /* uint32 [R][L]  their keys                         */
   size_t sel_score;  /* float  [R][L]  s_t of list[r][i], i < k           */
-  size_t w;          /* float  [R][n_atoms] unnormalised per-atom weights */
-  size_t part;       /* float  partial sums of w D_V                      */
+  size_t w;          /* bf16   [3][R][n_atoms] the per-atom weights w[r]
+                        (softmax-normalised) as three parts, w = w[0] +
+                        w[1] + w[2], each the bf16 rounding of what the
+                        previous parts leave                              */
+  size_t part;       /* (empty)                                           */
   size_t total;      /* total bytes                                       */
   size_t row;        /* elements per head in keys, list, cand_t, cand_key
                         and sel_score: max_len rounded up to a multiple of

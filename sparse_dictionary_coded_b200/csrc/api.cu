@@ -372,7 +372,7 @@ static sdk_status build_decode_params(const float* q, int32_t B, int32_t Hq, int
   p.cand_t = reinterpret_cast<int32_t*>(ws + l.cand_t);
   p.cand_key = reinterpret_cast<uint32_t*>(ws + l.cand_key);
   p.sel_score = reinterpret_cast<float*>(ws + l.sel_score);
-  p.w = reinterpret_cast<float*>(ws + l.w);
+  p.w = reinterpret_cast<uint16_t*>(ws + l.w);
   p.part = reinterpret_cast<float*>(ws + l.part);
   p.cap = cap;
   p.L = (int64_t)l.row;   // row stride of the per-token regions

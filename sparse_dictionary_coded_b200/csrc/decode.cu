@@ -1110,6 +1110,19 @@ __device__ __forceinline__ void for_records(const int32_t* list, int e0, int e1,
 // for_records without a per-entry value
 __device__ __forceinline__ float no_pay(int, int) { return 0.0f; }
 
+// x = h0 + h1 + h2 in bf16 parts, each the bf16 rounding of what the
+// previous parts leave (the remainder is below 2^-24 |x| for normal x)
+__device__ __forceinline__ void split3_bf16(float x, uint16_t& h0, uint16_t& h1, uint16_t& h2) {
+  const __nv_bfloat16 b0 = __float2bfloat16_rn(x);
+  x -= __bfloat162float(b0);
+  const __nv_bfloat16 b1 = __float2bfloat16_rn(x);
+  x -= __bfloat162float(b1);
+  const __nv_bfloat16 b2 = __float2bfloat16_rn(x);
+  h0 = __bfloat16_as_ushort(b0);
+  h1 = __bfloat16_as_ushort(b1);
+  h2 = __bfloat16_as_ushort(b2);
+}
+
 // block-wide reduction of one float per thread into s_red[0] (max or sum)
 template <bool kMax>
 __device__ __forceinline__ float block_reduce(float v, float* s_red) {
@@ -1415,7 +1428,9 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
   cluster.sync();
   const int ng = (n + 3) >> 2;
   const int g0 = (int)((int64_t)ng * rank / C), g1 = (int)((int64_t)ng * (rank + 1) / C);
-  float* gw = p.w + (int64_t)r * n;
+  // w as three bf16 parts (the operand layout of the tensor-core w D_V)
+  const int64_t plane = (int64_t)p.R * n;
+  uint16_t* gw = p.w + (int64_t)r * n;
   const int4* tiles[8];
   bool isf[8];
 #pragma unroll
@@ -1438,9 +1453,22 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
 #pragma unroll
       for (int u = 0; u < 4; ++u) sum[u] += isf[cc] ? __int_as_float(vv[u]) : (float)vv[u] * kFixInv;
     }
+    uint16_t parts[3][4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (4 * g + u < n) gw[4 * g + u] = sum[u];
+    for (int u = 0; u < 4; ++u) split3_bf16(sum[u], parts[0][u], parts[1][u], parts[2][u]);
+    if (4 * g + 3 < n && (n & 3) == 0) {
+#pragma unroll
+      for (int s3 = 0; s3 < 3; ++s3)
+        *reinterpret_cast<uint2*>(gw + s3 * plane + 4 * g) =
+            make_uint2(parts[s3][0] | ((uint32_t)parts[s3][1] << 16),
+                       parts[s3][2] | ((uint32_t)parts[s3][3] << 16));
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (4 * g + u < n)
+#pragma unroll
+          for (int s3 = 0; s3 < 3; ++s3) gw[s3 * plane + 4 * g + u] = parts[s3][u];
+    }
   }
   if (rank == 0 && tid == 0) {
     st->z = ztot;
@@ -1463,6 +1491,14 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
 // accumulators over the CTA's atoms): per atom one 8-byte value load and two
 // broadcast weight loads feed 32 FMAs.  The partial sums are added into
 // `out` (zeroed by qd_kernel) with one vector reduction per row.
+// w[r][a] from its three bf16 parts
+__device__ __forceinline__ float w_at(const DecodeParams& p, int r, int a) {
+  const int64_t plane = (int64_t)p.R * p.n, o = (int64_t)r * p.n + a;
+  const float w0 = __uint_as_float((uint32_t)__ldg(p.w + o) << 16);
+  const float w1 = __uint_as_float((uint32_t)__ldg(p.w + plane + o) << 16);
+  const float w2 = __uint_as_float((uint32_t)__ldg(p.w + 2 * plane + o) << 16);
+  return w0 + (w1 + w2);
+}
 constexpr int out_smem_bytes(int d, int rb, int tiles) {
   return tiles * kGvAtoms * d * 2 + rb * kGvAtoms * 32 * 4;
 }
@@ -1509,8 +1545,7 @@ __global__ void __launch_bounds__(D * RB) out_kernel(DecodeParams p) {
       for (int u = 0; u < kWPer; ++u) {
         const int e = e0 + u * kThreads;
         const int a = e % kGvAtoms, rr = e / kGvAtoms;
-        v[u] = (e < kW && r0 + rr < R && ta0 + a < n) ? __ldg(p.w + (int64_t)(r0 + rr) * n + ta0 + a)
-                                                        : 0.0f;
+        v[u] = (e < kW && r0 + rr < R && ta0 + a < n) ? w_at(p, r0 + rr, ta0 + a) : 0.0f;
       }
 #pragma unroll
       for (int u = 0; u < kWPer; ++u) {
@@ -1573,7 +1608,7 @@ sdk_decode_layout decode_layout(int B, int Hq, int d, int n, int64_t L) {
   l.cand_t = take(R * L * 4);
   l.cand_key = take(R * L * 4);
   l.sel_score = take(R * L * 4);
-  l.w = take(R * n * 4);
+  l.w = take(3 * R * n * 2);
   l.part = take(0);
   l.total = off;
   return l;
@@ -1738,10 +1773,10 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
   return SDK_OK;
   }
   default: {  // w D_V
-  // w D_V: tensor cores above 32 query rows; at 32 or fewer the CUDA-core
-  // kernel was measured faster (the tensor-core CTAs are latency-bound)
+  // w D_V on the tensor cores (the CUDA-core kernel where they are off or
+  // the shapes do not allow tensor maps)
   bool out_tc = false;
-  if (out_tensor_cores() && p.R > 32) {
+  if (out_tensor_cores()) {
     const sdk_status st = launch_out_tc(p, stream, &out_tc);
     if (st != SDK_OK) return st;
   }

@@ -1,22 +1,25 @@
 // out += w D_V on the 5th-generation tensor cores (decode step D6).
 //
-// out[r][c] = sum_a w[r][a] D_V[a][c]: M = R query rows, N = head_dim,
-// K = n atoms.  Each CTA takes 128 atoms (split-K) and up to 128 rows:
-//   * the atoms' value rows (bf16 [128 atoms][head_dim], 32 KB) and the rows'
-//     weights (fp32 [rows][128 atoms]) arrive with cp.async;
-//   * the value tile is transposed in shared memory into the K-major,
-//     128-byte-swizzled B operand ([head_dim][128 atoms]); the weights are
-//     split per element into three bf16 parts (w = w_hi + w_mid + w_lo, the
-//     remainder below 2^-24 |w| for normal values) forming three A operands;
-//   * one thread issues 3 x 8 tcgen05.mma (M=128, N=head_dim, K=16) into one
-//     TMEM accumulator (fp32);
-//   * four warps read it back (one row per thread) into shared memory;
-//   * CTAs run in clusters of kOCluster adjacent atom slices: CTA k of a
-//     cluster sums rows [k 128/kOCluster, (k+1) 128/kOCluster) over the
-//     cluster's partial tiles (distributed shared memory) and adds them into
-//     `out` (zeroed by the QD kernel of the call) with vector reductions, so
-//     every output element takes n / (128 kOCluster) global reductions.
-// The single wait on the MMA completion is bounded (1 s; SDK_ERR_TIMEOUT).
+// out[r][c] = sum_a w[r][a] D_V[a][c], computed transposed: out^T = D_V^T
+// w^T with M = head_dim (128; 64-dim heads use the lower half), N = up to
+// 128 query rows, K = the n atoms (split over the CTAs).  Both operands come
+// straight from global memory with TMA, in the layouts they already have:
+//   * A = a chunk of 64 atoms of D_V (bf16 [atom][head_dim], head_dim
+//     contiguous), read as an MN-major operand: two 64-element halves of the
+//     head dimension, each 64 atom rows of 128 bytes (128-byte swizzle);
+//   * B = the same 64 atoms of the three bf16 parts of w (attend writes w as
+//     w_0 + w_1 + w_2, the remainder below 2^-24 |w| for normal values),
+//     K-major ([part][row][atom], one 3-D box per chunk).
+// One thread streams the chunks through a ring of kStages stages, one thread
+// issues 3 x 4 tcgen05.mma (M=128, N, K=16) per chunk into one fp32 TMEM
+// accumulator, and the four warps read it back (thread = output column).
+// CTAs run in clusters of kWCluster consecutive atom ranges: after the
+// MMAs each CTA parks its partial tile [N][head_dim] in shared memory, and
+// CTA k of the cluster sums a quarter of the rows over the cluster's tiles
+// (distributed shared memory) and adds it into `out` (zeroed by the QD
+// kernel of the call) with vector reductions.  Every mbarrier wait is
+// bounded (1 s): on expiry the CTA records SDK_ERR_TIMEOUT, contributes a
+// zero tile and still completes the cluster's synchronisation.
 #include <cooperative_groups.h>
 
 #include "tc_ptx.cuh"
@@ -24,201 +27,210 @@
 namespace sdk {
 namespace tc {
 
-constexpr int kORows = 128;    // MMA M
-constexpr int kOAtoms = 128;   // K per CTA
-constexpr int kOThreads = 128;
-constexpr int kOSplit = 3;
-constexpr int kOCluster = 4;   // CTAs (atom slices) summed on chip per reduction
+constexpr int kWM = 128;        // MMA M (head_dim rows of out^T)
+constexpr int kWChunk = 64;     // atoms per stage: one 128-byte row of a w part
+constexpr int kWThreads = 128;  // producer lane, MMA lane, four epilogue warps
+constexpr int kWSplit = 3;      // bf16 parts of w
+constexpr int kWCluster = 4;    // CTAs whose partial tiles are summed on chip
 
-template <int D>
-struct OCfg {
-  static constexpr int kBBytes = D * kOAtoms * 2;         // B operand, bf16 [D][atoms]
-  static constexpr int kABytes = kORows * kOAtoms * 2;    // one bf16 part [rows][atoms]
-  static constexpr int kVBytes = kOAtoms * D * 2;         // staged values [atoms][D]
-  static constexpr int kWBytes = kORows * kOAtoms * 4;    // staged weights fp32
-  static constexpr int kOffB = 0;
-  static constexpr int kOffA = kOffB + kBBytes;
-  static constexpr int kOffV = kOffA + kOSplit * kABytes;
-  static constexpr int kOffW = kOffV + kVBytes;
-  // the partial tile fp32 [128][D + 4] reuses the value and weight staging
-  static constexpr int kPStride = D + 4;
-  static_assert(kORows * kPStride * 4 <= kVBytes + kWBytes, "partial tile must fit");
-  static constexpr int kOffBar = kOffW + kWBytes;
-  static constexpr int kOffMisc = kOffBar + 8;
-  static constexpr int kSmem = kOffMisc + 16 + 1024;     // + 1024-byte alignment slack
+template <int N>
+struct WCfg {
+  static constexpr int kABytes = kWM * kWChunk * 2;          // two 8 KB halves
+  static constexpr int kBBytes = kWSplit * N * kWChunk * 2;  // [part][N][64]
+  static constexpr int kStage = kABytes + kBBytes;
+  static constexpr int kStages = N <= 64 ? 4 : 3;
+  static constexpr int kPStride = kWM + 4;                   // partial tile row (floats)
+  static_assert(N * kPStride * 4 <= kStages * kStage, "partial tile must fit the ring");
+  static constexpr int kOffBar = kStages * kStage;
+  static constexpr int kNumBars = 2 * kStages + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmem = kOffMisc + 16 + 1024;         // + 1024-byte alignment slack
   static_assert(kSmem <= 232448, "exceeds the 227 KB shared memory of one sm_100 CTA");
+  static constexpr uint32_t kTmemCols = N < 32 ? 32u : (uint32_t)N;
+  // instruction descriptor: D f32, A and B bf16, A MN-major (bit 15),
+  // B K-major, N, M = 128
+  static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) |
+                                     ((uint32_t)(N >> 3) << 17) | ((uint32_t)(kWM >> 4) << 24);
 };
 
-// Instruction descriptor: D f32, A and B bf16, both K-major, N = D, M = 128.
-template <int D>
-struct OIdesc {
-  static constexpr uint32_t value = (1u << 4) | (1u << 7) | (1u << 10) |
-                                    ((uint32_t)(D >> 3) << 17) | ((uint32_t)(kORows >> 4) << 24);
-};
-
-// byte offset of the 16-byte chunk (row, chunk c) in a K-major
-// 128-byte-swizzled operand with 128 rows per 64-element K block
-__device__ __forceinline__ uint32_t swz_off(int row, int c, int rows) {
-  return (uint32_t)((c >> 3) * (rows * 128) + row * 128 + (((c & 7) ^ (row & 7)) << 4));
-}
-
-template <int D>
-__global__ void __launch_bounds__(kOThreads, 1) out_tc_kernel(DecodeParams p) {
-  using C = OCfg<D>;
+template <int D, int N>
+__global__ void __launch_bounds__(kWThreads, 1)
+    out_tc_kernel(const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap wmap,
+                  DecodeParams p) {
+  using C = WCfg<N>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem_1k(smem_raw);
-  const uint32_t bar = smem_u32(smem + C::kOffBar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
-  volatile uint32_t* s_tmem = misc;
+  volatile uint32_t* s_abort = misc + 0;
+  volatile uint32_t* s_tmem = misc + 1;
+  auto bar_full = [&](int s) { return smem_u32(&bars[s]); };
+  auto bar_empty = [&](int s) { return smem_u32(&bars[C::kStages + s]); };
+  const uint32_t bar_done = smem_u32(&bars[2 * C::kStages]);
+  const uint32_t s0 = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n = p.n, R = p.R;
-  const int a0 = blockIdx.x * kOAtoms;
-  const int r0 = blockIdx.y * kORows;
+  const int R = p.R;
+  const int nchunks = (p.n + kWChunk - 1) / kWChunk;
+  const int c0 = (int)((int64_t)nchunks * blockIdx.x / gridDim.x);
+  const int c1 = (int)((int64_t)nchunks * (blockIdx.x + 1) / gridDim.x);
+  const int r0 = blockIdx.y * N;
 
   if (tid == 0) {
-    mbar_init(bar, 1);
+    *s_abort = 0u;
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bar_full(s), 1);
+      mbar_init(bar_empty(s), 1);
+    }
+    mbar_init(bar_done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32((const void*)s_tmem)),
-                 "r"(D)
+                 "r"(C::kTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  // stage the value rows and the weights (all copies of a thread in flight)
-  const uint16_t* dv = p.dv + (int64_t)a0 * D;
-  uint4* vst = reinterpret_cast<uint4*>(smem + C::kOffV);
-  for (int e = tid; e < kOAtoms * (D / 8); e += kOThreads) {
-    const int a = e / (D / 8);
-    const bool v = a0 + a < n;
-    cp_async16(vst + e, reinterpret_cast<const uint4*>(v ? dv : p.dv) + (v ? e : 0), v);
+  if (D < kWM) {
+    // 64-dim heads: the upper half of every A stage (rows 64..127 of out^T)
+    // stays zero; TMA writes only the lower half
+    for (int s = 0; s < C::kStages; ++s)
+      for (int e = tid; e < 8192 / 16; e += kWThreads)
+        reinterpret_cast<uint4*>(smem + s * C::kStage + 8192)[e] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async();
   }
-  float* wst = reinterpret_cast<float*>(smem + C::kOffW);
-  for (int e = tid; e < kORows * (kOAtoms / 4); e += kOThreads) {
-    const int i = e / (kOAtoms / 4), c4 = e % (kOAtoms / 4);
-    const bool v = r0 + i < R && a0 + 4 * c4 + 3 < n;
-    const float* src = v ? p.w + (int64_t)(r0 + i) * n + a0 + 4 * c4 : p.w;
-    cp_async16(wst + i * kOAtoms + 4 * c4, src, v);
-  }
-  cp_async_commit();
-  cp_async_wait<0>();
-  __syncthreads();
-  // weights of a partial last tile that do not fill 16 bytes: plain loads
-  if (a0 + kOAtoms > n) {
-    for (int e = tid; e < kORows * kOAtoms; e += kOThreads) {
-      const int i = e / kOAtoms, a = e % kOAtoms;
-      const int c4 = a >> 2;
-      const bool vec = r0 + i < R && a0 + 4 * c4 + 3 < n;
-      if (!vec) wst[e] = (r0 + i < R && a0 + a < n) ? p.w[(int64_t)(r0 + i) * n + a0 + a] : 0.0f;
-    }
-    __syncthreads();
-  }
-  // B operand: transpose [atoms][D] -> K-major [D][atoms]; thread takes
-  // 8 consecutive atoms of one column c (one 16-byte chunk of the operand)
-  const uint16_t* vs = reinterpret_cast<const uint16_t*>(smem + C::kOffV);
-  for (int e = tid; e < D * (kOAtoms / 8); e += kOThreads) {
-    const int c = e % D, ch = e / D;            // c: column (operand row), ch: atom chunk
-    uint32_t w4[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const uint32_t lo = vs[(ch * 8 + 2 * u) * D + c];
-      const uint32_t hi = vs[(ch * 8 + 2 * u + 1) * D + c];
-      w4[u] = lo | (hi << 16);
-    }
-    *reinterpret_cast<uint4*>(smem + C::kOffB + swz_off(c, ch, D)) =
-        make_uint4(w4[0], w4[1], w4[2], w4[3]);
-  }
-  // A operands: three bf16 parts of the weights
-  for (int e = tid; e < kORows * (kOAtoms / 8); e += kOThreads) {
-    const int i = e / (kOAtoms / 8), ch = e % (kOAtoms / 8);
-    const float4 x0 = *reinterpret_cast<const float4*>(wst + i * kOAtoms + ch * 8);
-    const float4 x1 = *reinterpret_cast<const float4*>(wst + i * kOAtoms + ch * 8 + 4);
-    const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-    uint32_t w[kOSplit][4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      float a0f = v[2 * u], a1f = v[2 * u + 1];
-#pragma unroll
-      for (int s = 0; s < kOSplit; ++s) {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(a0f, a1f);
-        w[s][u] = *reinterpret_cast<const uint32_t*>(&h);
-        a0f -= __low2float(h);
-        a1f -= __high2float(h);
-      }
-    }
-#pragma unroll
-    for (int s = 0; s < kOSplit; ++s)
-      *reinterpret_cast<uint4*>(smem + C::kOffA + s * C::kABytes + swz_off(i, ch, kORows)) =
-          make_uint4(w[s][0], w[s][1], w[s][2], w[s][3]);
-  }
-  fence_proxy_async();   // generic stores of the operands before the MMAs read them
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
-  if (tid == 0) {
-    const uint32_t sA = smem_u32(smem + C::kOffA), sB = smem_u32(smem + C::kOffB);
-#pragma unroll
-    for (int s = 0; s < kOSplit; ++s)
-#pragma unroll
-      for (int ks = 0; ks < kOAtoms / 16; ++ks) {
-        const uint32_t koffA = (ks >> 2) * (kORows * 128) + (ks & 3) * 32;
-        const uint32_t koffB = (ks >> 2) * (D * 128) + (ks & 3) * 32;
-        tc_mma(tmem, smem_desc(sA + s * C::kABytes + koffA), smem_desc(sB + koffB),
-               OIdesc<D>::value, (s > 0 || ks > 0) ? 1u : 0u);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, issued_mask = 0, last_phase = 0;
+      bool ok = true;
+      for (int c = c0; c < c1; ++c) {
+        if (!mbar_wait(bar_empty(stage), phase ^ 1u, s_abort)) {
+          ok = false;
+          break;
+        }
+        const uint32_t st = s0 + stage * C::kStage;
+        mbar_expect_tx(bar_full(stage), (uint32_t)(D * kWChunk * 2 + C::kBBytes));
+        tma_load_2d(st, &vmap, 0, c * kWChunk, bar_full(stage));
+        if (D > 64) tma_load_2d(st + 8192, &vmap, 64, c * kWChunk, bar_full(stage));
+        tma_load_3d(st + C::kABytes, &wmap, c * kWChunk, r0, 0, bar_full(stage));
+        issued_mask |= 1u << stage;
+        last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
       }
-    tc_commit(bar);
+      if (!ok) {
+        record_error(p.hdr, SDK_ERR_TIMEOUT, 0x54000000u | blockIdx.x);
+        *s_abort = 1u;
+      }
+      // every copy issued has landed before the CTA may leave
+      for (int s = 0; s < C::kStages; ++s)
+        if (issued_mask & (1u << s)) {
+          uint32_t dummy = 0u;
+          mbar_wait(bar_full(s), (last_phase >> s) & 1u, &dummy, 100000000ull);
+        }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, issued = false;
+      for (int c = c0; c < c1; ++c) {
+        if (!mbar_wait(bar_full(stage), phase, s_abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = s0 + stage * C::kStage, sb = sa + C::kABytes;
+#pragma unroll
+        for (int s = 0; s < kWSplit; ++s)
+#pragma unroll
+          for (int ks = 0; ks < kWChunk / 16; ++ks) {
+            // A: 16 atoms = two 8-row swizzle atoms (2048 bytes); the two
+            // halves of the head dimension are 8192 bytes apart.  B: 16
+            // atoms = 32 bytes along the K-major rows of part s.
+            tc_mma(tmem, smem_desc_mn(sa + ks * 2048, 8192u, 1024u),
+                   smem_desc(sb + s * (N * 128) + ks * 32), C::kIdesc,
+                   (issued || s > 0 || ks > 0) ? 1u : 0u);
+          }
+        issued = true;
+        tc_commit(bar_empty(stage));
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) {
+        record_error(p.hdr, SDK_ERR_TIMEOUT, 0x55000000u | blockIdx.x);
+        *s_abort = 1u;
+      }
+      // arrives once every MMA issued has completed (at once if none was)
+      tc_commit(bar_done);
+    }
   }
   __syncwarp();
-  // every warp waits for the accumulator (lane 0 waits, bounded)
+
+  // ------------------------------------------------------------ epilogue
+  // thread i = TMEM lane i = column i of out (row i of out^T)
   uint32_t never = 0u;
-  const bool got = lane == 0 ? mbar_wait(bar, 0u, &never) : true;
-  const bool ok = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
-  if (!ok && lane == 0) record_error(p.hdr, SDK_ERR_TIMEOUT, 0x53000000u | blockIdx.x);
+  const bool got = lane == 0 ? mbar_wait(bar_done, 0u, &never) : true;
+  const bool done = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+  if (!done && lane == 0) record_error(p.hdr, SDK_ERR_TIMEOUT, 0x56000000u | blockIdx.x);
   tc_fence_after();
-  // the accumulator into shared memory, one row per thread (zeros if the
-  // MMAs timed out: the error is recorded, the cluster still completes)
-  float* part = reinterpret_cast<float*>(smem + C::kOffV);
+  __syncthreads();   // the ring is free: the partial tile [N][kPStride] reuses it
+  const bool have = done && c1 > c0 && *s_abort == 0u;
+  float* part = reinterpret_cast<float*>(smem);
   {
     const int i = warp * 32 + lane;
 #pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
+    for (int cb = 0; cb < N; cb += 32) {
       uint32_t v[32];
-      if (ok) {
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c0, v);
+      if (have && warp * 32 < D) {
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + cb, v);
         tmem_ld_wait();
       } else {
 #pragma unroll
         for (int u = 0; u < 32; ++u) v[u] = 0u;
       }
+      if (i < D) {
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        *reinterpret_cast<uint4*>(part + i * C::kPStride + c0 + 4 * u) =
-            make_uint4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+        for (int u = 0; u < 32; ++u)
+          if (cb + u < N) part[(cb + u) * C::kPStride + i] = __uint_as_float(v[u]);
+      }
     }
   }
   tc_fence_before();
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   cluster.sync();
-  // this CTA's rows of the cluster's sum, into `out`
   {
     const int cr = (int)cluster.block_rank();
-    constexpr int kRowsPer = kORows / kOCluster;
-    const float* parts[kOCluster];
+    constexpr int kRowsPer = N / kWCluster;
+    const float* parts[kWCluster];
 #pragma unroll
-    for (int k = 0; k < kOCluster; ++k) parts[k] = cluster.map_shared_rank(part, k);
-    for (int e = tid; e < kRowsPer * (D / 4); e += kOThreads) {
+    for (int k = 0; k < kWCluster; ++k) parts[k] = cluster.map_shared_rank(part, k);
+    for (int e = tid; e < kRowsPer * (D / 4); e += kWThreads) {
       const int i = cr * kRowsPer + e / (D / 4), c4 = e % (D / 4);
       if (r0 + i >= R) continue;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 x[kWCluster];
 #pragma unroll
-      for (int k = 0; k < kOCluster; ++k) {
-        const float4 x = *reinterpret_cast<const float4*>(parts[k] + i * C::kPStride + 4 * c4);
-        acc.x += x.x;
-        acc.y += x.y;
-        acc.z += x.z;
-        acc.w += x.w;
+      for (int k = 0; k < kWCluster; ++k)
+        x[k] = *reinterpret_cast<const float4*>(parts[k] + i * C::kPStride + 4 * c4);
+      float4 acc = x[0];
+#pragma unroll
+      for (int k = 1; k < kWCluster; ++k) {
+        acc.x += x[k].x;
+        acc.y += x[k].y;
+        acc.z += x[k].z;
+        acc.w += x[k].w;
       }
       float* dst = p.out + (int64_t)(r0 + i) * D + 4 * c4;
       asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(acc.x),
@@ -227,47 +239,106 @@ __global__ void __launch_bounds__(kOThreads, 1) out_tc_kernel(DecodeParams p) {
     }
   }
   cluster.sync();   // the peers' tiles are read before any CTA leaves
-  __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(D)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(C::kTmemCols)
                  : "memory");
   }
 }
 
-}  // namespace tc
-
-// w D_V on the tensor cores; *taken = false when not available.
-sdk_status launch_out_tc(const DecodeParams& p, cudaStream_t stream, bool* taken) {
-  *taken = false;
-  // 16-byte weight copies need rows of a multiple of 4 atoms
-  if ((p.d != 64 && p.d != 128) || (p.n & 3) != 0) return SDK_OK;
-  *taken = true;
+// Launches out_tc_kernel<D, N> over ty row tiles and up to gx atom ranges
+// (fewer when fewer clusters of this kernel fit the device at once).
+template <int D, int N>
+static cudaError_t launch_w(const CUtensorMap& vmap, const CUtensorMap& wmap, const DecodeParams& p,
+                            int gx, int ty, cudaStream_t stream) {
   static unsigned long long attr_set = 0ull;
-  if (device_needs_setup(&attr_set)) {
-    cudaFuncSetAttribute(tc::out_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         tc::OCfg<128>::kSmem);
-    cudaFuncSetAttribute(tc::out_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         tc::OCfg<64>::kSmem);
-    device_setup_done(&attr_set);
-  }
-  // atom slices rounded up to whole clusters (slices past n are zero)
-  int slices = (p.n + tc::kOAtoms - 1) / tc::kOAtoms;
-  slices = (slices + tc::kOCluster - 1) / tc::kOCluster * tc::kOCluster;
+  static int max_clusters[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)slices, (unsigned)((p.R + tc::kORows - 1) / tc::kORows));
-  cfg.blockDim = dim3(tc::kOThreads);
-  cfg.dynamicSmemBytes = p.d == 128 ? tc::OCfg<128>::kSmem : tc::OCfg<64>::kSmem;
+  cfg.blockDim = dim3(kWThreads);
+  cfg.dynamicSmemBytes = WCfg<N>::kSmem;
   cfg.stream = stream;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = tc::kOCluster;
+  at[0].val.clusterDim.x = kWCluster;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  const cudaError_t e = p.d == 128 ? cudaLaunchKernelEx(&cfg, tc::out_tc_kernel<128>, p)
-                                   : cudaLaunchKernelEx(&cfg, tc::out_tc_kernel<64>, p);
+  if (device_needs_setup(&attr_set)) {
+    cudaFuncSetAttribute(out_tc_kernel<D, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         WCfg<N>::kSmem);
+    int mc = 0;
+    cfg.gridDim = dim3(kWCluster);
+    if (cudaOccupancyMaxActiveClusters(&mc, out_tc_kernel<D, N>, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      mc = 0;
+    }
+    if (dev >= 0 && dev < 64) max_clusters[dev] = mc;
+    device_setup_done(&attr_set);
+  }
+  const int mc = (dev >= 0 && dev < 64) ? max_clusters[dev] : 0;
+  if (mc > 0 && gx * ty > mc * kWCluster) gx = mc * kWCluster / ty / kWCluster * kWCluster;
+  if (gx < kWCluster) gx = kWCluster;
+  cfg.gridDim = dim3((unsigned)gx, (unsigned)ty);
+  cfg.blockDim = dim3(kWThreads);
+  return cudaLaunchKernelEx(&cfg, out_tc_kernel<D, N>, vmap, wmap, p);
+}
+
+}  // namespace tc
+
+// w D_V on the tensor cores; *taken = false when the path is not available
+// (head_dim other than 64/128, rows of w that are not a multiple of 16
+// bytes, or no driver entry point for tensor maps).
+sdk_status launch_out_tc(const DecodeParams& p, cudaStream_t stream, bool* taken) {
+  *taken = false;
+  if ((p.d != 64 && p.d != 128) || (p.n % 8) != 0 || p.R < 1) return SDK_OK;
+  auto fn = tc::encode_fn();
+  if (fn == nullptr) return SDK_OK;
+  // D_V [n][d] bf16: boxes of 64 head-dim elements x 64 atoms
+  CUtensorMap vmap, wmap;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)p.d, (cuuint64_t)p.n};
+    const cuuint64_t strides[1] = {(cuuint64_t)p.d * 2};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)tc::kWChunk};
+    const cuuint32_t estr[2] = {1u, 1u};
+    if (fn(&vmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(p.dv), dims, strides,
+           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return SDK_OK;
+  }
+  // rows per tile: the smallest of 32 / 64 / 128 that holds R (128 above)
+  const int N = p.R <= 32 ? 32 : (p.R <= 64 ? 64 : 128);
+  {
+    // w parts [3][R][n] bf16: boxes of 64 atoms x N rows x 3 parts (rows
+    // past R read as zero)
+    const cuuint64_t dims[3] = {(cuuint64_t)p.n, (cuuint64_t)p.R, (cuuint64_t)tc::kWSplit};
+    const cuuint64_t strides[2] = {(cuuint64_t)p.n * 2, (cuuint64_t)p.R * p.n * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)tc::kWChunk, (cuuint32_t)N, (cuuint32_t)tc::kWSplit};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    if (fn(&wmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.w, dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return SDK_OK;
+  }
+  *taken = true;
+  // atom ranges: whole clusters, about one CTA per SM over all row tiles
+  const int ty = (p.R + N - 1) / N;
+  const int nchunks = (p.n + tc::kWChunk - 1) / tc::kWChunk;
+  int gx = num_sms() / ty;
+  if (gx > nchunks) gx = nchunks;
+  gx = gx / tc::kWCluster * tc::kWCluster;
+  cudaError_t e;
+  if (p.d == 128)
+    e = N == 32 ? tc::launch_w<128, 32>(vmap, wmap, p, gx, ty, stream)
+        : N == 64 ? tc::launch_w<128, 64>(vmap, wmap, p, gx, ty, stream)
+                  : tc::launch_w<128, 128>(vmap, wmap, p, gx, ty, stream);
+  else
+    e = N == 32 ? tc::launch_w<64, 32>(vmap, wmap, p, gx, ty, stream)
+        : N == 64 ? tc::launch_w<64, 64>(vmap, wmap, p, gx, ty, stream)
+                  : tc::launch_w<64, 128>(vmap, wmap, p, gx, ty, stream);
   return e == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
 }
 

@@ -170,7 +170,7 @@ struct DecodeParams {
   int32_t* cand_t;
   uint32_t* cand_key;
   float* sel_score;
-  float* w;
+  uint16_t* w;           // bf16 [3][R][n]: w = w[0] + w[1] + w[2] per (row, atom)
   float* part;
   WsHeader* hdr;
   int64_t cap;

@@ -346,16 +346,22 @@ def test_full_size_layer_sampled_heads(name, isoft):
         assert np.max(np.abs(outn[b, h] - ref["out"])) <= OUT_TOL
 
 
+_QD_PATH_NAMES = ("b1", "b2", "b4", "b2-640", "b1-d64", "b2-128", "b8", "b3-h12")
 _QD_PATH_CASE = r"""
 import sys, numpy as np, torch
+CASES = (("b1", (81, 1, 32, 8, 2000, 128, 32768)),
+         ("b2", (83, 2, 32, 8, 900, 64, 2048)),
+         ("b4", (82, 4, 32, 8, 600, 128, 4096)),
+         ("b2-640", (84, 2, 32, 8, 700, 128, 640)),
+         ("b1-d64", (86, 1, 32, 8, 1500, 64, 4096)),
+         ("b2-128", (85, 2, 32, 8, 300, 128, 128)),
+         ("b8", (87, 8, 32, 8, 200, 128, 2048)),
+         ("b3-h12", (88, 3, 12, 4, 400, 128, 1024)))
 sys.path.insert(0, sys.argv[1])
 sys.path.insert(0, sys.argv[1] + "/tests")
 import workloads, sparse_dictionary_coded_b200 as sdk
 from test_gpu_decode import _random_case, _store
-for name, args in (("b1", (81, 1, 32, 8, 2000, 128, 32768)),
-                   ("b2", (83, 2, 32, 8, 900, 64, 2048)),
-                   ("b4", (82, 4, 32, 8, 600, 128, 4096)),
-                   ("b2-640", (84, 2, 32, 8, 700, 128, 640))):
+for name, args in CASES:
     q, DK, DV, kw, vw, lens = _random_case(*args)
     B, Hq, d = q.shape
     store = _store(kw, vw, lens)
@@ -376,10 +382,12 @@ def test_gemvs_on_cuda_cores_match_tensor_cores(tmp_path):
     """D1 and D6 run on the tensor cores (q and w split into three bf16
     parts) unless SDK_DECODE_QD_TC=0 / SDK_DECODE_OUT_TC=0 select the fp32
     CUDA-core kernels (read once per process, hence child processes): both
-    give QD within fp32 rounding of each other and the same outputs, at 32,
-    64 (head_dim 64) and 128 query rows, and with 640 atoms (five atom
-    slices: the tensor-core w D_V runs clusters of four, three of them
-    empty)."""
+    give QD within fp32 rounding of each other and the same outputs.  The
+    w D_V cases cover 32, 64 and 128 query rows (row tiles of 32, 64, 128),
+    256 rows (two row tiles of 128), 36 rows (a tile of 64 with 28 empty
+    rows), head_dim 64 at 32 and 64 rows (the zero upper half of the
+    operand), 640 atoms (ten chunks over eight CTAs) and 128 atoms (two
+    chunks: two of the cluster's four CTAs have no atoms)."""
     import os
     import subprocess
     import sys
@@ -393,7 +401,7 @@ def test_gemvs_on_cuda_cores_match_tensor_cores(tmp_path):
                            env=env, capture_output=True, text=True, timeout=600)
         assert r.returncode == 0, r.stdout + r.stderr
         res[mode] = d
-    for name in ("b1", "b2", "b4", "b2-640"):
+    for name in _QD_PATH_NAMES:
         qa = np.load(res["1"] / ("qd_" + name + ".npy"))
         qb = np.load(res["0"] / ("qd_" + name + ".npy"))
         assert np.max(np.abs(qa - qb)) <= 2e-6 * np.max(np.abs(qb))
