@@ -181,7 +181,7 @@ SDK_API size_t sdk_append_workspace_bytes(int32_t B, int32_t Hkv, int32_t n_new,
  *   w[a]    = sum_t p_t sum_j c^V_tj [idx^V_tj == a] (over the softmax domain)
  *   out     = w D_V
  *
- *   q          device, float [B][Hq][head_dim]
+ *   q          device, float [B][Hq][head_dim], 16-byte aligned
  *   dict_k/_v  device, bf16 [n_atoms][head_dim]
  *   lens_host  host, int32 [B], 1 <= lens[b] <= cap
  *   klow       1 .. khigh;  khigh  klow .. 16

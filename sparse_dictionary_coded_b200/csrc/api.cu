@@ -341,7 +341,7 @@ static sdk_status build_decode_params(const float* q, int32_t B, int32_t Hq, int
   if (!q || !dict_k || !dict_v || !k_lo || !k_full || !v_full || !out || !lens_host || !workspace)
     return SDK_ERR_INVALID_ARG;
   if (!aligned(workspace, SDK_WS_ALIGN) || !aligned(dict_k, 16) || !aligned(dict_v, 16) ||
-      !aligned(k_full, 16) || !aligned(v_full, 16) || !aligned(k_lo, 4) || !aligned(q, 4) ||
+      !aligned(k_full, 16) || !aligned(v_full, 16) || !aligned(k_lo, 4) || !aligned(q, 16) ||
       !aligned(out, 16))
     return SDK_ERR_INVALID_ARG;
   int64_t max_len = 0;

@@ -1,20 +1,24 @@
 // QD = q D_K^T on the 5th-generation tensor cores (decode step D1).
 //
-// QD[r][a] = sum_k q[r][k] D_K[a][k] for R query rows against all n atoms:
-// a dense contraction (M = R, N = n, K = head_dim) whose B operand is the
-// bf16 dictionary itself.  q is fp32; to keep fp32 accuracy it is split per
-// element into three bf16 parts, q = q_hi + q_mid + q_lo (each the bf16
-// rounding of what the previous parts leave; the remainder is below 2^-24
-// |q| for normal values), and the three products with the exact bf16 atoms
-// accumulate in fp32 in tensor memory: 3 x (head_dim / 16) MMAs per atom
-// tile.
+// QD[r][a] = sum_k q[r][k] D_K[a][k] for R query rows against all n atoms,
+// computed transposed: QD^T = D_K q^T with M = 128 atoms per tile, N = up
+// to 128 query rows, K = head_dim.  The A operand is the bf16 dictionary
+// tile itself (TMA, 128-byte swizzle, K-major); q is fp32, and to keep fp32
+// accuracy each element is split into three bf16 parts, q = q_hi + q_mid +
+// q_lo (each the bf16 rounding of what the previous parts leave; the
+// remainder is below 2^-24 |q| for normal values), written by the CTA's
+// threads as three K-major B operands.  The three products with the exact
+// bf16 atoms accumulate in fp32 in tensor memory: 3 x (head_dim / 16) MMAs
+// per atom tile.
 //
-// One CTA per (row block of 128 query rows, strided set of 128-atom tiles),
-// 6 warps: warp 0 streams dictionary tiles with TMA through a kQStages ring
-// (128-byte swizzle, K-major), warp 1 issues tcgen05.mma (M=128, N=128,
-// K=16) into one of two TMEM accumulators, warps 2..5 read the accumulator
-// of a tile (tcgen05.ld, one row per thread) and store it to QD.  Rows past
-// R are zero in the A operand and are not stored.  Every mbarrier wait is
+// One CTA per (row tile of N query rows, strided set of 128-atom tiles), 6
+// warps: warp 0 streams dictionary tiles with TMA through a kQStages ring
+// from the first instruction on, warps 1..5 meanwhile zero the per-call
+// state and build the q parts, then warp 1 issues tcgen05.mma (M=128, N,
+// K=16) into one of two TMEM accumulators and warps 2..5 read an
+// accumulator back (tcgen05.ld, thread = atom, columns = query rows) and
+// store it to QD, 128 consecutive atoms of a row per warp store.  Rows past
+// R are zero in the B operand and are not stored.  Every mbarrier wait is
 // bounded (1 s); on expiry the CTA records SDK_ERR_TIMEOUT and stops.
 //
 // Like the CUDA-core QD kernel this first kernel of a decode call also
@@ -24,42 +28,41 @@
 namespace sdk {
 namespace tc {
 
-constexpr int kQRows = 128;     // MMA M
-constexpr int kQAtoms = 128;    // MMA N
+constexpr int kQAtoms = 128;    // MMA M
 constexpr int kQStages = 3;
 constexpr int kQThreads = 192;  // producer, MMA issuer, 4 epilogue warps
 constexpr int kQSplit = 3;      // bf16 parts of q
 
-template <int D>
+template <int D, int N>
 struct QCfg {
   static constexpr int KB = D / 64;                     // 128-byte K blocks
   static constexpr int KSTEPS = D / 16;
-  static constexpr int kStageBytes = kQAtoms * D * 2;
-  static constexpr int kABytes = kQRows * D * 2;        // one bf16 part
-  static constexpr int kOffA = kQStages * kStageBytes;
-  static constexpr int kOffBar = kOffA + kQSplit * kABytes;
+  static constexpr int kStageBytes = kQAtoms * D * 2;   // one dictionary tile
+  static constexpr int kBBytes = N * D * 2;             // one bf16 part of q
+  static constexpr int kOffB = kQStages * kStageBytes;
+  static constexpr int kOffBar = kOffB + kQSplit * kBBytes;
   static constexpr int kNumBars = 2 * kQStages + 2 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmem = kOffMisc + 64 + 1024;   // + 1024-byte alignment slack
   static_assert(kSmem <= 232448, "exceeds the 227 KB shared memory of one sm_100 CTA");
+  static constexpr uint32_t kTmemCols = 2 * N < 32 ? 32u : (uint32_t)(2 * N);
+  // instruction descriptor: D f32, A and B bf16, both K-major, N, M = 128
+  static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                                     ((uint32_t)(N >> 3) << 17) | ((uint32_t)(kQAtoms >> 4) << 24);
 };
 
-// Instruction descriptor: D f32, A and B bf16, both K-major, N=128, M=128.
-constexpr uint32_t kQIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                             ((uint32_t)(kQAtoms >> 3) << 17) | ((uint32_t)(kQRows >> 4) << 24);
-
-template <int D>
+template <int D, int N>
 __global__ void __launch_bounds__(kQThreads, 1)
     qd_tc_kernel(const __grid_constant__ CUtensorMap tmap, DecodeParams p) {
-  using C = QCfg<D>;
+  using C = QCfg<D, N>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem_1k(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile uint32_t* s_abort = misc + 0;
   volatile uint32_t* s_tmem = misc + 1;
-  const uint32_t sB = smem_u32(smem);
-  const uint32_t sA = smem_u32(smem + C::kOffA);
+  const uint32_t sA = smem_u32(smem);
+  const uint32_t sB = smem_u32(smem + C::kOffB);
   auto bar_full = [&](int s) { return smem_u32(&bars[s]); };
   auto bar_empty = [&](int s) { return smem_u32(&bars[kQStages + s]); };
   auto bar_tfull = [&](int b) { return smem_u32(&bars[2 * kQStages + b]); };
@@ -67,13 +70,76 @@ __global__ void __launch_bounds__(kQThreads, 1)
   const uint32_t bar_done = smem_u32(&bars[2 * kQStages + 4]);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = p.n, R = p.R;
-  const int r0 = blockIdx.y * kQRows;
+  const int r0 = blockIdx.y * N;
   const int n_atom_tiles = (n + kQAtoms - 1) / kQAtoms;
 
-  // per-call state: selection state, histograms, out
+  if (tid == 0) {
+    *s_abort = 0u;
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(bar_full(s), 1);
+      mbar_init(bar_empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_tfull(b), 1);
+      mbar_init(bar_tempty(b), 4);
+    }
+    mbar_init(bar_done, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32((const void*)s_tmem)),
+                 "r"(C::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, issued_mask = 0, last_phase = 0;
+      bool ok = true;
+      for (int a = blockIdx.x; ok && a < n_atom_tiles; a += gridDim.x) {
+        if (!mbar_wait(bar_empty(stage), phase ^ 1u, s_abort)) {
+          ok = false;
+          break;
+        }
+        mbar_expect_tx(bar_full(stage), (uint32_t)C::kStageBytes);
+#pragma unroll
+        for (int kb = 0; kb < C::KB; ++kb)
+          tma_load_2d(sA + stage * C::kStageBytes + kb * (kQAtoms * 128), &tmap, kb * 64,
+                      a * kQAtoms, bar_full(stage));
+        issued_mask |= 1u << stage;
+        last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
+        if (++stage == kQStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) {
+        record_error(p.hdr, SDK_ERR_TIMEOUT, 0x50000000u | blockIdx.x);
+        *s_abort = 1u;
+      }
+      for (int s = 0; s < kQStages; ++s)
+        if (issued_mask & (1u << s)) {
+          uint32_t dummy = 0u;
+          mbar_wait(bar_full(s), (last_phase >> s) & 1u, &dummy, 100000000ull);
+        }
+    }
+    return;
+  }
+
+  // ---- warps 1..5, while the first tiles load: the per-call state
+  // (selection state, histograms, out) and the B operands
   {
-    const int64_t nthr = (int64_t)gridDim.x * gridDim.y * kQThreads;
-    const int64_t g0 = ((int64_t)blockIdx.y * gridDim.x + blockIdx.x) * kQThreads + tid;
+    constexpr int kT = kQThreads - 32;
+    const int t = tid - 32;
+    const int64_t nthr = (int64_t)gridDim.x * gridDim.y * kT;
+    const int64_t g0 = ((int64_t)blockIdx.y * gridDim.x + blockIdx.x) * kT + t;
     const int64_t hwords = (int64_t)R * 4096;
     for (int64_t e = g0; e < hwords; e += nthr) {
       p.hist1[e] = 0u;
@@ -93,110 +159,63 @@ __global__ void __launch_bounds__(kQThreads, 1)
       st.pad[0] = st.pad[1] = 0u;
       p.st[e] = st;
     }
+    // B operands: the three bf16 parts of the tile's query rows in the
+    // 128-byte-swizzled K-major layout (8 elements = one 16-byte chunk;
+    // chunk c of K block kb of row i lives at kb*N*128 + i*128 +
+    // ((c^(i&7))*16)); rows past R are zero
+    // (the loads of kQBatch chunks are in flight before the first is used)
+    constexpr int kItems = N * (D / 8), kQBatch = 8;
+    for (int e0 = t; e0 < kItems; e0 += kQBatch * kT) {
+      float4 x[kQBatch][2];
+#pragma unroll
+      for (int u = 0; u < kQBatch; ++u) {
+        const int e = e0 + u * kT;
+        const int i = e / (D / 8), kc = e % (D / 8);
+        if (e < kItems && r0 + i < R) {   // q is 16-byte aligned (checked by the API)
+          const float4* src =
+              reinterpret_cast<const float4*>(p.q + (int64_t)(r0 + i) * D + kc * 8);
+          x[u][0] = __ldg(src);
+          x[u][1] = __ldg(src + 1);
+        } else {
+          x[u][0] = x[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kQBatch; ++u) {
+        const int e = e0 + u * kT;
+        if (e >= kItems) break;
+        const int i = e / (D / 8), kc = e % (D / 8);
+        const float v[8] = {x[u][0].x, x[u][0].y, x[u][0].z, x[u][0].w,
+                            x[u][1].x, x[u][1].y, x[u][1].z, x[u][1].w};
+        uint32_t w[kQSplit][4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float a0 = v[2 * c], a1 = v[2 * c + 1];
+#pragma unroll
+          for (int s = 0; s < kQSplit; ++s) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(a0, a1);
+            w[s][c] = *reinterpret_cast<const uint32_t*>(&h);
+            a0 -= __low2float(h);       // exact: the rounding error of a0
+            a1 -= __high2float(h);
+          }
+        }
+        const int kb = kc >> 3, c16 = kc & 7;
+#pragma unroll
+        for (int s = 0; s < kQSplit; ++s) {
+          uint4* dst = reinterpret_cast<uint4*>(smem + C::kOffB + s * C::kBBytes +
+                                                kb * (N * 128) + i * 128 + ((c16 ^ (i & 7)) << 4));
+          *dst = make_uint4(w[s][0], w[s][1], w[s][2], w[s][3]);
+        }
+      }
+    }
+    fence_proxy_async();   // generic-proxy stores of B before the MMAs read them
+    asm volatile("bar.sync 1, %0;" ::"r"(kT) : "memory");
   }
 
-  if (tid == 0) {
-    *s_abort = 0u;
-    for (int s = 0; s < kQStages; ++s) {
-      mbar_init(bar_full(s), 1);
-      mbar_init(bar_empty(s), 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar_tfull(b), 1);
-      mbar_init(bar_tempty(b), 4);
-    }
-    mbar_init(bar_done, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32((const void*)s_tmem)),
-                 "r"(256)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  // A operand: the three bf16 parts of the block's query rows, written in
-  // the 128-byte-swizzled K-major layout (8 elements = one 16-byte chunk;
-  // chunk c of K block kb of row i lives at kb*128*128 + i*128 + ((c^(i&7))*16)).
-  // The fp32 rows first land in the (still unused) B ring with cp.async, all
-  // of a thread's copies in flight at once.
-  float* qs = reinterpret_cast<float*>(smem);   // [kQRows][D] fp32, < the B ring
-  static_assert(kQRows * D * 4 <= kQStages * C::kStageBytes, "q staging must fit the B ring");
-  for (int e = tid; e < kQRows * (D / 4); e += kQThreads) {
-    const int i = e / (D / 4), c4 = e % (D / 4);
-    const bool v = r0 + i < R;
-    cp_async16(qs + i * D + 4 * c4, p.q + (int64_t)(v ? r0 + i : 0) * D + 4 * c4, v);
-  }
-  cp_async_commit();
-  cp_async_wait<0>();
-  __syncthreads();
-  for (int e = tid; e < kQRows * (D / 8); e += kQThreads) {
-    const int i = e / (D / 8), kc = e % (D / 8);
-    const float4 x0 = *reinterpret_cast<const float4*>(qs + i * D + kc * 8);
-    const float4 x1 = *reinterpret_cast<const float4*>(qs + i * D + kc * 8 + 4);
-    const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-    uint32_t w[kQSplit][4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      float a0 = v[2 * u], a1 = v[2 * u + 1];
-#pragma unroll
-      for (int s = 0; s < kQSplit; ++s) {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(a0, a1);
-        w[s][u] = *reinterpret_cast<const uint32_t*>(&h);
-        a0 -= __low2float(h);       // exact: the rounding error of a0
-        a1 -= __high2float(h);
-      }
-    }
-    const int kb = kc >> 3, c16 = kc & 7;
-#pragma unroll
-    for (int s = 0; s < kQSplit; ++s) {
-      uint4* dst = reinterpret_cast<uint4*>(smem + C::kOffA + s * C::kABytes + kb * (kQRows * 128) +
-                                            i * 128 + ((c16 ^ (i & 7)) << 4));
-      *dst = make_uint4(w[s][0], w[s][1], w[s][2], w[s][3]);
-    }
-  }
-  __syncthreads();   // the staged rows are read before the producer refills the ring
-  fence_proxy_async();   // generic-proxy stores of A before the MMAs read them
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *s_tmem;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0, issued_mask = 0, last_phase = 0;
-      bool ok = true;
-      for (int a = blockIdx.x; ok && a < n_atom_tiles; a += gridDim.x) {
-        if (!mbar_wait(bar_empty(stage), phase ^ 1u, s_abort)) {
-          ok = false;
-          break;
-        }
-        mbar_expect_tx(bar_full(stage), (uint32_t)C::kStageBytes);
-#pragma unroll
-        for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_2d(sB + stage * C::kStageBytes + kb * (kQAtoms * 128), &tmap, kb * 64,
-                      a * kQAtoms, bar_full(stage));
-        issued_mask |= 1u << stage;
-        last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
-        if (++stage == kQStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
-      }
-      if (!ok) {
-        record_error(p.hdr, SDK_ERR_TIMEOUT, 0x50000000u | blockIdx.x);
-        *s_abort = 1u;
-      }
-      for (int s = 0; s < kQStages; ++s)
-        if (issued_mask & (1u << s)) {
-          uint32_t dummy = 0u;
-          mbar_wait(bar_full(s), (last_phase >> s) & 1u, &dummy, 100000000ull);
-        }
-    }
-  } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
+      tc_fence_after();
       int stage = 0;
       uint32_t phase = 0, tbuf = 0, tphase = 0;
       bool ok = true, issued = false;
@@ -207,16 +226,16 @@ __global__ void __launch_bounds__(kQThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t bbase = sB + stage * C::kStageBytes;
-        const uint32_t d_tmem = tmem + tbuf * kQAtoms;
+        const uint32_t abase = sA + stage * C::kStageBytes;
+        const uint32_t d_tmem = tmem + tbuf * N;
 #pragma unroll
         for (int s = 0; s < kQSplit; ++s)
 #pragma unroll
           for (int ks = 0; ks < C::KSTEPS; ++ks) {
-            const uint32_t koff = (ks >> 2) * (kQRows * 128) + (ks & 3) * 32;
-            const uint32_t boff = (ks >> 2) * (kQAtoms * 128) + (ks & 3) * 32;
-            tc_mma(d_tmem, smem_desc(sA + s * C::kABytes + koff), smem_desc(bbase + boff), kQIdesc,
-                   (s > 0 || ks > 0) ? 1u : 0u);
+            const uint32_t aoff = (ks >> 2) * (kQAtoms * 128) + (ks & 3) * 32;
+            const uint32_t boff = (ks >> 2) * (N * 128) + (ks & 3) * 32;
+            tc_mma(d_tmem, smem_desc(abase + aoff), smem_desc(sB + s * C::kBBytes + boff),
+                   C::kIdesc, (s > 0 || ks > 0) ? 1u : 0u);
           }
         issued = true;
         tc_commit(bar_empty(stage));
@@ -238,11 +257,12 @@ __global__ void __launch_bounds__(kQThreads, 1)
         mbar_wait(bar_done, 0u, &dummy, 100000000ull);
       }
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    // warp w reads TMEM lanes 32*(w%4) .. +31: one query row per thread
+    // warp w reads TMEM lanes 32*(w%4) .. +31: one atom per thread, the
+    // tile's query rows along the columns
     const int quarter = warp & 3;
-    const int row = r0 + quarter * 32 + lane;
     uint32_t tbuf = 0, tphase = 0;
     for (int a = blockIdx.x; a < n_atom_tiles; a += gridDim.x) {
       // lane 0 waits (false on timeout or abort), the warp follows its answer
@@ -255,30 +275,23 @@ __global__ void __launch_bounds__(kQThreads, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + tbuf * kQAtoms;
-      uint32_t v[4][32];
+      const int atom = a * kQAtoms + quarter * 32 + lane;
+      const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + tbuf * N;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(taddr + c * 32, v[c]);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_tempty(tbuf));
-      const int a0 = a * kQAtoms;
-      if (row < R) {
-        float* dst = p.qd + (int64_t)row * n + a0;
-        if (a0 + kQAtoms <= n && (n & 3) == 0) {
+      for (int cb = 0; cb < N; cb += 32) {
+        uint32_t v[32];
+        tmem_ld32(taddr + cb, v);
+        tmem_ld_wait();
+        if (cb + 32 >= N) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_tempty(tbuf));
+        }
+        if (atom < n) {
+          float* dst = p.qd + (int64_t)(r0 + cb) * n + atom;
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              reinterpret_cast<uint4*>(dst + c * 32)[u] =
-                  make_uint4(v[c][4 * u], v[c][4 * u + 1], v[c][4 * u + 2], v[c][4 * u + 3]);
-        } else {
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int u = 0; u < 32; ++u)
-              if (a0 + c * 32 + u < n) dst[c * 32 + u] = __uint_as_float(v[c][u]);
+          for (int c = 0; c < 32; ++c)
+            if (r0 + cb + c < R) dst[(int64_t)c * n] = __uint_as_float(v[c]);
         }
       }
       tbuf ^= 1u;
@@ -286,12 +299,25 @@ __global__ void __launch_bounds__(kQThreads, 1)
     }
   }
 
-  __syncthreads();
+  asm volatile("bar.sync 1, %0;" ::"r"(kQThreads - 32) : "memory");
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(C::kTmemCols)
                  : "memory");
   }
+}
+
+template <int D, int N>
+static void qd_launch(const CUtensorMap& map, const DecodeParams& p, dim3 grid,
+                      cudaStream_t stream) {
+  static unsigned long long attr_set = 0ull;
+  if (device_needs_setup(&attr_set)) {
+    cudaFuncSetAttribute(qd_tc_kernel<D, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         QCfg<D, N>::kSmem);
+    device_setup_done(&attr_set);
+  }
+  qd_tc_kernel<D, N><<<grid, kQThreads, QCfg<D, N>::kSmem, stream>>>(map, p);
 }
 
 }  // namespace tc
@@ -313,22 +339,23 @@ sdk_status launch_qd_tc(const DecodeParams& p, cudaStream_t stream, bool* taken)
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return SDK_OK;   // fall back to the CUDA-core kernel
   *taken = true;
-  static unsigned long long attr_set = 0ull;
-  if (device_needs_setup(&attr_set)) {
-    cudaFuncSetAttribute(tc::qd_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         tc::QCfg<128>::kSmem);
-    cudaFuncSetAttribute(tc::qd_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         tc::QCfg<64>::kSmem);
-    device_setup_done(&attr_set);
-  }
+  // rows per tile: the smallest of 32 / 64 / 128 that holds R (128 above)
+  const int N = p.R <= 32 ? 32 : (p.R <= 64 ? 64 : 128);
+  const int ty = (p.R + N - 1) / N;
   const int tiles = (p.n + tc::kQAtoms - 1) / tc::kQAtoms;
-  int gx = num_sms();
+  int gx = num_sms() / ty;
+  if (gx < 1) gx = 1;
   if (gx > tiles) gx = tiles;
-  const dim3 grid((unsigned)gx, (unsigned)((p.R + tc::kQRows - 1) / tc::kQRows));
-  if (p.d == 128)
-    tc::qd_tc_kernel<128><<<grid, tc::kQThreads, tc::QCfg<128>::kSmem, stream>>>(map, p);
-  else
-    tc::qd_tc_kernel<64><<<grid, tc::kQThreads, tc::QCfg<64>::kSmem, stream>>>(map, p);
+  const dim3 grid((unsigned)gx, (unsigned)ty);
+  if (p.d == 128) {
+    if (N == 32) tc::qd_launch<128, 32>(map, p, grid, stream);
+    else if (N == 64) tc::qd_launch<128, 64>(map, p, grid, stream);
+    else tc::qd_launch<128, 128>(map, p, grid, stream);
+  } else {
+    if (N == 32) tc::qd_launch<64, 32>(map, p, grid, stream);
+    else if (N == 64) tc::qd_launch<64, 64>(map, p, grid, stream);
+    else tc::qd_launch<64, 128>(map, p, grid, stream);
+  }
   return cudaGetLastError() == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
 }
 

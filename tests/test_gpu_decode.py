@@ -272,8 +272,8 @@ def test_integer_softmax(full):
 
 
 def test_decode_flags_are_checked():
-    """Flag bits other than the two defined ones are rejected before any
-    launch."""
+    """Flag bits other than the two defined ones, and a query array that is
+    not 16-byte aligned, are rejected before any launch."""
     q, DK, DV, kw, vw, lens = _random_case(17, 1, 2, 1, 64, 64, 1000)
     store = _store(kw, vw)
     lib = sdk.load()
@@ -285,6 +285,13 @@ def test_decode_flags_are_checked():
     rc = lib.sdk_decode_attn(qd.data_ptr(), 1, 2, 1, 64, DKd.data_ptr(), DVd.data_ptr(), 1000,
                              store.k_lo.data_ptr(), store.k_full.data_ptr(),
                              store.v_full.data_ptr(), store.cap, lens_c, 3, 16, 1, 10, 4,
+                             0.125, out.data_ptr(), ws.data_ptr(), ws.numel(), None)
+    assert rc == 1
+    qbuf = torch.zeros(1 + q.numel(), device="cuda")
+    qbuf[1:] = qd.reshape(-1)
+    rc = lib.sdk_decode_attn(qbuf.data_ptr() + 4, 1, 2, 1, 64, DKd.data_ptr(), DVd.data_ptr(),
+                             1000, store.k_lo.data_ptr(), store.k_full.data_ptr(),
+                             store.v_full.data_ptr(), store.cap, lens_c, 3, 16, 1, 10, 0,
                              0.125, out.data_ptr(), ws.data_ptr(), ws.numel(), None)
     assert rc == 1
 
