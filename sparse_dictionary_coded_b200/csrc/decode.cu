@@ -35,24 +35,40 @@
 namespace sdk {
 
 
-// Walk the flattened (head, entry) range [G0, G1).  Heads of sequence b have
-// cnt[b] entries each; off[b] = sum_{b' < b} Hq * cnt[b'].  f(b, h, i0, i1)
-// is called with block-uniform arguments.
+// Work split over the heads of a layer.  A CTA pays a fixed start-up for
+// every head it touches (staging, histogram search, flush, pipeline fill)
+// on top of a cost per token, so the token range is split uniformly over a
+// virtual space in which each head of sequence b spans `a` start-up units
+// and then its cnt[b] tokens: a CTA that crosses into another head takes
+// `a` fewer tokens.  off[b] = sum_{b' < b} Hq * cnt[b'] (real tokens);
+// head (b, h) starts at virtual position off[b] + a*Hq*b + h*(cnt[b] + a).
+__device__ __forceinline__ int64_t virtual_total(const int64_t* off, int B, int Hq, int64_t a) {
+  return off[B] + a * Hq * (int64_t)B;
+}
+
+// Walks this CTA's share [V0, V1) of the virtual space: f(b, h, i0, i1) is
+// called with block-uniform arguments for every head whose tokens
+// [i0, i1) (i1 > i0) fall in the share.
 template <class F>
-__device__ __forceinline__ void for_segments(const int64_t* off, const int* cnt,
-                                             int B, int64_t G0, int64_t G1,
-                                             F f) {
-  int64_t G = G0;
+__device__ __forceinline__ void for_segments(const int64_t* off, const int* cnt, int B, int Hq,
+                                             int64_t a, F f) {
+  const int64_t VT = virtual_total(off, B, Hq, a);
+  const int64_t V0 = VT * blockIdx.x / gridDim.x;
+  const int64_t V1 = VT * (blockIdx.x + 1) / gridDim.x;
+  int64_t V = V0;
   int b = 0;
-  while (G < G1) {
-    while (b + 1 < B && off[b + 1] <= G) ++b;
-    const int64_t local = G - off[b];
-    const int c = cnt[b];
-    const int h = (int)(local / c);
-    const int64_t i = local - (int64_t)h * c;
-    const int64_t take = min(G1 - G, (int64_t)c - i);
-    f(b, h, i, i + take);
-    G += take;
+  while (V < V1) {
+    while (b + 1 < B && off[b + 1] + a * Hq * (int64_t)(b + 1) <= V) ++b;
+    const int64_t vb = off[b] + a * Hq * (int64_t)b;
+    const int64_t hl = (int64_t)cnt[b] + a;           // virtual length of one head
+    const int64_t local = V - vb;
+    const int h = (int)(local / hl);
+    const int64_t hs = vb + (int64_t)h * hl;          // virtual start of head h
+    const int64_t e = min(V1, hs + hl);
+    const int64_t i0 = max(V - hs - a, (int64_t)0);
+    const int64_t i1 = e - hs - a;
+    if (i1 > i0) f(b, h, i0, i1);
+    V = e;
   }
 }
 
@@ -254,6 +270,13 @@ __global__ void __launch_bounds__(64 * kGvTiles * RB, (RB > 1 ? 2 : 1)) qd_kerne
 // key bits 31..20 of every head (shared-memory atomics, flushed once per
 // segment).
 constexpr int kScanThreads = 512;
+// Start-up cost of one head segment in token units, from per-CTA timings at
+// 256K tokens (CTAs that touched two heads against those that touched one):
+// the Klow scan pays about 4 us of table staging, flush and pipeline fill
+// per segment (about 11K tokens of scan), pass 2 about 5 us (histogram
+// search, flush, pipeline fill: about 28K tokens).
+constexpr int64_t kKlowSegCost = 11000;
+constexpr int64_t kPass2SegCost = 28000;
 constexpr int kKlowThreads = 1024;
 
 // QD row -> table[0..kTable), zero past n.  Eight 16-byte loads per thread
@@ -291,13 +314,10 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
   float* table = reinterpret_cast<float*>(smem4);
   uint32_t* sh = reinterpret_cast<uint32_t*>(table + kTable);
   const int n = p.n, tid = threadIdx.x;
-  const int64_t total = p.tok_off[p.B];
-  const int64_t G0 = total * blockIdx.x / gridDim.x;
-  const int64_t G1 = total * (blockIdx.x + 1) / gridDim.x;
   const int nlo = min(p.klow, kLoPlanes);
   uint32_t maxidx = 0u;
 
-  for_segments(p.tok_off, p.lens, p.B, G0, G1, [&](int b, int h, int64_t t0l, int64_t t1l) {
+  for_segments(p.tok_off, p.lens, p.B, p.Hq, kKlowSegCost, [&](int b, int h, int64_t t0l, int64_t t1l) {
     const int r = b * p.Hq + h, kvh = h / p.g;
     const int t0 = (int)t0l, t1 = (int)t1l;    // token indices fit 31 bits
     stage_table(table, p.qd + (int64_t)r * n, n);
@@ -766,12 +786,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) pass2_kernel(DecodeParams p) 
   uint32_t* s_ck = reinterpret_cast<uint32_t*>(s_ct + kCandBuf);
   uint32_t* s_h2 = s_ck + kCandBuf;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t total = p.tok_off[p.B];
-  const int64_t G0 = total * blockIdx.x / gridDim.x;
-  const int64_t G1 = total * (blockIdx.x + 1) / gridDim.x;
   constexpr int kWarps = kScanThreads / 32;
 
-  for_segments(p.tok_off, p.lens, p.B, G0, G1, [&](int b, int h, int64_t t0l, int64_t t1l) {
+  for_segments(p.tok_off, p.lens, p.B, p.Hq, kPass2SegCost, [&](int b, int h, int64_t t0l, int64_t t1l) {
     const int r = b * p.Hq + h;
     const int Nb = p.lens[b];
     const int t0 = (int)t0l, t1 = (int)t1l;
@@ -1621,6 +1638,20 @@ static int grid_for(int64_t work, int64_t per_cta, int cap_ctas) {
   return (int)g;
 }
 
+// CTAs for a segment scan (klow, pass 2) over `total` tokens of R heads with
+// a start-up cost of `a` tokens per head touched: up to g CTAs splitting the
+// virtual space, or the largest multiple of R below g, whose boundaries fall
+// on head starts when the heads are equally long (no CTA pays a second
+// start-up), whichever gives the smaller cost per CTA.
+static int scan_grid(int64_t total, int64_t R, int64_t a, int64_t per_cta, int sms) {
+  const int g = grid_for(total, per_cta, sms);
+  if (R > g) return g;
+  const int64_t ga = R * (g / R);
+  const double c_split = (double)(total + a * (g + R)) / g;
+  const double c_aligned = (double)total / ga + (double)a;
+  return c_aligned <= c_split ? (int)ga : g;
+}
+
 // Optional launch with programmatic stream serialization (the kernel may
 // start while the previous one drains; every decode kernel waits for it
 // before touching memory).  Off by default: measured on B200 it made the
@@ -1738,7 +1769,7 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
     if (e != cudaSuccess) return SDK_ERR_CUDA;
   }
   {
-    const int g = grid_for(p.tok_off[p.B], 2048, sms);
+    const int g = scan_grid(p.tok_off[p.B], p.R, kKlowSegCost, 2048, sms);
     const int vec = (p.cap % 4 == 0) && ((reinterpret_cast<uintptr_t>(p.k_lo) & 15u) == 0u);
     e = launch_pdl(klow_kernel, dim3(g), dim3(kKlowThreads), (size_t)kTable * 4 + 4096 * 4, stream,
                    1, p, vec);
@@ -1747,7 +1778,7 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
   return SDK_OK;
   }
   case 1: {   // pass 2 of the selection
-    const int g = grid_for(p.tok_off[p.B], 8192, sms);
+    const int g = scan_grid(p.tok_off[p.B], p.R, kPass2SegCost, 8192, sms);
     e = launch_pdl(pass2_kernel, dim3(g), dim3(kScanThreads), (size_t)kPass2Smem, stream, 1, p);
     return e == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
   }
