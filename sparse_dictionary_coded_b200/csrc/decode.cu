@@ -475,36 +475,29 @@ __device__ void final_head(const DecodeParams& p, int r, uint32_t* s_cand, uint3
   const int32_t* ct = p.cand_t + (int64_t)r * p.L;
   int32_t* list = p.list + (int64_t)r * p.L;
   const uint32_t k1 = k - n_above;
-  // candidates in shared memory when they fit (one coalesced pass over the
-  // global copy; the passes below then read shared memory).  Otherwise the
-  // passes read global memory that no CTA of this SM has loaded before.
-  if (n_cand <= (uint32_t)kFinalStage) {
-    // eight loads of each array in flight per thread before any store
-    for (uint32_t i0 = tid; i0 < n_cand; i0 += 8 * kScanThreads) {
-      uint32_t kv[8], tv[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const uint32_t i = i0 + u * kScanThreads;
-        kv[u] = i < n_cand ? __ldcg(ck + i) : 0u;
-        tv[u] = i < n_cand ? (uint32_t)__ldcg(ct + i) : 0u;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const uint32_t i = i0 + u * kScanThreads;
-        if (i < n_cand) {
-          s_cand[i] = kv[u];
-          s_cand[kFinalStage + i] = tv[u];
-        }
-      }
+  // candidates in shared memory when they fit: asynchronous 16-byte copies
+  // (rows are 16-byte aligned; the last copy of each array reads only the
+  // remaining words) that land while the second digit is searched in hist2.
+  // Otherwise the passes read global memory.
+  const bool staged = n_cand <= (uint32_t)kFinalStage;
+  if (staged) {
+    for (uint32_t i4 = tid; 4 * i4 < n_cand; i4 += kScanThreads) {
+      const unsigned bytes = 4u * min(4u, n_cand - 4 * i4);
+      cp_async16_n(s_cand + 4 * i4, ck + 4 * i4, bytes);
+      cp_async16_n(s_cand + kFinalStage + 4 * i4, ct + 4 * i4, bytes);
     }
-    __syncthreads();
-    ck = s_cand;
-    ct = reinterpret_cast<const int32_t*>(s_cand + kFinalStage);
+    cp_async_commit();
   }
 
   uint32_t b2, above2, cnt2, b3, above3, cnt3;
   bool bad;
   block_find_desc<4096, true>(p.hist2 + (int64_t)r * 4096, k1, s_tmp, b2, above2, cnt2, bad);
+  if (staged) {
+    cp_async_wait<0>();
+    __syncthreads();
+    ck = s_cand;
+    ct = reinterpret_cast<const int32_t*>(s_cand + kFinalStage);
+  }
   if (bad) {
     if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x21000000u | r);
     return;
@@ -543,34 +536,52 @@ __device__ void final_head(const DecodeParams& p, int r, uint32_t* s_cand, uint3
     s_cnt[1] = __ldcg(&st->n_comp);
   }
   __syncthreads();
+  // a warp takes 4 x 32 candidates per round: one slot atomic per kind
   uint32_t cmax = 0u;
-  for (uint32_t i0 = (uint32_t)warp * 32; i0 < n_cand; i0 += kScanThreads) {
-    const uint32_t i = i0 + lane;
-    uint32_t key = 0u, t = 0u;
-    bool sel = false, comp = false;
-    if (i < n_cand) {
-      key = ck[i];
-      t = (uint32_t)ct[i];
-      sel = key > T || (key == T && t <= t_cut);
-      comp = !sel && p.full;
+  constexpr int kU = 4;
+  for (uint32_t i0 = (uint32_t)warp * 32 * kU; i0 < n_cand; i0 += kScanThreads * kU) {
+    uint32_t key[kU], t[kU];
+    unsigned msel[kU], mcomp[kU];
+    uint32_t ns = 0u, nc = 0u;
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const uint32_t i = i0 + 32 * u + lane;
+      key[u] = 0u;
+      t[u] = 0u;
+      bool sel = false, comp = false;
+      if (i < n_cand) {
+        key[u] = ck[i];
+        t[u] = (uint32_t)ct[i];
+        sel = key[u] > T || (key[u] == T && t[u] <= t_cut);
+        comp = !sel && p.full;
+      }
+      msel[u] = __ballot_sync(0xffffffffu, sel);
+      mcomp[u] = __ballot_sync(0xffffffffu, comp);
+      ns += (uint32_t)__popc(msel[u]);
+      nc += (uint32_t)__popc(mcomp[u]);
     }
-    const unsigned msel = __ballot_sync(0xffffffffu, sel);
-    const unsigned mcomp = __ballot_sync(0xffffffffu, comp);
     uint32_t bs = 0, bo = 0;
     if (lane == 0) {
-      if (msel) bs = atomicAdd(&s_cnt[0], (uint32_t)__popc(msel));
-      if (mcomp) bo = atomicAdd(&s_cnt[1], (uint32_t)__popc(mcomp));
+      if (ns) bs = atomicAdd(&s_cnt[0], ns);
+      if (nc) bo = atomicAdd(&s_cnt[1], nc);
     }
-    bs = __shfl_sync(0xffffffffu, bs, 0) + __popc(msel & lt);
-    bo = __shfl_sync(0xffffffffu, bo, 0) + __popc(mcomp & lt);
-    if (sel) {
-      if (bs < k) list[bs] = (int32_t)t;
-      else record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x26000000u | r);
-    }
-    if (comp) {
-      if (bo < (uint32_t)Nb) list[Nb - 1 - (int64_t)bo] = (int32_t)t;
-      else record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x27000000u | r);
-      cmax = max(cmax, key);
+    bs = __shfl_sync(0xffffffffu, bs, 0);
+    bo = __shfl_sync(0xffffffffu, bo, 0);
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      if (msel[u] & (1u << lane)) {
+        const uint32_t pos = bs + (uint32_t)__popc(msel[u] & lt);
+        if (pos < k) list[pos] = (int32_t)t[u];
+        else record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x26000000u | r);
+      }
+      if (mcomp[u] & (1u << lane)) {
+        const uint32_t pos = bo + (uint32_t)__popc(mcomp[u] & lt);
+        if (pos < (uint32_t)Nb) list[Nb - 1 - (int64_t)pos] = (int32_t)t[u];
+        else record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x27000000u | r);
+        cmax = max(cmax, key[u]);
+      }
+      bs += (uint32_t)__popc(msel[u]);
+      bo += (uint32_t)__popc(mcomp[u]);
     }
   }
   if (p.full) {

@@ -123,6 +123,13 @@ __device__ __forceinline__ void cp_async16_64B(void* smem_dst, const void* gsrc,
                "r"(valid ? 16 : 0)
                : "memory");
 }
+// 16-byte copy of which only the first `bytes` (0..16) are read; the rest
+// of the 16 destination bytes is zero-filled.
+__device__ __forceinline__ void cp_async16_n(void* smem_dst, const void* gsrc, unsigned bytes) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(smem_dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gsrc), "r"(bytes)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
