@@ -763,17 +763,19 @@ __global__ void __launch_bounds__(kScanThreads) shard_select_kernel(DecodeParams
 // become candidates (with a histogram of key bits 19..8), the others go to
 // the complement (full-softmax flag only).  A warp takes 512 tokens per
 // step: each lane takes 16 consecutive keys (four 16-byte copies streamed
-// through a per-lane shared-memory ring three steps ahead, about 6 KB per
-// warp in flight), counts its tokens of each kind, and a warp scan gives
-// every lane its output slots behind one atomic per warp and kind.  Candidates and their
-// histogram go through shared memory (flushed once per segment; slots past
-// the buffer go straight to global memory).  The few tokens before the
-// first 16-byte boundary of a segment and after its last one take a scalar
-// path.
+// through a per-lane shared-memory ring one step ahead), counts its tokens
+// of each kind, and a warp scan gives every lane its output slots behind
+// one atomic per warp and kind.  The steps are chains of dependent warp
+// operations, so the CTA runs 32 warps with a short ring (measured faster
+// than 16 or 24 warps with deeper rings).  Candidates and their histogram
+// go through shared memory (flushed once per segment; slots past the
+// buffer go straight to global memory).  The few tokens before the first
+// 16-byte boundary of a segment and after its last one take a scalar path.
 constexpr int kCandBuf = 2048;
-constexpr int kP2Stages = 4;                            // key ring depth per lane
+constexpr int kP2Threads = 1024;
+constexpr int kP2Stages = 2;                            // key ring depth per lane
 constexpr int kP2RingOff = 2 * kCandBuf + 4096;         // in words
-constexpr int kPass2Smem = (kP2RingOff + kP2Stages * (kScanThreads / 32) * 128 * 4) * 4;
+constexpr int kPass2Smem = (kP2RingOff + kP2Stages * (kP2Threads / 32) * 128 * 4) * 4;
 
 __device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v, uint32_t& total) {
   const int lane = threadIdx.x & 31;
@@ -787,7 +789,7 @@ __device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v, uint32_t& total) 
   return x - v;
 }
 
-__global__ void __launch_bounds__(kScanThreads, 1) pass2_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kP2Threads, 1) pass2_kernel(DecodeParams p) {
   pdl_wait();     // nothing global is touched before the previous kernel is done
   pdl_launch();
   __shared__ uint32_t s_tmp[48];
@@ -797,7 +799,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) pass2_kernel(DecodeParams p) 
   uint32_t* s_ck = reinterpret_cast<uint32_t*>(s_ct + kCandBuf);
   uint32_t* s_h2 = s_ck + kCandBuf;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int kWarps = kScanThreads / 32;
+  constexpr int kWarps = kP2Threads / 32;
 
   for_segments(p.tok_off, p.lens, p.B, p.Hq, kPass2SegCost, [&](int b, int h, int64_t t0l, int64_t t1l) {
     const int r = b * p.Hq + h;
@@ -806,7 +808,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) pass2_kernel(DecodeParams p) 
     sdk_select_state* st = p.st + r;
     uint32_t b1, above1, cnt1;
     bool bad;
-    for (int i = tid; i < 4096; i += kScanThreads) s_h2[i] = 0u;
+    for (int i = tid; i < 4096; i += kP2Threads) s_h2[i] = 0u;
     if (tid == 0) s_ncand = 0u;
     block_find_desc<4096>(p.hist1 + (int64_t)r * 4096, (uint32_t)p.kcnt[b], s_tmp, b1, above1,
                           cnt1, bad);   // ends with a barrier
@@ -1020,13 +1022,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) pass2_kernel(DecodeParams p) 
     }
     __syncthreads();
     const uint32_t ncand = s_ncand, cbase = s_cbase;
-    for (uint32_t i = tid; i < ncand; i += kScanThreads)
+    for (uint32_t i = tid; i < ncand; i += kP2Threads)
       if (cbase + i < (uint32_t)Nb) {
         ct[cbase + i] = s_ct[i];
         ck[cbase + i] = s_ck[i];
       }
     uint32_t* h2 = p.hist2 + (int64_t)r * 4096;
-    for (int i = tid; i < 4096; i += kScanThreads)
+    for (int i = tid; i < 4096; i += kP2Threads)
       if (s_h2[i]) atomicAdd(&h2[i], s_h2[i]);
     if (full) {
       cmax = warp_umax(cmax);
@@ -1790,7 +1792,7 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
   }
   case 1: {   // pass 2 of the selection
     const int g = scan_grid(p.tok_off[p.B], p.R, kPass2SegCost, 8192, sms);
-    e = launch_pdl(pass2_kernel, dim3(g), dim3(kScanThreads), (size_t)kPass2Smem, stream, 1, p);
+    e = launch_pdl(pass2_kernel, dim3(g), dim3(kP2Threads), (size_t)kPass2Smem, stream, 1, p);
     return e == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
   }
   case 2:     // the final selection (whole context)
