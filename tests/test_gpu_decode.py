@@ -180,6 +180,19 @@ def test_ragged_batch_small_and_odd_sizes():
         _compare(q, DK, DV, kw, vw, lens, full=full)
 
 
+@pytest.mark.parametrize("full", [False, True])
+def test_ragged_batch_many_ctas(full):
+    """B=4 with lengths 9000, 40000, 2500 and 23000 (GQA 8/2, d=128, 4096
+    atoms): the Klow scan and pass 2 split these unequal heads over many
+    CTAs (the work split charges every head a start-up cost, so CTA bounds
+    fall at arbitrary tokens of heads of different lengths).  Every head's
+    keys, set and output are checked, so a token range that no CTA scanned,
+    or that two did, fails."""
+    q, DK, DV, kw, vw, _ = _random_case(91, 4, 8, 2, 40000, 128, 4096)
+    lens = [9000, 40000, 2500, 23000]
+    _compare(q, DK, DV, kw, vw, lens, full=full)
+
+
 def test_dense_special_case_matches_sdpa():
     """Klow=Khigh=16, top 100%: dense attention over the decoded keys and
     values, checked against torch SDPA in fp64 on the CPU."""
