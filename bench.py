@@ -45,6 +45,9 @@ def enc_flop_per_vector(n_atoms, head_dim):
 ENC_KERNELS_PER_CALL = 3
 # kernels of one decode layer: qd, klow, pass2, final, attend, out
 DEC_KERNELS_PER_LAYER = 6
+# DRAM bytes (read + write) of one attend_kernel launch from an ncu capture
+# of the current kernel (one 256K-token layer, cold L2): 141.48 + 5.64 MB
+ATTEND_TRAFFIC = {"decode256k": 147.12e6}
 ENC_DTYPE = ("f32 (residuals and re-scoring; tensor-core operands fp16 with "
              "fp32 accumulation; bf16 dictionaries; fp16 coefficients)")
 
@@ -510,6 +513,24 @@ def bench_decode(args, world, rank, pk, name):
                "ms_per_step": t,
                "h2d_bytes_per_step": sum(h.numel() * 4 for h in hq),
                "d2h_bytes_per_step": hout.numel() * 4}
+    # the dominant kernel (attend_kernel: Khigh rescore, softmax, value
+    # scatter), timed live: a second capture of the step in which the
+    # library brackets every attention launch with CUDA events on the
+    # launching stream (sdk_timing_enable), replayed with the L2 flushed
+    # before each replay; the headline step time above has no events in it
+    sdk.sdk_timing_enable(True)
+    gt = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gt):
+        step()
+    sdk.sdk_timing_enable(False)
+    att = []
+    for _ in range(max(3, args.steps // 2)):
+        flush()
+        gt.replay()
+        torch.cuda.synchronize()
+        att += sdk.sdk_timing_read(L)
+    del gt
+    att_ms = max_over_ranks(statistics.mean(att), world)
     for ly in layers:
         rc, _ = sdk.sdk_check_status(ly["ws"])
         assert rc == 0, "device check failed in decode"
@@ -520,16 +541,32 @@ def bench_decode(args, world, rank, pk, name):
                                 Hkv, N, k, args.full_softmax)
     alg = code_bytes + L * 2 * n * d * 2
     gbs = alg / (step_ms * 1e-3) / 1e9
+    # attend's algorithmic bytes per launch: the code bytes of the layer
+    # without the Klow scan's 12 B per token per KV head
+    att_alg = (code_bytes - L * 12 * N * B * Hkv) / L
+    att_gbs = att_alg / (att_ms * 1e-3) / 1e9
+    traffic = ATTEND_TRAFFIC.get(name) if not (args.full_softmax or args.int_softmax) else None
     return {
         "value": world * B * N / (step_ms * 1e-3),
         "unit": "ctx tokens/s/step (%d layers)" % L,
         "ms_per_step": step_ms,
         "ms_per_step_no_graph": statistics.mean(ms_nog),
-        "roofline": {"bound": "hbm", "kernel": "decode step (all kernels, "
-                     "%d layers)" % L, "achieved": gbs, "peak": pk["hbm"],
-                     "unit": "GB/s", "frac": gbs / pk["hbm"],
-                     "traffic": None, "alg_bytes_per_step": alg,
-                     "union_tokens_per_step": U},
+        "roofline": {"bound": "hbm",
+                     "kernel": "attend_kernel (Khigh rescore, softmax and "
+                               "value scatter; the step's largest kernel)",
+                     "achieved": att_gbs, "peak": pk["hbm"], "unit": "GB/s",
+                     "frac": att_gbs / pk["hbm"],
+                     "traffic": traffic,
+                     "traffic_source": ("dram__bytes_read.sum + dram__bytes_write.sum "
+                                        "of one launch, ncu --set full, cold L2"
+                                        if traffic else None),
+                     "alg_bytes_per_launch": att_alg,
+                     "ms_per_launch": att_ms, "launches_timed": len(att),
+                     "step": {"kernels": "all %d per layer, %d layers"
+                                         % (DEC_KERNELS_PER_LAYER, L),
+                              "achieved": gbs, "frac": gbs / pk["hbm"],
+                              "alg_bytes_per_step": alg,
+                              "union_tokens_per_step": U}},
         "clocks": ck,
         "config": {"workload": name, "layers": L, "B": B, "Hq": Hq,
                    "Hkv": Hkv, "head_dim": d, "n_atoms": n, "n_tokens": N,

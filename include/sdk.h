@@ -365,6 +365,25 @@ SDK_API sdk_status sdk_workspace_init(void* workspace, size_t ws_bytes,
 SDK_API sdk_status sdk_check_status(void* workspace, sdk_stream_t stream,
                             uint32_t* counters_out);
 
+/* Kernel timing, for measurement.  While enabled (a process-wide switch),
+ * every launch of the decode attention kernel (the Khigh rescore, softmax
+ * and value scatter: one per sdk_decode_attn call, one in each of stages 5
+ * and 6 of sdk_decode_attn_shard) is bracketed by a pair of CUDA events
+ * recorded on the call's stream; the pairs are the current device's slots
+ * 0, 1, 2, ... of SDK_TIMING_SLOTS, reused round-robin.  Calls captured in
+ * a CUDA graph keep their slots, and every replay records them again.
+ * sdk_timing_enable(on): sets the switch; turning it on (outside any stream
+ * capture: it creates the current device's events the first time) restarts
+ * at slot 0.
+ * sdk_timing_read: waits for the events of slots 0 .. n-1, n = min(max_n,
+ * slots used since the last enable, SDK_TIMING_SLOTS), writes their
+ * durations in milliseconds to ms_out (host, >= max_n floats) and returns
+ * n; -1 on a CUDA error (SDK_ERR_CUDA semantics).
+ */
+#define SDK_TIMING_SLOTS 256
+SDK_API sdk_status sdk_timing_enable(int32_t on);
+SDK_API int32_t sdk_timing_read(float* ms_out, int32_t max_n);
+
 #ifdef __cplusplus
 }
 #endif

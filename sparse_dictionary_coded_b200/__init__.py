@@ -25,7 +25,8 @@ __all__ = [
     "sdk_decode_attn", "sdk_encode_workspace_bytes",
     "sdk_append_workspace_bytes", "sdk_decode_workspace_bytes",
     "sdk_decode_layout_of", "sdk_workspace_init", "sdk_check_status",
-    "new_workspace", "CodeStore", "read_select_state",
+    "new_workspace", "CodeStore", "read_select_state", "sdk_timing_enable",
+    "sdk_timing_read",
 ]
 
 
@@ -86,6 +87,22 @@ def sdk_check_status(ws, stream=None):
     buf = (ctypes.c_uint32 * 4)()
     rc = load().sdk_check_status(_ptr(ws), _stream(stream), buf)
     return rc, list(buf)
+
+
+def sdk_timing_enable(on):
+    """Brackets every decode attention-kernel launch with CUDA events
+    (include/sdk.h, sdk_timing_enable); turning it on restarts at slot 0."""
+    _check(load().sdk_timing_enable(1 if on else 0), "sdk_timing_enable")
+
+
+def sdk_timing_read(max_n=_capi.SDK_TIMING_SLOTS):
+    """Durations (ms) of the attention-kernel launches recorded in slots
+    0 .. n-1 since the last enable (waits for them)."""
+    buf = (ctypes.c_float * max(1, max_n))()
+    n = load().sdk_timing_read(buf, max_n)
+    if n < 0:
+        raise SdkError(4, "sdk_timing_read")      # SDK_ERR_CUDA
+    return [float(buf[i]) for i in range(n)]
 
 
 def sdk_encode_workspace_bytes(n_vec, head_dim, n_atoms):

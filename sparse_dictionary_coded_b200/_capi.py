@@ -24,6 +24,8 @@ DECODE_STATIC_WS_BYTES = 16 << 20
 # every symbol include/sdk.h declares, with (restype, argtypes)
 _vp, _i32, _i64, _sz, _f32 = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64,
                               ctypes.c_size_t, ctypes.c_float)
+SDK_TIMING_SLOTS = 256
+
 SIGNATURES = {
     "sdk_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "sdk_version": (_i32, []),
@@ -55,6 +57,8 @@ SIGNATURES = {
                                             _vp]),
     "sdk_workspace_init": (ctypes.c_int, [_vp, _sz, _vp]),
     "sdk_check_status": (ctypes.c_int, [_vp, _vp, _vp]),
+    "sdk_timing_enable": (ctypes.c_int, [_i32]),
+    "sdk_timing_read": (_i32, [_vp, _i32]),
 }
 
 

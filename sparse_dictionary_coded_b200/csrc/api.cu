@@ -449,6 +449,10 @@ sdk_status sdk_decode_attn_shard(int32_t stage, int32_t rank, int32_t world, con
   return launch_decode(p, reinterpret_cast<cudaStream_t>(stream), stage, rank);
 }
 
+sdk_status sdk_timing_enable(int32_t on) { return timing_enable(on != 0); }
+
+int32_t sdk_timing_read(float* ms_out, int32_t max_n) { return timing_read(ms_out, max_n); }
+
 sdk_status sdk_workspace_init(void* workspace, size_t ws_bytes, sdk_stream_t stream) {
   if (workspace == nullptr || !aligned(workspace, SDK_WS_ALIGN) || ws_bytes < sizeof(WsHeader))
     return SDK_ERR_INVALID_ARG;

@@ -28,6 +28,8 @@
 //                    `out`, zeroed by qd_kernel).
 #include <cooperative_groups.h>
 #include <stdlib.h>
+#include <atomic>
+#include <mutex>
 #include <type_traits>
 
 #include "sdk_internal.cuh"
@@ -1726,6 +1728,84 @@ static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+// ---- attention-kernel timing (sdk_timing_enable / sdk_timing_read) -------
+namespace {
+constexpr int kTimingDevices = 64;
+std::atomic<bool> g_timing_on{false};
+std::mutex g_timing_mu;
+struct TimingPool {
+  cudaEvent_t ev[SDK_TIMING_SLOTS][2];
+  bool made = false;
+  int used = 0;
+};
+TimingPool g_timing[kTimingDevices];
+
+// The event pair of the next slot of the current device (nulls when timing
+// is off, or was not turned on for this device).
+void timing_slot(cudaEvent_t* e0, cudaEvent_t* e1) {
+  *e0 = *e1 = nullptr;
+  if (!g_timing_on.load(std::memory_order_acquire)) return;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kTimingDevices) return;
+  std::lock_guard<std::mutex> lock(g_timing_mu);
+  TimingPool& tp = g_timing[dev];
+  if (!tp.made) return;   // enabled on another device
+  const int i = tp.used % SDK_TIMING_SLOTS;
+  ++tp.used;
+  *e0 = tp.ev[i][0];
+  *e1 = tp.ev[i][1];
+}
+// Records e on stream; inside a stream capture as an external record (an
+// event-record node of the graph, executed by every replay), which a plain
+// record there is not.
+cudaError_t timing_record(cudaEvent_t e, cudaStream_t stream) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return cudaErrorUnknown;
+  return cs == cudaStreamCaptureStatusActive
+             ? cudaEventRecordWithFlags(e, stream, cudaEventRecordExternal)
+             : cudaEventRecord(e, stream);
+}
+}  // namespace
+
+// The current device's events are made here, outside any stream capture.
+sdk_status timing_enable(bool on) {
+  std::lock_guard<std::mutex> lock(g_timing_mu);
+  if (on) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kTimingDevices)
+      return SDK_ERR_CUDA;
+    TimingPool& tp = g_timing[dev];
+    if (!tp.made) {
+      for (int i = 0; i < SDK_TIMING_SLOTS; ++i)
+        for (int j = 0; j < 2; ++j)
+          if (cudaEventCreate(&tp.ev[i][j]) != cudaSuccess) return SDK_ERR_CUDA;
+      tp.made = true;
+    }
+    tp.used = 0;
+  }
+  g_timing_on.store(on, std::memory_order_release);
+  return SDK_OK;
+}
+
+int timing_read(float* ms_out, int max_n) {
+  if (ms_out == nullptr || max_n < 0) return -1;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kTimingDevices) return -1;
+  std::lock_guard<std::mutex> lock(g_timing_mu);
+  TimingPool& tp = g_timing[dev];
+  if (!tp.made) return 0;
+  int n = tp.used < SDK_TIMING_SLOTS ? tp.used : SDK_TIMING_SLOTS;
+  if (n > max_n) n = max_n;
+  for (int i = 0; i < n; ++i) {
+    if (cudaEventSynchronize(tp.ev[i][1]) != cudaSuccess ||
+        cudaEventElapsedTime(&ms_out[i], tp.ev[i][0], tp.ev[i][1]) != cudaSuccess) {
+      cudaGetLastError();   // not sticky: leave no error for the next call
+      return -1;
+    }
+  }
+  return n;
+}
+
 sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, int rank_id) {
   const int sms = num_sms();
   static unsigned long long attr_set = 0ull;
@@ -1801,6 +1881,9 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
     return e == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
   case 3: {   // attend
   {
+    cudaEvent_t t0 = nullptr, t1 = nullptr;
+    timing_slot(&t0, &t1);
+    if (t0 != nullptr && timing_record(t0, stream) != cudaSuccess) return SDK_ERR_CUDA;
     // one cluster of C CTAs per query head, C a power of two <= 8 while the
     // clusters fit the SMs and every CTA keeps >= 1024 entries
     int64_t dmax = 0;
@@ -1813,6 +1896,7 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
     e = launch_pdl(kern, dim3((unsigned)(p.R * C)), dim3(kAttThreads), (size_t)kAttSmem, stream,
                    (unsigned)C, p, C);
     if (e != cudaSuccess) return SDK_ERR_CUDA;
+    if (t1 != nullptr && timing_record(t1, stream) != cudaSuccess) return SDK_ERR_CUDA;
   }
   return SDK_OK;
   }

@@ -309,6 +309,48 @@ def test_decode_flags_are_checked():
     assert rc == 1
 
 
+def test_attention_kernel_timing():
+    """sdk_timing_enable brackets every attention-kernel launch with CUDA
+    events: two decode calls give two positive durations; once disabled,
+    further calls record nothing; enabling again restarts at slot 0; two
+    calls captured in a CUDA graph give two durations at every replay."""
+    q, DK, DV, kw, vw, lens = _random_case(19, 1, 8, 2, 2000, 128, 4096)
+    store = _store(kw, vw)
+    sdk.sdk_timing_enable(True)
+    try:
+        for _ in range(2):
+            _run(q, DK, DV, store)
+        ms = sdk.sdk_timing_read(8)
+        assert len(ms) == 2 and all(0.0 < t < 1000.0 for t in ms), ms
+        sdk.sdk_timing_enable(False)
+        _run(q, DK, DV, store)
+        assert len(sdk.sdk_timing_read(8)) == 2
+        sdk.sdk_timing_enable(True)
+        assert sdk.sdk_timing_read(8) == []
+        # calls captured in a CUDA graph keep their slots; every replay
+        # records them again
+        B, Hq, d = q.shape
+        ws = sdk.new_workspace(sdk.sdk_decode_workspace_bytes(B, Hq, d, DK.shape[0], 2000))
+        qd, DKd, DVd = q.cuda(), DK.cuda(), DV.cuda()
+        out = torch.empty(B, Hq, d, device="cuda")
+        sdk.sdk_decode_attn(qd, DKd, DVd, store, out=out, workspace=ws)
+        torch.cuda.synchronize()
+        sdk.sdk_timing_enable(True)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            sdk.sdk_decode_attn(qd, DKd, DVd, store, out=out, workspace=ws)
+            sdk.sdk_decode_attn(qd, DKd, DVd, store, out=out, workspace=ws)
+        sdk.sdk_timing_enable(False)
+        for _ in range(2):
+            g.replay()
+            torch.cuda.synchronize()
+            ms = sdk.sdk_timing_read(8)
+            assert len(ms) == 2 and all(0.0 < t < 1000.0 for t in ms), ms
+        assert sdk.sdk_check_status(ws)[0] == 0
+    finally:
+        sdk.sdk_timing_enable(False)
+
+
 def test_bad_atom_index_is_reported_not_trapped():
     """Codes naming atom 1500 of a 1000-atom dictionary: the kernels skip
     the term and record SDK_ERR_DEVICE_CHECK with the index."""
