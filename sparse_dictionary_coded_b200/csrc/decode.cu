@@ -4,8 +4,9 @@
 // 15x compression: only 3 atoms score most tokens).
 //
 // One layer, B sequences, R = B*Hq query heads.  Kernels, in stream order:
-//   qd_kernel        QD[r][a] = <q_r, D_K[a]> (fp32 CUDA cores), and zeroes
-//                    the per-head selection state, histograms and w.
+//   qd_tc_kernel     (qd_tc.cu) QD[r][a] = <q_r, D_K[a]> on the tensor cores,
+//                    and zeroes the per-head selection state, histograms
+//                    and `out`; qd_kernel here is the fp32 CUDA-core form.
 //   klow_kernel      s_lo for every token from the 3 k_lo planes (12 B per
 //                    token, coalesced) and QD staged in shared memory;
 //                    writes order-preserving keys and the 12-bit radix
@@ -23,9 +24,11 @@
 //                    shared-memory per-atom weight tile (fixed-point
 //                    atomics); one cluster of CTAs per head shares the
 //                    softmax statistics and sums its tiles through
-//                    distributed shared memory.
-//   out_kernel       out += w D_V over atom tiles (vector reductions into
-//                    `out`, zeroed by qd_kernel).
+//                    distributed shared memory into w (three bf16 parts).
+//   out_tc_kernel    (out_tc.cu) out += w D_V on the tensor cores; out_kernel
+//                    here is the fp32 CUDA-core form.
+// The Klow scan and pass 2 split the layer's tokens over their CTAs with a
+// start-up cost charged per head (for_segments).
 #include <cooperative_groups.h>
 #include <stdlib.h>
 #include <atomic>
