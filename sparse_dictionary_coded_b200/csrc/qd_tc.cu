@@ -140,10 +140,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const int t = tid - 32;
     const int64_t nthr = (int64_t)gridDim.x * gridDim.y * kT;
     const int64_t g0 = ((int64_t)blockIdx.y * gridDim.x + blockIdx.x) * kT + t;
-    const int64_t hwords = (int64_t)R * 4096;
-    for (int64_t e = g0; e < hwords; e += nthr) {
-      p.hist1[e] = 0u;
-      p.hist2[e] = 0u;
+    const int64_t hquads = (int64_t)R * 1024;   // both histograms, 16-byte stores
+    for (int64_t e = g0; e < hquads; e += nthr) {
+      reinterpret_cast<uint4*>(p.hist1)[e] = make_uint4(0u, 0u, 0u, 0u);
+      reinterpret_cast<uint4*>(p.hist2)[e] = make_uint4(0u, 0u, 0u, 0u);
     }
     for (int64_t e = g0; e < (int64_t)R * D; e += nthr) p.out[e] = 0.0f;
     for (int64_t e = g0; e < (int64_t)R; e += nthr) {
