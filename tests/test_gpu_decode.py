@@ -193,6 +193,16 @@ def test_ragged_batch_many_ctas(full):
     _compare(q, DK, DV, kw, vw, lens, full=full)
 
 
+@pytest.mark.parametrize("full", [False, True])
+def test_atom_count_not_a_multiple_of_eight(full):
+    """1001 atoms (not a multiple of 4 or 8): the dictionary tensor maps
+    read past n as zero, the weight parts of the last atoms take the scalar
+    stores, and w D_V runs on the CUDA-core kernel (the tensor-core one needs
+    16-byte rows of w)."""
+    q, DK, DV, kw, vw, lens = _random_case(93, 2, 8, 2, 900, 128, 1001)
+    _compare(q, DK, DV, kw, vw, lens, full=full)
+
+
 def test_dense_special_case_matches_sdpa():
     """Klow=Khigh=16, top 100%: dense attention over the decoded keys and
     values, checked against torch SDPA in fp64 on the CPU."""
