@@ -91,6 +91,8 @@ def _decode(lib, **kw):
     (dict(ws=MISALIGNED), 1), (dict(lens=(ctypes.c_int32 * 1)(0)), 1),
     (dict(lens=(ctypes.c_int32 * 1)(257)), 1),
     (dict(ws_bytes=1024), 3),                 # workspace too small
+    (dict(q=MISALIGNED), 1),                  # q must be 16-byte aligned
+    (dict(full=4), 1),                        # unknown flag bit
 ])
 def test_decode_rejects_bad_arguments(lib, kw, status):
     assert _decode(lib, **kw) == status
@@ -142,3 +144,11 @@ def test_workspace_helpers_reject_bad_pointers(lib):
     assert lib.sdk_workspace_init(FAKE, 16, None) == 1
     assert lib.sdk_check_status(None, None, None) == 1
     assert lib.sdk_decode_layout_of(1, 4, 64, 1024, 256, None) == 1
+
+
+def test_timing_calls_check_their_arguments(lib):
+    # machine-independent: no device is queried for these
+    assert lib.sdk_timing_read(None, 4) == -1
+    buf = (ctypes.c_float * 4)()
+    assert lib.sdk_timing_read(buf, -1) == -1
+    assert lib.sdk_timing_enable(0) == 0
