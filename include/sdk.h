@@ -273,7 +273,7 @@ SDK_API sdk_status sdk_decode_attn_shard(int32_t stage, int32_t rank, int32_t wo
  *              max_len) <= SDK_DECODE_STATIC_WS_BYTES, else SDK_ERR_CAPACITY
  *              before anything is launched (for example one sequence with
  *              32 query heads over 32768-atom dictionaries fits up to
- *              about 11,000 tokens).
+ *              about 8,100 tokens).
  *   zeroing    the array's header words must start at zero: they are zero
  *              when the module loads and status_out re-zeroes them; the
  *              kernels write every other byte before reading it.
