@@ -37,7 +37,9 @@ def klow_scores(q, kwords, DK):
 
 
 def hashed_mask(N, head, m):
-    """About m of N tokens, chosen by a multiplicative hash of (token, head)."""
+    """About m of N tokens, chosen by a hash of (token, head): the golden-ratio
+    increment and mixing steps of the SplitMix64 generator (Steele, Lea and
+    Flood, OOPSLA 2014), taken modulo N / m."""
     t = np.arange(N, dtype=np.uint64)
     with np.errstate(over="ignore"):      # arithmetic modulo 2^64 is intended
         h = t * np.uint64(0x9E3779B97F4A7C15) + np.uint64(head) * np.uint64(0xBF58476D1CE4E5B9)
