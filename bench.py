@@ -1,16 +1,22 @@
 """Benchmark of the dictionary-coded KV cache hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sdk|reference]
-                    [--workload layer4k|decode256k|decode32k_b4|prefill256k_vec]
+                    [--workload decode256k|decode32k_b4|prefill256k_vec|layer4k|
+                                append_token_b1|append_token_b4]
 
-Default workload 'layer4k' (one Llama-3.1-8B attention layer, batch 1, 32 q /
-8 KV heads, d=128, 32768-atom bf16 K and V dictionaries, 4096 tokens): one
-step is the whole hot path on that layer -- greedy-pursuit encode of all
-4096 x 8 x 2 = 65,536 K/V vectors written into the code store (sdk_append),
-then one decode-attention step over the 4096 tokens (sdk_decode_attn).
-'decode256k' / 'decode32k_b4' time a 32-layer decode step, 'prefill256k_vec'
-the encode of 262,144 vectors, 'append_token_b1' / 'append_token_b4' the
-append of one generated token to all 32 layers (batch 1 / batch 4).
+Default workload 'decode256k': one decode step of a 32-layer Llama-3.1-8B KV
+shape at batch 1 over 262,144 context tokens (32 q / 8 KV heads, d=128,
+32768-atom bf16 K and V dictionaries per layer, 16-atom codes), the 32 layer
+calls (sdk_decode_attn) replayed as one CUDA graph; the headline value is
+context tokens attended per second per decode step.  The same line carries
+the prefill encode of 16384 tokens x 8 KV heads x 2 streams = 262,144
+vectors (sdk_encode, greedy pursuit over one layer's dictionaries) as the
+keyed sub-record "prefill_encode" (encoded vectors/s, tensor roofline, its
+own e2e); --no-prefill leaves it out.  Other workloads: 'decode32k_b4' (32
+layers, batch 4, 32K tokens), 'prefill256k_vec' alone, 'layer4k' (encode +
+append 65,536 vectors of one layer, then one decode step over 4096 tokens),
+'append_token_b1' / 'append_token_b4' (one generated token appended to all
+32 layers).
 
 Timing: W untimed warm-up steps, then K steps, each timed with CUDA events on
 the launching stream; the L2 is flushed (256 MiB memset) between steps,
@@ -45,9 +51,37 @@ def enc_flop_per_vector(n_atoms, head_dim):
 ENC_KERNELS_PER_CALL = 3
 # kernels of one decode layer: qd, klow, pass2, final, attend, out
 DEC_KERNELS_PER_LAYER = 6
-# DRAM bytes (read + write) of one attend_kernel launch from an ncu capture
-# of the current kernel (one 256K-token layer, cold L2): 141.48 + 5.64 MB
-ATTEND_TRAFFIC = {"decode256k": 147.12e6}
+DECODE_UNIT = "ctx tokens/s/step"
+ENCODE_UNIT = "encoded KV vecs/s"
+
+
+def _sha256(path):
+    import hashlib
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def profiled_traffic(kernel, workload):
+    """DRAM bytes (read + write) per launch of `kernel` on `workload` from
+    the committed ncu summary profiles/<kernel>_<workload>.md, whose lines
+    'traffic_bytes_per_launch: T' and 'source_sha256: H' record the capture
+    and the sha256 of the kernel's source file when it was taken.  None
+    when no summary exists or the source has changed since (the counters
+    then describe another kernel).  Returns (bytes or None, note)."""
+    import re
+    path = os.path.join(ROOT, "profiles", "%s_%s.md" % (kernel, workload))
+    if not os.path.exists(path):
+        return None, "no ncu summary for this kernel and workload"
+    txt = open(path).read()
+    mt = re.search(r"^traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt, re.M)
+    ms = re.search(r"^source_sha256:\s*([0-9a-f]{64})\s+(\S+)", txt, re.M)
+    if not mt or not ms:
+        return None, "summary holds no traffic line"
+    src = os.path.join(ROOT, ms.group(2))
+    if not os.path.exists(src) or _sha256(src) != ms.group(1):
+        return None, "kernel source changed since the capture in %s" % os.path.relpath(path, ROOT)
+    return float(mt.group(1)), ("dram__bytes_read.sum + dram__bytes_write.sum per launch, "
+                                "from %s" % os.path.relpath(path, ROOT))
 ENC_DTYPE = ("f32 (residuals and re-scoring; tensor-core operands fp16 with "
              "fp32 accumulation; bf16 dictionaries; fp16 coefficients)")
 
@@ -70,8 +104,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="sdk", choices=["sdk", "reference"])
-    ap.add_argument("--workload", default="layer4k",
-                    choices=["layer4k", "decode256k", "decode32k_b4",
+    ap.add_argument("--workload", default="decode256k",
+                    choices=["decode256k", "layer4k", "decode32k_b4",
                              "prefill256k_vec", "append_token_b1",
                              "append_token_b4"])
     ap.add_argument("--layers", type=int, default=None,
@@ -88,6 +122,8 @@ def parse():
                          "over the ranks (sdk_decode_attn_shard with NCCL "
                          "exchanges; strong scaling of one context) instead "
                          "of running one independent copy per rank")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="decode256k: leave out the prefill-encode sub-record")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -107,7 +143,12 @@ def peaks():
 # ----------------------------------------------------------------- clocks
 
 class Clocks:
-    """nvidia-smi samples (200 ms) of one GPU while the timed region runs."""
+    """nvidia-smi samples (every 20 ms) of one GPU.  start() returns once
+    the first sample has arrived, so the sampler is running when the timed
+    region begins; mark(True/False) brackets the timed region, and stop()
+    summarises the samples taken inside it (or, when the region is shorter
+    than the sampling period, the last sample before it and the first one
+    after it)."""
 
     Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,"
@@ -118,36 +159,54 @@ class Clocks:
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.lines = []
+        self.lines = []          # (monotonic time, line)
+        self.t0 = self.t1 = None
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
         except (OSError, ValueError):
             self.proc = None
+            return
+        deadline = time.monotonic() + 5.0
+        while not self.lines and time.monotonic() < deadline:
+            time.sleep(0.01)
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def mark(self, begin):
+        if begin:
+            self.t0 = time.monotonic()
+        else:
+            self.t1 = time.monotonic()
 
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        time.sleep(0.25)
+        time.sleep(0.1)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
+        t0 = self.t0 if self.t0 is not None else -1e30
+        t1 = self.t1 if self.t1 is not None else 1e30
+        inside = [ln for t, ln in self.lines if t0 <= t <= t1]
+        if not inside:
+            before = [ln for t, ln in self.lines if t < t0][-1:]
+            after = [ln for t, ln in self.lines if t > t1][:1]
+            inside = before + after
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
                  "sw_power_cap"]
-        for ln in self.lines:
+        for ln in inside:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 8:
                 continue
@@ -161,7 +220,9 @@ class Clocks:
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "timed_region_ms": ((t1 - t0) * 1e3 if self.t0 is not None
+                                    and self.t1 is not None else None)}
 
 
 # ---------------------------------------------------------- distributed
@@ -215,6 +276,8 @@ def timed_steps(step, steps, warmup, flush, world, clocks=None):
     torch.cuda.synchronize()
     if clocks:
         clocks.start()
+        torch.cuda.synchronize()
+        clocks.mark(True)
     evs = []
     for _ in range(steps):
         flush()
@@ -225,6 +288,8 @@ def timed_steps(step, steps, warmup, flush, world, clocks=None):
         b.record()
         evs.append((a, b))
     torch.cuda.synchronize()
+    if clocks:
+        clocks.mark(False)
     barrier(world)
     torch.cuda.synchronize()
     ck = clocks.stop() if clocks else None
@@ -263,6 +328,38 @@ def union_bytes(sdk, ws_list, lay, B, Hq, Hkv, N, k, full):
 
 
 # ---------------------------------------------------------- workloads
+
+def workload_config(name, args):
+    """The `config` object of a workload's line, shared by both arms."""
+    import workloads
+    if name == "prefill256k_vec":
+        return {"workload": name, "n_vectors": 262144, "tokens": 16384,
+                "Hkv": 8, "streams": 2, "head_dim": 128, "n_atoms": 32768,
+                "k_atoms": 16, "vectors": "dense Student-t (nu=4), 4 outlier "
+                "channels x10; correlated dictionaries",
+                "l2": "flushed between steps (256 MiB memset)"}
+    if name == "layer4k":
+        return {"workload": name, "B": 1, "Hq": 32, "Hkv": 8, "head_dim": 128,
+                "n_atoms": 32768, "n_tokens": 4096, "k_atoms": 16, "klow": 3,
+                "khigh": 16, "top": "1/10",
+                "l2": "flushed between steps (256 MiB memset)"}
+    if name in APPEND_WORKLOADS:
+        W = workloads.WORKLOADS[APPEND_WORKLOADS[name]]
+        L = W["L"] if args.layers is None else max(1, min(W["L"], args.layers))
+        return {"workload": name, "layers": L, "B": W["B"], "Hkv": W["Hkv"],
+                "head_dim": W["d"], "n_atoms": W["n_atoms"], "k_atoms": 16,
+                "n_new": 1, "l2": "flushed between steps; the layers' "
+                "dictionaries (%.0f MB) exceed L2" % (L * 2 * W["n_atoms"] * W["d"] * 2 / 1e6)}
+    W = workloads.WORKLOADS[name]
+    L = W["L"] if args.layers is None else max(1, min(W["L"], args.layers))
+    return {"workload": name, "layers": L, "B": W["B"], "Hq": W["Hq"],
+            "Hkv": W["Hkv"], "head_dim": W["d"], "n_atoms": W["n_atoms"],
+            "n_tokens": W["n_tokens"], "klow": 3, "khigh": 16, "top": "1/10",
+            "softmax": ("integer (INT16 logits)" if args.int_softmax else "fp32")
+                       + (", all tokens" if args.full_softmax else ", selected set"),
+            "l2": "flushed between steps; codes (%.1f GB) exceed L2"
+                  % (L * W["B"] * W["Hkv"] * W["n_tokens"] * 140 / 1e9)}
+
 
 def bench_layer4k(args, world, rank, pk):
     import torch
@@ -318,8 +415,9 @@ def bench_layer4k(args, world, rank, pk):
     enc_tflops = flops / (enc_ms * 1e-3) / 1e12
     res = {
         "value": world * n_vec / (step_ms * 1e-3),
-        "unit": "encoded KV vecs/s (whole step: encode+append 65,536 vectors, "
-                "then one decode step over 4096 tokens)",
+        "unit": ENCODE_UNIT,
+        "unit_note": "whole step: encode+append 65,536 vectors, then one "
+                     "decode step over 4096 tokens",
         "ms_per_step": step_ms,
         "encode": {"value": n_vec / (enc_ms * 1e-3), "unit": "vecs/s",
                    "ms": enc_ms, "tflops": enc_tflops},
@@ -331,11 +429,7 @@ def bench_layer4k(args, world, rank, pk):
                                     "encode (sdk_append: 2 x encode_tc_kernel"
                                     " + dictionary prep + scatter)"),
         "clocks": ck,
-        "config": {"workload": "layer4k", "B": 1, "Hq": Hq, "Hkv": Hkv,
-                   "head_dim": d, "n_atoms": n, "n_tokens": N, "k_atoms": 16,
-                   "klow": 3, "khigh": 16, "top": "1/10",
-                   "l2": "flushed between steps (256 MiB memset outside the "
-                         "per-step events)"},
+        "config": workload_config("layer4k", args),
         "dtype": ENC_DTYPE,
         # kernels per step: append = 2 x (dictionary statistics + fp16
         # dictionary copy + encode + scatter); decode = DEC_KERNELS_PER_LAYER
@@ -372,7 +466,7 @@ def e2e_layer4k(args, sdk, store, aws, dws, xk, xv, q, DK, DV, out, world,
     flush = make_flush()
     ms, _ = timed_steps(step, max(2, args.steps // 2), 1, flush, world)
     t = max_over_ranks(statistics.mean(ms), world)
-    return {"value": world * n_vec / (t * 1e-3), "unit": "encoded KV vecs/s",
+    return {"value": world * n_vec / (t * 1e-3), "unit": ENCODE_UNIT,
             "h2d_bytes_per_step": hxk.numel() * 4 + hxv.numel() * 4 + hq.numel() * 4,
             "d2h_bytes_per_step": hout.numel() * 4, "ms_per_step": t}
 
@@ -427,7 +521,8 @@ def bench_decode_sharded(args, world, rank, pk, name):
     gbs = alg / (step_ms * 1e-3) / 1e9
     return {
         "value": B * N / (step_ms * 1e-3),
-        "unit": "ctx tokens/s/step (%d layers, context split over %d GPUs)" % (L, world),
+        "unit": DECODE_UNIT,
+        "unit_note": "%d layers, context split over %d GPUs" % (L, world),
         "ms_per_step": step_ms,
         "scaling": "strong",
         "roofline": {"bound": "hbm", "kernel": "context-sharded decode step "
@@ -509,7 +604,7 @@ def bench_decode(args, world, rank, pk, name):
 
         ms_e, _ = timed_steps(e2e_step, max(2, args.steps // 2), 1, flush, world)
         t = max_over_ranks(statistics.mean(ms_e), world)
-        e2e = {"value": world * B * N / (t * 1e-3), "unit": "ctx tokens/s/step",
+        e2e = {"value": world * B * N / (t * 1e-3), "unit": DECODE_UNIT,
                "ms_per_step": t,
                "h2d_bytes_per_step": sum(h.numel() * 4 for h in hq),
                "d2h_bytes_per_step": hout.numel() * 4}
@@ -545,10 +640,12 @@ def bench_decode(args, world, rank, pk, name):
     # without the Klow scan's 12 B per token per KV head
     att_alg = (code_bytes - L * 12 * N * B * Hkv) / L
     att_gbs = att_alg / (att_ms * 1e-3) / 1e9
-    traffic = ATTEND_TRAFFIC.get(name) if not (args.full_softmax or args.int_softmax) else None
+    traffic, traffic_note = (profiled_traffic("attend_kernel", name)
+                             if not (args.full_softmax or args.int_softmax)
+                             else (None, "no ncu summary for this flag"))
     return {
         "value": world * B * N / (step_ms * 1e-3),
-        "unit": "ctx tokens/s/step (%d layers)" % L,
+        "unit": DECODE_UNIT,
         "ms_per_step": step_ms,
         "ms_per_step_no_graph": statistics.mean(ms_nog),
         "roofline": {"bound": "hbm",
@@ -557,9 +654,7 @@ def bench_decode(args, world, rank, pk, name):
                      "achieved": att_gbs, "peak": pk["hbm"], "unit": "GB/s",
                      "frac": att_gbs / pk["hbm"],
                      "traffic": traffic,
-                     "traffic_source": ("dram__bytes_read.sum + dram__bytes_write.sum "
-                                        "of one launch, ncu --set full, cold L2"
-                                        if traffic else None),
+                     "traffic_source": traffic_note,
                      "alg_bytes_per_launch": att_alg,
                      "ms_per_launch": att_ms, "launches_timed": len(att),
                      "step": {"kernels": "all %d per layer, %d layers"
@@ -568,14 +663,7 @@ def bench_decode(args, world, rank, pk, name):
                               "alg_bytes_per_step": alg,
                               "union_tokens_per_step": U}},
         "clocks": ck,
-        "config": {"workload": name, "layers": L, "B": B, "Hq": Hq,
-                   "Hkv": Hkv, "head_dim": d, "n_atoms": n, "n_tokens": N,
-                   "klow": 3, "khigh": 16, "top": "1/10",
-                   "softmax": ("integer (INT16 logits)" if args.int_softmax
-                               else "fp32") + (", all tokens" if args.full_softmax
-                                               else ", selected set"),
-                   "l2": "flushed between steps; codes (%.1f GB) exceed L2"
-                         % (L * B * Hkv * N * 140 / 1e9)},
+        "config": workload_config(name, args),
         "dtype": "f32 (bf16 dictionaries, fp16 coefficients)",
         "gpu_launches": args.steps * L * DEC_KERNELS_PER_LAYER,
         **({"e2e": e2e} if e2e else {}),
@@ -625,21 +713,19 @@ def bench_prefill(args, world, rank, pk):
 
         ms_e, _ = timed_steps(e2e_step, max(2, args.steps // 2), 1, flush, world)
         t = max_over_ranks(statistics.mean(ms_e), world)
-        e2e = {"value": world * 2 * nv / (t * 1e-3), "unit": "encoded KV vecs/s",
+        e2e = {"value": world * 2 * nv / (t * 1e-3), "unit": ENCODE_UNIT,
                "ms_per_step": t,
                "h2d_bytes_per_step": (hxk.numel() + hxv.numel()) * 4,
                "d2h_bytes_per_step": (hck.numel() + hcv.numel()) * 4}
     flops = 2 * nv * enc_flop_per_vector(n, d)
     tfl = flops / (step_ms * 1e-3) / 1e12
     return {
-        "value": world * 2 * nv / (step_ms * 1e-3), "unit": "encoded KV vecs/s",
+        "value": world * 2 * nv / (step_ms * 1e-3), "unit": ENCODE_UNIT,
         "ms_per_step": step_ms,
         "roofline": tensor_roofline(tfl, pk, "encode (2 x sdk_encode: "
                                     "encode_tc_kernel + dictionary prep)"),
         "clocks": ck,
-        "config": {"workload": "prefill256k_vec", "n_vectors": 2 * nv,
-                   "head_dim": d, "n_atoms": n, "k_atoms": 16,
-                   "l2": "flushed between steps"},
+        "config": workload_config("prefill256k_vec", args),
         "dtype": ENC_DTYPE,
         "gpu_launches": args.steps * 2 * ENC_KERNELS_PER_CALL,
         "enc_fallback_rows": hdr[2],
@@ -691,7 +777,8 @@ def bench_append(args, world, rank, pk, name):
     tfl = flops / (step_ms * 1e-3) / 1e12
     res = {
         "value": world * n_vec / (step_ms * 1e-3),
-        "unit": "encoded KV vecs/s (one token appended to all %d layers)" % L,
+        "unit": ENCODE_UNIT,
+        "unit_note": "one token appended to all %d layers" % L,
         "ms_per_step": step_ms,
         "us_per_token": step_ms * 1e3,
         "us_per_layer": step_ms * 1e3 / L,
@@ -704,10 +791,7 @@ def bench_append(args, world, rank, pk, name):
                               "%.1f us per step" % (step_ms * 1e3 / L / 16),
                          hbm_floor_us=L * 2 * n * d * 2 / (pk["hbm"] * 1e9) * 1e6),
         "clocks": ck,
-        "config": {"workload": name, "layers": L, "B": B, "Hkv": Hkv,
-                   "head_dim": d, "n_atoms": n, "k_atoms": 16, "n_new": 1,
-                   "l2": "flushed between steps; the %d layers' dictionaries "
-                         "(%.0f MB) exceed L2" % (L, L * 2 * n * d * 2 / 1e6)},
+        "config": workload_config(name, args),
         "dtype": ("f32 (residuals, exact re-scoring; tensor-core operands "
                   "bf16 with fp32 accumulation; fp16 coefficients)"),
         # per layer one kernel (the exchange words are cleared by a runtime
@@ -732,7 +816,7 @@ def bench_append(args, world, rank, pk, name):
         ms_e, _ = timed_steps(e2e_step, max(2, args.steps // 2), 1, flush, world)
         t = max_over_ranks(statistics.mean(ms_e), world)
         res["e2e"] = {"value": world * n_vec / (t * 1e-3),
-                      "unit": "encoded KV vecs/s", "ms_per_step": t,
+                      "unit": ENCODE_UNIT, "ms_per_step": t,
                       "h2d_bytes_per_step": sum(a.numel() * 4 + b.numel() * 4
                                                 for a, b in hx),
                       "d2h_bytes_per_step": hout.numel() * 4}
@@ -741,111 +825,141 @@ def bench_append(args, world, rank, pk, name):
 
 # ------------------------------------------------------ oracle timings
 
-def cpu_baseline(name, budget_s=15.0):
-    """The fp64 oracle on this host's cores, on a bounded sample of the
-    workload, scaled to the metric's unit."""
+def oracle_sampler(name):
+    """The fp64 oracle on this host's cores, prepared for a bounded sample
+    of the workload: returns run(budget_s) -> {value, unit, cores, kind,
+    sample}, the oracle's rate scaled to the metric's unit.  The sample's
+    inputs are generated once, outside every timing."""
     import numpy as np
     import torch
     import oracle
     import workloads
     cores = len(os.sched_getaffinity(0))
     torch.set_num_threads(cores)
+
+    def encode_runner(xs, Dn, per_step, what, extra=None):
+        def run(budget_s):
+            t0 = time.perf_counter()
+            nvec = 0
+            while (time.perf_counter() - t0 < budget_s * 0.8 or nvec == 0) \
+                    and nvec < xs.shape[0]:
+                oracle.encode_ref(xs[nvec:nvec + 4], Dn)
+                nvec += 4
+            t_vec = (time.perf_counter() - t0) / nvec
+            t_step = t_vec * per_step
+            sample = "%d %s encoded by the oracle" % (nvec, what)
+            if extra is not None:
+                t_extra, note = extra()
+                t_step += t_extra
+                sample += note
+            return {"value": per_step / t_step, "unit": ENCODE_UNIT,
+                    "cores": cores, "kind": "oracle",
+                    "sample": sample + "; rate scaled to the whole step"}
+        return run
+
     if name in APPEND_WORKLOADS:
         base = APPEND_WORKLOADS[name]
         W = workloads.WORKLOADS[base]
         a = workloads.append_token(base, 0)
         xs = a["xk"].reshape(-1, a["d"]).double().numpy()
         Dn = a["DK"].float().double().numpy()
-        t0 = time.perf_counter()
-        nvec = 0
-        while time.perf_counter() - t0 < budget_s * 0.8 and nvec < xs.shape[0]:
-            oracle.encode_ref(xs[nvec:nvec + 4], Dn)
-            nvec += 4
-        t_vec = (time.perf_counter() - t0) / nvec
         per_step = W["L"] * 2 * W["B"] * W["Hkv"]
-        return {"value": 1.0 / t_vec, "unit": "encoded KV vecs/s",
-                "cores": cores, "kind": "oracle",
-                "sample": "%d of the %d vectors of one token's append encoded "
-                          "by the oracle" % (nvec, per_step)}
-    if name in ("layer4k", "prefill256k_vec"):
-        if name == "layer4k":
-            w = workloads.layer4k()
-            x = w["xk"].reshape(-1, w["d"])
-            D = w["DK"]
-            per_step = 2 * w["Hkv"] * w["n_tokens"]
-        else:
-            w = workloads.prefill(n_tokens=64)
-            x = w["xk"].reshape(-1, w["d"])
-            D = w["DK"]
-            per_step = 2 * 8 * 16384
-        Dn = D.float().double().numpy()
-        xs = x.double().numpy()
-        t0 = time.perf_counter()
-        nvec = 0
-        while time.perf_counter() - t0 < budget_s * 0.8 and nvec < xs.shape[0]:
-            oracle.encode_ref(xs[nvec:nvec + 4], Dn)
-            nvec += 4
-        t_enc = (time.perf_counter() - t0) / nvec
-        sample = "%d vectors encoded by the oracle" % nvec
-        t_step = t_enc * per_step
-        if name == "layer4k":
-            # plus one decode head over 4096 tokens (x32 heads)
-            g = workloads.make_gen(5)
-            kw = workloads.random_codes((4096,), 32768, g).numpy().view(np.uint32)
-            vw = workloads.random_codes((4096,), 32768, g).numpy().view(np.uint32)
-            qh = np.random.default_rng(0).standard_normal(128)
+        return encode_runner(xs, Dn, per_step, "of the %d vectors of one token's "
+                             "append" % per_step)
+    if name == "layer4k":
+        w = workloads.layer4k()
+        xs = w["xk"].reshape(-1, w["d"]).double().numpy()
+        Dn = w["DK"].float().double().numpy()
+        per_step = 2 * w["Hkv"] * w["n_tokens"]
+        g = workloads.make_gen(5)
+        kw = workloads.random_codes((4096,), 32768, g).numpy().view(np.uint32)
+        vw = workloads.random_codes((4096,), 32768, g).numpy().view(np.uint32)
+        qh = np.random.default_rng(0).standard_normal(128)
+
+        def dec():
             t1 = time.perf_counter()
             oracle.decode_head_ref(qh, kw, vw, Dn, Dn)
-            t_dec = (time.perf_counter() - t1) * 32
-            t_step += t_dec
-            sample += " + 1 of 32 decode heads (4096 tokens)"
-        return {"value": per_step / t_step, "unit": "encoded KV vecs/s",
-                "cores": cores, "kind": "oracle",
-                "sample": sample + "; extrapolated to the full step"}
+            return (time.perf_counter() - t1) * 32, " + 1 of 32 decode heads (4096 tokens)"
+        return encode_runner(xs, Dn, per_step, "vectors", dec)
+    if name == "prefill256k_vec":
+        w = workloads.prefill(n_tokens=64)
+        xs = w["xk"].reshape(-1, w["d"]).double().numpy()
+        Dn = w["DK"].float().double().numpy()
+        return encode_runner(xs, Dn, 2 * 8 * 16384, "of the 262,144 vectors")
     # decode workloads: one head of one layer, x (L*B*Hq)
     W = workloads.WORKLOADS[name]
     lay = workloads.decode_layer(name, 0, B=1)
-    kw = lay["kwords"][0, 0].numpy().view(np.uint32)
-    vw = lay["vwords"][0, 0].numpy().view(np.uint32)
+    kw = lay["kwords"][0, 0].numpy().view(np.uint32).copy()
+    vw = lay["vwords"][0, 0].numpy().view(np.uint32).copy()
     qn = lay["q"][0, 0].double().numpy()
     Dk = lay["DK"].float().double().numpy()
     Dv = lay["DV"].float().double().numpy()
-    t0 = time.perf_counter()
-    oracle.decode_head_ref(qn, kw, vw, Dk, Dv)
-    t_head = time.perf_counter() - t0
-    t_step = t_head * W["L"] * W["B"] * W["Hq"]
-    return {"value": W["B"] * W["n_tokens"] / t_step,
-            "unit": "ctx tokens/s/step", "cores": cores, "kind": "oracle",
-            "sample": "1 query head of 1 layer (%d tokens), extrapolated x%d"
-                      % (W["n_tokens"], W["L"] * W["B"] * W["Hq"])}
+    del lay
+    heads = W["L"] * W["B"] * W["Hq"]
+
+    def run(budget_s):
+        t0 = time.perf_counter()
+        oracle.decode_head_ref(qn, kw, vw, Dk, Dv)
+        t_step = (time.perf_counter() - t0) * heads
+        return {"value": W["B"] * W["n_tokens"] / t_step, "unit": DECODE_UNIT,
+                "cores": cores, "kind": "oracle",
+                "sample": "1 query head of 1 layer (%d tokens), time x%d for the "
+                          "whole step" % (W["n_tokens"], heads)}
+    return run
+
+
+def cpu_baseline(name, budget_s=15.0):
+    """One bounded oracle sample of the workload (see oracle_sampler)."""
+    return oracle_sampler(name)(budget_s)
 
 
 def reference_arm(args):
     """The oracle as the reference implementation, timed on the host cores
-    with the same metric, unit and config as the sdk arm."""
+    with the same metric, unit and config as the sdk arm; with the default
+    workload it also carries the prefill-encode sub-record."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     name = args.workload
-    vals = []
-    for _ in range(args.warmup):
-        cpu_baseline(name, budget_s=0.5)
-    t0 = time.perf_counter()
-    for _ in range(max(1, args.steps)):
-        vals.append(cpu_baseline(name, budget_s=min(20.0, 120.0 / max(1, args.steps))))
-    wall = time.perf_counter() - t0
-    v = statistics.mean(x["value"] for x in vals)
-    cb = dict(vals[0])
-    cb["value"] = v
+
+    def arm(nm, steps, warmup):
+        run = oracle_sampler(nm)
+        for _ in range(warmup):
+            run(0.2)
+        vals = []
+        t0 = time.perf_counter()
+        for _ in range(max(1, steps)):
+            vals.append(run(min(20.0, 90.0 / max(1, steps))))
+        wall = time.perf_counter() - t0
+        v = statistics.mean(x["value"] for x in vals)
+        cb = dict(vals[0])
+        cb["value"] = v
+        return v, vals[0]["unit"], wall * 1e3 / max(1, steps), cb
+
+    v, unit, ms, cb = arm(name, args.steps, args.warmup)
     line = {"impl": "reference", "metric": METRIC, "value": v,
-            "unit": vals[0]["unit"], "n_gpus": args.gpus, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": wall * 1e3 / max(1, args.steps),
+            "unit": unit, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic",
-            "config": {"workload": name}, "cpu_baseline": cb,
-            "e2e": {"value": v, "unit": vals[0]["unit"],
+            "config": workload_config(name, args), "cpu_baseline": cb,
+            "e2e": {"value": v, "unit": unit,
                     "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    if with_prefill(args):
+        pv, pu, pms, pcb = arm("prefill256k_vec", max(1, args.steps // 4), 1)
+        line["prefill_encode"] = {
+            "value": pv, "unit": pu, "ms_per_step": pms,
+            "config": workload_config("prefill256k_vec", args),
+            "cpu_baseline": pcb,
+            "e2e": {"value": pv, "unit": pu, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def with_prefill(args):
+    """The default decode256k line carries the prefill-encode sub-record."""
+    return (args.workload == "decode256k" and not args.no_prefill and not
+            (args.full_softmax or args.int_softmax or args.context_shard))
 
 
 def main():
@@ -868,6 +982,12 @@ def main():
         res = bench_decode_sharded(args, world, rank, pk, args.workload)
     else:
         res = bench_decode(args, world, rank, pk, args.workload)
+    if with_prefill(args):
+        pre = bench_prefill(args, world, rank, pk)
+        pre["roofline"]["peak_source"] = pk["src"]
+        if world == 1 and not args.no_cpu_baseline:
+            pre["cpu_baseline"] = cpu_baseline("prefill256k_vec")
+        res["prefill_encode"] = pre
     if rank == 0:
         line = {"metric": METRIC, "value": res.pop("value"),
                 "unit": res.pop("unit"), "n_gpus": world, "steps": args.steps,

@@ -85,6 +85,19 @@ SDK_API const char* sdk_status_string(int status);
 /* Library ABI version (incremented on any signature change). */
 SDK_API int32_t sdk_version(void);
 
+/* Limit, in nanoseconds of the GPU's global timer, of every device-side
+ * wait for another CTA's result: the small-batch encoder's per-step
+ * exchange of slice winners (sdk_encode / sdk_append with at most 64
+ * vectors).  A wait that runs out records SDK_ERR_TIMEOUT in the
+ * workspace header (read by sdk_check_status); the kernel then leaves its
+ * loop, frees its tensor memory and returns, and the CTAs waiting for it
+ * run out in turn.  No copy or MMA of the CTA is in flight at these waits.
+ * Process-wide; default 1 s; 0 gives up at the first word that is not
+ * there yet.  Returns the previous limit.  The waits on the CTA's own
+ * copies and MMAs (mbarriers) keep their fixed 1 s limit.  The paper has
+ * no counterpart: this is the failure detection of the device waits. */
+SDK_API uint64_t sdk_set_exchange_timeout_ns(uint64_t ns);
+
 /* ------------------------------------------------------------------ encode
  * Greedy pursuit ("LLM Inference in a Flash!", review Summary): for every
  * input vector x, r = x; 16 times: i* = argmax_i |<r, d_i>| (ties: lowest
@@ -156,6 +169,10 @@ SDK_API size_t sdk_append_workspace_bytes(int32_t B, int32_t Hkv, int32_t n_new,
 /* decode flags */
 #define SDK_DECODE_FULL_SOFTMAX 1   /* softmax over every token, not only S   */
 #define SDK_DECODE_INT_SOFTMAX 2    /* integer softmax (see sdk_decode_attn)  */
+#define SDK_DECODE_KEEP_KEYS 4      /* also store every token's s_lo key in
+                                       the workspace region `keys` (for
+                                       inspection; costs 4 B per token and
+                                       query head of extra writes)           */
 
 /* ------------------------------------------------------------ decode attn
  * One layer of decode attention for B sequences over their code stores
@@ -277,9 +294,11 @@ SDK_API sdk_status sdk_decode_attn_shard(int32_t stage, int32_t rank, int32_t wo
  *   zeroing    the array's header words must start at zero: they are zero
  *              when the module loads and status_out re-zeroes them; the
  *              kernels write every other byte before reading it.
- *   setup      the first call on a device looks up the array's address
- *              (cudaGetSymbolAddress, which may load the module); make that
- *              first call before any stream capture.
+ *   setup      the first call in a device's context looks up the array's
+ *              address (cudaGetSymbolAddress, which may load the module);
+ *              make that first call before any stream capture.  The
+ *              address is kept per context and looked up again when the
+ *              current context changes (after cudaDeviceReset, for one).
  *   races      there is one array per device: calls that overlap in time
  *              on a device (other streams, other host threads) race on it
  *              and give undefined results; serialise them on one stream.
@@ -342,7 +361,13 @@ typedef struct {
   uint32_t isoft_sum[2];  /* integer softmax: E = sum of the integer
                              exponentials, low and high words              */
   uint32_t isoft_shift;   /* integer softmax: the overflow guard's shift   */
-  uint32_t pad[2];
+  uint32_t bracket_lo;    /* sampled bracket of the k-th key: tokens with  */
+  uint32_t bracket_hi;    /*   key > hi are selected during the Klow scan,
+                             lo <= key <= hi become candidates (0 and 0
+                             when the selection ran by radix histograms)   */
+  uint32_t select_path;   /* 0: histogram passes; 1: sampled bracket; 2:
+                             bracket missed, exact re-scan of the head     */
+  uint32_t pad[3];
 } sdk_select_state;
 
 SDK_API sdk_status sdk_decode_layout_of(int32_t B, int32_t Hq, int32_t head_dim,

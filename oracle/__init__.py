@@ -35,12 +35,12 @@ from .encode import (FP16_MAX, greedy_pursuit, encode_ref, store_coef_fp16,
                      pack_words, unpack_words)
 from .decode import (topk_count, select_top, decode_attn_ref,
                      decode_head_ref, decode_vectors, integer_softmax)
-from .certify import certify_codes
+from .certify import certify_codes, certify_codes_batched
 from .omp import omp, omp_ref
 
 __all__ = [
     "FP16_MAX", "greedy_pursuit", "encode_ref", "store_coef_fp16",
     "pack_words", "unpack_words", "topk_count", "select_top",
-    "decode_attn_ref", "decode_head_ref", "decode_vectors", "certify_codes",
+    "decode_attn_ref", "decode_head_ref", "decode_vectors", "certify_codes", "certify_codes_batched",
     "omp", "omp_ref", "integer_softmax",
 ]

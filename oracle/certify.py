@@ -54,3 +54,40 @@ def certify_codes(X, D, words, rel_tol=1e-4, coef_rel_tol=1e-3):
             r = r - exact * D[i]
     return {"pick_ratio": ratio, "coef_err": cerr, "ok_pick": ok_pick,
             "ok_coef": ok_coef}
+
+
+def certify_codes_batched(X, D, words, rel_tol=1e-4, coef_rel_tol=1e-3,
+                          batch=256):
+    """certify_codes for many vectors: the same replay, step for step, for a
+    batch of vectors at a time (each step's inner products of the batch's
+    residuals with all atoms as one matrix product).  Same return value."""
+    X = np.asarray(X, dtype=np.float64)
+    D = np.asarray(D, dtype=np.float64)
+    idx, coef_st = unpack_words(words)
+    m, k = idx.shape
+    ratio = np.ones((m, k))
+    cerr = np.zeros((m, k))
+    ok_pick = np.ones((m, k), dtype=bool)
+    ok_coef = np.ones((m, k), dtype=bool)
+    Dt = np.ascontiguousarray(D.T)
+    for v0 in range(0, m, batch):
+        sl = slice(v0, min(m, v0 + batch))
+        R = X[sl].copy()
+        rows = np.arange(R.shape[0])
+        xnorm = np.linalg.norm(R, axis=1)
+        for j in range(k):
+            C = R @ Dt                          # [b, n] all <r, d_i>
+            top = np.abs(C).max(axis=1)
+            i = idx[sl, j]
+            exact = C[rows, i]
+            nz = top > 0.0
+            ratio[sl, j] = np.where(nz, np.abs(exact) / np.where(nz, top, 1.0), 1.0)
+            ok_pick[sl, j] = np.where(nz, ratio[sl, j] >= 1.0 - rel_tol, True)
+            big = np.abs(exact) > 1e-12 * np.maximum(xnorm, 1e-300)
+            ce = np.abs(coef_st[sl, j] - exact) / np.where(big, np.abs(exact), 1.0)
+            cerr[sl, j] = np.where(big, ce, 0.0)
+            ok_coef[sl, j] = np.where(big, ce <= coef_rel_tol,
+                                      np.abs(coef_st[sl, j]) <= 1e-6 * np.maximum(xnorm, 1.0))
+            R = R - exact[:, None] * D[i]
+    return {"pick_ratio": ratio, "coef_err": cerr, "ok_pick": ok_pick,
+            "ok_coef": ok_coef}

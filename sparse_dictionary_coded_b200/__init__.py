@@ -18,7 +18,8 @@ import torch
 from . import _capi
 from ._capi import (SDK_OK, SDK_F32, SDK_BF16, MAX_ATOMS, K_ATOMS,
                     KLOW_PLANES, MAX_BATCH, SDK_DECODE_FULL_SOFTMAX,
-                    SDK_DECODE_INT_SOFTMAX, DecodeLayout, load)
+                    SDK_DECODE_INT_SOFTMAX, SDK_DECODE_KEEP_KEYS, DecodeLayout,
+                    load)
 
 __all__ = [
     "SdkError", "load", "sdk_encode", "sdk_encode_simt", "sdk_append",
@@ -26,6 +27,7 @@ __all__ = [
     "sdk_append_workspace_bytes", "sdk_decode_workspace_bytes",
     "sdk_decode_layout_of", "sdk_workspace_init", "sdk_check_status",
     "new_workspace", "CodeStore", "read_select_state", "sdk_timing_enable",
+    "sdk_set_exchange_timeout_ns", "decode_flags",
     "sdk_timing_read",
 ]
 
@@ -87,6 +89,12 @@ def sdk_check_status(ws, stream=None):
     buf = (ctypes.c_uint32 * 4)()
     rc = load().sdk_check_status(_ptr(ws), _stream(stream), buf)
     return rc, list(buf)
+
+
+def sdk_set_exchange_timeout_ns(ns):
+    """Limit (ns) of the device waits for other CTAs' results; returns the
+    previous limit (include/sdk.h, sdk_set_exchange_timeout_ns)."""
+    return int(load().sdk_set_exchange_timeout_ns(int(ns)))
 
 
 def sdk_timing_enable(on):
@@ -235,13 +243,21 @@ def sdk_append(store, xk, xv, dict_k, dict_v, workspace=None, stream=None):
 
 # ------------------------------------------------------------------ decode
 
+def decode_flags(full_softmax=False, int_softmax=False, keep_keys=False):
+    """The flags word of sdk_decode_attn."""
+    return ((SDK_DECODE_FULL_SOFTMAX if full_softmax else 0) |
+            (SDK_DECODE_INT_SOFTMAX if int_softmax else 0) |
+            (SDK_DECODE_KEEP_KEYS if keep_keys else 0))
+
+
 def sdk_decode_attn(q, dict_k, dict_v, store, klow=3, khigh=16, top_num=1,
                     top_den=10, full_softmax=False, scale=None, out=None,
-                    workspace=None, stream=None, int_softmax=False):
+                    workspace=None, stream=None, int_softmax=False,
+                    keep_keys=False):
     """One layer of decode attention.  q [B, Hq, head_dim] fp32.  Returns
     out [B, Hq, head_dim] fp32 (and leaves the intermediate results in the
-    workspace).  full_softmax / int_softmax set SDK_DECODE_FULL_SOFTMAX /
-    SDK_DECODE_INT_SOFTMAX."""
+    workspace).  full_softmax / int_softmax / keep_keys set
+    SDK_DECODE_FULL_SOFTMAX / SDK_DECODE_INT_SOFTMAX / SDK_DECODE_KEEP_KEYS."""
     lib = load()
     q = _cuda_contig(q, "q", (torch.float32,))
     dk = _cuda_contig(dict_k, "dict_k", (torch.bfloat16,))
@@ -262,8 +278,7 @@ def sdk_decode_attn(q, dict_k, dict_v, store, klow=3, khigh=16, top_num=1,
                              n_atoms, _ptr(store.k_lo), _ptr(store.k_full),
                              _ptr(store.v_full), store.cap, lens, klow, khigh,
                              top_num, top_den,
-                             (SDK_DECODE_FULL_SOFTMAX if full_softmax else 0) |
-                             (SDK_DECODE_INT_SOFTMAX if int_softmax else 0),
+                             decode_flags(full_softmax, int_softmax, keep_keys),
                              float(scale), _ptr(out), _ptr(workspace),
                              workspace.numel(), _stream(stream))
     _check(rc, "sdk_decode_attn")

@@ -17,7 +17,7 @@ STATUS_NAMES = {
     6: "SDK_ERR_DEVICE_CHECK",
 }
 SDK_F32, SDK_BF16 = 0, 1
-SDK_DECODE_FULL_SOFTMAX, SDK_DECODE_INT_SOFTMAX = 1, 2
+SDK_DECODE_FULL_SOFTMAX, SDK_DECODE_INT_SOFTMAX, SDK_DECODE_KEEP_KEYS = 1, 2, 4
 MAX_ATOMS, K_ATOMS, KLOW_PLANES, MAX_BATCH, WS_ALIGN = 32768, 16, 3, 64, 256
 DECODE_STATIC_WS_BYTES = 16 << 20
 
@@ -29,6 +29,7 @@ SDK_TIMING_SLOTS = 256
 SIGNATURES = {
     "sdk_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "sdk_version": (_i32, []),
+    "sdk_set_exchange_timeout_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
     "sdk_encode": (ctypes.c_int, [_vp, _i32, _i64, _i32, _vp, _i32, _i32, _vp,
                                   _vp, _vp, _sz, _vp]),
     "sdk_encode_simt": (ctypes.c_int, [_vp, _i32, _i64, _i32, _vp, _i32, _i32,
@@ -70,8 +71,9 @@ class DecodeLayout(ctypes.Structure):
 
 SELECT_STATE_FIELDS = ("kth_key", "k", "n_above", "n_cand", "n_sel", "n_comp",
                        "eq_total", "eq_taken", "max_score", "max_comp", "z",
-                       "isoft_sum_lo", "isoft_sum_hi", "isoft_shift")
-SELECT_STATE_WORDS = 16
+                       "isoft_sum_lo", "isoft_sum_hi", "isoft_shift",
+                       "bracket_lo", "bracket_hi", "select_path")
+SELECT_STATE_WORDS = 20
 
 _lib = None
 

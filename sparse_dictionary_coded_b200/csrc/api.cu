@@ -1,5 +1,6 @@
 // C ABI of libsdk.so: argument checks, workspace carving and stream-ordered
 // launches.  The operations are defined in include/sdk.h.
+#include <atomic>
 #include <cmath>
 #include <cstring>
 
@@ -8,6 +9,14 @@
 namespace sdk {
 
 
+
+namespace {
+std::atomic<unsigned long long> g_exchange_wait_ns{1000000000ull};
+}
+unsigned long long exchange_wait_ns() { return g_exchange_wait_ns.load(std::memory_order_relaxed); }
+unsigned long long set_exchange_wait_ns(unsigned long long ns) {
+  return g_exchange_wait_ns.exchange(ns, std::memory_order_relaxed);
+}
 
 int num_sms() {
   static int cache[64] = {0};
@@ -83,7 +92,9 @@ const char* sdk_status_string(int status) {
   }
 }
 
-int32_t sdk_version(void) { return 1; }
+int32_t sdk_version(void) { return 2; }
+
+uint64_t sdk_set_exchange_timeout_ns(uint64_t ns) { return sdk::set_exchange_wait_ns(ns); }
 
 size_t sdk_encode_workspace_bytes(int64_t n_vec, int32_t head_dim, int32_t n_atoms) {
   if (n_vec < 0) n_vec = 0;
@@ -319,6 +330,17 @@ sdk_status sdk_decode_layout_of(int32_t B, int32_t Hq, int32_t head_dim, int32_t
 
 }  // extern "C"
 
+// Selection by a sampled bracket of the k-th key unless SDK_DECODE_BRACKET=0
+// (read once per process; the radix histogram passes then run instead).
+static bool bracket_selection() {
+  static int on = -1;
+  if (on < 0) {
+    const char* v = getenv("SDK_DECODE_BRACKET");
+    on = (v != nullptr && v[0] == '0') ? 0 : 1;
+  }
+  return on == 1;
+}
+
 // Checks the decode arguments and fills the kernel parameter block.  With
 // glens (the sequences' whole lengths; context-sharded decode) the selected
 // set size k comes from glens[b] and lens_host holds this rank's shard.
@@ -337,7 +359,8 @@ static sdk_status build_decode_params(const float* q, int32_t B, int32_t Hq, int
   if (klow < 1 || khigh < klow || khigh > SDK_K_ATOMS) return SDK_ERR_INVALID_ARG;
   if (top_num < 1 || top_den < 1 || top_num > top_den) return SDK_ERR_INVALID_ARG;
   if (!(scale > 0.0f) || !std::isfinite(scale)) return SDK_ERR_INVALID_ARG;
-  if (flags & ~(SDK_DECODE_FULL_SOFTMAX | SDK_DECODE_INT_SOFTMAX)) return SDK_ERR_INVALID_ARG;
+  if (flags & ~(SDK_DECODE_FULL_SOFTMAX | SDK_DECODE_INT_SOFTMAX | SDK_DECODE_KEEP_KEYS))
+    return SDK_ERR_INVALID_ARG;
   if (!q || !dict_k || !dict_v || !k_lo || !k_full || !v_full || !out || !lens_host || !workspace)
     return SDK_ERR_INVALID_ARG;
   if (!aligned(workspace, SDK_WS_ALIGN) || !aligned(dict_k, 16) || !aligned(dict_v, 16) ||
@@ -386,6 +409,11 @@ static sdk_status build_decode_params(const float* q, int32_t B, int32_t Hq, int
   p.khigh = khigh;
   p.full = (flags & SDK_DECODE_FULL_SOFTMAX) ? 1 : 0;
   p.isoft = (flags & SDK_DECODE_INT_SOFTMAX) ? 1 : 0;
+  // the sampled-bracket selection unless the softmax runs over every token
+  // (that path needs every key and the complement list) or
+  // SDK_DECODE_BRACKET=0 is set in the environment
+  p.bracket = (!p.full && bracket_selection()) ? 1 : 0;
+  p.keep_keys = (flags & SDK_DECODE_KEEP_KEYS) ? 1 : 0;
   p.R = B * Hq;
   p.n_out_tiles = (n_atoms + 127) / 128;
   p.scale = scale;
@@ -446,6 +474,7 @@ sdk_status sdk_decode_attn_shard(int32_t stage, int32_t rank, int32_t world, con
   if (s != SDK_OK) return s;
   p.world = world;
   p.shard_in = gathered;
+  p.bracket = 0;   // the context-sharded stages exchange radix histograms
   return launch_decode(p, reinterpret_cast<cudaStream_t>(stream), stage, rank);
 }
 

@@ -169,23 +169,15 @@ __global__ void __launch_bounds__(64 * kGvTiles * RB, (RB > 1 ? 2 : 1)) qd_kerne
   {
     const int64_t nthr = (int64_t)gridDim.x * gridDim.y * kThreads;
     const int64_t g0 = ((int64_t)blockIdx.y * gridDim.x + blockIdx.x) * kThreads + tid;
-    const int64_t hwords = (int64_t)R * 4096;
+    const int64_t hwords = p.bracket ? 0 : (int64_t)R * 4096;   // radix selection path only
     for (int64_t e = g0; e < hwords; e += nthr) {
       p.hist1[e] = 0u;
       p.hist2[e] = 0u;
     }
     for (int64_t e = g0; e < (int64_t)R * D; e += nthr) p.out[e] = 0.0f;
     for (int64_t e = g0; e < (int64_t)R; e += nthr) {
-      sdk_select_state st;
-      st.kth_key = 0u;
+      sdk_select_state st = {};
       st.k = (uint32_t)p.kcnt[e / p.Hq];
-      st.n_above = st.n_cand = st.n_sel = st.n_comp = 0u;
-      st.eq_total = st.eq_taken = 0u;
-      st.max_score = 0u;
-      st.max_comp = 0u;
-      st.z = 0.0f;
-      st.isoft_sum[0] = st.isoft_sum[1] = st.isoft_shift = 0u;
-      st.pad[0] = st.pad[1] = 0u;
       p.st[e] = st;
     }
   }
@@ -269,11 +261,17 @@ __global__ void __launch_bounds__(64 * kGvTiles * RB, (RB > 1 ? 2 : 1)) qd_kerne
 // table (zero past n: every 15-bit index reads inside it, and an index >= n
 // is reported once per thread after the scan), the three k_lo planes read
 // four tokens at a time (16-byte loads when the planes are 16-byte
-// aligned), one gather and one FMA per word.  Writes the order-preserving
-// key of every token (one 16-byte store per quad; four 4-byte stores per
-// quad cost as much as the rest of the scan) and the 12-bit histogram of
-// key bits 31..20 of every head (shared-memory atomics, flushed once per
-// segment).
+// aligned), one gather and one FMA per word.
+//   kBracket = false: writes the order-preserving key of every token (one
+//     16-byte store per quad; four 4-byte stores per quad cost as much as
+//     the rest of the scan) and the 12-bit histogram of key bits 31..20 of
+//     every head (shared-memory atomics, flushed once per segment), for the
+//     radix selection of pass2_kernel and final_kernel.
+//   kBracket = true: classifies every token against the head's sampled
+//     bracket [lo, hi] of the k-th key (sample_kernel) as it is scored:
+//     key > hi goes to the front of the selected list, lo <= key <= hi to
+//     the candidates (token and key), the rest is dropped; slots come from
+//     one atomic per warp and kind.  Keys are stored only with keep_keys.
 constexpr int kScanThreads = 512;
 // Start-up cost of one head segment in token units, from per-CTA timings at
 // 256K tokens (CTAs that touched two heads against those that touched one):
@@ -312,26 +310,38 @@ __device__ __forceinline__ void stage_table(float* table, const float* src, int 
   for (int i = n + threadIdx.x; i < kTable; i += nt) table[i] = 0.0f;
 }
 
+template <bool kBracket>
 __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, int vec) {
   pdl_wait();     // nothing global is touched before the previous kernel is done
   pdl_launch();
   extern __shared__ float4 smem4[];
   float* table = reinterpret_cast<float*>(smem4);
   uint32_t* sh = reinterpret_cast<uint32_t*>(table + kTable);
-  const int n = p.n, tid = threadIdx.x;
+  const int n = p.n, tid = threadIdx.x, lane = tid & 31;
   const int nlo = min(p.klow, kLoPlanes);
+  const bool store_keys = !kBracket || p.keep_keys;
   uint32_t maxidx = 0u;
 
   for_segments(p.tok_off, p.lens, p.B, p.Hq, kKlowSegCost, [&](int b, int h, int64_t t0l, int64_t t1l) {
     const int r = b * p.Hq + h, kvh = h / p.g;
     const int t0 = (int)t0l, t1 = (int)t1l;    // token indices fit 31 bits
     stage_table(table, p.qd + (int64_t)r * n, n);
-    for (int i = tid; i < 4096; i += kKlowThreads) sh[i] = 0u;
+    if (!kBracket)
+      for (int i = tid; i < 4096; i += kKlowThreads) sh[i] = 0u;
     __syncthreads();
     const int64_t head = (int64_t)b * p.Hkv + kvh;
     const uint32_t* plane = p.k_lo + head * kLoPlanes * p.cap;
     const uint32_t* rec = p.k_full + head * p.cap * kAtoms;
     uint32_t* keys = p.keys + (int64_t)r * p.L;
+    sdk_select_state* st = p.st + r;
+    uint32_t lo = 0u, hi = 0u;
+    if (kBracket) {
+      lo = __ldcg(&st->bracket_lo);
+      hi = __ldcg(&st->bracket_hi);
+    }
+    int32_t* above_out = p.list + (int64_t)r * p.L;
+    int32_t* cand_t = p.cand_t + (int64_t)r * p.L;
+    uint32_t* cand_k = p.cand_key + (int64_t)r * p.L;
     // quads of 4 tokens [4q, 4q+4); the segment's edge quads are masked
     const int q0 = t0 >> 2, q1 = (t1 + 3) >> 2;
     auto load_quad = [&](int q, uint32_t (&w)[kLoPlanes][4]) {
@@ -370,10 +380,12 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
       }
     };
     uint32_t wc[kLoPlanes][4], wn[kLoPlanes][4];
-    int q = q0 + tid;
-    load_quad(q, wc);
-    prefetch(q + kKlowThreads);
-    for (; q < q1; q += kKlowThreads) {
+    load_quad(q0 + tid, wc);
+    prefetch(q0 + tid + kKlowThreads);
+    // every thread takes the same number of iterations (warp-wide slot
+    // assignment below); quads past q1 hold no tokens
+    for (int qb = q0; qb < q1; qb += kKlowThreads) {
+      const int q = qb + tid;
       load_quad(q + kKlowThreads, wn);
       prefetch(q + 2 * kKlowThreads);
       uint32_t kq[4];
@@ -395,18 +407,69 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
         }
         kq[u] = score_key(s);
       }
-      // keys: one 16-byte store per whole quad (rows are 16-byte aligned)
-      if (4 * q >= t0 && 4 * q + 4 <= t1) {
-        *reinterpret_cast<uint4*>(keys + 4 * q) = make_uint4(kq[0], kq[1], kq[2], kq[3]);
+      if (store_keys) {
+        // keys: one 16-byte store per whole quad (rows are 16-byte aligned)
+        if (4 * q >= t0 && 4 * q + 4 <= t1) {
+          *reinterpret_cast<uint4*>(keys + 4 * q) = make_uint4(kq[0], kq[1], kq[2], kq[3]);
+          if (!kBracket) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) atomicAdd(&sh[kq[u] >> 20], 1u);
-      } else if (q < q1) {
+            for (int u = 0; u < 4; ++u) atomicAdd(&sh[kq[u] >> 20], 1u);
+          }
+        } else if (q < q1) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int t = 4 * q + u;
+            if (t >= t0 && t < t1) {
+              keys[t] = kq[u];
+              if (!kBracket) atomicAdd(&sh[kq[u] >> 20], 1u);
+            }
+          }
+        }
+      }
+      if (kBracket) {
+        // classify; the warp's slots of each kind come from one atomic
+        unsigned fa = 0u, fc = 0u;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int t = 4 * q + u;
-          if (t >= t0 && t < t1) {
-            keys[t] = kq[u];
-            atomicAdd(&sh[kq[u] >> 20], 1u);
+          const bool valid = t >= t0 && t < t1;
+          const bool a = valid && kq[u] > hi;
+          const bool c = valid && !a && kq[u] >= lo;
+          fa |= (unsigned)a << u;
+          fc |= (unsigned)c << u;
+        }
+        const uint32_t mine = (uint32_t)__popc(fa) | ((uint32_t)__popc(fc) << 16);
+        uint32_t incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+        if (tot != 0u) {
+          uint32_t ba = 0u, bc = 0u;
+          if (lane == 31) {
+            if (tot & 0xFFFFu) ba = atomicAdd(&st->n_above, tot & 0xFFFFu);
+            if (tot >> 16) bc = atomicAdd(&st->n_cand, tot >> 16);
+          }
+          ba = __shfl_sync(0xffffffffu, ba, 31);
+          bc = __shfl_sync(0xffffffffu, bc, 31);
+          const uint32_t ex = incl - mine;
+          uint32_t pa = ba + (ex & 0xFFFFu), pc = bc + (ex >> 16);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int t = 4 * q + u;
+            if ((fa >> u) & 1u) {
+              if (pa < (uint32_t)p.L) above_out[pa] = t;
+              ++pa;
+            }
+            if ((fc >> u) & 1u) {
+              if (pc < (uint32_t)p.L) {
+                cand_t[pc] = t;
+                cand_k[pc] = kq[u];
+              }
+              ++pc;
+            }
           }
         }
       }
@@ -416,10 +479,12 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
         for (int u = 0; u < 4; ++u) wc[j][u] = wn[j][u];
     }
     __syncthreads();
-    uint32_t* gh = p.hist1 + (int64_t)r * 4096;
-    for (int i = tid; i < 4096; i += kKlowThreads)
-      if (sh[i]) atomicAdd(&gh[i], sh[i]);
-    __syncthreads();
+    if (!kBracket) {
+      uint32_t* gh = p.hist1 + (int64_t)r * 4096;
+      for (int i = tid; i < 4096; i += kKlowThreads)
+        if (sh[i]) atomicAdd(&gh[i], sh[i]);
+      __syncthreads();
+    }
   });
   if (maxidx >= (uint32_t)n) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, maxidx);
 }
@@ -615,6 +680,313 @@ __global__ void __launch_bounds__(kScanThreads) final_kernel(DecodeParams p) {
   __shared__ uint32_t s_cnt[2];
   extern __shared__ uint32_t s_cand[];   // 2 * kFinalStage words
   final_head(p, blockIdx.x, s_cand, s_tmp, sh, s_cnt);
+}
+
+// ------------------------------------------ sampled-bracket selection
+// The exact top k per query head without a second pass over the keys:
+//   sample_kernel  scores a sample of the head's tokens (one token per
+//                  block of blk = ceil(N / 8192) consecutive tokens, at
+//                  offset lowbias32(seed ^ block) mod the block's length,
+//                  seed = lowbias32(0x9E3779B9 * (b * Hkv + kvh + 1)); every
+//                  token when N <= 8192) with exactly the Klow scan's
+//                  arithmetic, and brackets the k-th key by two order
+//                  statistics of the sample, 6 standard deviations of the
+//                  sample rank on either side of the expected rank S k / N
+//                  (the whole population when N <= 8192: lo = hi = the k-th
+//                  key itself);
+//   klow_kernel<1> selects key > hi and collects lo <= key <= hi;
+//   select_kernel  finds the exact k-th key among the candidates when
+//                  n_above < k <= n_above + n_cand (ties: lower token), and
+//                  otherwise (the bracket missed, probability about 1e-9
+//                  per head for a representative sample) re-scores the
+//                  whole head and selects by radix histograms.
+// The result is the same set as the radix path in every case.
+constexpr int kSampleMax = 8192;
+constexpr int kSampleThreads = 1024;
+constexpr double kBracketSigmas = 6.0;
+
+// The rank-th largest (1-based) of n keys, by radix select over key digits
+// 31..21, 20..10, 9..0.  Also returns the number of keys equal to the
+// result (cnt) and the rank of the result among them (rank_in_ties:
+// rank - the number of larger keys).  keys: shared or global memory
+// (written before a __syncthreads of this block or by an earlier kernel);
+// hist: 2048 words of shared memory.
+__device__ uint32_t rank_desc(const uint32_t* keys, int n, uint32_t rank, uint32_t* hist,
+                              uint32_t* s_tmp, uint32_t& cnt, uint32_t& rank_in_ties, bool& bad) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  uint32_t prefix = 0u;
+  cnt = 0u;
+  for (int ps = 0; ps < 3; ++ps) {
+    const int shf = ps == 0 ? 21 : (ps == 1 ? 10 : 0);
+    const int wb = ps == 2 ? 10 : 11;
+    const uint32_t mask = (1u << wb) - 1u;
+    for (int i = tid; i < 2048; i += nt) hist[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < n; i += nt) {
+      const uint32_t key = keys[i];
+      if (ps == 0 || (key >> (shf + wb)) == prefix) atomicAdd(&hist[(key >> shf) & mask], 1u);
+    }
+    __syncthreads();
+    uint32_t bin, above;
+    block_find_desc<2048>(hist, rank, s_tmp, bin, above, cnt, bad);
+    if (bad) return 0u;
+    prefix = (prefix << wb) | bin;
+    rank -= above;
+  }
+  rank_in_ties = rank;
+  return prefix;
+}
+
+// The rank-th smallest token index (1-based) among tokens 0..n-1 whose key
+// equals T (tie_cut for keys indexed by token).  sh: 2048 words.
+__device__ uint32_t tie_cut_tokens(const uint32_t* keys, int n, uint32_t T, uint32_t rank,
+                                   uint32_t* s_tmp, uint32_t* sh, bool& bad) {
+  const int tid = threadIdx.x;
+  uint32_t prefix = 0u;
+  bad = false;
+  for (int ps = 0; ps < 3; ++ps) {
+    const int sh_lo = ps == 0 ? 21 : (ps == 1 ? 10 : 0);
+    const int wbits = ps == 2 ? 10 : 11;
+    const uint32_t nb = 1u << wbits;
+    for (int i = tid; i < 2048; i += blockDim.x) sh[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < n; i += blockDim.x) {
+      if (keys[i] != T) continue;
+      const uint32_t t = (uint32_t)i;
+      const uint32_t hi = (ps == 0) ? 0u : (t >> (sh_lo + wbits));
+      if (hi != prefix) continue;
+      atomicAdd(&sh[2047u - ((t >> sh_lo) & (nb - 1u))], 1u);
+    }
+    __syncthreads();
+    uint32_t bin, above, cnt;
+    block_find_desc<2048>(sh, rank, s_tmp, bin, above, cnt, bad);
+    if (bad) return 0u;
+    prefix = (prefix << wbits) | (2047u - bin);
+    rank -= above;
+  }
+  return prefix;
+}
+
+// s_lo of token t of a head exactly as klow_kernel computes it (the same
+// words, table values and FMA order; an index >= n reads 0).
+__device__ __forceinline__ float klow_score_at(const uint32_t* plane, int64_t cap,
+                                               const uint32_t* rec, int t, int klow, int nlo,
+                                               const float* tab, int n, bool global_tab) {
+  uint32_t w[kLoPlanes];
+#pragma unroll
+  for (int j = 0; j < kLoPlanes; ++j) w[j] = j < nlo ? __ldg(plane + j * cap + t) : 0u;
+  float s = 0.0f;
+#pragma unroll
+  for (int j = 0; j < kLoPlanes; ++j) {
+    const uint32_t idx = word_idx(w[j]);
+    const float v = global_tab ? (idx < (uint32_t)n ? __ldg(tab + idx) : 0.0f) : tab[idx];
+    s = fmaf(word_coef(w[j]), v, s);
+  }
+  for (int j = kLoPlanes; j < klow; ++j) {
+    const uint32_t wj = __ldg(rec + (int64_t)t * kAtoms + j);
+    const uint32_t idx = word_idx(wj);
+    const float v = global_tab ? (idx < (uint32_t)n ? __ldg(tab + idx) : 0.0f) : tab[idx];
+    s = fmaf(word_coef(wj), v, s);
+  }
+  return s;
+}
+
+// One CTA per query head: the sample, its keys and the bracket [lo, hi].
+__global__ void __launch_bounds__(kSampleThreads) sample_kernel(DecodeParams p) {
+  pdl_wait();
+  pdl_launch();
+  __shared__ uint32_t s_key[kSampleMax];
+  __shared__ uint32_t s_hist[2048];
+  __shared__ uint32_t s_tmp[48];
+  const int r = blockIdx.x, tid = threadIdx.x;
+  const int b = r / p.Hq, h = r % p.Hq, kvh = h / p.g;
+  const int N = p.lens[b], k = p.kcnt[b];
+  const int blk = N <= kSampleMax ? 1 : (N + kSampleMax - 1) / kSampleMax;
+  const int S = (N + blk - 1) / blk;
+  const int64_t head = (int64_t)b * p.Hkv + kvh;
+  const uint32_t* plane = p.k_lo + head * kLoPlanes * p.cap;
+  const uint32_t* rec = p.k_full + head * p.cap * kAtoms;
+  const float* qd = p.qd + (int64_t)r * p.n;
+  const uint32_t seed = lowbias32(0x9E3779B9u * (uint32_t)(head + 1));
+  const int nlo = min(p.klow, kLoPlanes);
+  // up to 8 samples per thread; all their word loads are issued first
+  constexpr int kPer = kSampleMax / kSampleThreads;
+  int tt[kPer];
+  uint32_t wv[kPer][kLoPlanes];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int i = tid + u * kSampleThreads;
+    tt[u] = -1;
+    if (i < S) {
+      const int len = min(blk, N - i * blk);
+      tt[u] = i * blk + (blk == 1 ? 0 : (int)(lowbias32(seed ^ (uint32_t)i) % (uint32_t)len));
+    }
+#pragma unroll
+    for (int j = 0; j < kLoPlanes; ++j)
+      wv[u][j] = (tt[u] >= 0 && j < nlo) ? __ldg(plane + j * p.cap + tt[u]) : 0u;
+  }
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    if (tt[u] < 0) continue;
+    float s = 0.0f;
+#pragma unroll
+    for (int j = 0; j < kLoPlanes; ++j) {
+      const uint32_t idx = word_idx(wv[u][j]);
+      s = fmaf(word_coef(wv[u][j]), idx < (uint32_t)p.n ? __ldg(qd + idx) : 0.0f, s);
+    }
+    for (int j = kLoPlanes; j < p.klow; ++j) {
+      const uint32_t wj = __ldg(rec + (int64_t)tt[u] * kAtoms + j);
+      const uint32_t idx = word_idx(wj);
+      s = fmaf(word_coef(wj), idx < (uint32_t)p.n ? __ldg(qd + idx) : 0.0f, s);
+    }
+    s_key[tid + u * kSampleThreads] = score_key(s);
+  }
+  __syncthreads();
+  // sample ranks of the bracket (1-based, descending); 0 = no upper end
+  // (nothing is selected directly), S + 1 = no lower end (every token not
+  // above hi is a candidate)
+  int rhi, rlo;
+  if (S == N) {
+    rhi = rlo = k;
+  } else if (k >= N) {
+    rhi = 0;
+    rlo = S + 1;
+  } else {
+    const double pp = (double)k / (double)N;
+    const double mu = (double)S * pp, sg = sqrt((double)S * pp * (1.0 - pp));
+    const double a = floor(mu - kBracketSigmas * sg), c = ceil(mu + kBracketSigmas * sg);
+    rhi = a < 1.0 ? 0 : (int)a;
+    rlo = c > (double)S ? S + 1 : (int)c;
+  }
+  uint32_t hi = 0xFFFFFFFFu, lo = 0u, cnt, rit;
+  bool bad = false;
+  if (rhi >= 1) hi = rank_desc(s_key, S, (uint32_t)rhi, s_hist, s_tmp, cnt, rit, bad);
+  if (!bad && rlo <= S) lo = rank_desc(s_key, S, (uint32_t)rlo, s_hist, s_tmp, cnt, rit, bad);
+  if (tid == 0) {
+    if (bad) {           // cannot happen for 1 <= rank <= S; select_kernel re-scans
+      hi = 0u;
+      lo = 0xFFFFFFFFu;
+      record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x28000000u | r);
+    }
+    sdk_select_state* st = p.st + r;
+    st->bracket_lo = lo;
+    st->bracket_hi = hi;
+    st->select_path = 1u;
+  }
+}
+
+constexpr int kSelThreads = 1024;
+constexpr int kSelStage = kTable / 2;      // staged candidates: keys + tokens = 128 KB
+constexpr int kSelSmem = kTable * 4;       // the same bytes hold the fallback's QD table
+
+// Appends the tokens selected by (key > T, or key == T and token <= t_cut)
+// among n entries (key_at(i), tok_at(i)) to list at slots from s_cnt[0].
+template <class KeyAt, class TokAt>
+__device__ __forceinline__ void append_selected(int n, uint32_t T, uint32_t t_cut, KeyAt key_at,
+                                                TokAt tok_at, int32_t* list, uint32_t k,
+                                                uint32_t* s_cnt, WsHeader* hdr, int r) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int i0 = tid - lane; i0 < n; i0 += kSelThreads) {
+    const int i = i0 + lane;
+    bool sel = false;
+    uint32_t t = 0u;
+    if (i < n) {
+      const uint32_t key = key_at(i);
+      t = tok_at(i);
+      sel = key > T || (key == T && t <= t_cut);
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, sel);
+    uint32_t base = 0u;
+    if (lane == 0 && m) base = atomicAdd(&s_cnt[0], (uint32_t)__popc(m));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    if (sel) {
+      const uint32_t pos = base + (uint32_t)__popc(m & lt);
+      if (pos < k) list[pos] = (int32_t)t;
+      else record_error(hdr, SDK_ERR_DEVICE_CHECK, 0x26000000u | r);
+    }
+  }
+}
+
+// One CTA per query head: the rest of the selected set (bracket path), or
+// the whole selection by an exact re-scan when the bracket missed.
+__global__ void __launch_bounds__(kSelThreads, 1) select_kernel(DecodeParams p) {
+  pdl_wait();
+  pdl_launch();
+  extern __shared__ float4 smem4[];
+  __shared__ uint32_t sh[2048];
+  __shared__ uint32_t s_tmp[48];
+  __shared__ uint32_t s_cnt[2];
+  const int r = blockIdx.x, tid = threadIdx.x;
+  const int b = r / p.Hq, h = r % p.Hq, kvh = h / p.g;
+  const int N = p.lens[b];
+  const uint32_t k = (uint32_t)p.kcnt[b];
+  sdk_select_state* st = p.st + r;
+  const uint32_t A = __ldcg(&st->n_above), C = __ldcg(&st->n_cand);
+  int32_t* list = p.list + (int64_t)r * p.L;
+  uint32_t T = 0u, eq_total = 0u, eq_take = 0u, t_cut = 0xFFFFFFFFu;
+  bool bad = false;
+  const bool hit = A < k && (uint64_t)A + C >= k && A + C <= (uint32_t)N;
+  if (hit) {
+    // the (k - A)-th largest candidate, staged in shared memory when the
+    // candidates fit (otherwise read through L2)
+    const uint32_t* ck = p.cand_key + (int64_t)r * p.L;
+    const int32_t* ct = p.cand_t + (int64_t)r * p.L;
+    if (C <= (uint32_t)kSelStage) {
+      uint32_t* s_ck = reinterpret_cast<uint32_t*>(smem4);
+      int32_t* s_ct = reinterpret_cast<int32_t*>(s_ck + kSelStage);
+      for (uint32_t i = tid; i < C; i += kSelThreads) {
+        s_ck[i] = __ldcg(ck + i);
+        s_ct[i] = __ldcg(ct + i);
+      }
+      __syncthreads();
+      ck = s_ck;
+      ct = s_ct;
+    }
+    const uint32_t k1 = k - A;
+    T = rank_desc(ck, (int)C, k1, sh, s_tmp, eq_total, eq_take, bad);
+    if (!bad && eq_total > eq_take) t_cut = tie_cut(ck, ct, C, T, eq_take, s_tmp, sh, bad);
+    if (bad) {
+      if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x29000000u | r);
+      return;
+    }
+    if (tid == 0) s_cnt[0] = A;
+    __syncthreads();
+    append_selected((int)C, T, t_cut, [&](int i) { return ck[i]; },
+                    [&](int i) { return (uint32_t)ct[i]; }, list, k, s_cnt, p.hdr, r);
+  } else {
+    // exact re-scan: every token's key into `keys`, then the radix select
+    float* table = reinterpret_cast<float*>(smem4);
+    stage_table(table, p.qd + (int64_t)r * p.n, p.n);
+    __syncthreads();
+    const int64_t head = (int64_t)b * p.Hkv + kvh;
+    const uint32_t* plane = p.k_lo + head * kLoPlanes * p.cap;
+    const uint32_t* rec = p.k_full + head * p.cap * kAtoms;
+    uint32_t* keys = p.keys + (int64_t)r * p.L;
+    const int nlo = min(p.klow, kLoPlanes);
+    for (int t = tid; t < N; t += kSelThreads)
+      keys[t] = score_key(klow_score_at(plane, p.cap, rec, t, p.klow, nlo, table, p.n, false));
+    __syncthreads();
+    T = rank_desc(keys, N, k, sh, s_tmp, eq_total, eq_take, bad);
+    if (!bad && eq_total > eq_take) t_cut = tie_cut_tokens(keys, N, T, eq_take, s_tmp, sh, bad);
+    if (bad) {
+      if (tid == 0) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x2A000000u | r);
+      return;
+    }
+    if (tid == 0) s_cnt[0] = 0u;
+    __syncthreads();
+    append_selected(N, T, t_cut, [&](int i) { return keys[i]; },
+                    [&](int i) { return (uint32_t)i; }, list, k, s_cnt, p.hdr, r);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    st->kth_key = T;
+    st->eq_total = eq_total;
+    st->eq_taken = eq_take;
+    st->n_sel = s_cnt[0];
+    st->select_path = hit ? 1u : 2u;
+    if (s_cnt[0] != k) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, 0x24000000u | r);
+  }
 }
 
 // ------------------------------------------- context-sharded final stages
@@ -1813,8 +2185,11 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
   const int sms = num_sms();
   static unsigned long long attr_set = 0ull;
   if (device_needs_setup(&attr_set)) {
-    cudaFuncSetAttribute(klow_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(klow_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kTable * 4 + 4096 * 4);
+    cudaFuncSetAttribute(klow_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kTable * 4 + 4096 * 4);
+    cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelSmem);
     cudaFuncSetAttribute(pass2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPass2Smem);
     cudaFuncSetAttribute(final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          2 * kFinalStage * 4);
@@ -1867,20 +2242,31 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
   {
     const int g = scan_grid(p.tok_off[p.B], p.R, kKlowSegCost, 2048, sms);
     const int vec = (p.cap % 4 == 0) && ((reinterpret_cast<uintptr_t>(p.k_lo) & 15u) == 0u);
-    e = launch_pdl(klow_kernel, dim3(g), dim3(kKlowThreads), (size_t)kTable * 4 + 4096 * 4, stream,
-                   1, p, vec);
+    if (p.bracket) {
+      e = launch_pdl(sample_kernel, dim3(p.R), dim3(kSampleThreads), 0, stream, 1, p);
+      if (e != cudaSuccess) return SDK_ERR_CUDA;
+      e = launch_pdl(klow_kernel<true>, dim3(g), dim3(kKlowThreads), (size_t)kTable * 4 + 4096 * 4,
+                     stream, 1, p, vec);
+    } else {
+      e = launch_pdl(klow_kernel<false>, dim3(g), dim3(kKlowThreads), (size_t)kTable * 4 + 4096 * 4,
+                     stream, 1, p, vec);
+    }
     if (e != cudaSuccess) return SDK_ERR_CUDA;
   }
   return SDK_OK;
   }
-  case 1: {   // pass 2 of the selection
+  case 1: {   // pass 2 of the selection (radix path only)
+    if (p.bracket) return SDK_OK;
     const int g = scan_grid(p.tok_off[p.B], p.R, kPass2SegCost, 8192, sms);
     e = launch_pdl(pass2_kernel, dim3(g), dim3(kP2Threads), (size_t)kPass2Smem, stream, 1, p);
     return e == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
   }
   case 2:     // the final selection (whole context)
-    e = launch_pdl(final_kernel, dim3(p.R), dim3(kScanThreads), (size_t)2 * kFinalStage * 4, stream,
-                   1, p);
+    if (p.bracket)
+      e = launch_pdl(select_kernel, dim3(p.R), dim3(kSelThreads), (size_t)kSelSmem, stream, 1, p);
+    else
+      e = launch_pdl(final_kernel, dim3(p.R), dim3(kScanThreads), (size_t)2 * kFinalStage * 4,
+                     stream, 1, p);
     return e == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
   case 3: {   // attend
   {

@@ -30,20 +30,58 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
+// Per device: the id of the context the address was looked up in, and the
+// address.  A __device__ array lives in the module loaded into one
+// context; after cudaDeviceReset (or anything else that destroys the
+// primary context) the module is loaded again, possibly at another
+// address, so the address is looked up again whenever the current
+// context's id differs (context ids are unique within a process; a
+// context handle may be reused).
+unsigned long long g_ws_ctx[kMaxDevices] = {};
 void* g_ws_ptr[kMaxDevices] = {};
 
-// Address of the array on the current device, looked up on the first call
-// for that device (that lookup loads the module if it is not loaded yet).
+// cuCtxGetCurrent and cuCtxGetId through the runtime's driver entry points
+// (null when the driver does not offer them).
+using CtxGetCurrentFn = int (*)(void**);
+using CtxGetIdFn = int (*)(void*, unsigned long long*);
+template <class Fn>
+Fn driver_fn(const char* name) {
+  void* ptr = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion(name, &ptr, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(ptr);
+}
+
+// Id of the calling thread's current context (0 if none or unknown).
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_ctx = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  void* ctx = nullptr;
+  unsigned long long id = 0ull;
+  if (get_ctx == nullptr || get_id == nullptr || get_ctx(&ctx) != 0 || ctx == nullptr) return 0ull;
+  if (get_id(ctx, &id) != 0) return 0ull;
+  return id;
+}
+
+// Address of the array in the current device's current context, looked up
+// on the first call in that context (the lookup loads the module if it is
+// not loaded yet, and makes the device's primary context current).
 sdk_status static_workspace(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SDK_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return SDK_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (g_ws_ptr[dev] == nullptr) {
+  unsigned long long id = current_ctx_id();
+  if (id == 0ull || g_ws_ptr[dev] == nullptr || g_ws_ctx[dev] != id) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress((void**)&ptr, g_decode_static_ws) != cudaSuccess || ptr == nullptr)
       return SDK_ERR_CUDA;
+    if (id == 0ull) id = current_ctx_id();
+    if (id == 0ull) return SDK_ERR_CUDA;
     g_ws_ptr[dev] = ptr;
+    g_ws_ctx[dev] = id;
   }
   *out = g_ws_ptr[dev];
   return SDK_OK;

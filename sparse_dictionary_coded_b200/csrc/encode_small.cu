@@ -94,6 +94,7 @@ struct SmallParams {
   int lens[32];
   WsHeader* hdr;
   unsigned long long* words;   // [2][grid][64], zero before the launch
+  unsigned long long wait_ns;  // limit of every poll for another CTA's word
 };
 
 // Word of a slice winner: bits 63..32 |c| (fp32 bits), 31..17 0x7fff - index,
@@ -123,11 +124,12 @@ __device__ __forceinline__ ulonglong2 ld_relaxed_v2(const unsigned long long* p)
 
 // Maximum over the words of one slot pair from CTAs c0, c0 + cstep, ...:
 // all loads issued at once, each word polled until it carries `tag`
-// (bounded by 1 s and the CTA's abort flag).  False on timeout.
+// (bounded by limit_ns and the CTA's abort flag).  False on timeout.
 template <int B>
 __device__ __forceinline__ bool gather_words(const unsigned long long* wb, int c0, int cstep, int G,
                                              int vr, bool v1, uint32_t tag,
-                                             volatile uint32_t* abort_flag, unsigned long long& mx0,
+                                             volatile uint32_t* abort_flag,
+                                             unsigned long long limit_ns, unsigned long long& mx0,
                                              unsigned long long& mx1) {
   for (int cb = c0; cb < G; cb += cstep * B) {
     ulonglong2 w[B];
@@ -146,7 +148,7 @@ __device__ __forceinline__ bool gather_words(const unsigned long long* wb, int c
         while (true) {
           x = ld_relaxed_v2(wb + (size_t)c * 64 + vr);
           if (word_tag(x.x) == tag && (!v1 || word_tag(x.y) == tag)) break;
-          if (*abort_flag || tc::globaltimer() - t0 > tc::kWaitNs) return false;
+          if (*abort_flag || tc::globaltimer() - t0 > limit_ns) return false;
           __nanosleep(20);
         }
       }
@@ -494,9 +496,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c0 = tid >> lg_np;
         unsigned long long mx0 = 0ull, mx1 = 0ull;
         if (cstep * 4 >= G)
-          ok = gather_words<4>(wb, c0, cstep, G, vr, v1, tag, s_abort, mx0, mx1);
+          ok = gather_words<4>(wb, c0, cstep, G, vr, v1, tag, s_abort, p.wait_ns, mx0, mx1);
         else
-          ok = gather_words<kBatch>(wb, c0, cstep, G, vr, v1, tag, s_abort, mx0, mx1);
+          ok = gather_words<kBatch>(wb, c0, cstep, G, vr, v1, tag, s_abort, p.wait_ns, mx0,
+                                    mx1);
         if (mx0) atomicMax(&s_best[vr], mx0);
         if (mx1) atomicMax(&s_best[vr + 1], mx1);
       }
@@ -673,6 +676,7 @@ sdk_status launch_encode_small(const SmallEncode& e, void* scratch, size_t scrat
   for (int b = 0; e.append && b < e.B; ++b) sp.lens[b] = e.lens[b];
   sp.hdr = e.p[0].hdr;
   sp.words = reinterpret_cast<unsigned long long*>(scratch);
+  sp.wait_ns = exchange_wait_ns();
   if (cudaMemsetAsync(sp.words, 0, (size_t)2 * grid * kSlots * 8, stream) != cudaSuccess)
     return SDK_ERR_CUDA;
   *taken = true;

@@ -140,23 +140,16 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const int t = tid - 32;
     const int64_t nthr = (int64_t)gridDim.x * gridDim.y * kT;
     const int64_t g0 = ((int64_t)blockIdx.y * gridDim.x + blockIdx.x) * kT + t;
-    const int64_t hquads = (int64_t)R * 1024;   // both histograms, 16-byte stores
+    // both histograms, 16-byte stores (the radix selection path only)
+    const int64_t hquads = p.bracket ? 0 : (int64_t)R * 1024;
     for (int64_t e = g0; e < hquads; e += nthr) {
       reinterpret_cast<uint4*>(p.hist1)[e] = make_uint4(0u, 0u, 0u, 0u);
       reinterpret_cast<uint4*>(p.hist2)[e] = make_uint4(0u, 0u, 0u, 0u);
     }
     for (int64_t e = g0; e < (int64_t)R * D; e += nthr) p.out[e] = 0.0f;
     for (int64_t e = g0; e < (int64_t)R; e += nthr) {
-      sdk_select_state st;
-      st.kth_key = 0u;
+      sdk_select_state st = {};
       st.k = (uint32_t)p.kcnt[e / p.Hq];
-      st.n_above = st.n_cand = st.n_sel = st.n_comp = 0u;
-      st.eq_total = st.eq_taken = 0u;
-      st.max_score = 0u;
-      st.max_comp = 0u;
-      st.z = 0.0f;
-      st.isoft_sum[0] = st.isoft_sum[1] = st.isoft_shift = 0u;
-      st.pad[0] = st.pad[1] = 0u;
       p.st[e] = st;
     }
     // B operands: the three bf16 parts of the tile's query rows in the

@@ -59,6 +59,18 @@ __device__ __forceinline__ float key_score(uint32_t k) {
   return __uint_as_float(b);
 }
 
+// Chris Wellons' "lowbias32" integer hash (from his 2018 search for 32-bit
+// hash functions with low bias): picks the sampled token of each block in
+// the sampled-bracket selection.
+__host__ __device__ __forceinline__ uint32_t lowbias32(uint32_t x) {
+  x ^= x >> 16;
+  x *= 0x7feb352dU;
+  x ^= x >> 15;
+  x *= 0x846ca68bU;
+  x ^= x >> 16;
+  return x;
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t v) {
   return __uint_as_float(v << 16);
 }
@@ -183,6 +195,10 @@ struct DecodeParams {
   int64_t cap;
   int64_t L;
   int B, Hq, Hkv, g, d, n, klow, khigh, full, isoft, R, n_out_tiles;
+  // selection by a sampled bracket of the k-th key (sample_kernel,
+  // klow_kernel<1>, select_kernel) instead of radix histograms; keep_keys:
+  // the Klow scan also stores every token's key (SDK_DECODE_KEEP_KEYS)
+  int bracket, keep_keys;
   // context-sharded decode: 0 = whole decode; 1 / 2 = attend's first /
   // second half (shard_in: the gathered softmax statistics); world ranks
   int att_mode, world;
@@ -210,6 +226,11 @@ struct EncodeParams {
 };
 
 int num_sms();  // cached multiprocessor count of the current device
+
+// Limit of the waits for other CTAs' results (sdk_set_exchange_timeout_ns;
+// 1 s by default); set_exchange_wait_ns returns the previous limit.
+unsigned long long exchange_wait_ns();
+unsigned long long set_exchange_wait_ns(unsigned long long ns);
 
 // Kernel attributes (the dynamic shared-memory limits) are set per device:
 // device_needs_setup tells whether the current device's bit in `flags` is

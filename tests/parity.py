@@ -34,9 +34,11 @@ def words_np(t):
     return t.detach().cpu().numpy().view(np.uint32)
 
 
-def check_encode(words_gpu, ref, coef_tol=COEF_TOL, gap_tol=GAP_TOL):
+def check_encode(words_gpu, ref, coef_tol=COEF_TOL, gap_tol=GAP_TOL,
+                 stopped=None):
     """Returns (steps_compared, vectors_that_diverged_at_a_near_tie).
-    Raises AssertionError on a violation."""
+    Raises AssertionError on a violation.  `stopped`, if a list, receives
+    the vectors whose walk ended early (a near tie or the residual floor)."""
     idx_g, coef_g = oracle.unpack_words(words_gpu)
     m, k = idx_g.shape
     compared = 0
@@ -45,6 +47,8 @@ def check_encode(words_gpu, ref, coef_tol=COEF_TOL, gap_tol=GAP_TOL):
         for j in range(k):
             if ref["rnorm"][v, j] <= RESID_FLOOR * ref["xnorm"][v]:
                 assert np.all(np.abs(coef_g[v, j:]) <= 1e-4 * ref["xnorm"][v])
+                if stopped is not None:
+                    stopped.append(v)
                 break
             if idx_g[v, j] != ref["idx"][v, j]:
                 assert ref["gap"][v, j] <= gap_tol, (
@@ -52,6 +56,8 @@ def check_encode(words_gpu, ref, coef_tol=COEF_TOL, gap_tol=GAP_TOL):
                     "gap %.3g" % (v, j, idx_g[v, j], ref["idx"][v, j],
                                   ref["gap"][v, j]))
                 diverged += 1
+                if stopped is not None:
+                    stopped.append(v)
                 break
             c_or = ref["coef"][v, j]
             err = abs(coef_g[v, j] - c_or)

@@ -74,11 +74,13 @@ def test_reference_arm_line(monkeypatch):
     monkeypatch.setenv("RANK", "0")
     calls = []
 
-    def fake(name, budget_s=15.0):
-        calls.append(budget_s)
-        return {"value": 100.0 + len(calls), "unit": "encoded KV vecs/s",
-                "cores": 4, "kind": "oracle", "sample": "s"}
-    monkeypatch.setattr(bench, "cpu_baseline", fake)
+    def fake_sampler(name):
+        def run(budget_s):
+            calls.append(budget_s)
+            return {"value": 100.0 + len(calls), "unit": bench.ENCODE_UNIT,
+                    "cores": 4, "kind": "oracle", "sample": "s"}
+        return run
+    monkeypatch.setattr(bench, "oracle_sampler", fake_sampler)
     args = type("A", (), dict(workload="layer4k", steps=2, warmup=3,
                               gpus=1))()
     buf = io.StringIO()
@@ -93,6 +95,34 @@ def test_reference_arm_line(monkeypatch):
     assert j["e2e"]["h2d_bytes_per_step"] == 0
     assert j["cpu_baseline"]["kind"] == "oracle"
     assert j["metric"] == bench.METRIC
+    # the same unit and config as the sdk arm prints for this workload
+    assert j["unit"] == bench.ENCODE_UNIT
+    assert j["config"] == bench.workload_config("layer4k", args)
+
+
+def test_reference_arm_default_line_carries_prefill(monkeypatch):
+    """The default workload's reference line has the decode unit and
+    config and a prefill-encode sub-record in the encode unit."""
+    import json
+    monkeypatch.setenv("RANK", "0")
+
+    def fake_sampler(name):
+        unit = bench.DECODE_UNIT if name == "decode256k" else bench.ENCODE_UNIT
+        return lambda budget_s: {"value": 7.0, "unit": unit, "cores": 4,
+                                 "kind": "oracle", "sample": "s"}
+    monkeypatch.setattr(bench, "oracle_sampler", fake_sampler)
+    args = type("A", (), dict(workload="decode256k", steps=2, warmup=1, gpus=1,
+                              no_prefill=False, full_softmax=False,
+                              int_softmax=False, context_shard=False,
+                              layers=None))()
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        bench.reference_arm(args)
+    j = json.loads(buf.getvalue().strip())
+    assert j["unit"] == bench.DECODE_UNIT and j["config"]["workload"] == "decode256k"
+    assert j["config"] == bench.workload_config("decode256k", args)
+    assert j["prefill_encode"]["unit"] == bench.ENCODE_UNIT
+    assert j["prefill_encode"]["config"]["workload"] == "prefill256k_vec"
 
 
 def test_clock_parsing():
@@ -101,12 +131,20 @@ def test_clock_parsing():
     c = bench.Clocks(0)
     c.proc = type("P", (), dict(terminate=lambda s: None,
                                 wait=lambda s, timeout=None: 0))()
-    c.lines = [
+    c.lines = [(float(i), ln) for i, ln in enumerate([
         "1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active",
         "1900, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active",
         "1950, 1965, 980.0, 0x4, Not Active, Not Active, Not Active, Active",
         "garbage",
-    ]
+    ])]
     r = c.stop()
     assert r["sm_mhz"] == 1950 and r["sm_max_mhz"] == 1965
     assert r["reasons"] == ["sw_power_cap"] and r["samples"] == 3
+    # only the samples inside the marked timed region count; a region
+    # shorter than the sampling period takes its neighbours
+    c.t0, c.t1 = 0.5, 1.5
+    r = c.stop()
+    assert r["sm_mhz"] == 1900 and r["samples"] == 1
+    c.t0, c.t1 = 1.2, 1.3
+    r = c.stop()
+    assert r["samples"] == 2 and r["sm_mhz"] == 1925

@@ -42,7 +42,7 @@ def test_status_strings(lib):
     for code, name in _capi.STATUS_NAMES.items():
         assert lib.sdk_status_string(code).decode().startswith(name)
     assert lib.sdk_status_string(99) == b"SDK_ERR_UNKNOWN"
-    assert lib.sdk_version() == 1
+    assert lib.sdk_version() == 2
 
 
 def test_workspace_sizes(lib):
@@ -92,7 +92,7 @@ def _decode(lib, **kw):
     (dict(lens=(ctypes.c_int32 * 1)(257)), 1),
     (dict(ws_bytes=1024), 3),                 # workspace too small
     (dict(q=MISALIGNED), 1),                  # q must be 16-byte aligned
-    (dict(full=4), 1),                        # unknown flag bit
+    (dict(full=8), 1),                        # unknown flag bit
 ])
 def test_decode_rejects_bad_arguments(lib, kw, status):
     assert _decode(lib, **kw) == status

@@ -42,12 +42,17 @@ def test_tiny_workload_all_vectors(fn):
     for x, D in ((w["xk"], w["DK"]), (w["xv"], w["DV"])):
         (codes, rsq), _ = _enc(fn, x, D, rsq=True)
         ref = _oracle(x, D)
-        compared, div = check_encode(words_np(codes), ref)
+        stopped = []
+        compared, div = check_encode(words_np(codes), ref, stopped=stopped)
         assert compared >= 0.9 * 256 * 16
-        # residual energy of the GPU encode vs the oracle's final residual
+        # residual energy of the GPU encode vs the oracle's final residual,
+        # for every vector whose walk ran all 16 steps (the others took a
+        # different but equally valid path at a near tie)
         r_or = np.sum(ref["resid"] ** 2, axis=1)
         ok = np.abs(rsq.cpu().double().numpy() - r_or) <= 1e-3 * (r_or + 1e-6)
-        assert ok.mean() >= 0.9
+        full = np.setdiff1d(np.arange(256), stopped)
+        assert full.size >= 0.9 * 256
+        assert ok[full].all(), np.flatnonzero(~ok)[:10]
 
 
 @pytest.mark.parametrize("fn", ENCODERS)
@@ -82,6 +87,37 @@ def test_prefill_sampled_vectors_and_certificate(fn):
                                     D.cpu().float().double().numpy(), ws)
         assert cert["ok_pick"].all()
         assert cert["ok_coef"].all()
+
+
+def _certify_many(x, D, codes, n, seed):
+    """fp64 replay certificate of n sampled vectors' GPU codes: every pick
+    within 1e-4 relative of its step's largest |<r, d>|, every stored
+    coefficient within 1e-3 of the exact projection."""
+    g = workloads.make_gen(seed)
+    sample = torch.randperm(x.shape[0], generator=g)[:n]
+    cert = oracle.certify_codes_batched(x.cpu()[sample].double().numpy(),
+                                        D.cpu().float().double().numpy(),
+                                        words_np(codes.cpu()[sample]))
+    bad = np.argwhere(~(cert["ok_pick"] & cert["ok_coef"]))
+    assert bad.size == 0, (bad[:5], cert["pick_ratio"][tuple(bad[0])] if bad.size else None)
+
+
+def test_certificate_4096_vectors_per_stream():
+    """The tensor-core encoder at full size: 4096 sampled vectors of each
+    stream of the prefill workload (262144 dense Student-t vectors,
+    correlated dictionaries) and 4096 of the layer4k keys, every pick and
+    coefficient certified by the fp64 replay (no oracle path of its own is
+    needed, so paths that diverged at a near tie are checked too)."""
+    w = workloads.prefill(device="cuda")
+    for s, (x, D) in enumerate(((w["xk"], w["DK"]), (w["xv"], w["DV"]))):
+        xf = x.reshape(-1, 128)
+        codes, _ = _enc("sdk_encode", xf, D)
+        _certify_many(xf, D, codes, 4096, 30 + s)
+    del w
+    w = workloads.layer4k()
+    x = w["xk"].reshape(-1, 128)
+    codes, _ = _enc("sdk_encode", x, w["DK"])
+    _certify_many(x, w["DK"], codes, 4096, 32)
 
 
 @pytest.mark.parametrize("fn", ENCODERS)
@@ -351,3 +387,37 @@ def test_small_batch_switch_off_uses_tensor_core_encoder():
                        capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "identical" in r.stdout
+
+
+def test_exchange_wait_runs_out_cleanly():
+    """The small-batch encoder's per-step exchange of slice winners is the
+    one device wait on other CTAs' results.  With its limit at 0 (the
+    first word not there yet gives up) a 16-vector encode records
+    SDK_ERR_TIMEOUT with the exchange's detail code, and the call returns.
+    With the default limit back, the next calls on the same device succeed
+    and their codes equal the CUDA-core encoder's bit for bit (the kernel
+    that gave up left its loop, freed its tensor memory and returned; no
+    copy or MMA was in flight at that wait)."""
+    g = workloads.make_gen(41)
+    D = workloads.gaussian_dictionary(32768, 128, g).cuda()
+    x = torch.randn(16, 128, generator=g).cuda()
+    prev = sdk.sdk_set_exchange_timeout_ns(0)
+    try:
+        seen = None
+        for _ in range(5):
+            ws = sdk.new_workspace(sdk.sdk_encode_workspace_bytes(16, 128, 32768))
+            sdk.sdk_encode(x, D, workspace=ws)
+            rc, hdr = sdk.sdk_check_status(ws)
+            assert rc in (0, 5), rc
+            if rc == 5:
+                seen = hdr
+                break
+        assert seen is not None, "no exchange wait ran out in 5 calls"
+        assert (seen[1] >> 24) == 0x63, hex(seen[1])
+    finally:
+        assert sdk.sdk_set_exchange_timeout_ns(prev) == 0
+    assert prev == 1000000000
+    for _ in range(2):
+        codes, _ = _enc("sdk_encode", x, D)
+        ref, _ = _enc("sdk_encode_simt", x, D)
+        assert torch.equal(codes.cpu(), ref.cpu())

@@ -61,8 +61,11 @@ def _reference(q, DK, DV, store, full=False):
 @pytest.mark.parametrize("full", [False, True])
 def test_layer_of_4096_tokens_twice_in_a_row(full):
     """B=1, 32 query heads over 8 KV heads, 4096 tokens, 32768 atoms, d=128
-    (11.5 MiB of workspace): two consecutive calls both match the call with
-    a caller-owned workspace, and report no device-side failure."""
+    (a decode workspace that fits the fixed array): two consecutive calls
+    both match the call with a caller-owned workspace, and report no
+    device-side failure."""
+    assert sdk.sdk_decode_workspace_bytes(1, 32, 128, 32768, 4096) <= \
+        _capi.DECODE_STATIC_WS_BYTES
     q, DK, DV, kw, vw, _ = _case(71, 1, 32, 8, 4096, 128, 32768)
     store = _store(kw, vw, [4096])
     ref = _reference(q, DK, DV, store, full)
