@@ -122,6 +122,11 @@ def parse():
                          "over the ranks (sdk_decode_attn_shard with NCCL "
                          "exchanges; strong scaling of one context) instead "
                          "of running one independent copy per rank")
+    ap.add_argument("--kv-layout", default="separate",
+                    choices=["separate", "interleaved"],
+                    help="decode workloads: key and value records in two "
+                         "arrays, or interleaved (a token's K and V records "
+                         "in one 128-byte line)")
     ap.add_argument("--no-prefill", action="store_true",
                     help="decode256k: leave out the prefill-encode sub-record")
     ap.add_argument("--no-e2e", action="store_true")
@@ -357,6 +362,7 @@ def workload_config(name, args):
             "n_tokens": W["n_tokens"], "klow": 3, "khigh": 16, "top": "1/10",
             "softmax": ("integer (INT16 logits)" if args.int_softmax else "fp32")
                        + (", all tokens" if args.full_softmax else ", selected set"),
+            "kv_layout": getattr(args, "kv_layout", "separate"),
             "l2": "flushed between steps; codes (%.1f GB) exceed L2"
                   % (L * W["B"] * W["Hkv"] * W["n_tokens"] * 140 / 1e9)}
 
@@ -556,7 +562,8 @@ def bench_decode(args, world, rank, pk, name):
     layers = []
     for l in range(L):
         lay = workloads.decode_layer(name, l + 1000 * rank, device="cuda")
-        k_lo, k_full, v_full = workloads.layout(lay["kwords"], lay["vwords"])
+        k_lo, k_full, v_full = workloads.layout(
+            lay["kwords"], lay["vwords"], interleaved=args.kv_layout == "interleaved")
         del lay["kwords"], lay["vwords"]
         store = sdk.CodeStore.from_tensors(k_lo, k_full, v_full, [N] * B)
         q = (lay["q"] / lay["q"].norm(dim=-1, keepdim=True)).contiguous()

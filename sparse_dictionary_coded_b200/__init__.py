@@ -195,16 +195,23 @@ def sdk_encode_simt(x, dictionary, k_atoms=K_ATOMS, codes=None,
 # ------------------------------------------------------------- code store
 
 class CodeStore:
-    """Device buffers of one layer's code store (layout of include/sdk.h)."""
+    """Device buffers of one layer's code store (layout of include/sdk.h).
+    interleaved: k_full and v_full are views of one [B, Hkv, cap, 2, 16]
+    array, so a token's key and value records form one 128-byte line."""
 
-    def __init__(self, B, Hkv, cap, device="cuda"):
+    def __init__(self, B, Hkv, cap, device="cuda", interleaved=False):
         self.B, self.Hkv, self.cap = B, Hkv, cap
         self.k_lo = torch.zeros(B, Hkv, KLOW_PLANES, cap, dtype=torch.int32,
                                 device=device)
-        self.k_full = torch.zeros(B, Hkv, cap, K_ATOMS, dtype=torch.int32,
-                                  device=device)
-        self.v_full = torch.zeros(B, Hkv, cap, K_ATOMS, dtype=torch.int32,
-                                  device=device)
+        if interleaved:
+            kv = torch.zeros(B, Hkv, cap, 2, K_ATOMS, dtype=torch.int32,
+                             device=device)
+            self.k_full, self.v_full = kv[:, :, :, 0], kv[:, :, :, 1]
+        else:
+            self.k_full = torch.zeros(B, Hkv, cap, K_ATOMS, dtype=torch.int32,
+                                      device=device)
+            self.v_full = torch.zeros(B, Hkv, cap, K_ATOMS, dtype=torch.int32,
+                                      device=device)
         self.lens = [0] * B
 
     @classmethod

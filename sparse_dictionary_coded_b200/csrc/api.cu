@@ -106,6 +106,12 @@ size_t sdk_encode_workspace_bytes(int64_t n_vec, int32_t head_dim, int32_t n_ato
 
 // Runs the encoder with an explicit header and scratch area (the scratch is
 // what the tensor-core encoder needs beyond its inputs and outputs).
+// Words between consecutive tokens' records: 32 when k_full and v_full point
+// into one interleaved array (v_full = k_full + 16 words), else 16.
+static int record_stride(const uint32_t* k_full, const uint32_t* v_full) {
+  return v_full == k_full + SDK_K_ATOMS ? 2 * SDK_K_ATOMS : SDK_K_ATOMS;
+}
+
 static sdk_status encode_core(bool allow_tc, const EncodeParams& p, int head_dim, void* scratch,
                               size_t scratch_bytes, cudaStream_t st) {
   if (p.n_vec == 0) return SDK_OK;
@@ -178,7 +184,7 @@ struct ScatterParams {
   uint32_t* full;         // [B][Hkv][cap][16]
   uint32_t* lo;           // [B][Hkv][3][cap] or null
   int64_t cap;
-  int Hkv, n_new;
+  int Hkv, n_new, rs;
   int64_t nv;
   int lens[kMaxBatch];
 };
@@ -193,7 +199,7 @@ __global__ void scatter_codes_kernel(ScatterParams p) {
   const int b = (int)(bk / p.Hkv);
   const int64_t t = (int64_t)p.lens[b] + i;
   const uint32_t w = p.codes[e];
-  p.full[(bk * p.cap + t) * kAtoms + j] = w;
+  p.full[(bk * p.cap + t) * p.rs + j] = w;
   if (p.lo != nullptr && j < kLoPlanes) p.lo[(bk * kLoPlanes + j) * p.cap + t] = w;
 }
 
@@ -261,6 +267,7 @@ sdk_status sdk_append(const void* xk, const void* xv, int32_t x_dtype, int32_t B
     e.Hkv = Hkv;
     e.n_new = n_new;
     e.lens = lens_host;
+    e.rs = record_stride(k_full, v_full);
     e.streams = 2;
     bool taken = false;
     sdk_status rc = launch_encode_small(e, scratch, scratch_bytes, st, &taken);
@@ -297,6 +304,7 @@ sdk_status sdk_append(const void* xk, const void* xv, int32_t x_dtype, int32_t B
     sp.cap = cap;
     sp.Hkv = Hkv;
     sp.n_new = n_new;
+    sp.rs = record_stride(k_full, v_full);
     sp.nv = nv;
     for (int b = 0; b < B; ++b) sp.lens[b] = lens_host[b];
     const int64_t tot = nv * kAtoms;
@@ -414,6 +422,7 @@ static sdk_status build_decode_params(const float* q, int32_t B, int32_t Hq, int
   // SDK_DECODE_BRACKET=0 is set in the environment
   p.bracket = (!p.full && bracket_selection()) ? 1 : 0;
   p.keep_keys = (flags & SDK_DECODE_KEEP_KEYS) ? 1 : 0;
+  p.rs = record_stride(k_full, v_full);
   p.R = B * Hq;
   p.n_out_tiles = (n_atoms + 127) / 128;
   p.scale = scale;

@@ -331,7 +331,7 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
     __syncthreads();
     const int64_t head = (int64_t)b * p.Hkv + kvh;
     const uint32_t* plane = p.k_lo + head * kLoPlanes * p.cap;
-    const uint32_t* rec = p.k_full + head * p.cap * kAtoms;
+    const uint32_t* rec = p.k_full + head * p.cap * p.rs;
     uint32_t* keys = p.keys + (int64_t)r * p.L;
     sdk_select_state* st = p.st + r;
     uint32_t lo = 0u, hi = 0u;
@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
           s = fmaf(word_coef(wc[j][u]), table[idx], s);
         }
         for (int j = kLoPlanes; j < p.klow; ++j) {      // klow > 3: k_full words
-          const uint32_t wj = (t >= t0 && t < t1) ? __ldg(rec + (int64_t)t * kAtoms + j) : 0u;
+          const uint32_t wj = (t >= t0 && t < t1) ? __ldg(rec + (int64_t)t * p.rs + j) : 0u;
           const uint32_t idx = word_idx(wj);
           maxidx = max(maxidx, idx);
           s = fmaf(word_coef(wj), table[idx], s);
@@ -770,7 +770,7 @@ __device__ uint32_t tie_cut_tokens(const uint32_t* keys, int n, uint32_t T, uint
 // s_lo of token t of a head exactly as klow_kernel computes it (the same
 // words, table values and FMA order; an index >= n reads 0).
 __device__ __forceinline__ float klow_score_at(const uint32_t* plane, int64_t cap,
-                                               const uint32_t* rec, int t, int klow, int nlo,
+                                               const uint32_t* rec, int rs, int t, int klow, int nlo,
                                                const float* tab, int n, bool global_tab) {
   uint32_t w[kLoPlanes];
 #pragma unroll
@@ -783,7 +783,7 @@ __device__ __forceinline__ float klow_score_at(const uint32_t* plane, int64_t ca
     s = fmaf(word_coef(w[j]), v, s);
   }
   for (int j = kLoPlanes; j < klow; ++j) {
-    const uint32_t wj = __ldg(rec + (int64_t)t * kAtoms + j);
+    const uint32_t wj = __ldg(rec + (int64_t)t * rs + j);
     const uint32_t idx = word_idx(wj);
     const float v = global_tab ? (idx < (uint32_t)n ? __ldg(tab + idx) : 0.0f) : tab[idx];
     s = fmaf(word_coef(wj), v, s);
@@ -805,7 +805,7 @@ __global__ void __launch_bounds__(kSampleThreads) sample_kernel(DecodeParams p) 
   const int S = (N + blk - 1) / blk;
   const int64_t head = (int64_t)b * p.Hkv + kvh;
   const uint32_t* plane = p.k_lo + head * kLoPlanes * p.cap;
-  const uint32_t* rec = p.k_full + head * p.cap * kAtoms;
+  const uint32_t* rec = p.k_full + head * p.cap * p.rs;
   const float* qd = p.qd + (int64_t)r * p.n;
   const uint32_t seed = lowbias32(0x9E3779B9u * (uint32_t)(head + 1));
   const int nlo = min(p.klow, kLoPlanes);
@@ -835,7 +835,7 @@ __global__ void __launch_bounds__(kSampleThreads) sample_kernel(DecodeParams p) 
       s = fmaf(word_coef(wv[u][j]), idx < (uint32_t)p.n ? __ldg(qd + idx) : 0.0f, s);
     }
     for (int j = kLoPlanes; j < p.klow; ++j) {
-      const uint32_t wj = __ldg(rec + (int64_t)tt[u] * kAtoms + j);
+      const uint32_t wj = __ldg(rec + (int64_t)tt[u] * p.rs + j);
       const uint32_t idx = word_idx(wj);
       s = fmaf(word_coef(wj), idx < (uint32_t)p.n ? __ldg(qd + idx) : 0.0f, s);
     }
@@ -961,11 +961,11 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(DecodeParams p) 
     __syncthreads();
     const int64_t head = (int64_t)b * p.Hkv + kvh;
     const uint32_t* plane = p.k_lo + head * kLoPlanes * p.cap;
-    const uint32_t* rec = p.k_full + head * p.cap * kAtoms;
+    const uint32_t* rec = p.k_full + head * p.cap * p.rs;
     uint32_t* keys = p.keys + (int64_t)r * p.L;
     const int nlo = min(p.klow, kLoPlanes);
     for (int t = tid; t < N; t += kSelThreads)
-      keys[t] = score_key(klow_score_at(plane, p.cap, rec, t, p.klow, nlo, table, p.n, false));
+      keys[t] = score_key(klow_score_at(plane, p.cap, rec, p.rs, t, p.klow, nlo, table, p.n, false));
     __syncthreads();
     T = rank_desc(keys, N, k, sh, s_tmp, eq_total, eq_take, bad);
     if (!bad && eq_total > eq_take) t_cut = tie_cut_tokens(keys, N, T, eq_take, s_tmp, sh, bad);
@@ -1453,29 +1453,36 @@ constexpr float kFixInv = 1.0f / 1048576.0f;
 // thread so the reads are free of bank conflicts): entries i + T and i + 2T
 // are in flight while i is used and the record of i + 3T is prefetched into
 // L2.  The list entries themselves are loaded six iterations ahead, so no
-// iteration waits on a list load.
-template <class Pay, class F>
+// iteration waits on a list load.  rs4: 16-byte units between consecutive
+// tokens' records (4, or 8 in the interleaved layout).  kLine: the copies
+// and the prefetch bring the record's whole 128-byte line into L2 (in the
+// interleaved layout the key pass thereby fetches the value record the
+// value pass reads next); otherwise exactly the record's 64 bytes, since
+// records sit at random token positions.
+template <bool kLine, class Pay, class F>
 __device__ __forceinline__ void for_records(const int32_t* list, int e0, int e1, const uint4* rec,
-                                            int Nb, WsHeader* hdr, uint32_t tag, uint4* ring,
-                                            Pay pay, F f) {
+                                            int rs4, int Nb, WsHeader* hdr, uint32_t tag,
+                                            uint4* ring, Pay pay, F f) {
   constexpr int T = kAttThreads;
   const int tid = threadIdx.x;
   const int sw = (tid >> 1) & 3;
   auto list_at = [&](int i) -> int { return i < e1 ? __ldg(list + i) : -1; };
   auto ok = [&](int t) { return (unsigned)t < (unsigned)Nb; };
-  // records sit at random token positions: both the copies and the L2
-  // prefetch ask for exactly the record's 64 bytes, not its 128-byte line
   auto issue = [&](int t, int slot) {
     const bool v = ok(t);
-    const uint4* a = rec + (int64_t)(v ? t : 0) * 4;
+    const uint4* a = rec + (int64_t)(v ? t : 0) * rs4;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) cp_async16_64B(ring + (slot * T + tid) * 4 + (u ^ sw), a + u, v);
+    for (int u = 0; u < 4; ++u) {
+      if (kLine) cp_async16_128B(ring + (slot * T + tid) * 4 + (u ^ sw), a + u, v);
+      else cp_async16_64B(ring + (slot * T + tid) * 4 + (u ^ sw), a + u, v);
+    }
     cp_async_commit();
   };
   auto prefetch = [&](int t) {
     if (ok(t)) {
-      const uint4* a = rec + (int64_t)t * 4;
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], 64;" ::"l"(a) : "memory");
+      const uint4* a = rec + (int64_t)t * rs4;
+      if (kLine) asm volatile("cp.async.bulk.prefetch.L2.global [%0], 128;" ::"l"(a) : "memory");
+      else asm volatile("cp.async.bulk.prefetch.L2.global [%0], 64;" ::"l"(a) : "memory");
     }
   };
   int i = e0 + tid;
@@ -1650,8 +1657,9 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
   const int c0 = k + (int)((int64_t)(Dr - k) * rank / C);
   const int c1 = k + (int)((int64_t)(Dr - k) * (rank + 1) / C);
   const int64_t head = (int64_t)b * p.Hkv + kvh;
-  const uint4* krec = reinterpret_cast<const uint4*>(p.k_full + head * p.cap * kAtoms);
-  const uint4* vrec = reinterpret_cast<const uint4*>(p.v_full + head * p.cap * kAtoms);
+  const uint4* krec = reinterpret_cast<const uint4*>(p.k_full + head * p.cap * p.rs);
+  const uint4* vrec = reinterpret_cast<const uint4*>(p.v_full + head * p.cap * p.rs);
+  const int rs4 = p.rs / 4;
   const int32_t* list = p.list + (int64_t)r * p.L;
   float* ss = p.sel_score + (int64_t)r * p.L;
   const uint32_t* keys = p.keys + (int64_t)r * p.L;
@@ -1683,7 +1691,13 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
   __syncthreads();
   float smax = -INFINITY, zrun = 0.0f;     // online softmax of this thread
   float smin = INFINITY;                   // for the integer softmax's scale
-  for_records(list, s0, s1, krec, Nb, p.hdr, 0x30000000u | r, ring, no_pay,
+  auto key_pass = [&](auto line, auto f) {
+    if constexpr (decltype(line)::value)
+      for_records<true>(list, s0, s1, krec, rs4, Nb, p.hdr, 0x30000000u | r, ring, no_pay, f);
+    else
+      for_records<false>(list, s0, s1, krec, rs4, Nb, p.hdr, 0x30000000u | r, ring, no_pay, f);
+  };
+  auto rescore = 
               [&](int i, int t, const uint4 (&w)[4], float) {
                 float s = 0.0f;
 #pragma unroll
@@ -1704,7 +1718,9 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
                 } else {
                   zrun += expf(s - smax);
                 }
-              });
+              };
+  if (p.rs == 2 * kAtoms) key_pass(std::true_type{}, rescore);
+  else key_pass(std::false_type{}, rescore);
   m = block_reduce<true>(smax, s_red);
   if (tid == 0) s_val = m;
   cluster.sync();
@@ -1814,11 +1830,11 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
     };
     // the logits load with the records: the rescored ones, and with the
     // flag the complement's scale * s_lo
-    for_records(list, s0, s1, vrec, Nb, p.hdr, 0x31000000u | r, ring,
+    for_records<false>(list, s0, s1, vrec, rs4, Nb, p.hdr, 0x31000000u | r, ring,
                 [&](int i, int) { return ss[i]; },
                 [&](int, int, const uint4 (&w)[4], float lg) { scatter(lg, w); });
     if (p.full)
-      for_records(list, c0, c1, vrec, Nb, p.hdr, 0x32000000u | r, ring,
+      for_records<false>(list, c0, c1, vrec, rs4, Nb, p.hdr, 0x32000000u | r, ring,
                   [&](int, int t) { return scale * key_score(keys[t]); },
                   [&](int, int, const uint4 (&w)[4], float lg) { scatter(lg, w); });
     // int32 range guard (also catches NaN): sum |p c| * 2^20 < 2^30

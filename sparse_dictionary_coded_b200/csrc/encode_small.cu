@@ -83,14 +83,14 @@ struct SmallParams {
   int k_atoms;
   int slice;             // atoms per CTA, multiple of 32, <= 256
   // outputs: plain mode writes codes[s][i * k_atoms + j]; append mode writes
-  // codes[s][(bk * cap + t) * 16 + j] (and lo[s][(bk * 3 + j) * cap + t] for
+  // codes[s][(bk * cap + t) * rs + j] (and lo[s][(bk * 3 + j) * cap + t] for
   // j < 3 when lo[s] is set) with bk = i / n_new, t = lens[bk / Hkv] + i % n_new
   uint32_t* codes[2];
   float* rsq[2];
   int append;
   uint32_t* lo[2];
   int64_t cap;
-  int n_new, Hkv;
+  int n_new, Hkv, rs;
   int lens[32];
   WsHeader* hdr;
   unsigned long long* words;   // [2][grid][64], zero before the launch
@@ -554,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           const int bk = i / p.n_new;
           const int64_t t = (int64_t)p.lens[bk / p.Hkv] + i % p.n_new;
-          p.codes[s][((int64_t)bk * p.cap + t) * kAtoms + j] = word;
+          p.codes[s][((int64_t)bk * p.cap + t) * p.rs + j] = word;
           if (p.lo[s] != nullptr && j < kLoPlanes)
             p.lo[s][((int64_t)bk * kLoPlanes + j) * p.cap + t] = word;
         }
@@ -673,6 +673,7 @@ sdk_status launch_encode_small(const SmallEncode& e, void* scratch, size_t scrat
   sp.cap = e.cap;
   sp.n_new = e.n_new;
   sp.Hkv = e.Hkv;
+  sp.rs = e.append ? e.rs : kAtoms;
   for (int b = 0; e.append && b < e.B; ++b) sp.lens[b] = e.lens[b];
   sp.hdr = e.p[0].hdr;
   sp.words = reinterpret_cast<unsigned long long*>(scratch);

@@ -127,6 +127,14 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, boo
                "r"(valid ? 16 : 0)
                : "memory");
 }
+// The same with the L2 fetch widened to the whole 128-byte line (for a
+// record whose line holds data needed later).
+__device__ __forceinline__ void cp_async16_128B(void* smem_dst, const void* gsrc, bool valid) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(smem_dst);
+  asm volatile("cp.async.cg.shared.global.L2::128B [%0], [%1], 16, %2;" ::"r"(d), "l"(gsrc),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
 // The same with the L2 prefetch size limited to 64 bytes (for 64-byte
 // records at scattered addresses).
 __device__ __forceinline__ void cp_async16_64B(void* smem_dst, const void* gsrc, bool valid) {
@@ -199,6 +207,11 @@ struct DecodeParams {
   // klow_kernel<1>, select_kernel) instead of radix histograms; keep_keys:
   // the Klow scan also stores every token's key (SDK_DECODE_KEEP_KEYS)
   int bracket, keep_keys;
+  // words between consecutive tokens' records in k_full / v_full: 16, or
+  // 32 when the two point into one interleaved array [..][cap][2][16]
+  // (v_full = k_full + 16: a token's key and value records form one
+  // 128-byte line)
+  int rs;
   // context-sharded decode: 0 = whole decode; 1 / 2 = attend's first /
   // second half (shard_in: the gathered softmax statistics); world ranks
   int att_mode, world;
@@ -271,6 +284,7 @@ struct SmallEncode {
   uint32_t* lo[2];
   int64_t cap;
   int B, Hkv, n_new;
+  int rs;               // words between tokens' records in the store (16 or 32)
   const int32_t* lens;  // host, [B]
 };
 // Sets *taken = false when it does not handle the call (too many rows,

@@ -349,6 +349,53 @@ def test_sampled_bracket_misses_on_both_sides():
         assert np.max(np.abs(out[0, h] - ref["out"])) <= OUT_TOL
 
 
+@pytest.mark.parametrize("full", [False, True])
+def test_interleaved_layout(full):
+    """k_full and v_full as views of one [B, Hkv, cap, 2, 16] array (a
+    token's key and value records in one 128-byte line): the library
+    detects the layout from v_full = k_full + 16 words; sets and outputs
+    against the oracle (ragged batch of 9000 / 40000 / 2500 tokens, so the
+    sampled bracket runs, and klow = 5 reads k_full words past the
+    planes)."""
+    q, DK, DV, kw, vw, _ = _random_case(94, 3, 8, 2, 40000, 128, 4096)
+    lens = [9000, 40000, 2500]
+    k_lo, k_full, v_full = workloads.layout(kw, vw, interleaved=True)
+    assert v_full.data_ptr() - k_full.data_ptr() == 64
+    store = sdk.CodeStore.from_tensors(k_lo.cuda(), k_full.cuda(), v_full.cuda(), lens)
+    out, ws, lay, rc = _run(q, DK, DV, store, full_softmax=full)
+    assert rc == 0
+    ref_store = _store(kw, vw, lens)
+    out_ref, _, _, rc = _run(q, DK, DV, ref_store, full_softmax=full)
+    assert rc == 0
+    assert np.max(np.abs(out - out_ref)) <= 1e-5
+    heads = [(0, 0), (1, 7), (2, 3)]
+    for klow in (3, 5):
+        _compare_store(q, DK, DV, kw, vw, lens, store, klow=klow, full=full, heads=heads)
+
+
+def _compare_store(q, DK, DV, kw, vw, lens, store, klow=3, full=False, heads=None):
+    """_compare on a given (possibly interleaved) code store."""
+    B, Hq, d = q.shape
+    out, ws, lay, rc = _run(q, DK, DV, store, klow=klow, full_softmax=full)
+    assert rc == 0
+    R = B * Hq
+    ks = [oracle.topk_count(lens[r // Hq], 1, 10) for r in range(R)]
+    sets = _gpu_sets(ws, lay, R, max(lens), ks)
+    qn = q.double().numpy()
+    kwn, vwn = words_np(kw), words_np(vw)
+    DKn, DVn = DK.float().double().numpy(), DV.float().double().numpy()
+    g = Hq // kw.shape[1]
+    for (b, h) in heads:
+        r = b * Hq + h
+        n_b = lens[b]
+        ref = oracle.decode_head_ref(qn[b, h], kwn[b, h // g, :n_b], vwn[b, h // g, :n_b],
+                                     DKn, DVn, klow, 16, 1, 10, full)
+        if check_selection(sets[r], ref["s_lo"], ks[r]):
+            ref = oracle.decode_head_ref(qn[b, h], kwn[b, h // g, :n_b], vwn[b, h // g, :n_b],
+                                         DKn, DVn, klow, 16, 1, 10, full, force_set=sets[r])
+        assert np.max(np.abs(out[b, h] - ref["out"])) <= OUT_TOL
+
+
 def test_klow_and_khigh_variants():
     q, DK, DV, kw, vw, lens = _random_case(12, 2, 8, 4, 700, 128, 4096)
     _compare(q, DK, DV, kw, vw, lens, klow=1, khigh=8, top_num=1, top_den=4)

@@ -183,17 +183,19 @@ def test_candidate_overflow_falls_back_to_exact_scan():
     assert torch.equal(codes.cpu(), b.cpu())
 
 
-def test_append_writes_the_layout():
+@pytest.mark.parametrize("interleaved", [False, True], ids=["separate", "interleaved"])
+def test_append_writes_the_layout(interleaved):
     """sdk_append encodes K and V and writes k_lo planes, k_full and v_full
-    records at positions lens[b]..lens[b]+n_new-1, leaving the rest."""
+    records at positions lens[b]..lens[b]+n_new-1, leaving the rest (also
+    with the key and value records interleaved in one array)."""
     g = workloads.make_gen(31)
     n, d, B, Hkv, cap = 2048, 128, 2, 4, 64
     DK = workloads.gaussian_dictionary(n, d, g).cuda()
     DV = workloads.gaussian_dictionary(n, d, g).cuda()
-    store = sdk.CodeStore(B, Hkv, cap)
+    store = sdk.CodeStore(B, Hkv, cap, interleaved=interleaved)
     store.lens = [3, 17]
-    sentinel = torch.full_like(store.k_full, 0x12345)
-    store.k_full.copy_(sentinel)
+    store.k_full.fill_(0x12345)
+    store.v_full.fill_(0x12345)
     xk = torch.randn(B, Hkv, 5, d, generator=g).cuda()
     xv = torch.randn(B, Hkv, 5, d, generator=g).cuda()
     ws = sdk.sdk_append(store, xk, xv, DK, DV)
@@ -207,8 +209,9 @@ def test_append_writes_the_layout():
         assert torch.equal(store.v_full[b, :, l0:l0 + 5], cv[b])
         assert torch.equal(store.k_lo[b, :, :, l0:l0 + 5],
                            ck[b, :, :, :3].transpose(-1, -2))
-        assert torch.all(store.k_full[b, :, :l0] == 0x12345)
-        assert torch.all(store.k_full[b, :, l0 + 5:] == 0x12345)
+        for t in (store.k_full, store.v_full):
+            assert torch.all(t[b, :, :l0] == 0x12345)
+            assert torch.all(t[b, :, l0 + 5:] == 0x12345)
     # capacity check: 22 + 50 > 64
     with pytest.raises(sdk.SdkError):
         sdk.sdk_append(store, torch.randn(B, Hkv, 50, d).cuda(),
@@ -320,8 +323,9 @@ APPEND_CASES = [
 ]
 
 
+@pytest.mark.parametrize("interleaved", [False, True], ids=["separate", "interleaved"])
 @pytest.mark.parametrize("case", APPEND_CASES, ids=lambda c: "B%d_H%d_n%d" % c[:3])
-def test_token_append_writes_exact_codes(case):
+def test_token_append_writes_exact_codes(case, interleaved):
     """Per-token append (the decode loop's shape): the encoder writes the
     words straight into the code store at lens[b]..lens[b]+n_new-1, the
     first 3 key words also into the k_lo planes; every word equals the
@@ -331,7 +335,7 @@ def test_token_append_writes_exact_codes(case):
     n, d, cap = 32768, 128, 40
     DK = workloads.gaussian_dictionary(n, d, g).cuda()
     DV = workloads.gaussian_dictionary(n, d, g).cuda()
-    store = sdk.CodeStore(B, Hkv, cap)
+    store = sdk.CodeStore(B, Hkv, cap, interleaved=interleaved)
     lens0 = [int(v) for v in torch.randint(0, cap - n_new + 1, (B,), generator=g)]
     store.lens = list(lens0)
     for t in (store.k_lo, store.k_full, store.v_full):

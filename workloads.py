@@ -177,13 +177,19 @@ def random_codes(shape, n_atoms, gen, device="cpu"):
     return words_from(idx, c)
 
 
-def layout(kwords, vwords, cap=None):
-    """Code-store layout from [B, Hkv, N, 16] word tensors (pure copies)."""
+def layout(kwords, vwords, cap=None, interleaved=False):
+    """Code-store layout from [B, Hkv, N, 16] word tensors (pure copies).
+    interleaved: k_full and v_full are views of one [B, Hkv, cap, 2, 16]
+    array (a token's key and value records adjacent)."""
     B, Hkv, N, _ = kwords.shape
     cap = N if cap is None else cap
     dev = kwords.device
-    k_full = torch.zeros(B, Hkv, cap, K_ATOMS, dtype=torch.int32, device=dev)
-    v_full = torch.zeros(B, Hkv, cap, K_ATOMS, dtype=torch.int32, device=dev)
+    if interleaved:
+        kv = torch.zeros(B, Hkv, cap, 2, K_ATOMS, dtype=torch.int32, device=dev)
+        k_full, v_full = kv[:, :, :, 0], kv[:, :, :, 1]
+    else:
+        k_full = torch.zeros(B, Hkv, cap, K_ATOMS, dtype=torch.int32, device=dev)
+        v_full = torch.zeros(B, Hkv, cap, K_ATOMS, dtype=torch.int32, device=dev)
     k_lo = torch.zeros(B, Hkv, KLOW_PLANES, cap, dtype=torch.int32,
                        device=dev)
     k_full[:, :, :N] = kwords
