@@ -19,8 +19,9 @@ append 65,536 vectors of one layer, then one decode step over 4096 tokens),
 32 layers).
 
 Timing: W untimed warm-up steps, then K steps, each timed with CUDA events on
-the launching stream; the L2 is flushed (256 MiB memset) between steps,
-outside the events.  Multi-GPU (torchrun): every rank runs its own
+the launching stream.  Encode workloads flush the L2 (256 MiB memset)
+between steps, outside the events; the decode workloads' inputs exceed the
+L2 (every layer's working set is larger than it), so they run unflushed.  Multi-GPU (torchrun): every rank runs its own
 independent copy of the workload (weak scaling, no collective on the data
 path); the time is the max over ranks.  Rank 0 prints one JSON line.
 """
@@ -46,9 +47,6 @@ def enc_flop_per_vector(n_atoms, head_dim):
     return 16 * n_atoms * head_dim * 2
 
 
-# kernels of one tensor-core encode call: dictionary statistics, fp16
-# dictionary copy, encoder
-ENC_KERNELS_PER_CALL = 3
 # kernels of one decode layer: qd, klow, pass2, final, attend, out
 DEC_KERNELS_PER_LAYER = 6
 DECODE_UNIT = "ctx tokens/s/step"
@@ -302,6 +300,10 @@ def timed_steps(step, steps, warmup, flush, world, clocks=None):
     return ms, ck
 
 
+def no_flush():
+    pass
+
+
 def make_flush():
     import torch
     buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
@@ -363,7 +365,8 @@ def workload_config(name, args):
             "softmax": ("integer (INT16 logits)" if args.int_softmax else "fp32")
                        + (", all tokens" if args.full_softmax else ", selected set"),
             "kv_layout": getattr(args, "kv_layout", "separate"),
-            "l2": "flushed between steps; codes (%.1f GB) exceed L2"
+            "l2": "not flushed: inputs larger than L2 (codes %.1f GB; every layer's "
+                  "working set exceeds the 126 MB L2)"
                   % (L * W["B"] * W["Hkv"] * W["n_tokens"] * 140 / 1e9)}
 
 
@@ -438,9 +441,9 @@ def bench_layer4k(args, world, rank, pk):
         "config": workload_config("layer4k", args),
         "dtype": ENC_DTYPE,
         # kernels per step: append = 2 x (dictionary statistics + fp16
-        # dictionary copy + encode + scatter); decode = DEC_KERNELS_PER_LAYER
-        "gpu_launches": args.steps * (2 * ENC_KERNELS_PER_CALL + 2 +
-                                      DEC_KERNELS_PER_LAYER),
+        # dictionary copy) + one encoder over both streams + 2 scatters;
+        # decode = DEC_KERNELS_PER_LAYER
+        "gpu_launches": args.steps * (2 * 2 + 1 + 2 + DEC_KERNELS_PER_LAYER),
         "enc_fallback_rows": hdr[2],
     }
     if not args.no_e2e:
@@ -589,7 +592,11 @@ def bench_decode(args, world, rank, pk, name):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         step()
-    flush = make_flush()
+    # no L2 flush: every layer's working set (codes, lists, QD: about 150
+    # MB) and the step's codes (gigabytes) exceed the 126 MB L2, so a step
+    # never finds the previous one's data there; a memset flush would
+    # only leave dirty lines whose write-back lands in the timed step
+    flush = no_flush
     clocks = Clocks(torch.cuda.current_device())
     ms, ck = timed_steps(g.replay, args.steps, args.warmup, flush, world, clocks)
     # serialised-layer variant without the graph, for reference
@@ -678,23 +685,25 @@ def bench_decode(args, world, rank, pk, name):
 
 
 def bench_prefill(args, world, rank, pk):
+    """The prefill encode: 16384 tokens x 8 KV heads of keys and values
+    (262,144 vectors) encoded against one layer's K and V dictionaries and
+    written into an empty code store, through one sdk_append call (both
+    streams' row tiles in one tensor-core launch)."""
     import torch
     import workloads
     import sparse_dictionary_coded_b200 as sdk
     w = workloads.prefill(device="cuda")
-    d, n = w["d"], w["n_atoms"]
-    xk = w["xk"].reshape(-1, d)
-    xv = w["xv"].reshape(-1, d)
+    d, n, Hkv, N = w["d"], w["n_atoms"], w["Hkv"], w["n_tokens"]
+    xk, xv = w["xk"].contiguous(), w["xv"].contiguous()
     if rank:
-        xk, xv = xv.flip(0).contiguous(), xk.flip(0).contiguous()
-    nv = xk.shape[0]
-    ck_ = torch.empty(nv, 16, dtype=torch.int32, device="cuda")
-    cv_ = torch.empty(nv, 16, dtype=torch.int32, device="cuda")
-    ws = sdk.new_workspace(sdk.sdk_encode_workspace_bytes(nv, d, n))
+        xk, xv = xv.flip(2).contiguous(), xk.flip(2).contiguous()
+    nv = Hkv * N
+    store = sdk.CodeStore(1, Hkv, N)
+    ws = sdk.new_workspace(sdk.sdk_append_workspace_bytes(1, Hkv, N, d, n))
 
     def step():
-        sdk.sdk_encode(xk, w["DK"], codes=ck_, workspace=ws)
-        sdk.sdk_encode(xv, w["DV"], codes=cv_, workspace=ws)
+        store.lens = [0]
+        sdk.sdk_append(store, xk, xv, w["DK"], w["DV"], workspace=ws)
 
     flush = make_flush()
     clocks = Clocks(torch.cuda.current_device())
@@ -704,19 +713,19 @@ def bench_prefill(args, world, rank, pk):
     step_ms = max_over_ranks(statistics.mean(ms), world)
     e2e = None
     if not args.no_e2e:
-        # host vectors in (pinned), codes back out, every step
+        # host vectors in (pinned), the appended code records back out
         hxk, hxv = xk.cpu().pin_memory(), xv.cpu().pin_memory()
-        hck = torch.empty(ck_.shape, dtype=ck_.dtype).pin_memory()
-        hcv = torch.empty(cv_.shape, dtype=cv_.dtype).pin_memory()
+        hck = torch.empty(store.k_full.shape, dtype=torch.int32).pin_memory()
+        hcv = torch.empty(store.v_full.shape, dtype=torch.int32).pin_memory()
         dxk, dxv = torch.empty_like(xk), torch.empty_like(xv)
 
         def e2e_step():
             dxk.copy_(hxk, non_blocking=True)
             dxv.copy_(hxv, non_blocking=True)
-            sdk.sdk_encode(dxk, w["DK"], codes=ck_, workspace=ws)
-            sdk.sdk_encode(dxv, w["DV"], codes=cv_, workspace=ws)
-            hck.copy_(ck_, non_blocking=True)
-            hcv.copy_(cv_, non_blocking=True)
+            store.lens = [0]
+            sdk.sdk_append(store, dxk, dxv, w["DK"], w["DV"], workspace=ws)
+            hck.copy_(store.k_full, non_blocking=True)
+            hcv.copy_(store.v_full, non_blocking=True)
 
         ms_e, _ = timed_steps(e2e_step, max(2, args.steps // 2), 1, flush, world)
         t = max_over_ranks(statistics.mean(ms_e), world)
@@ -729,12 +738,15 @@ def bench_prefill(args, world, rank, pk):
     return {
         "value": world * 2 * nv / (step_ms * 1e-3), "unit": ENCODE_UNIT,
         "ms_per_step": step_ms,
-        "roofline": tensor_roofline(tfl, pk, "encode (2 x sdk_encode: "
-                                    "encode_tc_kernel + dictionary prep)"),
+        "roofline": tensor_roofline(tfl, pk, "encode (sdk_append: dictionary prep, "
+                                    "one encode_tc_kernel over both streams' row "
+                                    "tiles, code scatter)"),
         "clocks": ck,
         "config": workload_config("prefill256k_vec", args),
         "dtype": ENC_DTYPE,
-        "gpu_launches": args.steps * 2 * ENC_KERNELS_PER_CALL,
+        # dictionary statistics + fp16 copy per stream, one encoder, one
+        # scatter per stream
+        "gpu_launches": args.steps * (2 * 2 + 1 + 2),
         "enc_fallback_rows": hdr[2],
         **({"e2e": e2e} if e2e else {}),
     }

@@ -211,6 +211,27 @@ SDK_API size_t sdk_append_workspace_bytes(int32_t B, int32_t Hkv, int32_t n_new,
  *              n_atoms, max_len) with max_len >= every lens[b]
  * Limits: B <= 64, Hq % Hkv == 0, head_dim in {64, 128}, B*Hq <= 2048,
  *         scale > 0.
+ * Selection (how S is found; the set is exact either way): without
+ * SDK_DECODE_FULL_SOFTMAX, a sample of every head's tokens is scored first
+ * and two of its order statistics bracket the k-th key; the Klow scan then
+ * selects the tokens above the bracket and keeps those inside it as
+ * candidates, among which the exact k-th key and the tie cut are found; a
+ * head whose k-th key falls outside the bracket is re-scanned exactly
+ * (state `select_path` 2).  The sample of KV head (b, kvh) with N tokens:
+ * every token when N <= 8192; else, with blk = 8 * ceil(ceil(N / 1024) / 8)
+ * and seed = lowbias32(0x9E3779B9 * (b * Hkv + kvh + 1)) (32-bit
+ * arithmetic; lowbias32 is Chris Wellons' integer hash x ^= x >> 16,
+ * x *= 0x7feb352d, x ^= x >> 15, x *= 0x846ca68b, x ^= x >> 16), block i
+ * of blk tokens (len_i = min(blk, N - i * blk)) contributes the 8 tokens
+ * from i * blk + 8 * (lowbias32(seed ^ i) mod (len_i / 8)), or all of its
+ * tokens when len_i < 8.  The bracket is the sample's order statistics
+ * 6 standard deviations of the sample rank above and below S * k / N.
+ * With SDK_DECODE_FULL_SOFTMAX (or SDK_DECODE_BRACKET=0 in the environment)
+ * the selection runs by radix histograms of all keys instead.
+ * Code store layout: k_full and v_full may also point into ONE array
+ * uint32 [B][Hkv][cap][2][16] with v_full = k_full + 16 (a token's key and
+ * value records adjacent in one 128-byte line); the library detects this
+ * from the two pointers (here and in sdk_append).
  */
 SDK_API sdk_status sdk_decode_attn(const float* q, int32_t B, int32_t Hq, int32_t Hkv,
                            int32_t head_dim, const void* dict_k,

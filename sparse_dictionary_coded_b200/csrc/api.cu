@@ -127,7 +127,7 @@ static sdk_status encode_core(bool allow_tc, const EncodeParams& p, int head_dim
   }
   if (allow_tc) {
     bool taken = false;
-    sdk_status s = launch_encode_tc(p, head_dim, scratch, scratch_bytes, st, &taken);
+    sdk_status s = launch_encode_tc(&p, 1, head_dim, scratch, scratch_bytes, st, &taken);
     if (taken) return s;
   }
   return launch_encode_simt(p, head_dim, st);
@@ -207,11 +207,16 @@ __global__ void scatter_codes_kernel(ScatterParams p) {
 
 extern "C" {
 
+// header, K and V code buffers [nv][16] each, then the encoder's scratch for
+// both streams in one launch (or the small encoder's)
 size_t sdk_append_workspace_bytes(int32_t B, int32_t Hkv, int32_t n_new, int32_t head_dim,
                                   int32_t n_atoms) {
   const int64_t nv = (int64_t)(B > 0 ? B : 0) * (Hkv > 0 ? Hkv : 0) * (n_new > 0 ? n_new : 0);
-  return align_up(sizeof(WsHeader), 256) + align_up((size_t)nv * kAtoms * 4, 256) +
-         sdk_encode_workspace_bytes(nv, head_dim, n_atoms);
+  size_t scratch = encode_tc_scratch_bytes(2 * nv, head_dim, n_atoms, 2);
+  const size_t one = sdk_encode_workspace_bytes(nv, head_dim, n_atoms) - align_up(sizeof(WsHeader), 256);
+  if (one > scratch) scratch = one;
+  return align_up(sizeof(WsHeader), 256) + 2 * align_up((size_t)nv * kAtoms * 4, 256) +
+         align_up(scratch, 256);
 }
 
 sdk_status sdk_append(const void* xk, const void* xv, int32_t x_dtype, int32_t B, int32_t Hkv,
@@ -237,9 +242,11 @@ sdk_status sdk_append(const void* xk, const void* xv, int32_t x_dtype, int32_t B
   const int64_t nv = (int64_t)B * Hkv * n_new;
   char* ws = reinterpret_cast<char*>(workspace);
   const size_t hb = align_up(sizeof(WsHeader), 256);
-  uint32_t* codes = reinterpret_cast<uint32_t*>(ws + hb);
-  char* scratch = ws + hb + align_up((size_t)nv * kAtoms * 4, 256);
-  const size_t scratch_bytes = sdk_encode_workspace_bytes(nv, head_dim, n_atoms) - hb;
+  const size_t cb = align_up((size_t)nv * kAtoms * 4, 256);
+  uint32_t* codes2[2] = {reinterpret_cast<uint32_t*>(ws + hb),
+                         reinterpret_cast<uint32_t*>(ws + hb + cb)};
+  char* scratch = ws + hb + 2 * cb;
+  const size_t scratch_bytes = sdk_append_workspace_bytes(B, Hkv, n_new, head_dim, n_atoms) - hb - 2 * cb;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // a few vectors: the atom-parallel encoder writes straight into the store,
   // K and V in one launch when both fit
@@ -284,21 +291,32 @@ sdk_status sdk_append(const void* xk, const void* xv, int32_t x_dtype, int32_t B
       return rc;
     }
   }
+  // K and V: one tensor-core launch over the row tiles of both streams
+  // (or, where it does not apply, one encode per stream), then the words
+  // go into the store
+  EncodeParams pe[2];
   for (int s = 0; s < 2; ++s) {
-    EncodeParams p;
+    EncodeParams& p = pe[s];
     p.x = s == 0 ? xk : xv;
     p.x_dtype = x_dtype;
     p.n_vec = nv;
     p.dict = reinterpret_cast<const uint16_t*>(s == 0 ? dict_k : dict_v);
     p.n = n_atoms;
     p.k_atoms = kAtoms;
-    p.codes = codes;
+    p.codes = codes2[s];
     p.rsq = nullptr;
     p.hdr = reinterpret_cast<WsHeader*>(ws);
-    sdk_status rc = encode_core(true, p, head_dim, scratch, scratch_bytes, st);
+  }
+  bool taken = false;
+  sdk_status rc = launch_encode_tc(pe, 2, head_dim, scratch, scratch_bytes, st, &taken);
+  if (rc != SDK_OK) return rc;
+  for (int s = 0; s < 2 && !taken; ++s) {
+    rc = encode_core(true, pe[s], head_dim, scratch, scratch_bytes, st);
     if (rc != SDK_OK) return rc;
+  }
+  for (int s = 0; s < 2; ++s) {
     ScatterParams sp;
-    sp.codes = codes;
+    sp.codes = codes2[s];
     sp.full = s == 0 ? k_full : v_full;
     sp.lo = s == 0 ? k_lo : nullptr;
     sp.cap = cap;

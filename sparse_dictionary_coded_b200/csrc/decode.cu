@@ -281,6 +281,12 @@ constexpr int kScanThreads = 512;
 constexpr int64_t kKlowSegCost = 11000;
 constexpr int64_t kPass2SegCost = 28000;
 constexpr int kKlowThreads = 1024;
+// bracket mode: per-segment buffers of selected tokens and candidates
+// (expected per segment at 256K tokens on 148 CTAs: about 4,500 and 2,300)
+constexpr int kKlowAboveBuf = 8192;
+constexpr int kKlowCandBuf = 4096;
+constexpr int kKlowSmemHist = kTable * 4 + 4096 * 4;
+constexpr int kKlowSmemBracket = kTable * 4 + (kKlowAboveBuf + 2 * kKlowCandBuf) * 4;
 
 // QD row -> table[0..kTable), zero past n.  Eight 16-byte loads per thread
 // are issued before any is stored, so the staging costs about one L2 round
@@ -317,10 +323,17 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
   extern __shared__ float4 smem4[];
   float* table = reinterpret_cast<float*>(smem4);
   uint32_t* sh = reinterpret_cast<uint32_t*>(table + kTable);
+  // bracket mode: the segment's selected tokens and candidates are
+  // collected here and reserved in the global lists once per segment
+  int32_t* s_ab = reinterpret_cast<int32_t*>(table + kTable);
+  int32_t* s_ct = s_ab + kKlowAboveBuf;
+  uint32_t* s_ck = reinterpret_cast<uint32_t*>(s_ct + kKlowCandBuf);
+  __shared__ uint32_t s_cnt[2], s_base[2];
   const int n = p.n, tid = threadIdx.x, lane = tid & 31;
   const int nlo = min(p.klow, kLoPlanes);
   const bool store_keys = !kBracket || p.keep_keys;
   uint32_t maxidx = 0u;
+  if (kBracket && tid == 0) s_cnt[0] = s_cnt[1] = 0u;
 
   for_segments(p.tok_off, p.lens, p.B, p.Hq, kKlowSegCost, [&](int b, int h, int64_t t0l, int64_t t1l) {
     const int r = b * p.Hq + h, kvh = h / p.g;
@@ -447,10 +460,12 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
         }
         const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
         if (tot != 0u) {
+          // slots in the shared-memory buffers (one shared atomic per kind
+          // and warp); past a buffer's end an entry takes a global slot
           uint32_t ba = 0u, bc = 0u;
           if (lane == 31) {
-            if (tot & 0xFFFFu) ba = atomicAdd(&st->n_above, tot & 0xFFFFu);
-            if (tot >> 16) bc = atomicAdd(&st->n_cand, tot >> 16);
+            if (tot & 0xFFFFu) ba = atomicAdd(&s_cnt[0], tot & 0xFFFFu);
+            if (tot >> 16) bc = atomicAdd(&s_cnt[1], tot >> 16);
           }
           ba = __shfl_sync(0xffffffffu, ba, 31);
           bc = __shfl_sync(0xffffffffu, bc, 31);
@@ -460,13 +475,24 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
           for (int u = 0; u < 4; ++u) {
             const int t = 4 * q + u;
             if ((fa >> u) & 1u) {
-              if (pa < (uint32_t)p.L) above_out[pa] = t;
+              if (pa < (uint32_t)kKlowAboveBuf) {
+                s_ab[pa] = t;
+              } else {
+                const uint32_t g = atomicAdd(&st->n_above, 1u);
+                if (g < (uint32_t)p.L) above_out[g] = t;
+              }
               ++pa;
             }
             if ((fc >> u) & 1u) {
-              if (pc < (uint32_t)p.L) {
-                cand_t[pc] = t;
-                cand_k[pc] = kq[u];
+              if (pc < (uint32_t)kKlowCandBuf) {
+                s_ct[pc] = t;
+                s_ck[pc] = kq[u];
+              } else {
+                const uint32_t g = atomicAdd(&st->n_cand, 1u);
+                if (g < (uint32_t)p.L) {
+                  cand_t[g] = t;
+                  cand_k[g] = kq[u];
+                }
               }
               ++pc;
             }
@@ -484,6 +510,30 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
       for (int i = tid; i < 4096; i += kKlowThreads)
         if (sh[i]) atomicAdd(&gh[i], sh[i]);
       __syncthreads();
+    } else {
+      // the segment's buffered entries: one global reservation per kind
+      if (tid == 0) {
+        const uint32_t na = min(s_cnt[0], (uint32_t)kKlowAboveBuf);
+        const uint32_t nc = min(s_cnt[1], (uint32_t)kKlowCandBuf);
+        s_base[0] = na ? atomicAdd(&st->n_above, na) : 0u;
+        s_base[1] = nc ? atomicAdd(&st->n_cand, nc) : 0u;
+      }
+      __syncthreads();
+      const uint32_t na = min(s_cnt[0], (uint32_t)kKlowAboveBuf);
+      const uint32_t nc = min(s_cnt[1], (uint32_t)kKlowCandBuf);
+      for (uint32_t i = tid; i < na; i += kKlowThreads) {
+        const uint32_t g = s_base[0] + i;
+        if (g < (uint32_t)p.L) above_out[g] = s_ab[i];
+      }
+      for (uint32_t i = tid; i < nc; i += kKlowThreads) {
+        const uint32_t g = s_base[1] + i;
+        if (g < (uint32_t)p.L) {
+          cand_t[g] = s_ct[i];
+          cand_k[g] = s_ck[i];
+        }
+      }
+      __syncthreads();
+      if (tid == 0) s_cnt[0] = s_cnt[1] = 0u;
     }
   });
   if (maxidx >= (uint32_t)n) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, maxidx);
@@ -684,11 +734,9 @@ __global__ void __launch_bounds__(kScanThreads) final_kernel(DecodeParams p) {
 
 // ------------------------------------------ sampled-bracket selection
 // The exact top k per query head without a second pass over the keys:
-//   sample_kernel  scores a sample of the head's tokens (one token per
-//                  block of blk = ceil(N / 8192) consecutive tokens, at
-//                  offset lowbias32(seed ^ block) mod the block's length,
-//                  seed = lowbias32(0x9E3779B9 * (b * Hkv + kvh + 1)); every
-//                  token when N <= 8192) with exactly the Klow scan's
+//   sample_kernel  scores a sample of the head's tokens (sample_geom: every
+//                  token when N <= 8192, else 1024 hashed runs of 8
+//                  consecutive tokens) with exactly the Klow scan's
 //                  arithmetic, and brackets the k-th key by two order
 //                  statistics of the sample, 6 standard deviations of the
 //                  sample rank on either side of the expected rank S k / N
@@ -697,44 +745,83 @@ __global__ void __launch_bounds__(kScanThreads) final_kernel(DecodeParams p) {
 //   klow_kernel<1> selects key > hi and collects lo <= key <= hi;
 //   select_kernel  finds the exact k-th key among the candidates when
 //                  n_above < k <= n_above + n_cand (ties: lower token), and
-//                  otherwise (the bracket missed, probability about 1e-9
-//                  per head for a representative sample) re-scores the
-//                  whole head and selects by radix histograms.
+//                  otherwise (the bracket missed, rare for a representative
+//                  sample) re-scores the whole head and selects by radix
+//                  histograms.
 // The result is the same set as the radix path in every case.
 constexpr int kSampleMax = 8192;
 constexpr int kSampleThreads = 1024;
 constexpr double kBracketSigmas = 6.0;
 
-// The rank-th largest (1-based) of n keys, by radix select over key digits
-// 31..21, 20..10, 9..0.  Also returns the number of keys equal to the
-// result (cnt) and the rank of the result among them (rank_in_ties:
-// rank - the number of larger keys).  keys: shared or global memory
-// (written before a __syncthreads of this block or by an earlier kernel);
-// hist: 2048 words of shared memory.
+// The rank-th largest (1-based) of n keys.  The result lies in [lo, hi],
+// first the keys' own range; every pass histograms (key - lo) >> shift
+// over 2048 bins with the smallest shift that covers the range, keeps the
+// bin that holds the rank-th key and narrows [lo, hi] to it, until shift
+// is 0.  Scaling the bins to the range (instead of fixed key digits)
+// spreads keys that share their high bits, e.g. the scores inside a
+// bracket, over many bins, so the shared-memory atomics rarely collide.
+// Also returns the number of keys equal to the result (cnt) and the rank
+// of the result among them (rank_in_ties: rank - the number of larger
+// keys).  keys: shared or global memory (written before a __syncthreads of
+// this block or by an earlier kernel); hist: 2048 words of shared memory.
 __device__ uint32_t rank_desc(const uint32_t* keys, int n, uint32_t rank, uint32_t* hist,
                               uint32_t* s_tmp, uint32_t& cnt, uint32_t& rank_in_ties, bool& bad) {
-  const int tid = threadIdx.x, nt = blockDim.x;
-  uint32_t prefix = 0u;
+  const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+  for (int i = tid; i < n; i += nt) {
+    const uint32_t key = keys[i];
+    mn = min(mn, key);
+    mx = max(mx, key);
+  }
+  mx = warp_umax(mx);
+  mn = ~warp_umax(~mn);
+  if (lane == 0) {
+    s_tmp[warp] = mx;
+    hist[warp] = mn;        // hist is free until the first pass clears it
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = nt >> 5;
+    uint32_t a = lane < nw ? s_tmp[lane] : 0u, c = lane < nw ? hist[lane] : 0xFFFFFFFFu;
+    a = warp_umax(a);
+    c = ~warp_umax(~c);
+    if (lane == 0) {
+      s_tmp[40] = c;
+      s_tmp[41] = a;
+    }
+  }
+  __syncthreads();
+  uint32_t lo = s_tmp[40], hi = s_tmp[41];
+  __syncthreads();
   cnt = 0u;
-  for (int ps = 0; ps < 3; ++ps) {
-    const int shf = ps == 0 ? 21 : (ps == 1 ? 10 : 0);
-    const int wb = ps == 2 ? 10 : 11;
-    const uint32_t mask = (1u << wb) - 1u;
+  bad = false;
+  if (n <= 0 || lo > hi) {
+    bad = true;
+    return 0u;
+  }
+  while (true) {
+    const uint32_t range = hi - lo;
+    const int shift = range < 2048u ? 0 : (32 - __clz((int)range)) - 11;
     for (int i = tid; i < 2048; i += nt) hist[i] = 0u;
     __syncthreads();
     for (int i = tid; i < n; i += nt) {
       const uint32_t key = keys[i];
-      if (ps == 0 || (key >> (shf + wb)) == prefix) atomicAdd(&hist[(key >> shf) & mask], 1u);
+      if (key >= lo && key <= hi) atomicAdd(&hist[(key - lo) >> shift], 1u);
     }
     __syncthreads();
     uint32_t bin, above;
     block_find_desc<2048>(hist, rank, s_tmp, bin, above, cnt, bad);
     if (bad) return 0u;
-    prefix = (prefix << wb) | bin;
     rank -= above;
+    const uint32_t nlo = lo + (bin << shift);
+    if (shift == 0) {
+      rank_in_ties = rank;
+      return nlo;
+    }
+    const uint64_t top = (uint64_t)nlo + ((1ull << shift) - 1ull);
+    hi = top < (uint64_t)hi ? (uint32_t)top : hi;
+    lo = nlo;
   }
-  rank_in_ties = rank;
-  return prefix;
 }
 
 // The rank-th smallest token index (1-based) among tokens 0..n-1 whose key
@@ -791,53 +878,84 @@ __device__ __forceinline__ float klow_score_at(const uint32_t* plane, int64_t ca
   return s;
 }
 
+// Geometry of the sample of an N-token head: every token when N <= 8192;
+// otherwise runs of 8 consecutive tokens, one run per block of blk tokens
+// (blk = 8 ceil(ceil(N / 1024) / 8)), the run of block i starting at
+// i blk + 8 (lowbias32(seed ^ i) mod (len_i / 8)) with len_i = min(blk,
+// N - i blk), or covering the whole block when len_i < 8.  A run of 8
+// keeps every sampled plane read inside one 32-byte sector.
+struct SampleGeom {
+  int blk, nb, S;
+};
+__device__ __forceinline__ SampleGeom sample_geom(int N) {
+  SampleGeom g;
+  if (N <= kSampleMax) {
+    g.blk = 1;
+    g.nb = N;
+    g.S = N;
+  } else {
+    g.blk = 8 * ((((N + 1023) / 1024) + 7) / 8);
+    g.nb = (N + g.blk - 1) / g.blk;
+    const int last = N - (g.nb - 1) * g.blk;
+    g.S = 8 * (g.nb - 1) + min(8, last);
+  }
+  return g;
+}
+// Token of sample i (0 <= i < S).
+__device__ __forceinline__ int sample_token(const SampleGeom& g, int N, uint32_t seed, int i) {
+  if (g.blk == 1) return i;
+  const int run = i >> 3, pos = i & 7;
+  const int len = min(g.blk, N - run * g.blk);
+  const int off = len < 8 ? 0 : 8 * (int)(lowbias32(seed ^ (uint32_t)run) % (uint32_t)(len / 8));
+  return run * g.blk + off + pos;
+}
+
 // One CTA per query head: the sample, its keys and the bracket [lo, hi].
-__global__ void __launch_bounds__(kSampleThreads) sample_kernel(DecodeParams p) {
+// QD of the head is staged in shared memory as in the Klow scan (the same
+// table values, so a sampled token's key equals its scan key).
+constexpr int kSampleSmem = kTable * 4;
+__global__ void __launch_bounds__(kSampleThreads, 1) sample_kernel(DecodeParams p) {
   pdl_wait();
   pdl_launch();
+  extern __shared__ float4 smem4[];
+  float* table = reinterpret_cast<float*>(smem4);
   __shared__ uint32_t s_key[kSampleMax];
   __shared__ uint32_t s_hist[2048];
   __shared__ uint32_t s_tmp[48];
   const int r = blockIdx.x, tid = threadIdx.x;
   const int b = r / p.Hq, h = r % p.Hq, kvh = h / p.g;
   const int N = p.lens[b], k = p.kcnt[b];
-  const int blk = N <= kSampleMax ? 1 : (N + kSampleMax - 1) / kSampleMax;
-  const int S = (N + blk - 1) / blk;
+  const SampleGeom gm = sample_geom(N);
+  const int S = gm.S;
   const int64_t head = (int64_t)b * p.Hkv + kvh;
   const uint32_t* plane = p.k_lo + head * kLoPlanes * p.cap;
   const uint32_t* rec = p.k_full + head * p.cap * p.rs;
-  const float* qd = p.qd + (int64_t)r * p.n;
   const uint32_t seed = lowbias32(0x9E3779B9u * (uint32_t)(head + 1));
   const int nlo = min(p.klow, kLoPlanes);
-  // up to 8 samples per thread; all their word loads are issued first
+  // up to 8 samples per thread; their plane words are requested before the
+  // table is staged, so the two round trips overlap
   constexpr int kPer = kSampleMax / kSampleThreads;
   int tt[kPer];
   uint32_t wv[kPer][kLoPlanes];
 #pragma unroll
   for (int u = 0; u < kPer; ++u) {
     const int i = tid + u * kSampleThreads;
-    tt[u] = -1;
-    if (i < S) {
-      const int len = min(blk, N - i * blk);
-      tt[u] = i * blk + (blk == 1 ? 0 : (int)(lowbias32(seed ^ (uint32_t)i) % (uint32_t)len));
-    }
+    tt[u] = i < S ? sample_token(gm, N, seed, i) : -1;
 #pragma unroll
     for (int j = 0; j < kLoPlanes; ++j)
       wv[u][j] = (tt[u] >= 0 && j < nlo) ? __ldg(plane + j * p.cap + tt[u]) : 0u;
   }
+  stage_table(table, p.qd + (int64_t)r * p.n, p.n);
+  __syncthreads();
 #pragma unroll
   for (int u = 0; u < kPer; ++u) {
     if (tt[u] < 0) continue;
     float s = 0.0f;
 #pragma unroll
-    for (int j = 0; j < kLoPlanes; ++j) {
-      const uint32_t idx = word_idx(wv[u][j]);
-      s = fmaf(word_coef(wv[u][j]), idx < (uint32_t)p.n ? __ldg(qd + idx) : 0.0f, s);
-    }
+    for (int j = 0; j < kLoPlanes; ++j) s = fmaf(word_coef(wv[u][j]), table[word_idx(wv[u][j])], s);
     for (int j = kLoPlanes; j < p.klow; ++j) {
       const uint32_t wj = __ldg(rec + (int64_t)tt[u] * p.rs + j);
-      const uint32_t idx = word_idx(wj);
-      s = fmaf(word_coef(wj), idx < (uint32_t)p.n ? __ldg(qd + idx) : 0.0f, s);
+      s = fmaf(word_coef(wj), table[word_idx(wj)], s);
     }
     s_key[tid + u * kSampleThreads] = score_key(s);
   }
@@ -858,10 +976,58 @@ __global__ void __launch_bounds__(kSampleThreads) sample_kernel(DecodeParams p) 
     rhi = a < 1.0 ? 0 : (int)a;
     rlo = c > (double)S ? S + 1 : (int)c;
   }
-  uint32_t hi = 0xFFFFFFFFu, lo = 0u, cnt, rit;
+  // Both ends from ONE histogram of the sample keys over their own range
+  // (2048 bins of (key - min) >> shift): hi is the upper edge of the bin
+  // holding the rhi-th largest key, lo the lower edge of the bin holding
+  // the rlo-th.  That widens the bracket by at most one bin on each side
+  // (a few sampled keys), never narrows it, and saves the further passes
+  // of an exact rank search (the bracket need not be exact; the selection
+  // is).
+  uint32_t hi = 0xFFFFFFFFu, lo = 0u;
   bool bad = false;
-  if (rhi >= 1) hi = rank_desc(s_key, S, (uint32_t)rhi, s_hist, s_tmp, cnt, rit, bad);
-  if (!bad && rlo <= S) lo = rank_desc(s_key, S, (uint32_t)rlo, s_hist, s_tmp, cnt, rit, bad);
+  {
+    uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+    for (int i = tid; i < S; i += kSampleThreads) {
+      mn = min(mn, s_key[i]);
+      mx = max(mx, s_key[i]);
+    }
+    mx = warp_umax(mx);
+    mn = ~warp_umax(~mn);
+    const int lane = tid & 31, warp = tid >> 5;
+    if (lane == 0) {
+      s_tmp[warp] = mx;
+      s_hist[warp] = mn;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t a = s_tmp[lane], c = s_hist[lane];
+      a = warp_umax(a);
+      c = ~warp_umax(~c);
+      if (lane == 0) {
+        s_tmp[40] = c;
+        s_tmp[41] = a;
+      }
+    }
+    __syncthreads();
+    const uint32_t kmn = s_tmp[40], kmx = s_tmp[41];
+    __syncthreads();
+    const uint32_t range = kmx - kmn;
+    const int shift = range < 2048u ? 0 : (32 - __clz((int)range)) - 11;
+    for (int i = tid; i < 2048; i += kSampleThreads) s_hist[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < S; i += kSampleThreads) atomicAdd(&s_hist[(s_key[i] - kmn) >> shift], 1u);
+    __syncthreads();
+    uint32_t bin, above, cnt;
+    if (rhi >= 1) {
+      block_find_desc<2048>(s_hist, (uint32_t)rhi, s_tmp, bin, above, cnt, bad);
+      const uint64_t top = (uint64_t)kmn + ((uint64_t)bin << shift) + ((1ull << shift) - 1ull);
+      hi = top < (uint64_t)kmx ? (uint32_t)top : kmx;
+    }
+    if (!bad && rlo <= S) {
+      block_find_desc<2048>(s_hist, (uint32_t)rlo, s_tmp, bin, above, cnt, bad);
+      lo = kmn + (bin << shift);
+    }
+  }
   if (tid == 0) {
     if (bad) {           // cannot happen for 1 <= rank <= S; select_kernel re-scans
       hi = 0u;
@@ -1439,8 +1605,10 @@ __global__ void __launch_bounds__(kP2Threads, 1) pass2_kernel(DecodeParams p) {
 //   phase 3  each CTA sums its slice of the atoms over the cluster's tiles
 //            and writes the normalised w[r].
 constexpr int kAttThreads = 768;
+constexpr int kAttThreadsReg = 640;          // records in registers: up to 96 per thread
 // shared memory: the QD / weight table, then a two-slot record ring
 constexpr int kAttSmem = kTable * 4 + 2 * kAttThreads * 64;
+constexpr int kAttSmemReg = kTable * 4;      // records in registers: the table only
 constexpr float kFixScale = 1048576.0f;       // 2^20
 constexpr float kFixInv = 1.0f / 1048576.0f;
 
@@ -1523,6 +1691,108 @@ __device__ __forceinline__ void for_records(const int32_t* list, int e0, int e1,
 }
 // for_records without a per-entry value
 __device__ __forceinline__ float no_pay(int, int) { return 0.0f; }
+
+// 16 bytes of read-only global memory, not allocated in L1 (the records
+// are read once), under the L2 eviction policy pol (createpolicy);
+// kLine also asks L2 to fetch the whole 128-byte line.
+template <bool kLine>
+__device__ __forceinline__ uint4 ld_record16(const uint4* a, uint64_t pol) {
+  uint4 v;
+  if (kLine)
+    asm("ld.global.nc.L1::no_allocate.L2::cache_hint.L2::128B.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(a), "l"(pol));
+  else
+    asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(a), "l"(pol));
+  return v;
+}
+// L2 policies: keep a line (evict last) / let it go first
+__device__ __forceinline__ uint64_t l2_evict_last() {
+  uint64_t pol;
+  asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// for_records with the records in registers instead of a shared-memory
+// ring: each thread holds the records of its next two entries (four
+// 16-byte loads each, issued a whole entry ahead of their use) and
+// prefetches the records two entries further into L2; no shared-memory
+// traffic is spent on moving records.  Same contract as for_records.
+// kLine (the key pass over interleaved records): the whole 128-byte line
+// is fetched and marked evict-last in L2, so the value record next to the
+// key record is still there for the value pass, which reads with
+// evict-first (each line is done with after it).
+template <bool kLine, class Pay, class F>
+__device__ __forceinline__ void for_records_reg(const int32_t* list, int e0, int e1,
+                                                const uint4* rec, int rs4, int Nb, WsHeader* hdr,
+                                                uint32_t tag, Pay pay, F f) {
+  constexpr int T = kAttThreadsReg;
+  const int tid = threadIdx.x;
+  const uint64_t pol = kLine ? l2_evict_last() : (rs4 == 8 ? l2_evict_first() : 0ull);
+  const bool use_pol = kLine || rs4 == 8;
+  auto list_at = [&](int i) -> int { return i < e1 ? __ldg(list + i) : -1; };
+  auto ok = [&](int t) { return (unsigned)t < (unsigned)Nb; };
+  auto load = [&](int t, uint4 (&w)[4]) {
+    if (ok(t)) {
+      const uint4* a = rec + (int64_t)t * rs4;
+      if (use_pol) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) w[u] = ld_record16<kLine>(a + u, pol);
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+              : "=r"(w[u].x), "=r"(w[u].y), "=r"(w[u].z), "=r"(w[u].w) : "l"(a + u));
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) w[u] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  auto prefetch = [&](int t) {
+    if (ok(t)) {
+      const uint4* a = rec + (int64_t)t * rs4;
+      if (kLine)
+        asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], 128, %1;" ::"l"(a),
+                     "l"(pol)
+                     : "memory");
+      else
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], 64;" ::"l"(a) : "memory");
+    }
+  };
+  int i = e0 + tid;
+  if (i >= e1) return;
+  int t0 = list_at(i), t1 = list_at(i + T), t2 = list_at(i + 2 * T), t3 = list_at(i + 3 * T);
+  uint4 w0[4], w1[4];
+  load(t0, w0);
+  float x0 = ok(t0) ? pay(i, t0) : 0.0f;
+  load(t1, w1);
+  float x1 = ok(t1) ? pay(i + T, t1) : 0.0f;
+  prefetch(t2);
+  prefetch(t3);
+  for (; i < e1; i += 2 * T) {
+    if (ok(t0)) f(i, t0, w0, x0);
+    else record_error(hdr, SDK_ERR_DEVICE_CHECK, tag);
+    t0 = t2;
+    load(t0, w0);
+    x0 = ok(t0) ? pay(i + 2 * T, t0) : 0.0f;
+    t2 = list_at(i + 4 * T);
+    prefetch(t2);
+    if (i + T >= e1) break;
+    if (ok(t1)) f(i + T, t1, w1, x1);
+    else record_error(hdr, SDK_ERR_DEVICE_CHECK, tag);
+    t1 = t3;
+    load(t1, w1);
+    x1 = ok(t1) ? pay(i + 3 * T, t1) : 0.0f;
+    t3 = list_at(i + 5 * T);
+    prefetch(t3);
+  }
+}
 
 // x = h0 + h1 + h2 in bf16 parts, each the bf16 rounding of what the
 // previous parts leave (the remainder is below 2^-24 |x| for normal x)
@@ -1627,8 +1897,10 @@ __device__ __forceinline__ unsigned long long block_sum_u64(unsigned long long v
   return r;
 }
 
-template <bool kAll16, bool kCheck>
-__global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, int C) {
+template <bool kAll16, bool kCheck, bool kReg>
+__global__ void __launch_bounds__(kReg ? kAttThreadsReg : kAttThreads, 1)
+    attend_kernel(DecodeParams p, int C) {
+  constexpr int kT = kReg ? kAttThreadsReg : kAttThreads;
   pdl_wait();     // nothing global is touched before the previous kernel is done
   pdl_launch();
   extern __shared__ float4 smem4[];
@@ -1662,6 +1934,13 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
   const int rs4 = p.rs / 4;
   const int32_t* list = p.list + (int64_t)r * p.L;
   float* ss = p.sel_score + (int64_t)r * p.L;
+  // the records of list entries [a0, a1): in registers (kReg) or through
+  // the shared-memory ring
+  auto recs = [&](auto line, int a0, int a1, const uint4* rc, uint32_t tag, auto pay, auto f) {
+    constexpr bool kL = decltype(line)::value;
+    if constexpr (kReg) for_records_reg<kL>(list, a0, a1, rc, rs4, Nb, p.hdr, tag, pay, f);
+    else for_records<kL>(list, a0, a1, rc, rs4, Nb, p.hdr, tag, ring, pay, f);
+  };
   const uint32_t* keys = p.keys + (int64_t)r * p.L;
   const float scale = p.scale;
   const int khigh = p.khigh;
@@ -1691,12 +1970,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
   __syncthreads();
   float smax = -INFINITY, zrun = 0.0f;     // online softmax of this thread
   float smin = INFINITY;                   // for the integer softmax's scale
-  auto key_pass = [&](auto line, auto f) {
-    if constexpr (decltype(line)::value)
-      for_records<true>(list, s0, s1, krec, rs4, Nb, p.hdr, 0x30000000u | r, ring, no_pay, f);
-    else
-      for_records<false>(list, s0, s1, krec, rs4, Nb, p.hdr, 0x30000000u | r, ring, no_pay, f);
-  };
+  auto key_pass = [&](auto line, auto f) { recs(line, s0, s1, krec, 0x30000000u | r, no_pay, f); };
   auto rescore = 
               [&](int i, int t, const uint4 (&w)[4], float) {
                 float s = 0.0f;
@@ -1733,7 +2007,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
     // z: the own selected entries (rescaled to m) and complement entries
     float z = smax > -INFINITY ? zrun * expf(smax - m) : 0.0f;
 #pragma unroll 4
-    for (int i = c0 + tid; i < c1; i += kAttThreads) {
+    for (int i = c0 + tid; i < c1; i += kT) {
       const int t = list[i];
       if ((unsigned)t < (unsigned)Nb) z += expf(scale * key_score(keys[t]) - m);
     }
@@ -1749,7 +2023,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
     // the smallest logit of the domain (own selected and complement
     // entries), then the INT16 scale, the integer exponentials and their sum
 #pragma unroll 4
-    for (int i = c0 + tid; i < c1; i += kAttThreads) {
+    for (int i = c0 + tid; i < c1; i += kT) {
       const int t = list[i];
       if ((unsigned)t < (unsigned)Nb) smin = fminf(smin, scale * key_score(keys[t]));
     }
@@ -1763,9 +2037,9 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
     const float lo_abs = lo < INFINITY ? fabsf(lo) : 0.0f;
     ic = isoft_setup(fmaxf(hi_abs, lo_abs), m > -INFINITY ? m : 0.0f);
     unsigned long long e = 0ull;
-    for (int i = s0 + tid; i < s1; i += kAttThreads) e += isoft_exp(ss[i], ic);
+    for (int i = s0 + tid; i < s1; i += kT) e += isoft_exp(ss[i], ic);
 #pragma unroll 4
-    for (int i = c0 + tid; i < c1; i += kAttThreads) {
+    for (int i = c0 + tid; i < c1; i += kT) {
       const int t = list[i];
       if ((unsigned)t < (unsigned)Nb) e += isoft_exp(scale * key_score(keys[t]), ic);
     }
@@ -1800,7 +2074,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
     constexpr bool kFloat = decltype(fl)::value;
     {
       uint4* t4 = reinterpret_cast<uint4*>(smem4);
-      for (int i = tid; i < kTable / 4; i += kAttThreads) t4[i] = make_uint4(0u, 0u, 0u, 0u);
+      for (int i = tid; i < kTable / 4; i += kT) t4[i] = make_uint4(0u, 0u, 0u, 0u);
     }
     __syncthreads();
     // fixed point: p already carries the 2^20 scale
@@ -1830,11 +2104,11 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
     };
     // the logits load with the records: the rescored ones, and with the
     // flag the complement's scale * s_lo
-    for_records<false>(list, s0, s1, vrec, rs4, Nb, p.hdr, 0x31000000u | r, ring,
+    recs(std::false_type{}, s0, s1, vrec, 0x31000000u | r,
                 [&](int i, int) { return ss[i]; },
                 [&](int, int, const uint4 (&w)[4], float lg) { scatter(lg, w); });
     if (p.full)
-      for_records<false>(list, c0, c1, vrec, rs4, Nb, p.hdr, 0x32000000u | r, ring,
+      recs(std::false_type{}, c0, c1, vrec, 0x32000000u | r,
                   [&](int, int t) { return scale * key_score(keys[t]); },
                   [&](int, int, const uint4 (&w)[4], float lg) { scatter(lg, w); });
     // int32 range guard (also catches NaN): sum |p c| * 2^20 < 2^30
@@ -1863,7 +2137,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(DecodeParams p, 
       isf[cc] = *cluster.map_shared_rank(&s_float, cc) != 0;
     }
   }
-  for (int g = g0 + tid; g < g1; g += kAttThreads) {
+  for (int g = g0 + tid; g < g1; g += kT) {
     int4 v[8];
 #pragma unroll
     for (int cc = 0; cc < 8; ++cc)
@@ -2072,6 +2346,17 @@ static bool pdl_enabled() {
   return on == 1;
 }
 
+// The attention kernel streams records through a shared-memory ring when
+// SDK_ATTEND_RING=1, else through registers.
+static bool attend_ring() {
+  static int on = -1;
+  if (on < 0) {
+    const char* v = getenv("SDK_ATTEND_RING");
+    on = (v != nullptr && v[0] == '1') ? 1 : 0;
+  }
+  return on == 1;
+}
+
 // QD on the tensor cores (three bf16 parts of q) unless SDK_DECODE_QD_TC=0.
 static bool qd_tensor_cores() {
   static int on = -1;
@@ -2202,10 +2487,11 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
   static unsigned long long attr_set = 0ull;
   if (device_needs_setup(&attr_set)) {
     cudaFuncSetAttribute(klow_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kTable * 4 + 4096 * 4);
+                         kKlowSmemHist);
     cudaFuncSetAttribute(klow_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kTable * 4 + 4096 * 4);
+                         kKlowSmemBracket);
     cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelSmem);
+    cudaFuncSetAttribute(sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSampleSmem);
     cudaFuncSetAttribute(pass2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPass2Smem);
     cudaFuncSetAttribute(final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          2 * kFinalStage * 4);
@@ -2218,14 +2504,22 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
     cudaFuncSetAttribute(out_kernel<64, 2, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          out_smem_bytes(64, 2, 4));
 
-    cudaFuncSetAttribute(attend_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kAttSmem);
-    cudaFuncSetAttribute(attend_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kAttSmem);
-    cudaFuncSetAttribute(attend_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kAttSmem);
-    cudaFuncSetAttribute(attend_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kAttSmem);
+    cudaFuncSetAttribute(attend_kernel<true, true, false>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, kAttSmem);
+    cudaFuncSetAttribute(attend_kernel<true, false, false>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, kAttSmem);
+    cudaFuncSetAttribute(attend_kernel<false, true, false>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, kAttSmem);
+    cudaFuncSetAttribute(attend_kernel<false, false, false>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, kAttSmem);
+    cudaFuncSetAttribute(attend_kernel<true, true, true>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, kAttSmemReg);
+    cudaFuncSetAttribute(attend_kernel<true, false, true>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, kAttSmemReg);
+    cudaFuncSetAttribute(attend_kernel<false, true, true>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, kAttSmemReg);
+    cudaFuncSetAttribute(attend_kernel<false, false, true>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, kAttSmemReg);
     device_setup_done(&attr_set);
   }
   cudaError_t e = cudaSuccess;
@@ -2259,12 +2553,13 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
     const int g = scan_grid(p.tok_off[p.B], p.R, kKlowSegCost, 2048, sms);
     const int vec = (p.cap % 4 == 0) && ((reinterpret_cast<uintptr_t>(p.k_lo) & 15u) == 0u);
     if (p.bracket) {
-      e = launch_pdl(sample_kernel, dim3(p.R), dim3(kSampleThreads), 0, stream, 1, p);
+      e = launch_pdl(sample_kernel, dim3(p.R), dim3(kSampleThreads), (size_t)kSampleSmem, stream,
+                     1, p);
       if (e != cudaSuccess) return SDK_ERR_CUDA;
-      e = launch_pdl(klow_kernel<true>, dim3(g), dim3(kKlowThreads), (size_t)kTable * 4 + 4096 * 4,
+      e = launch_pdl(klow_kernel<true>, dim3(g), dim3(kKlowThreads), (size_t)kKlowSmemBracket,
                      stream, 1, p, vec);
     } else {
-      e = launch_pdl(klow_kernel<false>, dim3(g), dim3(kKlowThreads), (size_t)kTable * 4 + 4096 * 4,
+      e = launch_pdl(klow_kernel<false>, dim3(g), dim3(kKlowThreads), (size_t)kKlowSmemHist,
                      stream, 1, p, vec);
     }
     if (e != cudaSuccess) return SDK_ERR_CUDA;
@@ -2296,10 +2591,13 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
     int C = 1;
     while (C < 8 && (int64_t)p.R * C * 2 <= sms && dmax / (2 * C) >= 1024) C *= 2;
     const bool all16 = p.khigh == kAtoms, check = p.n < kTable;
-    auto kern = all16 ? (check ? attend_kernel<true, true> : attend_kernel<true, false>)
-                      : (check ? attend_kernel<false, true> : attend_kernel<false, false>);
-    e = launch_pdl(kern, dim3((unsigned)(p.R * C)), dim3(kAttThreads), (size_t)kAttSmem, stream,
-                   (unsigned)C, p, C);
+    const bool reg = !attend_ring();
+    auto kern = reg ? (all16 ? (check ? attend_kernel<true, true, true> : attend_kernel<true, false, true>)
+                             : (check ? attend_kernel<false, true, true> : attend_kernel<false, false, true>))
+                    : (all16 ? (check ? attend_kernel<true, true, false> : attend_kernel<true, false, false>)
+                             : (check ? attend_kernel<false, true, false> : attend_kernel<false, false, false>));
+    e = launch_pdl(kern, dim3((unsigned)(p.R * C)), dim3(reg ? kAttThreadsReg : kAttThreads),
+                   (size_t)(reg ? kAttSmemReg : kAttSmem), stream, (unsigned)C, p, C);
     if (e != cudaSuccess) return SDK_ERR_CUDA;
     if (t1 != nullptr && timing_record(t1, stream) != cudaSuccess) return SDK_ERR_CUDA;
   }

@@ -107,21 +107,27 @@ __device__ __forceinline__ float pow2_scale(float amax) {
   return ldexpf(1.0f, min(14 - (ex - 127), 126));
 }
 
+// One or two streams (e.g. the keys and the values of an append), each
+// with its own vectors, dictionary, codes and residual energies; the
+// row tiles of stream 0 come first, then those of stream 1, so one launch
+// spreads the tiles of both over the SMs.
 struct TcParams {
-  const void* x;
+  const void* x[2];
   int x_dtype;
-  int64_t n_vec;
-  const uint16_t* dict;
+  int64_t n_vec[2];
+  const uint16_t* dict[2];
   int n;
   int k_atoms;
-  uint32_t* codes;
-  float* rsq;
+  uint32_t* codes[2];
+  float* rsq[2];
   WsHeader* hdr;
   float* resid;        // [grid][D][kTileRows] fp32
-  // dictionary statistics: [0] max_i ||d_i||, [1] max_i ||t d_i - fp16(t d_i)||
-  // (f16 operands; 0 for bf16), [2] max_ij |d_ij| as bits; t = dict_scale([2])
-  const float* dmax;
-  int n_tiles;
+  // dictionary statistics per stream: [0] max_i ||d_i||, [1] max_i
+  // ||t d_i - fp16(t d_i)|| (f16 operands; 0 for bf16), [2] max_ij |d_ij| as
+  // bits; t = dict_scale([2])
+  const float* dmax[2];
+  int tiles0;          // row tiles of stream 0
+  int n_tiles;         // row tiles of both streams
   int n_atom_tiles;
 };
 
@@ -149,7 +155,8 @@ __device__ __forceinline__ float bf16_round(float v) {
 // ---- the kernel --------------------------------------------------------------
 template <int D, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
-    encode_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcParams p) {
+    encode_tc_kernel(const __grid_constant__ CUtensorMap tmap0,
+                     const __grid_constant__ CUtensorMap tmap1, TcParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem_1k(smem_raw);
@@ -222,8 +229,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_expect_tx(bar_full(stage), (uint32_t)C::kStageBytes);
 #pragma unroll
             for (int kb = 0; kb < C::KB; ++kb)
-              tma_load_2d(sB + stage * C::kStageBytes + kb * (kAtomTile * 128), &tmap, kb * 64,
-                          a * kAtomTile, bar_full(stage));
+              tma_load_2d(sB + stage * C::kStageBytes + kb * (kAtomTile * 128),
+                          tile < p.tiles0 ? &tmap0 : &tmap1, kb * 64, a * kAtomTile,
+                          bar_full(stage));
             issued_mask |= 1u << stage;
             last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
             if (++stage == kStages) {
@@ -305,6 +313,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // scans 64 of the 128 columns of one residual row per atom tile; the
     // "lead" thread of the row (column half 0) merges both candidate lists
     // at the end of a step, picks, and updates the residual.
+    // the current row tile's stream
+    const uint16_t* cdict = p.dict[0];
+    const float* cdmax = p.dmax[0];
+    uint32_t* ccodes = p.codes[0];
+    float* crsq = p.rsq[0];
     const int e = warp - 2;
     const int combo = e >> 2;
     const int rs = combo >> 1, half = combo & 1;
@@ -324,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the operand atom norms ||fp16(t d_i)||
     // (read where used, to keep them out of the scan loop's registers)
     auto tdict_of = [&] {
-      return F16 ? pow2_scale(__int_as_float(__ldg(reinterpret_cast<const int*>(p.dmax) + 2)))
+      return F16 ? pow2_scale(__int_as_float(__ldg(reinterpret_cast<const int*>(cdmax) + 2)))
                  : 1.0f;
     };
     uint8_t* arow = smem + C::kOffA + rs * C::kABytes + rin * 128;
@@ -378,14 +391,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // twice the bound on |c~ - s c| (scaled units): rounding of s r
       // (Cauchy-Schwarz with the largest operand atom norm), conversion of
       // the dictionary to the operand type, and slack for the accumulation
-      const float econv = F16 ? __ldg(p.dmax + 1) : 0.0f;
-      const float dmax = __ldg(p.dmax) * tdict_of() + econv;
+      const float econv = F16 ? __ldg(cdmax + 1) : 0.0f;
+      const float dmax = __ldg(cdmax) * tdict_of() + econv;
       const float rn = sqrtf(n2);
       return 2.0f * dmax * sqrtf(e2) + 2.0f * econv * rn + 0.000244140625f * dmax * rn;
     };
     // fp32 correlation in k order (the CUDA-core encoder's arithmetic)
     auto dot_atom = [&](uint32_t i) {
-      const uint4* dp = reinterpret_cast<const uint4*>(p.dict + (int64_t)i * D);
+      const uint4* dp = reinterpret_cast<const uint4*>(cdict + (int64_t)i * D);
       float sd = 0.0f;
 #pragma unroll 4
       for (int kc = 0; kc < D / 8; ++kc) {
@@ -404,8 +417,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto cand_val = [](uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); };
 
     for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
-      const int64_t grow = (int64_t)tile * kTileRows + row;
-      const bool valid = grow < p.n_vec;
+      const int sidx = tile < p.tiles0 ? 0 : 1;
+      cdict = p.dict[sidx];
+      cdmax = p.dmax[sidx];
+      ccodes = p.codes[sidx];
+      crsq = p.rsq[sidx];
+      const void* cx = p.x[sidx];
+      const int64_t grow = (int64_t)(tile - (sidx ? p.tiles0 : 0)) * kTileRows + row;
+      const bool valid = grow < p.n_vec[sidx];
       if (lead && !*s_abort) {
         // residual <- x; A <- operand(scale * x)
         float amax = 0.0f;
@@ -415,13 +434,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (valid) {
             if (p.x_dtype == SDK_F32) {
               const float4* xp = reinterpret_cast<const float4*>(
-                  reinterpret_cast<const float*>(p.x) + grow * D + kc * 8);
+                  reinterpret_cast<const float*>(cx) + grow * D + kc * 8);
               const float4 xa = __ldg(xp), xb = __ldg(xp + 1);
               r8[0] = xa.x; r8[1] = xa.y; r8[2] = xa.z; r8[3] = xa.w;
               r8[4] = xb.x; r8[5] = xb.y; r8[6] = xb.z; r8[7] = xb.w;
             } else {
               const uint4 xv = __ldg(reinterpret_cast<const uint4*>(
-                  reinterpret_cast<const uint16_t*>(p.x) + grow * D + kc * 8));
+                  reinterpret_cast<const uint16_t*>(cx) + grow * D + kc * 8));
               const uint32_t vw[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
@@ -610,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int e2 = 0; e2 < kCand; ++e2) {
                 if (!ok_e[e2]) continue;
-                const uint4 dv = __ldg(reinterpret_cast<const uint4*>(p.dict + (int64_t)ix[e2] * D) + kc);
+                const uint4 dv = __ldg(reinterpret_cast<const uint4*>(cdict + (int64_t)ix[e2] * D) + kc);
                 float sd = acc[e2];
                 sd = fmaf(r8[0], bf16_lo(dv.x), sd);
                 sd = fmaf(r8[1], bf16_hi(dv.x), sd);
@@ -687,7 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t bi = 0u;
 #pragma unroll 1
             for (int i = lane; i < p.n; i += 32) {
-              const uint4* dp = reinterpret_cast<const uint4*>(p.dict + (int64_t)i * D);
+              const uint4* dp = reinterpret_cast<const uint4*>(cdict + (int64_t)i * D);
               float sd = 0.0f;
 #pragma unroll 4
               for (int kc = 0; kc < D / 8; ++kc) {
@@ -731,12 +750,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             pick = 0u;
             coef = 0.0f;
           }
-          if (valid) p.codes[grow * p.k_atoms + j] = make_word(coef, pick);
+          if (valid) ccodes[grow * p.k_atoms + j] = make_word(coef, pick);
 
           // residual update r -= coef * d_pick; next A operand
           if (active) {
             float amax = 0.0f;
-            const uint4* dp = reinterpret_cast<const uint4*>(p.dict + (int64_t)pick * D);
+            const uint4* dp = reinterpret_cast<const uint4*>(cdict + (int64_t)pick * D);
 #pragma unroll 1
             for (int kc = 0; kc < D / 8; ++kc) {
               const uint4 dv = __ldg(dp + kc);
@@ -780,13 +799,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ru < (uint32_t)p.n) best_next = fabsf(dot_atom(ru)) * s_scl[row] * tdict_of() - 0.5f * band;
         }
       }
-      if (lead && valid && p.rsq != nullptr && !*s_abort) {
+      if (lead && valid && crsq != nullptr && !*s_abort) {
         float sq = 0.0f;
         for (int k = 0; k < D; ++k) {
           const float r = rres[k * kTileRows];
           sq = fmaf(r, r, sq);
         }
-        p.rsq[grow] = sq;
+        crsq[grow] = sq;
       }
     }
     n_rescored = __reduce_add_sync(0xffffffffu, n_rescored);
@@ -897,29 +916,40 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 }  // namespace tc
 
-// scratch: 256 B of dictionary statistics, the fp16 operand copy of the
-// dictionary (256-byte aligned), then one fp32 residual tile per CTA
+// scratch: 256 B of dictionary statistics per stream, the fp16 operand
+// copy of every stream's dictionary (256-byte aligned), then one fp32
+// residual tile per CTA
 static size_t dict_copy_bytes(int head_dim, int n_atoms) {
   return ((size_t)n_atoms * head_dim * 2 + 255) & ~(size_t)255;
 }
 
-size_t encode_tc_scratch_bytes(int64_t n_vec, int head_dim, int n_atoms) {
+size_t encode_tc_scratch_bytes(int64_t n_vec, int head_dim, int n_atoms, int streams) {
   if ((head_dim != 64 && head_dim != 128) || n_vec <= 0) return 256;
-  int64_t tiles = (n_vec + tc::kTileRows - 1) / tc::kTileRows;
+  int64_t tiles = (n_vec + tc::kTileRows - 1) / tc::kTileRows + (streams - 1);
   if (tiles > tc::kMaxCtas) tiles = tc::kMaxCtas;
-  return 256 + dict_copy_bytes(head_dim, n_atoms) + (size_t)tiles * head_dim * tc::kTileRows * 4;
+  return (size_t)streams * (256 + dict_copy_bytes(head_dim, n_atoms)) +
+         (size_t)tiles * head_dim * tc::kTileRows * 4;
 }
 
-sdk_status launch_encode_tc(const EncodeParams& p, int head_dim, void* scratch,
+sdk_status launch_encode_tc(const EncodeParams* ps, int streams, int head_dim, void* scratch,
                             size_t scratch_bytes, cudaStream_t stream, bool* taken) {
   *taken = false;
   if (head_dim != 64 && head_dim != 128) return SDK_OK;
-  if (p.n_vec <= 0) return SDK_OK;
-  // vectorised 16-byte loads of x rows need a 16-byte aligned x
-  if ((reinterpret_cast<uintptr_t>(p.x) & 15u) != 0u) return SDK_OK;
+  if (streams < 1 || streams > 2) return SDK_OK;
+  if (streams == 2 && (ps[1].n != ps[0].n || ps[1].k_atoms != ps[0].k_atoms ||
+                       ps[1].x_dtype != ps[0].x_dtype))
+    return SDK_OK;
+  int64_t tiles_s[2] = {0, 0};
+  for (int s = 0; s < streams; ++s) {
+    if (ps[s].n_vec <= 0) return SDK_OK;
+    // vectorised 16-byte loads of x rows need a 16-byte aligned x
+    if ((reinterpret_cast<uintptr_t>(ps[s].x) & 15u) != 0u) return SDK_OK;
+    tiles_s[s] = (ps[s].n_vec + tc::kTileRows - 1) / tc::kTileRows;
+  }
   auto fn = tc::encode_fn();
   if (fn == nullptr) return SDK_OK;  // no driver entry point: CUDA-core path
-  const int64_t tiles = (p.n_vec + tc::kTileRows - 1) / tc::kTileRows;
+  const EncodeParams& p = ps[0];
+  const int64_t tiles = tiles_s[0] + tiles_s[1];
   int64_t grid = tiles;
   const int sms = num_sms();
   if (grid > sms) grid = sms;
@@ -927,45 +957,58 @@ sdk_status launch_encode_tc(const EncodeParams& p, int head_dim, void* scratch,
   const bool f16 = tc::operands_f16();
   const size_t per_cta = (size_t)head_dim * tc::kTileRows * 4;
   const size_t dict_bytes = dict_copy_bytes(head_dim, p.n);
-  if (scratch_bytes < 256 + dict_bytes + (size_t)grid * per_cta) return SDK_ERR_CAPACITY;
-  float* stats = reinterpret_cast<float*>(scratch);
-  __half* dict16 = reinterpret_cast<__half*>(reinterpret_cast<char*>(scratch) + 256);
+  const size_t per_stream = 256 + dict_bytes;
+  if (scratch_bytes < (size_t)streams * per_stream + (size_t)grid * per_cta) return SDK_ERR_CAPACITY;
 
-  CUtensorMap map;
-  const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)p.n};
-  const cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
-  const cuuint32_t box[2] = {64u, (cuuint32_t)tc::kAtomTile};
-  const cuuint32_t estr[2] = {1u, 1u};
-  void* base = f16 ? static_cast<void*>(dict16) : const_cast<uint16_t*>(p.dict);
-  CUresult cr = fn(&map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                   base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (cr != CUDA_SUCCESS) return SDK_ERR_INVALID_ARG;
+  CUtensorMap maps[2];
+  float* stats[2];
+  __half* dict16[2];
+  for (int s = 0; s < streams; ++s) {
+    char* base_s = reinterpret_cast<char*>(scratch) + (size_t)s * per_stream;
+    stats[s] = reinterpret_cast<float*>(base_s);
+    dict16[s] = reinterpret_cast<__half*>(base_s + 256);
+    const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)p.n};
+    const cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)tc::kAtomTile};
+    const cuuint32_t estr[2] = {1u, 1u};
+    void* base = f16 ? static_cast<void*>(dict16[s]) : const_cast<uint16_t*>(ps[s].dict);
+    CUresult cr = fn(&maps[s], f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                     2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return SDK_ERR_INVALID_ARG;
+  }
+  if (streams == 1) maps[1] = maps[0];
   *taken = true;
 
-  if (cudaMemsetAsync(stats, 0, 4 * sizeof(float), stream) != cudaSuccess) return SDK_ERR_CUDA;
   const unsigned dgrid = (unsigned)((p.n + 127) / 128);
-  if (head_dim == 128) {
-    tc::dict_stats_kernel<128><<<dgrid, 128, 0, stream>>>(p.dict, p.n, stats);
-    if (f16) tc::dict_f16_kernel<128><<<dgrid, 128, 0, stream>>>(p.dict, p.n, stats, dict16);
-  } else {
-    tc::dict_stats_kernel<64><<<dgrid, 128, 0, stream>>>(p.dict, p.n, stats);
-    if (f16) tc::dict_f16_kernel<64><<<dgrid, 128, 0, stream>>>(p.dict, p.n, stats, dict16);
+  for (int s = 0; s < streams; ++s) {
+    if (cudaMemsetAsync(stats[s], 0, 4 * sizeof(float), stream) != cudaSuccess) return SDK_ERR_CUDA;
+    if (head_dim == 128) {
+      tc::dict_stats_kernel<128><<<dgrid, 128, 0, stream>>>(ps[s].dict, p.n, stats[s]);
+      if (f16) tc::dict_f16_kernel<128><<<dgrid, 128, 0, stream>>>(ps[s].dict, p.n, stats[s], dict16[s]);
+    } else {
+      tc::dict_stats_kernel<64><<<dgrid, 128, 0, stream>>>(ps[s].dict, p.n, stats[s]);
+      if (f16) tc::dict_f16_kernel<64><<<dgrid, 128, 0, stream>>>(ps[s].dict, p.n, stats[s], dict16[s]);
+    }
   }
 
   tc::TcParams tp;
-  tp.x = p.x;
+  for (int s = 0; s < 2; ++s) {
+    const int u = s < streams ? s : 0;
+    tp.x[s] = ps[u].x;
+    tp.n_vec[s] = s < streams ? ps[s].n_vec : 0;
+    tp.dict[s] = ps[u].dict;
+    tp.codes[s] = ps[u].codes;
+    tp.rsq[s] = ps[u].rsq;
+    tp.dmax[s] = stats[u];
+  }
   tp.x_dtype = p.x_dtype;
-  tp.n_vec = p.n_vec;
-  tp.dict = p.dict;
   tp.n = p.n;
   tp.k_atoms = p.k_atoms;
-  tp.codes = p.codes;
-  tp.rsq = p.rsq;
   tp.hdr = p.hdr;
-  tp.resid = reinterpret_cast<float*>(reinterpret_cast<char*>(scratch) + 256 + dict_bytes);
-  tp.dmax = stats;
+  tp.resid = reinterpret_cast<float*>(reinterpret_cast<char*>(scratch) + (size_t)streams * per_stream);
+  tp.tiles0 = (int)tiles_s[0];
   tp.n_tiles = (int)tiles;
   tp.n_atom_tiles = (p.n + tc::kAtomTile - 1) / tc::kAtomTile;
 
@@ -984,14 +1027,14 @@ sdk_status launch_encode_tc(const EncodeParams& p, int head_dim, void* scratch,
   const dim3 g((unsigned)grid);
   if (head_dim == 128) {
     if (f16)
-      tc::encode_tc_kernel<128, true><<<g, tc::kThreads, tc::Cfg<128>::kSmem, stream>>>(map, tp);
+      tc::encode_tc_kernel<128, true><<<g, tc::kThreads, tc::Cfg<128>::kSmem, stream>>>(maps[0], maps[1], tp);
     else
-      tc::encode_tc_kernel<128, false><<<g, tc::kThreads, tc::Cfg<128>::kSmem, stream>>>(map, tp);
+      tc::encode_tc_kernel<128, false><<<g, tc::kThreads, tc::Cfg<128>::kSmem, stream>>>(maps[0], maps[1], tp);
   } else {
     if (f16)
-      tc::encode_tc_kernel<64, true><<<g, tc::kThreads, tc::Cfg<64>::kSmem, stream>>>(map, tp);
+      tc::encode_tc_kernel<64, true><<<g, tc::kThreads, tc::Cfg<64>::kSmem, stream>>>(maps[0], maps[1], tp);
     else
-      tc::encode_tc_kernel<64, false><<<g, tc::kThreads, tc::Cfg<64>::kSmem, stream>>>(map, tp);
+      tc::encode_tc_kernel<64, false><<<g, tc::kThreads, tc::Cfg<64>::kSmem, stream>>>(maps[0], maps[1], tp);
   }
   return cudaGetLastError() == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
 }

@@ -266,11 +266,14 @@ sdk_status timing_enable(bool on);
 int timing_read(float* ms_out, int max_n);
 sdk_decode_layout decode_layout(int B, int Hq, int d, int n, int64_t L);
 sdk_status launch_encode_simt(const EncodeParams& p, int head_dim, cudaStream_t stream);
-// Tensor-core encoder; sets *taken = false when it does not handle the
-// shape (the caller then runs the CUDA-core encoder).
-sdk_status launch_encode_tc(const EncodeParams& p, int head_dim, void* scratch,
+// Tensor-core encoder of one or two streams (ps[0..streams-1]; two
+// streams need equal n, k_atoms and x_dtype) in one launch; sets *taken =
+// false when it does not handle the shape (the caller then runs the
+// CUDA-core encoder).
+sdk_status launch_encode_tc(const EncodeParams* ps, int streams, int head_dim, void* scratch,
                             size_t scratch_bytes, cudaStream_t stream, bool* taken);
-size_t encode_tc_scratch_bytes(int64_t n_vec, int head_dim, int n_atoms);
+// scratch of launch_encode_tc for n_vec vectors in all over `streams` streams
+size_t encode_tc_scratch_bytes(int64_t n_vec, int head_dim, int n_atoms, int streams = 1);
 
 // Atom-parallel encoder for a few vectors of one or two streams (rows per
 // call: 64 in total, the second stream starting at an even slot).  In

@@ -275,15 +275,24 @@ def _lowbias32(x):
 
 def _sampled_tokens(N, b, Hkv, kvh):
     """The tokens the decode's selection samples for KV head (b, kvh), by
-    the rule include/sdk.h states for the sampled bracket (one token per
-    block of ceil(N / 8192) tokens, at lowbias32(seed ^ block) mod the
-    block's length)."""
-    blk = 1 if N <= 8192 else -(-N // 8192)
-    S = -(-N // blk)
+    the rule include/sdk.h states for the sampled bracket: every token when
+    N <= 8192, else runs of 8 tokens, one per block of blk = 8 ceil(ceil(N /
+    1024) / 8) tokens, starting 8 (lowbias32(seed ^ block) mod (len / 8))
+    into the block (the whole block when it holds fewer than 8 tokens)."""
+    if N <= 8192:
+        return np.arange(N)
+    blk = 8 * ((-(-N // 1024) + 7) // 8)
+    nb = -(-N // blk)
     seed = int(_lowbias32((0x9E3779B9 * (b * Hkv + kvh + 1)) & 0xFFFFFFFF))
-    i = np.arange(S, dtype=np.uint64)
-    ln = np.minimum(blk, N - i * blk)
-    return (i * blk + _lowbias32(seed ^ i) % ln).astype(np.int64)
+    out = []
+    for i in range(nb):
+        ln = min(blk, N - i * blk)
+        if ln < 8:
+            out.extend(range(i * blk, i * blk + ln))
+        else:
+            off = 8 * int(_lowbias32(seed ^ i) % (ln // 8))
+            out.extend(range(i * blk + off, i * blk + off + 8))
+    return np.asarray(out, dtype=np.int64)
 
 
 def test_sampled_bracket_misses_on_both_sides():

@@ -425,3 +425,29 @@ def test_exchange_wait_runs_out_cleanly():
         codes, _ = _enc("sdk_encode", x, D)
         ref, _ = _enc("sdk_encode_simt", x, D)
         assert torch.equal(codes.cpu(), ref.cpu())
+
+
+@pytest.mark.parametrize("interleaved", [False, True], ids=["separate", "interleaved"])
+def test_append_both_streams_in_one_launch(interleaved):
+    """An append of 600 tokens x 8 KV heads (4800 key and 4800 value
+    vectors: 19 row tiles each, one tensor-core launch over all 38, the
+    value tiles after the key tiles, each with its own dictionary): every
+    word in the store equals the CUDA-core encoder's for its own stream,
+    bf16 and fp32 inputs."""
+    g = workloads.make_gen(57)
+    n, d, B, Hkv, n_new, cap = 32768, 128, 1, 8, 600, 640
+    DK = workloads.correlated_dictionary(n, d, g).cuda()
+    DV = workloads.gaussian_dictionary(n, d, g).cuda()
+    for dt in (torch.float32, torch.bfloat16):
+        store = sdk.CodeStore(B, Hkv, cap, interleaved=interleaved)
+        store.lens = [13]
+        xk = torch.randn(B, Hkv, n_new, d, generator=g).to(dt).cuda()
+        xv = torch.randn(B, Hkv, n_new, d, generator=g).to(dt).cuda()
+        ws = sdk.sdk_append(store, xk, xv, DK, DV)
+        torch.cuda.synchronize()
+        assert sdk.sdk_check_status(ws)[0] == 0
+        ck = sdk.sdk_encode_simt(xk, DK).view(B, Hkv, n_new, 16)
+        cv = sdk.sdk_encode_simt(xv, DV).view(B, Hkv, n_new, 16)
+        assert torch.equal(store.k_full[:, :, 13:13 + n_new], ck)
+        assert torch.equal(store.v_full[:, :, 13:13 + n_new], cv)
+        assert torch.equal(store.k_lo[:, :, :, 13:13 + n_new], ck[..., :3].transpose(-1, -2))
