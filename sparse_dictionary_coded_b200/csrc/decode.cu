@@ -30,6 +30,7 @@
 // The Klow scan and pass 2 split the layer's tokens over their CTAs with a
 // start-up cost charged per head (for_segments).
 #include <cooperative_groups.h>
+#include <stdio.h>
 #include <stdlib.h>
 #include <atomic>
 #include <mutex>
@@ -325,9 +326,10 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
   uint32_t* sh = reinterpret_cast<uint32_t*>(table + kTable);
   // bracket mode: the segment's selected tokens and candidates are
   // collected here and reserved in the global lists once per segment
+  const int cap_ab = p.klow_buf, cap_cd = p.klow_buf / 2;
   int32_t* s_ab = reinterpret_cast<int32_t*>(table + kTable);
-  int32_t* s_ct = s_ab + kKlowAboveBuf;
-  uint32_t* s_ck = reinterpret_cast<uint32_t*>(s_ct + kKlowCandBuf);
+  int32_t* s_ct = s_ab + cap_ab;
+  uint32_t* s_ck = reinterpret_cast<uint32_t*>(s_ct + cap_cd);
   __shared__ uint32_t s_cnt[2], s_base[2];
   const int n = p.n, tid = threadIdx.x, lane = tid & 31;
   const int nlo = min(p.klow, kLoPlanes);
@@ -475,7 +477,7 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
           for (int u = 0; u < 4; ++u) {
             const int t = 4 * q + u;
             if ((fa >> u) & 1u) {
-              if (pa < (uint32_t)kKlowAboveBuf) {
+              if (pa < (uint32_t)cap_ab) {
                 s_ab[pa] = t;
               } else {
                 const uint32_t g = atomicAdd(&st->n_above, 1u);
@@ -484,7 +486,7 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
               ++pa;
             }
             if ((fc >> u) & 1u) {
-              if (pc < (uint32_t)kKlowCandBuf) {
+              if (pc < (uint32_t)cap_cd) {
                 s_ct[pc] = t;
                 s_ck[pc] = kq[u];
               } else {
@@ -513,14 +515,14 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
     } else {
       // the segment's buffered entries: one global reservation per kind
       if (tid == 0) {
-        const uint32_t na = min(s_cnt[0], (uint32_t)kKlowAboveBuf);
-        const uint32_t nc = min(s_cnt[1], (uint32_t)kKlowCandBuf);
+        const uint32_t na = min(s_cnt[0], (uint32_t)cap_ab);
+        const uint32_t nc = min(s_cnt[1], (uint32_t)cap_cd);
         s_base[0] = na ? atomicAdd(&st->n_above, na) : 0u;
         s_base[1] = nc ? atomicAdd(&st->n_cand, nc) : 0u;
       }
       __syncthreads();
-      const uint32_t na = min(s_cnt[0], (uint32_t)kKlowAboveBuf);
-      const uint32_t nc = min(s_cnt[1], (uint32_t)kKlowCandBuf);
+      const uint32_t na = min(s_cnt[0], (uint32_t)cap_ab);
+      const uint32_t nc = min(s_cnt[1], (uint32_t)cap_cd);
       for (uint32_t i = tid; i < na; i += kKlowThreads) {
         const uint32_t g = s_base[0] + i;
         if (g < (uint32_t)p.L) above_out[g] = s_ab[i];
@@ -976,58 +978,10 @@ __global__ void __launch_bounds__(kSampleThreads, 1) sample_kernel(DecodeParams 
     rhi = a < 1.0 ? 0 : (int)a;
     rlo = c > (double)S ? S + 1 : (int)c;
   }
-  // Both ends from ONE histogram of the sample keys over their own range
-  // (2048 bins of (key - min) >> shift): hi is the upper edge of the bin
-  // holding the rhi-th largest key, lo the lower edge of the bin holding
-  // the rlo-th.  That widens the bracket by at most one bin on each side
-  // (a few sampled keys), never narrows it, and saves the further passes
-  // of an exact rank search (the bracket need not be exact; the selection
-  // is).
-  uint32_t hi = 0xFFFFFFFFu, lo = 0u;
+  uint32_t hi = 0xFFFFFFFFu, lo = 0u, cnt, rit;
   bool bad = false;
-  {
-    uint32_t mn = 0xFFFFFFFFu, mx = 0u;
-    for (int i = tid; i < S; i += kSampleThreads) {
-      mn = min(mn, s_key[i]);
-      mx = max(mx, s_key[i]);
-    }
-    mx = warp_umax(mx);
-    mn = ~warp_umax(~mn);
-    const int lane = tid & 31, warp = tid >> 5;
-    if (lane == 0) {
-      s_tmp[warp] = mx;
-      s_hist[warp] = mn;
-    }
-    __syncthreads();
-    if (warp == 0) {
-      uint32_t a = s_tmp[lane], c = s_hist[lane];
-      a = warp_umax(a);
-      c = ~warp_umax(~c);
-      if (lane == 0) {
-        s_tmp[40] = c;
-        s_tmp[41] = a;
-      }
-    }
-    __syncthreads();
-    const uint32_t kmn = s_tmp[40], kmx = s_tmp[41];
-    __syncthreads();
-    const uint32_t range = kmx - kmn;
-    const int shift = range < 2048u ? 0 : (32 - __clz((int)range)) - 11;
-    for (int i = tid; i < 2048; i += kSampleThreads) s_hist[i] = 0u;
-    __syncthreads();
-    for (int i = tid; i < S; i += kSampleThreads) atomicAdd(&s_hist[(s_key[i] - kmn) >> shift], 1u);
-    __syncthreads();
-    uint32_t bin, above, cnt;
-    if (rhi >= 1) {
-      block_find_desc<2048>(s_hist, (uint32_t)rhi, s_tmp, bin, above, cnt, bad);
-      const uint64_t top = (uint64_t)kmn + ((uint64_t)bin << shift) + ((1ull << shift) - 1ull);
-      hi = top < (uint64_t)kmx ? (uint32_t)top : kmx;
-    }
-    if (!bad && rlo <= S) {
-      block_find_desc<2048>(s_hist, (uint32_t)rlo, s_tmp, bin, above, cnt, bad);
-      lo = kmn + (bin << shift);
-    }
-  }
+  if (rhi >= 1) hi = rank_desc(s_key, S, (uint32_t)rhi, s_hist, s_tmp, cnt, rit, bad);
+  if (!bad && rlo <= S) lo = rank_desc(s_key, S, (uint32_t)rlo, s_hist, s_tmp, cnt, rit, bad);
   if (tid == 0) {
     if (bad) {           // cannot happen for 1 <= rank <= S; select_kernel re-scans
       hi = 0u;
@@ -2346,15 +2300,28 @@ static bool pdl_enabled() {
   return on == 1;
 }
 
-// The attention kernel streams records through a shared-memory ring when
-// SDK_ATTEND_RING=1, else through registers.
+// The attention kernel streams records through a shared-memory ring unless
+// SDK_ATTEND_RING=0 (then through registers; measured slower at 256K: 67.8
+// against 62.5 us per launch).
 static bool attend_ring() {
   static int on = -1;
   if (on < 0) {
     const char* v = getenv("SDK_ATTEND_RING");
-    on = (v != nullptr && v[0] == '1') ? 1 : 0;
+    on = (v != nullptr && v[0] == '0') ? 0 : 1;
   }
   return on == 1;
+}
+
+// Entries of the Klow scan's per-segment buffer of selected tokens in the
+// bracket path (candidates: half as many); SDK_KLOW_BUF overrides.
+static int klow_above_buf() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("SDK_KLOW_BUF");
+    int x = e != nullptr ? atoi(e) : 0;
+    v = (x >= 256 && x <= kKlowAboveBuf) ? (x & ~255) : kKlowAboveBuf;
+  }
+  return v;
 }
 
 // QD on the tensor cores (three bf16 parts of q) unless SDK_DECODE_QD_TC=0.
@@ -2375,6 +2342,35 @@ static bool out_tensor_cores() {
     on = (v != nullptr && v[0] == '0') ? 0 : 1;
   }
   return on == 1;
+}
+
+// With SDK_DEBUG=1 in the environment a failed launch is reported on
+// stderr with the CUDA error (the call still returns SDK_ERR_CUDA).
+static bool debug_launches() {
+  static int on = -1;
+  if (on < 0) {
+    const char* v = getenv("SDK_DEBUG");
+    on = (v != nullptr && v[0] == '1') ? 1 : 0;
+  }
+  return on == 1;
+}
+
+template <class... KArgs, class... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, unsigned cluster, Args... args);
+
+template <class... KArgs, class... Args>
+static cudaError_t launch_checked(const char* name, void (*kern)(KArgs...), dim3 grid, dim3 block,
+                                  size_t smem, cudaStream_t stream, unsigned cluster,
+                                  Args... args) {
+  const cudaError_t e = launch_pdl(kern, grid, block, smem, stream, cluster, args...);
+  if (debug_launches()) {
+    const cudaError_t e2 = e != cudaSuccess ? e : cudaPeekAtLastError();
+    if (e2 != cudaSuccess)
+      fprintf(stderr, "sdk: launch of %s (grid %u, block %u, smem %zu, cluster %u): %s\n", name,
+              grid.x, block.x, smem, cluster, cudaGetErrorString(e2));
+  }
+  return e;
 }
 
 template <class... KArgs, class... Args>
@@ -2541,11 +2537,11 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
     const size_t sm = qd_smem_bytes(p.d, gv_rb, gv_tiles);
     const unsigned th = 64 * gv_tiles * gv_rb;
     if (p.d == 128) {
-      e = wide ? launch_pdl(qd_kernel<128, 2, 4>, gv_grid, dim3(th), sm, stream, 1, p)
-               : launch_pdl(qd_kernel<128, 1, 1>, gv_grid, dim3(th), sm, stream, 1, p);
+      e = wide ? launch_checked("qd_kernel", qd_kernel<128, 2, 4>, gv_grid, dim3(th), sm, stream, 1, p)
+               : launch_checked("qd_kernel", qd_kernel<128, 1, 1>, gv_grid, dim3(th), sm, stream, 1, p);
     } else {
-      e = wide ? launch_pdl(qd_kernel<64, 2, 4>, gv_grid, dim3(th), sm, stream, 1, p)
-               : launch_pdl(qd_kernel<64, 1, 1>, gv_grid, dim3(th), sm, stream, 1, p);
+      e = wide ? launch_checked("qd_kernel", qd_kernel<64, 2, 4>, gv_grid, dim3(th), sm, stream, 1, p)
+               : launch_checked("qd_kernel", qd_kernel<64, 1, 1>, gv_grid, dim3(th), sm, stream, 1, p);
     }
     if (e != cudaSuccess) return SDK_ERR_CUDA;
   }
@@ -2553,13 +2549,15 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
     const int g = scan_grid(p.tok_off[p.B], p.R, kKlowSegCost, 2048, sms);
     const int vec = (p.cap % 4 == 0) && ((reinterpret_cast<uintptr_t>(p.k_lo) & 15u) == 0u);
     if (p.bracket) {
-      e = launch_pdl(sample_kernel, dim3(p.R), dim3(kSampleThreads), (size_t)kSampleSmem, stream,
+      e = launch_checked("sample_kernel", sample_kernel, dim3(p.R), dim3(kSampleThreads), (size_t)kSampleSmem, stream,
                      1, p);
       if (e != cudaSuccess) return SDK_ERR_CUDA;
-      e = launch_pdl(klow_kernel<true>, dim3(g), dim3(kKlowThreads), (size_t)kKlowSmemBracket,
+      p.klow_buf = klow_above_buf();
+      e = launch_checked("klow_kernel", klow_kernel<true>, dim3(g), dim3(kKlowThreads),
+                         (size_t)kTable * 4 + (size_t)p.klow_buf * 8,
                      stream, 1, p, vec);
     } else {
-      e = launch_pdl(klow_kernel<false>, dim3(g), dim3(kKlowThreads), (size_t)kKlowSmemHist,
+      e = launch_checked("klow_kernel", klow_kernel<false>, dim3(g), dim3(kKlowThreads), (size_t)kKlowSmemHist,
                      stream, 1, p, vec);
     }
     if (e != cudaSuccess) return SDK_ERR_CUDA;
@@ -2569,14 +2567,14 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
   case 1: {   // pass 2 of the selection (radix path only)
     if (p.bracket) return SDK_OK;
     const int g = scan_grid(p.tok_off[p.B], p.R, kPass2SegCost, 8192, sms);
-    e = launch_pdl(pass2_kernel, dim3(g), dim3(kP2Threads), (size_t)kPass2Smem, stream, 1, p);
+    e = launch_checked("pass2_kernel", pass2_kernel, dim3(g), dim3(kP2Threads), (size_t)kPass2Smem, stream, 1, p);
     return e == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
   }
   case 2:     // the final selection (whole context)
     if (p.bracket)
-      e = launch_pdl(select_kernel, dim3(p.R), dim3(kSelThreads), (size_t)kSelSmem, stream, 1, p);
+      e = launch_checked("select_kernel", select_kernel, dim3(p.R), dim3(kSelThreads), (size_t)kSelSmem, stream, 1, p);
     else
-      e = launch_pdl(final_kernel, dim3(p.R), dim3(kScanThreads), (size_t)2 * kFinalStage * 4,
+      e = launch_checked("final_kernel", final_kernel, dim3(p.R), dim3(kScanThreads), (size_t)2 * kFinalStage * 4,
                      stream, 1, p);
     return e == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
   case 3: {   // attend
@@ -2596,7 +2594,7 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
                              : (check ? attend_kernel<false, true, true> : attend_kernel<false, false, true>))
                     : (all16 ? (check ? attend_kernel<true, true, false> : attend_kernel<true, false, false>)
                              : (check ? attend_kernel<false, true, false> : attend_kernel<false, false, false>));
-    e = launch_pdl(kern, dim3((unsigned)(p.R * C)), dim3(reg ? kAttThreadsReg : kAttThreads),
+    e = launch_checked("attend_kernel", kern, dim3((unsigned)(p.R * C)), dim3(reg ? kAttThreadsReg : kAttThreads),
                    (size_t)(reg ? kAttSmemReg : kAttSmem), stream, (unsigned)C, p, C);
     if (e != cudaSuccess) return SDK_ERR_CUDA;
     if (t1 != nullptr && timing_record(t1, stream) != cudaSuccess) return SDK_ERR_CUDA;
@@ -2614,13 +2612,13 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
   if (!out_tc) {
     if (wide) {
       const size_t sm = out_smem_bytes(p.d, gv_rb, gv_tiles);
-      e = p.d == 128 ? launch_pdl(out_kernel<128, 2, 4>, gv_grid, dim3(256), sm, stream, 1, p)
-                     : launch_pdl(out_kernel<64, 2, 4>, gv_grid, dim3(128), sm, stream, 1, p);
+      e = p.d == 128 ? launch_checked("out_kernel", out_kernel<128, 2, 4>, gv_grid, dim3(256), sm, stream, 1, p)
+                     : launch_checked("out_kernel", out_kernel<64, 2, 4>, gv_grid, dim3(128), sm, stream, 1, p);
     } else {
       // up to 32 rows: 64 atoms per CTA (measured faster than 128 or 256)
       const size_t sm = out_smem_bytes(p.d, 1, 1);
-      e = p.d == 128 ? launch_pdl(out_kernel<128, 1, 1>, gv_grid, dim3(128), sm, stream, 1, p)
-                     : launch_pdl(out_kernel<64, 1, 1>, gv_grid, dim3(64), sm, stream, 1, p);
+      e = p.d == 128 ? launch_checked("out_kernel", out_kernel<128, 1, 1>, gv_grid, dim3(128), sm, stream, 1, p)
+                     : launch_checked("out_kernel", out_kernel<64, 1, 1>, gv_grid, dim3(64), sm, stream, 1, p);
     }
     if (e != cudaSuccess) return SDK_ERR_CUDA;
   }
@@ -2642,15 +2640,15 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
       case 1: st = run(0); break;
       case 2: st = run(1); break;
       case 3:
-        e = launch_pdl(shard_digit3_kernel, dim3(p.R), dim3(kScanThreads), 0, stream, 1, p);
+        e = launch_checked("shard_digit3_kernel", shard_digit3_kernel, dim3(p.R), dim3(kScanThreads), 0, stream, 1, p);
         st = e == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
         break;
       case 4:
-        e = launch_pdl(shard_ties_kernel, dim3(p.R), dim3(kScanThreads), 0, stream, 1, p);
+        e = launch_checked("shard_ties_kernel", shard_ties_kernel, dim3(p.R), dim3(kScanThreads), 0, stream, 1, p);
         st = e == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
         break;
       case 5:
-        e = launch_pdl(shard_select_kernel, dim3(p.R), dim3(kScanThreads), 0, stream, 1, p,
+        e = launch_checked("shard_select_kernel", shard_select_kernel, dim3(p.R), dim3(kScanThreads), 0, stream, 1, p,
                        reinterpret_cast<const uint32_t*>(p.shard_in), rank_id);
         if (e != cudaSuccess) return SDK_ERR_CUDA;
         p.att_mode = 1;
@@ -2667,7 +2665,10 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
     }
     if (st != SDK_OK) return st;
   }
-  return cudaGetLastError() == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
+  const cudaError_t last = cudaGetLastError();
+  if (last != cudaSuccess && debug_launches())
+    fprintf(stderr, "sdk: decode launches: %s\n", cudaGetErrorString(last));
+  return last == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
 }
 
 }  // namespace sdk

@@ -212,6 +212,7 @@ struct DecodeParams {
   // (v_full = k_full + 16: a token's key and value records form one
   // 128-byte line)
   int rs;
+  int klow_buf;          // bracket-path Klow scan: buffer entries (selected; candidates half)
   // context-sharded decode: 0 = whole decode; 1 / 2 = attend's first /
   // second half (shard_in: the gathered softmax statistics); world ranks
   int att_mode, world;
