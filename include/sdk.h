@@ -173,6 +173,12 @@ SDK_API size_t sdk_append_workspace_bytes(int32_t B, int32_t Hkv, int32_t n_new,
                                        the workspace region `keys` (for
                                        inspection; costs 4 B per token and
                                        query head of extra writes)           */
+#define SDK_DECODE_SELECT_RADIX 8   /* find the top-k set by radix histograms
+                                       of all keys                           */
+#define SDK_DECODE_SELECT_BRACKET 16 /* find it through a sampled bracket of
+                                       the k-th key (ignored with
+                                       SDK_DECODE_FULL_SOFTMAX); without
+                                       either flag the library's default     */
 
 /* ------------------------------------------------------------ decode attn
  * One layer of decode attention for B sequences over their code stores

@@ -18,7 +18,8 @@ import torch
 from . import _capi
 from ._capi import (SDK_OK, SDK_F32, SDK_BF16, MAX_ATOMS, K_ATOMS,
                     KLOW_PLANES, MAX_BATCH, SDK_DECODE_FULL_SOFTMAX,
-                    SDK_DECODE_INT_SOFTMAX, SDK_DECODE_KEEP_KEYS, DecodeLayout,
+                    SDK_DECODE_INT_SOFTMAX, SDK_DECODE_KEEP_KEYS,
+                    SDK_DECODE_SELECT_RADIX, SDK_DECODE_SELECT_BRACKET, DecodeLayout,
                     load)
 
 __all__ = [
@@ -250,17 +251,22 @@ def sdk_append(store, xk, xv, dict_k, dict_v, workspace=None, stream=None):
 
 # ------------------------------------------------------------------ decode
 
-def decode_flags(full_softmax=False, int_softmax=False, keep_keys=False):
-    """The flags word of sdk_decode_attn."""
+def decode_flags(full_softmax=False, int_softmax=False, keep_keys=False, select=None):
+    """The flags word of sdk_decode_attn; select: None (the library's
+    default), "radix" or "bracket"."""
+    if select not in (None, "radix", "bracket"):
+        raise ValueError("select must be None, 'radix' or 'bracket'")
     return ((SDK_DECODE_FULL_SOFTMAX if full_softmax else 0) |
             (SDK_DECODE_INT_SOFTMAX if int_softmax else 0) |
-            (SDK_DECODE_KEEP_KEYS if keep_keys else 0))
+            (SDK_DECODE_KEEP_KEYS if keep_keys else 0) |
+            (SDK_DECODE_SELECT_RADIX if select == "radix" else 0) |
+            (SDK_DECODE_SELECT_BRACKET if select == "bracket" else 0))
 
 
 def sdk_decode_attn(q, dict_k, dict_v, store, klow=3, khigh=16, top_num=1,
                     top_den=10, full_softmax=False, scale=None, out=None,
                     workspace=None, stream=None, int_softmax=False,
-                    keep_keys=False):
+                    keep_keys=False, select=None):
     """One layer of decode attention.  q [B, Hq, head_dim] fp32.  Returns
     out [B, Hq, head_dim] fp32 (and leaves the intermediate results in the
     workspace).  full_softmax / int_softmax / keep_keys set
@@ -285,7 +291,7 @@ def sdk_decode_attn(q, dict_k, dict_v, store, klow=3, khigh=16, top_num=1,
                              n_atoms, _ptr(store.k_lo), _ptr(store.k_full),
                              _ptr(store.v_full), store.cap, lens, klow, khigh,
                              top_num, top_den,
-                             decode_flags(full_softmax, int_softmax, keep_keys),
+                             decode_flags(full_softmax, int_softmax, keep_keys, select),
                              float(scale), _ptr(out), _ptr(workspace),
                              workspace.numel(), _stream(stream))
     _check(rc, "sdk_decode_attn")

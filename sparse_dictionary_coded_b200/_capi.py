@@ -18,6 +18,7 @@ STATUS_NAMES = {
 }
 SDK_F32, SDK_BF16 = 0, 1
 SDK_DECODE_FULL_SOFTMAX, SDK_DECODE_INT_SOFTMAX, SDK_DECODE_KEEP_KEYS = 1, 2, 4
+SDK_DECODE_SELECT_RADIX, SDK_DECODE_SELECT_BRACKET = 8, 16
 MAX_ATOMS, K_ATOMS, KLOW_PLANES, MAX_BATCH, WS_ALIGN = 32768, 16, 3, 64, 256
 DECODE_STATIC_WS_BYTES = 16 << 20
 

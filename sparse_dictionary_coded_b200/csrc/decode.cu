@@ -473,30 +473,50 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
           bc = __shfl_sync(0xffffffffu, bc, 31);
           const uint32_t ex = incl - mine;
           uint32_t pa = ba + (ex & 0xFFFFu), pc = bc + (ex >> 16);
+          // warp-uniform: do all of the warp's entries fit the buffers?
+          const bool fits = ba + (tot & 0xFFFFu) <= (uint32_t)cap_ab &&
+                            bc + (tot >> 16) <= (uint32_t)cap_cd;
+          if (fits) {
+            // common path: predicated shared-memory stores, no branches
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int t = 4 * q + u;
-            if ((fa >> u) & 1u) {
-              if (pa < (uint32_t)cap_ab) {
-                s_ab[pa] = t;
-              } else {
-                const uint32_t g = atomicAdd(&st->n_above, 1u);
-                if (g < (uint32_t)p.L) above_out[g] = t;
-              }
-              ++pa;
-            }
-            if ((fc >> u) & 1u) {
-              if (pc < (uint32_t)cap_cd) {
+            for (int u = 0; u < 4; ++u) {
+              const int t = 4 * q + u;
+              const bool a = (fa >> u) & 1u, c = (fc >> u) & 1u;
+              if (a) s_ab[pa] = t;
+              if (c) {
                 s_ct[pc] = t;
                 s_ck[pc] = kq[u];
-              } else {
-                const uint32_t g = atomicAdd(&st->n_cand, 1u);
-                if (g < (uint32_t)p.L) {
-                  cand_t[g] = t;
-                  cand_k[g] = kq[u];
-                }
               }
-              ++pc;
+              pa += a ? 1u : 0u;
+              pc += c ? 1u : 0u;
+            }
+          } else {
+            // a buffer is full: entries past its end take global slots
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int t = 4 * q + u;
+              if ((fa >> u) & 1u) {
+                if (pa < (uint32_t)cap_ab) {
+                  s_ab[pa] = t;
+                } else {
+                  const uint32_t g = atomicAdd(&st->n_above, 1u);
+                  if (g < (uint32_t)p.L) above_out[g] = t;
+                }
+                ++pa;
+              }
+              if ((fc >> u) & 1u) {
+                if (pc < (uint32_t)cap_cd) {
+                  s_ct[pc] = t;
+                  s_ck[pc] = kq[u];
+                } else {
+                  const uint32_t g = atomicAdd(&st->n_cand, 1u);
+                  if (g < (uint32_t)p.L) {
+                    cand_t[g] = t;
+                    cand_k[g] = kq[u];
+                  }
+                }
+                ++pc;
+              }
             }
           }
         }
@@ -1053,12 +1073,17 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(DecodeParams p) 
     const uint32_t* ck = p.cand_key + (int64_t)r * p.L;
     const int32_t* ct = p.cand_t + (int64_t)r * p.L;
     if (C <= (uint32_t)kSelStage) {
+      // 16-byte asynchronous copies, all of a thread's in flight at once
+      // (rows are 16-byte aligned; the last copy reads only what is left)
       uint32_t* s_ck = reinterpret_cast<uint32_t*>(smem4);
       int32_t* s_ct = reinterpret_cast<int32_t*>(s_ck + kSelStage);
-      for (uint32_t i = tid; i < C; i += kSelThreads) {
-        s_ck[i] = __ldcg(ck + i);
-        s_ct[i] = __ldcg(ct + i);
+      for (uint32_t i4 = tid; 4 * i4 < C; i4 += kSelThreads) {
+        const unsigned bytes = 4u * min(4u, C - 4 * i4);
+        cp_async16_n(s_ck + 4 * i4, ck + 4 * i4, bytes);
+        cp_async16_n(s_ct + 4 * i4, ct + 4 * i4, bytes);
       }
+      cp_async_commit();
+      cp_async_wait<0>();
       __syncthreads();
       ck = s_ck;
       ct = s_ct;
@@ -1566,6 +1591,18 @@ constexpr int kAttSmemReg = kTable * 4;      // records in registers: the table 
 constexpr float kFixScale = 1048576.0f;       // 2^20
 constexpr float kFixInv = 1.0f / 1048576.0f;
 
+// L2 policies: keep a line (evict last) / let it go first
+__device__ __forceinline__ uint64_t l2_evict_last() {
+  uint64_t pol;
+  asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 // Calls f(i, t, w, x) for every entry i in [e0, e1) of `list` owned by this
 // thread (i = e0 + tid + j*T); w holds the 16 words of token t's record and
 // x = pay(i, t), a per-entry value whose load is issued together with the
@@ -1590,12 +1627,16 @@ __device__ __forceinline__ void for_records(const int32_t* list, int e0, int e1,
   const int sw = (tid >> 1) & 3;
   auto list_at = [&](int i) -> int { return i < e1 ? __ldg(list + i) : -1; };
   auto ok = [&](int t) { return (unsigned)t < (unsigned)Nb; };
+  // interleaved records: the key pass (kLine) keeps each whole line
+  // evict-last in L2 for the value pass, which reads with evict-first
+  const uint64_t pol = kLine ? l2_evict_last() : l2_evict_first();
+  const bool inter = rs4 == 8;
   auto issue = [&](int t, int slot) {
     const bool v = ok(t);
     const uint4* a = rec + (int64_t)(v ? t : 0) * rs4;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      if (kLine) cp_async16_128B(ring + (slot * T + tid) * 4 + (u ^ sw), a + u, v);
+      if (kLine) cp_async16_128B_pol(ring + (slot * T + tid) * 4 + (u ^ sw), a + u, v, pol);
       else cp_async16_64B(ring + (slot * T + tid) * 4 + (u ^ sw), a + u, v);
     }
     cp_async_commit();
@@ -1603,8 +1644,16 @@ __device__ __forceinline__ void for_records(const int32_t* list, int e0, int e1,
   auto prefetch = [&](int t) {
     if (ok(t)) {
       const uint4* a = rec + (int64_t)t * rs4;
-      if (kLine) asm volatile("cp.async.bulk.prefetch.L2.global [%0], 128;" ::"l"(a) : "memory");
-      else asm volatile("cp.async.bulk.prefetch.L2.global [%0], 64;" ::"l"(a) : "memory");
+      if (kLine)
+        asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], 128, %1;" ::"l"(a),
+                     "l"(pol)
+                     : "memory");
+      else if (inter)
+        asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], 64, %1;" ::"l"(a),
+                     "l"(pol)
+                     : "memory");
+      else
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], 64;" ::"l"(a) : "memory");
     }
   };
   int i = e0 + tid;
@@ -1659,17 +1708,6 @@ __device__ __forceinline__ uint4 ld_record16(const uint4* a, uint64_t pol) {
     asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(a), "l"(pol));
   return v;
-}
-// L2 policies: keep a line (evict last) / let it go first
-__device__ __forceinline__ uint64_t l2_evict_last() {
-  uint64_t pol;
-  asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
-__device__ __forceinline__ uint64_t l2_evict_first() {
-  uint64_t pol;
-  asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
 }
 
 // for_records with the records in registers instead of a shared-memory

@@ -135,6 +135,15 @@ __device__ __forceinline__ void cp_async16_128B(void* smem_dst, const void* gsrc
                "r"(valid ? 16 : 0)
                : "memory");
 }
+// The same under an L2 eviction policy (createpolicy), fetching the whole
+// 128-byte line.
+__device__ __forceinline__ void cp_async16_128B_pol(void* smem_dst, const void* gsrc, bool valid,
+                                                    uint64_t pol) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(smem_dst);
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint.L2::128B [%0], [%1], 16, %2, %3;" ::"r"(d),
+               "l"(gsrc), "r"(valid ? 16 : 0), "l"(pol)
+               : "memory");
+}
 // The same with the L2 prefetch size limited to 64 bytes (for 64-byte
 // records at scattered addresses).
 __device__ __forceinline__ void cp_async16_64B(void* smem_dst, const void* gsrc, bool valid) {

@@ -92,7 +92,8 @@ def _decode(lib, **kw):
     (dict(lens=(ctypes.c_int32 * 1)(257)), 1),
     (dict(ws_bytes=1024), 3),                 # workspace too small
     (dict(q=MISALIGNED), 1),                  # q must be 16-byte aligned
-    (dict(full=8), 1),                        # unknown flag bit
+    (dict(full=32), 1),                       # unknown flag bit
+    (dict(full=24), 1),                       # both selection flags
 ])
 def test_decode_rejects_bad_arguments(lib, kw, status):
     assert _decode(lib, **kw) == status

@@ -81,7 +81,7 @@ def _isoft_logits(ws, lay, r, k, n_b, full, keys_r, scale):
 
 
 def _compare(q, DK, DV, kw, vw, lens, klow=3, khigh=16, top_num=1, top_den=10,
-             full=False, heads=None, isoft=False):
+             full=False, heads=None, isoft=False, select=None):
     """Runs GPU decode and checks sets, s_lo and outputs against the oracle
     for the given (b, h) heads (all if None).  isoft: integer softmax on
     both sides, and the kernel's integer sum and guard shift recomputed
@@ -90,7 +90,7 @@ def _compare(q, DK, DV, kw, vw, lens, klow=3, khigh=16, top_num=1, top_den=10,
     store = _store(kw, vw, lens)
     out, ws, lay, rc = _run(q, DK, DV, store, klow=klow, khigh=khigh,
                             top_num=top_num, top_den=top_den,
-                            full_softmax=full, int_softmax=isoft)
+                            full_softmax=full, int_softmax=isoft, select=select)
     assert rc == 0, "device check failed"
     L = max(lens)
     R = B * Hq
@@ -111,9 +111,15 @@ def _compare(q, DK, DV, kw, vw, lens, klow=3, khigh=16, top_num=1, top_den=10,
         n_b = lens[b]
         kvh = h // g
         assert int(st["n_sel"][r]) == ks[r]
-        # full softmax: radix selection (0); otherwise the sampled bracket
-        # (1), or its exact re-scan when the bracket missed (2)
-        assert int(st["select_path"][r]) == (0 if full else 1), int(st["select_path"][r])
+        # full softmax or select="radix": radix selection (0); select=
+        # "bracket": the sampled bracket (1); the library's default: either
+        path = int(st["select_path"][r])
+        if full or select == "radix":
+            assert path == 0, path
+        elif select == "bracket":
+            assert path == 1, path
+        else:
+            assert path in (0, 1), path
         ref = oracle.decode_head_ref(qn[b, h], kwn[b, kvh, :n_b],
                                      vwn[b, kvh, :n_b], DKn, DVn, klow, khigh,
                                      top_num, top_den, full, int_softmax=isoft)
@@ -169,12 +175,12 @@ def test_tiny_workload_oracle_encoded_codes():
         _compare(q, w["DK"], w["DV"], kw, vw, [N], full=full)
 
 
-@pytest.mark.parametrize("full", [False, True])
-def test_layer4k_shape_random_codes(full):
+@pytest.mark.parametrize("full,select", [(False, "radix"), (False, "bracket"), (True, None)])
+def test_layer4k_shape_random_codes(full, select):
     """Workload 'layer4k' shape: 32 q / 8 KV heads, d=128, 32768 atoms,
-    4096 tokens (random codes from the input generator)."""
+    4096 tokens (random codes from the input generator), both selections."""
     q, DK, DV, kw, vw, lens = _random_case(77, 1, 32, 8, 4096, 128, 32768)
-    _compare(q, DK, DV, kw, vw, lens, full=full)
+    _compare(q, DK, DV, kw, vw, lens, full=full, select=select)
 
 
 def test_ragged_batch_small_and_odd_sizes():
@@ -186,8 +192,8 @@ def test_ragged_batch_small_and_odd_sizes():
         _compare(q, DK, DV, kw, vw, lens, full=full)
 
 
-@pytest.mark.parametrize("full", [False, True])
-def test_ragged_batch_many_ctas(full):
+@pytest.mark.parametrize("full,select", [(False, "radix"), (False, "bracket"), (True, None)])
+def test_ragged_batch_many_ctas(full, select):
     """B=4 with lengths 9000, 40000, 2500 and 23000 (GQA 8/2, d=128, 4096
     atoms): the Klow scan and pass 2 split these unequal heads over many
     CTAs (the work split charges every head a start-up cost, so CTA bounds
@@ -196,7 +202,7 @@ def test_ragged_batch_many_ctas(full):
     or that two did, fails."""
     q, DK, DV, kw, vw, _ = _random_case(91, 4, 8, 2, 40000, 128, 4096)
     lens = [9000, 40000, 2500, 23000]
-    _compare(q, DK, DV, kw, vw, lens, full=full)
+    _compare(q, DK, DV, kw, vw, lens, full=full, select=select)
 
 
 @pytest.mark.parametrize("full", [False, True])
@@ -239,12 +245,13 @@ def test_all_tokens_tie(full):
     vw = workloads.random_codes((1, 1, N), n, g)
     q = _unit(workloads.queries(1, 2, d, g))
     store = _store(kw, vw)
-    out, ws, lay, rc = _run(q, DK, DV, store, full_softmax=full)
-    assert rc == 0
-    sets = _gpu_sets(ws, lay, 2, N, [100, 100])
-    for r in range(2):
-        assert sorted(sets[r].tolist()) == list(range(100))
-    _compare(q, DK, DV, kw, vw, [N], full=full)
+    for select in ("radix", "bracket"):
+        out, ws, lay, rc = _run(q, DK, DV, store, full_softmax=full, select=select)
+        assert rc == 0
+        sets = _gpu_sets(ws, lay, 2, N, [100, 100])
+        for r in range(2):
+            assert sorted(sets[r].tolist()) == list(range(100))
+        _compare(q, DK, DV, kw, vw, [N], full=full, select=None if full else select)
 
 
 def test_partial_ties_at_threshold():
@@ -258,7 +265,8 @@ def test_partial_ties_at_threshold():
     kw[0, 0, 1::2] = kw[0, 0, 7]
     vw = workloads.random_codes((1, 1, N), n, g)
     q = _unit(workloads.queries(1, 4, d, g))
-    _compare(q, DK, DV, kw, vw, [N])
+    _compare(q, DK, DV, kw, vw, [N], select="radix")
+    _compare(q, DK, DV, kw, vw, [N], select="bracket")
     _compare(q, DK, DV, kw, vw, [N], full=True)
 
 
@@ -337,7 +345,7 @@ def test_sampled_bracket_misses_on_both_sides():
     q = torch.zeros(1, Hkv, d)
     q[0, :, 0] = 1.0
     store = _store(kw, vw)
-    out, ws, lay, rc = _run(q, DK, DV, store)
+    out, ws, lay, rc = _run(q, DK, DV, store, select="bracket")
     assert rc == 0
     st = sdk.read_select_state(ws, lay, Hkv)
     assert [int(v) for v in st["select_path"]] == [2, 2, 1]
@@ -444,7 +452,7 @@ def test_integer_softmax(full):
 
 
 def test_decode_flags_are_checked():
-    """Flag bits other than the three defined ones, and a query array that is
+    """Flag bits other than the defined ones, and a query array that is
     not 16-byte aligned, are rejected before any launch."""
     q, DK, DV, kw, vw, lens = _random_case(17, 1, 2, 1, 64, 64, 1000)
     store = _store(kw, vw)
@@ -456,7 +464,7 @@ def test_decode_flags_are_checked():
     lens_c = (ctypes.c_int32 * 1)(64)
     rc = lib.sdk_decode_attn(qd.data_ptr(), 1, 2, 1, 64, DKd.data_ptr(), DVd.data_ptr(), 1000,
                              store.k_lo.data_ptr(), store.k_full.data_ptr(),
-                             store.v_full.data_ptr(), store.cap, lens_c, 3, 16, 1, 10, 8,
+                             store.v_full.data_ptr(), store.cap, lens_c, 3, 16, 1, 10, 32,
                              0.125, out.data_ptr(), ws.data_ptr(), ws.numel(), None)
     assert rc == 1
     qbuf = torch.zeros(1 + q.numel(), device="cuda")
@@ -529,8 +537,9 @@ def _full_size_layer(name):
     return lay, store
 
 
-@pytest.mark.parametrize("name", ["decode32k_b4", "decode256k"])
-def test_full_size_layer_every_head(name):
+@pytest.mark.parametrize("name,select", [("decode32k_b4", "bracket"), ("decode256k", "bracket"),
+                                         ("decode256k", "radix")])
+def test_full_size_layer_every_head(name, select):
     """One layer of the full-size decode workloads (256K tokens: 32 heads;
     32K tokens at batch 4: 128 heads) in the bench's launch configuration:
     for EVERY query head the selected set against the oracle's exact top k
@@ -542,16 +551,18 @@ def test_full_size_layer_every_head(name):
     R, g = B * Hq, Hq // Hkv
     q = _unit(lay["q"])
     ws = sdk.new_workspace(sdk.sdk_decode_workspace_bytes(B, Hq, 128, 32768, N))
-    out = sdk.sdk_decode_attn(q, lay["DK"], lay["DV"], store, workspace=ws)
+    out = sdk.sdk_decode_attn(q, lay["DK"], lay["DV"], store, workspace=ws, select=select)
     torch.cuda.synchronize()
     assert sdk.sdk_check_status(ws)[0] == 0
     layd = sdk.sdk_decode_layout_of(B, Hq, 128, 32768, N)
     k = oracle.topk_count(N, 1, 10)
     st = sdk.read_select_state(ws, layd, R)
-    assert torch.all(st["n_sel"] == k) and torch.all(st["select_path"] == 1)
+    assert torch.all(st["n_sel"] == k)
+    assert torch.all(st["select_path"] == (1 if select == "bracket" else 0))
     sets = _gpu_sets(ws, layd, R, N, [k] * R)
     outn = out.cpu().double().numpy()
-    out2 = sdk.sdk_decode_attn(q, lay["DK"], lay["DV"], store, workspace=ws, keep_keys=True)
+    out2 = sdk.sdk_decode_attn(q, lay["DK"], lay["DV"], store, workspace=ws, keep_keys=True,
+                               select=select)
     torch.cuda.synchronize()
     assert sdk.sdk_check_status(ws)[0] == 0
     sets2 = _gpu_sets(ws, layd, R, N, [k] * R)
