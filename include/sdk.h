@@ -420,7 +420,8 @@ SDK_API sdk_status sdk_check_status(void* workspace, sdk_stream_t stream,
 /* Kernel timing, for measurement.  While enabled (a process-wide switch),
  * every launch of the decode attention kernel (the Khigh rescore, softmax
  * and value scatter: one per sdk_decode_attn call, one in each of stages 5
- * and 6 of sdk_decode_attn_shard) is bracketed by a pair of CUDA events
+ * and 6 of sdk_decode_attn_shard) and of the tensor-core encoder (one per
+ * sdk_encode / sdk_append call that takes it) is bracketed by a pair of CUDA events
  * recorded on the call's stream; the pairs are the current device's slots
  * 0, 1, 2, ... of SDK_TIMING_SLOTS, reused round-robin.  Calls captured in
  * a CUDA graph keep their slots, and every replay records them again.

@@ -2450,6 +2450,8 @@ struct TimingPool {
 };
 TimingPool g_timing[kTimingDevices];
 
+}  // namespace
+
 // The event pair of the next slot of the current device (nulls when timing
 // is off, or was not turned on for this device).
 void timing_slot(cudaEvent_t* e0, cudaEvent_t* e1) {
@@ -2475,7 +2477,7 @@ cudaError_t timing_record(cudaEvent_t e, cudaStream_t stream) {
              ? cudaEventRecordWithFlags(e, stream, cudaEventRecordExternal)
              : cudaEventRecord(e, stream);
 }
-}  // namespace
+
 
 // The current device's events are made here, outside any stream capture.
 sdk_status timing_enable(bool on) {

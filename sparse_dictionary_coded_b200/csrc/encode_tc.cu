@@ -1025,6 +1025,9 @@ sdk_status launch_encode_tc(const EncodeParams* ps, int streams, int head_dim, v
     device_setup_done(&attr_set);
   }
   const dim3 g((unsigned)grid);
+  cudaEvent_t t0 = nullptr, t1 = nullptr;
+  timing_slot(&t0, &t1);
+  if (t0 != nullptr && timing_record(t0, stream) != cudaSuccess) return SDK_ERR_CUDA;
   if (head_dim == 128) {
     if (f16)
       tc::encode_tc_kernel<128, true><<<g, tc::kThreads, tc::Cfg<128>::kSmem, stream>>>(maps[0], maps[1], tp);
@@ -1036,6 +1039,7 @@ sdk_status launch_encode_tc(const EncodeParams* ps, int streams, int head_dim, v
     else
       tc::encode_tc_kernel<64, false><<<g, tc::kThreads, tc::Cfg<64>::kSmem, stream>>>(maps[0], maps[1], tp);
   }
+  if (t1 != nullptr && timing_record(t1, stream) != cudaSuccess) return SDK_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? SDK_OK : SDK_ERR_CUDA;
 }
 

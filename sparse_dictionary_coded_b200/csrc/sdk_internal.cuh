@@ -271,9 +271,13 @@ sdk_status launch_out_tc(const DecodeParams& p, cudaStream_t stream, bool* taken
 // decode for rank rank_id (sdk_decode_attn_shard)
 sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage = 0,
                          int rank_id = 0);
-// attention-kernel timing (sdk_timing_enable / sdk_timing_read)
+// kernel timing (sdk_timing_enable / sdk_timing_read): the next slot's
+// event pair (nulls when timing is off) and a record that also works inside
+// a stream capture
 sdk_status timing_enable(bool on);
 int timing_read(float* ms_out, int max_n);
+void timing_slot(cudaEvent_t* e0, cudaEvent_t* e1);
+cudaError_t timing_record(cudaEvent_t e, cudaStream_t stream);
 sdk_decode_layout decode_layout(int B, int Hq, int d, int n, int64_t L);
 sdk_status launch_encode_simt(const EncodeParams& p, int head_dim, cudaStream_t stream);
 // Tensor-core encoder of one or two streams (ps[0..streams-1]; two
