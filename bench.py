@@ -512,12 +512,35 @@ def bench_decode_sharded(args, world, rank, pk, name):
             if world > 1:
                 sharded.run_exchanges(gen)
             else:
-                for _ in gen:
-                    pass
+                # one rank: a sum over ranks is the identity, a gather a copy
+                for kind, t, into in gen:
+                    if kind == "gather":
+                        into.copy_(t)
 
-    flush = make_flush()
+    flush = no_flush      # inputs larger than L2, as for the unsharded decode
+    timed = step
+    graph = None
+    if world == 1:
+        # one rank: every exchange is the identity, so the stages of all
+        # layers are replayed as one CUDA graph (as the unsharded step is);
+        # with several ranks the NCCL exchanges run between host-driven
+        # stages
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            step()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        timed = graph.replay
     clocks = Clocks(torch.cuda.current_device())
-    ms, ck = timed_steps(step, args.steps, args.warmup, flush, world, clocks)
+    ms, ck = timed_steps(timed, args.steps, args.warmup, flush, world, clocks)
+    ms_nog = None
+    if graph is not None:
+        ms_nog, _ = timed_steps(step, max(2, args.steps // 2), 1, flush, world)
+        del graph
     for plan in plans:
         rc, _ = sdk.sdk_check_status(plan.ws)
         assert rc == 0, "device check failed in sharded decode"
@@ -531,8 +554,10 @@ def bench_decode_sharded(args, world, rank, pk, name):
     return {
         "value": B * N / (step_ms * 1e-3),
         "unit": DECODE_UNIT,
-        "unit_note": "%d layers, context split over %d GPUs" % (L, world),
+        "unit_note": "%d layers, context split over %d GPUs%s" % (
+            L, world, " (one CUDA graph)" if world == 1 else ""),
         "ms_per_step": step_ms,
+        **({"ms_per_step_no_graph": statistics.mean(ms_nog)} if ms_nog else {}),
         "scaling": "strong",
         "roofline": {"bound": "hbm", "kernel": "context-sharded decode step "
                      "(all stages, %d layers)" % L, "achieved": gbs,

@@ -217,8 +217,11 @@ SDK_API size_t sdk_append_workspace_bytes(int32_t B, int32_t Hkv, int32_t n_new,
  *              n_atoms, max_len) with max_len >= every lens[b]
  * Limits: B <= 64, Hq % Hkv == 0, head_dim in {64, 128}, B*Hq <= 2048,
  *         scale > 0.
- * Selection (how S is found; the set is exact either way): without
- * SDK_DECODE_FULL_SOFTMAX, a sample of every head's tokens is scored first
+ * Selection (how S is found; the set is exact either way): by default
+ * (and always with SDK_DECODE_FULL_SOFTMAX) a radix select over the keys
+ * of all tokens (histograms of their digits).  With
+ * SDK_DECODE_SELECT_BRACKET (or SDK_DECODE_BRACKET=1 in the environment
+ * as the default), a sample of every head's tokens is scored first
  * and two of its order statistics bracket the k-th key; the Klow scan then
  * selects the tokens above the bracket and keeps those inside it as
  * candidates, among which the exact k-th key and the tie cut are found; a
@@ -232,8 +235,6 @@ SDK_API size_t sdk_append_workspace_bytes(int32_t B, int32_t Hkv, int32_t n_new,
  * from i * blk + 8 * (lowbias32(seed ^ i) mod (len_i / 8)), or all of its
  * tokens when len_i < 8.  The bracket is the sample's order statistics
  * 6 standard deviations of the sample rank above and below S * k / N.
- * With SDK_DECODE_FULL_SOFTMAX (or SDK_DECODE_BRACKET=0 in the environment)
- * the selection runs by radix histograms of all keys instead.
  * Code store layout: k_full and v_full may also point into ONE array
  * uint32 [B][Hkv][cap][2][16] with v_full = k_full + 16 (a token's key and
  * value records adjacent in one 128-byte line); the library detects this

@@ -148,3 +148,22 @@ def test_clock_parsing():
     c.t0, c.t1 = 1.2, 1.3
     r = c.stop()
     assert r["samples"] == 2 and r["sm_mhz"] == 1925
+
+
+def test_profiled_traffic_only_for_the_captured_source(tmp_path, monkeypatch):
+    """roofline.traffic comes from a committed ncu summary only while the
+    kernel's source file still has the sha256 the summary records."""
+    import hashlib
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1")
+    (tmp_path / "profiles").mkdir()
+    sha = hashlib.sha256(b"kernel v1").hexdigest()
+    (tmp_path / "profiles" / "attend_kernel_w.md").write_text(
+        "traffic_bytes_per_launch: 123456789\nsource_sha256: %s k.cu\n" % sha)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    t, note = bench.profiled_traffic("attend_kernel", "w")
+    assert t == 123456789.0 and "attend_kernel_w.md" in note
+    src.write_text("kernel v2")
+    t, note = bench.profiled_traffic("attend_kernel", "w")
+    assert t is None and "changed" in note
+    assert bench.profiled_traffic("attend_kernel", "other")[0] is None
