@@ -317,7 +317,9 @@ __device__ __forceinline__ void stage_table(float* table, const float* src, int 
   for (int i = n + threadIdx.x; i < kTable; i += nt) table[i] = 0.0f;
 }
 
-template <bool kBracket>
+// kCheck: the dictionary has fewer than 32768 atoms, so an index can lie
+// past it and is reported (with 32768 atoms every 15-bit index is valid).
+template <bool kBracket, bool kCheck>
 __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, int vec) {
   pdl_wait();     // nothing global is touched before the previous kernel is done
   pdl_launch();
@@ -411,13 +413,13 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
 #pragma unroll
         for (int j = 0; j < kLoPlanes; ++j) {
           const uint32_t idx = word_idx(wc[j][u]);
-          maxidx = max(maxidx, idx);
+          if (kCheck) maxidx = max(maxidx, idx);
           s = fmaf(word_coef(wc[j][u]), table[idx], s);
         }
         for (int j = kLoPlanes; j < p.klow; ++j) {      // klow > 3: k_full words
           const uint32_t wj = (t >= t0 && t < t1) ? __ldg(rec + (int64_t)t * p.rs + j) : 0u;
           const uint32_t idx = word_idx(wj);
-          maxidx = max(maxidx, idx);
+          if (kCheck) maxidx = max(maxidx, idx);
           s = fmaf(word_coef(wj), table[idx], s);
         }
         kq[u] = score_key(s);
@@ -558,7 +560,7 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
       if (tid == 0) s_cnt[0] = s_cnt[1] = 0u;
     }
   });
-  if (maxidx >= (uint32_t)n) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, maxidx);
+  if (kCheck && maxidx >= (uint32_t)n) record_error(p.hdr, SDK_ERR_DEVICE_CHECK, maxidx);
 }
 
 // ------------------------------------------------------- final selection
@@ -2522,9 +2524,13 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
   const int sms = num_sms();
   static unsigned long long attr_set = 0ull;
   if (device_needs_setup(&attr_set)) {
-    cudaFuncSetAttribute(klow_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(klow_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kKlowSmemHist);
-    cudaFuncSetAttribute(klow_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(klow_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kKlowSmemHist);
+    cudaFuncSetAttribute(klow_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kKlowSmemBracket);
+    cudaFuncSetAttribute(klow_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kKlowSmemBracket);
     cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelSmem);
     cudaFuncSetAttribute(sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSampleSmem);
@@ -2593,11 +2599,13 @@ sdk_status launch_decode(DecodeParams p, cudaStream_t stream, int shard_stage, i
                      1, p);
       if (e != cudaSuccess) return SDK_ERR_CUDA;
       p.klow_buf = klow_above_buf();
-      e = launch_checked("klow_kernel", klow_kernel<true>, dim3(g), dim3(kKlowThreads),
+      e = launch_checked("klow_kernel", p.n < kTable ? klow_kernel<true, true> : klow_kernel<true, false>,
+                         dim3(g), dim3(kKlowThreads),
                          (size_t)kTable * 4 + (size_t)p.klow_buf * 8,
                      stream, 1, p, vec);
     } else {
-      e = launch_checked("klow_kernel", klow_kernel<false>, dim3(g), dim3(kKlowThreads), (size_t)kKlowSmemHist,
+      e = launch_checked("klow_kernel", p.n < kTable ? klow_kernel<false, true> : klow_kernel<false, false>,
+                         dim3(g), dim3(kKlowThreads), (size_t)kKlowSmemHist,
                      stream, 1, p, vec);
     }
     if (e != cudaSuccess) return SDK_ERR_CUDA;
