@@ -286,7 +286,10 @@ constexpr int kKlowThreads = 1024;
 // (expected per segment at 256K tokens on 148 CTAs: about 4,500 and 2,300)
 constexpr int kKlowAboveBuf = 8192;
 constexpr int kKlowCandBuf = 4096;
-constexpr int kKlowSmemHist = kTable * 4 + 4096 * 4;
+// radix mode: two copies of the 4096-bin histogram (even and odd warps),
+// which halves the collisions of the histogram atomics (a head's keys
+// fall into few bins); the copies are summed when the segment flushes
+constexpr int kKlowSmemHist = kTable * 4 + 2 * 4096 * 4;
 constexpr int kKlowSmemBracket = kTable * 4 + (kKlowAboveBuf + 2 * kKlowCandBuf) * 4;
 
 // QD row -> table[0..kTable), zero past n.  Eight 16-byte loads per thread
@@ -326,6 +329,7 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
   extern __shared__ float4 smem4[];
   float* table = reinterpret_cast<float*>(smem4);
   uint32_t* sh = reinterpret_cast<uint32_t*>(table + kTable);
+  uint32_t* shw = sh + ((threadIdx.x >> 5) & 1) * 4096;   // this warp's histogram copy
   // bracket mode: the segment's selected tokens and candidates are
   // collected here and reserved in the global lists once per segment
   const int cap_ab = p.klow_buf, cap_cd = p.klow_buf / 2;
@@ -344,7 +348,7 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
     const int t0 = (int)t0l, t1 = (int)t1l;    // token indices fit 31 bits
     stage_table(table, p.qd + (int64_t)r * n, n);
     if (!kBracket)
-      for (int i = tid; i < 4096; i += kKlowThreads) sh[i] = 0u;
+      for (int i = tid; i < 2 * 4096; i += kKlowThreads) sh[i] = 0u;
     __syncthreads();
     const int64_t head = (int64_t)b * p.Hkv + kvh;
     const uint32_t* plane = p.k_lo + head * kLoPlanes * p.cap;
@@ -430,7 +434,7 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
           *reinterpret_cast<uint4*>(keys + 4 * q) = make_uint4(kq[0], kq[1], kq[2], kq[3]);
           if (!kBracket) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) atomicAdd(&sh[kq[u] >> 20], 1u);
+            for (int u = 0; u < 4; ++u) atomicAdd(&shw[kq[u] >> 20], 1u);
           }
         } else if (q < q1) {
 #pragma unroll
@@ -438,7 +442,7 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
             const int t = 4 * q + u;
             if (t >= t0 && t < t1) {
               keys[t] = kq[u];
-              if (!kBracket) atomicAdd(&sh[kq[u] >> 20], 1u);
+              if (!kBracket) atomicAdd(&shw[kq[u] >> 20], 1u);
             }
           }
         }
@@ -531,8 +535,10 @@ __global__ void __launch_bounds__(kKlowThreads, 1) klow_kernel(DecodeParams p, i
     __syncthreads();
     if (!kBracket) {
       uint32_t* gh = p.hist1 + (int64_t)r * 4096;
-      for (int i = tid; i < 4096; i += kKlowThreads)
-        if (sh[i]) atomicAdd(&gh[i], sh[i]);
+      for (int i = tid; i < 4096; i += kKlowThreads) {
+        const uint32_t c = sh[i] + sh[4096 + i];
+        if (c) atomicAdd(&gh[i], c);
+      }
       __syncthreads();
     } else {
       // the segment's buffered entries: one global reservation per kind
